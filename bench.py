@@ -1,0 +1,325 @@
+"""Benchmark of the BigBird ITC block-sparse attention forward on B200.
+
+One step = one forward pass (every row of the pattern: global rows, second
+rows, middle rows, epilogue) over one batch of the BigBird-base attention
+workload (B=4, H=12, L=4096, d=64, block=64, r=3, bf16, valid lengths
+U[2048, 4096]) by default. Metric: sparse TFLOP/s = 4 * B * H * L *
+keys_per_row * d / t.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+With N > 1 (launched by torch.distributed.run) every rank runs its own batch
+of the workload (weak scaling: heads/batches are independent; no data-path
+collective); time = max over ranks. `--impl reference` times the fp64 CPU
+oracle on a bounded sample of the same workload on the host cores.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "block-sparse attention TFLOP/s and % of BF16 tensor peak at L=4096, 1×B200"
+UNIT = "TFLOP/s"
+DEFAULT_WORKLOAD = "bigbird_base_l4096"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+def _dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle sampling; keeps the samples taken inside the
+    timed window [t0, t1] (host wall clock)."""
+
+    QUERY = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"bb_clocks_{os.getpid()}.csv")
+        self.t0 = self.t1 = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                 "-lms", "50"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        from datetime import datetime
+        rows = []
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 10:
+                continue
+            try:
+                ts = datetime.strptime(f[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                rows.append((ts, float(f[2]), float(f[3]), f[6], f[7], f[8], f[9]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        inside = [r for r in rows if self.t0 is not None and self.t0 <= r[0] <= self.t1]
+        if not inside:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        reasons = set()
+        for r in inside:
+            for name, val in zip(("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"),
+                                 r[3:]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": float(np.median([r[1] for r in inside])), "sm_max_mhz": max(r[2] for r in inside),
+                "reasons": sorted(reasons), "samples": len(inside)}
+
+
+def _oracle_sample(w, inp, ra, budget_s: float):
+    """Time the oracle, as it stands, on whole (b, h) heads until budget_s is
+    spent. Returns (sparse FLOPs processed, seconds, heads, threads)."""
+    import oracle
+    from threadpoolctl import threadpool_info
+
+    threads = max([t.get("num_threads", 1) for t in threadpool_info()] or [1])
+    per_head = oracle.sparse_flops(1, 1, w.L, w.d, w.block, w.r)
+    done, heads = 0.0, 0
+    t0 = time.perf_counter()
+    for b in range(w.B):
+        for h in range(w.H):
+            sub = {x: inp[x][b:b + 1, h:h + 1] for x in "qkv"}
+            sm = None if inp["seq_mask"] is None else inp["seq_mask"][b:b + 1].numpy()
+            oracle.attention(sub["q"], sub["k"], sub["v"], None if ra is None else ra[h:h + 1], sm, w.block, w.r)
+            done += per_head
+            heads += 1
+            if time.perf_counter() - t0 >= budget_s:
+                return done, time.perf_counter() - t0, heads, threads
+    return done, time.perf_counter() - t0, heads, threads
+
+
+def run_reference(args):
+    """The oracle on the host cores: the reference arm of this benchmark."""
+    world, rank, _ = _dist_env()
+    if rank != 0:
+        return 0
+    import oracle
+    from block_sparse_long_attention_b200.workloads import WORKLOADS, make_inputs
+    w = WORKLOADS[args.workload]
+    inp = make_inputs(w)
+    ra = None if oracle.is_fallback(w.L, w.block, w.r) else oracle.rand_attn_generate(w.H, w.L, w.block, w.r, seed=w.seed)
+    step_budget = float(os.environ.get("BB_REF_STEP_SECONDS", "5"))
+    for _ in range(args.warmup):
+        _oracle_sample(w, inp, ra, 0.0)
+    tot_flops, tot_s, heads, threads = 0.0, 0.0, 0, 1
+    for _ in range(args.steps):
+        f, s, hh, threads = _oracle_sample(w, inp, ra, step_budget)
+        tot_flops += f
+        tot_s += s
+        heads += hh
+    value = tot_flops / tot_s / 1e12
+    sample = f"{heads} whole (b,h) heads of {w.name} over {args.steps} steps (~{step_budget:.0f} s each)"
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": tot_s / args.steps * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+        "config": _config(w, world, "oracle on host cores; no L2 flush (CPU)"),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def _config(w, world, l2):
+    return {"workload": w.name, "B": w.B, "H": w.H, "L": w.L, "d": w.d, "block": w.block, "r": w.r,
+            "padding": "none" if w.pad is None else str(w.pad), "global_batch": w.B * world,
+            "seq_len": w.L, "parallelism": f"dp{world} (independent batches per GPU)", "l2": l2}
+
+
+def run_cuda(args):
+    import torch
+    import torch.distributed as dist
+
+    import block_sparse_long_attention_b200 as bb
+    from block_sparse_long_attention_b200.workloads import WORKLOADS, make_inputs
+
+    world, rank, local = _dist_env()
+    if world > 1:
+        from datetime import timedelta
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local if world > 1 else 0)
+    torch.cuda.set_device(dev)
+    w = WORKLOADS[args.workload]
+    inp = make_inputs(w, seed=w.seed + rank)
+    nb = w.L // w.block
+    sparse = not bb.is_fallback(w.L, w.block, w.r)
+    ra_h = bb.rand_attn_generate(w.H, w.L, w.block, w.r, seed=w.seed) if sparse else None
+
+    # device-resident inputs
+    q, k, v = (inp[x].to(dev) for x in "qkv")
+    sm = None if inp["seq_mask"] is None else inp["seq_mask"].to(dev)
+    ra = None if ra_h is None else torch.from_numpy(ra_h).to(dev)
+    out = torch.empty_like(q)
+    ws = torch.empty(max(bb.workspace_size(w.B, w.H, w.L, w.d, w.block, w.r), 1), dtype=torch.uint8, device=dev)
+    props = torch.cuda.get_device_properties(dev)
+    flush = torch.empty(2 * int(props.L2_cache_size) // 4 + (1 << 20), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        bb.fwd(q, k, v, ra, sm, block=w.block, r=w.r, out=out, workspace=ws)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize(dev)
+    if bb.device_status() != 0:
+        raise RuntimeError("device error during warm-up")
+
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    sampler = ClockSampler(dev.index if world == 1 else local)
+    sampler.start()
+    time.sleep(1.0)  # nvidia-smi start-up
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    sampler.t0 = time.time()
+    reps = max(1, int(args.repeat))
+    for _ in range(reps):
+        for i in range(args.steps):
+            flush.zero_()  # L2 flush between timed iterations (outside the events)
+            starts[i].record(stream)
+            step()
+            ends[i].record(stream)
+    torch.cuda.synchronize(dev)
+    sampler.t1 = time.time()
+    clocks = sampler.stop()
+    if world > 1:
+        dist.barrier()
+    ms = float(np.mean([s.elapsed_time(e) for s, e in zip(starts, ends)]))
+    if bb.device_status() != 0:
+        raise RuntimeError("device error during the timed region")
+
+    # end to end through the public API: pinned host inputs in, host result out
+    pin = {x: inp[x].pin_memory() for x in "qkv"}
+    sm_pin = None if inp["seq_mask"] is None else inp["seq_mask"].pin_memory()
+    ra_pin = None if ra_h is None else torch.from_numpy(ra_h).pin_memory()
+    out_pin = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    h2d = sum(pin[x].numel() * pin[x].element_size() for x in "qkv")
+    h2d += 0 if sm_pin is None else sm_pin.numel()
+    h2d += 0 if ra_pin is None else ra_pin.numel() * 4
+    d2h = out_pin.numel() * out_pin.element_size()
+
+    def e2e_step():
+        for x, dst in (("q", q), ("k", k), ("v", v)):
+            dst.copy_(pin[x], non_blocking=True)
+        if sm is not None:
+            sm.copy_(sm_pin, non_blocking=True)
+        if ra is not None:
+            ra.copy_(ra_pin, non_blocking=True)
+        step()
+        out_pin.copy_(out, non_blocking=True)
+
+    for _ in range(max(1, args.warmup)):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    e_steps = max(3, min(args.steps, 50))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e0.elapsed_time(e1) / e_steps
+
+    if world > 1:
+        t = torch.tensor([ms, e2e_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms, e2e_ms = float(t[0]), float(t[1])
+
+    import oracle  # work accounting only (FLOP count formula)
+    flops = oracle.sparse_flops(w.B, w.H, w.L, w.d, w.block, w.r)
+    value = flops * world / (ms * 1e-3) / 1e12
+    e2e_value = flops * world / (e2e_ms * 1e-3) / 1e12
+    peaks, src = _peaks()
+    peak = float(peaks["bf16_tflops"])
+    achieved = flops / (ms * 1e-3) / 1e12
+    roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+            "frac": achieved / peak, "traffic": None,
+            "kernel": "bigbird_fwd_kernel + bigbird_merge_kernel (one fwd call)",
+            "peak_source": f"{src} bf16 dense burst (kernel timed alone)"}
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": _config(w, world, "L2 flushed (2x L2 write) before every timed step"),
+        "roofline": roof,
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+                "ms_per_step": e2e_ms},
+        "gpu_launches": (2 if (sparse and bb.workspace_size(w.B, w.H, w.L) > 0) else 1) * args.steps * reps,
+        "clocks": clocks,
+    }
+    if rank == 0:
+        if world == 1 and not args.no_cpu_baseline:
+            budget = float(os.environ.get("BB_CPU_BASELINE_SECONDS", "15"))
+            ra_o = None if ra_h is None else oracle.rand_attn_generate(w.H, w.L, w.block, w.r, seed=w.seed)
+            f, s, heads, threads = _oracle_sample(w, inp, ra_o, budget)
+            line["cpu_baseline"] = {"value": f / s / 1e12, "unit": UNIT, "cores": threads, "kind": "oracle",
+                                    "sample": f"{heads} whole (b,h) heads of {w.name} ({s:.1f} s)"}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=4000)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--repeat", type=int, default=1, help="repeat the timed loop (longer clock sampling)")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_cuda(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

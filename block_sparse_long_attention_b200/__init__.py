@@ -1,0 +1,203 @@
+"""BigBird ITC block-sparse attention forward on B200 (sm_100a).
+
+Thin Python binding over the C ABI of ``libbigbird_attn.so`` (declared in
+``include/bigbird_attn.h``): argument marshalling only. Every step of the
+forward pass runs in the library's CUDA kernels; PyTorch supplies device
+memory and the current stream. There is no CPU fallback: if the library is
+missing or no sm_100 device is present the calls raise.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libbigbird_attn.so")
+
+BB_OK, BB_ERR_INVALID_ARG, BB_ERR_UNSUPPORTED, BB_ERR_CUDA, BB_ERR_BAD_RAND_ATTN, BB_ERR_DEVICE = range(6)
+BB_OUT_BF16, BB_OUT_F32 = 0, 1
+BB_FLAG_FORCE_SPARSE, BB_FLAG_DEBUG_CHECKS = 1, 2
+
+_lib = None
+
+
+class BigBirdError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {status_string(status)} ({status})")
+
+
+def _load():
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing: build it with `python -m block_sparse_long_attention_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I, U, Z, U64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_uint, ctypes.c_size_t, ctypes.c_uint64
+    sig = {
+        "bigbird_attn_fwd": (I, [P, P, P, P, P, P, I, I, I, I, I, I, P]),
+        "bigbird_attn_fwd_ex": (I, [P, P, P, P, P, P, I, I, I, I, I, I, I, U, P, Z, P]),
+        "bigbird_attn_workspace_size": (Z, [I, I, I, I, I, I, U]),
+        "bigbird_attn_is_fallback": (I, [I, I, I]),
+        "bigbird_rand_attn_generate": (I, [P, I, I, I, I, U64, I]),
+        "bigbird_rand_attn_validate": (I, [P, I, I, I, I, I]),
+        "bigbird_mask_prep": (I, [P, I, I, I, P, P, P, P]),
+        "bigbird_pattern_table": (I, [P, I, I, I, I, P]),
+        "bigbird_device_status": (I, [P, ctypes.POINTER(ctypes.c_uint32)]),
+        "bigbird_status_string": (ctypes.c_char_p, [I]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype, fn.argtypes = res, args
+    _lib = lib
+    return lib
+
+
+def lib():
+    """The loaded ctypes library (raises ImportError if it is not built)."""
+    return _load()
+
+
+def status_string(status: int) -> str:
+    return _load().bigbird_status_string(int(status)).decode()
+
+
+def _check(status: int, what: str):
+    if status != BB_OK:
+        raise BigBirdError(status, what)
+
+
+def _np_ptr(a: np.ndarray):
+    return ctypes.c_void_p(a.ctypes.data)
+
+
+# ------------------------------------------------------------------ host prep
+
+def is_fallback(L: int, block: int = 64, r: int = 3) -> bool:
+    res = _load().bigbird_attn_is_fallback(L, block, r)
+    if res < 0:
+        raise BigBirdError(BB_ERR_INVALID_ARG, "is_fallback")
+    return bool(res)
+
+
+def rand_attn_generate(H: int, L: int, block: int = 64, r: int = 3, seed: int = 0, last_idx: int = 0) -> np.ndarray:
+    """Seeded random adjacency int32 [H, nb-2, r] (host)."""
+    nb = L // block if block > 0 else 0
+    out = np.empty((H, max(nb - 2, 0), r), dtype=np.int32)
+    _check(_load().bigbird_rand_attn_generate(_np_ptr(out), H, L, block, r, seed & (2**64 - 1), last_idx),
+           "rand_attn_generate")
+    return out
+
+
+def rand_attn_validate(rand_attn, H: int, L: int, block: int = 64, r: int = 3, last_idx: int = 0) -> int:
+    """Status of the generator-rule check of a host rand_attn (BB_OK or an error code)."""
+    ra = np.ascontiguousarray(rand_attn, dtype=np.int32)
+    nb = L // block
+    if ra.shape != (H, nb - 2, r):
+        return BB_ERR_INVALID_ARG
+    return _load().bigbird_rand_attn_validate(_np_ptr(ra), H, L, block, r, last_idx)
+
+
+def mask_prep(seq_mask, block: int = 64):
+    """(blocked [B,nb,bs], band [B,nb-4,bs,3bs], from_mask [B,L], to_mask [B,L]) uint8."""
+    m = np.ascontiguousarray(np.asarray(seq_mask), dtype=np.uint8)
+    B, L = m.shape
+    nb = L // block
+    blocked = np.empty((B, nb, block), np.uint8)
+    band = np.empty((B, max(nb - 4, 0), block, 3 * block), np.uint8)
+    frm = np.empty((B, L), np.uint8)
+    to = np.empty((B, L), np.uint8)
+    _check(_load().bigbird_mask_prep(_np_ptr(m), B, L, block, _np_ptr(blocked), _np_ptr(band), _np_ptr(frm),
+                                     _np_ptr(to)), "mask_prep")
+    return blocked, band, frm, to
+
+
+def pattern_table(rand_attn, H: int, L: int, block: int = 64, r: int = 3) -> np.ndarray:
+    """Sorted distinct key blocks per non-global query block: int32 [H, nb-2, 5+r], -1 padded."""
+    ra = np.ascontiguousarray(rand_attn, dtype=np.int32)
+    nb = L // block
+    out = np.empty((H, nb - 2, 5 + r), np.int32)
+    _check(_load().bigbird_pattern_table(_np_ptr(ra), H, L, block, r, _np_ptr(out)), "pattern_table")
+    return out
+
+
+# ------------------------------------------------------------------ forward
+
+def workspace_size(B: int, H: int, L: int, d: int = 64, block: int = 64, r: int = 3, force_sparse: bool = False) -> int:
+    flags = BB_FLAG_FORCE_SPARSE if force_sparse else 0
+    return int(_load().bigbird_attn_workspace_size(B, H, L, d, block, r, flags))
+
+
+def _stream_handle(stream):
+    import torch
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def fwd(q, k, v, rand_attn, seq_mask=None, *, block: int = 64, r: int = 3, out=None, out_dtype=None,
+        force_sparse: bool = False, debug_checks: bool = False, workspace=None, stream=None):
+    """BigBird ITC attention forward: returns out [B, H, L, d] (bf16, or fp32
+    with out_dtype=torch.float32). q, k, v: contiguous bf16 CUDA tensors
+    [B, H, L, d]; rand_attn: int32 CUDA tensor [H, nb-2, r] (or None in the
+    full-attention fallback); seq_mask: uint8 CUDA tensor [B, L] (1 = valid
+    key) or None. Runs on the current torch stream (or `stream`)."""
+    import torch
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if not (t.is_cuda and t.dtype == torch.bfloat16 and t.is_contiguous() and t.dim() == 4):
+            raise ValueError(f"{name} must be a contiguous bf16 CUDA tensor [B, H, L, d]")
+    B, H, L, d = q.shape
+    if k.shape != q.shape or v.shape != q.shape:
+        raise ValueError("q, k, v shapes differ")
+    if out_dtype is None:
+        out_dtype = torch.bfloat16 if out is None else out.dtype
+    if out_dtype not in (torch.bfloat16, torch.float32):
+        raise ValueError("out_dtype must be bf16 or fp32")
+    if out is None:
+        out = torch.empty((B, H, L, d), dtype=out_dtype, device=q.device)
+    elif not (out.is_cuda and out.dtype == out_dtype and out.is_contiguous() and out.shape == q.shape):
+        raise ValueError("out must be a contiguous CUDA tensor of q's shape and out_dtype")
+    ra_ptr = None
+    if rand_attn is not None:
+        if not (rand_attn.is_cuda and rand_attn.dtype == torch.int32 and rand_attn.is_contiguous()):
+            raise ValueError("rand_attn must be a contiguous int32 CUDA tensor [H, nb-2, r]")
+        if rand_attn.shape != (H, L // block - 2, r):
+            raise ValueError(f"rand_attn shape {tuple(rand_attn.shape)} != {(H, L // block - 2, r)}")
+        ra_ptr = rand_attn.data_ptr()
+    sm_ptr = None
+    if seq_mask is not None:
+        if not (seq_mask.is_cuda and seq_mask.dtype == torch.uint8 and seq_mask.is_contiguous()
+                and seq_mask.shape == (B, L)):
+            raise ValueError("seq_mask must be a contiguous uint8 CUDA tensor [B, L]")
+        sm_ptr = seq_mask.data_ptr()
+    flags = (BB_FLAG_FORCE_SPARSE if force_sparse else 0) | (BB_FLAG_DEBUG_CHECKS if debug_checks else 0)
+    lib_ = _load()
+    ws_bytes = int(lib_.bigbird_attn_workspace_size(B, H, L, d, block, r, flags))
+    ws_ptr = None
+    if ws_bytes:
+        if workspace is None or workspace.numel() * workspace.element_size() < ws_bytes:
+            workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
+        ws_ptr = workspace.data_ptr()
+    st = lib_.bigbird_attn_fwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), ra_ptr, sm_ptr, out.data_ptr(),
+                                  B, H, L, d, block, r, BB_OUT_F32 if out_dtype == torch.float32 else BB_OUT_BF16,
+                                  flags, ws_ptr, ws_bytes, _stream_handle(stream))
+    _check(st, "bigbird_attn_fwd_ex")
+    return out
+
+
+def device_status(stream=None) -> int:
+    """Synchronise the stream, then read and clear the device error word
+    (bit 1: out-of-range rand_attn entry skipped; bit 2: a kernel wait timed out)."""
+    v = ctypes.c_uint32(0)
+    _check(_load().bigbird_device_status(_stream_handle(stream), ctypes.byref(v)), "device_status")
+    return int(v.value)
+
+
+__all__ = [
+    "BigBirdError", "fwd", "workspace_size", "is_fallback", "rand_attn_generate", "rand_attn_validate",
+    "mask_prep", "pattern_table", "device_status", "status_string", "lib", "LIB_PATH",
+]

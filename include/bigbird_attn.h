@@ -1,0 +1,176 @@
+/*
+ * bigbird_attn.h -- C ABI of the B200 (sm_100a) BigBird ITC block-sparse
+ * attention forward pass and its host-side preparation routines.
+ *
+ * Pages cited below:
+ *   [TFG-BigBird] "models 仓库中的 BigBird：线性复杂度稀疏注意力与长序列训练的完整实践"
+ *                 (TensorFlow Model Garden official/projects/bigbird)
+ *   [HF-Pegasus]  "BigBirdPegasus 长序列条件生成模型详解从稀疏注意力原理到 Transformers 实战"
+ *                 (Hugging Face modeling_bigbird_pegasus.py)
+ *
+ * Conventions for every entry point:
+ *   - Tensors are dense, row-major, with no padding between rows.
+ *     Q, K, V, O: [B, H, L, d]; seq_mask: [B, L]; rand_attn: [H, nb-2, r],
+ *     where nb = L / block.
+ *   - "device" pointers are CUDA global memory of the current device;
+ *     "host" pointers are ordinary CPU memory. The caller owns every buffer;
+ *     no function keeps a pointer after it returns.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default
+ *     stream). Device work is enqueued asynchronously on it; no entry point
+ *     synchronises the stream unless its comment says so.
+ *   - Return value: a bb_status. On any error nothing is launched and no
+ *     output is written, except BB_ERR_CUDA after a launch.
+ */
+#ifndef BIGBIRD_ATTN_H
+#define BIGBIRD_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  BB_OK = 0,
+  BB_ERR_INVALID_ARG = 1,   /* NULL pointer, non-positive size, L % block != 0, r < 1 */
+  BB_ERR_UNSUPPORTED = 2,   /* d != 64 or block != 64, misaligned pointer, no sm_100 device */
+  BB_ERR_CUDA = 3,          /* a CUDA runtime call or launch failed */
+  BB_ERR_BAD_RAND_ATTN = 4, /* rand_attn breaks the generator's rules (validator / debug checks) */
+  BB_ERR_DEVICE = 5         /* a kernel reported a device-side error (see bigbird_device_status) */
+} bb_status;
+
+/* Output element type of the forward pass. */
+enum { BB_OUT_BF16 = 0, BB_OUT_F32 = 1 };
+
+/* Flags of bigbird_attn_fwd_ex. */
+enum {
+  /* Use the sparse pattern even when nb <= 5 + 2r (requires nb >= 5 + r). */
+  BB_FLAG_FORCE_SPARSE = 1u,
+  /* Copy rand_attn to the host and validate it before launching; synchronises the stream. */
+  BB_FLAG_DEBUG_CHECKS = 2u
+};
+
+/*
+ * bigbird_attn_fwd -- BigBird ITC block-sparse attention forward, bf16 in, bf16 out.
+ *
+ * For every (b, h) and query block i (rows i*block .. i*block+block-1):
+ *   - i = 0 and i = nb-1 attend to all L keys (global rows)
+ *     [TFG-BigBird, section "BigBird：从二次方注意力到线性稀疏注意力"; HF-Pegasus,
+ *     section "三类注意力组合"];
+ *   - every other i attends to key blocks {0, nb-1} (global), {i-1, i, i+1}
+ *     (sliding window) and rand_attn[h][i-1][0..r) (random)
+ *     [same sections; TFG-BigBird, section "随机块掩码是如何生成的"].
+ * The key set of a row is a set: a random entry equal to a window or global
+ * block, or repeated, adds nothing. Scores are (q . k) / sqrt(d), plus -10000
+ * for keys with seq_mask == 0 [TFG-BigBird, "BigBird：从二次方注意力到线性稀疏注意力"];
+ * out = softmax(scores) . V with fp32 accumulation.
+ * If nb <= 5 + 2r the call computes full attention and ignores rand_attn
+ * [HF-Pegasus, section "序列过短时的自动回退"].
+ *
+ *   q, k, v    device, bf16 [B, H, L, d], 16-byte aligned.
+ *   rand_attn  device, int32 [H, nb-2, r]; entries must lie in [0, nb) (an
+ *              entry outside is skipped and flagged in bigbird_device_status).
+ *              May be NULL only in the full-attention fallback.
+ *   seq_mask   device, uint8 [B, L], nonzero = valid key; NULL = all valid.
+ *   out        device, bf16 [B, H, L, d], 16-byte aligned; must not alias q/k/v.
+ *   B, H, L, d, block, r  sizes; v1 supports d = 64 and block = 64 only.
+ *   stream     cudaStream_t.
+ * Errors: BB_ERR_INVALID_ARG for L % block != 0 [HF-Pegasus, section
+ * "序列长度的块对齐要求"] or r < 1 [HF-Pegasus, section "使用限制与注意事项"];
+ * BB_ERR_UNSUPPORTED for other d/block or misalignment. Scratch memory for
+ * the split global rows, when needed, is taken with cudaMallocAsync on
+ * `stream` and released the same way.
+ */
+int bigbird_attn_fwd(const void* q, const void* k, const void* v, const int32_t* rand_attn,
+                     const uint8_t* seq_mask, void* out, int B, int H, int L, int d, int block, int r,
+                     void* stream);
+
+/*
+ * Bytes of device scratch bigbird_attn_fwd_ex needs for these sizes and
+ * flags (0 when none). The scratch holds the partial (unnormalised output,
+ * running max, running sum) of each key range of the split global rows.
+ */
+size_t bigbird_attn_workspace_size(int B, int H, int L, int d, int block, int r, unsigned flags);
+
+/*
+ * bigbird_attn_fwd_ex -- bigbird_attn_fwd with an output type, flags and an
+ * optional caller-provided workspace.
+ *   out_dtype  BB_OUT_BF16 (out is bf16) or BB_OUT_F32 (out is fp32 [B,H,L,d]).
+ *   flags      BB_FLAG_* bits.
+ *   workspace  device, 256-byte aligned, at least
+ *              bigbird_attn_workspace_size(...) bytes; NULL = allocate with
+ *              cudaMallocAsync on `stream` when needed. Calls that share a
+ *              workspace must not overlap on the GPU.
+ */
+int bigbird_attn_fwd_ex(const void* q, const void* k, const void* v, const int32_t* rand_attn,
+                        const uint8_t* seq_mask, void* out, int B, int H, int L, int d, int block, int r,
+                        int out_dtype, unsigned flags, void* workspace, size_t workspace_bytes, void* stream);
+
+/* 1 if (L, block, r) runs full attention (nb <= 5 + 2r), 0 if sparse, <0 on
+ * invalid sizes [HF-Pegasus, section "序列过短时的自动回退"]. */
+int bigbird_attn_is_fallback(int L, int block, int r);
+
+/*
+ * bigbird_rand_attn_generate -- seeded random adjacency (host).
+ *   host_out  host, int32 [H, nb-2, r]; row i-1 holds query block i's random blocks.
+ * Row i draws a uniformly random r-subset, in random order, of its candidate
+ * pool: blocks 1..nb-2 without i-1, i, i+1 [TFG-BigBird, section
+ * "随机块掩码是如何生成的"]; with last_idx > 0 only blocks j with
+ * (j+1)*block <= last_idx qualify (the page's last_idx = 1024 cap; 0 = off).
+ * The draw is a partial Fisher-Yates shuffle of the ascending pool; draw t of
+ * row (h, i) takes the SplitMix64 output of state `seed` at counter
+ * ((h*(nb-2) + i-1) << 20) + 1 + t' (t' counts the row's draws, rejections
+ * included), bounded without bias by rejecting u < (2^64 - n) mod n.
+ * Deterministic for a given seed; heads get distinct streams.
+ * Errors: BB_ERR_INVALID_ARG for bad sizes or a row with fewer than r candidates.
+ */
+int bigbird_rand_attn_generate(int32_t* host_out, int H, int L, int block, int r, uint64_t seed, int last_idx);
+
+/*
+ * bigbird_rand_attn_validate -- check a host rand_attn [H, nb-2, r] against the
+ * generator's rules: every entry a candidate of its row (range, not in the
+ * row's window or global blocks, before last_idx when > 0) and no repeats
+ * within a row [TFG-BigBird, section "随机块掩码是如何生成的"].
+ * Returns BB_OK or BB_ERR_BAD_RAND_ATTN (BB_ERR_INVALID_ARG for bad sizes).
+ */
+int bigbird_rand_attn_validate(const int32_t* host_ra, int H, int L, int block, int r, int last_idx);
+
+/*
+ * bigbird_mask_prep -- the BigBirdMasks tensors from a [B, L] mask (host)
+ * [TFG-BigBird, section "随机块掩码是如何生成的", the four-mask tuple]:
+ *   blocked   host uint8 [B, nb, block]          seq_mask cut into blocks
+ *   band      host uint8 [B, nb-4, block, 3*block]
+ *             band[b, i-2, x, w*block + y] = m[b, i*block + x] * m[b, (i-1+w)*block + y]
+ *             for middle query block i in [2, nb-3], window slot w in {0,1,2}
+ *   from_mask host uint8 [B, L] (query side), to_mask host uint8 [B, L] (key side)
+ * Output values are 0/1. Any output pointer may be NULL to skip it. Requires nb >= 4.
+ */
+int bigbird_mask_prep(const uint8_t* seq_mask, int B, int L, int block, uint8_t* blocked, uint8_t* band,
+                      uint8_t* from_mask, uint8_t* to_mask);
+
+/*
+ * bigbird_pattern_table -- the sparse pattern as lists (host):
+ *   out  host int32 [H, nb-2, 5+r]; row i-1 lists query block i's distinct key
+ *        blocks in ascending order, padded with -1. Rows 0 and nb-1 attend to
+ *        every block and are not listed.
+ * Entries of host_ra outside [0, nb) give BB_ERR_BAD_RAND_ATTN.
+ */
+int bigbird_pattern_table(const int32_t* host_ra, int H, int L, int block, int r, int32_t* out);
+
+/*
+ * bigbird_device_status -- read and clear the library's device error word
+ * after synchronising `stream`. Bit 1: a rand_attn entry outside [0, nb) was
+ * skipped; bit 2: a kernel wait timed out (a lost completion). *host_status
+ * receives the word. Returns BB_OK, or BB_ERR_CUDA if the copy failed.
+ */
+int bigbird_device_status(void* stream, uint32_t* host_status);
+
+/* Static, human-readable text of a bb_status. */
+const char* bigbird_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BIGBIRD_ATTN_H */
