@@ -55,7 +55,6 @@ constexpr uint32_t kTileBytes = kBlock * kHeadDim * 2;  // one 64x64 bf16 tile
 constexpr uint32_t kTmemCols = 256;
 constexpr uint32_t kColO = 128;        // O accumulator columns [128, 192)
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr float kMaskedBiasLog2 = -10000.0f * kLog2e;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr float kNegInit = -1.0e30f;
 
@@ -93,15 +92,16 @@ struct FwdParams {
   int total_units;
   int out_f32;
   float scale_log2;  // log2(e) / sqrt(d)
+  float bias_raw;    // -10000 * sqrt(d): the masked-key bias in units of q.k
 };
 
 struct __align__(1024) SharedStorage {
   uint8_t q[2][kRows * kHeadDim * 2];   // 2 x 16 KB, SW128, 1024-aligned
   uint8_t k[kStages][kTileBytes];       // 8 KB each
   uint8_t v[kStages][kTileBytes];
-  UnitInfo unit[2];
+  UnitInfo unit[4];
   uint64_t q_full[2];
-  uint64_t slot_free[2];
+  uint64_t q_free[2];
   uint64_t kv_full[kStages];
   uint64_t kv_empty[kStages];
   uint64_t s_full[2];
@@ -128,8 +128,9 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity) {
   return __all_sync(0xffffffffu, mbar_wait(bar, parity));
 }
 
-// Decode unit u and build its key-block list (one thread).
-__device__ void build_unit(const FwdParams& p, int u, UnitInfo& ui) {
+// Decode unit u and build its key-block list. Called by a whole warp: the
+// lanes fetch the unit's random entries in parallel, lane 0 builds the list.
+__device__ void build_unit(const FwdParams& p, int u, UnitInfo& ui, int lane) {
   int n = 0;
   auto add = [&](int kb, int hm) {
     if (kb < 0 || kb >= p.nb) {
@@ -161,13 +162,16 @@ __device__ void build_unit(const FwdParams& p, int u, UnitInfo& ui) {
       qtop = 2 * pp;
       qbot = 2 * pp + 1 < p.nb ? 2 * pp + 1 : -1;
     }
-    const int k0 = s * p.split_blocks;
-    const int k1 = min(p.nb, k0 + p.split_blocks);
-    for (int kb = k0; kb < k1; ++kb) add(kb, 3);
-    ui.bh = bh;
-    ui.qtop = qtop;
-    ui.qbot = qbot;
-    ui.split = p.nsplit > 1 ? s : -1;
+    if (lane == 0) {
+      const int k0 = s * p.split_blocks;
+      const int k1 = min(p.nb, k0 + p.split_blocks);
+      for (int kb = k0; kb < k1; ++kb) add(kb, 3);
+      ui.bh = bh;
+      ui.qtop = qtop;
+      ui.qbot = qbot;
+      ui.split = p.nsplit > 1 ? s : -1;
+      ui.n = n;
+    }
   } else {
     const int v = u - p.n_glob_units;
     const int bh = v / p.n_pairs;
@@ -176,79 +180,115 @@ __device__ void build_unit(const FwdParams& p, int u, UnitInfo& ui) {
     const int qbot = (2 + 2 * pp <= p.nb - 2) ? 2 + 2 * pp : -1;
     const int h = bh % p.H;
     const int both = qbot >= 0 ? 3 : 1;
-    add(qtop - 1, 1);
-    add(qtop, both);
-    add(qtop + 1, both);
-    if (qbot >= 0) add(qtop + 2, 2);
-    add(0, both);
-    add(p.nb - 1, both);
+    // rand_attn rows qtop-1 and qtop (= qbot-1) are adjacent: lane t < r reads
+    // the top row's entry t, lane r + t the bottom row's entry t.
+    const int nrand = qbot >= 0 ? 2 * p.r : p.r;
     const int32_t* ra = p.rand_attn + (static_cast<size_t>(h) * (p.nb - 2) + (qtop - 1)) * p.r;
-    for (int t = 0; t < p.r; ++t) add(__ldg(ra + t), 1);
-    if (qbot >= 0)
-      for (int t = 0; t < p.r; ++t) add(__ldg(ra + p.r + t), 2);
-    ui.bh = bh;
-    ui.qtop = qtop;
-    ui.qbot = qbot;
-    ui.split = -1;
+    const int rv = lane < nrand ? __ldg(ra + lane) : -1;
+    if (lane == 0) {
+      add(qtop - 1, 1);
+      add(qtop, both);
+      add(qtop + 1, both);
+      if (qbot >= 0) add(qtop + 2, 2);
+      add(0, both);
+      add(p.nb - 1, both);
+    }
+    for (int t = 0; t < nrand; ++t) {
+      const int x = __shfl_sync(0xffffffffu, rv, t);
+      if (lane == 0) add(x, t < p.r ? 1 : 2);
+    }
+    if (lane == 0) {
+      ui.bh = bh;
+      ui.qtop = qtop;
+      ui.qbot = qbot;
+      ui.split = -1;
+      ui.n = n;
+    }
   }
-  ui.n = n;
+}
+
+// 64 validity bits of key block kb of batch b (bit c: seq_mask of key c != 0).
+__device__ __forceinline__ uint64_t key_valid_bits(const uint8_t* seq_mask, int L, int b, int kb) {
+  const uint4* src = reinterpret_cast<const uint4*>(seq_mask + static_cast<size_t>(b) * L + static_cast<size_t>(kb) * kBlock);
+  uint64_t bits = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint4 w = __ldg(src + i);
+    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      // one bit per byte (byte != 0), packed into 4 bits by a carry-free multiply
+      const uint32_t m = __vcmpne4(ws[j], 0u) & 0x01010101u;
+      bits |= static_cast<uint64_t>((m * 0x01020408u) >> 24) << (16 * i + 4 * j);
+    }
+  }
+  return bits;
 }
 
 // ---------------------------------------------------------------- producer
 
+// Prepare unit u's info (list, half masks, key validity bits). Whole warp.
+__device__ void prep_unit(const FwdParams& p, int u, UnitInfo& ui, int lane) {
+  build_unit(p, u, ui, lane);
+  __syncwarp();
+  const int n = ui.n;
+  const int b = ui.bh / p.H;
+  // Key validity bits: lane e handles list entries e and e + 32.
+  for (int e = lane; e < n; e += 32)
+    ui.vm[e] = p.seq_mask ? key_valid_bits(p.seq_mask, p.L, b, ui.kb[e]) : ~0ull;
+  __syncwarp();
+}
+
+// The next unit's info is prepared while the current unit's first K/V tiles
+// are in flight, so the list-building loads never stall the TMA ring at a
+// unit boundary. Four info slots: a slot is rewritten three units after its
+// last use, when every consumer is provably done with it.
 __device__ void producer_role(SharedStorage& s, const FwdParams& p, const CUtensorMap* tmQ, const CUtensorMap* tmK,
                               const CUtensorMap* tmV) {
   const int lane = threadIdx.x & 31;
   const uint64_t pol_kv = l2_policy_evict_last();
   const uint64_t pol_q = l2_policy_evict_first();
   uint32_t unit_it = 0, kv_it = 0;
-  for (int u = blockIdx.x; u < p.total_units; u += gridDim.x, ++unit_it) {
-    const int slot = unit_it & 1;
+  int u = blockIdx.x;
+  if (u < p.total_units) prep_unit(p, u, s.unit[0], lane);
+  for (; u < p.total_units; u += gridDim.x, ++unit_it) {
+    const int qs = unit_it & 1;
     const uint32_t ph = (unit_it >> 1) & 1;
-    if (lane == 0) {
-      if (!mbar_wait(smem_u32(&s.slot_free[slot]), ph ^ 1)) flag_timeout(s, p);
+    const UnitInfo& ui = s.unit[unit_it & 3];
+    int ok = 1;
+    if (lane == 0) ok = mbar_wait(smem_u32(&s.q_free[qs]), ph ^ 1);
+    if (!__shfl_sync(0xffffffffu, ok, 0)) {
+      if (lane == 0) flag_timeout(s, p);
+      return;
     }
-    __syncwarp();
-    if (aborted(s)) return;
-    UnitInfo& ui = s.unit[slot];
-    if (lane == 0) build_unit(p, u, ui);
-    __syncwarp();
     const int n = ui.n;
-    const int b = ui.bh / p.H;
-    // Key validity bits: lane l reads keys l and l+32 of each listed block.
-    for (int e = 0; e < n; ++e) {
-      uint64_t vm = ~0ull;
-      if (p.seq_mask) {
-        const uint8_t* m = p.seq_mask + static_cast<size_t>(b) * p.L + static_cast<size_t>(ui.kb[e]) * kBlock;
-        const uint32_t lo = __ballot_sync(0xffffffffu, __ldg(m + lane) != 0);
-        const uint32_t hi = __ballot_sync(0xffffffffu, __ldg(m + 32 + lane) != 0);
-        vm = (static_cast<uint64_t>(hi) << 32) | lo;
-      }
-      if (lane == 0) ui.vm[e] = vm;
-    }
-    __syncwarp();
+    const int32_t row0 = ui.bh * p.L;
+    const int nxt = u + gridDim.x;
+    const int prep_at = min(n, kStages) - 1;
     if (lane == 0) {
-      const int32_t row0 = ui.bh * p.L;
-      const uint32_t qbar = smem_u32(&s.q_full[slot]);
+      const uint32_t qbar = smem_u32(&s.q_full[qs]);
       mbar_arrive_expect_tx(qbar, ui.qbot >= 0 ? 2 * kTileBytes : kTileBytes);
-      tma_load_2d(smem_u32(s.q[slot]), tmQ, qbar, 0, row0 + ui.qtop * kBlock, pol_q);
-      if (ui.qbot >= 0) tma_load_2d(smem_u32(s.q[slot]) + kTileBytes, tmQ, qbar, 0, row0 + ui.qbot * kBlock, pol_q);
-      for (int j = 0; j < n; ++j, ++kv_it) {
-        const int st = kv_it % kStages;
-        const uint32_t kph = (kv_it / kStages) & 1;
-        if (!mbar_wait(smem_u32(&s.kv_empty[st]), kph ^ 1)) {
-          flag_timeout(s, p);
-          break;
-        }
-        const uint32_t kbar = smem_u32(&s.kv_full[st]);
-        mbar_arrive_expect_tx(kbar, 2 * kTileBytes);
-        const int32_t krow = row0 + ui.kb[j] * kBlock;
-        tma_load_2d(smem_u32(s.k[st]), tmK, kbar, 0, krow, pol_kv);
-        tma_load_2d(smem_u32(s.v[st]), tmV, kbar, 0, krow, pol_kv);
-      }
+      tma_load_2d(smem_u32(s.q[qs]), tmQ, qbar, 0, row0 + ui.qtop * kBlock, pol_q);
+      if (ui.qbot >= 0) tma_load_2d(smem_u32(s.q[qs]) + kTileBytes, tmQ, qbar, 0, row0 + ui.qbot * kBlock, pol_q);
     }
-    __syncwarp();
-    if (aborted(s)) return;
+    for (int j = 0; j < n; ++j, ++kv_it) {
+      if (lane == 0) {
+        const int st = kv_it % kStages;
+        ok = mbar_wait(smem_u32(&s.kv_empty[st]), ((kv_it / kStages) & 1) ^ 1);
+        if (ok) {
+          const uint32_t kbar = smem_u32(&s.kv_full[st]);
+          mbar_arrive_expect_tx(kbar, 2 * kTileBytes);
+          const int32_t krow = row0 + ui.kb[j] * kBlock;
+          tma_load_2d(smem_u32(s.k[st]), tmK, kbar, 0, krow, pol_kv);
+          tma_load_2d(smem_u32(s.v[st]), tmV, kbar, 0, krow, pol_kv);
+        }
+      }
+      if (!__shfl_sync(0xffffffffu, ok, 0)) {
+        if (lane == 0) flag_timeout(s, p);
+        return;
+      }
+      if (j == prep_at && nxt < p.total_units) prep_unit(p, nxt, s.unit[(unit_it + 1) & 3], lane);
+    }
   }
 }
 
@@ -256,14 +296,17 @@ __device__ void producer_role(SharedStorage& s, const FwdParams& p, const CUtens
 
 __device__ void mma_role(SharedStorage& s, const FwdParams& p, uint32_t tmem) {
   const uint32_t idesc_s = idesc_bf16_f32(kRows, kBlock, false);
-  const uint32_t idesc_o = idesc_bf16_f32(kRows, kHeadDim, true);
+  // P.V runs in fp16: P is written as fp16 and V is converted to fp16 in shared
+  // memory (exact for bf16 values in the fp16 normal range); fp16 keeps three
+  // more mantissa bits of P than bf16 would.
+  const uint32_t idesc_o = idesc_f32acc(kRows, kHeadDim, false, true);
   uint32_t unit_it = 0, kv_it = 0, g = 0;
   bool ok = true;
   for (int u = blockIdx.x; u < p.total_units && ok; u += gridDim.x, ++unit_it) {
     const int slot = unit_it & 1;
     const uint32_t ph = (unit_it >> 1) & 1;
     if (!mbar_wait(smem_u32(&s.q_full[slot]), ph)) { ok = false; break; }
-    const int n = s.unit[slot].n;
+    const int n = s.unit[unit_it & 3].n;
     const uint32_t q_addr = smem_u32(s.q[slot]);
 
     auto issue_pv = [&](int jj) -> bool {
@@ -304,7 +347,7 @@ __device__ void mma_role(SharedStorage& s, const FwdParams& p, uint32_t tmem) {
     }
     if (!ok) break;
     if (n > 0 && !issue_pv(n - 1)) { ok = false; break; }
-    mma_commit(smem_u32(&s.slot_free[slot]));
+    mma_commit(smem_u32(&s.q_free[slot]));
     mma_commit(smem_u32(&s.o_full));
     kv_it += n;
     g += n;
@@ -333,7 +376,7 @@ __device__ void softmax_role(SharedStorage& s, const FwdParams& p, uint32_t tmem
     const int slot = unit_it & 1;
     const uint32_t ph = (unit_it >> 1) & 1;
     if (!warp_wait(smem_u32(&s.q_full[slot]), ph)) { flag_timeout(s, p); return; }
-    const UnitInfo& ui = s.unit[slot];
+    const UnitInfo& ui = s.unit[unit_it & 3];
     const int n = ui.n;
     const int bh = ui.bh;
     const int qblk = half ? ui.qbot : ui.qtop;
@@ -349,7 +392,7 @@ __device__ void softmax_role(SharedStorage& s, const FwdParams& p, uint32_t tmem
       const bool used = exists && ((ui.hm[j] >> half) & 1);
       uint32_t pk[32];
       if (used) {
-        float x[64];
+        float x[64];  // raw scores q.k (+ the masked-key bias in the same units)
         {
           uint32_t r0[32], r1[32];
           tmem_ld32(tmem + lane_addr + sb * 64, r0);
@@ -357,21 +400,21 @@ __device__ void softmax_role(SharedStorage& s, const FwdParams& p, uint32_t tmem
           tmem_wait_ld();
 #pragma unroll
           for (int c = 0; c < 32; ++c) {
-            x[c] = __uint_as_float(r0[c]) * p.scale_log2;
-            x[32 + c] = __uint_as_float(r1[c]) * p.scale_log2;
+            x[c] = __uint_as_float(r0[c]);
+            x[32 + c] = __uint_as_float(r1[c]);
           }
         }
         const uint64_t vm = ui.vm[j];
         if (vm != ~0ull) {
 #pragma unroll
-          for (int c = 0; c < 64; ++c) x[c] += ((vm >> c) & 1ull) ? 0.f : kMaskedBiasLog2;
+          for (int c = 0; c < 64; ++c) x[c] += ((vm >> c) & 1ull) ? 0.f : p.bias_raw;
         }
         float mx;
         {
           float t[16];
 #pragma unroll
           for (int c = 0; c < 16; ++c) t[c] = fmaxf(fmaxf(x[c], x[16 + c]), fmaxf(x[32 + c], x[48 + c]));
-          mx = fmax_tree(t);
+          mx = fmax_tree(t) * p.scale_log2;
         }
         float factor = 1.f;
         bool rescale_o = false;
@@ -380,13 +423,14 @@ __device__ void softmax_role(SharedStorage& s, const FwdParams& p, uint32_t tmem
           rescale_o = l_run > 0.f;
           m_ref = mx;
         }
+        const float neg_m = -m_ref;
         float sum = 0.f;
 #pragma unroll
         for (int c = 0; c < 32; ++c) {
-          const float e0 = ex2_approx(x[2 * c] - m_ref);
-          const float e1 = ex2_approx(x[2 * c + 1] - m_ref);
+          const float e0 = ex2_approx(fmaf(x[2 * c], p.scale_log2, neg_m));
+          const float e1 = ex2_approx(fmaf(x[2 * c + 1], p.scale_log2, neg_m));
           sum += e0 + e1;
-          pk[c] = pack_bf16x2(e0, e1);
+          pk[c] = pack_f16x2(e0, e1);
         }
         l_run = l_run * factor + sum;
         if (__any_sync(0xffffffffu, rescale_o)) {
@@ -408,6 +452,23 @@ __device__ void softmax_role(SharedStorage& s, const FwdParams& p, uint32_t tmem
 #pragma unroll
         for (int c = 0; c < 32; ++c) pk[c] = 0u;
       }
+      {
+        // Convert this thread's 64-byte slice of V_j to fp16 in place (the
+        // block counter is also the K/V ring counter).
+        const int st = gg % kStages;
+        if (!warp_wait(smem_u32(&s.kv_full[st]), (gg / kStages) & 1)) { flag_timeout(s, p); return; }
+        uint4* vp = reinterpret_cast<uint4*>(s.v[st]) + tid * 4;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          uint4 w = vp[i];
+          w.x = bf16x2_to_f16x2(w.x);
+          w.y = bf16x2_to_f16x2(w.y);
+          w.z = bf16x2_to_f16x2(w.z);
+          w.w = bf16x2_to_f16x2(w.w);
+          vp[i] = w;
+        }
+        fence_proxy_async_smem();
+      }
       tmem_st32(tmem + lane_addr + sb * 64, pk);
       tmem_wait_st();
       tc_fence_before();
@@ -426,7 +487,6 @@ __device__ void softmax_role(SharedStorage& s, const FwdParams& p, uint32_t tmem
     __syncwarp();
     if (lane == 0) {
       mbar_arrive(smem_u32(&s.o_free));
-      mbar_arrive(smem_u32(&s.slot_free[slot]));
     }
     if (exists) {
       const int row_in_blk = tid & 63;
@@ -490,7 +550,7 @@ bigbird_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
   if (threadIdx.x == 0) {
     for (int i = 0; i < 2; ++i) {
       mbar_init(smem_u32(&s.q_full[i]), 1);
-      mbar_init(smem_u32(&s.slot_free[i]), 1 + 4);
+      mbar_init(smem_u32(&s.q_free[i]), 1);
       mbar_init(smem_u32(&s.s_full[i]), 1);
       mbar_init(smem_u32(&s.p_full[i]), 4);
       mbar_init(smem_u32(&s.pv_done[i]), 1);
@@ -530,52 +590,43 @@ bigbird_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
   }
 }
 
-// Combine the partial results of the key ranges of the global rows: one
-// thread per query row of a unit, log-sum-exp weights in log2 units.
-__global__ void __launch_bounds__(kRows)
+// Combine the partial results of the key ranges of the global rows by
+// log-sum-exp (log2 units). 16 threads per query row, 4 columns each; a CTA
+// covers 16 rows, grid = (B*H, 128 / 16).
+constexpr int kMergeRowsPerCta = 16;
+
+__global__ void __launch_bounds__(256)
 bigbird_merge_kernel(const float* __restrict__ part_o, const float* __restrict__ part_ml, void* out, int nsplit,
                      int L, int nb, int out_f32) {
   const int bh = blockIdx.x;
-  const int row = threadIdx.x;
+  const int row = blockIdx.y * kMergeRowsPerCta + (threadIdx.x >> 4);
+  const int c4 = threadIdx.x & 15;
   const size_t base = static_cast<size_t>(bh) * nsplit * kRows + row;
   const float2* ml = reinterpret_cast<const float2*>(part_ml);
   float mmax = kNegInit;
-  for (int s = 0; s < nsplit; ++s) mmax = fmaxf(mmax, ml[base + static_cast<size_t>(s) * kRows].x);
-  float acc[kHeadDim];
-#pragma unroll
-  for (int c = 0; c < kHeadDim; ++c) acc[c] = 0.f;
+  for (int s = 0; s < nsplit; ++s) mmax = fmaxf(mmax, __ldg(&ml[base + static_cast<size_t>(s) * kRows].x));
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
   float l = 0.f;
   for (int s = 0; s < nsplit; ++s) {
     const size_t idx = base + static_cast<size_t>(s) * kRows;
-    const float2 e = ml[idx];
+    const float2 e = __ldg(&ml[idx]);
     const float w = ex2_approx(e.x - mmax);
     l += w * e.y;
-    const float4* src = reinterpret_cast<const float4*>(part_o + idx * kHeadDim);
-#pragma unroll
-    for (int c = 0; c < kHeadDim / 4; ++c) {
-      const float4 t = src[c];
-      acc[4 * c] += w * t.x;
-      acc[4 * c + 1] += w * t.y;
-      acc[4 * c + 2] += w * t.z;
-      acc[4 * c + 3] += w * t.w;
-    }
+    const float4 t = __ldg(reinterpret_cast<const float4*>(part_o + idx * kHeadDim) + c4);
+    acc.x += w * t.x;
+    acc.y += w * t.y;
+    acc.z += w * t.z;
+    acc.w += w * t.w;
   }
   const float inv = 1.f / l;
   const int qblk = row < kBlock ? 0 : nb - 1;
   const size_t orow = static_cast<size_t>(bh) * L + static_cast<size_t>(qblk) * kBlock + (row & (kBlock - 1));
   if (out_f32) {
-    float4* dst = reinterpret_cast<float4*>(static_cast<float*>(out) + orow * kHeadDim);
-#pragma unroll
-    for (int c = 0; c < kHeadDim / 4; ++c)
-      dst[c] = make_float4(acc[4 * c] * inv, acc[4 * c + 1] * inv, acc[4 * c + 2] * inv, acc[4 * c + 3] * inv);
+    reinterpret_cast<float4*>(static_cast<float*>(out) + orow * kHeadDim)[c4] =
+        make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
   } else {
-    uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(out) + orow * kHeadDim);
-#pragma unroll
-    for (int c = 0; c < kHeadDim / 8; ++c)
-      dst[c] = make_uint4(pack_bf16x2(acc[8 * c] * inv, acc[8 * c + 1] * inv),
-                          pack_bf16x2(acc[8 * c + 2] * inv, acc[8 * c + 3] * inv),
-                          pack_bf16x2(acc[8 * c + 4] * inv, acc[8 * c + 5] * inv),
-                          pack_bf16x2(acc[8 * c + 6] * inv, acc[8 * c + 7] * inv));
+    reinterpret_cast<uint2*>(static_cast<uint16_t*>(out) + orow * kHeadDim)[c4] =
+        make_uint2(pack_bf16x2(acc.x * inv, acc.y * inv), pack_bf16x2(acc.z * inv, acc.w * inv));
   }
 }
 
@@ -739,6 +790,7 @@ int bigbird_attn_fwd_ex(const void* q, const void* k, const void* v, const int32
   }
   p.out_f32 = out_dtype == BB_OUT_F32 ? 1 : 0;
   p.scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(d));
+  p.bias_raw = -10000.0f * sqrtf(static_cast<float>(d));
 
   p.status = di->status;
 
@@ -758,7 +810,8 @@ int bigbird_attn_fwd_ex(const void* q, const void* k, const void* v, const int32
   bigbird_fwd_kernel<<<grid, kThreads, smem, stream>>>(tq, tk, tv, p);
   cudaError_t e = cudaGetLastError();
   if (e == cudaSuccess && pl.nsplit > 1) {
-    bigbird_merge_kernel<<<p.BH, kRows, 0, stream>>>(p.part_o, p.part_ml, out, pl.nsplit, L, pl.nb, p.out_f32);
+    bigbird_merge_kernel<<<dim3(p.BH, kRows / kMergeRowsPerCta), 256, 0, stream>>>(p.part_o, p.part_ml, out, pl.nsplit,
+                                                                               L, pl.nb, p.out_f32);
     e = cudaGetLastError();
   }
   if (owned) cudaFreeAsync(ws, stream);

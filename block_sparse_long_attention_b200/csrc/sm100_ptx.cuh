@@ -133,15 +133,19 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, ui
          (static_cast<uint64_t>(sbo >> 4) << 32) | (1ull << 46) | (2ull << 61);
 }
 
-// Instruction descriptor of kind::f16: bf16 x bf16 -> fp32, dense.
+// Instruction descriptor of kind::f16 with fp32 accumulation, dense.
+// ab_bf16: A and B are bf16 (else fp16; the two operands always share a type).
 // b_mn_major: B operand stored with its N dimension contiguous.
-__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool b_mn_major) {
+__host__ __device__ constexpr uint32_t idesc_f32acc(int M, int N, bool ab_bf16, bool b_mn_major) {
   return (1u << 4)                                   // D format f32
-         | (1u << 7)                                 // A format bf16
-         | (1u << 10)                                // B format bf16
+         | ((ab_bf16 ? 1u : 0u) << 7)                // A format: 0 f16, 1 bf16
+         | ((ab_bf16 ? 1u : 0u) << 10)               // B format
          | ((b_mn_major ? 1u : 0u) << 16)            // B major
          | (static_cast<uint32_t>(N >> 3) << 17)     // N / 8
          | (static_cast<uint32_t>(M >> 4) << 24);    // M / 16
+}
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool b_mn_major) {
+  return idesc_f32acc(M, N, true, b_mn_major);
 }
 
 // D[tmem] (+)= A[smem] * B[smem]
@@ -235,6 +239,19 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
+}
+
+// Two fp32 -> packed f16x2 (round to nearest even); lo goes to the low half.
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// Packed bf16x2 -> packed f16x2. Exact for every bf16 value whose magnitude
+// lies in the fp16 normal range [2^-14, 65504].
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w) {
+  return pack_f16x2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
 }
 
 }  // namespace bb
