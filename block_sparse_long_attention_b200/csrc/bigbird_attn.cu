@@ -16,23 +16,37 @@
 //     "随机块掩码是如何生成的"; HF-Pegasus, section "三类注意力组合"]. A half that
 //     does not use a block writes P = 0 for it, so the pair shares every MMA.
 //
-// Warp roles (192 threads): warps 0-3 run the softmax and the epilogue, one
-// query row per thread (thread t owns TMEM lane t); warp 4 builds the unit's
-// key-block list and key-validity masks and issues the TMA loads; warp 5
-// allocates TMEM and issues the tcgen05 MMAs from one thread.
+// A unit's key blocks are processed in chunks of two (128 keys): one
+// S = Q K^T MMA of N = 128 (the tensor core needs N >= 128 per instruction to
+// run at full rate), one softmax round, one O += P V MMA of K = 128.
 //
-// Per key block j of a unit:  S_j = Q K_j^T        (SS MMA, 128x64x64, TMEM)
-//                             P_j = exp2(S_j*c + bias - m)   (softmax warps, bf16
-//                                   written back over S_j in TMEM)
-//                             O  += P_j V_j        (TS MMA, P from TMEM)
-// with an online softmax whose reference max is moved only when it grows by
-// more than 2^8 (the O rescale is skipped otherwise; the final O / l is exact
-// either way). Padded keys get -10000 added to the scaled score.
+// Warp roles (256 threads, two CTAs per SM):
+//   warps 0-3  softmax and epilogue, one query row per thread (thread t owns
+//              TMEM lane t);
+//   warp 4     TMA: Q per unit, K and V per chunk on separate rings, the V
+//              stream one chunk behind the K stream (K is needed a round
+//              earlier);
+//   warp 5     TMEM allocation and the tcgen05 MMAs (one thread);
+//   warp 6     unit preparation (key-block list, half masks, key-validity
+//              bits) up to four units ahead, so its dependent global loads
+//              never stall the pipeline;
+//   warp 7     converts each V chunk bf16 -> fp16 in shared memory.
+//
+// TMEM (256 columns): S [0,128) fp32, P [128,192) fp16 (written by the softmax,
+// read by the TS MMA), O [192,256) fp32. Because P has its own columns, the
+// next chunk's S MMA is issued as soon as the softmax has read S, and runs
+// while the softmax computes the exponentials.
+//
+// Softmax: the reference max moves only when it grows by more than 2^8 (the O
+// rescale is skipped otherwise; the final O / l is exact either way). Padded
+// keys get -10000 added to the scaled score. P.V runs in fp16: P is written as
+// fp16 and each V tile is converted bf16 -> fp16 in shared memory (exact in the
+// fp16 normal range), which keeps three more mantissa bits of P than bf16.
 #include <cuda.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 #include <algorithm>
-#include <atomic>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -46,15 +60,19 @@ namespace bb {
 constexpr int kBlock = 64;             // tokens per block
 constexpr int kHeadDim = 64;           // head dimension
 constexpr int kRows = 128;             // query rows per unit (two blocks)
-constexpr int kStages = 4;             // K/V ring depth
+constexpr int kChunk = 2;              // key blocks per chunk
+constexpr int kKStages = 2;            // K ring depth (chunks)
+constexpr int kVStages = 2;            // V ring depth (chunks)
 constexpr int kMaxList = 40;           // key blocks per unit
 constexpr int kMaxR = 16;              // random blocks per row supported
 constexpr int kSplitBlocks = 8;        // key blocks per global-row range
-constexpr int kThreads = 192;
+constexpr int kThreads = 256;
 constexpr uint32_t kTileBytes = kBlock * kHeadDim * 2;  // one 64x64 bf16 tile
+constexpr uint32_t kChunkBytes = kChunk * kTileBytes;
 constexpr uint32_t kTmemCols = 256;
-constexpr uint32_t kColO = 128;        // O accumulator columns [128, 192)
-constexpr float kLog2e = 1.4426950408889634f;
+constexpr uint32_t kColS = 0;          // S: 128 fp32 columns
+constexpr uint32_t kColP = 128;        // P: 128 fp16 keys = 64 columns
+constexpr uint32_t kColO = 192;        // O: 64 fp32 columns
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr float kNegInit = -1.0e30f;
 
@@ -77,6 +95,9 @@ struct UnitInfo {
 };
 
 struct FwdParams {
+  const uint16_t* q;  // bf16 [B*H*L, 64], for L2 prefetch (loads go through the tensor maps)
+  const uint16_t* k;
+  const uint16_t* v;
   const int32_t* rand_attn;
   const uint8_t* seq_mask;
   void* out;
@@ -96,17 +117,25 @@ struct FwdParams {
 };
 
 struct __align__(1024) SharedStorage {
-  uint8_t q[2][kRows * kHeadDim * 2];   // 2 x 16 KB, SW128, 1024-aligned
-  uint8_t k[kStages][kTileBytes];       // 8 KB each
-  uint8_t v[kStages][kTileBytes];
+  uint8_t q[2][kRows * kHeadDim * 2];   // Q per unit, double buffered (SW128)
+  uint8_t k[kKStages][kChunkBytes];     // K chunk = two adjacent 64x64 tiles
+  uint8_t v[kVStages][kChunkBytes];     // V chunk
   UnitInfo unit[4];
+  uint64_t info_full[4];
+  uint64_t info_empty[4];
   uint64_t q_full[2];
   uint64_t q_free[2];
-  uint64_t kv_full[kStages];
-  uint64_t kv_empty[kStages];
-  uint64_t s_full[2];
-  uint64_t p_full[2];
-  uint64_t pv_done[2];
+  uint64_t k_full[kKStages];
+  uint64_t k_empty[kKStages];
+  uint64_t v_full[kVStages];
+  uint64_t v_conv[kVStages];
+  uint64_t v_empty[kVStages];
+  uint64_t s_full;
+  uint64_t s_free;
+  uint64_t p_lo;     // P of the chunk's block 0 written (4 softmax warps)
+  uint64_t p_hi;     // P of block 1 written (always arrived, also for one-block chunks)
+  uint64_t pv_lo;    // P.V of block 0 complete
+  uint64_t pv_hi;    // P.V of block 1 complete (committed for every chunk)
   uint64_t o_full;
   uint64_t o_free;
   uint32_t tmem_base;
@@ -118,15 +147,13 @@ __device__ __forceinline__ void flag_timeout(SharedStorage& s, const FwdParams& 
   *reinterpret_cast<volatile int32_t*>(&s.abort_flag) = 1;
 }
 
-__device__ __forceinline__ bool aborted(SharedStorage& s) {
-  return *reinterpret_cast<volatile int32_t*>(&s.abort_flag) != 0;
-}
-
 // Every lane waits (and acquires); the warp agrees on the outcome so that a
 // timeout never splits the warp before a .sync.aligned instruction.
 __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity) {
   return __all_sync(0xffffffffu, mbar_wait(bar, parity));
 }
+
+__device__ __forceinline__ int chunk_count(int n) { return (n + kChunk - 1) / kChunk; }
 
 // Decode unit u and build its key-block list. Called by a whole warp: the
 // lanes fetch the unit's random entries in parallel, lane 0 builds the list.
@@ -239,125 +266,243 @@ __device__ void prep_unit(const FwdParams& p, int u, UnitInfo& ui, int lane) {
   __syncwarp();
 }
 
-// The next unit's info is prepared while the current unit's first K/V tiles
-// are in flight, so the list-building loads never stall the TMA ring at a
-// unit boundary. Four info slots: a slot is rewritten three units after its
-// last use, when every consumer is provably done with it.
+// Unit preparation, up to four units ahead of the TMA warp: slot ut & 3 is
+// refilled once every consumer of unit ut - 4 has released it.
+__device__ void prep_role(SharedStorage& s, const FwdParams& p) {
+  const int lane = threadIdx.x & 31;
+  uint32_t ut = 0;
+  for (int u = blockIdx.x; u < p.total_units; u += gridDim.x, ++ut) {
+    const int slot = ut & 3;
+    int ok = 1;
+    if (lane == 0) ok = mbar_wait(smem_u32(&s.info_empty[slot]), ((ut >> 2) & 1) ^ 1);
+    if (!__shfl_sync(0xffffffffu, ok, 0)) {
+      if (lane == 0) flag_timeout(s, p);
+      return;
+    }
+    prep_unit(p, u, s.unit[slot], lane);
+    if (lane == 0) mbar_arrive(smem_u32(&s.info_full[slot]));
+    // Pull the unit's tiles into L2 now (it is up to four units ahead of the
+    // TMA warp), so its TMA loads hit L2 instead of HBM: one 8 KB tile per
+    // lane, lanes 0..n-1 K, n..2n-1 V, 2n and 2n+1 the query blocks.
+    const UnitInfo& ui = s.unit[slot];
+    const size_t row0 = static_cast<size_t>(ui.bh) * p.L;
+    const int n = ui.n;
+    for (int t = lane; t < 2 * n + 2; t += 32) {
+      const uint16_t* base;
+      int blk;
+      if (t < n) { base = p.k; blk = ui.kb[t]; }
+      else if (t < 2 * n) { base = p.v; blk = ui.kb[t - n]; }
+      else { base = p.q; blk = (t == 2 * n) ? ui.qtop : ui.qbot; }
+      if (blk >= 0) prefetch_l2_bulk(base + (row0 + static_cast<size_t>(blk) * kBlock) * kHeadDim, kTileBytes);
+    }
+  }
+}
+
+// V chunks are converted bf16 -> fp16 in place (exact in the fp16 normal
+// range) in the order the TMA warp loads them; the P.V MMA waits for v_conv.
+__device__ void convert_role(SharedStorage& s, const FwdParams& p) {
+  const int lane = threadIdx.x & 31;
+  uint32_t ut = 0, gv = 0;
+  for (int u = blockIdx.x; u < p.total_units; u += gridDim.x, ++ut) {
+    if (!warp_wait(smem_u32(&s.info_full[ut & 3]), (ut >> 2) & 1)) { if (lane == 0) flag_timeout(s, p); return; }
+    const int n = s.unit[ut & 3].n;
+    const int nch = chunk_count(n);
+    for (int c = 0; c < nch; ++c, ++gv) {
+      const int st = gv % kVStages;
+      const int nblk = min(kChunk, n - c * kChunk);
+      if (!warp_wait(smem_u32(&s.v_full[st]), (gv / kVStages) & 1)) { if (lane == 0) flag_timeout(s, p); return; }
+      uint4* vp = reinterpret_cast<uint4*>(s.v[st]) + lane;
+      const int nvec = nblk * (kTileBytes / 16) / 32;  // uint4 per lane
+#pragma unroll 4
+      for (int i = 0; i < nvec; ++i) {
+        uint4 w = vp[32 * i];
+        w.x = bf16x2_to_f16x2(w.x);
+        w.y = bf16x2_to_f16x2(w.y);
+        w.z = bf16x2_to_f16x2(w.z);
+        w.w = bf16x2_to_f16x2(w.w);
+        vp[32 * i] = w;
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&s.v_conv[st]));
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(smem_u32(&s.info_empty[ut & 3]));
+  }
+}
+
+// Two cursors walk this CTA's chunk sequence: the K cursor (which also loads
+// each unit's Q when it enters the unit) and the V cursor one chunk behind it.
 __device__ void producer_role(SharedStorage& s, const FwdParams& p, const CUtensorMap* tmQ, const CUtensorMap* tmK,
                               const CUtensorMap* tmV) {
   const int lane = threadIdx.x & 31;
   const uint64_t pol_kv = l2_policy_evict_last();
   const uint64_t pol_q = l2_policy_evict_first();
-  uint32_t unit_it = 0, kv_it = 0;
-  int u = blockIdx.x;
-  if (u < p.total_units) prep_unit(p, u, s.unit[0], lane);
-  for (; u < p.total_units; u += gridDim.x, ++unit_it) {
-    const int qs = unit_it & 1;
-    const uint32_t ph = (unit_it >> 1) & 1;
-    const UnitInfo& ui = s.unit[unit_it & 3];
-    int ok = 1;
-    if (lane == 0) ok = mbar_wait(smem_u32(&s.q_free[qs]), ph ^ 1);
-    if (!__shfl_sync(0xffffffffu, ok, 0)) {
-      if (lane == 0) flag_timeout(s, p);
-      return;
-    }
-    const int n = ui.n;
-    const int32_t row0 = ui.bh * p.L;
-    const int nxt = u + gridDim.x;
-    const int prep_at = min(n, kStages) - 1;
-    if (lane == 0) {
-      const uint32_t qbar = smem_u32(&s.q_full[qs]);
-      mbar_arrive_expect_tx(qbar, ui.qbot >= 0 ? 2 * kTileBytes : kTileBytes);
-      tma_load_2d(smem_u32(s.q[qs]), tmQ, qbar, 0, row0 + ui.qtop * kBlock, pol_q);
-      if (ui.qbot >= 0) tma_load_2d(smem_u32(s.q[qs]) + kTileBytes, tmQ, qbar, 0, row0 + ui.qbot * kBlock, pol_q);
-    }
-    for (int j = 0; j < n; ++j, ++kv_it) {
+  if (static_cast<int>(blockIdx.x) >= p.total_units) return;
+  uint32_t kut = 0, vut = 0, gk = 0, gv = 0;
+  int ku = blockIdx.x, kc = 0, vc = 0;
+  bool kdone = false;
+  while (!(kdone && gv == gk)) {
+    if (!kdone) {
+      int ok = 1;
+      if (kc == 0) ok = mbar_wait(smem_u32(&s.info_full[kut & 3]), (kut >> 2) & 1);
+      if (!__all_sync(0xffffffffu, ok)) {
+        if (lane == 0) flag_timeout(s, p);
+        return;
+      }
+      const UnitInfo& ui = s.unit[kut & 3];
+      const int n = ui.n;
+      const int nch = chunk_count(n);
+      const int32_t row0 = ui.bh * p.L;
       if (lane == 0) {
-        const int st = kv_it % kStages;
-        ok = mbar_wait(smem_u32(&s.kv_empty[st]), ((kv_it / kStages) & 1) ^ 1);
+        if (kc == 0) {
+          const int qs = kut & 1;
+          ok = mbar_wait(smem_u32(&s.q_free[qs]), ((kut >> 1) & 1) ^ 1);
+          if (ok) {
+            const uint32_t qbar = smem_u32(&s.q_full[qs]);
+            mbar_arrive_expect_tx(qbar, ui.qbot >= 0 ? 2 * kTileBytes : kTileBytes);
+            tma_load_2d(smem_u32(s.q[qs]), tmQ, qbar, 0, row0 + ui.qtop * kBlock, pol_q);
+            if (ui.qbot >= 0)
+              tma_load_2d(smem_u32(s.q[qs]) + kTileBytes, tmQ, qbar, 0, row0 + ui.qbot * kBlock, pol_q);
+          }
+        }
         if (ok) {
-          const uint32_t kbar = smem_u32(&s.kv_full[st]);
-          mbar_arrive_expect_tx(kbar, 2 * kTileBytes);
-          const int32_t krow = row0 + ui.kb[j] * kBlock;
-          tma_load_2d(smem_u32(s.k[st]), tmK, kbar, 0, krow, pol_kv);
-          tma_load_2d(smem_u32(s.v[st]), tmV, kbar, 0, krow, pol_kv);
+          const int st = gk % kKStages;
+          ok = mbar_wait(smem_u32(&s.k_empty[st]), ((gk / kKStages) & 1) ^ 1);
+          if (ok) {
+            const int e0 = kc * kChunk;
+            const int nblk = min(kChunk, n - e0);
+            const uint32_t kbar = smem_u32(&s.k_full[st]);
+            mbar_arrive_expect_tx(kbar, nblk * kTileBytes);
+            for (int e = 0; e < nblk; ++e)
+              tma_load_2d(smem_u32(s.k[st]) + e * kTileBytes, tmK, kbar, 0, row0 + ui.kb[e0 + e] * kBlock, pol_kv);
+          }
         }
       }
       if (!__shfl_sync(0xffffffffu, ok, 0)) {
         if (lane == 0) flag_timeout(s, p);
         return;
       }
-      if (j == prep_at && nxt < p.total_units) prep_unit(p, nxt, s.unit[(unit_it + 1) & 3], lane);
+      ++gk;
+      if (++kc == nch) {
+        kc = 0;
+        ++kut;
+        ku += gridDim.x;
+        kdone = ku >= p.total_units;
+      }
+    }
+    if (gv + 1 < gk || (kdone && gv < gk)) {
+      const UnitInfo& ui = s.unit[vut & 3];
+      const int n = ui.n;
+      const int32_t row0 = ui.bh * p.L;
+      int ok = 1;
+      if (lane == 0) {
+        const int st = gv % kVStages;
+        ok = mbar_wait(smem_u32(&s.v_empty[st]), ((gv / kVStages) & 1) ^ 1);
+        if (ok) {
+          const int e0 = vc * kChunk;
+          const int nblk = min(kChunk, n - e0);
+          const uint32_t vbar = smem_u32(&s.v_full[st]);
+          mbar_arrive_expect_tx(vbar, nblk * kTileBytes);
+          for (int e = 0; e < nblk; ++e)
+            tma_load_2d(smem_u32(s.v[st]) + e * kTileBytes, tmV, vbar, 0, row0 + ui.kb[e0 + e] * kBlock, pol_kv);
+        }
+      }
+      if (!__shfl_sync(0xffffffffu, ok, 0)) {
+        if (lane == 0) flag_timeout(s, p);
+        return;
+      }
+      ++gv;
+      if (++vc == chunk_count(n)) {
+        // both cursors are done with this unit's info
+        if (lane == 0) mbar_arrive(smem_u32(&s.info_empty[vut & 3]));
+        vc = 0;
+        ++vut;
+      }
     }
   }
 }
 
 // ---------------------------------------------------------------- MMA issuer
 
+// Per chunk g: S(g) once the softmax has read S(g-1); then the P.V of the
+// previous chunk's block 1 (PV-hi, when its P is written) and of this chunk's
+// block 0 (PV-lo, written half way through the softmax). Splitting P.V in two
+// frees the P buffer in halves, so the softmax never waits for a whole P.V.
 __device__ void mma_role(SharedStorage& s, const FwdParams& p, uint32_t tmem) {
-  const uint32_t idesc_s = idesc_bf16_f32(kRows, kBlock, false);
-  // P.V runs in fp16: P is written as fp16 and V is converted to fp16 in shared
-  // memory (exact for bf16 values in the fp16 normal range); fp16 keeps three
-  // more mantissa bits of P than bf16 would.
-  const uint32_t idesc_o = idesc_f32acc(kRows, kHeadDim, false, true);
-  uint32_t unit_it = 0, kv_it = 0, g = 0;
+  const uint32_t idesc_s2 = idesc_f32acc(kRows, 2 * kBlock, true, false);  // S of a 2-block chunk
+  const uint32_t idesc_s1 = idesc_f32acc(kRows, kBlock, true, false);      // S of a 1-block chunk
+  const uint32_t idesc_o = idesc_f32acc(kRows, kHeadDim, false, true);     // fp16 P . fp16 V
+  uint32_t ut = 0, gc = 0;
   bool ok = true;
-  for (int u = blockIdx.x; u < p.total_units && ok; u += gridDim.x, ++unit_it) {
-    const int slot = unit_it & 1;
-    const uint32_t ph = (unit_it >> 1) & 1;
-    if (!mbar_wait(smem_u32(&s.q_full[slot]), ph)) { ok = false; break; }
-    const int n = s.unit[unit_it & 3].n;
-    const uint32_t q_addr = smem_u32(s.q[slot]);
+  for (int u = blockIdx.x; u < p.total_units && ok; u += gridDim.x, ++ut) {
+    const int qs = ut & 1;
+    if (!mbar_wait(smem_u32(&s.q_full[qs]), (ut >> 1) & 1)) { ok = false; break; }
+    const int n = s.unit[ut & 3].n;
+    const int nch = chunk_count(n);
+    const uint32_t q_addr = smem_u32(s.q[qs]);
 
-    auto issue_pv = [&](int jj) -> bool {
-      const uint32_t gg = g + jj;
-      const int sb = gg & 1;
-      const int st = (kv_it + jj) % kStages;
-      if (!mbar_wait(smem_u32(&s.p_full[sb]), (gg >> 1) & 1)) return false;
-      if (jj == 0 && !mbar_wait(smem_u32(&s.o_free), (unit_it & 1) ^ 1)) return false;
-      tc_fence_after();
-      const uint32_t v_addr = smem_u32(s.v[st]);
-#pragma unroll
-      for (int kk = 0; kk < kBlock / 16; ++kk) {
-        const uint64_t bdesc = sdesc_sw128(v_addr + kk * 2048, 8192, 1024);
-        mma_ts(tmem + kColO, tmem + sb * 64 + kk * 8, bdesc, idesc_o, (jj > 0 || kk > 0) ? 1u : 0u);
+    // P.V of one block (bi = 0: lo, 1: hi) of chunk c.
+    auto issue_pv = [&](int c, int bi) -> bool {
+      const uint32_t g = gc + c;
+      const int st = g % kVStages;
+      const int nblk = min(kChunk, n - c * kChunk);
+      if (bi == 0) {
+        if (!mbar_wait(smem_u32(&s.v_conv[st]), (g / kVStages) & 1)) return false;
+        if (c == 0 && !mbar_wait(smem_u32(&s.o_free), (ut & 1) ^ 1)) return false;
       }
-      mma_commit(smem_u32(&s.pv_done[sb]));
-      mma_commit(smem_u32(&s.kv_empty[st]));
+      if (!mbar_wait(smem_u32(bi == 0 ? &s.p_lo : &s.p_hi), g & 1)) return false;
+      tc_fence_after();
+      if (bi < nblk) {
+        const uint32_t v_addr = smem_u32(s.v[st]) + bi * kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < kBlock / 16; ++kk) {
+          const uint64_t bdesc = sdesc_sw128(v_addr + kk * 2048, 8192, 1024);
+          mma_ts(tmem + kColO, tmem + kColP + bi * 32 + kk * 8, bdesc, idesc_o,
+                 (c > 0 || bi > 0 || kk > 0) ? 1u : 0u);
+        }
+      }
+      if (bi == 0) {
+        mma_commit(smem_u32(&s.pv_lo));
+      } else {
+        mma_commit(smem_u32(&s.pv_hi));
+        mma_commit(smem_u32(&s.v_empty[st]));
+      }
       return true;
     };
 
-    for (int j = 0; j < n && ok; ++j) {
-      const uint32_t gg = g + j;
-      const int sb = gg & 1;
-      const uint32_t kvi = kv_it + j;
-      const int st = kvi % kStages;
-      if (!mbar_wait(smem_u32(&s.kv_full[st]), (kvi / kStages) & 1)) { ok = false; break; }
-      if (gg >= 2 && !mbar_wait(smem_u32(&s.pv_done[sb]), ((gg >> 1) - 1) & 1)) { ok = false; break; }
+    for (int c = 0; c < nch && ok; ++c) {
+      const uint32_t g = gc + c;
+      const int st = g % kKStages;
+      const int nblk = min(kChunk, n - c * kChunk);
+      if (!mbar_wait(smem_u32(&s.k_full[st]), (g / kKStages) & 1)) { ok = false; break; }
+      if (g >= 1 && !mbar_wait(smem_u32(&s.s_free), (g - 1) & 1)) { ok = false; break; }
       tc_fence_after();
       const uint32_t k_addr = smem_u32(s.k[st]);
 #pragma unroll
       for (int kk = 0; kk < kHeadDim / 16; ++kk) {
         const uint64_t adesc = sdesc_sw128(q_addr + kk * 32, 16, 1024);
         const uint64_t bdesc = sdesc_sw128(k_addr + kk * 32, 16, 1024);
-        mma_ss(tmem + sb * 64, adesc, bdesc, idesc_s, kk > 0 ? 1u : 0u);
+        mma_ss(tmem + kColS, adesc, bdesc, nblk == 2 ? idesc_s2 : idesc_s1, kk > 0 ? 1u : 0u);
       }
-      mma_commit(smem_u32(&s.s_full[sb]));
-      if (j >= 1 && !issue_pv(j - 1)) { ok = false; break; }
+      mma_commit(smem_u32(&s.s_full));
+      mma_commit(smem_u32(&s.k_empty[st]));
+      if (c >= 1 && !issue_pv(c - 1, 1)) { ok = false; break; }
+      if (!issue_pv(c, 0)) { ok = false; break; }
     }
     if (!ok) break;
-    if (n > 0 && !issue_pv(n - 1)) { ok = false; break; }
-    mma_commit(smem_u32(&s.q_free[slot]));
+    if (!issue_pv(nch - 1, 1)) { ok = false; break; }
+    mma_commit(smem_u32(&s.q_free[qs]));
     mma_commit(smem_u32(&s.o_full));
-    kv_it += n;
-    g += n;
+    mbar_arrive(smem_u32(&s.info_empty[ut & 3]));
+    gc += nch;
   }
   if (!ok) flag_timeout(s, p);
 }
 
 // ---------------------------------------------------------------- softmax + epilogue
 
-__device__ __forceinline__ float fmax_tree(const float (&x)[16]) {
+__device__ __forceinline__ float fmax_tree16(const float (&x)[16]) {
   float a = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
   float b = fmaxf(fmaxf(x[4], x[5]), fmaxf(x[6], x[7]));
   float c = fmaxf(fmaxf(x[8], x[9]), fmaxf(x[10], x[11]));
@@ -365,129 +510,241 @@ __device__ __forceinline__ float fmax_tree(const float (&x)[16]) {
   return fmaxf(fmaxf(a, b), fmaxf(c, d));
 }
 
+// Per-block key validity: all keys valid (no bias), all masked (one uniform
+// bias, folded into the exponent offset and the max), or mixed (per-key bias;
+// only the block holding a sequence's padding boundary).
+__device__ __forceinline__ bool block_mixed(uint64_t vm) { return vm != ~0ull && vm != 0ull; }
+__device__ __forceinline__ float block_offset(uint64_t vm, float bias) { return vm == 0ull ? bias : 0.f; }
+
+// Add the per-key bias of a mixed block to 32 raw scores (in place) and
+// return their max plus the block's uniform offset (q.k units).
+__device__ __forceinline__ float piece_prepare(uint32_t (&r)[32], bool mixed, uint32_t vm, float bias, float off) {
+  if (mixed) {
+#pragma unroll
+    for (int c = 0; c < 32; ++c) r[c] = __float_as_uint(__uint_as_float(r[c]) + (((vm >> c) & 1u) ? 0.f : bias));
+  }
+  float a = fmaxf(__uint_as_float(r[0]), __uint_as_float(r[1]));
+  float b = fmaxf(__uint_as_float(r[2]), __uint_as_float(r[3]));
+#pragma unroll
+  for (int i = 1; i < 8; ++i) {
+    a = fmax3(a, __uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]));
+    b = fmax3(b, __uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3]));
+  }
+  return fmaxf(a, b) + off;
+}
+
+// p = exp2(r * scale + off) for 32 scores, packed to fp16x2 into pk[0..16);
+// the sum accumulates into two packed pairs (shorter dependency chains).
+__device__ __forceinline__ void piece_exp(const uint32_t (&r)[32], uint64_t scale2, uint64_t off2, uint32_t* pk,
+                                          uint64_t& acc0, uint64_t& acc1) {
+#pragma unroll
+  for (int c = 0; c < 16; ++c) {
+    float t0, t1;
+    f2_unpack(f2_fma(f2_pack(__uint_as_float(r[2 * c]), __uint_as_float(r[2 * c + 1])), scale2, off2), t0, t1);
+    const float e0 = ex2_approx(t0);
+    const float e1 = ex2_approx(t1);
+    if (c & 1) acc1 = f2_add(acc1, f2_pack(e0, e1));
+    else acc0 = f2_add(acc0, f2_pack(e0, e1));
+    pk[c] = pack_f16x2(e0, e1);
+  }
+}
+
+// Multiply 16 packed fp16x2 values by f (rare path: a later max increase).
+__device__ __forceinline__ void scale_packed16(uint32_t* pk, float f) {
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    __half2 h = *reinterpret_cast<__half2*>(&pk[i]);
+    const float2 v = __half22float2(h);
+    pk[i] = pack_f16x2(v.x * f, v.y * f);
+  }
+}
+
+// Per-row online-softmax state of one unit.
+struct RowState {
+  float m_ref;     // reference max (scaled log2 units)
+  float l_run;     // sum of p over the chunks before the current one
+  uint64_t acc0, acc1;  // packed partial sums of the current chunk
+  float o_factor;  // rescale owed to the O accumulator
+};
+
+// Max, rescale bookkeeping and exponentials of one 32-column piece.
+// hi: the block's lo piece is already in pk[-16..0).
+__device__ __forceinline__ void process_piece(uint32_t (&r)[32], bool mixed, uint32_t vm, float off, bool hi,
+                                              const FwdParams& p, uint32_t* pk, RowState& st) {
+  const float mx = piece_prepare(r, mixed, vm, p.bias_raw, off) * p.scale_log2;
+  const bool need = mx > st.m_ref + kRescaleThreshold;
+  if (__any_sync(0xffffffffu, need)) {
+    float f = 1.f;
+    if (need) {
+      f = ex2_approx(st.m_ref - mx);
+      st.m_ref = mx;
+    }
+    const uint64_t f2 = f2_pack(f, f);
+    st.l_run *= f;
+    st.acc0 = f2_fma(st.acc0, f2, 0ull);
+    st.acc1 = f2_fma(st.acc1, f2, 0ull);
+    st.o_factor *= f;
+    if (hi) scale_packed16(pk - 16, f);
+  }
+  const float o = fmaf(off, p.scale_log2, -st.m_ref);
+  piece_exp(r, f2_pack(p.scale_log2, p.scale_log2), f2_pack(o, o), pk, st.acc0, st.acc1);
+}
+
+// O (64 fp32 columns of this thread's row) *= f, in 16-column pieces.
+__device__ __forceinline__ void rescale_o(uint32_t taddr, float f) {
+#pragma unroll 1
+  for (int c0 = 0; c0 < 64; c0 += 16) {
+    uint32_t t[16];
+    tmem_ld16(taddr + c0, t);
+    tmem_wait_ld();
+#pragma unroll
+    for (int i = 0; i < 16; ++i) t[i] = __float_as_uint(__uint_as_float(t[i]) * f);
+    tmem_st16(taddr + c0, t);
+  }
+  tmem_wait_st();
+}
+
 __device__ void softmax_role(SharedStorage& s, const FwdParams& p, uint32_t tmem) {
   const int tid = threadIdx.x;  // 0..127 == TMEM lane
   const int warp = tid >> 5;
   const int lane = tid & 31;
   const int half = warp >> 1;   // 0: rows 0..63, 1: rows 64..127
-  const uint32_t lane_addr = static_cast<uint32_t>(warp * 32) << 16;
-  uint32_t unit_it = 0, g = 0;
-  for (int u = blockIdx.x; u < p.total_units; u += gridDim.x, ++unit_it) {
-    const int slot = unit_it & 1;
-    const uint32_t ph = (unit_it >> 1) & 1;
-    if (!warp_wait(smem_u32(&s.q_full[slot]), ph)) { flag_timeout(s, p); return; }
-    const UnitInfo& ui = s.unit[unit_it & 3];
+  const uint32_t lane_addr = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+  uint32_t ut = 0, gc = 0;
+  for (int u = blockIdx.x; u < p.total_units; u += gridDim.x, ++ut) {
+    if (!warp_wait(smem_u32(&s.q_full[ut & 1]), (ut >> 1) & 1)) { flag_timeout(s, p); return; }
+    const UnitInfo& ui = s.unit[ut & 3];
     const int n = ui.n;
+    const int nch = chunk_count(n);
     const int bh = ui.bh;
     const int qblk = half ? ui.qbot : ui.qtop;
     const int split = ui.split;
     const bool exists = qblk >= 0;
-    float m_ref = kNegInit, l_run = 0.f;
+    RowState st;
+    st.m_ref = kNegInit;
+    st.l_run = 0.f;
 
-    for (int j = 0; j < n; ++j) {
-      const uint32_t gg = g + j;
-      const int sb = gg & 1;
-      if (!warp_wait(smem_u32(&s.s_full[sb]), (gg >> 1) & 1)) { flag_timeout(s, p); return; }
+    for (int c = 0; c < nch; ++c) {
+      const uint32_t g = gc + c;
+      const int e0 = c * kChunk;
+      const int nblk = min(kChunk, n - e0);
+      if (!warp_wait(smem_u32(&s.s_full), g & 1)) { flag_timeout(s, p); return; }
       tc_fence_after();
-      const bool used = exists && ((ui.hm[j] >> half) & 1);
+      const bool used0 = exists && ((ui.hm[e0] >> half) & 1);
+      const bool used1 = nblk == 2 && exists && ((ui.hm[e0 + 1] >> half) & 1);
+      st.acc0 = st.acc1 = 0ull;
+      st.o_factor = 1.f;
       uint32_t pk[32];
-      if (used) {
-        float x[64];  // raw scores q.k (+ the masked-key bias in the same units)
-        {
-          uint32_t r0[32], r1[32];
-          tmem_ld32(tmem + lane_addr + sb * 64, r0);
-          tmem_ld32(tmem + lane_addr + sb * 64 + 32, r1);
-          tmem_wait_ld();
-#pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            x[c] = __uint_as_float(r0[c]);
-            x[32 + c] = __uint_as_float(r1[c]);
-          }
+      uint32_t ra[32], rb[32];
+      // Single pass over the used blocks in 32-column pieces; the TMEM read of
+      // piece k+1 is in flight while piece k is exponentiated. S is released
+      // as soon as its last piece has been read.
+      if (used0 || used1) {
+        tmem_ld32(lane_addr + kColS + (used0 ? 0 : kBlock), ra);
+        tmem_wait_ld();
+      } else {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&s.s_free));
+      }
+      // ---- block 0
+      if (used0) {
+        const uint64_t vm = ui.vm[e0];
+        const bool mixed = block_mixed(vm);
+        const float off = block_offset(vm, p.bias_raw);
+        tmem_ld32(lane_addr + kColS + 32, rb);
+        process_piece(ra, mixed, static_cast<uint32_t>(vm), off, false, p, pk, st);
+        tmem_wait_ld();
+        if (!used1) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(smem_u32(&s.s_free));
         }
-        const uint64_t vm = ui.vm[j];
-        if (vm != ~0ull) {
-#pragma unroll
-          for (int c = 0; c < 64; ++c) x[c] += ((vm >> c) & 1ull) ? 0.f : p.bias_raw;
-        }
-        float mx;
-        {
-          float t[16];
-#pragma unroll
-          for (int c = 0; c < 16; ++c) t[c] = fmaxf(fmaxf(x[c], x[16 + c]), fmaxf(x[32 + c], x[48 + c]));
-          mx = fmax_tree(t) * p.scale_log2;
-        }
-        float factor = 1.f;
-        bool rescale_o = false;
-        if (mx > m_ref + kRescaleThreshold) {
-          factor = ex2_approx(m_ref - mx);
-          rescale_o = l_run > 0.f;
-          m_ref = mx;
-        }
-        const float neg_m = -m_ref;
-        float sum = 0.f;
-#pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          const float e0 = ex2_approx(fmaf(x[2 * c], p.scale_log2, neg_m));
-          const float e1 = ex2_approx(fmaf(x[2 * c + 1], p.scale_log2, neg_m));
-          sum += e0 + e1;
-          pk[c] = pack_f16x2(e0, e1);
-        }
-        l_run = l_run * factor + sum;
-        if (__any_sync(0xffffffffu, rescale_o)) {
-          // O rows are final only once the previous block's P.V has landed.
-          const uint32_t gp = gg - 1;
-          if (!warp_wait(smem_u32(&s.pv_done[gp & 1]), (gp >> 1) & 1)) { flag_timeout(s, p); return; }
-          tc_fence_after();
-#pragma unroll
-          for (int c0 = 0; c0 < 64; c0 += 32) {
-            uint32_t o[32];
-            tmem_ld32(tmem + lane_addr + kColO + c0, o);
-            tmem_wait_ld();
-#pragma unroll
-            for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * factor);
-            tmem_st32(tmem + lane_addr + kColO + c0, o);
-          }
-        }
+        process_piece(rb, mixed, static_cast<uint32_t>(vm >> 32), off, true, p, pk + 16, st);
       } else {
 #pragma unroll
-        for (int c = 0; c < 32; ++c) pk[c] = 0u;
+        for (int i = 0; i < 32; ++i) pk[i] = 0u;
       }
-      {
-        // Convert this thread's 64-byte slice of V_j to fp16 in place (the
-        // block counter is also the K/V ring counter).
-        const int st = gg % kStages;
-        if (!warp_wait(smem_u32(&s.kv_full[st]), (gg / kStages) & 1)) { flag_timeout(s, p); return; }
-        uint4* vp = reinterpret_cast<uint4*>(s.v[st]) + tid * 4;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          uint4 w = vp[i];
-          w.x = bf16x2_to_f16x2(w.x);
-          w.y = bf16x2_to_f16x2(w.y);
-          w.z = bf16x2_to_f16x2(w.z);
-          w.w = bf16x2_to_f16x2(w.w);
-          vp[i] = w;
+      // P columns of block 0 are free once the previous chunk's PV-lo is done.
+      if (g >= 1 && !warp_wait(smem_u32(&s.pv_lo), (g - 1) & 1)) { flag_timeout(s, p); return; }
+      tc_fence_after();
+      if (__any_sync(0xffffffffu, st.o_factor != 1.f)) {
+        // The max grew: O (all of the previous chunk's P.V) scales by o_factor.
+        if (c > 0) {
+          if (!warp_wait(smem_u32(&s.pv_hi), (g - 1) & 1)) { flag_timeout(s, p); return; }
+          tc_fence_after();
+          rescale_o(lane_addr + kColO, st.o_factor);
         }
-        fence_proxy_async_smem();
+        st.o_factor = 1.f;
       }
-      tmem_st32(tmem + lane_addr + sb * 64, pk);
+      tmem_st32(lane_addr + kColP, pk);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&s.p_full[sb]));
+      if (lane == 0) mbar_arrive(smem_u32(&s.p_lo));
+      // ---- block 1
+      if (nblk == 2) {
+        if (used1) {
+          const uint64_t vm = ui.vm[e0 + 1];
+          const bool mixed = block_mixed(vm);
+          const float off = block_offset(vm, p.bias_raw);
+          if (used0) {
+            tmem_ld32(lane_addr + kColS + kBlock, ra);
+            tmem_wait_ld();
+          }
+          tmem_ld32(lane_addr + kColS + kBlock + 32, rb);
+          process_piece(ra, mixed, static_cast<uint32_t>(vm), off, false, p, pk, st);
+          tmem_wait_ld();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(smem_u32(&s.s_free));
+          process_piece(rb, mixed, static_cast<uint32_t>(vm >> 32), off, true, p, pk + 16, st);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) pk[i] = 0u;
+        }
+        if (g >= 1 && !warp_wait(smem_u32(&s.pv_hi), (g - 1) & 1)) { flag_timeout(s, p); return; }
+        tc_fence_after();
+        if (__any_sync(0xffffffffu, st.o_factor != 1.f)) {
+          // The max grew after block 0's P went out: once this chunk's PV-lo has
+          // landed, O (earlier chunks and block 0) scales by o_factor.
+          if (!warp_wait(smem_u32(&s.pv_lo), g & 1)) { flag_timeout(s, p); return; }
+          tc_fence_after();
+          rescale_o(lane_addr + kColO, st.o_factor);
+          st.o_factor = 1.f;
+        }
+        tmem_st32(lane_addr + kColP + 32, pk);
+        tmem_wait_st();
+      } else if (g >= 1) {
+        // One-block chunk: nothing to write, but p_hi must not run two phases
+        // ahead of the MMA thread's wait on it.
+        if (!warp_wait(smem_u32(&s.pv_hi), (g - 1) & 1)) { flag_timeout(s, p); return; }
+      }
+      {
+        float a0, a1, b0, b1;
+        f2_unpack(st.acc0, a0, a1);
+        f2_unpack(st.acc1, b0, b1);
+        st.l_run += (a0 + a1) + (b0 + b1);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&s.p_hi));
     }
+    const float m_ref = st.m_ref;
+    const float l_run = st.l_run;
+    __syncwarp();
+    if (lane == 0) mbar_arrive(smem_u32(&s.info_empty[ut & 3]));
 
     // ---- epilogue
-    if (!warp_wait(smem_u32(&s.o_full), unit_it & 1)) { flag_timeout(s, p); return; }
+    if (!warp_wait(smem_u32(&s.o_full), ut & 1)) { flag_timeout(s, p); return; }
     tc_fence_after();
     uint32_t o0[32], o1[32];
-    tmem_ld32(tmem + lane_addr + kColO, o0);
-    tmem_ld32(tmem + lane_addr + kColO + 32, o1);
+    tmem_ld32(lane_addr + kColO, o0);
+    tmem_ld32(lane_addr + kColO + 32, o1);
     tmem_wait_ld();
     tc_fence_before();
     __syncwarp();
-    if (lane == 0) {
-      mbar_arrive(smem_u32(&s.o_free));
-    }
+    if (lane == 0) mbar_arrive(smem_u32(&s.o_free));
     if (exists) {
       const int row_in_blk = tid & 63;
       if (split >= 0) {
@@ -532,7 +789,7 @@ __device__ void softmax_role(SharedStorage& s, const FwdParams& p, uint32_t tmem
         }
       }
     }
-    g += n;
+    gc += nch;
   }
 }
 
@@ -548,17 +805,29 @@ bigbird_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     tmem_relinquish();
   }
   if (threadIdx.x == 0) {
+    for (int i = 0; i < 4; ++i) {
+      mbar_init(smem_u32(&s.info_full[i]), 1);
+      mbar_init(smem_u32(&s.info_empty[i]), 1 + 1 + 4 + 1);  // TMA, MMA, 4 softmax warps, converter
+    }
     for (int i = 0; i < 2; ++i) {
       mbar_init(smem_u32(&s.q_full[i]), 1);
       mbar_init(smem_u32(&s.q_free[i]), 1);
-      mbar_init(smem_u32(&s.s_full[i]), 1);
-      mbar_init(smem_u32(&s.p_full[i]), 4);
-      mbar_init(smem_u32(&s.pv_done[i]), 1);
     }
-    for (int i = 0; i < kStages; ++i) {
-      mbar_init(smem_u32(&s.kv_full[i]), 1);
-      mbar_init(smem_u32(&s.kv_empty[i]), 1);
+    for (int i = 0; i < kKStages; ++i) {
+      mbar_init(smem_u32(&s.k_full[i]), 1);
+      mbar_init(smem_u32(&s.k_empty[i]), 1);
     }
+    for (int i = 0; i < kVStages; ++i) {
+      mbar_init(smem_u32(&s.v_full[i]), 1);
+      mbar_init(smem_u32(&s.v_conv[i]), 1);
+      mbar_init(smem_u32(&s.v_empty[i]), 1);
+    }
+    mbar_init(smem_u32(&s.s_full), 1);
+    mbar_init(smem_u32(&s.s_free), 4);
+    mbar_init(smem_u32(&s.p_lo), 4);
+    mbar_init(smem_u32(&s.p_hi), 4);
+    mbar_init(smem_u32(&s.pv_lo), 1);
+    mbar_init(smem_u32(&s.pv_hi), 1);
     mbar_init(smem_u32(&s.o_full), 1);
     mbar_init(smem_u32(&s.o_free), 4);
     s.abort_flag = 0;
@@ -578,8 +847,12 @@ bigbird_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     softmax_role(s, p, tmem);
   } else if (warp == 4) {
     producer_role(s, p, &tmQ, &tmK, &tmV);
-  } else if (lane == 0) {
-    mma_role(s, p, tmem);
+  } else if (warp == 5) {
+    if (lane == 0) mma_role(s, p, tmem);
+  } else if (warp == 6) {
+    prep_role(s, p);
+  } else {
+    convert_role(s, p);
   }
   tc_fence_before();
   __syncthreads();
@@ -685,6 +958,9 @@ static DeviceInfo* device_info(int dev) {
       const int smem = static_cast<int>(sizeof(SharedStorage) + 1024);
       if (cudaFuncSetAttribute(bigbird_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
         return nullptr;
+      // Two CTAs per SM need the largest shared-memory carve-out.
+      if (cudaFuncSetAttribute(bigbird_fwd_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100) != cudaSuccess)
+        return nullptr;
       if (cudaGetSymbolAddress(reinterpret_cast<void**>(&di.status), g_status) != cudaSuccess) return nullptr;
     }
     di.attr_set = true;
@@ -767,6 +1043,9 @@ int bigbird_attn_fwd_ex(const void* q, const void* k, const void* v, const int32
   if (!make_map(&tq, q, rows) || !make_map(&tk, k, rows) || !make_map(&tv, v, rows)) return BB_ERR_CUDA;
 
   FwdParams p{};
+  p.q = static_cast<const uint16_t*>(q);
+  p.k = static_cast<const uint16_t*>(k);
+  p.v = static_cast<const uint16_t*>(v);
   p.rand_attn = rand_attn;
   p.seq_mask = seq_mask;
   p.out = out;
