@@ -1,0 +1,69 @@
+"""Multi-rank host logic on CPU (gloo, world size 2): each rank computes its
+shard of a global batch independently; the gathered result equals the
+single-process one, with no data-path exchange beyond the final gather."""
+
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+from block_sparse_long_attention_b200.sharding import batch_shard
+
+
+def test_batch_shard_covers_exactly():
+    for gb in range(0, 13):
+        for world in range(1, 6):
+            owned = []
+            for r in range(world):
+                lo, hi = batch_shard(gb, world, r)
+                owned.extend(range(lo, hi))
+                assert hi - lo in (gb // world, gb // world + 1)
+            assert owned == list(range(gb))
+    with pytest.raises(ValueError):
+        batch_shard(4, 2, 2)
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+def _worker(rank, world, port, result_path):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    from datetime import timedelta
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=timedelta(seconds=60))
+    import oracle
+    from block_sparse_long_attention_b200.workloads import Workload, make_inputs
+    w = Workload("dist", 3, 2, 14 * 64, pad=("fixed", [896, 500, 700]), seed=31)
+    inp = make_inputs(w)
+    ra = oracle.rand_attn_generate(w.H, w.L, w.block, w.r, seed=w.seed)
+    lo, hi = batch_shard(w.B, world, rank)
+    part = oracle.attention(inp["q"][lo:hi], inp["k"][lo:hi], inp["v"][lo:hi], ra, inp["seq_mask"][lo:hi].numpy(),
+                            w.block, w.r)
+    # pad to the largest shard so all_gather sees equal shapes
+    maxn = max(b - a for a, b in (batch_shard(w.B, world, r) for r in range(world)))
+    buf = torch.zeros((maxn,) + part.shape[1:], dtype=torch.float64)
+    buf[: hi - lo] = torch.from_numpy(part)
+    gathered = [torch.zeros_like(buf) for _ in range(world)]
+    dist.all_gather(gathered, buf)
+    if rank == 0:
+        pieces = [g[: b - a] for g, (a, b) in zip(gathered, (batch_shard(w.B, world, r) for r in range(world)))]
+        full = torch.cat(pieces).numpy()
+        ref = oracle.attention(inp["q"], inp["k"], inp["v"], ra, inp["seq_mask"].numpy(), w.block, w.r)
+        np.save(result_path, np.array([np.abs(full - ref).max()]))
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+def test_two_gloo_ranks_equal_single_process(tmp_path):
+    path = str(tmp_path / "res.npy")
+    mp.start_processes(_worker, args=(2, _free_port(), path), nprocs=2, join=True, start_method="spawn")
+    assert float(np.load(path)[0]) == 0.0
