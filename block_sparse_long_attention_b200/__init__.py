@@ -50,6 +50,8 @@ def _load():
         "bigbird_pattern_table": (I, [P, I, I, I, I, P]),
         "bigbird_device_status": (I, [P, ctypes.POINTER(ctypes.c_uint32)]),
         "bigbird_status_string": (ctypes.c_char_p, [I]),
+        "bigbird_attn_fwd_noalloc": (I, [P, P, P, P, P, P, I, I, I, I, I, I, I, U, P]),
+        "bigbird_attn_noalloc_scratch_bytes": (Z, []),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)

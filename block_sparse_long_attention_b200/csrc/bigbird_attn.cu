@@ -1114,3 +1114,54 @@ int bigbird_device_status(void* stream_, uint32_t* host_status) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------- no-allocation entry point
+//
+// Some callers cannot allocate device memory while they run this op: an
+// inference server or real-time pipeline that reserves all device memory at
+// start-up and forbids allocation (and the device-wide synchronisation that
+// cudaMalloc/cudaFree can cause) inside its steady-state loop. For them,
+// bigbird_attn_fwd_noalloc uses this fixed scratch region, which lives in the
+// library's module: every GPU that loads the library holds it until the
+// process exits.
+
+namespace bb {
+
+constexpr size_t kStaticScratchBytes = size_t(32) << 20;  // 32 MiB
+
+static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
+
+// Device address of g_static_scratch on device `dev` (which must be current).
+// The host-side name is only a stand-in for the symbol: a kernel must be given
+// this looked-up address, never &g_static_scratch. Looked up once per device.
+static void* static_scratch_address(int dev) {
+  static void* addr[64];
+  static std::once_flag once[64];
+  if (dev < 0 || dev >= 64) return nullptr;
+  std::call_once(once[dev], [dev] {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_static_scratch) == cudaSuccess) addr[dev] = ptr;
+  });
+  return addr[dev];
+}
+
+}  // namespace bb
+
+extern "C" int bigbird_attn_fwd_noalloc(const void* q, const void* k, const void* v, const int32_t* rand_attn,
+                                        const uint8_t* seq_mask, void* out, int B, int H, int L, int d, int block,
+                                        int r, int out_dtype, unsigned flags, void* stream) {
+  // The debug checks copy rand_attn into a host buffer that they allocate.
+  if (flags & BB_FLAG_DEBUG_CHECKS) return BB_ERR_UNSUPPORTED;
+  bb::Plan pl;
+  const int st = bb::make_plan(B, H, L, d, block, r, flags, pl);
+  if (st != BB_OK) return st;
+  if (pl.ws_bytes > bb::kStaticScratchBytes) return BB_ERR_UNSUPPORTED;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return BB_ERR_CUDA;
+  void* scratch = bb::static_scratch_address(dev);
+  if (!scratch) return BB_ERR_CUDA;
+  return bigbird_attn_fwd_ex(q, k, v, rand_attn, seq_mask, out, B, H, L, d, block, r, out_dtype, flags, scratch,
+                             bb::kStaticScratchBytes, stream);
+}
+
+extern "C" size_t bigbird_attn_noalloc_scratch_bytes(void) { return bb::kStaticScratchBytes; }

@@ -166,6 +166,36 @@ int bigbird_pattern_table(const int32_t* host_ra, int H, int L, int block, int r
  */
 int bigbird_device_status(void* stream, uint32_t* host_status);
 
+/*
+ * bigbird_attn_fwd_noalloc -- bigbird_attn_fwd_ex without any device memory
+ * allocation. (The pages have no counterpart: this entry point exists for
+ * callers that cannot allocate device memory while they run, e.g. a server or
+ * real-time loop that reserves all GPU memory at start-up and must not hit the
+ * allocator, or its device-wide synchronisation, inside a step.)
+ *
+ * The scratch for the split global rows comes from a fixed region of
+ * bigbird_attn_noalloc_scratch_bytes() bytes (32 MiB) that the library's module
+ * holds on every GPU that loads it, until the process exits. Arguments and
+ * results are those of bigbird_attn_fwd_ex, except:
+ *   - there is no workspace argument;
+ *   - a problem whose scratch need (bigbird_attn_workspace_size) exceeds the
+ *     fixed region returns BB_ERR_UNSUPPORTED before anything is launched
+ *     (32 MiB covers, e.g., B*H = 48 heads at L = 4096 or 8 heads at L = 32768);
+ *   - BB_FLAG_DEBUG_CHECKS returns BB_ERR_UNSUPPORTED (that check allocates a
+ *     host buffer).
+ * The first call on a device looks up the region's device address (once per
+ * device, with that device current); make that first call before any stream
+ * capture. All calls share the one region and every call rewrites what it
+ * uses (nothing needs to start at zero): calls that overlap on the GPU -- on
+ * different streams, or from different threads -- race on it.
+ */
+int bigbird_attn_fwd_noalloc(const void* q, const void* k, const void* v, const int32_t* rand_attn,
+                             const uint8_t* seq_mask, void* out, int B, int H, int L, int d, int block, int r,
+                             int out_dtype, unsigned flags, void* stream);
+
+/* Size in bytes of the fixed scratch region of bigbird_attn_fwd_noalloc. */
+size_t bigbird_attn_noalloc_scratch_bytes(void);
+
 /* Static, human-readable text of a bb_status. */
 const char* bigbird_status_string(int status);
 
