@@ -287,7 +287,10 @@ def run_cuda(args):
         "roofline": roof,
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                 "ms_per_step": e2e_ms},
-        "gpu_launches": (2 if (sparse and bb.workspace_size(w.B, w.H, w.L) > 0) else 1) * args.steps * reps,
+        # per forward call: the attention kernel, plus the merge kernel when the
+        # global rows are split into key ranges (sparse and more than 8 blocks);
+        # the 4-byte counter reset before each call is a cudaMemsetAsync
+        "gpu_launches": (2 if (sparse and w.L // w.block > 8) else 1) * args.steps * reps,
         "clocks": clocks,
     }
     if rank == 0:

@@ -88,7 +88,7 @@ struct UnitInfo {
   int32_t qtop;  // query block of rows 0..63
   int32_t qbot;  // query block of rows 64..127, or -1
   int32_t split; // key range index of a partial global unit, or -1
-  int32_t pad_;
+  int32_t stop;  // 1: no more units for this CTA (every role leaves its loop)
   int32_t kb[kMaxList];
   uint64_t vm[kMaxList];  // bit c set: key c of the block is valid
   uint8_t hm[kMaxList];   // bit 0: rows 0..63 use the block, bit 1: rows 64..127
@@ -104,11 +104,12 @@ struct FwdParams {
   float* part_o;   // [BH, nsplit, 128, 64]
   float* part_ml;  // [BH, nsplit, 128, 2]
   uint32_t* status;
+  int* sched;       // unit tickets handed out so far beyond the first gridDim.x (zeroed before launch)
   int B, H, L, nb, r, BH;
   int sparse;
   int nsplit;        // key ranges per global unit (1 = write the output directly)
   int split_blocks;  // key blocks per range
-  int n_glob_units;
+  int n_pair_units;  // pair units come first (they are the longer ones)
   int n_pairs;       // pair units per head
   int total_units;
   int out_f32;
@@ -173,7 +174,8 @@ __device__ void build_unit(const FwdParams& p, int u, UnitInfo& ui, int lane) {
     ui.hm[n] = static_cast<uint8_t>(hm);
     ++n;
   };
-  if (u < p.n_glob_units) {
+  if (u >= p.n_pair_units) {
+    u -= p.n_pair_units;
     int bh, s, qtop, qbot;
     if (p.sparse) {
       bh = u / p.nsplit;
@@ -198,9 +200,10 @@ __device__ void build_unit(const FwdParams& p, int u, UnitInfo& ui, int lane) {
       ui.qbot = qbot;
       ui.split = p.nsplit > 1 ? s : -1;
       ui.n = n;
+      ui.stop = 0;
     }
   } else {
-    const int v = u - p.n_glob_units;
+    const int v = u;
     const int bh = v / p.n_pairs;
     const int pp = v % p.n_pairs;
     const int qtop = 1 + 2 * pp;
@@ -230,6 +233,7 @@ __device__ void build_unit(const FwdParams& p, int u, UnitInfo& ui, int lane) {
       ui.qbot = qbot;
       ui.split = -1;
       ui.n = n;
+      ui.stop = 0;
     }
   }
 }
@@ -267,11 +271,15 @@ __device__ void prep_unit(const FwdParams& p, int u, UnitInfo& ui, int lane) {
 }
 
 // Unit preparation, up to four units ahead of the TMA warp: slot ut & 3 is
-// refilled once every consumer of unit ut - 4 has released it.
+// refilled once every consumer of unit ut - 4 has released it. The prep warp
+// also schedules: a CTA's first unit is blockIdx.x, every later one is a
+// ticket from a device-wide counter (units are numbered longest first), so
+// CTAs that run faster take more units and all finish together. Once the
+// tickets run out it publishes a stop slot, which ends every role's loop.
 __device__ void prep_role(SharedStorage& s, const FwdParams& p) {
   const int lane = threadIdx.x & 31;
-  uint32_t ut = 0;
-  for (int u = blockIdx.x; u < p.total_units; u += gridDim.x, ++ut) {
+  int u = blockIdx.x;
+  for (uint32_t ut = 0;; ++ut) {
     const int slot = ut & 3;
     int ok = 1;
     if (lane == 0) ok = mbar_wait(smem_u32(&s.info_empty[slot]), ((ut >> 2) & 1) ^ 1);
@@ -279,12 +287,22 @@ __device__ void prep_role(SharedStorage& s, const FwdParams& p) {
       if (lane == 0) flag_timeout(s, p);
       return;
     }
-    prep_unit(p, u, s.unit[slot], lane);
+    UnitInfo& ui = s.unit[slot];
+    if (u >= p.total_units) {
+      if (lane == 0) {
+        ui.stop = 1;
+        mbar_arrive(smem_u32(&s.info_full[slot]));
+      }
+      return;
+    }
+    // Claim the next unit now, so the atomic's round trip overlaps this one's preparation.
+    int next = 0;
+    if (lane == 0) next = static_cast<int>(gridDim.x) + atomicAdd(p.sched, 1);
+    prep_unit(p, u, ui, lane);
     if (lane == 0) mbar_arrive(smem_u32(&s.info_full[slot]));
     // Pull the unit's tiles into L2 now (it is up to four units ahead of the
     // TMA warp), so its TMA loads hit L2 instead of HBM: one 8 KB tile per
     // lane, lanes 0..n-1 K, n..2n-1 V, 2n and 2n+1 the query blocks.
-    const UnitInfo& ui = s.unit[slot];
     const size_t row0 = static_cast<size_t>(ui.bh) * p.L;
     const int n = ui.n;
     for (int t = lane; t < 2 * n + 2; t += 32) {
@@ -295,6 +313,7 @@ __device__ void prep_role(SharedStorage& s, const FwdParams& p) {
       else { base = p.q; blk = (t == 2 * n) ? ui.qtop : ui.qbot; }
       if (blk >= 0) prefetch_l2_bulk(base + (row0 + static_cast<size_t>(blk) * kBlock) * kHeadDim, kTileBytes);
     }
+    u = __shfl_sync(0xffffffffu, next, 0);
   }
 }
 
@@ -302,9 +321,10 @@ __device__ void prep_role(SharedStorage& s, const FwdParams& p) {
 // range) in the order the TMA warp loads them; the P.V MMA waits for v_conv.
 __device__ void convert_role(SharedStorage& s, const FwdParams& p) {
   const int lane = threadIdx.x & 31;
-  uint32_t ut = 0, gv = 0;
-  for (int u = blockIdx.x; u < p.total_units; u += gridDim.x, ++ut) {
+  uint32_t gv = 0;
+  for (uint32_t ut = 0;; ++ut) {
     if (!warp_wait(smem_u32(&s.info_full[ut & 3]), (ut >> 2) & 1)) { if (lane == 0) flag_timeout(s, p); return; }
+    if (s.unit[ut & 3].stop) break;
     const int n = s.unit[ut & 3].n;
     const int nch = chunk_count(n);
     for (int c = 0; c < nch; ++c, ++gv) {
@@ -338,9 +358,8 @@ __device__ void producer_role(SharedStorage& s, const FwdParams& p, const CUtens
   const int lane = threadIdx.x & 31;
   const uint64_t pol_kv = l2_policy_evict_last();
   const uint64_t pol_q = l2_policy_evict_first();
-  if (static_cast<int>(blockIdx.x) >= p.total_units) return;
   uint32_t kut = 0, vut = 0, gk = 0, gv = 0;
-  int ku = blockIdx.x, kc = 0, vc = 0;
+  int kc = 0, vc = 0;
   bool kdone = false;
   while (!(kdone && gv == gk)) {
     if (!kdone) {
@@ -351,6 +370,10 @@ __device__ void producer_role(SharedStorage& s, const FwdParams& p, const CUtens
         return;
       }
       const UnitInfo& ui = s.unit[kut & 3];
+      if (ui.stop) {
+        kdone = true;
+        continue;
+      }
       const int n = ui.n;
       const int nch = chunk_count(n);
       const int32_t row0 = ui.bh * p.L;
@@ -387,8 +410,6 @@ __device__ void producer_role(SharedStorage& s, const FwdParams& p, const CUtens
       if (++kc == nch) {
         kc = 0;
         ++kut;
-        ku += gridDim.x;
-        kdone = ku >= p.total_units;
       }
     }
     if (gv + 1 < gk || (kdone && gv < gk)) {
@@ -433,9 +454,11 @@ __device__ void mma_role(SharedStorage& s, const FwdParams& p, uint32_t tmem) {
   const uint32_t idesc_s2 = idesc_f32acc(kRows, 2 * kBlock, true, false);  // S of a 2-block chunk
   const uint32_t idesc_s1 = idesc_f32acc(kRows, kBlock, true, false);      // S of a 1-block chunk
   const uint32_t idesc_o = idesc_f32acc(kRows, kHeadDim, false, true);     // fp16 P . fp16 V
-  uint32_t ut = 0, gc = 0;
+  uint32_t gc = 0;
   bool ok = true;
-  for (int u = blockIdx.x; u < p.total_units && ok; u += gridDim.x, ++ut) {
+  for (uint32_t ut = 0; ok; ++ut) {
+    if (!mbar_wait(smem_u32(&s.info_full[ut & 3]), (ut >> 2) & 1)) { ok = false; break; }
+    if (s.unit[ut & 3].stop) break;
     const int qs = ut & 1;
     if (!mbar_wait(smem_u32(&s.q_full[qs]), (ut >> 1) & 1)) { ok = false; break; }
     const int n = s.unit[ut & 3].n;
@@ -610,10 +633,12 @@ __device__ void softmax_role(SharedStorage& s, const FwdParams& p, uint32_t tmem
   const int lane = tid & 31;
   const int half = warp >> 1;   // 0: rows 0..63, 1: rows 64..127
   const uint32_t lane_addr = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-  uint32_t ut = 0, gc = 0;
-  for (int u = blockIdx.x; u < p.total_units; u += gridDim.x, ++ut) {
-    if (!warp_wait(smem_u32(&s.q_full[ut & 1]), (ut >> 1) & 1)) { flag_timeout(s, p); return; }
+  uint32_t gc = 0;
+  for (uint32_t ut = 0;; ++ut) {
+    if (!warp_wait(smem_u32(&s.info_full[ut & 3]), (ut >> 2) & 1)) { flag_timeout(s, p); return; }
     const UnitInfo& ui = s.unit[ut & 3];
+    if (ui.stop) break;
+    if (!warp_wait(smem_u32(&s.q_full[ut & 1]), (ut >> 1) & 1)) { flag_timeout(s, p); return; }
     const int n = ui.n;
     const int nch = chunk_count(n);
     const int bh = ui.bh;
@@ -968,6 +993,8 @@ static DeviceInfo* device_info(int dev) {
   return &di;
 }
 
+constexpr size_t kSchedBytes = 256;  // the scheduling counter's slot at the start of the workspace
+
 struct Plan {
   int nb = 0;
   bool sparse = false;
@@ -990,8 +1017,11 @@ static int make_plan(int B, int H, int L, int d, int block, int r, unsigned flag
     pl.split_blocks = pl.nb;  // nb <= 5 + 2r <= kMaxList
     pl.nsplit = 1;
   }
+  // Workspace: the unit-ticket counter, then (split global rows only) the
+  // partial outputs [B*H, nsplit, 128, 64] and their (max, sum) [B*H, nsplit, 128, 2].
+  pl.ws_bytes = kSchedBytes;
   if (pl.nsplit > 1)
-    pl.ws_bytes = static_cast<size_t>(B) * H * pl.nsplit * kRows * (kHeadDim + 2) * sizeof(float);
+    pl.ws_bytes += static_cast<size_t>(B) * H * pl.nsplit * kRows * (kHeadDim + 2) * sizeof(float);
   return BB_OK;
 }
 
@@ -1059,13 +1089,13 @@ int bigbird_attn_fwd_ex(const void* q, const void* k, const void* v, const int32
   p.nsplit = pl.nsplit;
   p.split_blocks = pl.split_blocks;
   if (pl.sparse) {
-    p.n_glob_units = p.BH * pl.nsplit;
     p.n_pairs = (pl.nb - 2 + 1) / 2;
-    p.total_units = p.n_glob_units + p.BH * p.n_pairs;
+    p.n_pair_units = p.BH * p.n_pairs;
+    p.total_units = p.n_pair_units + p.BH * pl.nsplit;
   } else {
-    p.n_glob_units = p.BH * ((pl.nb + 1) / 2);
     p.n_pairs = 0;
-    p.total_units = p.n_glob_units;
+    p.n_pair_units = 0;
+    p.total_units = p.BH * ((pl.nb + 1) / 2);
   }
   p.out_f32 = out_dtype == BB_OUT_F32 ? 1 : 0;
   p.scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(d));
@@ -1075,13 +1105,19 @@ int bigbird_attn_fwd_ex(const void* q, const void* k, const void* v, const int32
 
   void* ws = workspace;
   bool owned = false;
-  if (pl.ws_bytes > 0 && !ws) {
+  if (!ws) {
     if (cudaMallocAsync(&ws, pl.ws_bytes, stream) != cudaSuccess) return BB_ERR_CUDA;
     owned = true;
   }
-  if (pl.ws_bytes > 0) {
-    p.part_o = static_cast<float*>(ws);
+  p.sched = static_cast<int*>(ws);
+  if (pl.nsplit > 1) {
+    p.part_o = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + kSchedBytes);
     p.part_ml = p.part_o + static_cast<size_t>(p.BH) * pl.nsplit * kRows * kHeadDim;
+  }
+  // Unit tickets start from zero on every call.
+  if (cudaMemsetAsync(p.sched, 0, sizeof(int), stream) != cudaSuccess) {
+    if (owned) cudaFreeAsync(ws, stream);
+    return BB_ERR_CUDA;
   }
 
   const int grid = std::min(p.total_units, 2 * di->sms);

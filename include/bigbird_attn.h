@@ -88,8 +88,11 @@ int bigbird_attn_fwd(const void* q, const void* k, const void* v, const int32_t*
 
 /*
  * Bytes of device scratch bigbird_attn_fwd_ex needs for these sizes and
- * flags (0 when none). The scratch holds the partial (unnormalised output,
- * running max, running sum) of each key range of the split global rows.
+ * flags (0 if the sizes are invalid). The scratch starts with a 256-byte slot
+ * for the counter through which the CTAs share out the work units (every call
+ * zeroes it with cudaMemsetAsync on its stream before the launch); when the
+ * global rows are split into key ranges (sparse pattern, nb > 8) it also holds
+ * each range's partial result (unnormalised output, running max, running sum).
  */
 size_t bigbird_attn_workspace_size(int B, int H, int L, int d, int block, int r, unsigned flags);
 
@@ -100,8 +103,9 @@ size_t bigbird_attn_workspace_size(int B, int H, int L, int d, int block, int r,
  *   flags      BB_FLAG_* bits.
  *   workspace  device, 256-byte aligned, at least
  *              bigbird_attn_workspace_size(...) bytes; NULL = allocate with
- *              cudaMallocAsync on `stream` when needed. Calls that share a
- *              workspace must not overlap on the GPU.
+ *              cudaMallocAsync on `stream` (freed with cudaFreeAsync after
+ *              the launch). Its contents need no initialisation. Calls that
+ *              share a workspace must not overlap on the GPU.
  */
 int bigbird_attn_fwd_ex(const void* q, const void* k, const void* v, const int32_t* rand_attn,
                         const uint8_t* seq_mask, void* out, int B, int H, int L, int d, int block, int r,

@@ -111,10 +111,11 @@ def test_fallback_rule_matches_oracle():
 
 
 def test_workspace_size():
-    assert bb.workspace_size(1, 2, 704) == 0  # fallback: no split rows
+    sched = 256  # the work-unit counter's slot
+    assert bb.workspace_size(1, 2, 704) == sched  # fallback: no split rows
     nb = 4096 // 64
     nsplit = (nb + 7) // 8
-    assert bb.workspace_size(4, 12, 4096) == 4 * 12 * nsplit * 128 * 66 * 4
+    assert bb.workspace_size(4, 12, 4096) == sched + 4 * 12 * nsplit * 128 * 66 * 4
     assert bb.workspace_size(1, 1, 1000) == 0  # invalid sizes
 
 
