@@ -572,16 +572,6 @@ __device__ __forceinline__ void piece_exp(const uint32_t (&r)[32], uint64_t scal
   }
 }
 
-// Multiply 16 packed fp16x2 values by f (rare path: a later max increase).
-__device__ __forceinline__ void scale_packed16(uint32_t* pk, float f) {
-#pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    __half2 h = *reinterpret_cast<__half2*>(&pk[i]);
-    const float2 v = __half22float2(h);
-    pk[i] = pack_f16x2(v.x * f, v.y * f);
-  }
-}
-
 // Per-row online-softmax state of one unit.
 struct RowState {
   float m_ref;     // reference max (scaled log2 units)
@@ -590,11 +580,17 @@ struct RowState {
   float o_factor;  // rescale owed to the O accumulator
 };
 
-// Max, rescale bookkeeping and exponentials of one 32-column piece.
-// hi: the block's lo piece is already in pk[-16..0).
-__device__ __forceinline__ void process_piece(uint32_t (&r)[32], bool mixed, uint32_t vm, float off, bool hi,
-                                              const FwdParams& p, uint32_t* pk, RowState& st) {
-  const float mx = piece_prepare(r, mixed, vm, p.bias_raw, off) * p.scale_log2;
+// One 64-key block of a row (ra: keys 0..31, rb: keys 32..63): one max, at
+// most one change of the reference max, then 64 exponentials packed to fp16
+// into pk. The reference moves only at block boundaries, so P already written
+// never needs rescaling; O and the running sums do (o_factor, l_run, acc).
+__device__ __forceinline__ void process_block(uint32_t (&ra)[32], uint32_t (&rb)[32], uint64_t vm,
+                                              const FwdParams& p, uint32_t (&pk)[32], RowState& st) {
+  const bool mixed = block_mixed(vm);
+  const float off = block_offset(vm, p.bias_raw);
+  const float ma = piece_prepare(ra, mixed, static_cast<uint32_t>(vm), p.bias_raw, off);
+  const float mb = piece_prepare(rb, mixed, static_cast<uint32_t>(vm >> 32), p.bias_raw, off);
+  const float mx = fmaxf(ma, mb) * p.scale_log2;
   const bool need = mx > st.m_ref + kRescaleThreshold;
   if (__any_sync(0xffffffffu, need)) {
     float f = 1.f;
@@ -607,10 +603,12 @@ __device__ __forceinline__ void process_piece(uint32_t (&r)[32], bool mixed, uin
     st.acc0 = f2_fma(st.acc0, f2, 0ull);
     st.acc1 = f2_fma(st.acc1, f2, 0ull);
     st.o_factor *= f;
-    if (hi) scale_packed16(pk - 16, f);
   }
   const float o = fmaf(off, p.scale_log2, -st.m_ref);
-  piece_exp(r, f2_pack(p.scale_log2, p.scale_log2), f2_pack(o, o), pk, st.acc0, st.acc1);
+  const uint64_t scale2 = f2_pack(p.scale_log2, p.scale_log2);
+  const uint64_t off2 = f2_pack(o, o);
+  piece_exp(ra, scale2, off2, pk, st.acc0, st.acc1);
+  piece_exp(rb, scale2, off2, pk + 16, st.acc0, st.acc1);
 }
 
 // O (64 fp32 columns of this thread's row) *= f, in 16-column pieces.
@@ -661,32 +659,22 @@ __device__ void softmax_role(SharedStorage& s, const FwdParams& p, uint32_t tmem
       st.o_factor = 1.f;
       uint32_t pk[32];
       uint32_t ra[32], rb[32];
-      // Single pass over the used blocks in 32-column pieces; the TMEM read of
-      // piece k+1 is in flight while piece k is exponentiated. S is released
-      // as soon as its last piece has been read.
-      if (used0 || used1) {
-        tmem_ld32(lane_addr + kColS + (used0 ? 0 : kBlock), ra);
-        tmem_wait_ld();
-      } else {
+      // Each used block is read whole (two 32-column loads) and processed in
+      // one pass; S is released once its last used block has been read.
+      auto release_s = [&]() {
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&s.s_free));
-      }
+      };
       // ---- block 0
       if (used0) {
-        const uint64_t vm = ui.vm[e0];
-        const bool mixed = block_mixed(vm);
-        const float off = block_offset(vm, p.bias_raw);
+        tmem_ld32(lane_addr + kColS, ra);
         tmem_ld32(lane_addr + kColS + 32, rb);
-        process_piece(ra, mixed, static_cast<uint32_t>(vm), off, false, p, pk, st);
         tmem_wait_ld();
-        if (!used1) {
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(smem_u32(&s.s_free));
-        }
-        process_piece(rb, mixed, static_cast<uint32_t>(vm >> 32), off, true, p, pk + 16, st);
+        if (!used1) release_s();
+        process_block(ra, rb, ui.vm[e0], p, pk, st);
       } else {
+        if (!used1) release_s();
 #pragma unroll
         for (int i = 0; i < 32; ++i) pk[i] = 0u;
       }
@@ -710,20 +698,11 @@ __device__ void softmax_role(SharedStorage& s, const FwdParams& p, uint32_t tmem
       // ---- block 1
       if (nblk == 2) {
         if (used1) {
-          const uint64_t vm = ui.vm[e0 + 1];
-          const bool mixed = block_mixed(vm);
-          const float off = block_offset(vm, p.bias_raw);
-          if (used0) {
-            tmem_ld32(lane_addr + kColS + kBlock, ra);
-            tmem_wait_ld();
-          }
+          tmem_ld32(lane_addr + kColS + kBlock, ra);
           tmem_ld32(lane_addr + kColS + kBlock + 32, rb);
-          process_piece(ra, mixed, static_cast<uint32_t>(vm), off, false, p, pk, st);
           tmem_wait_ld();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(smem_u32(&s.s_free));
-          process_piece(rb, mixed, static_cast<uint32_t>(vm >> 32), off, true, p, pk + 16, st);
+          release_s();
+          process_block(ra, rb, ui.vm[e0 + 1], p, pk, st);
         } else {
 #pragma unroll
           for (int i = 0; i < 32; ++i) pk[i] = 0u;
