@@ -16,29 +16,34 @@
 //     "随机块掩码是如何生成的"; HF-Pegasus, section "三类注意力组合"]. A half that
 //     does not use a block writes P = 0 for it, so the pair shares every MMA.
 //
-// A unit's key blocks are processed in chunks of two (128 keys): one
-// S = Q K^T MMA of N = 128 (the tensor core needs N >= 128 per instruction to
-// run at full rate), one softmax round, one O += P V MMA of K = 128.
+// Units are handed out dynamically (longest first): a CTA's first unit is its
+// block index, later ones are tickets from a device-wide counter.
 //
-// Warp roles (256 threads, two CTAs per SM):
+// A unit's key blocks are processed one at a time through a serial chain:
+// S = Q K^T (tcgen05 SS-MMA, 128x64x16 steps) -> softmax -> fp16 P written
+// back over the S columns -> O += P V (TS-MMA, A = P from TMEM). Each CTA
+// needs only 128 TMEM columns, so four CTAs (four independent chains) share
+// an SM and interleave on its tensor pipe, exp unit and issue slots.
+//
+// Warp roles (256 threads, 64 registers, four CTAs per SM):
 //   warps 0-3  softmax and epilogue, one query row per thread (thread t owns
 //              TMEM lane t);
-//   warp 4     TMA: Q per unit, K and V per chunk on separate rings, the V
-//              stream one chunk behind the K stream (K is needed a round
-//              earlier);
+//   warp 4     TMA: Q per unit (one buffer, loaded once the previous unit's
+//              last S is done), K and V per block on 2-deep rings;
 //   warp 5     TMEM allocation and the tcgen05 MMAs (one thread);
-//   warp 6     unit preparation (key-block list, half masks, key-validity
-//              bits) up to four units ahead, so its dependent global loads
-//              never stall the pipeline;
-//   warp 7     converts each V chunk bf16 -> fp16 in shared memory.
+//   warp 6     scheduling and unit preparation (key-block list, half masks,
+//              key-validity bits) up to four units ahead, plus L2 prefetch,
+//              so its dependent global loads never stall the pipeline;
+//   warp 7     converts each V block bf16 -> fp16 in shared memory.
 //
-// TMEM (256 columns): S [0,128) fp32, P [128,192) fp16 (written by the softmax,
-// read by the TS MMA), O [192,256) fp32. Because P has its own columns, the
-// next chunk's S MMA is issued as soon as the softmax has read S, and runs
-// while the softmax computes the exponentials.
+// TMEM (128 columns): S [0,64) fp32, with P (fp16, 32 columns) written over
+// [0,32) once read; O [64,128) fp32. The next S waits for the P.V that reads
+// P (tcgen05 only orders MMAs that share an accumulator).
 //
-// Softmax: the reference max moves only when it grows by more than 2^8 (the O
-// rescale is skipped otherwise; the final O / l is exact either way). Padded
+// Softmax: a max pass and an exponential pass over each block's 64 columns;
+// the reference max moves only at block boundaries and only when it grows by
+// more than 2^8 (the O rescale is skipped otherwise; the final O / l is exact
+// either way). Padded
 // keys get -10000 added to the scaled score. P.V runs in fp16: P is written as
 // fp16 and each V tile is converted bf16 -> fp16 in shared memory (exact in the
 // fp16 normal range), which keeps three more mantissa bits of P than bf16.
@@ -60,19 +65,17 @@ namespace bb {
 constexpr int kBlock = 64;             // tokens per block
 constexpr int kHeadDim = 64;           // head dimension
 constexpr int kRows = 128;             // query rows per unit (two blocks)
-constexpr int kChunk = 2;              // key blocks per chunk
-constexpr int kKStages = 2;            // K ring depth (chunks)
-constexpr int kVStages = 2;            // V ring depth (chunks)
+constexpr int kKStages = 2;            // K ring depth (blocks)
+constexpr int kVStages = 2;            // V ring depth (blocks)
 constexpr int kMaxList = 40;           // key blocks per unit
 constexpr int kMaxR = 16;              // random blocks per row supported
 constexpr int kSplitBlocks = 8;        // key blocks per global-row range
 constexpr int kThreads = 256;
+constexpr int kCtasPerSm = 4;          // four independent unit pipelines per SM
 constexpr uint32_t kTileBytes = kBlock * kHeadDim * 2;  // one 64x64 bf16 tile
-constexpr uint32_t kChunkBytes = kChunk * kTileBytes;
-constexpr uint32_t kTmemCols = 256;
-constexpr uint32_t kColS = 0;          // S: 128 fp32 columns
-constexpr uint32_t kColP = 128;        // P: 128 fp16 keys = 64 columns
-constexpr uint32_t kColO = 192;        // O: 64 fp32 columns
+constexpr uint32_t kTmemCols = 128;
+constexpr uint32_t kColS = 0;          // S of one key block: 64 fp32 columns; P (fp16) overwrites the first 32
+constexpr uint32_t kColO = 64;         // O: 64 fp32 columns
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr float kNegInit = -1.0e30f;
 
@@ -118,25 +121,22 @@ struct FwdParams {
 };
 
 struct __align__(1024) SharedStorage {
-  uint8_t q[2][kRows * kHeadDim * 2];   // Q per unit, double buffered (SW128)
-  uint8_t k[kKStages][kChunkBytes];     // K chunk = two adjacent 64x64 tiles
-  uint8_t v[kVStages][kChunkBytes];     // V chunk
+  uint8_t q[kRows * kHeadDim * 2];      // Q of the current unit (two 64x64 tiles, SW128)
+  uint8_t k[kKStages][kTileBytes];      // K blocks
+  uint8_t v[kVStages][kTileBytes];      // V blocks, converted to fp16 in place
   UnitInfo unit[4];
   uint64_t info_full[4];
   uint64_t info_empty[4];
-  uint64_t q_full[2];
-  uint64_t q_free[2];
+  uint64_t q_full;
+  uint64_t q_free;
   uint64_t k_full[kKStages];
   uint64_t k_empty[kKStages];
   uint64_t v_full[kVStages];
   uint64_t v_conv[kVStages];
   uint64_t v_empty[kVStages];
-  uint64_t s_full;
-  uint64_t s_free;
-  uint64_t p_lo;     // P of the chunk's block 0 written (4 softmax warps)
-  uint64_t p_hi;     // P of block 1 written (always arrived, also for one-block chunks)
-  uint64_t pv_lo;    // P.V of block 0 complete
-  uint64_t pv_hi;    // P.V of block 1 complete (committed for every chunk)
+  uint64_t s_full;   // S of the current key block is in TMEM
+  uint64_t p_full;   // P of the current key block is in TMEM (4 softmax warps)
+  uint64_t pv_done;  // P.V of the current key block is complete (S/P columns reusable)
   uint64_t o_full;
   uint64_t o_free;
   uint32_t tmem_base;
@@ -153,8 +153,6 @@ __device__ __forceinline__ void flag_timeout(SharedStorage& s, const FwdParams& 
 __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity) {
   return __all_sync(0xffffffffu, mbar_wait(bar, parity));
 }
-
-__device__ __forceinline__ int chunk_count(int n) { return (n + kChunk - 1) / kChunk; }
 
 // Decode unit u and build its key-block list. Called by a whole warp: the
 // lanes fetch the unit's random entries in parallel, lane 0 builds the list.
@@ -317,7 +315,7 @@ __device__ void prep_role(SharedStorage& s, const FwdParams& p) {
   }
 }
 
-// V chunks are converted bf16 -> fp16 in place (exact in the fp16 normal
+// V blocks are converted bf16 -> fp16 in place (exact in the fp16 normal
 // range) in the order the TMA warp loads them; the P.V MMA waits for v_conv.
 __device__ void convert_role(SharedStorage& s, const FwdParams& p) {
   const int lane = threadIdx.x & 31;
@@ -326,15 +324,12 @@ __device__ void convert_role(SharedStorage& s, const FwdParams& p) {
     if (!warp_wait(smem_u32(&s.info_full[ut & 3]), (ut >> 2) & 1)) { if (lane == 0) flag_timeout(s, p); return; }
     if (s.unit[ut & 3].stop) break;
     const int n = s.unit[ut & 3].n;
-    const int nch = chunk_count(n);
-    for (int c = 0; c < nch; ++c, ++gv) {
+    for (int e = 0; e < n; ++e, ++gv) {
       const int st = gv % kVStages;
-      const int nblk = min(kChunk, n - c * kChunk);
       if (!warp_wait(smem_u32(&s.v_full[st]), (gv / kVStages) & 1)) { if (lane == 0) flag_timeout(s, p); return; }
       uint4* vp = reinterpret_cast<uint4*>(s.v[st]) + lane;
-      const int nvec = nblk * (kTileBytes / 16) / 32;  // uint4 per lane
 #pragma unroll 4
-      for (int i = 0; i < nvec; ++i) {
+      for (int i = 0; i < static_cast<int>(kTileBytes / 16 / 32); ++i) {
         uint4 w = vp[32 * i];
         w.x = bf16x2_to_f16x2(w.x);
         w.y = bf16x2_to_f16x2(w.y);
@@ -351,20 +346,48 @@ __device__ void convert_role(SharedStorage& s, const FwdParams& p) {
   }
 }
 
-// Two cursors walk this CTA's chunk sequence: the K cursor (which also loads
-// each unit's Q when it enters the unit) and the V cursor one chunk behind it.
+// Two cursors walk this CTA's key blocks: the V cursor (at most as far as the
+// K cursor) and the K cursor, which also loads each unit's Q when it enters
+// the unit (single Q buffer: after every S of the previous unit is done).
 __device__ void producer_role(SharedStorage& s, const FwdParams& p, const CUtensorMap* tmQ, const CUtensorMap* tmK,
                               const CUtensorMap* tmV) {
   const int lane = threadIdx.x & 31;
   const uint64_t pol_kv = l2_policy_evict_last();
   const uint64_t pol_q = l2_policy_evict_first();
   uint32_t kut = 0, vut = 0, gk = 0, gv = 0;
-  int kc = 0, vc = 0;
+  int ke = 0, ve = 0;
   bool kdone = false;
   while (!(kdone && gv == gk)) {
+    // V first, so that the block the K cursor has just loaded gets its V
+    // before the K cursor can block on the next unit's Q buffer.
+    if (gv < gk) {
+      const UnitInfo& ui = s.unit[vut & 3];
+      int ok = 1;
+      if (lane == 0) {
+        const int st = gv % kVStages;
+        ok = mbar_wait(smem_u32(&s.v_empty[st]), ((gv / kVStages) & 1) ^ 1);
+        if (ok) {
+          const uint32_t vbar = smem_u32(&s.v_full[st]);
+          mbar_arrive_expect_tx(vbar, kTileBytes);
+          tma_load_2d(smem_u32(s.v[st]), tmV, vbar, 0, ui.bh * p.L + ui.kb[ve] * kBlock, pol_kv);
+        }
+      }
+      if (!__shfl_sync(0xffffffffu, ok, 0)) {
+        if (lane == 0) flag_timeout(s, p);
+        return;
+      }
+      ++gv;
+      if (++ve == ui.n) {
+        // both cursors are done with this unit's info
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&s.info_empty[vut & 3]));
+        ve = 0;
+        ++vut;
+      }
+    }
     if (!kdone) {
       int ok = 1;
-      if (kc == 0) ok = mbar_wait(smem_u32(&s.info_full[kut & 3]), (kut >> 2) & 1);
+      if (ke == 0) ok = mbar_wait(smem_u32(&s.info_full[kut & 3]), (kut >> 2) & 1);
       if (!__all_sync(0xffffffffu, ok)) {
         if (lane == 0) flag_timeout(s, p);
         return;
@@ -374,31 +397,24 @@ __device__ void producer_role(SharedStorage& s, const FwdParams& p, const CUtens
         kdone = true;
         continue;
       }
-      const int n = ui.n;
-      const int nch = chunk_count(n);
       const int32_t row0 = ui.bh * p.L;
       if (lane == 0) {
-        if (kc == 0) {
-          const int qs = kut & 1;
-          ok = mbar_wait(smem_u32(&s.q_free[qs]), ((kut >> 1) & 1) ^ 1);
+        if (ke == 0) {
+          ok = mbar_wait(smem_u32(&s.q_free), (kut & 1) ^ 1);
           if (ok) {
-            const uint32_t qbar = smem_u32(&s.q_full[qs]);
+            const uint32_t qbar = smem_u32(&s.q_full);
             mbar_arrive_expect_tx(qbar, ui.qbot >= 0 ? 2 * kTileBytes : kTileBytes);
-            tma_load_2d(smem_u32(s.q[qs]), tmQ, qbar, 0, row0 + ui.qtop * kBlock, pol_q);
-            if (ui.qbot >= 0)
-              tma_load_2d(smem_u32(s.q[qs]) + kTileBytes, tmQ, qbar, 0, row0 + ui.qbot * kBlock, pol_q);
+            tma_load_2d(smem_u32(s.q), tmQ, qbar, 0, row0 + ui.qtop * kBlock, pol_q);
+            if (ui.qbot >= 0) tma_load_2d(smem_u32(s.q) + kTileBytes, tmQ, qbar, 0, row0 + ui.qbot * kBlock, pol_q);
           }
         }
         if (ok) {
           const int st = gk % kKStages;
           ok = mbar_wait(smem_u32(&s.k_empty[st]), ((gk / kKStages) & 1) ^ 1);
           if (ok) {
-            const int e0 = kc * kChunk;
-            const int nblk = min(kChunk, n - e0);
             const uint32_t kbar = smem_u32(&s.k_full[st]);
-            mbar_arrive_expect_tx(kbar, nblk * kTileBytes);
-            for (int e = 0; e < nblk; ++e)
-              tma_load_2d(smem_u32(s.k[st]) + e * kTileBytes, tmK, kbar, 0, row0 + ui.kb[e0 + e] * kBlock, pol_kv);
+            mbar_arrive_expect_tx(kbar, kTileBytes);
+            tma_load_2d(smem_u32(s.k[st]), tmK, kbar, 0, row0 + ui.kb[ke] * kBlock, pol_kv);
           }
         }
       }
@@ -407,38 +423,9 @@ __device__ void producer_role(SharedStorage& s, const FwdParams& p, const CUtens
         return;
       }
       ++gk;
-      if (++kc == nch) {
-        kc = 0;
+      if (++ke == ui.n) {
+        ke = 0;
         ++kut;
-      }
-    }
-    if (gv + 1 < gk || (kdone && gv < gk)) {
-      const UnitInfo& ui = s.unit[vut & 3];
-      const int n = ui.n;
-      const int32_t row0 = ui.bh * p.L;
-      int ok = 1;
-      if (lane == 0) {
-        const int st = gv % kVStages;
-        ok = mbar_wait(smem_u32(&s.v_empty[st]), ((gv / kVStages) & 1) ^ 1);
-        if (ok) {
-          const int e0 = vc * kChunk;
-          const int nblk = min(kChunk, n - e0);
-          const uint32_t vbar = smem_u32(&s.v_full[st]);
-          mbar_arrive_expect_tx(vbar, nblk * kTileBytes);
-          for (int e = 0; e < nblk; ++e)
-            tma_load_2d(smem_u32(s.v[st]) + e * kTileBytes, tmV, vbar, 0, row0 + ui.kb[e0 + e] * kBlock, pol_kv);
-        }
-      }
-      if (!__shfl_sync(0xffffffffu, ok, 0)) {
-        if (lane == 0) flag_timeout(s, p);
-        return;
-      }
-      ++gv;
-      if (++vc == chunk_count(n)) {
-        // both cursors are done with this unit's info
-        if (lane == 0) mbar_arrive(smem_u32(&s.info_empty[vut & 3]));
-        vc = 0;
-        ++vut;
       }
     }
   }
@@ -446,92 +433,55 @@ __device__ void producer_role(SharedStorage& s, const FwdParams& p, const CUtens
 
 // ---------------------------------------------------------------- MMA issuer
 
-// Per chunk g: S(g) once the softmax has read S(g-1); then the P.V of the
-// previous chunk's block 1 (PV-hi, when its P is written) and of this chunk's
-// block 0 (PV-lo, written half way through the softmax). Splitting P.V in two
-// frees the P buffer in halves, so the softmax never waits for a whole P.V.
+// Per key block g of this CTA: S(g) = Q . K(g)^T into the S columns once the
+// previous block's P.V has consumed the P that shares them, then, once the
+// softmax has written P(g), O += P(g) . V(g). The chain is serial within a
+// CTA; the four CTAs of an SM interleave on the tensor pipe.
 __device__ void mma_role(SharedStorage& s, const FwdParams& p, uint32_t tmem) {
-  const uint32_t idesc_s2 = idesc_f32acc(kRows, 2 * kBlock, true, false);  // S of a 2-block chunk
-  const uint32_t idesc_s1 = idesc_f32acc(kRows, kBlock, true, false);      // S of a 1-block chunk
-  const uint32_t idesc_o = idesc_f32acc(kRows, kHeadDim, false, true);     // fp16 P . fp16 V
-  uint32_t gc = 0;
+  const uint32_t idesc_s = idesc_f32acc(kRows, kBlock, true, false);    // bf16 Q . K^T, N = 64
+  const uint32_t idesc_o = idesc_f32acc(kRows, kHeadDim, false, true);  // fp16 P . fp16 V
+  const uint32_t q_addr = smem_u32(s.q);
+  uint32_t g = 0;
   bool ok = true;
   for (uint32_t ut = 0; ok; ++ut) {
     if (!mbar_wait(smem_u32(&s.info_full[ut & 3]), (ut >> 2) & 1)) { ok = false; break; }
     if (s.unit[ut & 3].stop) break;
-    const int qs = ut & 1;
-    if (!mbar_wait(smem_u32(&s.q_full[qs]), (ut >> 1) & 1)) { ok = false; break; }
+    if (!mbar_wait(smem_u32(&s.q_full), ut & 1)) { ok = false; break; }
     const int n = s.unit[ut & 3].n;
-    const int nch = chunk_count(n);
-    const uint32_t q_addr = smem_u32(s.q[qs]);
-
-    // P.V of one block (bi = 0: lo, 1: hi) of chunk c.
-    auto issue_pv = [&](int c, int bi) -> bool {
-      const uint32_t g = gc + c;
-      const int st = g % kVStages;
-      const int nblk = min(kChunk, n - c * kChunk);
-      if (bi == 0) {
-        if (!mbar_wait(smem_u32(&s.v_conv[st]), (g / kVStages) & 1)) return false;
-        if (c == 0 && !mbar_wait(smem_u32(&s.o_free), (ut & 1) ^ 1)) return false;
-      }
-      if (!mbar_wait(smem_u32(bi == 0 ? &s.p_lo : &s.p_hi), g & 1)) return false;
+    for (int e = 0; e < n; ++e, ++g) {
+      const int kst = g % kKStages;
+      if (!mbar_wait(smem_u32(&s.k_full[kst]), (g / kKStages) & 1)) { ok = false; break; }
+      if (g >= 1 && !mbar_wait(smem_u32(&s.pv_done), (g - 1) & 1)) { ok = false; break; }
       tc_fence_after();
-      if (bi < nblk) {
-        const uint32_t v_addr = smem_u32(s.v[st]) + bi * kTileBytes;
+      const uint32_t k_addr = smem_u32(s.k[kst]);
 #pragma unroll
-        for (int kk = 0; kk < kBlock / 16; ++kk) {
-          const uint64_t bdesc = sdesc_sw128(v_addr + kk * 2048, 8192, 1024);
-          mma_ts(tmem + kColO, tmem + kColP + bi * 32 + kk * 8, bdesc, idesc_o,
-                 (c > 0 || bi > 0 || kk > 0) ? 1u : 0u);
-        }
-      }
-      if (bi == 0) {
-        mma_commit(smem_u32(&s.pv_lo));
-      } else {
-        mma_commit(smem_u32(&s.pv_hi));
-        mma_commit(smem_u32(&s.v_empty[st]));
-      }
-      return true;
-    };
-
-    for (int c = 0; c < nch && ok; ++c) {
-      const uint32_t g = gc + c;
-      const int st = g % kKStages;
-      const int nblk = min(kChunk, n - c * kChunk);
-      if (!mbar_wait(smem_u32(&s.k_full[st]), (g / kKStages) & 1)) { ok = false; break; }
-      if (g >= 1 && !mbar_wait(smem_u32(&s.s_free), (g - 1) & 1)) { ok = false; break; }
-      tc_fence_after();
-      const uint32_t k_addr = smem_u32(s.k[st]);
-#pragma unroll
-      for (int kk = 0; kk < kHeadDim / 16; ++kk) {
-        const uint64_t adesc = sdesc_sw128(q_addr + kk * 32, 16, 1024);
-        const uint64_t bdesc = sdesc_sw128(k_addr + kk * 32, 16, 1024);
-        mma_ss(tmem + kColS, adesc, bdesc, nblk == 2 ? idesc_s2 : idesc_s1, kk > 0 ? 1u : 0u);
-      }
+      for (int kk = 0; kk < kHeadDim / 16; ++kk)
+        mma_ss(tmem + kColS, sdesc_sw128(q_addr + kk * 32, 16, 1024), sdesc_sw128(k_addr + kk * 32, 16, 1024),
+               idesc_s, kk > 0 ? 1u : 0u);
       mma_commit(smem_u32(&s.s_full));
-      mma_commit(smem_u32(&s.k_empty[st]));
-      if (c >= 1 && !issue_pv(c - 1, 1)) { ok = false; break; }
-      if (!issue_pv(c, 0)) { ok = false; break; }
+      mma_commit(smem_u32(&s.k_empty[kst]));
+      if (e == n - 1) mma_commit(smem_u32(&s.q_free));
+      const int vst = g % kVStages;
+      if (!mbar_wait(smem_u32(&s.v_conv[vst]), (g / kVStages) & 1)) { ok = false; break; }
+      if (e == 0 && !mbar_wait(smem_u32(&s.o_free), (ut & 1) ^ 1)) { ok = false; break; }
+      if (!mbar_wait(smem_u32(&s.p_full), g & 1)) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t v_addr = smem_u32(s.v[vst]);
+#pragma unroll
+      for (int kk = 0; kk < kBlock / 16; ++kk)
+        mma_ts(tmem + kColO, tmem + kColS + kk * 8, sdesc_sw128(v_addr + kk * 2048, 8192, 1024), idesc_o,
+               (e > 0 || kk > 0) ? 1u : 0u);
+      mma_commit(smem_u32(&s.pv_done));
+      mma_commit(smem_u32(&s.v_empty[vst]));
+      if (e == n - 1) mma_commit(smem_u32(&s.o_full));
     }
     if (!ok) break;
-    if (!issue_pv(nch - 1, 1)) { ok = false; break; }
-    mma_commit(smem_u32(&s.q_free[qs]));
-    mma_commit(smem_u32(&s.o_full));
     mbar_arrive(smem_u32(&s.info_empty[ut & 3]));
-    gc += nch;
   }
   if (!ok) flag_timeout(s, p);
 }
 
 // ---------------------------------------------------------------- softmax + epilogue
-
-__device__ __forceinline__ float fmax_tree16(const float (&x)[16]) {
-  float a = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
-  float b = fmaxf(fmaxf(x[4], x[5]), fmaxf(x[6], x[7]));
-  float c = fmaxf(fmaxf(x[8], x[9]), fmaxf(x[10], x[11]));
-  float d = fmaxf(fmaxf(x[12], x[13]), fmaxf(x[14], x[15]));
-  return fmaxf(fmaxf(a, b), fmaxf(c, d));
-}
 
 // Per-block key validity: all keys valid (no bias), all masked (one uniform
 // bias, folded into the exponent offset and the max), or mixed (per-key bias;
@@ -539,29 +489,28 @@ __device__ __forceinline__ float fmax_tree16(const float (&x)[16]) {
 __device__ __forceinline__ bool block_mixed(uint64_t vm) { return vm != ~0ull && vm != 0ull; }
 __device__ __forceinline__ float block_offset(uint64_t vm, float bias) { return vm == 0ull ? bias : 0.f; }
 
-// Add the per-key bias of a mixed block to 32 raw scores (in place) and
-// return their max plus the block's uniform offset (q.k units).
-__device__ __forceinline__ float piece_prepare(uint32_t (&r)[32], bool mixed, uint32_t vm, float bias, float off) {
+// Add the per-key bias of a mixed block to 16 raw scores (in place; vm16 bit
+// c: key c valid) and return their max (q.k units, without the block offset).
+__device__ __forceinline__ float piece16_prepare(uint32_t (&r)[16], bool mixed, uint32_t vm16, float bias) {
   if (mixed) {
 #pragma unroll
-    for (int c = 0; c < 32; ++c) r[c] = __float_as_uint(__uint_as_float(r[c]) + (((vm >> c) & 1u) ? 0.f : bias));
+    for (int c = 0; c < 16; ++c) r[c] = __float_as_uint(__uint_as_float(r[c]) + (((vm16 >> c) & 1u) ? 0.f : bias));
   }
-  float a = fmaxf(__uint_as_float(r[0]), __uint_as_float(r[1]));
-  float b = fmaxf(__uint_as_float(r[2]), __uint_as_float(r[3]));
-#pragma unroll
-  for (int i = 1; i < 8; ++i) {
-    a = fmax3(a, __uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]));
-    b = fmax3(b, __uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3]));
-  }
-  return fmaxf(a, b) + off;
+  float a = fmax3(__uint_as_float(r[0]), __uint_as_float(r[1]), __uint_as_float(r[2]));
+  float b = fmax3(__uint_as_float(r[3]), __uint_as_float(r[4]), __uint_as_float(r[5]));
+  a = fmax3(a, __uint_as_float(r[6]), __uint_as_float(r[7]));
+  b = fmax3(b, __uint_as_float(r[8]), __uint_as_float(r[9]));
+  a = fmax3(a, __uint_as_float(r[10]), __uint_as_float(r[11]));
+  b = fmax3(b, __uint_as_float(r[12]), __uint_as_float(r[13]));
+  return fmax3(a, b, fmaxf(__uint_as_float(r[14]), __uint_as_float(r[15])));
 }
 
-// p = exp2(r * scale + off) for 32 scores, packed to fp16x2 into pk[0..16);
-// the sum accumulates into two packed pairs (shorter dependency chains).
-__device__ __forceinline__ void piece_exp(const uint32_t (&r)[32], uint64_t scale2, uint64_t off2, uint32_t* pk,
-                                          uint64_t& acc0, uint64_t& acc1) {
+// p = exp2(r * scale + off) for 16 scores, packed to fp16x2 into pk; the sum
+// accumulates into two packed pairs.
+__device__ __forceinline__ void piece16_exp(const uint32_t (&r)[16], uint64_t scale2, uint64_t off2, uint32_t (&pk)[8],
+                                            uint64_t& acc0, uint64_t& acc1) {
 #pragma unroll
-  for (int c = 0; c < 16; ++c) {
+  for (int c = 0; c < 8; ++c) {
     float t0, t1;
     f2_unpack(f2_fma(f2_pack(__uint_as_float(r[2 * c]), __uint_as_float(r[2 * c + 1])), scale2, off2), t0, t1);
     const float e0 = ex2_approx(t0);
@@ -570,45 +519,6 @@ __device__ __forceinline__ void piece_exp(const uint32_t (&r)[32], uint64_t scal
     else acc0 = f2_add(acc0, f2_pack(e0, e1));
     pk[c] = pack_f16x2(e0, e1);
   }
-}
-
-// Per-row online-softmax state of one unit.
-struct RowState {
-  float m_ref;     // reference max (scaled log2 units)
-  float l_run;     // sum of p over the chunks before the current one
-  uint64_t acc0, acc1;  // packed partial sums of the current chunk
-  float o_factor;  // rescale owed to the O accumulator
-};
-
-// One 64-key block of a row (ra: keys 0..31, rb: keys 32..63): one max, at
-// most one change of the reference max, then 64 exponentials packed to fp16
-// into pk. The reference moves only at block boundaries, so P already written
-// never needs rescaling; O and the running sums do (o_factor, l_run, acc).
-__device__ __forceinline__ void process_block(uint32_t (&ra)[32], uint32_t (&rb)[32], uint64_t vm,
-                                              const FwdParams& p, uint32_t (&pk)[32], RowState& st) {
-  const bool mixed = block_mixed(vm);
-  const float off = block_offset(vm, p.bias_raw);
-  const float ma = piece_prepare(ra, mixed, static_cast<uint32_t>(vm), p.bias_raw, off);
-  const float mb = piece_prepare(rb, mixed, static_cast<uint32_t>(vm >> 32), p.bias_raw, off);
-  const float mx = fmaxf(ma, mb) * p.scale_log2;
-  const bool need = mx > st.m_ref + kRescaleThreshold;
-  if (__any_sync(0xffffffffu, need)) {
-    float f = 1.f;
-    if (need) {
-      f = ex2_approx(st.m_ref - mx);
-      st.m_ref = mx;
-    }
-    const uint64_t f2 = f2_pack(f, f);
-    st.l_run *= f;
-    st.acc0 = f2_fma(st.acc0, f2, 0ull);
-    st.acc1 = f2_fma(st.acc1, f2, 0ull);
-    st.o_factor *= f;
-  }
-  const float o = fmaf(off, p.scale_log2, -st.m_ref);
-  const uint64_t scale2 = f2_pack(p.scale_log2, p.scale_log2);
-  const uint64_t off2 = f2_pack(o, o);
-  piece_exp(ra, scale2, off2, pk, st.acc0, st.acc1);
-  piece_exp(rb, scale2, off2, pk + 16, st.acc0, st.acc1);
 }
 
 // O (64 fp32 columns of this thread's row) *= f, in 16-column pieces.
@@ -625,179 +535,161 @@ __device__ __forceinline__ void rescale_o(uint32_t taddr, float f) {
   tmem_wait_st();
 }
 
+// Store 16 columns [c0, c0+16) of one output row: o * inv as bf16 or fp32.
+__device__ __forceinline__ void store16(const FwdParams& p, size_t row, int c0, const uint32_t (&o)[16], float inv) {
+  if (p.out_f32) {
+    float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + row * kHeadDim + c0);
+#pragma unroll
+    for (int c = 0; c < 4; ++c)
+      dst[c] = make_float4(__uint_as_float(o[4 * c]) * inv, __uint_as_float(o[4 * c + 1]) * inv,
+                           __uint_as_float(o[4 * c + 2]) * inv, __uint_as_float(o[4 * c + 3]) * inv);
+  } else {
+    uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) + row * kHeadDim + c0);
+#pragma unroll
+    for (int c = 0; c < 2; ++c)
+      dst[c] = make_uint4(pack_bf16x2(__uint_as_float(o[8 * c]) * inv, __uint_as_float(o[8 * c + 1]) * inv),
+                          pack_bf16x2(__uint_as_float(o[8 * c + 2]) * inv, __uint_as_float(o[8 * c + 3]) * inv),
+                          pack_bf16x2(__uint_as_float(o[8 * c + 4]) * inv, __uint_as_float(o[8 * c + 5]) * inv),
+                          pack_bf16x2(__uint_as_float(o[8 * c + 6]) * inv, __uint_as_float(o[8 * c + 7]) * inv));
+  }
+}
+
+// Warps 0..3, one query row per thread (TMEM lane = row of the unit). Per key
+// block: a max pass over the block's 64 S columns (16 at a time), at most one
+// change of the reference max (lazy: only when it grows by more than 2^8;
+// O is rescaled once the previous P.V has landed), then an exponential pass
+// that writes fp16 P over the S columns it has already read (16 keys = 8
+// columns per piece) and hands the block to the MMA.
 __device__ void softmax_role(SharedStorage& s, const FwdParams& p, uint32_t tmem) {
   const int tid = threadIdx.x;  // 0..127 == TMEM lane
   const int warp = tid >> 5;
   const int lane = tid & 31;
   const int half = warp >> 1;   // 0: rows 0..63, 1: rows 64..127
   const uint32_t lane_addr = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-  uint32_t gc = 0;
+  const uint32_t s_addr = lane_addr + kColS;
+  const uint64_t scale2 = f2_pack(p.scale_log2, p.scale_log2);
+  uint32_t g = 0;
   for (uint32_t ut = 0;; ++ut) {
     if (!warp_wait(smem_u32(&s.info_full[ut & 3]), (ut >> 2) & 1)) { flag_timeout(s, p); return; }
     const UnitInfo& ui = s.unit[ut & 3];
     if (ui.stop) break;
-    if (!warp_wait(smem_u32(&s.q_full[ut & 1]), (ut >> 1) & 1)) { flag_timeout(s, p); return; }
     const int n = ui.n;
-    const int nch = chunk_count(n);
     const int bh = ui.bh;
     const int qblk = half ? ui.qbot : ui.qtop;
     const int split = ui.split;
     const bool exists = qblk >= 0;
-    RowState st;
-    st.m_ref = kNegInit;
-    st.l_run = 0.f;
-
-    for (int c = 0; c < nch; ++c) {
-      const uint32_t g = gc + c;
-      const int e0 = c * kChunk;
-      const int nblk = min(kChunk, n - e0);
+    float m_ref = kNegInit;
+    float l_run = 0.f;
+    for (int e = 0; e < n; ++e, ++g) {
+      const bool used = exists && ((ui.hm[e] >> half) & 1);
       if (!warp_wait(smem_u32(&s.s_full), g & 1)) { flag_timeout(s, p); return; }
       tc_fence_after();
-      const bool used0 = exists && ((ui.hm[e0] >> half) & 1);
-      const bool used1 = nblk == 2 && exists && ((ui.hm[e0 + 1] >> half) & 1);
-      st.acc0 = st.acc1 = 0ull;
-      st.o_factor = 1.f;
-      uint32_t pk[32];
-      uint32_t ra[32], rb[32];
-      // Each used block is read whole (two 32-column loads) and processed in
-      // one pass; S is released once its last used block has been read.
-      auto release_s = [&]() {
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(&s.s_free));
-      };
-      // ---- block 0
-      if (used0) {
-        tmem_ld32(lane_addr + kColS, ra);
-        tmem_ld32(lane_addr + kColS + 32, rb);
+      if (used) {
+        const uint64_t vm = ui.vm[e];
+        const bool mixed = block_mixed(vm);
+        const float off = block_offset(vm, p.bias_raw);
+        uint32_t r0[16], r1[16];
+        // ---- max pass
+        tmem_ld16(s_addr, r0);
+        tmem_ld16(s_addr + 16, r1);
         tmem_wait_ld();
-        if (!used1) release_s();
-        process_block(ra, rb, ui.vm[e0], p, pk, st);
-      } else {
-        if (!used1) release_s();
-#pragma unroll
-        for (int i = 0; i < 32; ++i) pk[i] = 0u;
-      }
-      // P columns of block 0 are free once the previous chunk's PV-lo is done.
-      if (g >= 1 && !warp_wait(smem_u32(&s.pv_lo), (g - 1) & 1)) { flag_timeout(s, p); return; }
-      tc_fence_after();
-      if (__any_sync(0xffffffffu, st.o_factor != 1.f)) {
-        // The max grew: O (all of the previous chunk's P.V) scales by o_factor.
-        if (c > 0) {
-          if (!warp_wait(smem_u32(&s.pv_hi), (g - 1) & 1)) { flag_timeout(s, p); return; }
-          tc_fence_after();
-          rescale_o(lane_addr + kColO, st.o_factor);
+        float mx = fmaxf(piece16_prepare(r0, mixed, static_cast<uint32_t>(vm) & 0xFFFFu, p.bias_raw),
+                         piece16_prepare(r1, mixed, static_cast<uint32_t>(vm >> 16) & 0xFFFFu, p.bias_raw));
+        tmem_ld16(s_addr + 32, r0);
+        tmem_ld16(s_addr + 48, r1);
+        tmem_wait_ld();
+        mx = fmax3(mx, piece16_prepare(r0, mixed, static_cast<uint32_t>(vm >> 32) & 0xFFFFu, p.bias_raw),
+                   piece16_prepare(r1, mixed, static_cast<uint32_t>(vm >> 48) & 0xFFFFu, p.bias_raw));
+        mx = (mx + off) * p.scale_log2;
+        const bool need = mx > m_ref + kRescaleThreshold;
+        if (__any_sync(0xffffffffu, need)) {
+          float f = 1.f;
+          if (need) {
+            f = ex2_approx(m_ref - mx);
+            m_ref = mx;
+          }
+          l_run *= f;
+          // O holds the P.V of the earlier blocks (none yet for e == 0: the
+          // first P.V of the unit overwrites O).
+          if (e > 0 && __any_sync(0xffffffffu, f != 1.f)) {
+            if (!warp_wait(smem_u32(&s.pv_done), (g - 1) & 1)) { flag_timeout(s, p); return; }
+            tc_fence_after();
+            rescale_o(lane_addr + kColO, f);
+          }
         }
-        st.o_factor = 1.f;
+        // ---- exponential pass; P piece q goes to columns 8q..8q+7, inside S
+        // columns already read (piece q-1's or this piece's own).
+        const float o = fmaf(off, p.scale_log2, -m_ref);
+        const uint64_t off2 = f2_pack(o, o);
+        uint64_t acc0 = 0ull, acc1 = 0ull;
+        tmem_ld16(s_addr, r0);
+        tmem_wait_ld();
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          uint32_t (&cur)[16] = (q & 1) ? r1 : r0;
+          uint32_t (&nxt)[16] = (q & 1) ? r0 : r1;
+          if (q < 3) tmem_ld16(s_addr + 16 * (q + 1), nxt);
+          piece16_prepare(cur, mixed, static_cast<uint32_t>(vm >> (16 * q)) & 0xFFFFu, p.bias_raw);
+          uint32_t pk[8];
+          piece16_exp(cur, scale2, off2, pk, acc0, acc1);
+          if (q < 3) tmem_wait_ld();
+          tmem_st8(s_addr + 8 * q, pk);
+        }
+        float a0, a1, b0, b1;
+        f2_unpack(acc0, a0, a1);
+        f2_unpack(acc1, b0, b1);
+        l_run += (a0 + a1) + (b0 + b1);
+      } else {
+        // No row of this warp uses the block: P = 0.
+        uint32_t z[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) z[i] = 0u;
+        tmem_st16(s_addr, z);
+        tmem_st16(s_addr + 16, z);
       }
-      tmem_st32(lane_addr + kColP, pk);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&s.p_lo));
-      // ---- block 1
-      if (nblk == 2) {
-        if (used1) {
-          tmem_ld32(lane_addr + kColS + kBlock, ra);
-          tmem_ld32(lane_addr + kColS + kBlock + 32, rb);
-          tmem_wait_ld();
-          release_s();
-          process_block(ra, rb, ui.vm[e0 + 1], p, pk, st);
-        } else {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) pk[i] = 0u;
-        }
-        if (g >= 1 && !warp_wait(smem_u32(&s.pv_hi), (g - 1) & 1)) { flag_timeout(s, p); return; }
-        tc_fence_after();
-        if (__any_sync(0xffffffffu, st.o_factor != 1.f)) {
-          // The max grew after block 0's P went out: once this chunk's PV-lo has
-          // landed, O (earlier chunks and block 0) scales by o_factor.
-          if (!warp_wait(smem_u32(&s.pv_lo), g & 1)) { flag_timeout(s, p); return; }
-          tc_fence_after();
-          rescale_o(lane_addr + kColO, st.o_factor);
-          st.o_factor = 1.f;
-        }
-        tmem_st32(lane_addr + kColP + 32, pk);
-        tmem_wait_st();
-      } else if (g >= 1) {
-        // One-block chunk: nothing to write, but p_hi must not run two phases
-        // ahead of the MMA thread's wait on it.
-        if (!warp_wait(smem_u32(&s.pv_hi), (g - 1) & 1)) { flag_timeout(s, p); return; }
-      }
-      {
-        float a0, a1, b0, b1;
-        f2_unpack(st.acc0, a0, a1);
-        f2_unpack(st.acc1, b0, b1);
-        st.l_run += (a0 + a1) + (b0 + b1);
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&s.p_hi));
+      if (lane == 0) mbar_arrive(smem_u32(&s.p_full));
     }
-    const float m_ref = st.m_ref;
-    const float l_run = st.l_run;
     __syncwarp();
     if (lane == 0) mbar_arrive(smem_u32(&s.info_empty[ut & 3]));
 
-    // ---- epilogue
+    // ---- epilogue: O in 16-column pieces, freed after the last piece
     if (!warp_wait(smem_u32(&s.o_full), ut & 1)) { flag_timeout(s, p); return; }
     tc_fence_after();
-    uint32_t o0[32], o1[32];
-    tmem_ld32(lane_addr + kColO, o0);
-    tmem_ld32(lane_addr + kColO + 32, o1);
-    tmem_wait_ld();
+    if (split >= 0) {
+      const size_t base = (static_cast<size_t>(bh) * p.nsplit + split) * kRows + tid;
+#pragma unroll 1
+      for (int c0 = 0; c0 < kHeadDim; c0 += 16) {
+        uint32_t o[16];
+        tmem_ld16(lane_addr + kColO + c0, o);
+        tmem_wait_ld();
+        float4* dst = reinterpret_cast<float4*>(p.part_o + base * kHeadDim + c0);
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          dst[c] = make_float4(__uint_as_float(o[4 * c]), __uint_as_float(o[4 * c + 1]), __uint_as_float(o[4 * c + 2]),
+                               __uint_as_float(o[4 * c + 3]));
+      }
+      reinterpret_cast<float2*>(p.part_ml)[base] = make_float2(m_ref, l_run);
+    } else if (exists) {
+      const float inv = 1.f / l_run;
+      const size_t row = static_cast<size_t>(bh) * p.L + static_cast<size_t>(qblk) * kBlock + (tid & 63);
+#pragma unroll 1
+      for (int c0 = 0; c0 < kHeadDim; c0 += 16) {
+        uint32_t o[16];
+        tmem_ld16(lane_addr + kColO + c0, o);
+        tmem_wait_ld();
+        store16(p, row, c0, o, inv);
+      }
+    }
     tc_fence_before();
     __syncwarp();
     if (lane == 0) mbar_arrive(smem_u32(&s.o_free));
-    if (exists) {
-      const int row_in_blk = tid & 63;
-      if (split >= 0) {
-        const size_t base = (static_cast<size_t>(bh) * p.nsplit + split) * kRows + tid;
-        float4* dst = reinterpret_cast<float4*>(p.part_o + base * kHeadDim);
-#pragma unroll
-        for (int c = 0; c < 8; ++c)
-          dst[c] = make_float4(__uint_as_float(o0[4 * c]), __uint_as_float(o0[4 * c + 1]),
-                               __uint_as_float(o0[4 * c + 2]), __uint_as_float(o0[4 * c + 3]));
-#pragma unroll
-        for (int c = 0; c < 8; ++c)
-          dst[8 + c] = make_float4(__uint_as_float(o1[4 * c]), __uint_as_float(o1[4 * c + 1]),
-                                   __uint_as_float(o1[4 * c + 2]), __uint_as_float(o1[4 * c + 3]));
-        reinterpret_cast<float2*>(p.part_ml)[base] = make_float2(m_ref, l_run);
-      } else {
-        const float inv = 1.f / l_run;
-        const size_t row = static_cast<size_t>(bh) * p.L + static_cast<size_t>(qblk) * kBlock + row_in_blk;
-        if (p.out_f32) {
-          float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + row * kHeadDim);
-#pragma unroll
-          for (int c = 0; c < 8; ++c)
-            dst[c] = make_float4(__uint_as_float(o0[4 * c]) * inv, __uint_as_float(o0[4 * c + 1]) * inv,
-                                 __uint_as_float(o0[4 * c + 2]) * inv, __uint_as_float(o0[4 * c + 3]) * inv);
-#pragma unroll
-          for (int c = 0; c < 8; ++c)
-            dst[8 + c] = make_float4(__uint_as_float(o1[4 * c]) * inv, __uint_as_float(o1[4 * c + 1]) * inv,
-                                     __uint_as_float(o1[4 * c + 2]) * inv, __uint_as_float(o1[4 * c + 3]) * inv);
-        } else {
-          uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) + row * kHeadDim);
-#pragma unroll
-          for (int c = 0; c < 4; ++c)
-            dst[c] = make_uint4(pack_bf16x2(__uint_as_float(o0[8 * c]) * inv, __uint_as_float(o0[8 * c + 1]) * inv),
-                                pack_bf16x2(__uint_as_float(o0[8 * c + 2]) * inv, __uint_as_float(o0[8 * c + 3]) * inv),
-                                pack_bf16x2(__uint_as_float(o0[8 * c + 4]) * inv, __uint_as_float(o0[8 * c + 5]) * inv),
-                                pack_bf16x2(__uint_as_float(o0[8 * c + 6]) * inv, __uint_as_float(o0[8 * c + 7]) * inv));
-#pragma unroll
-          for (int c = 0; c < 4; ++c)
-            dst[4 + c] = make_uint4(pack_bf16x2(__uint_as_float(o1[8 * c]) * inv, __uint_as_float(o1[8 * c + 1]) * inv),
-                                    pack_bf16x2(__uint_as_float(o1[8 * c + 2]) * inv, __uint_as_float(o1[8 * c + 3]) * inv),
-                                    pack_bf16x2(__uint_as_float(o1[8 * c + 4]) * inv, __uint_as_float(o1[8 * c + 5]) * inv),
-                                    pack_bf16x2(__uint_as_float(o1[8 * c + 6]) * inv, __uint_as_float(o1[8 * c + 7]) * inv));
-        }
-      }
-    }
-    gc += nch;
   }
 }
 
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(kThreads, kCtasPerSm)
 bigbird_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -813,10 +705,8 @@ bigbird_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       mbar_init(smem_u32(&s.info_full[i]), 1);
       mbar_init(smem_u32(&s.info_empty[i]), 1 + 1 + 4 + 1);  // TMA, MMA, 4 softmax warps, converter
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(smem_u32(&s.q_full[i]), 1);
-      mbar_init(smem_u32(&s.q_free[i]), 1);
-    }
+    mbar_init(smem_u32(&s.q_full), 1);
+    mbar_init(smem_u32(&s.q_free), 1);
     for (int i = 0; i < kKStages; ++i) {
       mbar_init(smem_u32(&s.k_full[i]), 1);
       mbar_init(smem_u32(&s.k_empty[i]), 1);
@@ -827,11 +717,8 @@ bigbird_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       mbar_init(smem_u32(&s.v_empty[i]), 1);
     }
     mbar_init(smem_u32(&s.s_full), 1);
-    mbar_init(smem_u32(&s.s_free), 4);
-    mbar_init(smem_u32(&s.p_lo), 4);
-    mbar_init(smem_u32(&s.p_hi), 4);
-    mbar_init(smem_u32(&s.pv_lo), 1);
-    mbar_init(smem_u32(&s.pv_hi), 1);
+    mbar_init(smem_u32(&s.p_full), 4);
+    mbar_init(smem_u32(&s.pv_done), 1);
     mbar_init(smem_u32(&s.o_full), 1);
     mbar_init(smem_u32(&s.o_free), 4);
     s.abort_flag = 0;
@@ -962,7 +849,7 @@ static DeviceInfo* device_info(int dev) {
       const int smem = static_cast<int>(sizeof(SharedStorage) + 1024);
       if (cudaFuncSetAttribute(bigbird_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
         return nullptr;
-      // Two CTAs per SM need the largest shared-memory carve-out.
+      // Four CTAs per SM need the largest shared-memory carve-out.
       if (cudaFuncSetAttribute(bigbird_fwd_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100) != cudaSuccess)
         return nullptr;
       if (cudaGetSymbolAddress(reinterpret_cast<void**>(&di.status), g_status) != cudaSuccess) return nullptr;
@@ -1099,7 +986,7 @@ int bigbird_attn_fwd_ex(const void* q, const void* k, const void* v, const int32
     return BB_ERR_CUDA;
   }
 
-  const int grid = std::min(p.total_units, 2 * di->sms);
+  const int grid = std::min(p.total_units, kCtasPerSm * di->sms);
   const size_t smem = sizeof(SharedStorage) + 1024;
   bigbird_fwd_kernel<<<grid, kThreads, smem, stream>>>(tq, tk, tv, p);
   cudaError_t e = cudaGetLastError();
