@@ -42,7 +42,7 @@
 //
 // Softmax: a max pass and an exponential pass over each block's 64 columns;
 // the reference max moves only at block boundaries and only when it grows by
-// more than 2^8 (the O rescale is skipped otherwise; the final O / l is exact
+// more than 2^14 (the O rescale is skipped otherwise; the final O / l is exact
 // either way). Padded
 // keys get -10000 added to the scaled score. P.V runs in fp16: P is written as
 // fp16 and each V tile is converted bf16 -> fp16 in shared memory (exact in the
@@ -76,7 +76,10 @@ constexpr uint32_t kTileBytes = kBlock * kHeadDim * 2;  // one 64x64 bf16 tile
 constexpr uint32_t kTmemCols = 128;
 constexpr uint32_t kColS = 0;          // S of one key block: 64 fp32 columns; P (fp16) overwrites the first 32
 constexpr uint32_t kColO = 64;         // O: 64 fp32 columns
-constexpr float kRescaleThreshold = 8.0f;  // log2 units
+// The reference max moves only when a score exceeds it by more than 2^14: P
+// (fp16, largest finite 65504) then stays <= 2^14 with headroom, and the
+// repairs of already-written P and O stay rare even for wide score ranges.
+constexpr float kRescaleThreshold = 14.0f;  // log2 units
 constexpr float kNegInit = -1.0e30f;
 
 // status word bits
@@ -521,6 +524,24 @@ __device__ __forceinline__ void piece16_exp(const uint32_t (&r)[16], uint64_t sc
   }
 }
 
+// Rare path: the reference max grew inside a block after `npieces` 16-key
+// pieces of P were already written (fp16, 8 columns each): scale them by f.
+__device__ __noinline__ void rescale_p(uint32_t s_addr, int npieces, float f) {
+  tmem_wait_st();
+  for (int i = 0; i < npieces; ++i) {
+    uint32_t t[8];
+    tmem_ld8(s_addr + 8 * i, t);
+    tmem_wait_ld();
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const float2 v = __half22float2(*reinterpret_cast<const __half2*>(&t[j]));
+      t[j] = pack_f16x2(v.x * f, v.y * f);
+    }
+    tmem_st8(s_addr + 8 * i, t);
+  }
+  tmem_wait_st();
+}
+
 // O (64 fp32 columns of this thread's row) *= f, in 16-column pieces.
 __device__ __forceinline__ void rescale_o(uint32_t taddr, float f) {
 #pragma unroll 1
@@ -555,11 +576,11 @@ __device__ __forceinline__ void store16(const FwdParams& p, size_t row, int c0, 
 }
 
 // Warps 0..3, one query row per thread (TMEM lane = row of the unit). Per key
-// block: a max pass over the block's 64 S columns (16 at a time), at most one
-// change of the reference max (lazy: only when it grows by more than 2^8;
-// O is rescaled once the previous P.V has landed), then an exponential pass
-// that writes fp16 P over the S columns it has already read (16 keys = 8
-// columns per piece) and hands the block to the MMA.
+// block: one pass over its 64 S columns, 16 at a time -- max, a change of the
+// reference max when a score exceeds it by more than 2^14 (rare; the P pieces
+// already written and, after the previous P.V has landed, O are rescaled),
+// exponentials, fp16 P written over the S columns already read (16 keys = 8
+// columns per piece) -- then the block goes to the MMA.
 __device__ void softmax_role(SharedStorage& s, const FwdParams& p, uint32_t tmem) {
   const int tid = threadIdx.x;  // 0..127 == TMEM lane
   const int warp = tid >> 5;
@@ -588,40 +609,14 @@ __device__ void softmax_role(SharedStorage& s, const FwdParams& p, uint32_t tmem
         const uint64_t vm = ui.vm[e];
         const bool mixed = block_mixed(vm);
         const float off = block_offset(vm, p.bias_raw);
-        uint32_t r0[16], r1[16];
-        // ---- max pass
-        tmem_ld16(s_addr, r0);
-        tmem_ld16(s_addr + 16, r1);
-        tmem_wait_ld();
-        float mx = fmaxf(piece16_prepare(r0, mixed, static_cast<uint32_t>(vm) & 0xFFFFu, p.bias_raw),
-                         piece16_prepare(r1, mixed, static_cast<uint32_t>(vm >> 16) & 0xFFFFu, p.bias_raw));
-        tmem_ld16(s_addr + 32, r0);
-        tmem_ld16(s_addr + 48, r1);
-        tmem_wait_ld();
-        mx = fmax3(mx, piece16_prepare(r0, mixed, static_cast<uint32_t>(vm >> 32) & 0xFFFFu, p.bias_raw),
-                   piece16_prepare(r1, mixed, static_cast<uint32_t>(vm >> 48) & 0xFFFFu, p.bias_raw));
-        mx = (mx + off) * p.scale_log2;
-        const bool need = mx > m_ref + kRescaleThreshold;
-        if (__any_sync(0xffffffffu, need)) {
-          float f = 1.f;
-          if (need) {
-            f = ex2_approx(m_ref - mx);
-            m_ref = mx;
-          }
-          l_run *= f;
-          // O holds the P.V of the earlier blocks (none yet for e == 0: the
-          // first P.V of the unit overwrites O).
-          if (e > 0 && __any_sync(0xffffffffu, f != 1.f)) {
-            if (!warp_wait(smem_u32(&s.pv_done), (g - 1) & 1)) { flag_timeout(s, p); return; }
-            tc_fence_after();
-            rescale_o(lane_addr + kColO, f);
-          }
-        }
-        // ---- exponential pass; P piece q goes to columns 8q..8q+7, inside S
-        // columns already read (piece q-1's or this piece's own).
-        const float o = fmaf(off, p.scale_log2, -m_ref);
-        const uint64_t off2 = f2_pack(o, o);
+        const float off_s = off * p.scale_log2;
+        float o_factor = 1.f;  // rescale owed to O (the P.V of the earlier blocks)
         uint64_t acc0 = 0ull, acc1 = 0ull;
+        uint32_t r0[16], r1[16];
+        // One pass over the block's 64 columns, 16 at a time with the next
+        // piece's TMEM read in flight: max, a change of the reference max when
+        // it grows by more than 2^14, exponentials, and fp16 P written over S
+        // columns already read (piece q -> columns 8q..8q+7).
         tmem_ld16(s_addr, r0);
         tmem_wait_ld();
 #pragma unroll
@@ -629,9 +624,26 @@ __device__ void softmax_role(SharedStorage& s, const FwdParams& p, uint32_t tmem
           uint32_t (&cur)[16] = (q & 1) ? r1 : r0;
           uint32_t (&nxt)[16] = (q & 1) ? r0 : r1;
           if (q < 3) tmem_ld16(s_addr + 16 * (q + 1), nxt);
-          piece16_prepare(cur, mixed, static_cast<uint32_t>(vm >> (16 * q)) & 0xFFFFu, p.bias_raw);
+          const float mx = fmaf(piece16_prepare(cur, mixed, static_cast<uint32_t>(vm >> (16 * q)) & 0xFFFFu,
+                                                p.bias_raw),
+                                p.scale_log2, off_s);
+          const bool need = mx > m_ref + kRescaleThreshold;
+          if (__any_sync(0xffffffffu, need)) {
+            float f = 1.f;
+            if (need) {
+              f = ex2_approx(m_ref - mx);
+              m_ref = mx;
+            }
+            l_run *= f;
+            const uint64_t f2 = f2_pack(f, f);
+            acc0 = f2_fma(acc0, f2, 0ull);
+            acc1 = f2_fma(acc1, f2, 0ull);
+            o_factor *= f;
+            if (q > 0 && __any_sync(0xffffffffu, f != 1.f)) rescale_p(s_addr, q, f);
+          }
+          const float o = off_s - m_ref;
           uint32_t pk[8];
-          piece16_exp(cur, scale2, off2, pk, acc0, acc1);
+          piece16_exp(cur, scale2, f2_pack(o, o), pk, acc0, acc1);
           if (q < 3) tmem_wait_ld();
           tmem_st8(s_addr + 8 * q, pk);
         }
@@ -639,6 +651,13 @@ __device__ void softmax_role(SharedStorage& s, const FwdParams& p, uint32_t tmem
         f2_unpack(acc0, a0, a1);
         f2_unpack(acc1, b0, b1);
         l_run += (a0 + a1) + (b0 + b1);
+        // O holds the P.V of the earlier blocks (none yet for e == 0: the
+        // first P.V of the unit overwrites O); rescale it once that P.V is done.
+        if (e > 0 && __any_sync(0xffffffffu, o_factor != 1.f)) {
+          if (!warp_wait(smem_u32(&s.pv_done), (g - 1) & 1)) { flag_timeout(s, p); return; }
+          tc_fence_after();
+          rescale_o(lane_addr + kColO, o_factor);
+        }
       } else {
         // No row of this warp uses the block: P = 0.
         uint32_t z[16];

@@ -200,6 +200,25 @@ def test_set_semantics_and_all_padded():
     _check(got, want, "edge")
 
 
+def test_max_growth_inside_and_across_blocks():
+    """Scores that rise by about 16 (log2 units) from each 16-key piece of a
+    block to the next and by about 17 from block to block: the lazy rescale
+    (threshold 14) fires inside every block, after P of earlier pieces is
+    written, and between blocks, after earlier P.V is in O; both repairs must
+    give the oracle's softmax."""
+    B, H, L = 1, 2, 12 * 64
+    j = torch.arange(L, dtype=torch.float32)
+    a = 0.35 * (j % 64) + 6.0 * (j // 64)     # score = q.k / 8 = 2a
+    q = torch.full((B, H, L, 64), 0.25).to(torch.bfloat16)
+    k = (a[:, None] * torch.ones(64)).expand(B, H, L, 64).contiguous().to(torch.bfloat16)
+    v = torch.randn(B, H, L, 64, generator=torch.Generator().manual_seed(3)).to(torch.bfloat16)
+    w = Workload("growth", B, H, L, seed=0)
+    ra, ra_o = _rand_attn_pair(w, seed=31)
+    got = _cuda_fwd({"q": q, "k": k, "v": v, "seq_mask": None}, w, ra, torch.float32)
+    want = oracle.attention(q, k, v, ra_o, None, w.block, w.r)
+    _check(got, want, "growth")
+
+
 def test_out_of_range_rand_attn_is_flagged():
     w = Workload("oor", 1, 1, 16 * 64, seed=18)
     inp = make_inputs(w)
