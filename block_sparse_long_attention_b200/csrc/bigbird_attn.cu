@@ -743,6 +743,8 @@ bigbird_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     s.abort_flag = 0;
     fence_barrier_init();
   }
+  // Dependent grids (the merge) may launch now; they wait for this grid's completion.
+  asm volatile("griddepcontrol.launch_dependents;");
   if (warp == 4 && lane == 0) {
     tma_prefetch_desc(&tmQ);
     tma_prefetch_desc(&tmK);
@@ -781,6 +783,9 @@ constexpr int kMergeRowsPerCta = 16;
 __global__ void __launch_bounds__(256)
 bigbird_merge_kernel(const float* __restrict__ part_o, const float* __restrict__ part_ml, void* out, int nsplit,
                      int L, int nb, int out_f32) {
+  // Launched as a programmatic dependent of the attention kernel: wait until
+  // that grid has completed and its partials are visible.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int bh = blockIdx.x;
   const int row = blockIdx.y * kMergeRowsPerCta + (threadIdx.x >> 4);
   const int c4 = threadIdx.x & 15;
@@ -1010,9 +1015,21 @@ int bigbird_attn_fwd_ex(const void* q, const void* k, const void* v, const int32
   bigbird_fwd_kernel<<<grid, kThreads, smem, stream>>>(tq, tk, tv, p);
   cudaError_t e = cudaGetLastError();
   if (e == cudaSuccess && pl.nsplit > 1) {
-    bigbird_merge_kernel<<<dim3(p.BH, kRows / kMergeRowsPerCta), 256, 0, stream>>>(p.part_o, p.part_ml, out, pl.nsplit,
-                                                                               L, pl.nb, p.out_f32);
-    e = cudaGetLastError();
+    // Programmatic dependent launch: the merge grid is launched while the
+    // attention kernel runs and waits (griddepcontrol.wait) for its completion,
+    // which hides the launch gap between the two.
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(p.BH, kRows / kMergeRowsPerCta);
+    cfg.blockDim = dim3(256);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, bigbird_merge_kernel, static_cast<const float*>(p.part_o),
+                           static_cast<const float*>(p.part_ml), out, pl.nsplit, L, pl.nb, p.out_f32);
   }
   if (owned) cudaFreeAsync(ws, stream);
   return e == cudaSuccess ? BB_OK : BB_ERR_CUDA;
