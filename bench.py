@@ -275,9 +275,13 @@ def run_cuda(args):
     peaks, src = _peaks()
     peak = float(peaks["bf16_tflops"])
     achieved = flops / (ms * 1e-3) / 1e12
+    # DRAM bytes (read + write) of one bigbird_fwd_kernel launch on the default
+    # workload, from the ncu capture summarised in
+    # profiles/bigbird_fwd_l4096_b4h12.md; valid for that kernel source only.
+    traffic = 86.20e6 if (w.name == DEFAULT_WORKLOAD and world == 1) else None
     roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-            "frac": achieved / peak, "traffic": None,
-            "kernel": "bigbird_fwd_kernel + bigbird_merge_kernel (one fwd call)",
+            "frac": achieved / peak, "traffic": traffic,
+            "kernel": "bigbird_fwd_kernel + bigbird_merge_kernel (one fwd call; traffic: fwd kernel, ncu)",
             "peak_source": f"{src} bf16 dense burst (kernel timed alone)"}
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
