@@ -340,3 +340,49 @@ def test_bf16_inputs_used_exactly():
 def test_sparse_flops():
     assert oracle.sparse_flops(4, 12, 4096, 64, 64, 3) == 4.0 * 4 * 12 * 4096 * 622 * 64
     assert math.isclose(oracle.sparse_flops(4, 12, 4096, 64, 64, 3) / 1e9, 31.31, rel_tol=1e-3)
+
+
+# --------------------------------------------------------------------------
+# The C sparse brute-force reference (the timed CPU baseline) against the
+# dense-mask oracle: both are fp64 statements of the same definition, one by
+# per-row key gathering in C, the other by an [L, L] mask in NumPy.
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("case", ["sparse_padded", "fallback", "forced_sparse", "set_semantics", "all_padded"])
+def test_c_sparse_reference_matches_oracle(case):
+    from oracle import sparse_ref
+    from block_sparse_long_attention_b200.workloads import Workload
+
+    force = False
+    if case == "sparse_padded":
+        w = Workload("c", 2, 3, 21 * 64, pad=("fixed", [1300, 900]), seed=41)
+    elif case == "fallback":
+        w = Workload("c", 1, 2, 704, pad=("fixed", [500]), seed=42)
+    elif case == "forced_sparse":
+        w = Workload("c", 1, 2, 9 * 64, seed=43)
+        force = True
+    elif case == "set_semantics":
+        w = Workload("c", 1, 2, 16 * 64, seed=44)
+    else:
+        w = Workload("c", 1, 1, 12 * 64, pad=("fixed", [0]), seed=45)
+    inp = make_inputs(w)
+    nb = w.L // w.block
+    sparse = force or nb > 5 + 2 * w.r
+    ra = oracle.rand_attn_generate(w.H, w.L, w.block, w.r, seed=7) if sparse else None
+    if case == "set_semantics":
+        ra[0] = 0                   # all-zero adjacency (global block repeated)
+        ra[1, 4, :] = 5             # window overlap, repeated
+    want = oracle.attention(inp["q"], inp["k"], inp["v"], ra, inp["seq_mask"], w.block, w.r, force_sparse=force)
+    got = sparse_ref.sparse_attention(inp["q"], inp["k"], inp["v"], ra, inp["seq_mask"], w.block, w.r,
+                                      force_sparse=force, threads=2)
+    assert np.abs(got - want).max() < 1e-12
+
+
+def test_c_sparse_reference_rejects_bad_input():
+    from oracle import sparse_ref
+
+    q = torch.zeros(1, 1, 12 * 64, 64, dtype=torch.bfloat16)
+    ra = np.zeros((1, 10, 3), dtype=np.int32)
+    ra[0, 2, 1] = 99
+    with pytest.raises(ValueError):
+        sparse_ref.sparse_attention(q, q, q, ra, None, 64, 3)
