@@ -17,7 +17,10 @@ Page abbreviations used in the citations of this package:
 from .bigbird_oracle import (  # noqa: F401
     BIAS_MASKED,
     attention,
+    attention_backward,
+    attention_lse,
     attention_rows,
+    backward_flops,
     block_mask,
     brute_force_rows,
     check_shape,

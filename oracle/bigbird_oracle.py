@@ -368,6 +368,73 @@ def pattern_table(rand_attn: np.ndarray, H: int, L: int, block: int, r: int) -> 
 
 
 # --------------------------------------------------------------------------
+# Backward pass (gradients of the same definition)
+# --------------------------------------------------------------------------
+
+def attention_lse(q, k, rand_attn, seq_mask, block: int, r: int, force_sparse: bool = False) -> np.ndarray:
+    """Natural-log log-sum-exp of each row's scores, lse[B, H, L] in fp64:
+    log sum_k exp(s[q, k]) over the row's attended keys (the softmax
+    normaliser the backward pass recomputes P from)."""
+    q, k = _as_f64(q), _as_f64(k)
+    B, H, L, d = q.shape
+    nb, sparse = _mode(L, block, r, force_sparse)
+    tok_blk = np.arange(L) // block
+    out = np.empty((B, H, L), dtype=np.float64)
+    for b in range(B):
+        bias = _key_bias(seq_mask, b, L)
+        for h in range(H):
+            bm = block_mask(nb, r, None if rand_attn is None else np.asarray(rand_attn)[h], sparse)
+            allowed = bm[tok_blk][:, tok_blk]
+            s = (q[b, h] @ k[b, h].T) / math.sqrt(d) + bias[None, :]
+            s = np.where(allowed, s, -np.inf)
+            m = s.max(axis=1)
+            out[b, h] = m + np.log(np.exp(s - m[:, None]).sum(axis=1))
+    return out
+
+
+def attention_backward(q, k, v, rand_attn, seq_mask, block: int, r: int, dout,
+                       force_sparse: bool = False):
+    """Gradients (dq, dk, dv), each [B, H, L, d] fp64, of the scalar
+    sum(dout * attention(q, k, v, ...)).
+
+    Plain chain rule through the masked softmax of each row: with
+    p = softmax(s), s = q k^T / sqrt(d) + bias (bias is a constant),
+    dv = p^T dout, dp = dout v^T, ds = p * (dp - rowsum(dp * p)),
+    dq = ds k / sqrt(d), dk = ds^T q / sqrt(d). Keys outside a row's pattern
+    have p = 0 and receive nothing from it.
+    """
+    q, k, v, do = _as_f64(q), _as_f64(k), _as_f64(v), _as_f64(dout)
+    B, H, L, d = q.shape
+    nb, sparse = _mode(L, block, r, force_sparse)
+    tok_blk = np.arange(L) // block
+    dq = np.zeros_like(q)
+    dk = np.zeros_like(k)
+    dv = np.zeros_like(v)
+    c = 1.0 / math.sqrt(d)
+    for b in range(B):
+        bias = _key_bias(seq_mask, b, L)
+        for h in range(H):
+            bm = block_mask(nb, r, None if rand_attn is None else np.asarray(rand_attn)[h], sparse)
+            allowed = bm[tok_blk][:, tok_blk]
+            s = (q[b, h] @ k[b, h].T) * c + bias[None, :]
+            s = np.where(allowed, s, -np.inf)
+            p = np.exp(s - s.max(axis=1, keepdims=True))
+            p /= p.sum(axis=1, keepdims=True)
+            dv[b, h] = p.T @ do[b, h]
+            dp = do[b, h] @ v[b, h].T
+            ds = p * (dp - (dp * p).sum(axis=1, keepdims=True))
+            dq[b, h] = ds @ k[b, h] * c
+            dk[b, h] = ds.T @ q[b, h] * c
+    return dq, dk, dv
+
+
+def backward_flops(B: int, H: int, L: int, d: int, block: int, r: int) -> float:
+    """Algorithmic FLOPs of one backward: 10 * B * H * L * keys_per_row * d
+    (2 each for recomputing q k^T, dout v^T, p^T dout, ds k and ds^T q)."""
+    return 10.0 * B * H * L * keys_per_row(L, block, r) * d
+
+
+# --------------------------------------------------------------------------
 # Work accounting (the metric's FLOP count)
 # --------------------------------------------------------------------------
 

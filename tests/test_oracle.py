@@ -386,3 +386,69 @@ def test_c_sparse_reference_rejects_bad_input():
     ra[0, 2, 1] = 99
     with pytest.raises(ValueError):
         sparse_ref.sparse_attention(q, q, q, ra, None, 64, 3)
+
+
+# --------------------------------------------------------------------------
+# Backward pass of the oracle: pinned by finite differences of the forward
+# (an independent route to the same derivatives) and by exact identities.
+# --------------------------------------------------------------------------
+
+def _fd_case(L, pad, seed):
+    rng = np.random.default_rng(seed)
+    B, H, d = 1, 2, 64
+    q = rng.standard_normal((B, H, L, d)) * 0.5
+    k = rng.standard_normal((B, H, L, d)) * 0.5
+    v = rng.standard_normal((B, H, L, d))
+    do = rng.standard_normal((B, H, L, d))
+    sm = None if pad is None else mask_from_lengths(B, L, [pad]).numpy()
+    ra = None if oracle.is_fallback(L, 64, 3) else oracle.rand_attn_generate(H, L, 64, 3, seed=seed)
+    return q, k, v, do, sm, ra
+
+
+@pytest.mark.parametrize("L,pad", [(12 * 64, 700), (704, None)], ids=["sparse_padded", "fallback"])
+def test_backward_matches_finite_differences(L, pad):
+    q, k, v, do, sm, ra = _fd_case(L, pad, seed=5)
+    dq, dk, dv = oracle.attention_backward(q, k, v, ra, sm, 64, 3, do)
+
+    def loss(qq, kk, vv):
+        return float((oracle.attention(qq, kk, vv, ra, sm, 64, 3) * do).sum())
+
+    rng = np.random.default_rng(11)
+    eps = 1e-5
+    for name, g in (("q", dq), ("k", dk), ("v", dv)):
+        for _ in range(8):
+            idx = (0, int(rng.integers(2)), int(rng.integers(L)), int(rng.integers(64)))
+            plus = {"q": q.copy(), "k": k.copy(), "v": v.copy()}
+            minus = {"q": q.copy(), "k": k.copy(), "v": v.copy()}
+            plus[name][idx] += eps
+            minus[name][idx] -= eps
+            fd = (loss(plus["q"], plus["k"], plus["v"]) - loss(minus["q"], minus["k"], minus["v"])) / (2 * eps)
+            assert abs(fd - g[idx]) <= 1e-6 * (1 + abs(fd)), (name, idx, fd, g[idx])
+
+
+def test_backward_identities():
+    """Exact for any input: the rows of ds sum to zero, so sum_k dk = 0; the
+    rows of p sum to one, so sum_k dv = sum_q dout. A padded key (-10000)
+    receives nothing."""
+    q, k, v, do, sm, ra = _fd_case(16 * 64, 900, seed=8)
+    dq, dk, dv = oracle.attention_backward(q, k, v, ra, sm, 64, 3, do)
+    assert np.abs(dk.sum(axis=2)).max() < 1e-10
+    assert np.abs(dv.sum(axis=2) - do.sum(axis=2)).max() < 1e-10
+    assert np.abs(dk[:, :, 900:]).max() == 0.0 and np.abs(dv[:, :, 900:]).max() == 0.0
+    # identical keys: every score of a row is equal, so q gets no gradient
+    kc = np.broadcast_to(k[:, :, :1], k.shape).copy()
+    dq2, _, _ = oracle.attention_backward(q, kc, v, ra, None, 64, 3, do)
+    assert np.abs(dq2).max() < 1e-12
+
+
+def test_lse_is_the_softmax_normaliser():
+    q, k, v, do, sm, ra = _fd_case(12 * 64, 600, seed=9)
+    lse = oracle.attention_lse(q, k, ra, sm, 64, 3)
+    # with v = one-hot of key t, the output is p[:, t] = exp(s[:, t] - lse)
+    L = q.shape[2]
+    t = 5
+    e = np.zeros_like(v)
+    e[..., t, 0] = 1.0
+    p_t = oracle.attention(q, k, e, ra, sm, 64, 3)[..., 0]
+    s_t = (q @ k[:, :, t:t + 1].transpose(0, 1, 3, 2))[..., 0] / 8.0   # key t is in block 0 (a global block)
+    assert np.abs(p_t - np.exp(s_t - lse)).max() < 1e-12
