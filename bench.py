@@ -355,6 +355,75 @@ def run_cuda(args):
     return 0
 
 
+def run_bwd(args):
+    """Backward pass (bigbird_attn_bwd) on the same workload: one step = the
+    gradients dq, dk, dv of one batch, with the forward's out and lse (from
+    bigbird_attn_fwd_train) and dout resident. Single GPU."""
+    import torch
+
+    import block_sparse_long_attention_b200 as bb
+    from block_sparse_long_attention_b200.workloads import WORKLOADS, make_inputs
+
+    world, rank, local = _dist_env()
+    if rank != 0:
+        return 0
+    dev = torch.device("cuda", local if world > 1 else 0)
+    torch.cuda.set_device(dev)
+    w = WORKLOADS[args.workload]
+    inp = make_inputs(w)
+    sparse = not bb.is_fallback(w.L, w.block, w.r)
+    q, k, v = (inp[x].to(dev) for x in "qkv")
+    sm = None if inp["seq_mask"] is None else inp["seq_mask"].to(dev)
+    ra = torch.from_numpy(bb.rand_attn_generate(w.H, w.L, w.block, w.r, seed=w.seed)).to(dev) if sparse else None
+    dout = torch.randn(q.shape, generator=torch.Generator().manual_seed(w.seed)).to(torch.bfloat16).to(dev)
+    out, lse = bb.fwd_train(q, k, v, ra, sm, block=w.block, r=w.r)
+    props = torch.cuda.get_device_properties(dev)
+    flush = torch.empty(2 * int(props.L2_cache_size) // 4 + (1 << 20), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(args.warmup):
+        flush.zero_()
+        bb.bwd(q, k, v, out, dout, lse, ra, sm, block=w.block, r=w.r)
+    torch.cuda.synchronize(dev)
+    steps = min(args.steps, 50)
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    sampler = ClockSampler(dev.index)
+    sampler.start()
+    time.sleep(1.0)
+    torch.cuda.synchronize(dev)
+    sampler.t0 = time.time()
+    for i in range(steps):
+        flush.zero_()
+        starts[i].record(stream)
+        bb.bwd(q, k, v, out, dout, lse, ra, sm, block=w.block, r=w.r)
+        ends[i].record(stream)
+    torch.cuda.synchronize(dev)
+    sampler.t1 = time.time()
+    clocks = sampler.stop()
+    if bb.device_status() != 0:
+        raise RuntimeError("device error during the timed region")
+    ms = float(np.mean([a.elapsed_time(b) for a, b in zip(starts, ends)]))
+    import oracle  # work accounting only (FLOP count formula)
+    flops = oracle.backward_flops(w.B, w.H, w.L, w.d, w.block, w.r)
+    value = flops / (ms * 1e-3) / 1e12
+    # fp32 CUDA-core peak from unit counts and clocks: SMs x 128 FMA lanes x 2 FLOP x max SM clock
+    sm_ghz = (clocks or {}).get("sm_max_mhz") or 1965.0
+    peak = props.multi_processor_count * 128 * 2 * float(sm_ghz) * 1e-3 / 1e3
+    line = {
+        "metric": "block-sparse attention backward TFLOP/s (dq, dk, dv) at L=4096, 1xB200", "value": value,
+        "unit": UNIT, "n_gpus": 1, "steps": steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32 (bf16 inputs)",
+        "data": "synthetic", "pass": "bwd",
+        "config": _config(w, 1, "L2 flushed (2x L2 write) before every timed step"),
+        "roofline": {"bound": "alu", "achieved": value, "peak": peak, "unit": "TFLOP/s", "frac": value / peak,
+                     "traffic": None, "kernel": "bigbird_bwd_kernel (fp32 CUDA cores, fp32 atomics for dk, dv)",
+                     "peak_source": "SMs x 128 fp32 FMA lanes x 2 x max SM clock"},
+        "gpu_launches": steps, "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -364,11 +433,15 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--pass", dest="pass_", default="fwd", choices=["fwd", "bwd"],
+                    help="fwd (default, the headline) or bwd (the backward pass)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":
         return run_reference(args)
+    if args.pass_ == "bwd":
+        return run_bwd(args)
     return run_cuda(args)
 
 

@@ -52,6 +52,8 @@ def _load():
         "bigbird_status_string": (ctypes.c_char_p, [I]),
         "bigbird_attn_fwd_noalloc": (I, [P, P, P, P, P, P, I, I, I, I, I, I, I, U, P]),
         "bigbird_attn_noalloc_scratch_bytes": (Z, []),
+        "bigbird_attn_fwd_train": (I, [P, P, P, P, P, P, P, I, I, I, I, I, I, I, U, P, Z, P]),
+        "bigbird_attn_bwd": (I, [P, P, P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, U, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -141,6 +143,77 @@ def _stream_handle(stream):
     return ctypes.c_void_p(s.cuda_stream)
 
 
+def _check_inputs(q, k, v, rand_attn, seq_mask, block, r):
+    import torch
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if not (t.is_cuda and t.dtype == torch.bfloat16 and t.is_contiguous() and t.dim() == 4):
+            raise ValueError(f"{name} must be a contiguous bf16 CUDA tensor [B, H, L, d]")
+    B, H, L, d = q.shape
+    if k.shape != q.shape or v.shape != q.shape:
+        raise ValueError("q, k, v shapes differ")
+    ra_ptr = None
+    if rand_attn is not None:
+        if not (rand_attn.is_cuda and rand_attn.dtype == torch.int32 and rand_attn.is_contiguous()):
+            raise ValueError("rand_attn must be a contiguous int32 CUDA tensor [H, nb-2, r]")
+        if rand_attn.shape != (H, L // block - 2, r):
+            raise ValueError(f"rand_attn shape {tuple(rand_attn.shape)} != {(H, L // block - 2, r)}")
+        ra_ptr = rand_attn.data_ptr()
+    sm_ptr = None
+    if seq_mask is not None:
+        if not (seq_mask.is_cuda and seq_mask.dtype == torch.uint8 and seq_mask.is_contiguous()
+                and seq_mask.shape == (B, L)):
+            raise ValueError("seq_mask must be a contiguous uint8 CUDA tensor [B, L]")
+        sm_ptr = seq_mask.data_ptr()
+    return B, H, L, d, ra_ptr, sm_ptr
+
+
+def fwd_train(q, k, v, rand_attn, seq_mask=None, *, block: int = 64, r: int = 3, out_dtype=None,
+              force_sparse: bool = False, workspace=None, stream=None):
+    """Forward for training: returns (out, lse) with lse [B, H, L] fp32 the
+    natural-log log-sum-exp of each row's scores (what bwd() needs)."""
+    import torch
+    B, H, L, d, ra_ptr, sm_ptr = _check_inputs(q, k, v, rand_attn, seq_mask, block, r)
+    out_dtype = torch.bfloat16 if out_dtype is None else out_dtype
+    if out_dtype not in (torch.bfloat16, torch.float32):
+        raise ValueError("out_dtype must be bf16 or fp32")
+    out = torch.empty((B, H, L, d), dtype=out_dtype, device=q.device)
+    lse = torch.empty((B, H, L), dtype=torch.float32, device=q.device)
+    flags = BB_FLAG_FORCE_SPARSE if force_sparse else 0
+    lib_ = _load()
+    ws_bytes = int(lib_.bigbird_attn_workspace_size(B, H, L, d, block, r, flags))
+    if workspace is None or workspace.numel() * workspace.element_size() < ws_bytes:
+        workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=q.device)
+    st = lib_.bigbird_attn_fwd_train(q.data_ptr(), k.data_ptr(), v.data_ptr(), ra_ptr, sm_ptr, out.data_ptr(),
+                                     lse.data_ptr(), B, H, L, d, block, r,
+                                     BB_OUT_F32 if out_dtype == torch.float32 else BB_OUT_BF16, flags,
+                                     workspace.data_ptr(), ws_bytes, _stream_handle(stream))
+    _check(st, "bigbird_attn_fwd_train")
+    return out, lse
+
+
+def bwd(q, k, v, out, dout, lse, rand_attn, seq_mask=None, *, block: int = 64, r: int = 3,
+        force_sparse: bool = False, stream=None):
+    """Backward: returns (dq, dk, dv), fp32 [B, H, L, d], the gradients of
+    sum(dout * out). out is the forward's output (bf16 or fp32), dout a bf16
+    tensor of its shape, lse from fwd_train()."""
+    import torch
+    B, H, L, d, ra_ptr, sm_ptr = _check_inputs(q, k, v, rand_attn, seq_mask, block, r)
+    if not (dout.is_cuda and dout.dtype == torch.bfloat16 and dout.is_contiguous() and dout.shape == q.shape):
+        raise ValueError("dout must be a contiguous bf16 CUDA tensor of q's shape")
+    if not (out.is_cuda and out.dtype in (torch.bfloat16, torch.float32) and out.is_contiguous()
+            and out.shape == q.shape):
+        raise ValueError("out must be the forward's output (bf16 or fp32, q's shape)")
+    if not (lse.is_cuda and lse.dtype == torch.float32 and lse.is_contiguous() and lse.shape == (B, H, L)):
+        raise ValueError("lse must be a contiguous fp32 CUDA tensor [B, H, L]")
+    dq, dk, dv = (torch.empty((B, H, L, d), dtype=torch.float32, device=q.device) for _ in range(3))
+    st = _load().bigbird_attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), dout.data_ptr(),
+                                  lse.data_ptr(), ra_ptr, sm_ptr, dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+                                  B, H, L, d, block, r, BB_OUT_F32 if out.dtype == torch.float32 else BB_OUT_BF16,
+                                  BB_FLAG_FORCE_SPARSE if force_sparse else 0, _stream_handle(stream))
+    _check(st, "bigbird_attn_bwd")
+    return dq, dk, dv
+
+
 def fwd(q, k, v, rand_attn, seq_mask=None, *, block: int = 64, r: int = 3, out=None, out_dtype=None,
         force_sparse: bool = False, debug_checks: bool = False, workspace=None, stream=None):
     """BigBird ITC attention forward: returns out [B, H, L, d] (bf16, or fp32
@@ -200,6 +273,6 @@ def device_status(stream=None) -> int:
 
 
 __all__ = [
-    "BigBirdError", "fwd", "workspace_size", "is_fallback", "rand_attn_generate", "rand_attn_validate",
+    "BigBirdError", "fwd", "fwd_train", "bwd", "workspace_size", "is_fallback", "rand_attn_generate", "rand_attn_validate",
     "mask_prep", "pattern_table", "device_status", "status_string", "lib", "LIB_PATH",
 ]

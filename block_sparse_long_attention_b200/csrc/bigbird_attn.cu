@@ -107,6 +107,7 @@ struct FwdParams {
   const int32_t* rand_attn;
   const uint8_t* seq_mask;
   void* out;
+  float* lse;      // [B*H*L] natural-log log-sum-exp of each row's scores, or null
   float* part_o;   // [BH, nsplit, 128, 64]
   float* part_ml;  // [BH, nsplit, 128, 2]
   uint32_t* status;
@@ -694,6 +695,8 @@ __device__ void softmax_role(SharedStorage& s, const FwdParams& p, uint32_t tmem
     } else if (exists) {
       const float inv = 1.f / l_run;
       const size_t row = static_cast<size_t>(bh) * p.L + static_cast<size_t>(qblk) * kBlock + (tid & 63);
+      // log sum_k exp(s_k) = ln 2 * (m_ref + log2 l), the scores in log2 units being s * log2(e).
+      if (p.lse) p.lse[row] = (m_ref + log2f(l_run)) * 0.69314718055994531f;
 #pragma unroll 1
       for (int c0 = 0; c0 < kHeadDim; c0 += 16) {
         uint32_t o[16];
@@ -781,8 +784,8 @@ bigbird_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
 constexpr int kMergeRowsPerCta = 16;
 
 __global__ void __launch_bounds__(256)
-bigbird_merge_kernel(const float* __restrict__ part_o, const float* __restrict__ part_ml, void* out, int nsplit,
-                     int L, int nb, int out_f32) {
+bigbird_merge_kernel(const float* __restrict__ part_o, const float* __restrict__ part_ml, void* out, float* lse,
+                     int nsplit, int L, int nb, int out_f32) {
   // Launched as a programmatic dependent of the attention kernel: wait until
   // that grid has completed and its partials are visible.
   asm volatile("griddepcontrol.wait;" ::: "memory");
@@ -809,6 +812,7 @@ bigbird_merge_kernel(const float* __restrict__ part_o, const float* __restrict__
   const float inv = 1.f / l;
   const int qblk = row < kBlock ? 0 : nb - 1;
   const size_t orow = static_cast<size_t>(bh) * L + static_cast<size_t>(qblk) * kBlock + (row & (kBlock - 1));
+  if (lse && c4 == 0) lse[orow] = (mmax + log2f(l)) * 0.69314718055994531f;
   if (out_f32) {
     reinterpret_cast<float4*>(static_cast<float*>(out) + orow * kHeadDim)[c4] =
         make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
@@ -927,9 +931,9 @@ size_t bigbird_attn_workspace_size(int B, int H, int L, int d, int block, int r,
   return pl.ws_bytes;
 }
 
-int bigbird_attn_fwd_ex(const void* q, const void* k, const void* v, const int32_t* rand_attn,
-                        const uint8_t* seq_mask, void* out, int B, int H, int L, int d, int block, int r,
-                        int out_dtype, unsigned flags, void* workspace, size_t workspace_bytes, void* stream_) {
+static int fwd_impl(const void* q, const void* k, const void* v, const int32_t* rand_attn, const uint8_t* seq_mask,
+                    void* out, float* lse, int B, int H, int L, int d, int block, int r, int out_dtype, unsigned flags,
+                    void* workspace, size_t workspace_bytes, void* stream_) {
   cudaStream_t stream = static_cast<cudaStream_t>(stream_);
   Plan pl;
   int st = make_plan(B, H, L, d, block, r, flags, pl);
@@ -969,6 +973,7 @@ int bigbird_attn_fwd_ex(const void* q, const void* k, const void* v, const int32
   p.rand_attn = rand_attn;
   p.seq_mask = seq_mask;
   p.out = out;
+  p.lse = lse;
   p.B = B;
   p.H = H;
   p.L = L;
@@ -1029,10 +1034,26 @@ int bigbird_attn_fwd_ex(const void* q, const void* k, const void* v, const int32
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     e = cudaLaunchKernelEx(&cfg, bigbird_merge_kernel, static_cast<const float*>(p.part_o),
-                           static_cast<const float*>(p.part_ml), out, pl.nsplit, L, pl.nb, p.out_f32);
+                           static_cast<const float*>(p.part_ml), out, p.lse, pl.nsplit, L, pl.nb, p.out_f32);
   }
   if (owned) cudaFreeAsync(ws, stream);
   return e == cudaSuccess ? BB_OK : BB_ERR_CUDA;
+}
+
+int bigbird_attn_fwd_ex(const void* q, const void* k, const void* v, const int32_t* rand_attn,
+                        const uint8_t* seq_mask, void* out, int B, int H, int L, int d, int block, int r,
+                        int out_dtype, unsigned flags, void* workspace, size_t workspace_bytes, void* stream) {
+  return fwd_impl(q, k, v, rand_attn, seq_mask, out, nullptr, B, H, L, d, block, r, out_dtype, flags, workspace,
+                  workspace_bytes, stream);
+}
+
+int bigbird_attn_fwd_train(const void* q, const void* k, const void* v, const int32_t* rand_attn,
+                           const uint8_t* seq_mask, void* out, float* lse, int B, int H, int L, int d, int block,
+                           int r, int out_dtype, unsigned flags, void* workspace, size_t workspace_bytes,
+                           void* stream) {
+  if (!lse) return BB_ERR_INVALID_ARG;
+  return fwd_impl(q, k, v, rand_attn, seq_mask, out, lse, B, H, L, d, block, r, out_dtype, flags, workspace,
+                  workspace_bytes, stream);
 }
 
 int bigbird_attn_fwd(const void* q, const void* k, const void* v, const int32_t* rand_attn, const uint8_t* seq_mask,

@@ -111,6 +111,41 @@ int bigbird_attn_fwd_ex(const void* q, const void* k, const void* v, const int32
                         const uint8_t* seq_mask, void* out, int B, int H, int L, int d, int block, int r,
                         int out_dtype, unsigned flags, void* workspace, size_t workspace_bytes, void* stream);
 
+/*
+ * bigbird_attn_fwd_train -- bigbird_attn_fwd_ex that also writes, for the
+ * backward pass, each row's natural-log log-sum-exp of its scores:
+ *   lse[b,h,t] = log sum_k exp(s[t,k]),  s = q.k / sqrt(d) + bias
+ * over the row's attended keys (the softmax normaliser).
+ *   lse  device fp32 [B, H, L], written in full; NULL -> BB_ERR_INVALID_ARG.
+ * Everything else as bigbird_attn_fwd_ex.
+ */
+int bigbird_attn_fwd_train(const void* q, const void* k, const void* v, const int32_t* rand_attn,
+                           const uint8_t* seq_mask, void* out, float* lse, int B, int H, int L, int d, int block,
+                           int r, int out_dtype, unsigned flags, void* workspace, size_t workspace_bytes,
+                           void* stream);
+
+/*
+ * bigbird_attn_bwd -- gradients of sum(dout * out) with respect to q, k, v
+ * for the same pattern as the forward [TFG-BigBird, section "BigBird：从二次方
+ * 注意力到线性稀疏注意力"; HF-Pegasus, section "三类注意力组合"], by the chain rule
+ * through each row's softmax (p recomputed as exp(s - lse)):
+ *   dv = p^T dout,  dp = dout v^T,  ds = p (dp - rowsum(dout * out)),
+ *   dq = ds k / sqrt(d),  dk = ds^T q / sqrt(d).
+ *   q, k, v, dout  device bf16 [B, H, L, d] (dout: gradient of out).
+ *   out            device [B, H, L, d]: the forward's output, bf16 or fp32 (out_dtype).
+ *   lse            device fp32 [B, H, L] from bigbird_attn_fwd_train.
+ *   rand_attn, seq_mask, B, H, L, d, block, r, BB_FLAG_FORCE_SPARSE: as the forward.
+ *   dq, dk, dv     device fp32 [B, H, L, d], written in full (dk and dv are
+ *                  zeroed with cudaMemsetAsync on `stream`, then accumulated).
+ * Asynchronous on `stream`; nothing is allocated. Errors as the forward
+ * (d != 64 or block != 64 -> BB_ERR_UNSUPPORTED). Out-of-range rand_attn
+ * entries are skipped.
+ */
+int bigbird_attn_bwd(const void* q, const void* k, const void* v, const void* out, const void* dout,
+                     const float* lse, const int32_t* rand_attn, const uint8_t* seq_mask, float* dq, float* dk,
+                     float* dv, int B, int H, int L, int d, int block, int r, int out_dtype, unsigned flags,
+                     void* stream);
+
 /* 1 if (L, block, r) runs full attention (nb <= 5 + 2r), 0 if sparse, <0 on
  * invalid sizes [HF-Pegasus, section "序列过短时的自动回退"]. */
 int bigbird_attn_is_fallback(int L, int block, int r);
