@@ -13,7 +13,10 @@
 // i (all of them for the global rows and the full-attention fallback; else
 // the set {0, nb-1, i-1, i, i+1} and the row's random blocks), keeps dq_i in
 // registers and adds its dk_j, dv_j contributions with fp32 atomics (a key
-// block receives from every query block that attends to it).
+// block receives from every query block that attends to it). Every product
+// is computed as 4x4 register tiles per thread (16 x 16 threads over a 64x64
+// result), reading 4-wide vectors along the summed dimension, so each shared-
+// memory load feeds four FMAs or more.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -26,7 +29,7 @@ namespace bbw {
 constexpr int kBlock = 64;
 constexpr int kDim = 64;
 constexpr int kThreads = 256;
-constexpr int kLd = kDim + 1;  // padded row stride of the fp32 tiles
+constexpr int kLd = kDim + 4;  // row stride of the fp32 tiles (16-byte aligned rows)
 constexpr int kMaxList = 5 + 16;
 
 struct BwdParams {
@@ -82,8 +85,10 @@ __global__ void __launch_bounds__(kThreads, 2) bigbird_bwd_kernel(const BwdParam
   const int b = bh / p.H;
   const int h = bh % p.H;
   const int t = threadIdx.x;
-  const int row = t >> 2;          // query row (S/dq phases) or key (dk/dv phase) of this thread
+  const int row = t >> 2;          // row of the D computation (4 threads per row)
   const int c0 = (t & 3) * 16;     // its 16 columns
+  const int ty = t >> 4;           // 4x4 result tile: rows (or keys) 4ty..4ty+3
+  const int tx = t & 15;           // and columns (keys or dims) 4tx..4tx+3
   const size_t head = static_cast<size_t>(bh) * p.L;
   const size_t q0 = head + static_cast<size_t>(i) * kBlock;
 
@@ -127,9 +132,11 @@ __global__ void __launch_bounds__(kThreads, 2) bigbird_bwd_kernel(const BwdParam
   const int nkb = all ? p.nb : s.nlist;
   const float log2e = 1.4426950408889634f;
 
-  float dq[16];
+  float dq[4][4];  // rows 4ty.., dims 4tx..
 #pragma unroll
-  for (int x = 0; x < 16; ++x) dq[x] = 0.f;
+  for (int a = 0; a < 4; ++a)
+#pragma unroll
+    for (int c = 0; c < 4; ++c) dq[a][c] = 0.f;
 
   for (int e = 0; e < nkb; ++e) {
     const int j = all ? e : s.list[e];
@@ -138,59 +145,106 @@ __global__ void __launch_bounds__(kThreads, 2) bigbird_bwd_kernel(const BwdParam
     load_tile(s.v, p.v, k0);
     if (t < kBlock) s.bias[t] = (p.seq_mask && !p.seq_mask[static_cast<size_t>(b) * p.L + j * kBlock + t]) ? -10000.f : 0.f;
     __syncthreads();
-    // p and ds of row `row`, keys c0..c0+15
+    // p and ds for rows 4ty..4ty+3 and keys 4tx..4tx+3 of the block
     {
-      const float lse2 = s.lse[row] * log2e;
-      const float dr = s.dsum[row];
-#pragma unroll 4
-      for (int c = c0; c < c0 + 16; ++c) {
-        float sc = 0.f, dp = 0.f;
-#pragma unroll 16
-        for (int x = 0; x < kDim; ++x) {
-          sc = fmaf(s.q[row][x], s.k[c][x], sc);
-          dp = fmaf(s.dout[row][x], s.v[c][x], dp);
+      float sc[4][4], dp[4][4];
+#pragma unroll
+      for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) sc[a][c] = dp[a][c] = 0.f;
+#pragma unroll 2
+      for (int x = 0; x < kDim; x += 4) {
+        float4 qa[4], ka[4], da[4], va[4];
+#pragma unroll
+        for (int a = 0; a < 4; ++a) {
+          qa[a] = *reinterpret_cast<const float4*>(&s.q[4 * ty + a][x]);
+          da[a] = *reinterpret_cast<const float4*>(&s.dout[4 * ty + a][x]);
+          ka[a] = *reinterpret_cast<const float4*>(&s.k[4 * tx + a][x]);
+          va[a] = *reinterpret_cast<const float4*>(&s.v[4 * tx + a][x]);
         }
-        const float pv = exp2f(fmaf(sc, p.scale, s.bias[c]) * log2e - lse2);
-        s.p[row][c] = pv;
-        s.ds[row][c] = pv * (dp - dr);
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            sc[a][c] = fmaf(qa[a].x, ka[c].x, fmaf(qa[a].y, ka[c].y, fmaf(qa[a].z, ka[c].z, fmaf(qa[a].w, ka[c].w, sc[a][c]))));
+            dp[a][c] = fmaf(da[a].x, va[c].x, fmaf(da[a].y, va[c].y, fmaf(da[a].z, va[c].z, fmaf(da[a].w, va[c].w, dp[a][c]))));
+          }
+      }
+#pragma unroll
+      for (int a = 0; a < 4; ++a) {
+        const int rr = 4 * ty + a;
+        const float lse2 = s.lse[rr] * log2e;
+        const float dr = s.dsum[rr];
+        float4 pv4, ds4;
+        float* pv = reinterpret_cast<float*>(&pv4);
+        float* dsv = reinterpret_cast<float*>(&ds4);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          pv[c] = exp2f(fmaf(sc[a][c], p.scale, s.bias[4 * tx + c]) * log2e - lse2);
+          dsv[c] = pv[c] * (dp[a][c] - dr);
+        }
+        *reinterpret_cast<float4*>(&s.p[rr][4 * tx]) = pv4;
+        *reinterpret_cast<float4*>(&s.ds[rr][4 * tx]) = ds4;
       }
     }
     __syncthreads();
-    // dq of row `row`, columns c0..c0+15: sum over the block's keys
+    // dq[rows 4ty.., dims 4tx..] += ds[rows, all keys] . k[all keys, dims]
 #pragma unroll 4
     for (int c = 0; c < kBlock; ++c) {
-      const float w = s.ds[row][c];
+      const float4 kv = *reinterpret_cast<const float4*>(&s.k[c][4 * tx]);
 #pragma unroll
-      for (int x = 0; x < 16; ++x) dq[x] = fmaf(w, s.k[c][c0 + x], dq[x]);
+      for (int a = 0; a < 4; ++a) {
+        const float w = s.ds[4 * ty + a][c];
+        dq[a][0] = fmaf(w, kv.x, dq[a][0]);
+        dq[a][1] = fmaf(w, kv.y, dq[a][1]);
+        dq[a][2] = fmaf(w, kv.z, dq[a][2]);
+        dq[a][3] = fmaf(w, kv.w, dq[a][3]);
+      }
     }
-    // dk and dv of key `row` of block j, columns c0..c0+15: sum over the query rows
+    // dk[keys 4ty.., dims 4tx..] += ds^T q,  dv[keys 4ty.., dims 4tx..] += p^T dout
     {
-      float dk[16], dv[16];
+      float dk[4][4], dv[4][4];
 #pragma unroll
-      for (int x = 0; x < 16; ++x) dk[x] = dv[x] = 0.f;
+      for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) dk[a][c] = dv[a][c] = 0.f;
 #pragma unroll 4
       for (int rr = 0; rr < kBlock; ++rr) {
-        const float w = s.ds[rr][row];
-        const float pw = s.p[rr][row];
+        const float4 w = *reinterpret_cast<const float4*>(&s.ds[rr][4 * ty]);
+        const float4 pw = *reinterpret_cast<const float4*>(&s.p[rr][4 * ty]);
+        const float4 qv = *reinterpret_cast<const float4*>(&s.q[rr][4 * tx]);
+        const float4 dv4 = *reinterpret_cast<const float4*>(&s.dout[rr][4 * tx]);
+        const float ws[4] = {w.x, w.y, w.z, w.w};
+        const float ps[4] = {pw.x, pw.y, pw.z, pw.w};
 #pragma unroll
-        for (int x = 0; x < 16; ++x) {
-          dk[x] = fmaf(w, s.q[rr][c0 + x], dk[x]);
-          dv[x] = fmaf(pw, s.dout[rr][c0 + x], dv[x]);
+        for (int a = 0; a < 4; ++a) {
+          dk[a][0] = fmaf(ws[a], qv.x, dk[a][0]);
+          dk[a][1] = fmaf(ws[a], qv.y, dk[a][1]);
+          dk[a][2] = fmaf(ws[a], qv.z, dk[a][2]);
+          dk[a][3] = fmaf(ws[a], qv.w, dk[a][3]);
+          dv[a][0] = fmaf(ps[a], dv4.x, dv[a][0]);
+          dv[a][1] = fmaf(ps[a], dv4.y, dv[a][1]);
+          dv[a][2] = fmaf(ps[a], dv4.z, dv[a][2]);
+          dv[a][3] = fmaf(ps[a], dv4.w, dv[a][3]);
         }
       }
-      float* dkp = p.dk + (k0 + row) * kDim + c0;
-      float* dvp = p.dv + (k0 + row) * kDim + c0;
 #pragma unroll
-      for (int x = 0; x < 16; ++x) {
-        atomicAdd(dkp + x, dk[x] * p.scale);
-        atomicAdd(dvp + x, dv[x]);
+      for (int a = 0; a < 4; ++a) {
+        float* dkp = p.dk + (k0 + 4 * ty + a) * kDim + 4 * tx;
+        float* dvp = p.dv + (k0 + 4 * ty + a) * kDim + 4 * tx;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          atomicAdd(dkp + c, dk[a][c] * p.scale);
+          atomicAdd(dvp + c, dv[a][c]);
+        }
       }
     }
     __syncthreads();
   }
-  float* dqp = p.dq + (q0 + row) * kDim + c0;
 #pragma unroll
-  for (int x = 0; x < 16; ++x) dqp[x] = dq[x] * p.scale;
+  for (int a = 0; a < 4; ++a)
+    *reinterpret_cast<float4*>(p.dq + (q0 + 4 * ty + a) * kDim + 4 * tx) =
+        make_float4(dq[a][0] * p.scale, dq[a][1] * p.scale, dq[a][2] * p.scale, dq[a][3] * p.scale);
 }
 
 }  // namespace bbw
