@@ -314,7 +314,7 @@ def run_cuda(args):
     # DRAM bytes (read + write) of one bigbird_fwd_kernel launch on the default
     # workload, from the ncu capture summarised in
     # profiles/bigbird_fwd_l4096_b4h12.md; valid for that kernel source only.
-    traffic = 86.20e6 if (w.name == DEFAULT_WORKLOAD and world == 1) else None
+    traffic = 88.87e6 if (w.name == DEFAULT_WORKLOAD and world == 1) else None
     roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
             "frac": achieved / peak, "traffic": traffic,
             "kernel": "bigbird_fwd_kernel + bigbird_merge_kernel (one fwd call; traffic: fwd kernel, ncu)",

@@ -54,6 +54,7 @@ def _load():
         "bigbird_attn_noalloc_scratch_bytes": (Z, []),
         "bigbird_attn_fwd_train": (I, [P, P, P, P, P, P, P, I, I, I, I, I, I, I, U, P, Z, P]),
         "bigbird_attn_bwd": (I, [P, P, P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, U, P]),
+        "bigbird_wait_probe": (I, [U, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)

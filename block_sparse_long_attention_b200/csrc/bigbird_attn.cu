@@ -822,6 +822,18 @@ bigbird_merge_kernel(const float* __restrict__ part_o, const float* __restrict__
   }
 }
 
+// Self-test of the bounded-wait path: one thread waits for an mbarrier that
+// nothing arrives on; the wait runs out after limit_ns and sets the timeout
+// bit of the status word, as a lost completion inside the forward would.
+__global__ void bigbird_wait_probe_kernel(uint32_t* status, uint64_t limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    fence_barrier_init();
+    if (!mbar_wait_for(smem_u32(&bar), 0, limit_ns)) atomicOr(status, kStatusTimeout);
+  }
+}
+
 // ---------------------------------------------------------------- host side
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -1060,6 +1072,17 @@ int bigbird_attn_fwd(const void* q, const void* k, const void* v, const int32_t*
                      void* out, int B, int H, int L, int d, int block, int r, void* stream) {
   return bigbird_attn_fwd_ex(q, k, v, rand_attn, seq_mask, out, B, H, L, d, block, r, BB_OUT_BF16, 0u, nullptr, 0,
                              stream);
+}
+
+int bigbird_wait_probe(unsigned limit_us, void* stream_) {
+  if (limit_us == 0 || limit_us > 2000000u) return BB_ERR_INVALID_ARG;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return BB_ERR_CUDA;
+  DeviceInfo* di = device_info(dev);
+  if (!di || !di->status) return BB_ERR_CUDA;
+  bigbird_wait_probe_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream_)>>>(
+      di->status, static_cast<uint64_t>(limit_us) * 1000ull);
+  return cudaGetLastError() == cudaSuccess ? BB_OK : BB_ERR_CUDA;
 }
 
 int bigbird_device_status(void* stream_, uint32_t* host_status) {

@@ -60,16 +60,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity, uin
 
 // Wait until the phase with the given parity has completed. The waiting
 // thread sleeps in the barrier (so it takes no issue slots from working
-// warps); returns false if the phase did not complete within kWaitTimeoutNs.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+// warps); returns false if the phase did not complete within limit_ns.
+__device__ __forceinline__ bool mbar_wait_for(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
   constexpr uint32_t kSuspendNs = 1000000;  // re-check the clock every millisecond
   if (mbar_try_wait(bar, parity, kSuspendNs)) return true;
   const uint64_t t0 = globaltimer_ns();
 #pragma unroll 1
   while (true) {
     if (mbar_try_wait(bar, parity, kSuspendNs)) return true;
-    if (globaltimer_ns() - t0 > kWaitTimeoutNs) return false;
+    if (globaltimer_ns() - t0 > limit_ns) return false;
   }
+}
+
+// The kernels' wait: bounded by kWaitTimeoutNs.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+  return mbar_wait_for(bar, parity, kWaitTimeoutNs);
 }
 
 // ------------------------------------------------------------------ TMA

@@ -146,6 +146,17 @@ int bigbird_attn_bwd(const void* q, const void* k, const void* v, const void* ou
                      float* dv, int B, int H, int L, int d, int block, int r, int out_dtype, unsigned flags,
                      void* stream);
 
+/*
+ * bigbird_wait_probe -- self-test of the failure-detection path. Launches one
+ * thread that waits, with the same bounded wait the kernels use, for an
+ * mbarrier nothing arrives on; after limit_us microseconds (1 .. 2e6) the
+ * wait gives up and sets the timeout bit (2) of the device status word, as
+ * a lost completion inside bigbird_attn_fwd would. Nothing faults or hangs;
+ * read the bit with bigbird_device_status. Returns BB_OK once launched,
+ * BB_ERR_INVALID_ARG for a limit out of range.
+ */
+int bigbird_wait_probe(unsigned limit_us, void* stream);
+
 /* 1 if (L, block, r) runs full attention (nb <= 5 + 2r), 0 if sparse, <0 on
  * invalid sizes [HF-Pegasus, section "序列过短时的自动回退"]. */
 int bigbird_attn_is_fallback(int L, int block, int r);

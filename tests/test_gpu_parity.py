@@ -231,3 +231,22 @@ def test_out_of_range_rand_attn_is_flagged():
         bb.fwd(q, k, v, torch.from_numpy(ra).cuda(), None, debug_checks=True)
     assert e.value.status == bb.BB_ERR_BAD_RAND_ATTN
     assert bb.device_status() == 0
+
+
+def test_bounded_wait_runs_out_and_is_reported():
+    """Failure detection without a fault: a wait on an mbarrier that nothing
+    arrives on gives up after its limit, the host reads the timeout bit, and
+    the context stays usable (a forward afterwards is correct and clean)."""
+    import ctypes
+    lib = bb.lib()
+    assert lib.bigbird_wait_probe(0, None) == bb.BB_ERR_INVALID_ARG
+    st = lib.bigbird_wait_probe(20000, ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert st == bb.BB_OK
+    assert bb.device_status() == 2
+    assert bb.device_status() == 0  # read-and-clear
+    w = WORKLOADS["tiny_l1024"]
+    inp = make_inputs(w)
+    ra, ra_o = _rand_attn_pair(w)
+    got = _cuda_fwd(inp, w, ra, torch.float32)
+    want = oracle.attention(inp["q"], inp["k"], inp["v"], ra_o, inp["seq_mask"], w.block, w.r)
+    _check(got, want, "after probe")
