@@ -40,13 +40,14 @@
 // [0,32) once read; O [64,128) fp32. The next S waits for the P.V that reads
 // P (tcgen05 only orders MMAs that share an accumulator).
 //
-// Softmax: a max pass and an exponential pass over each block's 64 columns;
-// the reference max moves only at block boundaries and only when it grows by
-// more than 2^14 (the O rescale is skipped otherwise; the final O / l is exact
-// either way). Padded
-// keys get -10000 added to the scaled score. P.V runs in fp16: P is written as
-// fp16 and each V tile is converted bf16 -> fp16 in shared memory (exact in the
-// fp16 normal range), which keeps three more mantissa bits of P than bf16.
+// Softmax: one pass over each block's 64 columns, 16 at a time; the
+// reference max moves only when a score exceeds it by more than 2^14 (rare:
+// then the P pieces already written in the block are rescaled in TMEM, and O
+// once the previous P.V has landed; the final O / l is exact either way).
+// Padded keys get -10000 added to the scaled score. P.V runs in fp16: P is
+// written as fp16 and each V tile is converted bf16 -> fp16 in shared memory
+// (exact in the fp16 normal range), which keeps three more mantissa bits of P
+// than bf16.
 #include <cuda.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
