@@ -19,6 +19,8 @@ from .bigbird_oracle import (  # noqa: F401
     attention,
     attention_backward,
     attention_lse,
+    attention_probs,
+    attention_probs_rows,
     attention_rows,
     backward_flops,
     block_mask,

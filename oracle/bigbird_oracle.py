@@ -1,4 +1,5 @@
-"""Plain fp64 CPU oracle of BigBird ITC block-sparse attention (forward).
+"""Plain fp64 CPU oracle of BigBird ITC block-sparse attention (forward, its
+attention probabilities, and the backward).
 
 TEST INFRASTRUCTURE ONLY (see the package docstring): the product path never
 imports this module. Every function below is a direct, unoptimised statement of
@@ -365,6 +366,54 @@ def pattern_table(rand_attn: np.ndarray, H: int, L: int, block: int, r: int) -> 
             blocks = np.nonzero(bm[i])[0]
             out[h, i - 1, :len(blocks)] = blocks
     return out
+
+
+# --------------------------------------------------------------------------
+# Attention probabilities (the output_attentions path)
+# --------------------------------------------------------------------------
+
+def attention_probs(q, k, rand_attn, seq_mask, block: int, r: int, force_sparse: bool = False) -> np.ndarray:
+    """The attention weights as the full matrix, probs[B, H, L, L] in fp64.
+
+    The block-sparse model computes the weights of each row group and writes
+    them back into a full (batch, heads, L, L) matrix, every position outside
+    the pattern left at zero [HF-Pegasus, section "三类注意力组合": four
+    scatter_ calls]; that matrix is mostly zeros and carries no gradient
+    [HF-Pegasus, section "使用限制与注意事项"]. Entry [b, h, q, k] is the
+    softmax weight of key k in row q (the same scores as attention()), and
+    exactly 0 where k is outside the row's pattern.
+    """
+    q, k = _as_f64(q), _as_f64(k)
+    B, H, L, d = q.shape
+    nb, sparse = _mode(L, block, r, force_sparse)
+    tok_blk = np.arange(L) // block
+    out = np.zeros((B, H, L, L), dtype=np.float64)
+    for b in range(B):
+        bias = _key_bias(seq_mask, b, L)
+        for h in range(H):
+            bm = block_mask(nb, r, None if rand_attn is None else np.asarray(rand_attn)[h], sparse)
+            out[b, h] = _probs_of_rows(q[b, h], k[b, h], bm[tok_blk][:, tok_blk], bias)
+    return out
+
+
+def attention_probs_rows(q, k, rand_attn, seq_mask, block: int, r: int, b: int, h: int, rows,
+                         force_sparse: bool = False) -> np.ndarray:
+    """Rows of attention_probs() for one (b, h): [len(rows), L] fp64."""
+    q, k = _as_f64(q), _as_f64(k)
+    L = q.shape[2]
+    nb, sparse = _mode(L, block, r, force_sparse)
+    rows = np.asarray(rows, dtype=np.int64)
+    tok_blk = np.arange(L) // block
+    bm = block_mask(nb, r, None if rand_attn is None else np.asarray(rand_attn)[h], sparse)
+    return _probs_of_rows(q[b, h, rows], k[b, h], bm[tok_blk[rows]][:, tok_blk], _key_bias(seq_mask, b, L))
+
+
+def _probs_of_rows(qr: np.ndarray, k: np.ndarray, allowed: np.ndarray, bias: np.ndarray) -> np.ndarray:
+    """Softmax weights of the rows qr over the allowed keys; 0 elsewhere."""
+    s = (qr @ k.T) / math.sqrt(qr.shape[-1]) + bias[None, :]
+    s = np.where(allowed, s, -np.inf)
+    w = np.exp(s - s.max(axis=1, keepdims=True))   # exp(-inf) = 0 outside the pattern
+    return w / w.sum(axis=1, keepdims=True)
 
 
 # --------------------------------------------------------------------------

@@ -452,3 +452,76 @@ def test_lse_is_the_softmax_normaliser():
     p_t = oracle.attention(q, k, e, ra, sm, 64, 3)[..., 0]
     s_t = (q @ k[:, :, t:t + 1].transpose(0, 1, 3, 2))[..., 0] / 8.0   # key t is in block 0 (a global block)
     assert np.abs(p_t - np.exp(s_t - lse)).max() < 1e-12
+
+
+# --------------------------------------------------------------------------
+# Attention probabilities of the oracle: pinned through attention() itself
+# (an identity value matrix turns its output into the weights) and through
+# the closed form exp(s - lse).
+# --------------------------------------------------------------------------
+
+_PROBS_CASES = [(12 * 64, 700, False), (704, 600, False), (8 * 64, 450, True)]
+
+
+@pytest.mark.parametrize("L,pad,force", _PROBS_CASES, ids=["sparse_padded", "fallback", "forced_sparse"])
+def test_probs_are_attention_of_identity_values(L, pad, force):
+    """With V = I (value of key k = the k-th unit vector) the output row q is
+    the weight vector of row q. Catches a probability matrix whose support,
+    scaling or normalisation differs from the (separately pinned) forward."""
+    rng = np.random.default_rng(21)
+    B, H, d, r = 1, 2, 64, 3
+    q = rng.standard_normal((B, H, L, d)) * 0.6
+    k = rng.standard_normal((B, H, L, d)) * 0.6
+    sm = mask_from_lengths(B, L, [pad]).numpy()
+    nb = L // 64
+    if force:   # nb = 5 + r: the random blocks are the rest of the middle rows
+        ra = np.zeros((H, nb - 2, r), dtype=np.int32)
+        for h in range(H):
+            for i in range(1, nb - 1):
+                rest = [j for j in range(1, nb - 1) if abs(j - i) > 1]
+                ra[h, i - 1, :len(rest)] = rest[:r]
+                ra[h, i - 1, len(rest):] = rest[0]
+    else:
+        ra = None if oracle.is_fallback(L, 64, r) else oracle.rand_attn_generate(H, L, 64, r, seed=3)
+    # V = I, 64 columns at a time (attention() takes values of the head width)
+    eye = np.eye(L)
+    want = np.concatenate([oracle.attention(q, k, np.broadcast_to(eye[:, c:c + d], (B, H, L, d)), ra, sm, 64, r,
+                                            force_sparse=force) for c in range(0, L, d)], axis=3)
+    got = oracle.attention_probs(q, k, ra, sm, 64, r, force_sparse=force)
+    assert np.abs(got - want).max() < 1e-12
+    assert np.abs(got.sum(axis=3) - 1.0).max() < 1e-12
+    rows = [0, 63, 64, 200, L - 65, L - 1]
+    assert np.array_equal(oracle.attention_probs_rows(q, k, ra, sm, 64, r, 0, 1, rows, force_sparse=force),
+                          got[0, 1, rows])
+
+
+def test_probs_closed_form_and_support():
+    """probs = exp(s - lse) on the pattern, exactly 0 off it and on padded keys
+    (for rows with a valid key). Catches a wrong score scale, a bias applied to
+    the wrong side, or weight leaking outside the pattern."""
+    rng = np.random.default_rng(22)
+    B, H, L, d, r = 2, 2, 16 * 64, 64, 3
+    q = rng.standard_normal((B, H, L, d)) * 0.5
+    k = rng.standard_normal((B, H, L, d)) * 0.5
+    sm = mask_from_lengths(B, L, [1000, 700]).numpy()
+    ra = oracle.rand_attn_generate(H, L, 64, r, seed=5)
+    p = oracle.attention_probs(q, k, ra, sm, 64, r)
+    lse = oracle.attention_lse(q, k, ra, sm, 64, r)
+    nb = L // 64
+    for b in range(B):
+        for h in range(H):
+            s = q[b, h] @ k[b, h].T / 8.0 + np.where(sm[b].astype(bool), 0.0, -10000.0)[None, :]
+            for i in range(nb):
+                # key blocks of query block i, listed from the rules as the pages state them
+                if i in (0, nb - 1):
+                    blocks = set(range(nb))
+                else:
+                    blocks = {0, nb - 1, i - 1, i, i + 1} | {int(x) for x in ra[h, i - 1]}
+                keys = np.concatenate([np.arange(j * 64, j * 64 + 64) for j in sorted(blocks)])
+                rows = slice(i * 64, i * 64 + 64)
+                off = np.setdiff1d(np.arange(L), keys)
+                assert np.all(p[b, h, rows][:, off] == 0.0)
+                want = np.exp(s[rows][:, keys] - lse[b, h, rows][:, None])
+                assert np.abs(p[b, h, rows][:, keys] - want).max() < 1e-13
+            valid = int(sm[b].sum())
+            assert np.all(p[b, h, :, valid:] == 0.0)
