@@ -424,6 +424,94 @@ def run_bwd(args):
     return 0
 
 
+def run_probs(args):
+    """Attention-probability export (bigbird_attn_probs, packed block-sparse
+    layout, fp32) on the same workload: one step = the weights of every
+    attended (query, key) pair of one batch, with q, k and the forward's lse
+    resident. HBM-bound: the algorithmic bytes are the weights written plus
+    q, k, lse and the mask read once. Single GPU."""
+    import torch
+
+    import block_sparse_long_attention_b200 as bb
+    from block_sparse_long_attention_b200.workloads import WORKLOADS, make_inputs
+
+    world, rank, local = _dist_env()
+    if rank != 0:
+        return 0
+    dev = torch.device("cuda", local if world > 1 else 0)
+    torch.cuda.set_device(dev)
+    w = WORKLOADS[args.workload]
+    inp = make_inputs(w)
+    sparse = not bb.is_fallback(w.L, w.block, w.r)
+    q, k, v = (inp[x].to(dev) for x in "qkv")
+    sm = None if inp["seq_mask"] is None else inp["seq_mask"].to(dev)
+    ra = torch.from_numpy(bb.rand_attn_generate(w.H, w.L, w.block, w.r, seed=w.seed)).to(dev) if sparse else None
+    _, lse = bb.fwd_train(q, k, v, ra, sm, block=w.block, r=w.r)
+    G, nbr, slots = bb.probs_layout(w.L, w.block, w.r, w.d)
+    props = torch.cuda.get_device_properties(dev)
+    flush = torch.empty(2 * int(props.L2_cache_size) // 4 + (1 << 20), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    res = {}
+    for dtype, esize in ((torch.float32, 4), (torch.bfloat16, 2)):
+        pg = torch.empty((w.B, w.H, G, w.block, w.L), dtype=dtype, device=dev)
+        pb = torch.empty((w.B, w.H, nbr, slots, w.block, w.block), dtype=dtype, device=dev) if nbr else None
+
+        def step():
+            bb.probs(q, k, lse, ra, sm, block=w.block, r=w.r, out_dtype=dtype, out=(pg, pb))
+
+        for _ in range(args.warmup):
+            flush.zero_()
+            step()
+        torch.cuda.synchronize(dev)
+        steps = min(args.steps, 200)
+        starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+        ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+        sampler = ClockSampler(dev.index)
+        sampler.start()
+        time.sleep(1.0)
+        torch.cuda.synchronize(dev)
+        sampler.t0 = time.time()
+        for i in range(steps):
+            flush.zero_()
+            starts[i].record(stream)
+            step()
+            ends[i].record(stream)
+        torch.cuda.synchronize(dev)
+        sampler.t1 = time.time()
+        clocks = sampler.stop()
+        if bb.device_status() != 0:
+            raise RuntimeError("device error during the timed region")
+        ms = float(np.mean([a.elapsed_time(b) for a, b in zip(starts, ends)]))
+        out_bytes = (pg.numel() + (0 if pb is None else pb.numel())) * esize
+        in_bytes = 2 * q.numel() * 2 + lse.numel() * 4 + (0 if sm is None else sm.numel())
+        res[str(dtype).split(".")[-1]] = (ms, out_bytes, in_bytes, steps, clocks)
+    ms, out_bytes, in_bytes, steps, clocks = res["float32"]
+    peaks, src = _peaks()
+    peak = float(peaks["hbm_gbs"])
+    gbs = (out_bytes + in_bytes) / (ms * 1e-3) / 1e9
+    bms, bout, bin_, _, _ = res["bfloat16"]
+    bgbs = (bout + bin_) / (bms * 1e-3) / 1e9
+    import oracle  # work accounting only (attended pairs)
+    pairs = w.B * w.H * w.L * oracle.keys_per_row(w.L, w.block, w.r)
+    line = {
+        "metric": "block-sparse attention-probability export GB/s (packed layout, fp32) at L=4096, 1xB200",
+        "value": gbs, "unit": "GB/s", "n_gpus": 1, "steps": steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32 (bf16 inputs)",
+        "data": "synthetic", "pass": "probs",
+        "config": _config(w, 1, "L2 flushed (2x L2 write) before every timed step"),
+        "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s", "frac": gbs / peak,
+                     "traffic": None, "kernel": "bigbird_probs_kernel",
+                     "algorithmic_bytes": out_bytes + in_bytes,
+                     "peak_source": f"{src} HBM copy bandwidth"},
+        "pairs_per_s": pairs / (ms * 1e-3),
+        "bf16_output": {"ms_per_step": bms, "value": bgbs, "unit": "GB/s", "frac": bgbs / peak,
+                        "algorithmic_bytes": bout + bin_},
+        "gpu_launches": steps, "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -433,8 +521,8 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--pass", dest="pass_", default="fwd", choices=["fwd", "bwd"],
-                    help="fwd (default, the headline) or bwd (the backward pass)")
+    ap.add_argument("--pass", dest="pass_", default="fwd", choices=["fwd", "bwd", "probs"],
+                    help="fwd (default, the headline), bwd (the backward pass) or probs (probability export)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -442,6 +530,8 @@ def main():
         return run_reference(args)
     if args.pass_ == "bwd":
         return run_bwd(args)
+    if args.pass_ == "probs":
+        return run_probs(args)
     return run_cuda(args)
 
 

@@ -55,6 +55,9 @@ def _load():
         "bigbird_attn_fwd_train": (I, [P, P, P, P, P, P, P, I, I, I, I, I, I, I, U, P, Z, P]),
         "bigbird_attn_bwd": (I, [P, P, P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, U, P]),
         "bigbird_wait_probe": (I, [U, P]),
+        "bigbird_attn_probs_layout": (I, [I, I, I, I, U, ctypes.POINTER(I), ctypes.POINTER(I), ctypes.POINTER(I)]),
+        "bigbird_attn_probs": (I, [P, P, P, P, P, P, P, I, I, I, I, I, I, I, U, P]),
+        "bigbird_attn_probs_dense": (I, [P, P, P, P, P, P, I, I, I, I, I, I, I, U, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -215,6 +218,76 @@ def bwd(q, k, v, out, dout, lse, rand_attn, seq_mask=None, *, block: int = 64, r
     return dq, dk, dv
 
 
+def probs_layout(L: int, block: int = 64, r: int = 3, d: int = 64, force_sparse: bool = False):
+    """(G, band_rows, band_slots) of the packed probability layout: G full
+    rows per head (2 sparse, nb in the fallback), band tiles
+    [nb-2, 5+r] per head (0, 0 in the fallback)."""
+    g, br, bs = ctypes.c_int(0), ctypes.c_int(0), ctypes.c_int(0)
+    st = _load().bigbird_attn_probs_layout(L, d, block, r, BB_FLAG_FORCE_SPARSE if force_sparse else 0,
+                                          ctypes.byref(g), ctypes.byref(br), ctypes.byref(bs))
+    _check(st, "bigbird_attn_probs_layout")
+    return g.value, br.value, bs.value
+
+
+def _probs_args(q, k, lse, rand_attn, seq_mask, block, r, out_dtype):
+    import torch
+    B, H, L, d, ra_ptr, sm_ptr = _check_inputs(q, k, k, rand_attn, seq_mask, block, r)
+    if not (lse.is_cuda and lse.dtype == torch.float32 and lse.is_contiguous() and lse.shape == (B, H, L)):
+        raise ValueError("lse must be a contiguous fp32 CUDA tensor [B, H, L] (from fwd_train)")
+    out_dtype = torch.float32 if out_dtype is None else out_dtype
+    if out_dtype not in (torch.bfloat16, torch.float32):
+        raise ValueError("out_dtype must be bf16 or fp32")
+    return B, H, L, d, ra_ptr, sm_ptr, out_dtype
+
+
+def probs(q, k, lse, rand_attn, seq_mask=None, *, block: int = 64, r: int = 3, out_dtype=None,
+          force_sparse: bool = False, out=None, stream=None):
+    """Attention weights in the packed block-sparse layout: returns
+    (probs_global [B, H, G, 64, L], probs_band [B, H, nb-2, 5+r, 64, 64] or
+    None in the fallback). Tile t of band row i is against key block
+    pattern_table(...)[h, i-1, t] (zeros where that entry is -1). lse comes
+    from fwd_train() on the same inputs. Default dtype fp32. `out` may be a
+    (probs_global, probs_band) pair of preallocated contiguous tensors."""
+    import torch
+    B, H, L, d, ra_ptr, sm_ptr, out_dtype = _probs_args(q, k, lse, rand_attn, seq_mask, block, r, out_dtype)
+    G, nbr, slots = probs_layout(L, block, r, d, force_sparse)
+    shapes = ((B, H, G, block, L), (B, H, nbr, slots, block, block) if nbr else None)
+    if out is None:
+        pg = torch.empty(shapes[0], dtype=out_dtype, device=q.device)
+        pb = torch.empty(shapes[1], dtype=out_dtype, device=q.device) if nbr else None
+    else:
+        pg, pb = out
+        for t, shp in ((pg, shapes[0]), (pb, shapes[1])):
+            if shp is None:
+                continue
+            if t is None or not (t.is_cuda and t.dtype == out_dtype and t.is_contiguous() and tuple(t.shape) == shp):
+                raise ValueError(f"out tensors must be contiguous CUDA tensors {shapes} of {out_dtype}")
+    st = _load().bigbird_attn_probs(q.data_ptr(), k.data_ptr(), lse.data_ptr(), ra_ptr, sm_ptr, pg.data_ptr(),
+                                    None if pb is None else pb.data_ptr(), B, H, L, d, block, r,
+                                    BB_OUT_F32 if out_dtype == torch.float32 else BB_OUT_BF16,
+                                    BB_FLAG_FORCE_SPARSE if force_sparse else 0, _stream_handle(stream))
+    _check(st, "bigbird_attn_probs")
+    return pg, pb
+
+
+def probs_dense(q, k, lse, rand_attn, seq_mask=None, *, block: int = 64, r: int = 3, out_dtype=None,
+                force_sparse: bool = False, out=None, stream=None):
+    """Attention weights as the full [B, H, L, L] matrix (zeros outside the
+    pattern), the layout the model returns for its attention outputs."""
+    import torch
+    B, H, L, d, ra_ptr, sm_ptr, out_dtype = _probs_args(q, k, lse, rand_attn, seq_mask, block, r, out_dtype)
+    if out is None:
+        out = torch.empty((B, H, L, L), dtype=out_dtype, device=q.device)
+    elif not (out.is_cuda and out.dtype == out_dtype and out.is_contiguous() and out.shape == (B, H, L, L)):
+        raise ValueError("out must be a contiguous CUDA tensor [B, H, L, L] of out_dtype")
+    st = _load().bigbird_attn_probs_dense(q.data_ptr(), k.data_ptr(), lse.data_ptr(), ra_ptr, sm_ptr,
+                                          out.data_ptr(), B, H, L, d, block, r,
+                                          BB_OUT_F32 if out_dtype == torch.float32 else BB_OUT_BF16,
+                                          BB_FLAG_FORCE_SPARSE if force_sparse else 0, _stream_handle(stream))
+    _check(st, "bigbird_attn_probs_dense")
+    return out
+
+
 def fwd(q, k, v, rand_attn, seq_mask=None, *, block: int = 64, r: int = 3, out=None, out_dtype=None,
         force_sparse: bool = False, debug_checks: bool = False, workspace=None, stream=None):
     """BigBird ITC attention forward: returns out [B, H, L, d] (bf16, or fp32
@@ -274,6 +347,6 @@ def device_status(stream=None) -> int:
 
 
 __all__ = [
-    "BigBirdError", "fwd", "fwd_train", "bwd", "workspace_size", "is_fallback", "rand_attn_generate", "rand_attn_validate",
+    "BigBirdError", "fwd", "fwd_train", "bwd", "probs", "probs_dense", "probs_layout", "workspace_size", "is_fallback", "rand_attn_generate", "rand_attn_validate",
     "mask_prep", "pattern_table", "device_status", "status_string", "lib", "LIB_PATH",
 ]

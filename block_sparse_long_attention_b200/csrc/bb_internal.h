@@ -1,0 +1,21 @@
+// Host-side helpers shared by the library's translation units (not part of
+// the C ABI). Implemented in bigbird_attn.cu.
+#pragma once
+
+#include <cuda.h>
+
+#include <cstdint>
+
+namespace bb {
+
+// Tensor map over a [rows, 64] bf16 matrix with 64x64 boxes and 128-byte
+// swizzle (one box = one block of one head). False if the driver entry point
+// is missing or the encoding is rejected.
+bool make_tile_map(CUtensorMap* map, const void* base, uint64_t rows);
+
+// Device address of the library's status word on the current device `dev`
+// (bit 1: an out-of-range rand_attn entry was skipped; bit 2: a bounded wait
+// timed out), or null if `dev` is not an sm_100 device or a query failed.
+uint32_t* status_word(int dev);
+
+}  // namespace bb

@@ -59,6 +59,7 @@
 #include <mutex>
 
 #include "../../include/bigbird_attn.h"
+#include "bb_internal.h"
 #include "sm100_ptx.cuh"
 
 namespace bb {
@@ -898,6 +899,13 @@ static DeviceInfo* device_info(int dev) {
     di.attr_set = true;
   }
   return &di;
+}
+
+bool make_tile_map(CUtensorMap* map, const void* base, uint64_t rows) { return make_map(map, base, rows); }
+
+uint32_t* status_word(int dev) {
+  DeviceInfo* di = device_info(dev);
+  return di && di->ok ? di->status : nullptr;
 }
 
 constexpr size_t kSchedBytes = 256;  // the scheduling counter's slot at the start of the workspace

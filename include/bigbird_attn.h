@@ -147,6 +147,55 @@ int bigbird_attn_bwd(const void* q, const void* k, const void* v, const void* ou
                      void* stream);
 
 /*
+ * Attention probabilities (the output_attentions path). The block-sparse model
+ * writes each row group's softmax weights into a full [B, H, L, L] matrix that
+ * is zero outside the pattern [HF-Pegasus, section "三类注意力组合": four
+ * scatter_ calls]; the matrix carries no gradient [HF-Pegasus, section
+ * "使用限制与注意事项"]. These calls recompute the weights from q, k and the
+ * row log-sum-exp that bigbird_attn_fwd_train wrote for the same inputs:
+ *   p[b,h,t,k] = exp(q_t.k_k / sqrt(d) + bias_k - lse[b,h,t])
+ * on the row's attended keys (bias_k = -10000 for a padded key), 0 elsewhere.
+ *
+ * bigbird_attn_probs_layout -- shapes of the packed layout (host, no GPU):
+ *   *global_rows  G: 2 in the sparse mode (query blocks 0 and nb-1), nb in the
+ *                 full-attention fallback;
+ *   *band_rows    nb - 2 in the sparse mode, 0 in the fallback;
+ *   *band_slots   5 + r in the sparse mode, 0 in the fallback.
+ * Any output pointer may be NULL. Errors as bigbird_attn_fwd_ex's arguments.
+ *
+ * bigbird_attn_probs -- the weights in the packed block-sparse layout:
+ *   q, k          device bf16 [B, H, L, d]; lse device fp32 [B, H, L];
+ *   rand_attn, seq_mask, B, H, L, d, block, r, BB_FLAG_FORCE_SPARSE: as the forward;
+ *   probs_global  device [B, H, G, 64, L]: row g's weights over every key
+ *                 (g = 0: query block 0, g = 1: query block nb-1; in the
+ *                 fallback g = every query block, i.e. the whole matrix);
+ *   probs_band    device [B, H, nb-2, 5+r, 64, 64]: tile t of query block i
+ *                 (1 <= i <= nb-2) holds its weights against key block
+ *                 bigbird_pattern_table(...)[h][i-1][t]; tiles whose table
+ *                 entry is -1 are written as zeros. Unused (may be NULL) in
+ *                 the fallback;
+ *   out_dtype     BB_OUT_F32 or BB_OUT_BF16 (both outputs).
+ * Every element of both outputs is written. Asynchronous on `stream`; nothing
+ * is allocated. Output pointers must be 16-byte aligned
+ * (BB_ERR_UNSUPPORTED otherwise). Out-of-range rand_attn entries are skipped
+ * and flagged (bit 1 of bigbird_device_status). Rows whose keys are all
+ * padded are accurate to ~1e-3 relative (their lse sits near -10000, where
+ * fp32 keeps ~3 decimal places); every other row to ~1e-5.
+ *
+ * bigbird_attn_probs_dense -- the same weights scattered into the full
+ * matrix: probs device [B, H, L, L] (B*H*L*L elements of out_dtype), zeros
+ * outside the pattern, every element written.
+ */
+int bigbird_attn_probs_layout(int L, int d, int block, int r, unsigned flags, int* global_rows, int* band_rows,
+                              int* band_slots);
+int bigbird_attn_probs(const void* q, const void* k, const float* lse, const int32_t* rand_attn,
+                       const uint8_t* seq_mask, void* probs_global, void* probs_band, int B, int H, int L, int d,
+                       int block, int r, int out_dtype, unsigned flags, void* stream);
+int bigbird_attn_probs_dense(const void* q, const void* k, const float* lse, const int32_t* rand_attn,
+                             const uint8_t* seq_mask, void* probs, int B, int H, int L, int d, int block, int r,
+                             int out_dtype, unsigned flags, void* stream);
+
+/*
  * bigbird_wait_probe -- self-test of the failure-detection path. Launches one
  * thread that waits, with the same bounded wait the kernels use, for an
  * mbarrier nothing arrives on; after limit_us microseconds (1 .. 2e6) the

@@ -146,3 +146,43 @@ def test_fwd_argument_errors_before_any_launch():
     assert lib.bigbird_attn_fwd_ex(fake, fake, fake, fake, None, fake, 1, 2, 7 * 64, 64, 64, 3, 0,
                                    bb.BB_FLAG_FORCE_SPARSE, None, 0, None) == bb.BB_ERR_INVALID_ARG
     assert bb.status_string(bb.BB_ERR_UNSUPPORTED) == "unsupported configuration"
+
+
+def test_probs_layout_and_argument_errors_before_any_launch():
+    # packed layout: G full rows per head, then [nb-2, 5+r] band tiles whose
+    # slot t is column t of the pattern table
+    assert bb.probs_layout(4096) == (2, 62, 8)
+    assert bb.probs_layout(2048, r=5) == (2, 30, 10)
+    assert bb.probs_layout(704) == (11, 0, 0)                    # fallback: the whole matrix
+    assert bb.probs_layout(8 * 64, force_sparse=True) == (2, 6, 8)
+    ra = oracle.rand_attn_generate(2, 4096, 64, 3, seed=1)
+    assert oracle.pattern_table(ra, 2, 4096, 64, 3).shape == (2, 62, 8)
+    with pytest.raises(bb.BigBirdError):
+        bb.probs_layout(1000)
+    lib = bb.lib()
+    P = ctypes.c_void_p
+    fake = P(0x10000)  # never dereferenced: every case fails argument checks first
+    base = dict(q=fake, k=fake, lse=fake, ra=fake, sm=None, pg=fake, pb=fake, B=1, H=2, L=4096, d=64, block=64, r=3,
+                dt=bb.BB_OUT_F32, fl=0)
+    cases = [
+        (dict(L=1000), bb.BB_ERR_INVALID_ARG),
+        (dict(r=0), bb.BB_ERR_INVALID_ARG),
+        (dict(d=128), bb.BB_ERR_UNSUPPORTED),
+        (dict(B=0), bb.BB_ERR_INVALID_ARG),
+        (dict(lse=None), bb.BB_ERR_INVALID_ARG),
+        (dict(pb=None), bb.BB_ERR_INVALID_ARG),       # the sparse mode needs the band output
+        (dict(ra=None), bb.BB_ERR_INVALID_ARG),       # and rand_attn
+        (dict(pg=P(0x10004)), bb.BB_ERR_UNSUPPORTED),  # misaligned output
+        (dict(dt=7), bb.BB_ERR_INVALID_ARG),
+        (dict(L=7 * 64, fl=bb.BB_FLAG_FORCE_SPARSE), bb.BB_ERR_INVALID_ARG),
+    ]
+    for kw, want in cases:
+        a = dict(base)
+        a.update(kw)
+        st = lib.bigbird_attn_probs(a["q"], a["k"], a["lse"], a["ra"], a["sm"], a["pg"], a["pb"], a["B"], a["H"],
+                                    a["L"], a["d"], a["block"], a["r"], a["dt"], a["fl"], None)
+        assert st == want, (kw, st)
+    assert lib.bigbird_attn_probs_dense(fake, fake, None, fake, None, fake, 1, 2, 4096, 64, 64, 3, bb.BB_OUT_F32, 0,
+                                        None) == bb.BB_ERR_INVALID_ARG
+    assert lib.bigbird_attn_probs_dense(fake, fake, fake, fake, None, P(0x10002), 1, 2, 4096, 64, 64, 3,
+                                        bb.BB_OUT_BF16, 0, None) == bb.BB_ERR_UNSUPPORTED
