@@ -6,8 +6,9 @@ fp32: s is the tensor cores' fp32 sum of exact bf16 products and lse the GPU
 forward's own log-sum-exp (fp32 sums of unrounded exponentials, ~1e-6
 absolute). For |x| up to ~60 the fp32 roundings of x stay below ~5e-6 (log2
 units) and ex2.approx adds ~2 ulp, so |dp| <~ 5e-6 p. Bars per element:
-|err| <= 2e-5 p + 1e-12 with fp32 output, 2e-3 p + 1e-12 with bf16 output
-(its half-ulp is 2^-9 p). Rows whose keys are all padded have lse near
+|err| <= 2e-5 p + 1e-12 with fp32 output, 4e-3 p + 1e-12 with bf16 output
+(8 significant bits: rounding to nearest moves a value by up to 2^-8 of
+itself). Rows whose keys are all padded have lse near
 -10000, where fp32 resolves ~1e-3: 4e-3 p there. Zeros (outside the pattern,
 padded keys of rows with a valid key, band slots past the end of a row's
 list) therefore have to be exact.
@@ -23,7 +24,7 @@ from block_sparse_long_attention_b200.workloads import WORKLOADS, Workload, make
 
 pytestmark = pytest.mark.gpu
 
-REL_F32, REL_BF16, REL_ALL_PADDED, ABS_FLOOR = 2e-5, 2e-3, 4e-3, 1e-12
+REL_F32, REL_BF16, REL_ALL_PADDED, ABS_FLOOR = 2e-5, 4e-3, 4e-3, 1e-12
 
 
 @pytest.fixture(scope="module", autouse=True)
