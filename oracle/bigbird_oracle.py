@@ -31,7 +31,7 @@ defaults]. A length that is not a multiple of block is an error
 [HF-Pegasus, section "序列长度的块对齐要求"]; r = 0 is unsupported
 [HF-Pegasus, section "使用限制与注意事项"].
 
-Readings where the pages leave a step open (each is listed in the design doc):
+Readings where the pages leave a step open:
 the random blocks of a row are a *set* (a duplicated or window-overlapping
 entry adds nothing); the second rows (1 and nb-2) follow the same three rules;
 the -10000 bias applies to padded keys only and is added after the 1/sqrt(d)
