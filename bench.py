@@ -463,7 +463,7 @@ def run_probs(args):
             flush.zero_()
             step()
         torch.cuda.synchronize(dev)
-        steps = min(args.steps, 200)
+        steps = min(args.steps, 4000)  # ~1 s of timed region: long enough for the clock samples
         starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
         ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
         sampler = ClockSampler(dev.index)

@@ -21,18 +21,23 @@
 //
 // A unit is one query block against up to 8 key-block tiles: a range of 8
 // blocks of a full row, a row's band list (packed), or a range of 8 blocks of
-// any row with its unlisted tiles zero (dense). One CTA per unit, 288 threads:
-//   warp 8     TMEM allocation, TMA loads of the Q block and the listed K
-//              tiles, and the MMAs. Scores are computed transposed,
-//              S^T = K Q^T, two key tiles at a time (M = 128 keys, N = 64
-//              queries, four tcgen05 128x64x16 steps), into one of two
-//              64-column TMEM buffers;
+// any row with its unlisted tiles zero (dense). The kernel is persistent
+// (three CTAs of 320 threads per SM, units dealt out evenly) and
+// warp-specialised, so one unit's setup, loads and MMAs overlap the previous
+// unit's stores:
+//   warp 8     plans each unit (its tiles and output offsets; the band list
+//              from rand_attn) into a 2-slot ring, and loads the Q block and
+//              the listed K tiles by TMA into 2-deep rings;
+//   warp 9     TMEM allocation and the MMAs: scores transposed, S^T = K Q^T,
+//              two key tiles at a time (M = 128 keys, N = 64 queries, four
+//              tcgen05 128x64x16 steps) into one of two 64-column TMEM
+//              buffers;
 //   warps 0-7  thread (warp w, lane l) reads TMEM lane 32 (w % 4) + l (one
 //              key) and the 32 query columns of half w / 4, and writes p for
 //              them. Consecutive lanes hold consecutive keys, so each store
 //              instruction of a warp covers 32 consecutive elements of one
 //              output row (128 bytes in fp32) with no shuffle. Zero tiles are
-//              written with 16-byte stores while the MMAs run.
+//              written with 16-byte stores.
 // Output stores are streaming (evict-first); Q and K loads are kept in L2
 // (each K block is read by every unit that lists it).
 #include <cuda.h>
@@ -54,7 +59,10 @@ constexpr int kDim = 64;
 constexpr int kTiles = 8;                   // key-block tiles per unit
 constexpr int kEpiWarps = 8;                // warps that turn scores into weights
 constexpr int kEpiThreads = kEpiWarps * 32;
-constexpr int kThreads = kEpiThreads + 32;  // + the TMEM / TMA / MMA warp
+constexpr int kProdWarp = kEpiWarps;        // planning + TMA
+constexpr int kMmaWarp = kEpiWarps + 1;     // TMEM + MMA
+constexpr int kThreads = kEpiThreads + 64;
+constexpr int kCtasPerSm = 3;
 constexpr int kMaxR = 16;
 constexpr uint32_t kTileBytes = kBlock * kDim * 2;
 constexpr uint32_t kTmemCols = 128;         // two 64-column S^T buffers
@@ -77,30 +85,50 @@ struct ProbsParams {
   int chunks;          // band chunks of kTiles slots per row (packed)
   int grows;           // full rows per head in the packed layout
   int units_per_head;
+  int total_units;
+  int units_per_cta;   // CTA c takes units [c * units_per_cta, (c + 1) * units_per_cta)
   float scale_log2;    // log2(e) / sqrt(d)
-  float bias_raw;      // -10000 * sqrt(d): the masked-key bias in units of q.k
+  float bias_log2;     // -10000 * log2(e): the masked-key bias in log2 units
+};
+
+struct UnitInfo {
+  long long tile_off[kTiles];  // element offset of each tile's (0, 0) in its output
+  int32_t tile_kb[kTiles];     // key block of each tile, or -1 for a zero tile
+  int32_t comp_tile[kTiles];   // compute slot -> tile index
+  int32_t n_tiles;             // < 0: no more units (every role leaves its loop)
+  int32_t n_comp, ld, bh, qblk, band;
 };
 
 struct __align__(1024) Smem {
-  uint8_t q[kTileBytes];          // the unit's Q block (SW128)
-  uint8_t k[kTiles][kTileBytes];  // listed K tiles in compute order; slots 2g, 2g+1 form one M = 128 operand
-  float lse2[kBlock];             // lse * log2(e) of the block's 64 rows
-  long long tile_off[kTiles];     // element offset of each tile's (0, 0) in its output
-  int32_t tile_kb[kTiles];        // key block of each tile, or -1 for a zero tile
-  int32_t comp_tile[kTiles];      // compute slot -> tile index
-  uint64_t ld_full;
-  uint64_t mma_done[2];
-  uint64_t tmem_free[2];
-  uint64_t mma_all;
+  uint8_t q[2][kTileBytes];     // Q block ring (SW128)
+  uint8_t k[2][2][kTileBytes];  // K ring: each slot holds the two key tiles of one MMA group (M = 128)
+  float nlse2[kBlock];          // -lse * log2(e) of the current unit's 64 rows (weight warps)
+  UnitInfo info[2];
+  uint64_t info_full[2], info_empty[2];
+  uint64_t q_full[2], q_empty[2];
+  uint64_t k_full[2], k_empty[2];
+  uint64_t mma_done[2], tmem_free[2];
   uint32_t tmem_base;
-  int32_t n_tiles, n_comp, ld, bh, qblk, band;
   int32_t abort_flag;
 };
+
+__device__ __forceinline__ bool aborted(const Smem& sm) {
+  return *reinterpret_cast<const volatile int32_t*>(&sm.abort_flag) != 0;
+}
+
+__device__ __forceinline__ void set_abort(Smem& sm, const ProbsParams& p) {
+  atomicOr(p.status, kStatusTimeout);
+  *reinterpret_cast<volatile int32_t*>(&sm.abort_flag) = 1;
+}
 
 // Sorted distinct key blocks of band row i (1 <= i <= nb-2) of head h: the
 // two global blocks, the window and the row's random blocks. Out-of-range
 // random entries are skipped and reported in the status word.
 __device__ int band_list(const ProbsParams& p, int h, int i, int32_t* lst) {
+  int32_t ra[kMaxR];
+  const int32_t* src = p.rand_attn + (static_cast<long long>(h) * (p.nb - 2) + (i - 1)) * p.r;
+#pragma unroll
+  for (int t = 0; t < kMaxR; ++t) ra[t] = t < p.r ? src[t] : 0;  // independent loads, issued together
   int n = 0;
   auto add = [&](int x) {
     int pos = 0;
@@ -115,7 +143,6 @@ __device__ int band_list(const ProbsParams& p, int h, int i, int32_t* lst) {
   add(i - 1);
   add(i);
   add(i + 1);
-  const int32_t* ra = p.rand_attn + (static_cast<long long>(h) * (p.nb - 2) + (i - 1)) * p.r;
   for (int t = 0; t < p.r; ++t) {
     const int x = ra[t];
     if (x < 0 || x >= p.nb) {
@@ -127,8 +154,8 @@ __device__ int band_list(const ProbsParams& p, int h, int i, int32_t* lst) {
   return n;
 }
 
-// Decode unit `unit` into its query block, tiles, output offsets (one thread).
-__device__ void plan_unit(const ProbsParams& p, Smem& sm, int unit) {
+// Decode unit `unit` into its query block, tiles and output offsets (one thread).
+__device__ void plan_unit(const ProbsParams& p, UnitInfo& in, int unit) {
   const int bh = unit / p.units_per_head;
   int w = unit - bh * p.units_per_head;
   const int h = bh % p.H;
@@ -146,8 +173,8 @@ __device__ void plan_unit(const ProbsParams& p, Smem& sm, int unit) {
       const int kb = kb0 + t;
       bool listed = full;
       for (int e = 0; e < n && !listed; ++e) listed = lst[e] == kb;
-      sm.tile_kb[t] = listed ? kb : -1;
-      sm.tile_off[t] = (static_cast<long long>(bh) * L + static_cast<long long>(i) * kBlock) * L +
+      in.tile_kb[t] = listed ? kb : -1;
+      in.tile_off[t] = (static_cast<long long>(bh) * L + static_cast<long long>(i) * kBlock) * L +
                        static_cast<long long>(kb) * kBlock;
     }
   } else if (w < p.grows * p.ranges) {
@@ -158,8 +185,8 @@ __device__ void plan_unit(const ProbsParams& p, Smem& sm, int unit) {
     n_tiles = min(kTiles, p.nb - kb0);
     for (int t = 0; t < n_tiles; ++t) {
       const int kb = kb0 + t;
-      sm.tile_kb[t] = kb;
-      sm.tile_off[t] = (static_cast<long long>(bh) * p.grows + g) * kBlock * L + static_cast<long long>(kb) * kBlock;
+      in.tile_kb[t] = kb;
+      in.tile_off[t] = (static_cast<long long>(bh) * p.grows + g) * kBlock * L + static_cast<long long>(kb) * kBlock;
     }
   } else {
     w -= p.grows * p.ranges;
@@ -173,27 +200,73 @@ __device__ void plan_unit(const ProbsParams& p, Smem& sm, int unit) {
     band = 1;
     for (int t = 0; t < n_tiles; ++t) {
       const int s = s0 + t;
-      sm.tile_kb[t] = s < n ? lst[s] : -1;
-      sm.tile_off[t] =
+      in.tile_kb[t] = s < n ? lst[s] : -1;
+      in.tile_off[t] =
           ((static_cast<long long>(bh) * (p.nb - 2) + (i - 1)) * slots + s) * static_cast<long long>(kBlock * kBlock);
     }
   }
   int nc = 0;
   for (int t = 0; t < n_tiles; ++t)
-    if (sm.tile_kb[t] >= 0) sm.comp_tile[nc++] = t;
-  sm.n_tiles = n_tiles;
-  sm.n_comp = nc;
-  sm.ld = ld;
-  sm.bh = bh;
-  sm.qblk = i;
-  sm.band = band;
+    if (in.tile_kb[t] >= 0) in.comp_tile[nc++] = t;
+  in.n_tiles = n_tiles;
+  in.n_comp = nc;
+  in.ld = ld;
+  in.bh = bh;
+  in.qblk = i;
+  in.band = band;
 }
 
 __device__ __forceinline__ void epi_bar_sync() {
   asm volatile("bar.sync 1, %0;" ::"r"(kEpiThreads) : "memory");
 }
 
-__global__ void __launch_bounds__(kThreads, 3)
+// Named barrier of the weight threads that also ORs a predicate over them:
+// every thread gets the same answer.
+__device__ __forceinline__ bool epi_bar_or(bool x) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, 1, %2, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(x)), "r"(kEpiThreads)
+      : "memory");
+  return r != 0;
+}
+
+// p for one key and 32 query rows: x = s log2(e)/sqrt(d) + (bias2 - lse2[q]),
+// two rows per packed f32x2 operation; row q of the tile is LD elements
+// after row q-1 (LD = 0: the runtime stride ld).
+template <int LD, bool F32>
+__device__ __forceinline__ void emit32(const uint32_t (&v)[32], const float* nlse2, float bias2, float scale, void* dst,
+                                       long long ld) {
+  const uint64_t scale2 = f2_pack(scale, scale);
+  const uint64_t bias22 = f2_pack(bias2, bias2);
+  const long long stride = LD ? LD : ld;
+#pragma unroll
+  for (int c = 0; c < 32; c += 4) {
+    const float4 nl = *reinterpret_cast<const float4*>(nlse2 + c);
+    const uint64_t x01 = f2_fma(f2_pack(__uint_as_float(v[c]), __uint_as_float(v[c + 1])), scale2,
+                                f2_add(f2_pack(nl.x, nl.y), bias22));
+    const uint64_t x23 = f2_fma(f2_pack(__uint_as_float(v[c + 2]), __uint_as_float(v[c + 3])), scale2,
+                                f2_add(f2_pack(nl.z, nl.w), bias22));
+    float x[4];
+    f2_unpack(x01, x[0], x[1]);
+    f2_unpack(x23, x[2], x[3]);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float pr = ex2_approx(x[e]);
+      if (F32)
+        __stcs(reinterpret_cast<float*>(dst) + (c + e) * stride, pr);
+      else
+        __stcs(reinterpret_cast<unsigned short*>(dst) + (c + e) * stride,
+               __bfloat16_as_ushort(__float2bfloat16_rn(pr)));
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kThreads, kCtasPerSm)
 bigbird_probs_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const ProbsParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -202,19 +275,21 @@ bigbird_probs_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
   const int warp = tid >> 5;
   const int lane = tid & 31;
 
-  if (warp == kEpiWarps) {
-    if (lane == 0) {
-      mbar_init(smem_u32(&sm.ld_full), 1);
-      for (int b = 0; b < 2; ++b) {
-        mbar_init(smem_u32(&sm.mma_done[b]), 1);
-        mbar_init(smem_u32(&sm.tmem_free[b]), kEpiThreads);
-      }
-      mbar_init(smem_u32(&sm.mma_all), 1);
-      fence_barrier_init();
-      sm.abort_flag = 0;
-      plan_unit(p, sm, blockIdx.x);
+  if (warp == kProdWarp && lane == 0) {
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(smem_u32(&sm.info_full[b]), 1);
+      mbar_init(smem_u32(&sm.info_empty[b]), 2);  // the MMA thread and the weight warps
+      mbar_init(smem_u32(&sm.q_full[b]), 1);
+      mbar_init(smem_u32(&sm.q_empty[b]), 1);
+      mbar_init(smem_u32(&sm.k_full[b]), 1);
+      mbar_init(smem_u32(&sm.k_empty[b]), 1);
+      mbar_init(smem_u32(&sm.mma_done[b]), 1);
+      mbar_init(smem_u32(&sm.tmem_free[b]), kEpiThreads);
     }
-    __syncwarp();
+    fence_barrier_init();
+    sm.abort_flag = 0;
+  }
+  if (warp == kMmaWarp) {
     tmem_alloc(smem_u32(&sm.tmem_base), kTmemCols);
     tmem_relinquish();
     tc_fence_before();
@@ -222,124 +297,195 @@ bigbird_probs_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
-  const int nc = sm.n_comp;
-  const int ngroups = (nc + 1) / 2;
-  uint8_t* out = static_cast<uint8_t*>(sm.band ? p.out_band : p.out_rows);
-  const int esize = p.out_f32 ? 4 : 2;
+  const int u0 = blockIdx.x * p.units_per_cta;
+  const int u1 = min(p.total_units, u0 + p.units_per_cta);
 
-  if (warp == kEpiWarps) {
-    // ---------------------------------------------------------------- TMA + MMA
-    if (lane == 0 && nc > 0) {  // (a unit of zero tiles only loads nothing)
-      const uint32_t full = smem_u32(&sm.ld_full);
+  if (warp == kProdWarp) {
+    // ------------------------------------------------------------ plan + TMA
+    if (lane == 0) {
       const uint64_t keep = l2_policy_evict_last();
-      const int row0 = sm.bh * p.L;
-      mbar_arrive_expect_tx(full, static_cast<uint32_t>(1 + nc) * kTileBytes);
-      tma_load_2d(smem_u32(sm.q), &tmQ, full, 0, row0 + sm.qblk * kBlock, keep);
-      for (int s = 0; s < nc; ++s)
-        tma_load_2d(smem_u32(sm.k[s]), &tmK, full, 0, row0 + sm.tile_kb[sm.comp_tile[s]] * kBlock, keep);
-      int issued = 0;
-      if (!mbar_wait(full, 0)) {
-        atomicOr(p.status, kStatusTimeout);
-        *reinterpret_cast<volatile int32_t*>(&sm.abort_flag) = 1;
-        mbar_arrive(smem_u32(&sm.mma_done[0]));
-        mbar_arrive(smem_u32(&sm.mma_done[1]));
-      } else {
-        tc_fence_after();
-        const uint32_t idesc = idesc_f32acc(2 * kBlock, kBlock, true, false);  // bf16 K . Q^T, M = 128, N = 64
-        const uint32_t qa = smem_u32(sm.q);
-        for (int g = 0; g < ngroups; ++g) {
-          const int buf = g & 1;
-          if (g >= 2 && !mbar_wait(smem_u32(&sm.tmem_free[buf]), ((g - 2) >> 1) & 1)) {
-            atomicOr(p.status, kStatusTimeout);
-            *reinterpret_cast<volatile int32_t*>(&sm.abort_flag) = 1;
-            mbar_arrive(smem_u32(&sm.mma_done[buf]));
+      int iq = 0, gk = 0;  // Q blocks and K groups loaded so far
+      for (int iu = 0;; ++iu) {
+        const int u = u0 + iu;
+        const int s = iu & 1;
+        if (iu >= 2 && !mbar_wait(smem_u32(&sm.info_empty[s]), ((iu - 2) >> 1) & 1)) {
+          set_abort(sm, p);
+          break;
+        }
+        UnitInfo& in = sm.info[s];
+        if (u >= u1 || aborted(sm)) {
+          in.n_tiles = -1;
+          mbar_arrive(smem_u32(&sm.info_full[s]));
+          break;
+        }
+        plan_unit(p, in, u);
+        mbar_arrive(smem_u32(&sm.info_full[s]));  // release: the plan is visible to the waiting roles
+        const int nc = in.n_comp;
+        if (nc == 0) continue;  // zero tiles only: nothing to load
+        const int row0 = in.bh * p.L;
+        const int qs = iq & 1;
+        if (iq >= 2 && !mbar_wait(smem_u32(&sm.q_empty[qs]), ((iq - 2) >> 1) & 1)) {
+          set_abort(sm, p);
+          break;
+        }
+        mbar_arrive_expect_tx(smem_u32(&sm.q_full[qs]), kTileBytes);
+        tma_load_2d(smem_u32(sm.q[qs]), &tmQ, smem_u32(&sm.q_full[qs]), 0, row0 + in.qblk * kBlock, keep);
+        ++iq;
+        bool ok = true;
+        for (int g = 0; g < (nc + 1) / 2; ++g, ++gk) {
+          const int ks = gk & 1;
+          if (gk >= 2 && !mbar_wait(smem_u32(&sm.k_empty[ks]), ((gk - 2) >> 1) & 1)) {
+            ok = false;
             break;
           }
-          tc_fence_after();
-          const uint32_t ka = smem_u32(sm.k[2 * g]);
-#pragma unroll
-          for (int kk = 0; kk < kDim / 16; ++kk)
-            mma_ss(tmem + static_cast<uint32_t>(buf) * kBlock, sdesc_sw128(ka + kk * 32, 16, 1024),
-                   sdesc_sw128(qa + kk * 32, 16, 1024), idesc, kk > 0 ? 1u : 0u);
-          mma_commit(smem_u32(&sm.mma_done[buf]));
-          issued = 1;
+          const int nt = min(2, nc - 2 * g);
+          mbar_arrive_expect_tx(smem_u32(&sm.k_full[ks]), static_cast<uint32_t>(nt) * kTileBytes);
+          for (int t = 0; t < nt; ++t)
+            tma_load_2d(smem_u32(sm.k[ks][t]), &tmK, smem_u32(&sm.k_full[ks]), 0,
+                        row0 + in.tile_kb[in.comp_tile[2 * g + t]] * kBlock, keep);
+        }
+        if (!ok) {
+          set_abort(sm, p);
+          break;
         }
       }
-      if (issued) mma_commit(smem_u32(&sm.mma_all));
-      // Before TMEM is released: every MMA has completed, and no copy is left
-      // in flight (both bounded; only an earlier failure makes them wait).
-      if (issued && !mbar_wait(smem_u32(&sm.mma_all), 0)) atomicOr(p.status, kStatusTimeout);
-      if (!mbar_wait(full, 0)) atomicOr(p.status, kStatusTimeout);
+      // No copy may still be in flight when the CTA exits: wait (bounded) for
+      // the last loads of both rings.
+      for (int j = max(0, iq - 2); j < iq; ++j) mbar_wait(smem_u32(&sm.q_full[j & 1]), (j >> 1) & 1);
+      for (int j = max(0, gk - 2); j < gk; ++j) mbar_wait(smem_u32(&sm.k_full[j & 1]), (j >> 1) & 1);
+    }
+    __syncwarp();
+  } else if (warp == kMmaWarp) {
+    // ------------------------------------------------------------ MMA
+    if (lane == 0) {
+      const uint32_t idesc = idesc_f32acc(2 * kBlock, kBlock, true, false);  // bf16 K . Q^T, M = 128, N = 64
+      int iq = 0, gk = 0, gt = 0;  // Q blocks, K groups, TMEM groups consumed
+      bool issued = false;
+      for (int iu = 0;; ++iu) {
+        const int s = iu & 1;
+        if (!mbar_wait(smem_u32(&sm.info_full[s]), (iu >> 1) & 1)) {
+          set_abort(sm, p);
+          break;
+        }
+        const UnitInfo& in = sm.info[s];
+        if (in.n_tiles < 0) break;
+        const int nc = in.n_comp;
+        if (nc > 0) {
+          const int qs = iq & 1;
+          bool ok = mbar_wait(smem_u32(&sm.q_full[qs]), (iq >> 1) & 1);
+          for (int g = 0; ok && g < (nc + 1) / 2; ++g, ++gk, ++gt) {
+            const int ks = gk & 1;
+            const int buf = gt & 1;
+            ok = mbar_wait(smem_u32(&sm.k_full[ks]), (gk >> 1) & 1) &&
+                 (gt < 2 || mbar_wait(smem_u32(&sm.tmem_free[buf]), ((gt - 2) >> 1) & 1));
+            if (!ok) break;
+            tc_fence_after();
+            const uint32_t ka = smem_u32(sm.k[ks][0]);
+            const uint32_t qa = smem_u32(sm.q[qs]);
+#pragma unroll
+            for (int kk = 0; kk < kDim / 16; ++kk)
+              mma_ss(tmem + static_cast<uint32_t>(buf) * kBlock, sdesc_sw128(ka + kk * 32, 16, 1024),
+                     sdesc_sw128(qa + kk * 32, 16, 1024), idesc, kk > 0 ? 1u : 0u);
+            mma_commit(smem_u32(&sm.mma_done[buf]));
+            mma_commit(smem_u32(&sm.k_empty[ks]));
+            issued = true;
+          }
+          if (!ok) {
+            set_abort(sm, p);
+            break;
+          }
+          mma_commit(smem_u32(&sm.q_empty[qs]));
+          ++iq;
+        }
+        mbar_arrive(smem_u32(&sm.info_empty[s]));
+      }
+      // Every MMA has completed before TMEM is released (bounded).
+      if (issued && gt > 0) mbar_wait(smem_u32(&sm.mma_done[(gt - 1) & 1]), ((gt - 1) >> 1) & 1);
     }
     __syncwarp();
   } else {
-    // ---------------------------------------------------------------- weights
-    const int et = tid;  // 0 .. 255
-    if (et < kBlock)
-      sm.lse2[et] = p.lse[static_cast<long long>(sm.bh) * p.L + sm.qblk * kBlock + et] * kLog2e;
-    // Zero tiles, while the loads and MMAs run.
-    const int vec_per_row = kBlock * esize / 16;
-    for (int t = 0; t < sm.n_tiles; ++t) {
-      if (sm.tile_kb[t] >= 0) continue;
-      uint8_t* base = out + sm.tile_off[t] * esize;
-      for (int idx = et; idx < kBlock * vec_per_row; idx += kEpiThreads) {
-        const int row = idx / vec_per_row;
-        const int col = idx - row * vec_per_row;
-        __stcs(reinterpret_cast<uint4*>(base + (static_cast<long long>(row) * sm.ld) * esize) + col,
-               make_uint4(0u, 0u, 0u, 0u));
-      }
-    }
-    epi_bar_sync();  // lse2 visible to every weight thread
-
-    const int quad = warp & 3;                 // TMEM lanes 32 quad .. 32 quad + 31
-    const int half = warp >> 2;                // query columns 32 half .. 32 half + 31
-    const int m = 32 * quad + lane;            // key row of the 128-key pair
-    const int b = sm.bh / p.H;
-    const long long ld = sm.ld;
-    for (int g = 0; g < ngroups; ++g) {
-      const int buf = g & 1;
-      const bool ok = mbar_wait(smem_u32(&sm.mma_done[buf]), (g >> 1) & 1);
-      if (!__all_sync(0xffffffffu, ok)) {
-        if (lane == 0) atomicOr(p.status, kStatusTimeout);
-        *reinterpret_cast<volatile int32_t*>(&sm.abort_flag) = 1;
-        break;
-      }
-      if (__any_sync(0xffffffffu, *reinterpret_cast<volatile int32_t*>(&sm.abort_flag) != 0)) break;
-      tc_fence_after();
-      uint32_t v[32];
-      tmem_ld32(tmem + (static_cast<uint32_t>(32 * quad) << 16) + static_cast<uint32_t>(buf * kBlock + 32 * half), v);
-      tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive(smem_u32(&sm.tmem_free[buf]));
-      const int cs = 2 * g + (m >> 6);
-      if (cs < nc) {
-        const int ti = sm.comp_tile[cs];
-        const int kb = sm.tile_kb[ti];
-        const int kk = m & (kBlock - 1);
-        const bool masked = p.seq_mask && !p.seq_mask[static_cast<long long>(b) * p.L + kb * kBlock + kk];
-        const float braw = masked ? p.bias_raw : 0.0f;
-        const long long base = sm.tile_off[ti] + kk + static_cast<long long>(32 * half) * ld;
-        if (p.out_f32) {
-          float* o = reinterpret_cast<float*>(out) + base;
+    // ------------------------------------------------------------ weights
+    // Every decision to leave the unit loop is taken jointly by the 256
+    // weight threads (bar.red.or), so they always meet at the same named
+    // barriers; a failed wait only skips work after that point.
+    const int et = tid;                 // 0 .. 255
+    const int quad = warp & 3;          // TMEM lanes 32 quad .. 32 quad + 31
+    const int half = warp >> 2;         // query columns 32 half .. 32 half + 31
+    const int m = 32 * quad + lane;     // key row of a 128-key MMA group
+    const int kk = m & (kBlock - 1);
+    const int esize = p.out_f32 ? 4 : 2;
+    int gt = 0;
+    for (int iu = 0;; ++iu) {
+      const int s = iu & 1;
+      const bool ok = !aborted(sm) && mbar_wait(smem_u32(&sm.info_full[s]), (iu >> 1) & 1);
+      if (!ok && !aborted(sm)) set_abort(sm, p);
+      const UnitInfo& in = sm.info[s];
+      const bool leave = epi_bar_or(!ok || in.n_tiles < 0);  // also: every thread is done with the previous unit
+      if (iu >= 1 && et == 0) mbar_arrive(smem_u32(&sm.info_empty[s ^ 1]));
+      if (leave) break;
+      const int nc = in.n_comp;
+      const int ngroups = (nc + 1) / 2;
+      uint8_t* out = static_cast<uint8_t*>(in.band ? p.out_band : p.out_rows);
+      const long long ld = in.ld;
+      if (et < kBlock) sm.nlse2[et] = -p.lse[static_cast<long long>(in.bh) * p.L + in.qblk * kBlock + et] * kLog2e;
+      // which of this thread's keys (one per group) are padded; loads issued before any wait
+      uint32_t masked = 0;
+      if (p.seq_mask) {
+        const uint8_t* sm_row = p.seq_mask + static_cast<long long>(in.bh / p.H) * p.L + kk;
 #pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            const float x = fmaf(__uint_as_float(v[c]) + braw, p.scale_log2, -sm.lse2[32 * half + c]);
-            __stcs(o + c * ld, ex2_approx(x));
+        for (int g = 0; g < kTiles / 2; ++g) {
+          const int cs = 2 * g + (m >> 6);
+          if (cs < nc && !sm_row[in.tile_kb[in.comp_tile[cs]] * kBlock]) masked |= 1u << g;
+        }
+      }
+      // zero tiles
+      const int vec_per_row = kBlock * esize / 16;
+      for (int t = 0; t < in.n_tiles; ++t) {
+        if (in.tile_kb[t] >= 0) continue;
+        uint8_t* base = out + in.tile_off[t] * esize;
+        for (int idx = et; idx < kBlock * vec_per_row; idx += kEpiThreads) {
+          const int row = idx / vec_per_row;
+          const int col = idx - row * vec_per_row;
+          __stcs(reinterpret_cast<uint4*>(base + (static_cast<long long>(row) * ld) * esize) + col,
+                 make_uint4(0u, 0u, 0u, 0u));
+        }
+      }
+      epi_bar_sync();  // nlse2 visible
+      for (int g = 0; g < ngroups; ++g, ++gt) {
+        const int buf = gt & 1;
+        const bool okw = !aborted(sm) && mbar_wait(smem_u32(&sm.mma_done[buf]), (gt >> 1) & 1);
+        if (__all_sync(0xffffffffu, okw)) {
+          tc_fence_after();
+          uint32_t v[32];
+          tmem_ld32(tmem + (static_cast<uint32_t>(32 * quad) << 16) + static_cast<uint32_t>(buf * kBlock + 32 * half),
+                    v);
+          tmem_wait_ld();
+          tc_fence_before();
+          mbar_arrive(smem_u32(&sm.tmem_free[buf]));
+          const int cs = 2 * g + (m >> 6);
+          if (cs < nc) {
+            const int ti = in.comp_tile[cs];
+            uint8_t* dst = out + (in.tile_off[ti] + kk + static_cast<long long>(32 * half) * ld) * esize;
+            const float* nl = sm.nlse2 + 32 * half;
+            const float bias2 = (masked >> g) & 1u ? p.bias_log2 : 0.0f;
+            if (in.band) {
+              if (p.out_f32) emit32<kBlock, true>(v, nl, bias2, p.scale_log2, dst, ld);
+              else emit32<kBlock, false>(v, nl, bias2, p.scale_log2, dst, ld);
+            } else {
+              if (p.out_f32) emit32<0, true>(v, nl, bias2, p.scale_log2, dst, ld);
+              else emit32<0, false>(v, nl, bias2, p.scale_log2, dst, ld);
+            }
           }
         } else {
-          unsigned short* o = reinterpret_cast<unsigned short*>(out) + base;
-#pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            const float x = fmaf(__uint_as_float(v[c]) + braw, p.scale_log2, -sm.lse2[32 * half + c]);
-            __stcs(o + c * ld, __bfloat16_as_ushort(__float2bfloat16_rn(ex2_approx(x))));
-          }
+          if (!aborted(sm)) set_abort(sm, p);
+          mbar_arrive(smem_u32(&sm.tmem_free[buf]));
         }
       }
     }
   }
 
   __syncthreads();
-  if (warp == kEpiWarps) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
@@ -416,18 +562,25 @@ static int probs_impl(const void* q, const void* k, const float* lse, const int3
   p.chunks = chunks;
   p.grows = lo.grows;
   p.units_per_head = static_cast<int>(per_head);
+  p.total_units = static_cast<int>(units);
   p.scale_log2 = kLog2e / sqrtf(static_cast<float>(d));
-  p.bias_raw = -10000.0f * sqrtf(static_cast<float>(d));
+  p.bias_log2 = -10000.0f * kLog2e;
+  // Persistent grid: kCtasPerSm CTAs per SM at most, each taking an equal
+  // run of consecutive units (neighbouring units share K tiles in L2).
+  int sms = 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0) return BB_ERR_CUDA;
+  const int64_t slots = static_cast<int64_t>(kCtasPerSm) * sms;
+  p.units_per_cta = static_cast<int>((units + slots - 1) / slots);
+  const int grid = static_cast<int>((units + p.units_per_cta - 1) / p.units_per_cta);
 
   const int smem = static_cast<int>(sizeof(Smem) + 1024);
   // (set on every call: the attribute is per device and the call is cheap)
   if (cudaFuncSetAttribute(bigbird_probs_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return BB_ERR_CUDA;
-  // Three CTAs (74 KB each) per SM need the largest shared-memory carve-out.
+  // Three CTAs per SM need a large shared-memory carve-out.
   if (cudaFuncSetAttribute(bigbird_probs_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100) != cudaSuccess)
     return BB_ERR_CUDA;
-  bigbird_probs_kernel<<<static_cast<unsigned>(units), kThreads, smem, static_cast<cudaStream_t>(stream_)>>>(tq, tk,
-                                                                                                            p);
+  bigbird_probs_kernel<<<grid, kThreads, smem, static_cast<cudaStream_t>(stream_)>>>(tq, tk, p);
   return cudaGetLastError() == cudaSuccess ? BB_OK : BB_ERR_CUDA;
 }
 
