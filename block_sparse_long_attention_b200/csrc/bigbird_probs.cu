@@ -63,6 +63,8 @@ constexpr int kProdWarp = kEpiWarps;        // planning + TMA
 constexpr int kMmaWarp = kEpiWarps + 1;     // TMEM + MMA
 constexpr int kThreads = kEpiThreads + 64;
 constexpr int kCtasPerSm = 3;
+constexpr int kKSlots = 2;                  // K ring depth (MMA groups of two key tiles)
+constexpr int kLdCols = 32;                 // TMEM columns a weight thread reads at a time
 constexpr int kMaxR = 16;
 constexpr uint32_t kTileBytes = kBlock * kDim * 2;
 constexpr uint32_t kTmemCols = 128;         // two 64-column S^T buffers
@@ -101,12 +103,12 @@ struct UnitInfo {
 
 struct __align__(1024) Smem {
   uint8_t q[2][kTileBytes];     // Q block ring (SW128)
-  uint8_t k[2][2][kTileBytes];  // K ring: each slot holds the two key tiles of one MMA group (M = 128)
+  uint8_t k[kKSlots][2][kTileBytes];  // K ring: each slot holds the two key tiles of one MMA group (M = 128)
   float nlse2[kBlock];          // -lse * log2(e) of the current unit's 64 rows (weight warps)
   UnitInfo info[2];
   uint64_t info_full[2], info_empty[2];
   uint64_t q_full[2], q_empty[2];
-  uint64_t k_full[2], k_empty[2];
+  uint64_t k_full[kKSlots], k_empty[kKSlots];
   uint64_t mma_done[2], tmem_free[2];
   uint32_t tmem_base;
   int32_t abort_flag;
@@ -235,17 +237,20 @@ __device__ __forceinline__ bool epi_bar_or(bool x) {
   return r != 0;
 }
 
-// p for one key and 32 query rows: x = s log2(e)/sqrt(d) + (bias2 - lse2[q]),
+__device__ __forceinline__ void tmem_ld_cols(uint32_t a, uint32_t (&r)[32]) { tmem_ld32(a, r); }
+__device__ __forceinline__ void tmem_ld_cols(uint32_t a, uint32_t (&r)[16]) { tmem_ld16(a, r); }
+
+// p for one key and N query rows: x = s log2(e)/sqrt(d) + (bias2 - lse2[q]),
 // two rows per packed f32x2 operation; row q of the tile is LD elements
 // after row q-1 (LD = 0: the runtime stride ld).
-template <int LD, bool F32>
-__device__ __forceinline__ void emit32(const uint32_t (&v)[32], const float* nlse2, float bias2, float scale, void* dst,
-                                       long long ld) {
+template <int N, int LD, bool F32>
+__device__ __forceinline__ void emit(const uint32_t (&v)[N], const float* nlse2, float bias2, float scale, void* dst,
+                                     long long ld) {
   const uint64_t scale2 = f2_pack(scale, scale);
   const uint64_t bias22 = f2_pack(bias2, bias2);
   const long long stride = LD ? LD : ld;
 #pragma unroll
-  for (int c = 0; c < 32; c += 4) {
+  for (int c = 0; c < N; c += 4) {
     const float4 nl = *reinterpret_cast<const float4*>(nlse2 + c);
     const uint64_t x01 = f2_fma(f2_pack(__uint_as_float(v[c]), __uint_as_float(v[c + 1])), scale2,
                                 f2_add(f2_pack(nl.x, nl.y), bias22));
@@ -281,10 +286,12 @@ bigbird_probs_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
       mbar_init(smem_u32(&sm.info_empty[b]), 2);  // the MMA thread and the weight warps
       mbar_init(smem_u32(&sm.q_full[b]), 1);
       mbar_init(smem_u32(&sm.q_empty[b]), 1);
-      mbar_init(smem_u32(&sm.k_full[b]), 1);
-      mbar_init(smem_u32(&sm.k_empty[b]), 1);
       mbar_init(smem_u32(&sm.mma_done[b]), 1);
       mbar_init(smem_u32(&sm.tmem_free[b]), kEpiThreads);
+    }
+    for (int b = 0; b < kKSlots; ++b) {
+      mbar_init(smem_u32(&sm.k_full[b]), 1);
+      mbar_init(smem_u32(&sm.k_empty[b]), 1);
     }
     fence_barrier_init();
     sm.abort_flag = 0;
@@ -333,8 +340,8 @@ bigbird_probs_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
         ++iq;
         bool ok = true;
         for (int g = 0; g < (nc + 1) / 2; ++g, ++gk) {
-          const int ks = gk & 1;
-          if (gk >= 2 && !mbar_wait(smem_u32(&sm.k_empty[ks]), ((gk - 2) >> 1) & 1)) {
+          const int ks = gk % kKSlots;
+          if (gk >= kKSlots && !mbar_wait(smem_u32(&sm.k_empty[ks]), (gk / kKSlots - 1) & 1)) {
             ok = false;
             break;
           }
@@ -352,7 +359,7 @@ bigbird_probs_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
       // No copy may still be in flight when the CTA exits: wait (bounded) for
       // the last loads of both rings.
       for (int j = max(0, iq - 2); j < iq; ++j) mbar_wait(smem_u32(&sm.q_full[j & 1]), (j >> 1) & 1);
-      for (int j = max(0, gk - 2); j < gk; ++j) mbar_wait(smem_u32(&sm.k_full[j & 1]), (j >> 1) & 1);
+      for (int j = max(0, gk - kKSlots); j < gk; ++j) mbar_wait(smem_u32(&sm.k_full[j % kKSlots]), (j / kKSlots) & 1);
     }
     __syncwarp();
   } else if (warp == kMmaWarp) {
@@ -374,9 +381,9 @@ bigbird_probs_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
           const int qs = iq & 1;
           bool ok = mbar_wait(smem_u32(&sm.q_full[qs]), (iq >> 1) & 1);
           for (int g = 0; ok && g < (nc + 1) / 2; ++g, ++gk, ++gt) {
-            const int ks = gk & 1;
+            const int ks = gk % kKSlots;
             const int buf = gt & 1;
-            ok = mbar_wait(smem_u32(&sm.k_full[ks]), (gk >> 1) & 1) &&
+            ok = mbar_wait(smem_u32(&sm.k_full[ks]), (gk / kKSlots) & 1) &&
                  (gt < 2 || mbar_wait(smem_u32(&sm.tmem_free[buf]), ((gt - 2) >> 1) & 1));
             if (!ok) break;
             tc_fence_after();
@@ -456,24 +463,30 @@ bigbird_probs_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
         const bool okw = !aborted(sm) && mbar_wait(smem_u32(&sm.mma_done[buf]), (gt >> 1) & 1);
         if (__all_sync(0xffffffffu, okw)) {
           tc_fence_after();
-          uint32_t v[32];
-          tmem_ld32(tmem + (static_cast<uint32_t>(32 * quad) << 16) + static_cast<uint32_t>(buf * kBlock + 32 * half),
-                    v);
-          tmem_wait_ld();
-          tc_fence_before();
-          mbar_arrive(smem_u32(&sm.tmem_free[buf]));
           const int cs = 2 * g + (m >> 6);
-          if (cs < nc) {
-            const int ti = in.comp_tile[cs];
-            uint8_t* dst = out + (in.tile_off[ti] + kk + static_cast<long long>(32 * half) * ld) * esize;
-            const float* nl = sm.nlse2 + 32 * half;
-            const float bias2 = (masked >> g) & 1u ? p.bias_log2 : 0.0f;
-            if (in.band) {
-              if (p.out_f32) emit32<kBlock, true>(v, nl, bias2, p.scale_log2, dst, ld);
-              else emit32<kBlock, false>(v, nl, bias2, p.scale_log2, dst, ld);
-            } else {
-              if (p.out_f32) emit32<0, true>(v, nl, bias2, p.scale_log2, dst, ld);
-              else emit32<0, false>(v, nl, bias2, p.scale_log2, dst, ld);
+          const bool act = cs < nc;
+          const long long off = act ? in.tile_off[in.comp_tile[cs]] : 0;
+          const float bias2 = (masked >> g) & 1u ? p.bias_log2 : 0.0f;
+#pragma unroll
+          for (int c0 = 0; c0 < 32; c0 += kLdCols) {
+            uint32_t v[kLdCols];
+            tmem_ld_cols(tmem + (static_cast<uint32_t>(32 * quad) << 16) +
+                             static_cast<uint32_t>(buf * kBlock + 32 * half + c0), v);
+            tmem_wait_ld();
+            if (c0 + kLdCols == 32) {  // the buffer is fully read: the next MMA may overwrite it
+              tc_fence_before();
+              mbar_arrive(smem_u32(&sm.tmem_free[buf]));
+            }
+            if (act) {
+              uint8_t* dst = out + (off + kk + static_cast<long long>(32 * half + c0) * ld) * esize;
+              const float* nl = sm.nlse2 + 32 * half + c0;
+              if (in.band) {
+                if (p.out_f32) emit<kLdCols, kBlock, true>(v, nl, bias2, p.scale_log2, dst, ld);
+                else emit<kLdCols, kBlock, false>(v, nl, bias2, p.scale_log2, dst, ld);
+              } else {
+                if (p.out_f32) emit<kLdCols, 0, true>(v, nl, bias2, p.scale_log2, dst, ld);
+                else emit<kLdCols, 0, false>(v, nl, bias2, p.scale_log2, dst, ld);
+              }
             }
           }
         } else {
