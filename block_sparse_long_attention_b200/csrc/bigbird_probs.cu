@@ -22,7 +22,7 @@
 // A unit is one query block against up to 8 key-block tiles: a range of 8
 // blocks of a full row, a row's band list (packed), or a range of 8 blocks of
 // any row with its unlisted tiles zero (dense). The kernel is persistent
-// (three CTAs of 320 threads per SM, units dealt out evenly) and
+// (four CTAs of 320 threads per SM, units dealt out evenly) and
 // warp-specialised, so one unit's setup, loads and MMAs overlap the previous
 // unit's stores:
 //   warp 8     plans each unit (its tiles and output offsets; the band list
@@ -33,8 +33,8 @@
 //              tcgen05 128x64x16 steps) into one of two 64-column TMEM
 //              buffers;
 //   warps 0-7  thread (warp w, lane l) reads TMEM lane 32 (w % 4) + l (one
-//              key) and the 32 query columns of half w / 4, and writes p for
-//              them. Consecutive lanes hold consecutive keys, so each store
+//              key) and the 32 query columns of half w / 4, 16 at a time,
+//              and writes p for them. Consecutive lanes hold consecutive keys, so each store
 //              instruction of a warp covers 32 consecutive elements of one
 //              output row (128 bytes in fp32) with no shuffle. Zero tiles are
 //              written with 16-byte stores.
@@ -62,9 +62,9 @@ constexpr int kEpiThreads = kEpiWarps * 32;
 constexpr int kProdWarp = kEpiWarps;        // planning + TMA
 constexpr int kMmaWarp = kEpiWarps + 1;     // TMEM + MMA
 constexpr int kThreads = kEpiThreads + 64;
-constexpr int kCtasPerSm = 3;
+constexpr int kCtasPerSm = 4;
 constexpr int kKSlots = 2;                  // K ring depth (MMA groups of two key tiles)
-constexpr int kLdCols = 32;                 // TMEM columns a weight thread reads at a time
+constexpr int kLdCols = 16;                 // TMEM columns a weight thread reads at a time (keeps 4 CTAs within 48 registers)
 constexpr int kMaxR = 16;
 constexpr uint32_t kTileBytes = kBlock * kDim * 2;
 constexpr uint32_t kTmemCols = 128;         // two 64-column S^T buffers
@@ -590,7 +590,7 @@ static int probs_impl(const void* q, const void* k, const float* lse, const int3
   // (set on every call: the attribute is per device and the call is cheap)
   if (cudaFuncSetAttribute(bigbird_probs_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return BB_ERR_CUDA;
-  // Three CTAs per SM need a large shared-memory carve-out.
+  // Four CTAs (51 KB each) per SM need a large shared-memory carve-out.
   if (cudaFuncSetAttribute(bigbird_probs_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100) != cudaSuccess)
     return BB_ERR_CUDA;
   bigbird_probs_kernel<<<grid, kThreads, smem, static_cast<cudaStream_t>(stream_)>>>(tq, tk, p);
