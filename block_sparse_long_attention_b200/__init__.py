@@ -1,10 +1,12 @@
-"""BigBird ITC block-sparse attention forward on B200 (sm_100a).
+"""BigBird ITC block-sparse attention on B200 (sm_100a): forward (fwd,
+fwd_train), backward (bwd) and the attention-probability export (probs,
+probs_dense).
 
 Thin Python binding over the C ABI of ``libbigbird_attn.so`` (declared in
-``include/bigbird_attn.h``): argument marshalling only. Every step of the
-forward pass runs in the library's CUDA kernels; PyTorch supplies device
-memory and the current stream. There is no CPU fallback: if the library is
-missing or no sm_100 device is present the calls raise.
+``include/bigbird_attn.h``): argument marshalling only. Every step runs in
+the library's CUDA kernels; PyTorch supplies device memory and the current
+stream. There is no CPU fallback: if the library is missing or no sm_100
+device is present the calls raise.
 """
 
 from __future__ import annotations

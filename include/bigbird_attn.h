@@ -1,6 +1,7 @@
 /*
  * bigbird_attn.h -- C ABI of the B200 (sm_100a) BigBird ITC block-sparse
- * attention forward pass and its host-side preparation routines.
+ * attention: the forward pass, its host-side preparation routines, the
+ * backward pass and the attention-probability export.
  *
  * Pages cited below:
  *   [TFG-BigBird] "models 仓库中的 BigBird：线性复杂度稀疏注意力与长序列训练的完整实践"
