@@ -499,11 +499,10 @@ def run_probs(args):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32 (bf16 inputs)",
         "data": "synthetic", "pass": "probs",
         "config": _config(w, 1, "L2 flushed (2x L2 write) before every timed step"),
-        # DRAM bytes (read + write) of one fp32 bigbird_probs_kernel launch on
-        # the default workload, from the ncu capture summarised in
-        # profiles/bigbird_probs_l4096_b4h12.md; valid for that kernel source only.
+        # traffic: null -- the kernel changed (warp-parallel unit planning) after
+        # the ncu capture summarised in profiles/bigbird_probs_l4096_b4h12.md.
         "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s", "frac": gbs / peak,
-                     "traffic": 492.98e6 if w.name == DEFAULT_WORKLOAD else None, "kernel": "bigbird_probs_kernel",
+                     "traffic": None, "kernel": "bigbird_probs_kernel",
                      "algorithmic_bytes": out_bytes + in_bytes,
                      "peak_source": f"{src} HBM copy bandwidth"},
         "pairs_per_s": pairs / (ms * 1e-3),

@@ -25,8 +25,9 @@
 // (four CTAs of 320 threads per SM, units dealt out evenly) and
 // warp-specialised, so one unit's setup, loads and MMAs overlap the previous
 // unit's stores:
-//   warp 8     plans each unit (its tiles and output offsets; the band list
-//              from rand_attn) into a 2-slot ring, and loads the Q block and
+//   warp 8     plans each unit with all 32 lanes (its tiles and output
+//              offsets; the band list from rand_attn, sorted and deduplicated
+//              with shuffles) into a 2-slot ring, and loads the Q block and
 //              the listed K tiles by TMA into 2-deep rings;
 //   warp 9     TMEM allocation and the MMAs: scores transposed, S^T = K Q^T,
 //              two key tiles at a time (M = 128 keys, N = 64 queries, four
@@ -123,99 +124,113 @@ __device__ __forceinline__ void set_abort(Smem& sm, const ProbsParams& p) {
   *reinterpret_cast<volatile int32_t*>(&sm.abort_flag) = 1;
 }
 
-// Sorted distinct key blocks of band row i (1 <= i <= nb-2) of head h: the
-// two global blocks, the window and the row's random blocks. Out-of-range
-// random entries are skipped and reported in the status word.
-__device__ int band_list(const ProbsParams& p, int h, int i, int32_t* lst) {
-  int32_t ra[kMaxR];
-  const int32_t* src = p.rand_attn + (static_cast<long long>(h) * (p.nb - 2) + (i - 1)) * p.r;
-#pragma unroll
-  for (int t = 0; t < kMaxR; ++t) ra[t] = t < p.r ? src[t] : 0;  // independent loads, issued together
-  int n = 0;
-  auto add = [&](int x) {
-    int pos = 0;
-    while (pos < n && lst[pos] < x) ++pos;
-    if (pos < n && lst[pos] == x) return;
-    for (int t = n; t > pos; --t) lst[t] = lst[t - 1];
-    lst[pos] = x;
-    ++n;
-  };
-  add(0);
-  add(p.nb - 1);
-  add(i - 1);
-  add(i);
-  add(i + 1);
-  for (int t = 0; t < p.r; ++t) {
-    const int x = ra[t];
-    if (x < 0 || x >= p.nb) {
-      atomicOr(p.status, kStatusBadRandAttn);
-      continue;
-    }
-    add(x);
-  }
-  return n;
-}
-
-// Decode unit `unit` into its query block, tiles and output offsets (one thread).
-__device__ void plan_unit(const ProbsParams& p, UnitInfo& in, int unit) {
+// Plan of unit `unit`, computed by all 32 lanes of the calling warp with
+// registers and shuffles only: its query block, tiles and output offsets.
+// The key blocks of a band row i (1 <= i <= nb-2) of head h are the set
+// {0, nb-1, i-1, i, i+1} and the row's random blocks, in ascending order:
+// lane c holds candidate c (lanes 5 .. 4+r load rand_attn[h][i-1][c-5]), a
+// candidate equal to one on a lower lane is a duplicate, and a distinct
+// candidate's slot is the number of distinct candidates below it.
+// Out-of-range random entries are skipped and reported in the status word.
+__device__ void plan_unit_warp(const ProbsParams& p, UnitInfo& in, int unit, int lane) {
+  constexpr unsigned kFull = 0xffffffffu;
+  constexpr int kNone = 0x7fffffff;
   const int bh = unit / p.units_per_head;
   int w = unit - bh * p.units_per_head;
   const int h = bh % p.H;
   const long long L = p.L;
-  int i = 0, n_tiles = 0, ld = p.L, band = 0;
-  int32_t lst[5 + kMaxR];
+  int i, g = 0, kb0 = 0, s0 = 0, n_tiles, ld = p.L, band = 0;
+  bool full;
   if (p.dense) {
     i = w / p.ranges;
-    const int j = w - i * p.ranges;
-    const bool full = !p.sparse || i == 0 || i == p.nb - 1;
-    const int n = full ? 0 : band_list(p, h, i, lst);
-    const int kb0 = j * kTiles;
+    kb0 = (w - i * p.ranges) * kTiles;
+    full = !p.sparse || i == 0 || i == p.nb - 1;
     n_tiles = min(kTiles, p.nb - kb0);
-    for (int t = 0; t < n_tiles; ++t) {
-      const int kb = kb0 + t;
-      bool listed = full;
-      for (int e = 0; e < n && !listed; ++e) listed = lst[e] == kb;
-      in.tile_kb[t] = listed ? kb : -1;
-      in.tile_off[t] = (static_cast<long long>(bh) * L + static_cast<long long>(i) * kBlock) * L +
-                       static_cast<long long>(kb) * kBlock;
-    }
   } else if (w < p.grows * p.ranges) {
-    const int g = w / p.ranges;
-    const int j = w - g * p.ranges;
+    g = w / p.ranges;
+    kb0 = (w - g * p.ranges) * kTiles;
     i = p.sparse ? (g == 0 ? 0 : p.nb - 1) : g;
-    const int kb0 = j * kTiles;
+    full = true;
     n_tiles = min(kTiles, p.nb - kb0);
-    for (int t = 0; t < n_tiles; ++t) {
-      const int kb = kb0 + t;
-      in.tile_kb[t] = kb;
-      in.tile_off[t] = (static_cast<long long>(bh) * p.grows + g) * kBlock * L + static_cast<long long>(kb) * kBlock;
-    }
   } else {
     w -= p.grows * p.ranges;
     i = 1 + w / p.chunks;
-    const int c = w - (i - 1) * p.chunks;
-    const int slots = 5 + p.r;
-    const int n = band_list(p, h, i, lst);
-    const int s0 = c * kTiles;
-    n_tiles = min(kTiles, slots - s0);
+    s0 = (w - (i - 1) * p.chunks) * kTiles;
+    full = false;
+    n_tiles = min(kTiles, 5 + p.r - s0);
     ld = kBlock;
     band = 1;
-    for (int t = 0; t < n_tiles; ++t) {
-      const int s = s0 + t;
-      in.tile_kb[t] = s < n ? lst[s] : -1;
-      in.tile_off[t] =
-          ((static_cast<long long>(bh) * (p.nb - 2) + (i - 1)) * slots + s) * static_cast<long long>(kBlock * kBlock);
+  }
+  // band rows: distinct candidates, their slots, and how many there are
+  int cand = kNone;
+  bool valid = false;
+  int rank = 0;
+  if (!full) {
+    if (lane < 5) {
+      cand = lane == 0 ? 0 : lane == 1 ? p.nb - 1 : i - 3 + lane;  // lanes 2, 3, 4: i-1, i, i+1
+    } else if (lane < 5 + p.r) {
+      const int x = p.rand_attn[(static_cast<long long>(h) * (p.nb - 2) + (i - 1)) * p.r + (lane - 5)];
+      if (x >= 0 && x < p.nb) cand = x;
+      else atomicOr(p.status, kStatusBadRandAttn);
+    }
+    bool dup = false;
+    for (int o = 0; o < 5 + kMaxR; ++o) {
+      const int v = __shfl_sync(kFull, cand, o);
+      dup |= (o < lane && v == cand);
+    }
+    valid = cand != kNone && !dup;
+    for (int o = 0; o < 5 + kMaxR; ++o) {
+      const int v = __shfl_sync(kFull, cand, o);
+      const bool vo = __shfl_sync(kFull, valid ? 1 : 0, o) != 0;
+      rank += (vo && v < cand) ? 1 : 0;
     }
   }
-  int nc = 0;
-  for (int t = 0; t < n_tiles; ++t)
-    if (in.tile_kb[t] >= 0) in.comp_tile[nc++] = t;
-  in.n_tiles = n_tiles;
-  in.n_comp = nc;
-  in.ld = ld;
-  in.bh = bh;
-  in.qblk = i;
-  in.band = band;
+  // tile t is lane t's: key block (or -1: a zero tile) and output offset
+  int kb = -1;
+  long long off = 0;
+  if (lane < n_tiles) {
+    if (p.dense) {
+      kb = kb0 + lane;
+      off = (static_cast<long long>(bh) * L + static_cast<long long>(i) * kBlock) * L + static_cast<long long>(kb) * kBlock;
+    } else if (!band) {
+      kb = kb0 + lane;
+      off = (static_cast<long long>(bh) * p.grows + g) * kBlock * L + static_cast<long long>(kb) * kBlock;
+    } else {
+      off = ((static_cast<long long>(bh) * (p.nb - 2) + (i - 1)) * (5 + p.r) + s0 + lane) *
+            static_cast<long long>(kBlock * kBlock);
+    }
+  }
+  if (!full) {
+    if (band) {
+      // slot s0 + t holds the candidate of rank s0 + t
+      for (int t = 0; t < kTiles; ++t) {
+        const unsigned owner = __ballot_sync(kFull, valid && rank == s0 + t);
+        const int v = __shfl_sync(kFull, cand, owner ? __ffs(owner) - 1 : 0);
+        if (lane == t) kb = owner ? v : -1;
+      }
+    } else {
+      // dense layout: block kb0 + t is computed only if it is in the row's set
+      const unsigned hit = __reduce_or_sync(
+          kFull, (valid && cand >= kb0 && cand < kb0 + n_tiles) ? (1u << (cand - kb0)) : 0u);
+      if (lane < n_tiles && !((hit >> lane) & 1u)) kb = -1;
+    }
+  }
+  const bool comp = lane < n_tiles && kb >= 0;
+  const unsigned cmask = __ballot_sync(kFull, comp);
+  if (lane < n_tiles) {
+    in.tile_kb[lane] = kb;
+    in.tile_off[lane] = off;
+  }
+  if (comp) in.comp_tile[__popc(cmask & ((1u << lane) - 1u))] = lane;
+  if (lane == 0) {
+    in.n_tiles = n_tiles;
+    in.n_comp = __popc(cmask);
+    in.ld = ld;
+    in.bh = bh;
+    in.qblk = i;
+    in.band = band;
+  }
+  __syncwarp();
 }
 
 __device__ __forceinline__ void epi_bar_sync() {
@@ -309,53 +324,60 @@ bigbird_probs_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
 
   if (warp == kProdWarp) {
     // ------------------------------------------------------------ plan + TMA
-    if (lane == 0) {
-      const uint64_t keep = l2_policy_evict_last();
-      int iq = 0, gk = 0;  // Q blocks and K groups loaded so far
-      for (int iu = 0;; ++iu) {
-        const int u = u0 + iu;
-        const int s = iu & 1;
+    // The whole warp plans each unit; lane 0 waits on the rings and issues
+    // the loads, and tells the other lanes when to stop.
+    const uint64_t keep = l2_policy_evict_last();
+    int iq = 0, gk = 0;  // Q blocks and K groups loaded so far (lane 0)
+    for (int iu = 0;; ++iu) {
+      const int u = u0 + iu;
+      const int s = iu & 1;
+      UnitInfo& in = sm.info[s];
+      int stop = 0;
+      if (lane == 0) {
         if (iu >= 2 && !mbar_wait(smem_u32(&sm.info_empty[s]), ((iu - 2) >> 1) & 1)) {
           set_abort(sm, p);
-          break;
-        }
-        UnitInfo& in = sm.info[s];
-        if (u >= u1 || aborted(sm)) {
+          stop = 1;
+        } else if (u >= u1 || aborted(sm)) {
           in.n_tiles = -1;
           mbar_arrive(smem_u32(&sm.info_full[s]));
-          break;
-        }
-        plan_unit(p, in, u);
-        mbar_arrive(smem_u32(&sm.info_full[s]));  // release: the plan is visible to the waiting roles
-        const int nc = in.n_comp;
-        if (nc == 0) continue;  // zero tiles only: nothing to load
-        const int row0 = in.bh * p.L;
-        const int qs = iq & 1;
-        if (iq >= 2 && !mbar_wait(smem_u32(&sm.q_empty[qs]), ((iq - 2) >> 1) & 1)) {
-          set_abort(sm, p);
-          break;
-        }
-        mbar_arrive_expect_tx(smem_u32(&sm.q_full[qs]), kTileBytes);
-        tma_load_2d(smem_u32(sm.q[qs]), &tmQ, smem_u32(&sm.q_full[qs]), 0, row0 + in.qblk * kBlock, keep);
-        ++iq;
-        bool ok = true;
-        for (int g = 0; g < (nc + 1) / 2; ++g, ++gk) {
-          const int ks = gk % kKSlots;
-          if (gk >= kKSlots && !mbar_wait(smem_u32(&sm.k_empty[ks]), (gk / kKSlots - 1) & 1)) {
-            ok = false;
-            break;
-          }
-          const int nt = min(2, nc - 2 * g);
-          mbar_arrive_expect_tx(smem_u32(&sm.k_full[ks]), static_cast<uint32_t>(nt) * kTileBytes);
-          for (int t = 0; t < nt; ++t)
-            tma_load_2d(smem_u32(sm.k[ks][t]), &tmK, smem_u32(&sm.k_full[ks]), 0,
-                        row0 + in.tile_kb[in.comp_tile[2 * g + t]] * kBlock, keep);
-        }
-        if (!ok) {
-          set_abort(sm, p);
-          break;
+          stop = 1;
         }
       }
+      if (__shfl_sync(0xffffffffu, stop, 0)) break;
+      plan_unit_warp(p, in, u, lane);  // ends with __syncwarp: lane 0 sees every lane's entries
+      if (lane == 0) {
+        mbar_arrive(smem_u32(&sm.info_full[s]));  // release: the plan is visible to the waiting roles
+        const int nc = in.n_comp;
+        if (nc > 0) {  // (a unit of zero tiles only loads nothing)
+          const int row0 = in.bh * p.L;
+          const int qs = iq & 1;
+          bool ok = !(iq >= 2 && !mbar_wait(smem_u32(&sm.q_empty[qs]), ((iq - 2) >> 1) & 1));
+          if (ok) {
+            mbar_arrive_expect_tx(smem_u32(&sm.q_full[qs]), kTileBytes);
+            tma_load_2d(smem_u32(sm.q[qs]), &tmQ, smem_u32(&sm.q_full[qs]), 0, row0 + in.qblk * kBlock, keep);
+            ++iq;
+          }
+          for (int g = 0; ok && g < (nc + 1) / 2; ++g, ++gk) {
+            const int ks = gk % kKSlots;
+            if (gk >= kKSlots && !mbar_wait(smem_u32(&sm.k_empty[ks]), (gk / kKSlots - 1) & 1)) {
+              ok = false;
+              break;
+            }
+            const int nt = min(2, nc - 2 * g);
+            mbar_arrive_expect_tx(smem_u32(&sm.k_full[ks]), static_cast<uint32_t>(nt) * kTileBytes);
+            for (int t = 0; t < nt; ++t)
+              tma_load_2d(smem_u32(sm.k[ks][t]), &tmK, smem_u32(&sm.k_full[ks]), 0,
+                          row0 + in.tile_kb[in.comp_tile[2 * g + t]] * kBlock, keep);
+          }
+          if (!ok) {
+            set_abort(sm, p);
+            stop = 1;
+          }
+        }
+      }
+      if (__shfl_sync(0xffffffffu, stop, 0)) break;
+    }
+    if (lane == 0) {
       // No copy may still be in flight when the CTA exits: wait (bounded) for
       // the last loads of both rings.
       for (int j = max(0, iq - 2); j < iq; ++j) mbar_wait(smem_u32(&sm.q_full[j & 1]), (j >> 1) & 1);
