@@ -186,3 +186,24 @@ def test_probs_layout_and_argument_errors_before_any_launch():
                                         None) == bb.BB_ERR_INVALID_ARG
     assert lib.bigbird_attn_probs_dense(fake, fake, fake, fake, None, P(0x10002), 1, 2, 4096, 64, 64, 3,
                                         bb.BB_OUT_BF16, 0, None) == bb.BB_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("block", [32, 128])
+def test_host_prep_other_block_sizes(block):
+    """The pages' only knob is block_size: the host routines (generator,
+    validator, masks, pattern table, fallback rule) follow the oracle bit for
+    bit at other block sizes too. (The GPU kernels take block 64 only.)"""
+    H, L, r = 3, 64 * block, 3
+    for seed, last_idx in ((5, 0), (2**63 + 1, 0), (9, 40 * block)):
+        got = bb.rand_attn_generate(H, L, block, r, seed=seed, last_idx=last_idx)
+        want = oracle.rand_attn_generate(H, L, block, r, seed=seed, last_idx=last_idx)
+        assert np.array_equal(got, want)
+        assert bb.rand_attn_validate(got, H, L, block, r, last_idx) == bb.BB_OK
+    ra = oracle.rand_attn_generate(H, L, block, r, seed=7)
+    assert np.array_equal(bb.pattern_table(ra, H, L, block, r), oracle.pattern_table(ra, H, L, block, r))
+    sm = mask_from_lengths(2, L, [L - 3 * block - 5, block]).numpy()
+    for g, w in zip(bb.mask_prep(sm, block), oracle.mask_prep(sm, block)):
+        assert g.shape == w.shape and np.array_equal(g, w)
+    for LL in range(block, block * 30, block):
+        assert bb.is_fallback(LL, block, r) == oracle.is_fallback(LL, block, r)
+    assert bb.is_fallback((5 + 2 * r) * block, block, r) and not bb.is_fallback((6 + 2 * r) * block, block, r)
