@@ -161,7 +161,7 @@ __device__ void plan_unit_warp(const ProbsParams& p, UnitInfo& in, int unit, int
     ld = kBlock;
     band = 1;
   }
-  // band rows: distinct candidates, their slots, and how many there are
+  // band rows: the distinct candidates and their slots
   int cand = kNone;
   bool valid = false;
   int rank = 0;
