@@ -309,16 +309,25 @@ def run_cuda(args):
     value = flops * world / (ms * 1e-3) / 1e12
     e2e_value = flops * world / (e2e_ms * 1e-3) / 1e12
     peaks, src = _peaks()
-    peak = float(peaks["bf16_tflops"])
     achieved = flops / (ms * 1e-3) / 1e12
-    # DRAM bytes (read + write) of one bigbird_fwd_kernel launch on the default
-    # workload, from the ncu capture summarised in
-    # profiles/bigbird_fwd_l4096_b4h12.md; valid for that kernel source only.
-    traffic = 88.87e6 if (w.name == DEFAULT_WORKLOAD and world == 1) else None
-    roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-            "frac": achieved / peak, "traffic": traffic,
-            "kernel": "bigbird_fwd_kernel + bigbird_merge_kernel (one fwd call; traffic: fwd kernel, ncu)",
-            "peak_source": f"{src} bf16 dense burst (kernel timed alone)"}
+    generic = (w.block, w.d) != (64, 64)
+    if generic:
+        # the CUDA-core kernel: fp32 peak from unit counts and clocks
+        sm_mhz = (clocks or {}).get("sm_max_mhz") or 1965.0
+        peak = props.multi_processor_count * 128 * 2 * float(sm_mhz) * 1e-6
+        roof = {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                "traffic": None, "kernel": "bigbird_generic_fwd_kernel (fp32 CUDA cores)",
+                "peak_source": "SMs x 128 fp32 FMA lanes x 2 x max SM clock"}
+    else:
+        peak = float(peaks["bf16_tflops"])
+        # DRAM bytes (read + write) of one bigbird_fwd_kernel launch on the default
+        # workload, from the ncu capture summarised in
+        # profiles/bigbird_fwd_l4096_b4h12.md; valid for that kernel source only.
+        traffic = 88.87e6 if (w.name == DEFAULT_WORKLOAD and world == 1) else None
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "traffic": traffic,
+                "kernel": "bigbird_fwd_kernel + bigbird_merge_kernel (one fwd call; traffic: fwd kernel, ncu)",
+                "peak_source": f"{src} bf16 dense burst (kernel timed alone)"}
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
@@ -330,7 +339,7 @@ def run_cuda(args):
         # per forward call: the attention kernel, plus the merge kernel when the
         # global rows are split into key ranges (sparse and more than 8 blocks);
         # the 4-byte counter reset before each call is a cudaMemsetAsync
-        "gpu_launches": (2 if (sparse and w.L // w.block > 8) else 1) * args.steps * reps,
+        "gpu_launches": (1 if generic else (2 if (sparse and w.L // w.block > 8) else 1)) * args.steps * reps,
         "warm_l2": {"ms_per_step": warm_ms, "value": flops * world / (warm_ms * 1e-3) / 1e12, "unit": UNIT,
                     "steps": n_warm, "note": "same calls back to back, no L2 flush (not the headline)"},
         "clocks": clocks,

@@ -16,7 +16,7 @@ CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libbigbird_attn.so")
 BUILD = os.path.join(ROOT, "_build")
 
-SOURCES = ["bigbird_attn.cu", "bigbird_bwd.cu", "bigbird_probs.cu", "host_prep.cpp"]
+SOURCES = ["bigbird_attn.cu", "bigbird_generic.cu", "bigbird_bwd.cu", "bigbird_probs.cu", "host_prep.cpp"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

@@ -18,4 +18,13 @@ bool make_tile_map(CUtensorMap* map, const void* base, uint64_t rows);
 // timed out), or null if `dev` is not an sm_100 device or a query failed.
 uint32_t* status_word(int dev);
 
+// The CUDA-core forward for the sizes the tensor-core kernel does not take
+// (bigbird_generic.cu): supported when d is 64 or 128 and block is 32, 64 or
+// 128, except d = block = 64. Arguments and results as bigbird_attn_fwd_train
+// with lse optional (null: not written); no workspace.
+bool generic_fwd_supported(int d, int block);
+int generic_fwd(const void* q, const void* k, const void* v, const int32_t* rand_attn, const uint8_t* seq_mask,
+                void* out, float* lse, int B, int H, int L, int d, int block, int r, int out_dtype, unsigned flags,
+                void* stream);
+
 }  // namespace bb

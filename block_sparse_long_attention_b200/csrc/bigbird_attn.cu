@@ -955,6 +955,9 @@ size_t bigbird_attn_workspace_size(int B, int H, int L, int d, int block, int r,
 static int fwd_impl(const void* q, const void* k, const void* v, const int32_t* rand_attn, const uint8_t* seq_mask,
                     void* out, float* lse, int B, int H, int L, int d, int block, int r, int out_dtype, unsigned flags,
                     void* workspace, size_t workspace_bytes, void* stream_) {
+  // Other supported sizes run the CUDA-core kernel (no workspace).
+  if (generic_fwd_supported(d, block))
+    return generic_fwd(q, k, v, rand_attn, seq_mask, out, lse, B, H, L, d, block, r, out_dtype, flags, stream_);
   cudaStream_t stream = static_cast<cudaStream_t>(stream_);
   Plan pl;
   int st = make_plan(B, H, L, d, block, r, flags, pl);
@@ -1143,6 +1146,10 @@ extern "C" int bigbird_attn_fwd_noalloc(const void* q, const void* k, const void
                                         int r, int out_dtype, unsigned flags, void* stream) {
   // The debug checks copy rand_attn into a host buffer that they allocate.
   if (flags & BB_FLAG_DEBUG_CHECKS) return BB_ERR_UNSUPPORTED;
+  // The CUDA-core kernel for other sizes needs no scratch.
+  if (bb::generic_fwd_supported(d, block))
+    return bigbird_attn_fwd_ex(q, k, v, rand_attn, seq_mask, out, B, H, L, d, block, r, out_dtype, flags, nullptr, 0,
+                               stream);
   bb::Plan pl;
   const int st = bb::make_plan(B, H, L, d, block, r, flags, pl);
   if (st != BB_OK) return st;

@@ -6,7 +6,8 @@ side derives rand_attn from the seed with its own implementation of the same
 generator definition.
 
 Workloads (the BigBird-base and BigBirdPegasus-large attention shapes, d = 64,
-block = 64, r = 3, at 1K to 32K tokens):
+block = 64, r = 3, at 1K to 32K tokens, and the BigBird-base shape at block 128
+and at d = 128):
 
 =====================  ==========================  =========================================
 name                   shape                       values / padding
@@ -16,6 +17,8 @@ bigbird_base_l4096     B4 H12 L4096                N(0,1)/sqrt(d); valid length 
 pegasus_large_l4096    B2 H16 L4096                N(0,1); no padding
 long_l16384            B1 H12 L16384 (256 blocks)  N(0,1); last 10 % of tokens padded
 extreme_l32768         B1 H8 L32768 (512 blocks)   N(0,1) x 2; valid length U[24576, 32768]
+base_l4096_block128    B4 H12 L4096, block 128     N(0,1)/sqrt(d); valid length U[2048, 4096]
+base_l4096_d128        B4 H12 L4096, d 128         N(0,1)/sqrt(d); valid length U[2048, 4096]
 =====================  ==========================  =========================================
 
 Recipe: a ``torch.Generator`` seeded with the workload seed draws fp32 N(0,1)
@@ -64,6 +67,11 @@ WORKLOADS = {
         Workload("long_l16384", 1, 12, 16384, pad=("last_frac", 0.1), seed=1004),
         Workload("extreme_l32768", 1, 8, 32768, value_scale=2.0,
                  pad=("uniform", 24576, 32768), seed=1005),
+        # the BigBird-base shape at the other sizes the pages allow (CUDA-core kernel)
+        Workload("base_l4096_block128", 4, 12, 4096, block=128, value_scale=1.0 / math.sqrt(64.0),
+                 pad=("uniform", 2048, 4096), seed=1006),
+        Workload("base_l4096_d128", 4, 12, 4096, d=128, value_scale=1.0 / math.sqrt(128.0),
+                 pad=("uniform", 2048, 4096), seed=1007),
     )
 }
 

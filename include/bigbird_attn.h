@@ -35,7 +35,7 @@ extern "C" {
 typedef enum {
   BB_OK = 0,
   BB_ERR_INVALID_ARG = 1,   /* NULL pointer, non-positive size, L % block != 0, r < 1 */
-  BB_ERR_UNSUPPORTED = 2,   /* d != 64 or block != 64, misaligned pointer, no sm_100 device */
+  BB_ERR_UNSUPPORTED = 2,   /* unsupported d / block, misaligned pointer, no sm_100 device */
   BB_ERR_CUDA = 3,          /* a CUDA runtime call or launch failed */
   BB_ERR_BAD_RAND_ATTN = 4, /* rand_attn breaks the generator's rules (validator / debug checks) */
   BB_ERR_DEVICE = 5         /* a kernel reported a device-side error (see bigbird_device_status) */
@@ -75,7 +75,10 @@ enum {
  *              May be NULL only in the full-attention fallback.
  *   seq_mask   device, uint8 [B, L], nonzero = valid key; NULL = all valid.
  *   out        device, bf16 [B, H, L, d], 16-byte aligned; must not alias q/k/v.
- *   B, H, L, d, block, r  sizes; v1 supports d = 64 and block = 64 only.
+ *   B, H, L, d, block, r  sizes: d in {64, 128}, block in {32, 64, 128}.
+ *              d = block = 64 runs the tensor-core kernel described above; the
+ *              other sizes run a CUDA-core kernel (fp32 arithmetic, one CTA per
+ *              query block, no workspace) with the same results.
  *   stream     cudaStream_t.
  * Errors: BB_ERR_INVALID_ARG for L % block != 0 [HF-Pegasus, section
  * "序列长度的块对齐要求"] or r < 1 [HF-Pegasus, section "使用限制与注意事项"];

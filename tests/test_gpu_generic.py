@@ -1,0 +1,131 @@
+"""The CUDA-core forward (block 32 or 128, d 64 or 128) through the C ABI
+against the fp64 oracle.
+
+Bars: bf16 output as the tensor-core path (max |err| <= 1e-2, mean <= 1e-3);
+fp32 output max |err| <= 1e-4, derived from the arithmetic: fp32 dot products
+and sums over at most L keys (~1e-6 relative), accurate exp2f, and one fp32
+rescale per 32-key chunk (<= ~60 per row: ~4e-6 relative), on outputs of
+magnitude <~ 4. lse (fwd_train) <= 1e-5 absolute.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import block_sparse_long_attention_b200 as bb
+from block_sparse_long_attention_b200.workloads import Workload, make_inputs
+
+pytestmark = pytest.mark.gpu
+
+SIZES = [(32, 64), (128, 64), (32, 128), (64, 128), (128, 128)]  # (block, d)
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from block_sparse_long_attention_b200 import build
+    build.build()
+    bb.device_status()
+    yield
+
+
+def _ra(w, seed=None):
+    if oracle.is_fallback(w.L, w.block, w.r):
+        return None
+    ra = bb.rand_attn_generate(w.H, w.L, w.block, w.r, seed=w.seed if seed is None else seed)
+    assert np.array_equal(ra, oracle.rand_attn_generate(w.H, w.L, w.block, w.r, seed=w.seed if seed is None else seed))
+    return ra
+
+
+def _run(w, inp, ra, out_dtype, train=False, force_sparse=False):
+    q, k, v = (inp[x].cuda() for x in "qkv")
+    sm = None if inp["seq_mask"] is None else inp["seq_mask"].cuda()
+    ra_d = None if ra is None else torch.from_numpy(np.ascontiguousarray(ra)).cuda()
+    if train:
+        out, lse = bb.fwd_train(q, k, v, ra_d, sm, block=w.block, r=w.r, out_dtype=out_dtype,
+                                force_sparse=force_sparse)
+    else:
+        out, lse = bb.fwd(q, k, v, ra_d, sm, block=w.block, r=w.r, out_dtype=out_dtype,
+                          force_sparse=force_sparse), None
+    torch.cuda.synchronize()
+    assert bb.device_status() == 0
+    return out.float().cpu().numpy().astype(np.float64), None if lse is None else lse.double().cpu().numpy()
+
+
+def _cases(block, d):
+    s = 10 * block + d
+    return [
+        Workload(f"sparse_b{block}_d{d}", 2, 2, 14 * block, d=d, block=block,
+                 value_scale=1.0, pad=("fixed", [14 * block - block - 5, 7 * block + 3]), seed=s),
+        Workload(f"fallback_b{block}_d{d}", 1, 2, 8 * block, d=d, block=block, pad=("fixed", [8 * block - 9]),
+                 seed=s + 1),
+        Workload(f"one_block_b{block}_d{d}", 1, 1, block, d=d, block=block, seed=s + 2),
+    ]
+
+
+@pytest.mark.parametrize("block,d", SIZES, ids=[f"b{b}_d{d}" for b, d in SIZES])
+def test_generic_all_rows(block, d):
+    for w in _cases(block, d):
+        inp = make_inputs(w)
+        ra = _ra(w)
+        want = oracle.attention(inp["q"], inp["k"], inp["v"], ra, inp["seq_mask"], w.block, w.r)
+        got, lse = _run(w, inp, ra, torch.float32, train=True)
+        err = np.abs(got - want)
+        assert err.max() <= 1e-4, (w.name, float(err.max()))
+        want_lse = oracle.attention_lse(inp["q"], inp["k"], ra, inp["seq_mask"], w.block, w.r)
+        assert np.abs(lse - want_lse).max() <= 1e-5, (w.name, float(np.abs(lse - want_lse).max()))
+        got16, _ = _run(w, inp, ra, torch.bfloat16)
+        err16 = np.abs(got16 - want)
+        assert err16.max() <= 1e-2 and err16.mean() <= 1e-3, (w.name, float(err16.max()), float(err16.mean()))
+
+
+@pytest.mark.parametrize("block,d", [(128, 64), (128, 128), (32, 64)], ids=["b128_d64", "b128_d128", "b32_d64"])
+def test_generic_l4096(block, d):
+    """4096 tokens (32 to 128 blocks), padded, every row of two heads."""
+    w = Workload(f"l4096_b{block}_d{d}", 1, 2, 4096, d=d, block=block, value_scale=1.0 / np.sqrt(d),
+                 pad=("fixed", [3001]), seed=3 * block + d)
+    inp = make_inputs(w)
+    ra = _ra(w)
+    got, _ = _run(w, inp, ra, torch.float32)
+    want = oracle.attention(inp["q"], inp["k"], inp["v"], ra, inp["seq_mask"], w.block, w.r)
+    assert np.abs(got - want).max() <= 1e-4
+
+
+def test_generic_set_semantics_forced_sparse_and_flags():
+    w = Workload("edge_b32", 1, 2, 16 * 32, d=64, block=32, pad=("fixed", [400]), seed=77)
+    inp = make_inputs(w)
+    ra = oracle.rand_attn_generate(w.H, w.L, w.block, w.r, seed=4)
+    ra[0] = 0
+    ra[1, 5, :] = ra[1, 5, 0]
+    ra[1, 9, 0] = 10
+    got, _ = _run(w, inp, ra, torch.float32)
+    want = oracle.attention(inp["q"], inp["k"], inp["v"], ra, inp["seq_mask"], w.block, w.r)
+    assert np.abs(got - want).max() <= 1e-4
+    # forced sparse at nb = 5 + r: the sparse definition everywhere, and rows
+    # 2 .. nb-3 (window + globals + the r remaining blocks) see every block;
+    # rows 1 and nb-2 hold 4 + r blocks, so they cannot
+    w2 = Workload("forced_b128", 1, 1, 8 * 128, d=128, block=128, seed=78)
+    inp2 = make_inputs(w2)
+    nb = 8
+    ra2 = np.zeros((1, nb - 2, 3), dtype=np.int32)
+    for i in range(1, nb - 1):
+        rest = [j for j in range(1, nb - 1) if abs(j - i) > 1]
+        ra2[0, i - 1] = (rest + [rest[0]] * 3)[:3]
+    got2, _ = _run(w2, inp2, ra2, torch.float32, force_sparse=True)
+    want2 = oracle.attention(inp2["q"], inp2["k"], inp2["v"], ra2, None, 128, 3, force_sparse=True)
+    assert np.abs(got2 - want2).max() <= 1e-4
+    full2 = oracle.attention(inp2["q"], inp2["k"], inp2["v"], None, None, 128, 3)  # full attention
+    mid = slice(2 * 128, (nb - 2) * 128)
+    assert np.abs(got2[:, :, mid] - full2[:, :, mid]).max() <= 1e-4
+    # an out-of-range entry is skipped and flagged
+    q, k, v = (inp[x].cuda() for x in "qkv")
+    bad = torch.from_numpy(np.ascontiguousarray(ra)).cuda()
+    bad[0, 3, 1] = 999
+    bb.device_status()
+    bb.fwd(q, k, v, bad, inp["seq_mask"].cuda(), block=32, r=3)
+    assert bb.device_status() & 1
+    # deterministic
+    a, _ = _run(w, inp, ra, torch.float32)
+    assert np.array_equal(a, got)

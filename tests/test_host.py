@@ -126,8 +126,10 @@ def test_fwd_argument_errors_before_any_launch():
     cases = [
         (dict(L=1000), bb.BB_ERR_INVALID_ARG),   # not a multiple of the block
         (dict(r=0), bb.BB_ERR_INVALID_ARG),      # r = 0 unsupported
-        (dict(d=128), bb.BB_ERR_UNSUPPORTED),
-        (dict(block=32), bb.BB_ERR_UNSUPPORTED),
+        (dict(d=96), bb.BB_ERR_UNSUPPORTED),
+        (dict(block=48, L=3072), bb.BB_ERR_UNSUPPORTED),
+        (dict(d=128, L=1000), bb.BB_ERR_INVALID_ARG),       # the CUDA-core sizes check their arguments too
+        (dict(block=32, r=0), bb.BB_ERR_INVALID_ARG),
         (dict(B=0), bb.BB_ERR_INVALID_ARG),
         (dict(r=17), bb.BB_ERR_UNSUPPORTED),
     ]
@@ -145,6 +147,21 @@ def test_fwd_argument_errors_before_any_launch():
     # forced sparse needs nb >= 5 + r
     assert lib.bigbird_attn_fwd_ex(fake, fake, fake, fake, None, fake, 1, 2, 7 * 64, 64, 64, 3, 0,
                                    bb.BB_FLAG_FORCE_SPARSE, None, 0, None) == bb.BB_ERR_INVALID_ARG
+    # the CUDA-core sizes (block 32 / 128, d 128) check the same before any device call
+    for d, block in ((64, 32), (64, 128), (128, 32), (128, 64), (128, 128)):
+        L = 16 * block
+        assert lib.bigbird_attn_fwd(None, fake, fake, fake, None, fake, 1, 2, L, d, block, 3, None) == \
+            bb.BB_ERR_INVALID_ARG
+        assert lib.bigbird_attn_fwd(fake, fake, fake, fake, None, P(0x10008), 1, 2, L, d, block, 3, None) == \
+            bb.BB_ERR_UNSUPPORTED
+        assert lib.bigbird_attn_fwd(fake, fake, fake, None, None, fake, 1, 2, L, d, block, 3, None) == \
+            bb.BB_ERR_INVALID_ARG
+        assert lib.bigbird_attn_fwd_ex(fake, fake, fake, fake, None, fake, 1, 2, 7 * block, d, block, 3, 0,
+                                       bb.BB_FLAG_FORCE_SPARSE, None, 0, None) == bb.BB_ERR_INVALID_ARG
+        assert bb.workspace_size(1, 2, L, d, block) == 0   # no workspace
+    # the backward and the probability export take d = block = 64 only
+    assert lib.bigbird_attn_probs(fake, fake, fake, fake, None, fake, fake, 1, 2, 4096, 128, 64, 3, 1, 0, None) == \
+        bb.BB_ERR_UNSUPPORTED
     assert bb.status_string(bb.BB_ERR_UNSUPPORTED) == "unsupported configuration"
 
 
