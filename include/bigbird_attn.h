@@ -92,7 +92,8 @@ int bigbird_attn_fwd(const void* q, const void* k, const void* v, const int32_t*
 
 /*
  * Bytes of device scratch bigbird_attn_fwd_ex needs for these sizes and
- * flags (0 if the sizes are invalid). The scratch starts with a 256-byte slot
+ * flags (0 if the sizes are invalid, and for the sizes the CUDA-core kernel
+ * runs, which need none). For d = block = 64 the scratch starts with a 256-byte slot
  * for the counter through which the CTAs share out the work units (every call
  * zeroes it with cudaMemsetAsync on its stream before the launch); when the
  * global rows are split into key ranges (sparse pattern, nb > 8) it also holds
