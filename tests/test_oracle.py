@@ -342,6 +342,25 @@ def test_sparse_flops():
     assert math.isclose(oracle.sparse_flops(4, 12, 4096, 64, 64, 3) / 1e9, 31.31, rel_tol=1e-3)
 
 
+@pytest.mark.parametrize("L,d", [(1024, 64), (20 * 64, 32), (11 * 64, 16)])
+def test_work_counts_match_the_attended_pairs(L, d):
+    """The forward and backward work counts equal a count of the attended
+    (query, key) pairs taken from the weight matrix itself: every attended
+    pair has a nonzero weight (no padding here), every other pair weight 0.
+    Per pair and head dimension the forward forms 2 products (q.k and p.v)
+    and the backward 5 (q.k recomputed, dout.v, p.dout, ds.k, ds.q), each
+    one multiply-add = 2 FLOP."""
+    B, H, block, r = 1, 2, 64, 3
+    q, k, _ = _rand_qkv(B, H, L, d, seed=41)
+    nb = L // block
+    ra = None if oracle.is_fallback(L, block, r) else oracle.rand_attn_generate(H, L, block, r, seed=42)
+    p = oracle.attention_probs(q, k, ra, None, block, r)
+    pairs = int(np.count_nonzero(p))
+    assert pairs > 0 and (pairs < B * H * L * L or nb <= 5 + 2 * r)
+    assert oracle.sparse_flops(B, H, L, d, block, r) == 4.0 * d * pairs
+    assert oracle.backward_flops(B, H, L, d, block, r) == 10.0 * d * pairs
+
+
 # --------------------------------------------------------------------------
 # The C sparse brute-force reference (the timed CPU baseline) against the
 # dense-mask oracle: both are fp64 statements of the same definition, one by
