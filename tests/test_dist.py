@@ -35,30 +35,35 @@ def _free_port():
     return port
 
 
+def _oracle_compute(q, k, v, ra_, sm, block, r):
+    import oracle
+    return torch.from_numpy(oracle.attention(q, k, v, None if ra_ is None else np.asarray(ra_),
+                                             None if sm is None else np.asarray(sm), block, r))
+
+
 def _worker(rank, world, port, result_path):
+    """Each rank runs the product's batch-sharded forward (its slice of the
+    sequences, then the all-gather along the batch axis) with the oracle as
+    the per-rank compute (no GPU here)."""
     os.environ["MASTER_ADDR"] = "127.0.0.1"
     os.environ["MASTER_PORT"] = str(port)
     from datetime import timedelta
     dist.init_process_group("gloo", rank=rank, world_size=world, timeout=timedelta(seconds=60))
     import oracle
+    from block_sparse_long_attention_b200.sharding import batch_sharded_fwd
     from block_sparse_long_attention_b200.workloads import Workload, make_inputs
     w = Workload("dist", 3, 2, 14 * 64, pad=("fixed", [896, 500, 700]), seed=31)
     inp = make_inputs(w)
     ra = oracle.rand_attn_generate(w.H, w.L, w.block, w.r, seed=w.seed)
+    full = batch_sharded_fwd(inp["q"], inp["k"], inp["v"], ra, inp["seq_mask"], block=w.block, r=w.r,
+                             compute=_oracle_compute)
+    mine = batch_sharded_fwd(inp["q"], inp["k"], inp["v"], ra, inp["seq_mask"], block=w.block, r=w.r,
+                             gather=False, compute=_oracle_compute)
     lo, hi = batch_shard(w.B, world, rank)
-    part = oracle.attention(inp["q"][lo:hi], inp["k"][lo:hi], inp["v"][lo:hi], ra, inp["seq_mask"][lo:hi].numpy(),
-                            w.block, w.r)
-    # pad to the largest shard so all_gather sees equal shapes
-    maxn = max(b - a for a, b in (batch_shard(w.B, world, r) for r in range(world)))
-    buf = torch.zeros((maxn,) + part.shape[1:], dtype=torch.float64)
-    buf[: hi - lo] = torch.from_numpy(part)
-    gathered = [torch.zeros_like(buf) for _ in range(world)]
-    dist.all_gather(gathered, buf)
+    assert mine.shape[0] == hi - lo
     if rank == 0:
-        pieces = [g[: b - a] for g, (a, b) in zip(gathered, (batch_shard(w.B, world, r) for r in range(world)))]
-        full = torch.cat(pieces).numpy()
         ref = oracle.attention(inp["q"], inp["k"], inp["v"], ra, inp["seq_mask"].numpy(), w.block, w.r)
-        np.save(result_path, np.array([np.abs(full - ref).max()]))
+        np.save(result_path, np.array([np.abs(full.numpy() - ref).max(), float(full.shape[0])]))
     dist.barrier()
     dist.destroy_process_group()
 
@@ -66,7 +71,8 @@ def _worker(rank, world, port, result_path):
 def test_two_gloo_ranks_equal_single_process(tmp_path):
     path = str(tmp_path / "res.npy")
     mp.start_processes(_worker, args=(2, _free_port(), path), nprocs=2, join=True, start_method="spawn")
-    assert float(np.load(path)[0]) == 0.0
+    err, nseq = np.load(path)
+    assert err == 0.0 and nseq == 3
 
 
 def _head_worker(rank, world, port, result_path):
@@ -81,10 +87,8 @@ def _head_worker(rank, world, port, result_path):
     inp = make_inputs(w)
     ra = torch.from_numpy(oracle.rand_attn_generate(w.H, w.L, w.block, w.r, seed=w.seed))
 
-    def compute(q, k, v, ra_, sm, block, r):
-        return torch.from_numpy(oracle.attention(q, k, v, ra_.numpy(), sm.numpy(), block, r))
-
-    full = sharded_fwd(inp["q"], inp["k"], inp["v"], ra, inp["seq_mask"], block=w.block, r=w.r, compute=compute)
+    full = sharded_fwd(inp["q"], inp["k"], inp["v"], ra, inp["seq_mask"], block=w.block, r=w.r,
+                       compute=_oracle_compute)
     if rank == 0:
         ref = oracle.attention(inp["q"], inp["k"], inp["v"], ra.numpy(), inp["seq_mask"].numpy(), w.block, w.r)
         np.save(result_path, np.array([np.abs(full.numpy() - ref).max(), float(full.shape[1])]))
