@@ -188,7 +188,7 @@ def fwd_train(q, k, v, rand_attn, seq_mask=None, *, block: int = 64, r: int = 3,
     lib_ = _load()
     ws_bytes = int(lib_.bigbird_attn_workspace_size(B, H, L, d, block, r, flags))
     if workspace is None or workspace.numel() * workspace.element_size() < ws_bytes:
-        workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=q.device)
+        workspace = torch.zeros(max(ws_bytes, 1), dtype=torch.uint8, device=q.device)
     st = lib_.bigbird_attn_fwd_train(q.data_ptr(), k.data_ptr(), v.data_ptr(), ra_ptr, sm_ptr, out.data_ptr(),
                                      lse.data_ptr(), B, H, L, d, block, r,
                                      BB_OUT_F32 if out_dtype == torch.float32 else BB_OUT_BF16, flags,
@@ -296,7 +296,10 @@ def fwd(q, k, v, rand_attn, seq_mask=None, *, block: int = 64, r: int = 3, out=N
     with out_dtype=torch.float32). q, k, v: contiguous bf16 CUDA tensors
     [B, H, L, d]; rand_attn: int32 CUDA tensor [H, nb-2, r] (or None in the
     full-attention fallback); seq_mask: uint8 CUDA tensor [B, L] (1 = valid
-    key) or None. Runs on the current torch stream (or `stream`)."""
+    key) or None. Runs on the current torch stream (or `stream`).
+    `workspace` (optional, reusable across calls): a uint8 CUDA tensor of at
+    least workspace_size(...) bytes, zero-filled before its first use (each
+    call leaves its counters at zero again, e.g. torch.zeros)."""
     import torch
     for name, t in (("q", q), ("k", k), ("v", v)):
         if not (t.is_cuda and t.dtype == torch.bfloat16 and t.is_contiguous() and t.dim() == 4):
@@ -331,7 +334,7 @@ def fwd(q, k, v, rand_attn, seq_mask=None, *, block: int = 64, r: int = 3, out=N
     ws_ptr = None
     if ws_bytes:
         if workspace is None or workspace.numel() * workspace.element_size() < ws_bytes:
-            workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
+            workspace = torch.zeros(ws_bytes, dtype=torch.uint8, device=q.device)
         ws_ptr = workspace.data_ptr()
     st = lib_.bigbird_attn_fwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), ra_ptr, sm_ptr, out.data_ptr(),
                                   B, H, L, d, block, r, BB_OUT_F32 if out_dtype == torch.float32 else BB_OUT_BF16,

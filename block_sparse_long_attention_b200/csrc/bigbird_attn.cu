@@ -17,7 +17,8 @@
 //     does not use a block writes P = 0 for it, so the pair shares every MMA.
 //
 // Units are handed out dynamically (longest first): a CTA's first unit is its
-// block index, later ones are tickets from a device-wide counter.
+// block index, later ones are tickets from a counter in the workspace; the
+// CTA that finishes last sets the workspace counters back to zero.
 //
 // A unit's key blocks are processed one at a time through a serial chain:
 // S = Q K^T (tcgen05 SS-MMA, 128x64x16 steps) -> softmax -> fp16 P written
@@ -47,7 +48,12 @@
 // Padded keys get -10000 added to the scaled score. P.V runs in fp16: P is
 // written as fp16 and each V tile is converted bf16 -> fp16 in shared memory
 // (exact in the fp16 normal range), which keeps three more mantissa bits of P
-// than bf16.
+// than bf16. fp16 cannot represent a magnitude >= 65536: the converter flags
+// such a value (in the workspace) as it converts, and a second instance of
+// this kernel, launched behind the first as its programmatic dependent, then
+// recomputes the whole call with bf16 P and V as loaded (8 significant bits of
+// P), so every finite bf16 V is taken. Without the flag the second instance
+// returns at once.
 #include <cuda.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -84,6 +90,16 @@ constexpr uint32_t kColO = 64;         // O: 64 fp32 columns
 constexpr float kRescaleThreshold = 14.0f;  // log2 units
 constexpr float kNegInit = -1.0e30f;
 
+// bf16 exponent field (bits 7..14 of a 16-bit value) of 2^16: a tile whose
+// largest exponent field reaches it holds a value fp16 cannot represent.
+constexpr uint32_t kBigExpField = 143u << 7;
+
+// Workspace counters (ints, in the first 256 bytes): [0] unit tickets handed
+// out beyond gridDim.x, [1] CTAs finished, [2] set when a V value fp16 cannot
+// represent was seen (the bf16 instance then recomputes the call).
+constexpr size_t kCounterBytes = 256;
+constexpr int kCtrTickets = 0, kCtrDone = 1, kCtrBigV = 2;
+
 // status word bits
 constexpr uint32_t kStatusBadRandAttn = 1u;
 constexpr uint32_t kStatusTimeout = 2u;
@@ -113,7 +129,7 @@ struct FwdParams {
   float* part_o;   // [BH, nsplit, 128, 64]
   float* part_ml;  // [BH, nsplit, 128, 2]
   uint32_t* status;
-  int* sched;       // unit tickets handed out so far beyond the first gridDim.x (zeroed before launch)
+  int* counters;    // workspace counters (zero at launch; the last CTA resets them)
   int B, H, L, nb, r, BH;
   int sparse;
   int nsplit;        // key ranges per global unit (1 = write the output directly)
@@ -301,7 +317,7 @@ __device__ void prep_role(SharedStorage& s, const FwdParams& p) {
     }
     // Claim the next unit now, so the atomic's round trip overlaps this one's preparation.
     int next = 0;
-    if (lane == 0) next = static_cast<int>(gridDim.x) + atomicAdd(p.sched, 1);
+    if (lane == 0) next = static_cast<int>(gridDim.x) + atomicAdd(&p.counters[kCtrTickets], 1);
     prep_unit(p, u, ui, lane);
     if (lane == 0) mbar_arrive(smem_u32(&s.info_full[slot]));
     // Pull the unit's tiles into L2 now (it is up to four units ahead of the
@@ -323,6 +339,11 @@ __device__ void prep_role(SharedStorage& s, const FwdParams& p) {
 
 // V blocks are converted bf16 -> fp16 in place (exact in the fp16 normal
 // range) in the order the TMA warp loads them; the P.V MMA waits for v_conv.
+// A value of magnitude >= 2^16 (its bf16 exponent field >= 143), which fp16
+// cannot represent, sets the workspace flag that makes the bf16 instance
+// recompute the call. The bf16 instance converts nothing: this warp only
+// keeps the unit bookkeeping.
+template <bool kBf16>
 __device__ void convert_role(SharedStorage& s, const FwdParams& p) {
   const int lane = threadIdx.x & 31;
   uint32_t gv = 0;
@@ -330,13 +351,18 @@ __device__ void convert_role(SharedStorage& s, const FwdParams& p) {
     if (!warp_wait(smem_u32(&s.info_full[ut & 3]), (ut >> 2) & 1)) { if (lane == 0) flag_timeout(s, p); return; }
     if (s.unit[ut & 3].stop) break;
     const int n = s.unit[ut & 3].n;
-    for (int e = 0; e < n; ++e, ++gv) {
+    for (int e = 0; e < n && !kBf16; ++e, ++gv) {
       const int st = gv % kVStages;
       if (!warp_wait(smem_u32(&s.v_full[st]), (gv / kVStages) & 1)) { if (lane == 0) flag_timeout(s, p); return; }
       uint4* vp = reinterpret_cast<uint4*>(s.v[st]) + lane;
+      uint32_t ex = 0;  // largest bf16 exponent field seen, per 16-bit half
 #pragma unroll 4
       for (int i = 0; i < static_cast<int>(kTileBytes / 16 / 32); ++i) {
         uint4 w = vp[32 * i];
+        ex = __vmaxu2(ex, w.x & 0x7F807F80u);
+        ex = __vmaxu2(ex, w.y & 0x7F807F80u);
+        ex = __vmaxu2(ex, w.z & 0x7F807F80u);
+        ex = __vmaxu2(ex, w.w & 0x7F807F80u);
         w.x = bf16x2_to_f16x2(w.x);
         w.y = bf16x2_to_f16x2(w.y);
         w.z = bf16x2_to_f16x2(w.z);
@@ -344,6 +370,8 @@ __device__ void convert_role(SharedStorage& s, const FwdParams& p) {
         vp[32 * i] = w;
       }
       fence_proxy_async_smem();
+      if (__any_sync(0xffffffffu, max(ex & 0xFFFFu, ex >> 16) >= kBigExpField) && lane == 0)
+        atomicExch(&p.counters[kCtrBigV], 1);
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&s.v_conv[st]));
     }
@@ -443,9 +471,11 @@ __device__ void producer_role(SharedStorage& s, const FwdParams& p, const CUtens
 // previous block's P.V has consumed the P that shares them, then, once the
 // softmax has written P(g), O += P(g) . V(g). The chain is serial within a
 // CTA; the four CTAs of an SM interleave on the tensor pipe.
+template <bool kBf16>
 __device__ void mma_role(SharedStorage& s, const FwdParams& p, uint32_t tmem) {
   const uint32_t idesc_s = idesc_f32acc(kRows, kBlock, true, false);    // bf16 Q . K^T, N = 64
-  const uint32_t idesc_o = idesc_f32acc(kRows, kHeadDim, false, true);  // fp16 P . fp16 V
+  // fp16 P . fp16 V, or bf16 P . bf16 V in the bf16 instance
+  const uint32_t idesc_o = idesc_f32acc(kRows, kHeadDim, kBf16, true);
   const uint32_t q_addr = smem_u32(s.q);
   uint32_t g = 0;
   bool ok = true;
@@ -468,7 +498,8 @@ __device__ void mma_role(SharedStorage& s, const FwdParams& p, uint32_t tmem) {
       mma_commit(smem_u32(&s.k_empty[kst]));
       if (e == n - 1) mma_commit(smem_u32(&s.q_free));
       const int vst = g % kVStages;
-      if (!mbar_wait(smem_u32(&s.v_conv[vst]), (g / kVStages) & 1)) { ok = false; break; }
+      // the V tile: converted (fp16), or as loaded (bf16 instance)
+      if (!mbar_wait(smem_u32(kBf16 ? &s.v_full[vst] : &s.v_conv[vst]), (g / kVStages) & 1)) { ok = false; break; }
       if (e == 0 && !mbar_wait(smem_u32(&s.o_free), (ut & 1) ^ 1)) { ok = false; break; }
       if (!mbar_wait(smem_u32(&s.p_full), g & 1)) { ok = false; break; }
       tc_fence_after();
@@ -511,8 +542,9 @@ __device__ __forceinline__ float piece16_prepare(uint32_t (&r)[16], bool mixed, 
   return fmax3(a, b, fmaxf(__uint_as_float(r[14]), __uint_as_float(r[15])));
 }
 
-// p = exp2(r * scale + off) for 16 scores, packed to fp16x2 into pk; the sum
-// accumulates into two packed pairs.
+// p = exp2(r * scale + off) for 16 scores, packed in pairs into pk (fp16, or
+// bf16 in the bf16 instance); the sum accumulates into two packed pairs.
+template <bool kBf16>
 __device__ __forceinline__ void piece16_exp(const uint32_t (&r)[16], uint64_t scale2, uint64_t off2, uint32_t (&pk)[8],
                                             uint64_t& acc0, uint64_t& acc1) {
 #pragma unroll
@@ -523,12 +555,14 @@ __device__ __forceinline__ void piece16_exp(const uint32_t (&r)[16], uint64_t sc
     const float e1 = ex2_approx(t1);
     if (c & 1) acc1 = f2_add(acc1, f2_pack(e0, e1));
     else acc0 = f2_add(acc0, f2_pack(e0, e1));
-    pk[c] = pack_f16x2(e0, e1);
+    pk[c] = kBf16 ? pack_bf16x2(e0, e1) : pack_f16x2(e0, e1);
   }
 }
 
 // Rare path: the reference max grew inside a block after `npieces` 16-key
-// pieces of P were already written (fp16, 8 columns each): scale them by f.
+// pieces of P were already written (fp16, or bf16 when kBf16; 8 columns
+// each): scale them by f.
+template <bool kBf16>
 __device__ __noinline__ void rescale_p(uint32_t s_addr, int npieces, float f) {
   tmem_wait_st();
   for (int i = 0; i < npieces; ++i) {
@@ -537,8 +571,12 @@ __device__ __noinline__ void rescale_p(uint32_t s_addr, int npieces, float f) {
     tmem_wait_ld();
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
-      const float2 v = __half22float2(*reinterpret_cast<const __half2*>(&t[j]));
-      t[j] = pack_f16x2(v.x * f, v.y * f);
+      if (kBf16) {
+        t[j] = pack_bf16x2(__uint_as_float(t[j] << 16) * f, __uint_as_float(t[j] & 0xFFFF0000u) * f);
+      } else {
+        const float2 v = __half22float2(*reinterpret_cast<const __half2*>(&t[j]));
+        t[j] = pack_f16x2(v.x * f, v.y * f);
+      }
     }
     tmem_st8(s_addr + 8 * i, t);
   }
@@ -584,6 +622,7 @@ __device__ __forceinline__ void store16(const FwdParams& p, size_t row, int c0, 
 // already written and, after the previous P.V has landed, O are rescaled),
 // exponentials, fp16 P written over the S columns already read (16 keys = 8
 // columns per piece) -- then the block goes to the MMA.
+template <bool kBf16>
 __device__ void softmax_role(SharedStorage& s, const FwdParams& p, uint32_t tmem) {
   const int tid = threadIdx.x;  // 0..127 == TMEM lane
   const int warp = tid >> 5;
@@ -642,11 +681,11 @@ __device__ void softmax_role(SharedStorage& s, const FwdParams& p, uint32_t tmem
             acc0 = f2_fma(acc0, f2, 0ull);
             acc1 = f2_fma(acc1, f2, 0ull);
             o_factor *= f;
-            if (q > 0 && __any_sync(0xffffffffu, f != 1.f)) rescale_p(s_addr, q, f);
+            if (q > 0 && __any_sync(0xffffffffu, f != 1.f)) rescale_p<kBf16>(s_addr, q, f);
           }
           const float o = off_s - m_ref;
           uint32_t pk[8];
-          piece16_exp(cur, scale2, f2_pack(o, o), pk, acc0, acc1);
+          piece16_exp<kBf16>(cur, scale2, f2_pack(o, o), pk, acc0, acc1);
           if (q < 3) tmem_wait_ld();
           tmem_st8(s_addr + 8 * q, pk);
         }
@@ -713,6 +752,10 @@ __device__ void softmax_role(SharedStorage& s, const FwdParams& p, uint32_t tmem
   }
 }
 
+// kBf16 = false: the fp16 instance (every call). kBf16 = true: the bf16
+// instance, launched behind it as its programmatic dependent, which does the
+// call again only when the fp16 instance saw a V value fp16 cannot represent.
+template <bool kBf16>
 __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 bigbird_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
@@ -720,6 +763,16 @@ bigbird_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
   SharedStorage& s = *reinterpret_cast<SharedStorage*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  if (kBf16) {
+    // Wait until the fp16 instance has completed (its writes visible), then
+    // do the call again only if it set the flag.
+    asm volatile("griddepcontrol.launch_dependents;");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    if (threadIdx.x == 0) s.abort_flag = *reinterpret_cast<volatile int*>(&p.counters[kCtrBigV]);
+    __syncthreads();
+    if (s.abort_flag == 0) return;
+    __syncthreads();
+  }
   if (warp == 5) {
     tmem_alloc(smem_u32(&s.tmem_base), kTmemCols);
     tmem_relinquish();
@@ -748,8 +801,9 @@ bigbird_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     s.abort_flag = 0;
     fence_barrier_init();
   }
-  // Dependent grids (the merge) may launch now; they wait for this grid's completion.
-  asm volatile("griddepcontrol.launch_dependents;");
+  // Dependent grids (the bf16 instance, the merge) may launch now; they wait
+  // for this grid's completion.
+  if (!kBf16) asm volatile("griddepcontrol.launch_dependents;");
   if (warp == 4 && lane == 0) {
     tma_prefetch_desc(&tmQ);
     tma_prefetch_desc(&tmK);
@@ -761,15 +815,15 @@ bigbird_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
   const uint32_t tmem = s.tmem_base;
 
   if (warp < 4) {
-    softmax_role(s, p, tmem);
+    softmax_role<kBf16>(s, p, tmem);
   } else if (warp == 4) {
     producer_role(s, p, &tmQ, &tmK, &tmV);
   } else if (warp == 5) {
-    if (lane == 0) mma_role(s, p, tmem);
+    if (lane == 0) mma_role<kBf16>(s, p, tmem);
   } else if (warp == 6) {
     prep_role(s, p);
   } else {
-    convert_role(s, p);
+    convert_role<kBf16>(s, p);
   }
   tc_fence_before();
   __syncthreads();
@@ -777,6 +831,17 @@ bigbird_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
   if (warp == 5) {
     __syncwarp();
     tmem_dealloc(tmem, kTmemCols);
+  }
+  // The CTA that finishes last puts the workspace counters back to zero for
+  // the next call (every other CTA is done with them).
+  // (The flag is left for the bf16 instance, which clears it when it runs.)
+  if (threadIdx.x == 0) {
+    __threadfence();
+    if (atomicAdd(&p.counters[kCtrDone], 1) == static_cast<int>(gridDim.x) - 1) {
+      p.counters[kCtrTickets] = 0;
+      p.counters[kCtrDone] = 0;
+      if (kBf16) p.counters[kCtrBigV] = 0;
+    }
   }
 }
 
@@ -889,11 +954,13 @@ static DeviceInfo* device_info(int dev) {
     di.sms = sms;
     if (di.ok) {
       const int smem = static_cast<int>(sizeof(SharedStorage) + 1024);
-      if (cudaFuncSetAttribute(bigbird_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-        return nullptr;
       // Four CTAs per SM need the largest shared-memory carve-out.
-      if (cudaFuncSetAttribute(bigbird_fwd_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100) != cudaSuccess)
-        return nullptr;
+      for (const void* fn : {reinterpret_cast<const void*>(bigbird_fwd_kernel<false>),
+                             reinterpret_cast<const void*>(bigbird_fwd_kernel<true>)}) {
+        if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) return nullptr;
+        if (cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout, 100) != cudaSuccess)
+          return nullptr;
+      }
       if (cudaGetSymbolAddress(reinterpret_cast<void**>(&di.status), g_status) != cudaSuccess) return nullptr;
     }
     di.attr_set = true;
@@ -908,7 +975,6 @@ uint32_t* status_word(int dev) {
   return di && di->ok ? di->status : nullptr;
 }
 
-constexpr size_t kSchedBytes = 256;  // the scheduling counter's slot at the start of the workspace
 
 struct Plan {
   int nb = 0;
@@ -932,9 +998,10 @@ static int make_plan(int B, int H, int L, int d, int block, int r, unsigned flag
     pl.split_blocks = pl.nb;  // nb <= 5 + 2r <= kMaxList
     pl.nsplit = 1;
   }
-  // Workspace: the unit-ticket counter, then (split global rows only) the
-  // partial outputs [B*H, nsplit, 128, 64] and their (max, sum) [B*H, nsplit, 128, 2].
-  pl.ws_bytes = kSchedBytes;
+  // Workspace: the counters (unit tickets, finished CTAs, the bf16 flag),
+  // then (split global rows only) the partial outputs [B*H, nsplit, 128, 64]
+  // and their (max, sum) [B*H, nsplit, 128, 2].
+  pl.ws_bytes = kCounterBytes;
   if (pl.nsplit > 1)
     pl.ws_bytes += static_cast<size_t>(B) * H * pl.nsplit * kRows * (kHeadDim + 2) * sizeof(float);
   return BB_OK;
@@ -1027,34 +1094,46 @@ static int fwd_impl(const void* q, const void* k, const void* v, const int32_t* 
   if (!ws) {
     if (cudaMallocAsync(&ws, pl.ws_bytes, stream) != cudaSuccess) return BB_ERR_CUDA;
     owned = true;
+    // a fresh workspace's counters start at zero
+    if (cudaMemsetAsync(ws, 0, kCounterBytes, stream) != cudaSuccess) {
+      cudaFreeAsync(ws, stream);
+      return BB_ERR_CUDA;
+    }
   }
-  p.sched = static_cast<int*>(ws);
+  p.counters = static_cast<int*>(ws);
   if (pl.nsplit > 1) {
-    p.part_o = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + kSchedBytes);
+    p.part_o = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + kCounterBytes);
     p.part_ml = p.part_o + static_cast<size_t>(p.BH) * pl.nsplit * kRows * kHeadDim;
   }
-  // Unit tickets start from zero on every call.
-  if (cudaMemsetAsync(p.sched, 0, sizeof(int), stream) != cudaSuccess) {
-    if (owned) cudaFreeAsync(ws, stream);
-    return BB_ERR_CUDA;
-  }
 
+  // The fp16 instance, then the bf16 instance and the merge, each a
+  // programmatic dependent of the kernel before it: launched while its
+  // predecessor runs, it waits (griddepcontrol.wait) for the predecessor's
+  // completion before it reads what that grid wrote, which hides the launch
+  // gaps.
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
   const int grid = std::min(p.total_units, kCtasPerSm * di->sms);
   const size_t smem = sizeof(SharedStorage) + 1024;
-  bigbird_fwd_kernel<<<grid, kThreads, smem, stream>>>(tq, tk, tv, p);
+  bigbird_fwd_kernel<false><<<grid, kThreads, smem, stream>>>(tq, tk, tv, p);
   cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess) {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, bigbird_fwd_kernel<true>, tq, tk, tv, p);
+  }
   if (e == cudaSuccess && pl.nsplit > 1) {
-    // Programmatic dependent launch: the merge grid is launched while the
-    // attention kernel runs and waits (griddepcontrol.wait) for its completion,
-    // which hides the launch gap between the two.
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3(p.BH, kRows / kMergeRowsPerCta);
     cfg.blockDim = dim3(256);
     cfg.dynamicSmemBytes = 0;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     e = cudaLaunchKernelEx(&cfg, bigbird_merge_kernel, static_cast<const float*>(p.part_o),
@@ -1158,6 +1237,10 @@ extern "C" int bigbird_attn_fwd_noalloc(const void* q, const void* k, const void
   if (cudaGetDevice(&dev) != cudaSuccess) return BB_ERR_CUDA;
   void* scratch = bb::static_scratch_address(dev);
   if (!scratch) return BB_ERR_CUDA;
+  // The region keeps whatever the previous call left; the counters must start
+  // at zero (a call that completes leaves them so, one that gave up may not).
+  if (cudaMemsetAsync(scratch, 0, bb::kCounterBytes, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return BB_ERR_CUDA;
   return bigbird_attn_fwd_ex(q, k, v, rand_attn, seq_mask, out, B, H, L, d, block, r, out_dtype, flags, scratch,
                              bb::kStaticScratchBytes, stream);
 }

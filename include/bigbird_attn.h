@@ -82,22 +82,36 @@ enum {
  *   stream     cudaStream_t.
  * Errors: BB_ERR_INVALID_ARG for L % block != 0 [HF-Pegasus, section
  * "序列长度的块对齐要求"] or r < 1 [HF-Pegasus, section "使用限制与注意事项"];
- * BB_ERR_UNSUPPORTED for other d/block or misalignment. Scratch memory for
- * the split global rows, when needed, is taken with cudaMallocAsync on
- * `stream` and released the same way.
+ * BB_ERR_UNSUPPORTED for other d/block or misalignment. Every finite bf16
+ * value is taken. For d = block = 64, P.V runs in fp16 (P and V converted in
+ * shared memory); when V holds a value of magnitude >= 65536, which fp16
+ * cannot represent, the call is done again with bf16 P and V (8 significant
+ * bits of P instead of 11), which about doubles its time. A call launches the
+ * fp16 kernel, then its bf16 instance (which returns at once unless that
+ * recompute is needed) and, when the global rows are split into key ranges,
+ * the merge of the ranges, each a programmatic dependent of the one before.
+ * The workspace (the work-unit counters and,
+ * for split global rows, their partial results; see
+ * bigbird_attn_workspace_size) is taken with cudaMallocAsync on `stream`,
+ * zeroed with cudaMemsetAsync and released with cudaFreeAsync: callers that
+ * must not allocate use bigbird_attn_fwd_ex with their own workspace, or
+ * bigbird_attn_fwd_noalloc.
  */
 int bigbird_attn_fwd(const void* q, const void* k, const void* v, const int32_t* rand_attn,
                      const uint8_t* seq_mask, void* out, int B, int H, int L, int d, int block, int r,
                      void* stream);
 
 /*
- * Bytes of device scratch bigbird_attn_fwd_ex needs for these sizes and
+ * Bytes of device workspace bigbird_attn_fwd_ex needs for these sizes and
  * flags (0 if the sizes are invalid, and for the sizes the CUDA-core kernel
- * runs, which need none). For d = block = 64 the scratch starts with a 256-byte slot
- * for the counter through which the CTAs share out the work units (every call
- * zeroes it with cudaMemsetAsync on its stream before the launch); when the
- * global rows are split into key ranges (sparse pattern, nb > 8) it also holds
- * each range's partial result (unnormalised output, running max, running sum).
+ * runs, which need none). For d = block = 64 it starts with 256 bytes of
+ * counters: the one through which the CTAs share out the work units, one that
+ * finds the CTA finishing last (which sets the counters back to zero), and
+ * the flag that asks for the bf16 recompute (cleared by the bf16 instance when
+ * it runs). When the global rows are split into key ranges (sparse pattern:
+ * ranges of 8 key blocks) each range's partial result follows (output
+ * normalised by its own sum, running max, running sum), merged by
+ * log-sum-exp in a separate kernel.
  */
 size_t bigbird_attn_workspace_size(int B, int H, int L, int d, int block, int r, unsigned flags);
 
@@ -107,10 +121,13 @@ size_t bigbird_attn_workspace_size(int B, int H, int L, int d, int block, int r,
  *   out_dtype  BB_OUT_BF16 (out is bf16) or BB_OUT_F32 (out is fp32 [B,H,L,d]).
  *   flags      BB_FLAG_* bits.
  *   workspace  device, 256-byte aligned, at least
- *              bigbird_attn_workspace_size(...) bytes; NULL = allocate with
- *              cudaMallocAsync on `stream` (freed with cudaFreeAsync after
- *              the launch). Its contents need no initialisation. Calls that
- *              share a workspace must not overlap on the GPU.
+ *              bigbird_attn_workspace_size(...) bytes, zero-filled before
+ *              its first use; every call that completes leaves its counters
+ *              at zero again, so a workspace is reused without clearing it.
+ *              NULL = allocate and zero one with cudaMallocAsync /
+ *              cudaMemsetAsync on `stream` (freed with cudaFreeAsync after
+ *              the launch). Calls that share a workspace must not overlap on
+ *              the GPU.
  */
 int bigbird_attn_fwd_ex(const void* q, const void* k, const void* v, const int32_t* rand_attn,
                         const uint8_t* seq_mask, void* out, int B, int H, int L, int d, int block, int r,
@@ -267,6 +284,11 @@ int bigbird_pattern_table(const int32_t* host_ra, int H, int L, int block, int r
  * after synchronising `stream`. Bit 1: a rand_attn entry outside [0, nb) was
  * skipped; bit 2: a kernel wait timed out (a lost completion). *host_status
  * receives the word. Returns BB_OK, or BB_ERR_CUDA if the copy failed.
+ * The word is one per device and process: every call of every entry point,
+ * on any stream and from any host thread, ORs its bits into the same word,
+ * and a read clears the bits of all of them. Read it where no other work of
+ * this library is in flight on the device, or attribute its bits to all the
+ * calls since the previous read.
  */
 int bigbird_device_status(void* stream, uint32_t* host_status);
 
@@ -277,9 +299,10 @@ int bigbird_device_status(void* stream, uint32_t* host_status);
  * real-time loop that reserves all GPU memory at start-up and must not hit the
  * allocator, or its device-wide synchronisation, inside a step.)
  *
- * The scratch for the split global rows comes from a fixed region of
- * bigbird_attn_noalloc_scratch_bytes() bytes (32 MiB) that the library's module
- * holds on every GPU that loads it, until the process exits. Arguments and
+ * The workspace (counters and the split global rows' partial results) comes
+ * from a fixed region of bigbird_attn_noalloc_scratch_bytes() bytes (32 MiB)
+ * that the library's module holds on every GPU that loads it, until the
+ * process exits. Arguments and
  * results are those of bigbird_attn_fwd_ex, except:
  *   - there is no workspace argument;
  *   - a problem whose scratch need (bigbird_attn_workspace_size) exceeds the
@@ -289,9 +312,11 @@ int bigbird_device_status(void* stream, uint32_t* host_status);
  *     host buffer).
  * The first call on a device looks up the region's device address (once per
  * device, with that device current); make that first call before any stream
- * capture. All calls share the one region and every call rewrites what it
- * uses (nothing needs to start at zero): calls that overlap on the GPU -- on
- * different streams, or from different threads -- race on it.
+ * capture. All calls share the one region, which keeps what the previous
+ * call left: each call first clears the counters at its start with
+ * cudaMemsetAsync on `stream` (the partial results are rewritten before they
+ * are read). Calls that overlap on the GPU -- on different streams, or from
+ * different threads -- race on the region.
  */
 int bigbird_attn_fwd_noalloc(const void* q, const void* k, const void* v, const int32_t* rand_attn,
                              const uint8_t* seq_mask, void* out, int B, int H, int L, int d, int block, int r,

@@ -219,6 +219,54 @@ def test_max_growth_inside_and_across_blocks():
     _check(got, want, "growth")
 
 
+@pytest.mark.parametrize("vmax", [65280.0, 1.0e5, 1.0e20], ids=["fp16_edge", "1e5", "1e20"])
+@pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])
+def test_v_beyond_fp16_range(vmax, out_dtype):
+    """One key block of V scaled so its largest magnitude is vmax: 65280 is the
+    largest bf16 value fp16 still holds, 1e5 and 1e20 are not representable in
+    fp16 (P.V of that tile then runs in bf16). Pair unit (5, 6) shares every
+    MMA between a half that attends to block 4 (window of 5) and one that does
+    not (window of 6), so the second half must be untouched.
+
+    Bars: rows that do not attend to block 4 at the forward's bar (max 1e-2,
+    mean 1e-3) and finite. Rows that do: attention is linear in V, and the
+    large tile's weights are rounded once to 16 bits (bf16: relative 2^-9) and,
+    with bf16 output, the output once more (2^-9 of |out| <= the same scale),
+    so |err| <= 1e-2 + 2^-7 * mass4 * max|v4|, mass4 = the row's attention
+    weight on block 4 (the oracle's output for V = 1 on block 4, 0 elsewhere)."""
+    w = Workload("bigv", 1, 2, 16 * 64, pad=("fixed", [1000]), seed=19)
+    j = 4
+    inp = make_inputs(w)
+    ra_c, ra_o = _rand_attn_pair(w)
+    for h in range(w.H):  # keep block 4 out of query block 6's random blocks
+        row = list(ra_o[h, 5])
+        if j in row:
+            row[row.index(j)] = [x for x in range(1, w.nb - 1) if x not in (5, 6, 7, j) and x not in row][0]
+            ra_o[h, 5] = row
+    assert bb.rand_attn_validate(ra_o, w.H, w.L, w.block, w.r) == bb.BB_OK
+    ra_c = ra_o.copy()
+    v = inp["v"].clone()
+    big = torch.randn(w.B, w.H, 64, 64, generator=torch.Generator().manual_seed(5))
+    v[:, :, j * 64:(j + 1) * 64] = (big / big.abs().max() * vmax).to(torch.bfloat16)
+    inp = dict(inp, v=v)
+    got = _cuda_fwd(inp, w, ra_c, out_dtype)
+    assert np.isfinite(got).all()
+    want = oracle.attention(inp["q"], inp["k"], v, ra_o, inp["seq_mask"], w.block, w.r)
+    ind = np.zeros(v.shape, np.float64)
+    ind[:, :, j * 64:(j + 1) * 64] = 1.0
+    mass = oracle.attention(inp["q"], inp["k"], ind, ra_o, inp["seq_mask"], w.block, w.r)[..., :1]
+    vmax4 = float(v[:, :, j * 64:(j + 1) * 64].float().abs().max())
+    err = np.abs(got.astype(np.float64) - want)
+    for h in range(w.H):
+        bm = oracle.block_mask(w.nb, w.r, ra_o[h], True)
+        attends = np.repeat(bm[:, j], 64)          # per query row
+        assert not attends[6 * 64] and attends[5 * 64], "pair (5, 6) must split on block 4"
+        e_off = err[0, h, ~attends]
+        assert e_off.max() <= MAX_ABS and e_off.mean() <= MEAN_ABS, (h, float(e_off.max()))
+        bar = 1e-2 + 2.0 ** -7 * mass[0, h, attends] * vmax4
+        assert (err[0, h, attends] <= bar).all(), (h, float((err[0, h, attends] / bar).max()))
+
+
 def test_out_of_range_rand_attn_is_flagged():
     w = Workload("oor", 1, 1, 16 * 64, seed=18)
     inp = make_inputs(w)

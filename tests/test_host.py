@@ -111,11 +111,13 @@ def test_fallback_rule_matches_oracle():
 
 
 def test_workspace_size():
-    sched = 256  # the work-unit counter's slot
-    assert bb.workspace_size(1, 2, 704) == sched  # fallback: no split rows
+    head = 256  # unit-ticket, finished-CTA and bf16-recompute counters
+    assert bb.workspace_size(1, 2, 704) == head  # fallback: no split rows
     nb = 4096 // 64
-    nsplit = (nb + 7) // 8
-    assert bb.workspace_size(4, 12, 4096) == sched + 4 * 12 * nsplit * 128 * 66 * 4
+    nsplit = (nb + 7) // 8  # global rows split into ranges of 8 key blocks
+    assert bb.workspace_size(4, 12, 4096) == head + 4 * 12 * nsplit * 128 * 66 * 4
+    nb = 125  # a ragged last range
+    assert bb.workspace_size(1, 3, nb * 64) == head + 3 * ((nb + 7) // 8) * 128 * 66 * 4
     assert bb.workspace_size(1, 1, 1000) == 0  # invalid sizes
 
 
