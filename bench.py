@@ -36,7 +36,10 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one forward
 # kernel launch per workload, from an ncu capture of the current kernel
 # source; an entry is removed whenever the kernel changes.
-FWD_DRAM_BYTES_PER_LAUNCH: dict = {}
+FWD_DRAM_BYTES_PER_LAUNCH: dict = {
+    # 77.85 MB read + 7.93 MB written, fp16 instance, one launch
+    "bigbird_base_l4096": 85.785344e6,
+}
 
 
 def _peaks():
