@@ -36,10 +36,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one forward
 # kernel launch per workload, from an ncu capture of the current kernel
 # source; an entry is removed whenever the kernel changes.
-FWD_DRAM_BYTES_PER_LAUNCH: dict = {
-    # 77.85 MB read + 7.93 MB written, fp16 instance, one launch
-    "bigbird_base_l4096": 85.785344e6,
-}
+FWD_DRAM_BYTES_PER_LAUNCH: dict = {}
 
 
 def _peaks():
@@ -333,13 +330,13 @@ def run_cuda(args):
     e2e_value = flops * world / (e2e_ms * 1e-3) / 1e12
     peaks, src = _peaks()
     achieved = flops / (ms * 1e-3) / 1e12
-    generic = (w.block, w.d) != (64, 64)
     # The tensor-core path launches the fp16 attention kernel and its bf16
     # instance (which returns at once unless V holds a value fp16 cannot
     # represent), plus the global-row merge when the global rows are split
-    # into key ranges (the workspace then holds more than its counters); the
-    # CUDA-core path launches one kernel.
+    # into key ranges (the workspace then holds more than its counters). It is
+    # the path that takes a workspace; the CUDA-core path launches one kernel.
     ws_bytes = bb.workspace_size(w.B, w.H, w.L, w.d, w.block, w.r)
+    generic = ws_bytes == 0
     launches_per_call = 1 if generic else (3 if ws_bytes > 256 else 2)
     if generic:
         # the CUDA-core kernel: fp32 peak from unit counts and clocks

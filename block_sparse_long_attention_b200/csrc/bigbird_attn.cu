@@ -70,14 +70,14 @@
 
 namespace bb {
 
-constexpr int kBlock = 64;             // tokens per block
+constexpr int kBlock = 64;             // tokens per tile: a block of 64, or half a block of 128
 constexpr int kHeadDim = 64;           // head dimension
-constexpr int kRows = 128;             // query rows per unit (two blocks)
+constexpr int kRows = 128;             // query rows per unit (two tiles)
 constexpr int kKStages = 2;            // K ring depth (blocks)
 constexpr int kVStages = 2;            // V ring depth (blocks)
-constexpr int kMaxList = 40;           // key blocks per unit
+constexpr int kMaxList = 42;           // key tiles per unit
 constexpr int kMaxR = 16;              // random blocks per row supported
-constexpr int kSplitBlocks = 8;        // key blocks per global-row range
+constexpr int kSplitBlocks = 8;        // key tiles per global-row range
 constexpr int kThreads = 256;
 constexpr int kCtasPerSm = 4;          // four independent unit pipelines per SM
 constexpr uint32_t kTileBytes = kBlock * kHeadDim * 2;  // one 64x64 bf16 tile
@@ -106,12 +106,15 @@ constexpr uint32_t kStatusTimeout = 2u;
 
 __device__ uint32_t g_status;
 
+// Everything below is counted in 64-token tiles: a block of 64 is one tile, a
+// block of 128 two. A unit is 128 query rows (two tiles) against a list of key
+// tiles.
 struct UnitInfo {
-  int32_t n;     // key blocks in the list
+  int32_t n;     // key tiles in the list
   int32_t bh;    // b * H + h
-  int32_t qtop;  // query block of rows 0..63
-  int32_t qbot;  // query block of rows 64..127, or -1
-  int32_t split; // key range index of a partial global unit, or -1
+  int32_t qtop;  // query tile of rows 0..63
+  int32_t qbot;  // query tile of rows 64..127, or -1
+  int32_t split; // partial-result slot of a split global unit (global unit * nsplit + range), or -1
   int32_t stop;  // 1: no more units for this CTA (every role leaves its loop)
   int32_t kb[kMaxList];
   uint64_t vm[kMaxList];  // bit c set: key c of the block is valid
@@ -126,16 +129,20 @@ struct FwdParams {
   const uint8_t* seq_mask;
   void* out;
   float* lse;      // [B*H*L] natural-log log-sum-exp of each row's scores, or null
-  float* part_o;   // [BH, nsplit, 128, 64]
-  float* part_ml;  // [BH, nsplit, 128, 2]
+  float* part_o;   // [BH, nparts, 128, 64]
+  float* part_ml;  // [BH, nparts, 128, 2]
   uint32_t* status;
   int* counters;    // workspace counters (zero at launch; the last CTA resets them)
   int B, H, L, nb, r, BH;
+  int nt;            // 64-token tiles per sequence (L / 64)
+  int bt;            // tiles per block: 1 (block 64) or 2 (block 128)
   int sparse;
   int nsplit;        // key ranges per global unit (1 = write the output directly)
-  int split_blocks;  // key blocks per range
-  int n_pair_units;  // pair units come first (they are the longer ones)
-  int n_pairs;       // pair units per head
+  int split_tiles;   // key tiles per range
+  int n_glob;        // global units per range: 1 (blocks 0 and nb-1 stacked) or 2 (one per global block)
+  int nparts;        // n_glob * nsplit
+  int n_pair_units;  // middle units come first (they are the longer ones)
+  int n_pairs;       // middle units per head
   int total_units;
   int out_f32;
   float scale_log2;  // log2(e) / sqrt(d)
@@ -176,76 +183,123 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity) {
   return __all_sync(0xffffffffu, mbar_wait(bar, parity));
 }
 
-// Decode unit u and build its key-block list. Called by a whole warp: the
+// Decode unit u and build its key-tile list. Called by a whole warp: the
 // lanes fetch the unit's random entries in parallel, lane 0 builds the list.
+// Units, in order (longest first):
+//   * middle units: with block 64, query blocks (i, i+1) for i = 1, 3, ...
+//     (the last alone when nb - 2 is odd) against the union of their key
+//     blocks, a half mask per tile telling which rows use it; with block 128,
+//     query block i (its two tiles) against its own key blocks. The key
+//     blocks of query block i: window i-1, i, i+1, the global blocks 0 and
+//     nb-1 and rand_attn[h][i-1] [TFG-BigBird, section "BigBird：从二次方注意力到线性稀疏注意力"
+//     and "随机块掩码是如何生成的"; HF-Pegasus, section "三类注意力组合"];
+//   * global units: the rows of query blocks 0 and nb-1 (which attend to
+//     every key) against one range of split_tiles key tiles -- both blocks in
+//     one unit with block 64, one unit per block with block 128;
+//   * full-attention fallback: query tiles (2j, 2j+1) against every key tile.
 __device__ void build_unit(const FwdParams& p, int u, UnitInfo& ui, int lane) {
   int n = 0;
-  auto add = [&](int kb, int hm) {
+  // one key tile, merging the half masks of a tile listed twice (set semantics)
+  auto add_tile = [&](int kt, int hm) {
+    for (int e = 0; e < n; ++e)
+      if (ui.kb[e] == kt) {
+        ui.hm[e] |= static_cast<uint8_t>(hm);
+        return;
+      }
+    ui.kb[n] = kt;
+    ui.hm[n] = static_cast<uint8_t>(hm);
+    ++n;
+  };
+  // one key block of the pattern (its bt tiles); an entry outside [0, nb) is
+  // skipped and reported
+  auto add_block = [&](int kb, int hm) {
     if (kb < 0 || kb >= p.nb) {
       atomicOr(p.status, kStatusBadRandAttn);
       return;
     }
-    for (int e = 0; e < n; ++e)
-      if (ui.kb[e] == kb) {
-        ui.hm[e] |= static_cast<uint8_t>(hm);
-        return;
-      }
-    ui.kb[n] = kb;
-    ui.hm[n] = static_cast<uint8_t>(hm);
-    ++n;
+    for (int t = 0; t < p.bt; ++t) add_tile(kb * p.bt + t, hm);
   };
   if (u >= p.n_pair_units) {
     u -= p.n_pair_units;
-    int bh, s, qtop, qbot;
+    int bh, s, qtop, qbot, part;
     if (p.sparse) {
-      bh = u / p.nsplit;
-      s = u % p.nsplit;
-      qtop = 0;
-      qbot = p.nb - 1;
+      bh = u / p.nparts;
+      part = u % p.nparts;
+      const int g = part / p.nsplit;  // global unit within the range
+      s = part % p.nsplit;
+      if (p.n_glob == 1) {
+        qtop = 0;
+        qbot = p.nt - 1;
+      } else {
+        qtop = g == 0 ? 0 : p.nt - 2;
+        qbot = qtop + 1;
+      }
     } else {
-      const int npair = (p.nb + 1) / 2;
+      const int npair = (p.nt + 1) / 2;
       bh = u / (npair * p.nsplit);
       const int rem = u % (npair * p.nsplit);
       const int pp = rem / p.nsplit;
       s = rem % p.nsplit;
+      part = s;
       qtop = 2 * pp;
-      qbot = 2 * pp + 1 < p.nb ? 2 * pp + 1 : -1;
+      qbot = 2 * pp + 1 < p.nt ? 2 * pp + 1 : -1;
     }
     if (lane == 0) {
-      const int k0 = s * p.split_blocks;
-      const int k1 = min(p.nb, k0 + p.split_blocks);
-      for (int kb = k0; kb < k1; ++kb) add(kb, 3);
+      const int k0 = s * p.split_tiles;
+      const int k1 = min(p.nt, k0 + p.split_tiles);
+      for (int kt = k0; kt < k1; ++kt) add_tile(kt, 3);
       ui.bh = bh;
       ui.qtop = qtop;
       ui.qbot = qbot;
-      ui.split = p.nsplit > 1 ? s : -1;
+      ui.split = p.nsplit > 1 ? part : -1;
       ui.n = n;
       ui.stop = 0;
     }
   } else {
-    const int v = u;
-    const int bh = v / p.n_pairs;
-    const int pp = v % p.n_pairs;
-    const int qtop = 1 + 2 * pp;
-    const int qbot = (2 + 2 * pp <= p.nb - 2) ? 2 + 2 * pp : -1;
+    const int bh = u / p.n_pairs;
+    const int pp = u % p.n_pairs;
     const int h = bh % p.H;
-    const int both = qbot >= 0 ? 3 : 1;
-    // rand_attn rows qtop-1 and qtop (= qbot-1) are adjacent: lane t < r reads
-    // the top row's entry t, lane r + t the bottom row's entry t.
-    const int nrand = qbot >= 0 ? 2 * p.r : p.r;
-    const int32_t* ra = p.rand_attn + (static_cast<size_t>(h) * (p.nb - 2) + (qtop - 1)) * p.r;
-    const int rv = lane < nrand ? __ldg(ra + lane) : -1;
-    if (lane == 0) {
-      add(qtop - 1, 1);
-      add(qtop, both);
-      add(qtop + 1, both);
-      if (qbot >= 0) add(qtop + 2, 2);
-      add(0, both);
-      add(p.nb - 1, both);
-    }
-    for (int t = 0; t < nrand; ++t) {
-      const int x = __shfl_sync(0xffffffffu, rv, t);
-      if (lane == 0) add(x, t < p.r ? 1 : 2);
+    int qtop, qbot;
+    if (p.bt == 1) {
+      const int i = 1 + 2 * pp;  // query blocks i and i + 1 (if still a middle block)
+      const bool pair = i + 1 <= p.nb - 2;
+      const int both = pair ? 3 : 1;
+      // rand_attn rows i-1 and i are adjacent: lane t < r reads the top
+      // row's entry t, lane r + t the bottom row's entry t.
+      const int nrand = pair ? 2 * p.r : p.r;
+      const int32_t* ra = p.rand_attn + (static_cast<size_t>(h) * (p.nb - 2) + (i - 1)) * p.r;
+      const int rv = lane < nrand ? __ldg(ra + lane) : -1;
+      if (lane == 0) {
+        add_block(i - 1, 1);
+        add_block(i, both);
+        add_block(i + 1, both);
+        if (pair) add_block(i + 2, 2);
+        add_block(0, both);
+        add_block(p.nb - 1, both);
+      }
+      for (int t = 0; t < nrand; ++t) {
+        const int x = __shfl_sync(0xffffffffu, rv, t);
+        if (lane == 0) add_block(x, t < p.r ? 1 : 2);
+      }
+      qtop = i;
+      qbot = pair ? i + 1 : -1;
+    } else {
+      const int i = 1 + pp;  // query block i: tiles 2i and 2i + 1, both using every key block
+      const int32_t* ra = p.rand_attn + (static_cast<size_t>(h) * (p.nb - 2) + (i - 1)) * p.r;
+      const int rv = lane < p.r ? __ldg(ra + lane) : -1;
+      if (lane == 0) {
+        add_block(i - 1, 3);
+        add_block(i, 3);
+        add_block(i + 1, 3);
+        add_block(0, 3);
+        add_block(p.nb - 1, 3);
+      }
+      for (int t = 0; t < p.r; ++t) {
+        const int x = __shfl_sync(0xffffffffu, rv, t);
+        if (lane == 0) add_block(x, 3);
+      }
+      qtop = 2 * i;
+      qbot = 2 * i + 1;
     }
     if (lane == 0) {
       ui.bh = bh;
@@ -258,7 +312,7 @@ __device__ void build_unit(const FwdParams& p, int u, UnitInfo& ui, int lane) {
   }
 }
 
-// 64 validity bits of key block kb of batch b (bit c: seq_mask of key c != 0).
+// 64 validity bits of key tile kb of batch b (bit c: seq_mask of key c != 0).
 __device__ __forceinline__ uint64_t key_valid_bits(const uint8_t* seq_mask, int L, int b, int kb) {
   const uint4* src = reinterpret_cast<const uint4*>(seq_mask + static_cast<size_t>(b) * L + static_cast<size_t>(kb) * kBlock);
   uint64_t bits = 0;
@@ -720,7 +774,7 @@ __device__ void softmax_role(SharedStorage& s, const FwdParams& p, uint32_t tmem
     if (!warp_wait(smem_u32(&s.o_full), ut & 1)) { flag_timeout(s, p); return; }
     tc_fence_after();
     if (split >= 0) {
-      const size_t base = (static_cast<size_t>(bh) * p.nsplit + split) * kRows + tid;
+      const size_t base = (static_cast<size_t>(bh) * p.nparts + split) * kRows + tid;
 #pragma unroll 1
       for (int c0 = 0; c0 < kHeadDim; c0 += 16) {
         uint32_t o[16];
@@ -847,19 +901,20 @@ bigbird_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
 
 // Combine the partial results of the key ranges of the global rows by
 // log-sum-exp (log2 units). 16 threads per query row, 4 columns each; a CTA
-// covers 16 rows, grid = (B*H, 128 / 16).
+// covers 16 rows of one global unit, grid = (B*H*n_glob, 128 / 16).
 constexpr int kMergeRowsPerCta = 16;
 
 __global__ void __launch_bounds__(256)
 bigbird_merge_kernel(const float* __restrict__ part_o, const float* __restrict__ part_ml, void* out, float* lse,
-                     int nsplit, int L, int nb, int out_f32) {
+                     int nsplit, int n_glob, int L, int nt, int out_f32) {
   // Launched as a programmatic dependent of the attention kernel: wait until
   // that grid has completed and its partials are visible.
   asm volatile("griddepcontrol.wait;" ::: "memory");
-  const int bh = blockIdx.x;
+  const int bh = blockIdx.x / n_glob;
+  const int g = blockIdx.x % n_glob;  // global unit: its partials follow those of unit g - 1
   const int row = blockIdx.y * kMergeRowsPerCta + (threadIdx.x >> 4);
   const int c4 = threadIdx.x & 15;
-  const size_t base = static_cast<size_t>(bh) * nsplit * kRows + row;
+  const size_t base = (static_cast<size_t>(bh) * n_glob + g) * nsplit * kRows + row;
   const float2* ml = reinterpret_cast<const float2*>(part_ml);
   float mmax = kNegInit;
   for (int s = 0; s < nsplit; ++s) mmax = fmaxf(mmax, __ldg(&ml[base + static_cast<size_t>(s) * kRows].x));
@@ -877,8 +932,10 @@ bigbird_merge_kernel(const float* __restrict__ part_o, const float* __restrict__
     acc.w += w * t.w;
   }
   const float inv = 1.f / l;
-  const int qblk = row < kBlock ? 0 : nb - 1;
-  const size_t orow = static_cast<size_t>(bh) * L + static_cast<size_t>(qblk) * kBlock + (row & (kBlock - 1));
+  // rows 0..63 and 64..127 of the unit: tiles 0 and nt-1 (block 64: blocks 0
+  // and nb-1 stacked), or the two tiles of block 0 (g = 0) or of block nb-1
+  const int qtile = n_glob == 1 ? (row < kBlock ? 0 : nt - 1) : (g == 0 ? 0 : nt - 2) + row / kBlock;
+  const size_t orow = static_cast<size_t>(bh) * L + static_cast<size_t>(qtile) * kBlock + (row & (kBlock - 1));
   if (lse && c4 == 0) lse[orow] = (mmax + log2f(l)) * 0.69314718055994531f;
   if (out_f32) {
     reinterpret_cast<float4*>(static_cast<float*>(out) + orow * kHeadDim)[c4] =
@@ -978,32 +1035,45 @@ uint32_t* status_word(int dev) {
 
 struct Plan {
   int nb = 0;
+  int nt = 0;
+  int bt = 1;
   bool sparse = false;
   int nsplit = 1;
-  int split_blocks = 0;
+  int split_tiles = 0;
+  int n_glob = 1;
   size_t ws_bytes = 0;
 };
 
+// Blocks of 64 or 128 tokens at d = 64 run on this kernel; other sizes return
+// BB_ERR_UNSUPPORTED here (the caller then tries the CUDA-core kernel).
 static int make_plan(int B, int H, int L, int d, int block, int r, unsigned flags, Plan& pl) {
   if (B <= 0 || H <= 0 || L <= 0 || d <= 0 || block <= 0 || r < 1 || L % block != 0) return BB_ERR_INVALID_ARG;
-  if (d != kHeadDim || block != kBlock || r > kMaxR) return BB_ERR_UNSUPPORTED;
+  if (d != kHeadDim || (block != kBlock && block != 2 * kBlock) || r > kMaxR) return BB_ERR_UNSUPPORTED;
   if (static_cast<int64_t>(B) * H * L >= (int64_t(1) << 31)) return BB_ERR_UNSUPPORTED;
   pl.nb = L / block;
+  pl.bt = block / kBlock;
+  pl.nt = L / kBlock;
   pl.sparse = (flags & BB_FLAG_FORCE_SPARSE) || pl.nb > 5 + 2 * r;
   if (pl.sparse && pl.nb < 5 + r) return BB_ERR_INVALID_ARG;
   if (pl.sparse) {
-    pl.split_blocks = kSplitBlocks;
-    pl.nsplit = (pl.nb + kSplitBlocks - 1) / kSplitBlocks;
+    // a middle unit lists at most 6 + 2r tiles (block 64: two query blocks'
+    // union) or 2 (5 + r) (block 128); both fit kMaxList for r <= kMaxR
+    pl.split_tiles = kSplitBlocks;
+    pl.nsplit = (pl.nt + kSplitBlocks - 1) / kSplitBlocks;
+    pl.n_glob = pl.bt == 1 ? 1 : 2;
   } else {
-    pl.split_blocks = pl.nb;  // nb <= 5 + 2r <= kMaxList
+    // full attention in one range: nt <= (5 + 2r) bt tiles must fit the list
+    if (pl.nt > kMaxList) return BB_ERR_UNSUPPORTED;
+    pl.split_tiles = pl.nt;
     pl.nsplit = 1;
+    pl.n_glob = 1;
   }
   // Workspace: the counters (unit tickets, finished CTAs, the bf16 flag),
-  // then (split global rows only) the partial outputs [B*H, nsplit, 128, 64]
-  // and their (max, sum) [B*H, nsplit, 128, 2].
+  // then (split global rows only) the partial outputs [B*H, n_glob*nsplit,
+  // 128, 64] and their (max, sum) [B*H, n_glob*nsplit, 128, 2].
   pl.ws_bytes = kCounterBytes;
   if (pl.nsplit > 1)
-    pl.ws_bytes += static_cast<size_t>(B) * H * pl.nsplit * kRows * (kHeadDim + 2) * sizeof(float);
+    pl.ws_bytes += static_cast<size_t>(B) * H * pl.n_glob * pl.nsplit * kRows * (kHeadDim + 2) * sizeof(float);
   return BB_OK;
 }
 
@@ -1022,12 +1092,12 @@ size_t bigbird_attn_workspace_size(int B, int H, int L, int d, int block, int r,
 static int fwd_impl(const void* q, const void* k, const void* v, const int32_t* rand_attn, const uint8_t* seq_mask,
                     void* out, float* lse, int B, int H, int L, int d, int block, int r, int out_dtype, unsigned flags,
                     void* workspace, size_t workspace_bytes, void* stream_) {
-  // Other supported sizes run the CUDA-core kernel (no workspace).
-  if (generic_fwd_supported(d, block))
-    return generic_fwd(q, k, v, rand_attn, seq_mask, out, lse, B, H, L, d, block, r, out_dtype, flags, stream_);
   cudaStream_t stream = static_cast<cudaStream_t>(stream_);
   Plan pl;
   int st = make_plan(B, H, L, d, block, r, flags, pl);
+  // Other supported sizes run the CUDA-core kernel (no workspace).
+  if (st == BB_ERR_UNSUPPORTED && generic_fwd_supported(d, block))
+    return generic_fwd(q, k, v, rand_attn, seq_mask, out, lse, B, H, L, d, block, r, out_dtype, flags, stream_);
   if (st != BB_OK) return st;
   if (!q || !k || !v || !out) return BB_ERR_INVALID_ARG;
   if (pl.sparse && !rand_attn) return BB_ERR_INVALID_ARG;
@@ -1072,16 +1142,21 @@ static int fwd_impl(const void* q, const void* k, const void* v, const int32_t* 
   p.r = r;
   p.BH = B * H;
   p.sparse = pl.sparse ? 1 : 0;
+  p.nt = pl.nt;
+  p.bt = pl.bt;
   p.nsplit = pl.nsplit;
-  p.split_blocks = pl.split_blocks;
+  p.split_tiles = pl.split_tiles;
+  p.n_glob = pl.n_glob;
+  p.nparts = pl.n_glob * pl.nsplit;
   if (pl.sparse) {
-    p.n_pairs = (pl.nb - 2 + 1) / 2;
+    // middle units: pairs of query blocks (block 64) or single blocks (block 128)
+    p.n_pairs = pl.bt == 1 ? (pl.nb - 2 + 1) / 2 : pl.nb - 2;
     p.n_pair_units = p.BH * p.n_pairs;
-    p.total_units = p.n_pair_units + p.BH * pl.nsplit;
+    p.total_units = p.n_pair_units + p.BH * p.nparts;
   } else {
     p.n_pairs = 0;
     p.n_pair_units = 0;
-    p.total_units = p.BH * ((pl.nb + 1) / 2);
+    p.total_units = p.BH * ((pl.nt + 1) / 2);
   }
   p.out_f32 = out_dtype == BB_OUT_F32 ? 1 : 0;
   p.scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(d));
@@ -1103,7 +1178,7 @@ static int fwd_impl(const void* q, const void* k, const void* v, const int32_t* 
   p.counters = static_cast<int*>(ws);
   if (pl.nsplit > 1) {
     p.part_o = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + kCounterBytes);
-    p.part_ml = p.part_o + static_cast<size_t>(p.BH) * pl.nsplit * kRows * kHeadDim;
+    p.part_ml = p.part_o + static_cast<size_t>(p.BH) * p.nparts * kRows * kHeadDim;
   }
 
   // The fp16 instance, then the bf16 instance and the merge, each a
@@ -1130,14 +1205,15 @@ static int fwd_impl(const void* q, const void* k, const void* v, const int32_t* 
   }
   if (e == cudaSuccess && pl.nsplit > 1) {
     cudaLaunchConfig_t cfg{};
-    cfg.gridDim = dim3(p.BH, kRows / kMergeRowsPerCta);
+    cfg.gridDim = dim3(p.BH * p.n_glob, kRows / kMergeRowsPerCta);
     cfg.blockDim = dim3(256);
     cfg.dynamicSmemBytes = 0;
     cfg.stream = stream;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     e = cudaLaunchKernelEx(&cfg, bigbird_merge_kernel, static_cast<const float*>(p.part_o),
-                           static_cast<const float*>(p.part_ml), out, p.lse, pl.nsplit, L, pl.nb, p.out_f32);
+                           static_cast<const float*>(p.part_ml), out, p.lse, pl.nsplit, pl.n_glob, L, pl.nt,
+                           p.out_f32);
   }
   if (owned) cudaFreeAsync(ws, stream);
   return e == cudaSuccess ? BB_OK : BB_ERR_CUDA;
@@ -1225,12 +1301,12 @@ extern "C" int bigbird_attn_fwd_noalloc(const void* q, const void* k, const void
                                         int r, int out_dtype, unsigned flags, void* stream) {
   // The debug checks copy rand_attn into a host buffer that they allocate.
   if (flags & BB_FLAG_DEBUG_CHECKS) return BB_ERR_UNSUPPORTED;
-  // The CUDA-core kernel for other sizes needs no scratch.
-  if (bb::generic_fwd_supported(d, block))
-    return bigbird_attn_fwd_ex(q, k, v, rand_attn, seq_mask, out, B, H, L, d, block, r, out_dtype, flags, nullptr, 0,
-                               stream);
   bb::Plan pl;
   const int st = bb::make_plan(B, H, L, d, block, r, flags, pl);
+  // The CUDA-core kernel for other sizes needs no scratch.
+  if (st == BB_ERR_UNSUPPORTED && bb::generic_fwd_supported(d, block))
+    return bigbird_attn_fwd_ex(q, k, v, rand_attn, seq_mask, out, B, H, L, d, block, r, out_dtype, flags, nullptr, 0,
+                               stream);
   if (st != BB_OK) return st;
   if (pl.ws_bytes > bb::kStaticScratchBytes) return BB_ERR_UNSUPPORTED;
   int dev = 0;
