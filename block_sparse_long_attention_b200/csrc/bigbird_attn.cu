@@ -71,7 +71,6 @@
 namespace bb {
 
 constexpr int kBlock = 64;             // tokens per tile: a block of 64, or half a block of 128
-constexpr int kHeadDim = 64;           // head dimension
 constexpr int kRows = 128;             // query rows per unit (two tiles)
 constexpr int kKStages = 2;            // K ring depth (blocks)
 constexpr int kVStages = 2;            // V ring depth (blocks)
@@ -79,11 +78,23 @@ constexpr int kMaxList = 42;           // key tiles per unit
 constexpr int kMaxR = 16;              // random blocks per row supported
 constexpr int kSplitBlocks = 8;        // key tiles per global-row range
 constexpr int kThreads = 256;
-constexpr int kCtasPerSm = 4;          // four independent unit pipelines per SM
-constexpr uint32_t kTileBytes = kBlock * kHeadDim * 2;  // one 64x64 bf16 tile
-constexpr uint32_t kTmemCols = 128;
-constexpr uint32_t kColS = 0;          // S of one key block: 64 fp32 columns; P (fp16) overwrites the first 32
-constexpr uint32_t kColO = 64;         // O: 64 fp32 columns
+constexpr uint32_t kColS = 0;          // S of one key tile: 64 fp32 columns; P (16-bit) overwrites the first 32
+constexpr uint32_t kColO = 64;         // O: d fp32 columns
+constexpr uint32_t kChunkBytes = kBlock * 64 * 2;  // 64 rows x 64 columns bf16: one TMA box, one 128-byte swizzle span
+
+// Sizes that follow from the head dimension d (64 or 128). A row of d values
+// is cut into d / 64 chunks of 64 columns; each tile is stored chunk by chunk
+// (chunk c of a K or V tile at c * 8 KB, of the unit's 128 Q rows at c * 16 KB).
+template <int kD>
+struct Geo {
+  static constexpr int kChunks = kD / 64;
+  static constexpr uint32_t kTileBytes = kBlock * kD * 2;    // one 64-token tile of K or V
+  static constexpr uint32_t kQChunkBytes = kRows * 64 * 2;   // one chunk of the unit's Q
+  // TMEM columns per CTA (S 64 + O d, rounded up to a power of two) and CTAs
+  // per SM: four at d = 64, two at d = 128 (TMEM and shared memory)
+  static constexpr uint32_t kTmemCols = kD == 64 ? 128 : 256;
+  static constexpr int kCtasPerSm = kD == 64 ? 4 : 2;
+};
 // The reference max moves only when a score exceeds it by more than 2^14: P
 // (fp16, largest finite 65504) then stays <= 2^14 with headroom, and the
 // repairs of already-written P and O stay rare even for wide score ranges.
@@ -149,10 +160,11 @@ struct FwdParams {
   float bias_raw;    // -10000 * sqrt(d): the masked-key bias in units of q.k
 };
 
+template <int kD>
 struct __align__(1024) SharedStorage {
-  uint8_t q[kRows * kHeadDim * 2];      // Q of the current unit (two 64x64 tiles, SW128)
-  uint8_t k[kKStages][kTileBytes];      // K blocks
-  uint8_t v[kVStages][kTileBytes];      // V blocks, converted to fp16 in place
+  uint8_t q[kRows * kD * 2];                   // Q of the current unit (chunks of two 64x64 tiles, SW128)
+  uint8_t k[kKStages][Geo<kD>::kTileBytes];    // K tiles
+  uint8_t v[kVStages][Geo<kD>::kTileBytes];    // V tiles, converted to fp16 in place
   UnitInfo unit[4];
   uint64_t info_full[4];
   uint64_t info_empty[4];
@@ -172,7 +184,8 @@ struct __align__(1024) SharedStorage {
   int32_t abort_flag;
 };
 
-__device__ __forceinline__ void flag_timeout(SharedStorage& s, const FwdParams& p) {
+template <class Smem>
+__device__ __forceinline__ void flag_timeout(Smem& s, const FwdParams& p) {
   atomicOr(p.status, kStatusTimeout);
   *reinterpret_cast<volatile int32_t*>(&s.abort_flag) = 1;
 }
@@ -350,7 +363,8 @@ __device__ void prep_unit(const FwdParams& p, int u, UnitInfo& ui, int lane) {
 // ticket from a device-wide counter (units are numbered longest first), so
 // CTAs that run faster take more units and all finish together. Once the
 // tickets run out it publishes a stop slot, which ends every role's loop.
-__device__ void prep_role(SharedStorage& s, const FwdParams& p) {
+template <int kD>
+__device__ void prep_role(SharedStorage<kD>& s, const FwdParams& p) {
   const int lane = threadIdx.x & 31;
   int u = blockIdx.x;
   for (uint32_t ut = 0;; ++ut) {
@@ -375,7 +389,7 @@ __device__ void prep_role(SharedStorage& s, const FwdParams& p) {
     prep_unit(p, u, ui, lane);
     if (lane == 0) mbar_arrive(smem_u32(&s.info_full[slot]));
     // Pull the unit's tiles into L2 now (it is up to four units ahead of the
-    // TMA warp), so its TMA loads hit L2 instead of HBM: one 8 KB tile per
+    // TMA warp), so its TMA loads hit L2 instead of HBM: one tile per
     // lane, lanes 0..n-1 K, n..2n-1 V, 2n and 2n+1 the query blocks.
     const size_t row0 = static_cast<size_t>(ui.bh) * p.L;
     const int n = ui.n;
@@ -385,7 +399,7 @@ __device__ void prep_role(SharedStorage& s, const FwdParams& p) {
       if (t < n) { base = p.k; blk = ui.kb[t]; }
       else if (t < 2 * n) { base = p.v; blk = ui.kb[t - n]; }
       else { base = p.q; blk = (t == 2 * n) ? ui.qtop : ui.qbot; }
-      if (blk >= 0) prefetch_l2_bulk(base + (row0 + static_cast<size_t>(blk) * kBlock) * kHeadDim, kTileBytes);
+      if (blk >= 0) prefetch_l2_bulk(base + (row0 + static_cast<size_t>(blk) * kBlock) * kD, Geo<kD>::kTileBytes);
     }
     u = __shfl_sync(0xffffffffu, next, 0);
   }
@@ -397,8 +411,8 @@ __device__ void prep_role(SharedStorage& s, const FwdParams& p) {
 // cannot represent, sets the workspace flag that makes the bf16 instance
 // recompute the call. The bf16 instance converts nothing: this warp only
 // keeps the unit bookkeeping.
-template <bool kBf16>
-__device__ void convert_role(SharedStorage& s, const FwdParams& p) {
+template <int kD, bool kBf16>
+__device__ void convert_role(SharedStorage<kD>& s, const FwdParams& p) {
   const int lane = threadIdx.x & 31;
   uint32_t gv = 0;
   for (uint32_t ut = 0;; ++ut) {
@@ -411,7 +425,7 @@ __device__ void convert_role(SharedStorage& s, const FwdParams& p) {
       uint4* vp = reinterpret_cast<uint4*>(s.v[st]) + lane;
       uint32_t ex = 0;  // largest bf16 exponent field seen, per 16-bit half
 #pragma unroll 4
-      for (int i = 0; i < static_cast<int>(kTileBytes / 16 / 32); ++i) {
+      for (int i = 0; i < static_cast<int>(Geo<kD>::kTileBytes / 16 / 32); ++i) {
         uint4 w = vp[32 * i];
         ex = __vmaxu2(ex, w.x & 0x7F807F80u);
         ex = __vmaxu2(ex, w.y & 0x7F807F80u);
@@ -437,7 +451,10 @@ __device__ void convert_role(SharedStorage& s, const FwdParams& p) {
 // Two cursors walk this CTA's key blocks: the V cursor (at most as far as the
 // K cursor) and the K cursor, which also loads each unit's Q when it enters
 // the unit (single Q buffer: after every S of the previous unit is done).
-__device__ void producer_role(SharedStorage& s, const FwdParams& p, const CUtensorMap* tmQ, const CUtensorMap* tmK,
+// Loads every chunk of a tile: K and V tiles are 64 rows x d, stored chunk by
+// chunk (x = 64 c of the tensor map, 8 KB apart).
+template <int kD>
+__device__ void producer_role(SharedStorage<kD>& s, const FwdParams& p, const CUtensorMap* tmQ, const CUtensorMap* tmK,
                               const CUtensorMap* tmV) {
   const int lane = threadIdx.x & 31;
   const uint64_t pol_kv = l2_policy_evict_last();
@@ -456,8 +473,11 @@ __device__ void producer_role(SharedStorage& s, const FwdParams& p, const CUtens
         ok = mbar_wait(smem_u32(&s.v_empty[st]), ((gv / kVStages) & 1) ^ 1);
         if (ok) {
           const uint32_t vbar = smem_u32(&s.v_full[st]);
-          mbar_arrive_expect_tx(vbar, kTileBytes);
-          tma_load_2d(smem_u32(s.v[st]), tmV, vbar, 0, ui.bh * p.L + ui.kb[ve] * kBlock, pol_kv);
+          mbar_arrive_expect_tx(vbar, Geo<kD>::kTileBytes);
+#pragma unroll
+          for (int c = 0; c < Geo<kD>::kChunks; ++c)
+            tma_load_2d(smem_u32(s.v[st]) + c * kChunkBytes, tmV, vbar, 64 * c, ui.bh * p.L + ui.kb[ve] * kBlock,
+                        pol_kv);
         }
       }
       if (!__shfl_sync(0xffffffffu, ok, 0)) {
@@ -491,9 +511,14 @@ __device__ void producer_role(SharedStorage& s, const FwdParams& p, const CUtens
           ok = mbar_wait(smem_u32(&s.q_free), (kut & 1) ^ 1);
           if (ok) {
             const uint32_t qbar = smem_u32(&s.q_full);
-            mbar_arrive_expect_tx(qbar, ui.qbot >= 0 ? 2 * kTileBytes : kTileBytes);
-            tma_load_2d(smem_u32(s.q), tmQ, qbar, 0, row0 + ui.qtop * kBlock, pol_q);
-            if (ui.qbot >= 0) tma_load_2d(smem_u32(s.q) + kTileBytes, tmQ, qbar, 0, row0 + ui.qbot * kBlock, pol_q);
+            mbar_arrive_expect_tx(qbar, (ui.qbot >= 0 ? 2 : 1) * Geo<kD>::kTileBytes);
+#pragma unroll
+            for (int c = 0; c < Geo<kD>::kChunks; ++c) {
+              // chunk c of the unit's 128 rows: the top tile, then the bottom one
+              const uint32_t qdst = smem_u32(s.q) + c * Geo<kD>::kQChunkBytes;
+              tma_load_2d(qdst, tmQ, qbar, 64 * c, row0 + ui.qtop * kBlock, pol_q);
+              if (ui.qbot >= 0) tma_load_2d(qdst + kChunkBytes, tmQ, qbar, 64 * c, row0 + ui.qbot * kBlock, pol_q);
+            }
           }
         }
         if (ok) {
@@ -501,8 +526,10 @@ __device__ void producer_role(SharedStorage& s, const FwdParams& p, const CUtens
           ok = mbar_wait(smem_u32(&s.k_empty[st]), ((gk / kKStages) & 1) ^ 1);
           if (ok) {
             const uint32_t kbar = smem_u32(&s.k_full[st]);
-            mbar_arrive_expect_tx(kbar, kTileBytes);
-            tma_load_2d(smem_u32(s.k[st]), tmK, kbar, 0, row0 + ui.kb[ke] * kBlock, pol_kv);
+            mbar_arrive_expect_tx(kbar, Geo<kD>::kTileBytes);
+#pragma unroll
+            for (int c = 0; c < Geo<kD>::kChunks; ++c)
+              tma_load_2d(smem_u32(s.k[st]) + c * kChunkBytes, tmK, kbar, 64 * c, row0 + ui.kb[ke] * kBlock, pol_kv);
           }
         }
       }
@@ -525,11 +552,11 @@ __device__ void producer_role(SharedStorage& s, const FwdParams& p, const CUtens
 // previous block's P.V has consumed the P that shares them, then, once the
 // softmax has written P(g), O += P(g) . V(g). The chain is serial within a
 // CTA; the four CTAs of an SM interleave on the tensor pipe.
-template <bool kBf16>
-__device__ void mma_role(SharedStorage& s, const FwdParams& p, uint32_t tmem) {
+template <int kD, bool kBf16>
+__device__ void mma_role(SharedStorage<kD>& s, const FwdParams& p, uint32_t tmem) {
   const uint32_t idesc_s = idesc_f32acc(kRows, kBlock, true, false);    // bf16 Q . K^T, N = 64
-  // fp16 P . fp16 V, or bf16 P . bf16 V in the bf16 instance
-  const uint32_t idesc_o = idesc_f32acc(kRows, kHeadDim, kBf16, true);
+  // fp16 P . fp16 V, or bf16 P . bf16 V in the bf16 instance; N = 64 per chunk of d
+  const uint32_t idesc_o = idesc_f32acc(kRows, 64, kBf16, true);
   const uint32_t q_addr = smem_u32(s.q);
   uint32_t g = 0;
   bool ok = true;
@@ -544,10 +571,11 @@ __device__ void mma_role(SharedStorage& s, const FwdParams& p, uint32_t tmem) {
       if (g >= 1 && !mbar_wait(smem_u32(&s.pv_done), (g - 1) & 1)) { ok = false; break; }
       tc_fence_after();
       const uint32_t k_addr = smem_u32(s.k[kst]);
+      // K = d in steps of 16: four steps (32 bytes apart) per 64-column chunk
 #pragma unroll
-      for (int kk = 0; kk < kHeadDim / 16; ++kk)
-        mma_ss(tmem + kColS, sdesc_sw128(q_addr + kk * 32, 16, 1024), sdesc_sw128(k_addr + kk * 32, 16, 1024),
-               idesc_s, kk > 0 ? 1u : 0u);
+      for (int kk = 0; kk < kD / 16; ++kk)
+        mma_ss(tmem + kColS, sdesc_sw128(q_addr + (kk >> 2) * Geo<kD>::kQChunkBytes + (kk & 3) * 32, 16, 1024),
+               sdesc_sw128(k_addr + (kk >> 2) * kChunkBytes + (kk & 3) * 32, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
       mma_commit(smem_u32(&s.s_full));
       mma_commit(smem_u32(&s.k_empty[kst]));
       if (e == n - 1) mma_commit(smem_u32(&s.q_free));
@@ -558,10 +586,13 @@ __device__ void mma_role(SharedStorage& s, const FwdParams& p, uint32_t tmem) {
       if (!mbar_wait(smem_u32(&s.p_full), g & 1)) { ok = false; break; }
       tc_fence_after();
       const uint32_t v_addr = smem_u32(s.v[vst]);
+      // O columns 64 c .. 64 c + 63 from V chunk c; K = 64 keys in steps of 16
 #pragma unroll
-      for (int kk = 0; kk < kBlock / 16; ++kk)
-        mma_ts(tmem + kColO, tmem + kColS + kk * 8, sdesc_sw128(v_addr + kk * 2048, 8192, 1024), idesc_o,
-               (e > 0 || kk > 0) ? 1u : 0u);
+      for (int c = 0; c < Geo<kD>::kChunks; ++c)
+#pragma unroll
+        for (int kk = 0; kk < kBlock / 16; ++kk)
+          mma_ts(tmem + kColO + 64 * c, tmem + kColS + kk * 8,
+                 sdesc_sw128(v_addr + c * kChunkBytes + kk * 2048, 8192, 1024), idesc_o, (e > 0 || kk > 0) ? 1u : 0u);
       mma_commit(smem_u32(&s.pv_done));
       mma_commit(smem_u32(&s.v_empty[vst]));
       if (e == n - 1) mma_commit(smem_u32(&s.o_full));
@@ -638,9 +669,10 @@ __device__ __noinline__ void rescale_p(uint32_t s_addr, int npieces, float f) {
 }
 
 // O (64 fp32 columns of this thread's row) *= f, in 16-column pieces.
+template <int kD>
 __device__ __forceinline__ void rescale_o(uint32_t taddr, float f) {
 #pragma unroll 1
-  for (int c0 = 0; c0 < 64; c0 += 16) {
+  for (int c0 = 0; c0 < kD; c0 += 16) {
     uint32_t t[16];
     tmem_ld16(taddr + c0, t);
     tmem_wait_ld();
@@ -652,15 +684,16 @@ __device__ __forceinline__ void rescale_o(uint32_t taddr, float f) {
 }
 
 // Store 16 columns [c0, c0+16) of one output row: o * inv as bf16 or fp32.
+template <int kD>
 __device__ __forceinline__ void store16(const FwdParams& p, size_t row, int c0, const uint32_t (&o)[16], float inv) {
   if (p.out_f32) {
-    float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + row * kHeadDim + c0);
+    float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + row * kD + c0);
 #pragma unroll
     for (int c = 0; c < 4; ++c)
       dst[c] = make_float4(__uint_as_float(o[4 * c]) * inv, __uint_as_float(o[4 * c + 1]) * inv,
                            __uint_as_float(o[4 * c + 2]) * inv, __uint_as_float(o[4 * c + 3]) * inv);
   } else {
-    uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) + row * kHeadDim + c0);
+    uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) + row * kD + c0);
 #pragma unroll
     for (int c = 0; c < 2; ++c)
       dst[c] = make_uint4(pack_bf16x2(__uint_as_float(o[8 * c]) * inv, __uint_as_float(o[8 * c + 1]) * inv),
@@ -676,8 +709,8 @@ __device__ __forceinline__ void store16(const FwdParams& p, size_t row, int c0, 
 // already written and, after the previous P.V has landed, O are rescaled),
 // exponentials, fp16 P written over the S columns already read (16 keys = 8
 // columns per piece) -- then the block goes to the MMA.
-template <bool kBf16>
-__device__ void softmax_role(SharedStorage& s, const FwdParams& p, uint32_t tmem) {
+template <int kD, bool kBf16>
+__device__ void softmax_role(SharedStorage<kD>& s, const FwdParams& p, uint32_t tmem) {
   const int tid = threadIdx.x;  // 0..127 == TMEM lane
   const int warp = tid >> 5;
   const int lane = tid & 31;
@@ -752,7 +785,7 @@ __device__ void softmax_role(SharedStorage& s, const FwdParams& p, uint32_t tmem
         if (e > 0 && __any_sync(0xffffffffu, o_factor != 1.f)) {
           if (!warp_wait(smem_u32(&s.pv_done), (g - 1) & 1)) { flag_timeout(s, p); return; }
           tc_fence_after();
-          rescale_o(lane_addr + kColO, o_factor);
+          rescale_o<kD>(lane_addr + kColO, o_factor);
         }
       } else {
         // No row of this warp uses the block: P = 0.
@@ -776,11 +809,11 @@ __device__ void softmax_role(SharedStorage& s, const FwdParams& p, uint32_t tmem
     if (split >= 0) {
       const size_t base = (static_cast<size_t>(bh) * p.nparts + split) * kRows + tid;
 #pragma unroll 1
-      for (int c0 = 0; c0 < kHeadDim; c0 += 16) {
+      for (int c0 = 0; c0 < kD; c0 += 16) {
         uint32_t o[16];
         tmem_ld16(lane_addr + kColO + c0, o);
         tmem_wait_ld();
-        float4* dst = reinterpret_cast<float4*>(p.part_o + base * kHeadDim + c0);
+        float4* dst = reinterpret_cast<float4*>(p.part_o + base * kD + c0);
 #pragma unroll
         for (int c = 0; c < 4; ++c)
           dst[c] = make_float4(__uint_as_float(o[4 * c]), __uint_as_float(o[4 * c + 1]), __uint_as_float(o[4 * c + 2]),
@@ -793,11 +826,11 @@ __device__ void softmax_role(SharedStorage& s, const FwdParams& p, uint32_t tmem
       // log sum_k exp(s_k) = ln 2 * (m_ref + log2 l), the scores in log2 units being s * log2(e).
       if (p.lse) p.lse[row] = (m_ref + log2f(l_run)) * 0.69314718055994531f;
 #pragma unroll 1
-      for (int c0 = 0; c0 < kHeadDim; c0 += 16) {
+      for (int c0 = 0; c0 < kD; c0 += 16) {
         uint32_t o[16];
         tmem_ld16(lane_addr + kColO + c0, o);
         tmem_wait_ld();
-        store16(p, row, c0, o, inv);
+        store16<kD>(p, row, c0, o, inv);
       }
     }
     tc_fence_before();
@@ -809,12 +842,14 @@ __device__ void softmax_role(SharedStorage& s, const FwdParams& p, uint32_t tmem
 // kBf16 = false: the fp16 instance (every call). kBf16 = true: the bf16
 // instance, launched behind it as its programmatic dependent, which does the
 // call again only when the fp16 instance saw a V value fp16 cannot represent.
-template <bool kBf16>
-__global__ void __launch_bounds__(kThreads, kCtasPerSm)
+// kD: the head dimension (64 or 128).
+template <int kD, bool kBf16>
+__global__ void __launch_bounds__(kThreads, Geo<kD>::kCtasPerSm)
 bigbird_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
   extern __shared__ uint8_t smem_raw[];
-  SharedStorage& s = *reinterpret_cast<SharedStorage*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  SharedStorage<kD>& s =
+      *reinterpret_cast<SharedStorage<kD>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   if (kBf16) {
@@ -828,7 +863,7 @@ bigbird_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     __syncthreads();
   }
   if (warp == 5) {
-    tmem_alloc(smem_u32(&s.tmem_base), kTmemCols);
+    tmem_alloc(smem_u32(&s.tmem_base), Geo<kD>::kTmemCols);
     tmem_relinquish();
   }
   if (threadIdx.x == 0) {
@@ -869,22 +904,22 @@ bigbird_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
   const uint32_t tmem = s.tmem_base;
 
   if (warp < 4) {
-    softmax_role<kBf16>(s, p, tmem);
+    softmax_role<kD, kBf16>(s, p, tmem);
   } else if (warp == 4) {
-    producer_role(s, p, &tmQ, &tmK, &tmV);
+    producer_role<kD>(s, p, &tmQ, &tmK, &tmV);
   } else if (warp == 5) {
-    if (lane == 0) mma_role<kBf16>(s, p, tmem);
+    if (lane == 0) mma_role<kD, kBf16>(s, p, tmem);
   } else if (warp == 6) {
-    prep_role(s, p);
+    prep_role<kD>(s, p);
   } else {
-    convert_role<kBf16>(s, p);
+    convert_role<kD, kBf16>(s, p);
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   if (warp == 5) {
     __syncwarp();
-    tmem_dealloc(tmem, kTmemCols);
+    tmem_dealloc(tmem, Geo<kD>::kTmemCols);
   }
   // The CTA that finishes last puts the workspace counters back to zero for
   // the next call (every other CTA is done with them).
@@ -900,20 +935,27 @@ bigbird_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
 }
 
 // Combine the partial results of the key ranges of the global rows by
-// log-sum-exp (log2 units). 16 threads per query row, 4 columns each; a CTA
-// covers 16 rows of one global unit, grid = (B*H*n_glob, 128 / 16).
-constexpr int kMergeRowsPerCta = 16;
+// log-sum-exp (log2 units). d / 4 threads per query row, 4 columns each; a
+// CTA of 256 threads covers 1024 / d rows of one global unit, grid =
+// (B*H*n_glob, 128 d / 1024).
+template <int kD>
+struct MergeGeo {
+  static constexpr int kThreadsPerRow = kD / 4;
+  static constexpr int kRowsPerCta = 256 / kThreadsPerRow;
+};
 
+template <int kD>
 __global__ void __launch_bounds__(256)
 bigbird_merge_kernel(const float* __restrict__ part_o, const float* __restrict__ part_ml, void* out, float* lse,
                      int nsplit, int n_glob, int L, int nt, int out_f32) {
+  constexpr int kTpr = MergeGeo<kD>::kThreadsPerRow;
   // Launched as a programmatic dependent of the attention kernel: wait until
   // that grid has completed and its partials are visible.
   asm volatile("griddepcontrol.wait;" ::: "memory");
   const int bh = blockIdx.x / n_glob;
   const int g = blockIdx.x % n_glob;  // global unit: its partials follow those of unit g - 1
-  const int row = blockIdx.y * kMergeRowsPerCta + (threadIdx.x >> 4);
-  const int c4 = threadIdx.x & 15;
+  const int row = blockIdx.y * MergeGeo<kD>::kRowsPerCta + static_cast<int>(threadIdx.x) / kTpr;
+  const int c4 = static_cast<int>(threadIdx.x) % kTpr;
   const size_t base = (static_cast<size_t>(bh) * n_glob + g) * nsplit * kRows + row;
   const float2* ml = reinterpret_cast<const float2*>(part_ml);
   float mmax = kNegInit;
@@ -925,7 +967,7 @@ bigbird_merge_kernel(const float* __restrict__ part_o, const float* __restrict__
     const float2 e = __ldg(&ml[idx]);
     const float w = ex2_approx(e.x - mmax);
     l += w * e.y;
-    const float4 t = __ldg(reinterpret_cast<const float4*>(part_o + idx * kHeadDim) + c4);
+    const float4 t = __ldg(reinterpret_cast<const float4*>(part_o + idx * kD) + c4);
     acc.x += w * t.x;
     acc.y += w * t.y;
     acc.z += w * t.z;
@@ -938,10 +980,10 @@ bigbird_merge_kernel(const float* __restrict__ part_o, const float* __restrict__
   const size_t orow = static_cast<size_t>(bh) * L + static_cast<size_t>(qtile) * kBlock + (row & (kBlock - 1));
   if (lse && c4 == 0) lse[orow] = (mmax + log2f(l)) * 0.69314718055994531f;
   if (out_f32) {
-    reinterpret_cast<float4*>(static_cast<float*>(out) + orow * kHeadDim)[c4] =
+    reinterpret_cast<float4*>(static_cast<float*>(out) + orow * kD)[c4] =
         make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
   } else {
-    reinterpret_cast<uint2*>(static_cast<uint16_t*>(out) + orow * kHeadDim)[c4] =
+    reinterpret_cast<uint2*>(static_cast<uint16_t*>(out) + orow * kD)[c4] =
         make_uint2(pack_bf16x2(acc.x * inv, acc.y * inv), pack_bf16x2(acc.z * inv, acc.w * inv));
   }
 }
@@ -978,12 +1020,14 @@ static EncodeTiledFn get_encode_fn() {
 }
 
 // Tensor map over [rows, 64] bf16 with 64x64 boxes and 128-byte swizzle.
-static bool make_map(CUtensorMap* map, const void* base, uint64_t rows) {
+// Tensor map over a [rows, d] bf16 matrix with 64x64 boxes (64 rows, one
+// 64-column chunk) and 128-byte swizzle.
+static bool make_map(CUtensorMap* map, const void* base, uint64_t rows, int d) {
   EncodeTiledFn enc = get_encode_fn();
   if (!enc) return false;
-  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(kHeadDim), static_cast<cuuint64_t>(rows)};
-  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(kHeadDim) * 2};
-  const cuuint32_t box[2] = {static_cast<cuuint32_t>(kHeadDim), static_cast<cuuint32_t>(kBlock)};
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(d) * 2};
+  const cuuint32_t box[2] = {64u, static_cast<cuuint32_t>(kBlock)};
   const cuuint32_t es[2] = {1, 1};
   return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -1010,12 +1054,20 @@ static DeviceInfo* device_info(int dev) {
     di.ok = (major == 10);
     di.sms = sms;
     if (di.ok) {
-      const int smem = static_cast<int>(sizeof(SharedStorage) + 1024);
-      // Four CTAs per SM need the largest shared-memory carve-out.
-      for (const void* fn : {reinterpret_cast<const void*>(bigbird_fwd_kernel<false>),
-                             reinterpret_cast<const void*>(bigbird_fwd_kernel<true>)}) {
-        if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) return nullptr;
-        if (cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout, 100) != cudaSuccess)
+      // Four (d 64) or two (d 128) CTAs per SM need the largest shared-memory carve-out.
+      const struct {
+        const void* fn;
+        int smem;
+      } kernels[] = {
+          {reinterpret_cast<const void*>(bigbird_fwd_kernel<64, false>), static_cast<int>(sizeof(SharedStorage<64>) + 1024)},
+          {reinterpret_cast<const void*>(bigbird_fwd_kernel<64, true>), static_cast<int>(sizeof(SharedStorage<64>) + 1024)},
+          {reinterpret_cast<const void*>(bigbird_fwd_kernel<128, false>), static_cast<int>(sizeof(SharedStorage<128>) + 1024)},
+          {reinterpret_cast<const void*>(bigbird_fwd_kernel<128, true>), static_cast<int>(sizeof(SharedStorage<128>) + 1024)},
+      };
+      for (const auto& kf : kernels) {
+        if (cudaFuncSetAttribute(kf.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, kf.smem) != cudaSuccess)
+          return nullptr;
+        if (cudaFuncSetAttribute(kf.fn, cudaFuncAttributePreferredSharedMemoryCarveout, 100) != cudaSuccess)
           return nullptr;
       }
       if (cudaGetSymbolAddress(reinterpret_cast<void**>(&di.status), g_status) != cudaSuccess) return nullptr;
@@ -1025,7 +1077,7 @@ static DeviceInfo* device_info(int dev) {
   return &di;
 }
 
-bool make_tile_map(CUtensorMap* map, const void* base, uint64_t rows) { return make_map(map, base, rows); }
+bool make_tile_map(CUtensorMap* map, const void* base, uint64_t rows) { return make_map(map, base, rows, 64); }
 
 uint32_t* status_word(int dev) {
   DeviceInfo* di = device_info(dev);
@@ -1044,11 +1096,11 @@ struct Plan {
   size_t ws_bytes = 0;
 };
 
-// Blocks of 64 or 128 tokens at d = 64 run on this kernel; other sizes return
+// Blocks of 64 or 128 tokens at d = 64 or 128 run on this kernel; other sizes return
 // BB_ERR_UNSUPPORTED here (the caller then tries the CUDA-core kernel).
 static int make_plan(int B, int H, int L, int d, int block, int r, unsigned flags, Plan& pl) {
   if (B <= 0 || H <= 0 || L <= 0 || d <= 0 || block <= 0 || r < 1 || L % block != 0) return BB_ERR_INVALID_ARG;
-  if (d != kHeadDim || (block != kBlock && block != 2 * kBlock) || r > kMaxR) return BB_ERR_UNSUPPORTED;
+  if ((d != 64 && d != 128) || (block != kBlock && block != 2 * kBlock) || r > kMaxR) return BB_ERR_UNSUPPORTED;
   if (static_cast<int64_t>(B) * H * L >= (int64_t(1) << 31)) return BB_ERR_UNSUPPORTED;
   pl.nb = L / block;
   pl.bt = block / kBlock;
@@ -1070,11 +1122,53 @@ static int make_plan(int B, int H, int L, int d, int block, int r, unsigned flag
   }
   // Workspace: the counters (unit tickets, finished CTAs, the bf16 flag),
   // then (split global rows only) the partial outputs [B*H, n_glob*nsplit,
-  // 128, 64] and their (max, sum) [B*H, n_glob*nsplit, 128, 2].
+  // 128, d] and their (max, sum) [B*H, n_glob*nsplit, 128, 2].
   pl.ws_bytes = kCounterBytes;
   if (pl.nsplit > 1)
-    pl.ws_bytes += static_cast<size_t>(B) * H * pl.n_glob * pl.nsplit * kRows * (kHeadDim + 2) * sizeof(float);
+    pl.ws_bytes += static_cast<size_t>(B) * H * pl.n_glob * pl.nsplit * kRows * (d + 2) * sizeof(float);
   return BB_OK;
+}
+
+// The launches of one call at head dimension kD: the fp16 instance, then the
+// bf16 instance and (split global rows) the merge.
+template <int kD>
+static cudaError_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const FwdParams& p,
+                              const Plan& pl, int sms, void* out, int L, cudaStream_t stream) {
+  // The fp16 instance, then the bf16 instance and the merge, each a
+  // programmatic dependent of the kernel before it: launched while its
+  // predecessor runs, it waits (griddepcontrol.wait) for the predecessor's
+  // completion before it reads what that grid wrote, which hides the launch
+  // gaps.
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  const int grid = std::min(p.total_units, Geo<kD>::kCtasPerSm * sms);
+  const size_t smem = sizeof(SharedStorage<kD>) + 1024;
+  bigbird_fwd_kernel<kD, false><<<grid, kThreads, smem, stream>>>(tq, tk, tv, p);
+  cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess) {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, bigbird_fwd_kernel<kD, true>, tq, tk, tv, p);
+  }
+  if (e == cudaSuccess && pl.nsplit > 1) {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(p.BH * p.n_glob, kRows / MergeGeo<kD>::kRowsPerCta);
+    cfg.blockDim = dim3(256);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, bigbird_merge_kernel<kD>, static_cast<const float*>(p.part_o),
+                           static_cast<const float*>(p.part_ml), out, p.lse, pl.nsplit, pl.n_glob, L, pl.nt,
+                           p.out_f32);
+  }
+  return e;
 }
 
 }  // namespace bb
@@ -1125,7 +1219,7 @@ static int fwd_impl(const void* q, const void* k, const void* v, const int32_t* 
 
   CUtensorMap tq, tk, tv;
   const uint64_t rows = static_cast<uint64_t>(B) * H * L;
-  if (!make_map(&tq, q, rows) || !make_map(&tk, k, rows) || !make_map(&tv, v, rows)) return BB_ERR_CUDA;
+  if (!make_map(&tq, q, rows, d) || !make_map(&tk, k, rows, d) || !make_map(&tv, v, rows, d)) return BB_ERR_CUDA;
 
   FwdParams p{};
   p.q = static_cast<const uint16_t*>(q);
@@ -1178,43 +1272,10 @@ static int fwd_impl(const void* q, const void* k, const void* v, const int32_t* 
   p.counters = static_cast<int*>(ws);
   if (pl.nsplit > 1) {
     p.part_o = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + kCounterBytes);
-    p.part_ml = p.part_o + static_cast<size_t>(p.BH) * p.nparts * kRows * kHeadDim;
+    p.part_ml = p.part_o + static_cast<size_t>(p.BH) * p.nparts * kRows * d;
   }
-
-  // The fp16 instance, then the bf16 instance and the merge, each a
-  // programmatic dependent of the kernel before it: launched while its
-  // predecessor runs, it waits (griddepcontrol.wait) for the predecessor's
-  // completion before it reads what that grid wrote, which hides the launch
-  // gaps.
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  const int grid = std::min(p.total_units, kCtasPerSm * di->sms);
-  const size_t smem = sizeof(SharedStorage) + 1024;
-  bigbird_fwd_kernel<false><<<grid, kThreads, smem, stream>>>(tq, tk, tv, p);
-  cudaError_t e = cudaGetLastError();
-  if (e == cudaSuccess) {
-    cudaLaunchConfig_t cfg{};
-    cfg.gridDim = dim3(grid);
-    cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = stream;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, bigbird_fwd_kernel<true>, tq, tk, tv, p);
-  }
-  if (e == cudaSuccess && pl.nsplit > 1) {
-    cudaLaunchConfig_t cfg{};
-    cfg.gridDim = dim3(p.BH * p.n_glob, kRows / kMergeRowsPerCta);
-    cfg.blockDim = dim3(256);
-    cfg.dynamicSmemBytes = 0;
-    cfg.stream = stream;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, bigbird_merge_kernel, static_cast<const float*>(p.part_o),
-                           static_cast<const float*>(p.part_ml), out, p.lse, pl.nsplit, pl.n_glob, L, pl.nt,
-                           p.out_f32);
-  }
+  const cudaError_t e = d == 64 ? launch_fwd<64>(tq, tk, tv, p, pl, di->sms, out, L, stream)
+                                : launch_fwd<128>(tq, tk, tv, p, pl, di->sms, out, L, stream);
   if (owned) cudaFreeAsync(ws, stream);
   return e == cudaSuccess ? BB_OK : BB_ERR_CUDA;
 }

@@ -1,6 +1,7 @@
 """The forward at the sizes other than block = d = 64, through the C ABI
-against the fp64 oracle: block 128 at d 64 on the tensor-core kernel (a block
-is two 64-token tiles), block 32 and d 128 on the CUDA-core kernel.
+against the fp64 oracle: blocks of 64 or 128 at d 64 or 128 on the
+tensor-core kernel (a block of 128 is two 64-token tiles, d 128 two 64-column
+chunks), block 32 on the CUDA-core kernel.
 
 Bars: bf16 output max |err| <= 1e-2, mean <= 1e-3 (the forward's bar) for
 both kernels. fp32 output: tensor-core sizes at the same bar (fp16 P, as at
@@ -21,7 +22,7 @@ from block_sparse_long_attention_b200.workloads import Workload, make_inputs
 pytestmark = pytest.mark.gpu
 
 SIZES = [(32, 64), (128, 64), (32, 128), (64, 128), (128, 128)]  # (block, d)
-TENSOR_CORE = {(128, 64)}  # sizes the tensor-core kernel takes (besides block = d = 64)
+TENSOR_CORE = {(128, 64), (64, 128), (128, 128)}  # sizes the tensor-core kernel takes (besides block = d = 64)
 
 
 def _check_f32(block, d, err, name):
@@ -184,3 +185,33 @@ def test_block128_tensor_core_edges():
     got3, _ = _run(w3, inp3, None, torch.float32)
     want3 = oracle.attention(inp3["q"], inp3["k"], inp3["v"], None, inp3["seq_mask"], 128, 9)
     assert np.abs(got3 - want3).max() <= 1e-4
+
+
+@pytest.mark.parametrize("block,d", [(64, 128), (128, 128)], ids=["b64_d128", "b128_d128"])
+def test_d128_v_beyond_fp16_range(block, d):
+    """d 128: one key block of V at magnitude 1e20 (fp16 cannot hold it, so
+    the call is redone with bf16 P and V). Every output is finite; rows with
+    no weight on that block meet the forward's bar; the others |err| <= 1e-2
+    + 2^-7 * mass * 1e20 (weights rounded once to bf16, relative 2^-9; mass =
+    the row's weight on the block, from the oracle with V = 1 there)."""
+    w = Workload(f"bigv_b{block}_d{d}", 1, 2, 16 * block, d=d, block=block, value_scale=1.0,
+                 pad=("fixed", [16 * block - 37]), seed=95)
+    j = 4
+    inp = make_inputs(w)
+    ra = _ra(w)
+    v = inp["v"].clone()
+    big = torch.randn(w.B, w.H, block, d, generator=torch.Generator().manual_seed(6))
+    v[:, :, j * block:(j + 1) * block] = (big / big.abs().max() * 1e20).to(torch.bfloat16)
+    inp = dict(inp, v=v)
+    got, _ = _run(w, inp, ra, torch.float32)
+    assert np.isfinite(got).all()
+    want = oracle.attention(inp["q"], inp["k"], v, ra, inp["seq_mask"], w.block, w.r)
+    ind = np.zeros(v.shape, np.float64)
+    ind[:, :, j * block:(j + 1) * block] = 1.0
+    mass = oracle.attention(inp["q"], inp["k"], ind, ra, inp["seq_mask"], w.block, w.r)[..., :1]
+    vmax = float(v[:, :, j * block:(j + 1) * block].float().abs().max())
+    err = np.abs(got - want)
+    off = (mass == 0)[..., 0]
+    assert off.any() and (~off).any()
+    assert err[off].max() <= 1e-2 and err[off].mean() <= 1e-3, float(err[off].max())
+    assert (err <= 1e-2 + 2.0 ** -7 * mass * vmax).all()

@@ -224,7 +224,7 @@ def test_max_growth_inside_and_across_blocks():
 def test_v_beyond_fp16_range(vmax, out_dtype):
     """One key block of V scaled so its largest magnitude is vmax: 65280 is the
     largest bf16 value fp16 still holds, 1e5 and 1e20 are not representable in
-    fp16 (P.V of that tile then runs in bf16). Pair unit (5, 6) shares every
+    fp16 (the call is then done again with bf16 P and V). Pair unit (5, 6) shares every
     MMA between a half that attends to block 4 (window of 5) and one that does
     not (window of 6), so the second half must be untouched.
 

@@ -149,7 +149,7 @@ def test_fwd_argument_errors_before_any_launch():
     # forced sparse needs nb >= 5 + r
     assert lib.bigbird_attn_fwd_ex(fake, fake, fake, fake, None, fake, 1, 2, 7 * 64, 64, 64, 3, 0,
                                    bb.BB_FLAG_FORCE_SPARSE, None, 0, None) == bb.BB_ERR_INVALID_ARG
-    # the other sizes (block 128 on tensor cores; block 32 and d 128 on CUDA
+    # the other sizes (block 128 and d 128 on tensor cores, block 32 on CUDA
     # cores) check the same before any device call
     for d, block in ((64, 32), (64, 128), (128, 32), (128, 64), (128, 128)):
         L = 16 * block
@@ -161,7 +161,7 @@ def test_fwd_argument_errors_before_any_launch():
             bb.BB_ERR_INVALID_ARG
         assert lib.bigbird_attn_fwd_ex(fake, fake, fake, fake, None, fake, 1, 2, 7 * block, d, block, 3, 0,
                                        bb.BB_FLAG_FORCE_SPARSE, None, 0, None) == bb.BB_ERR_INVALID_ARG
-        if (d, block) != (64, 128):
+        if block == 32:
             assert bb.workspace_size(1, 2, L, d, block) == 0   # CUDA cores: no workspace
     # block 128 at d 64: 64-token tiles, nt = L / 64, the global rows split
     # into ranges of 8 tiles, one partial-result set per global block
@@ -169,6 +169,9 @@ def test_fwd_argument_errors_before_any_launch():
     assert bb.workspace_size(1, 2, 2048, 64, 128) == 256 + 2 * 2 * ((nt + 7) // 8) * 128 * 66 * 4
     assert bb.workspace_size(1, 2, 8 * 128, 64, 128) == 256            # fallback: no split rows
     assert bb.workspace_size(1, 2, 22 * 128, 64, 128, r=9) == 0        # fallback wider than a unit: CUDA cores
+    # d 128: partial outputs of 128 columns (plus max and sum)
+    assert bb.workspace_size(1, 2, 4096, 128, 64) == 256 + 2 * 8 * 128 * 130 * 4
+    assert bb.workspace_size(1, 2, 4096, 128, 128) == 256 + 2 * 2 * 8 * 128 * 130 * 4
     # the backward and the probability export take d = block = 64 only
     assert lib.bigbird_attn_probs(fake, fake, fake, fake, None, fake, fake, 1, 2, 4096, 128, 64, 3, 1, 0, None) == \
         bb.BB_ERR_UNSUPPORTED
