@@ -210,6 +210,8 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity) {
 //     every key) against one range of split_tiles key tiles -- both blocks in
 //     one unit with block 64, one unit per block with block 128;
 //   * full-attention fallback: query tiles (2j, 2j+1) against every key tile.
+// kBt: tiles per block (1: block 64, 2: block 128).
+template <int kBt>
 __device__ void build_unit(const FwdParams& p, int u, UnitInfo& ui, int lane) {
   int n = 0;
   // one key tile, merging the half masks of a tile listed twice (set semantics)
@@ -230,7 +232,8 @@ __device__ void build_unit(const FwdParams& p, int u, UnitInfo& ui, int lane) {
       atomicOr(p.status, kStatusBadRandAttn);
       return;
     }
-    for (int t = 0; t < p.bt; ++t) add_tile(kb * p.bt + t, hm);
+#pragma unroll
+    for (int t = 0; t < kBt; ++t) add_tile(kb * kBt + t, hm);
   };
   if (u >= p.n_pair_units) {
     u -= p.n_pair_units;
@@ -273,7 +276,7 @@ __device__ void build_unit(const FwdParams& p, int u, UnitInfo& ui, int lane) {
     const int pp = u % p.n_pairs;
     const int h = bh % p.H;
     int qtop, qbot;
-    if (p.bt == 1) {
+    if (kBt == 1) {
       const int i = 1 + 2 * pp;  // query blocks i and i + 1 (if still a middle block)
       const bool pair = i + 1 <= p.nb - 2;
       const int both = pair ? 3 : 1;
@@ -346,8 +349,9 @@ __device__ __forceinline__ uint64_t key_valid_bits(const uint8_t* seq_mask, int 
 // ---------------------------------------------------------------- producer
 
 // Prepare unit u's info (list, half masks, key validity bits). Whole warp.
+template <int kBt>
 __device__ void prep_unit(const FwdParams& p, int u, UnitInfo& ui, int lane) {
-  build_unit(p, u, ui, lane);
+  build_unit<kBt>(p, u, ui, lane);
   __syncwarp();
   const int n = ui.n;
   const int b = ui.bh / p.H;
@@ -364,7 +368,7 @@ __device__ void prep_unit(const FwdParams& p, int u, UnitInfo& ui, int lane) {
 // CTAs that run faster take more units and all finish together. Once the
 // tickets run out it publishes a stop slot, which ends every role's loop.
 template <int kD>
-__device__ void prep_role(SharedStorage<kD>& s, const FwdParams& p) {
+__device__ void prep_role(SharedStorage<kD>& s, const FwdParams& p, int bt) {
   const int lane = threadIdx.x & 31;
   int u = blockIdx.x;
   for (uint32_t ut = 0;; ++ut) {
@@ -386,7 +390,8 @@ __device__ void prep_role(SharedStorage<kD>& s, const FwdParams& p) {
     // Claim the next unit now, so the atomic's round trip overlaps this one's preparation.
     int next = 0;
     if (lane == 0) next = static_cast<int>(gridDim.x) + atomicAdd(&p.counters[kCtrTickets], 1);
-    prep_unit(p, u, ui, lane);
+    if (bt == 1) prep_unit<1>(p, u, ui, lane);
+    else prep_unit<2>(p, u, ui, lane);
     if (lane == 0) mbar_arrive(smem_u32(&s.info_full[slot]));
     // Pull the unit's tiles into L2 now (it is up to four units ahead of the
     // TMA warp), so its TMA loads hit L2 instead of HBM: one tile per
@@ -910,7 +915,7 @@ bigbird_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
   } else if (warp == 5) {
     if (lane == 0) mma_role<kD, kBf16>(s, p, tmem);
   } else if (warp == 6) {
-    prep_role<kD>(s, p);
+    prep_role<kD>(s, p, p.bt);
   } else {
     convert_role<kD, kBf16>(s, p);
   }
