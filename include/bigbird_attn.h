@@ -76,14 +76,17 @@ enum {
  *   seq_mask   device, uint8 [B, L], nonzero = valid key; NULL = all valid.
  *   out        device, bf16 [B, H, L, d], 16-byte aligned; must not alias q/k/v.
  *   B, H, L, d, block, r  sizes: d in {64, 128}, block in {32, 64, 128}.
- *              d = block = 64 runs the tensor-core kernel described above; the
- *              other sizes run a CUDA-core kernel (fp32 arithmetic, one CTA per
- *              query block, no workspace) with the same results.
+ *              Blocks of 64 or 128 at d 64 or 128 run the tensor-core kernel
+ *              (64-token tiles: a block of 128 is two; d 128 is two 64-column
+ *              chunks per row); block 32, and full attention over more than
+ *              42 tiles (block 128 with r > 8), run a CUDA-core kernel (fp32
+ *              arithmetic, one CTA per query block, no workspace) with the
+ *              same results.
  *   stream     cudaStream_t.
  * Errors: BB_ERR_INVALID_ARG for L % block != 0 [HF-Pegasus, section
  * "序列长度的块对齐要求"] or r < 1 [HF-Pegasus, section "使用限制与注意事项"];
  * BB_ERR_UNSUPPORTED for other d/block or misalignment. Every finite bf16
- * value is taken. For d = block = 64, P.V runs in fp16 (P and V converted in
+ * value is taken. On the tensor-core kernel P.V runs in fp16 (P and V converted in
  * shared memory); when V holds a value of magnitude >= 65536, which fp16
  * cannot represent, the call is done again with bf16 P and V (8 significant
  * bits of P instead of 11), which about doubles its time. A call launches the
@@ -104,14 +107,15 @@ int bigbird_attn_fwd(const void* q, const void* k, const void* v, const int32_t*
 /*
  * Bytes of device workspace bigbird_attn_fwd_ex needs for these sizes and
  * flags (0 if the sizes are invalid, and for the sizes the CUDA-core kernel
- * runs, which need none). For d = block = 64 it starts with 256 bytes of
+ * runs, which need none). For the tensor-core kernel it starts with 256 bytes of
  * counters: the one through which the CTAs share out the work units, one that
  * finds the CTA finishing last (which sets the counters back to zero), and
  * the flag that asks for the bf16 recompute (cleared by the bf16 instance when
  * it runs). When the global rows are split into key ranges (sparse pattern:
- * ranges of 8 key blocks) each range's partial result follows (output
- * normalised by its own sum, running max, running sum), merged by
- * log-sum-exp in a separate kernel.
+ * ranges of 8 tiles of 64 keys) each range's partial result follows, per
+ * global unit (one unit holds both global blocks at block 64, one unit per
+ * global block at block 128): output normalised by its own sum [128 rows, d],
+ * running max and running sum, merged by log-sum-exp in a separate kernel.
  */
 size_t bigbird_attn_workspace_size(int B, int H, int L, int d, int block, int r, unsigned flags);
 
