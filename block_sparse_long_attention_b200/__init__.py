@@ -56,6 +56,8 @@ def _load():
         "bigbird_attn_noalloc_scratch_bytes": (Z, []),
         "bigbird_attn_fwd_train": (I, [P, P, P, P, P, P, P, I, I, I, I, I, I, I, U, P, Z, P]),
         "bigbird_attn_bwd": (I, [P, P, P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, U, P]),
+        "bigbird_attn_bwd_ex": (I, [P, P, P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, U, P, Z, P]),
+        "bigbird_attn_bwd_workspace_size": (Z, [I, I, I, I, I, I, U]),
         "bigbird_wait_probe": (I, [U, P]),
         "bigbird_attn_probs_layout": (I, [I, I, I, I, U, ctypes.POINTER(I), ctypes.POINTER(I), ctypes.POINTER(I)]),
         "bigbird_attn_probs": (I, [P, P, P, P, P, P, P, I, I, I, I, I, I, I, U, P]),
@@ -197,11 +199,19 @@ def fwd_train(q, k, v, rand_attn, seq_mask=None, *, block: int = 64, r: int = 3,
     return out, lse
 
 
+def bwd_workspace_size(B: int, H: int, L: int, d: int = 64, block: int = 64, r: int = 3,
+                       force_sparse: bool = False) -> int:
+    flags = BB_FLAG_FORCE_SPARSE if force_sparse else 0
+    return int(_load().bigbird_attn_bwd_workspace_size(B, H, L, d, block, r, flags))
+
+
 def bwd(q, k, v, out, dout, lse, rand_attn, seq_mask=None, *, block: int = 64, r: int = 3,
-        force_sparse: bool = False, stream=None):
+        force_sparse: bool = False, stream=None, workspace=None):
     """Backward: returns (dq, dk, dv), fp32 [B, H, L, d], the gradients of
     sum(dout * out). out is the forward's output (bf16 or fp32), dout a bf16
-    tensor of its shape, lse from fwd_train()."""
+    tensor of its shape, lse from fwd_train(). `workspace` (optional, reusable
+    across calls): a uint8 CUDA tensor of at least bwd_workspace_size(...)
+    bytes, zero-filled before its first use (e.g. torch.zeros)."""
     import torch
     B, H, L, d, ra_ptr, sm_ptr = _check_inputs(q, k, v, rand_attn, seq_mask, block, r)
     if not (dout.is_cuda and dout.dtype == torch.bfloat16 and dout.is_contiguous() and dout.shape == q.shape):
@@ -212,11 +222,19 @@ def bwd(q, k, v, out, dout, lse, rand_attn, seq_mask=None, *, block: int = 64, r
     if not (lse.is_cuda and lse.dtype == torch.float32 and lse.is_contiguous() and lse.shape == (B, H, L)):
         raise ValueError("lse must be a contiguous fp32 CUDA tensor [B, H, L]")
     dq, dk, dv = (torch.empty((B, H, L, d), dtype=torch.float32, device=q.device) for _ in range(3))
-    st = _load().bigbird_attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), dout.data_ptr(),
+    flags = BB_FLAG_FORCE_SPARSE if force_sparse else 0
+    lib_ = _load()
+    ws_bytes = int(lib_.bigbird_attn_bwd_workspace_size(B, H, L, d, block, r, flags))
+    ws_ptr = None
+    if workspace is not None:
+        if workspace.numel() * workspace.element_size() < ws_bytes:
+            raise ValueError(f"workspace too small: need {ws_bytes} bytes")
+        ws_ptr = workspace.data_ptr()
+    st = lib_.bigbird_attn_bwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), dout.data_ptr(),
                                   lse.data_ptr(), ra_ptr, sm_ptr, dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
                                   B, H, L, d, block, r, BB_OUT_F32 if out.dtype == torch.float32 else BB_OUT_BF16,
-                                  BB_FLAG_FORCE_SPARSE if force_sparse else 0, _stream_handle(stream))
-    _check(st, "bigbird_attn_bwd")
+                                  flags, ws_ptr, ws_bytes if ws_ptr else 0, _stream_handle(stream))
+    _check(st, "bigbird_attn_bwd_ex")
     return dq, dk, dv
 
 

@@ -4,292 +4,1013 @@
 // pattern as the forward [TFG-BigBird, section "BigBird：从二次方注意力到线性稀疏注意力";
 // HF-Pegasus, section "三类注意力组合"], by the chain rule through each row's
 // softmax: with p = exp(s - lse) recomputed from the forward's row
-// log-sum-exp, D = rowsum(dout * out),
-//   dv_k += p^T dout,  dp = dout v^T,  ds = p (dp - D),
-//   dq   += ds k / sqrt(d),  dk_k += ds^T q / sqrt(d).
+// log-sum-exp and D = rowsum(dout * out),
+//   dp = dout v^T,  ds = p (dp - D),
+//   dq = ds k / sqrt(d),  dk = ds^T q / sqrt(d),  dv = p^T dout.
 //
-// One CTA per (b, h, query block i), 256 threads, fp32 CUDA-core arithmetic
-// on 64x64 tiles staged in shared memory: the CTA walks the key blocks of row
-// i (all of them for the global rows and the full-attention fallback; else
-// the set {0, nb-1, i-1, i, i+1} and the row's random blocks), keeps dq_i in
-// registers and adds its dk_j, dv_j contributions with fp32 atomics (a key
-// block receives from every query block that attends to it). Every product
-// is computed as 4x4 register tiles per thread (16 x 16 threads over a 64x64
-// result), reading 4-wide vectors along the summed dimension, so each shared-
-// memory load feeds four FMAs or more.
+// Four launches, in stream order, nothing accumulated with atomics (the
+// gradients are the same bit for bit on every run):
+//   1. bwd_rowdot_kernel: D = rowsum(dout * out) into the workspace;
+//   2. bwd_kernel<false> (dq): query-stationary. A unit is the forward's: 128
+//      query rows (query blocks i, i+1, or the two global blocks against one
+//      range of key tiles) against a list of 64-key tiles. Per key tile:
+//      S = Q K^T and dP = dO V^T (tcgen05 SS-MMAs, M = 128, N = 64, K = 64,
+//      fp32 in TMEM), P and dS by one thread per query row (bf16, written
+//      back over the S and dP columns), then dQ += dS K (TS-MMA, dS from TMEM,
+//      K as loaded, d contiguous);
+//   3. bwd_kernel<true> (dk, dv): key-stationary. A unit is 128 key rows (key
+//      blocks j, j+1, or the two global key blocks against one range of query
+//      tiles) against the query tiles that attend either block -- the pattern
+//      transposed, found by scanning rand_attn (a long list goes out in
+//      chunks). Per query tile: S^T = K Q^T and dP^T = V dO^T, P^T and dS^T by
+//      one thread per key row (the query's lse and D from shared memory), then
+//      dV += P^T dO and dK += dS^T Q (two TS-MMAs);
+//   4. bwd_sum_kernel: the global rows' dq and the global key blocks' dk, dv
+//      are split over ranges; their partial sums (workspace) are added here.
+//
+// Both attention kernels are persistent (2 CTAs per SM, 256 TMEM columns:
+// S | dP | accumulator 1 | accumulator 2) and warp-specialised: warps 0-3 the
+// elementwise part and the epilogue, warp 4 TMA, warp 5 the MMAs (one
+// thread), warp 6 unit preparation and scheduling (tickets from a workspace
+// counter, reset by the CTA that finishes last). Every wait is bounded.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
+#include <cmath>
 #include <cstdint>
 
 #include "../../include/bigbird_attn.h"
+#include "bb_internal.h"
+#include "sm100_ptx.cuh"
 
 namespace bbw {
 
-constexpr int kBlock = 64;
-constexpr int kDim = 64;
-constexpr int kThreads = 256;
-constexpr int kLd = kDim + 4;  // row stride of the fp32 tiles (16-byte aligned rows)
-constexpr int kMaxList = 5 + 16;
+using namespace bb;
 
-struct BwdParams {
+constexpr int kBlock = 64;     // tokens per block (one 64x64 tile)
+constexpr int kDim = 64;       // head dimension
+constexpr int kRows = 128;     // stationary rows per unit (two tiles)
+constexpr int kStages = 2;     // moving-tile ring depth
+constexpr int kMaxList = 42;   // moving tiles per unit chunk
+constexpr int kMaxR = 16;
+constexpr int kSplit = 8;      // tiles per range of a global unit
+constexpr int kThreads = 256;
+constexpr int kCtasPerSm = 2;
+// Dynamic shared memory requested per CTA: more than the kernel uses, so that
+// at most two CTAs share an SM (each allocates half of its TMEM).
+constexpr int kSmemRequest = 112 * 1024;
+constexpr uint32_t kTileBytes = kBlock * kDim * 2;  // 8 KB
+constexpr uint32_t kTmemCols = 256;
+constexpr uint32_t kColX = 0;     // S (or S^T): 64 fp32 columns; P (bf16) overwrites the first 32, dS_lo the last 32
+constexpr uint32_t kColY = 64;    // dP (or dP^T): 64 fp32 columns; dS_hi (bf16) overwrites the first 32
+constexpr uint32_t kColA1 = 128;  // dQ, or dV
+constexpr uint32_t kColA2 = 192;  // dK
+
+constexpr uint32_t kStatusBadRandAttn = 1u;
+constexpr uint32_t kStatusTimeout = 2u;
+
+// Workspace: counters (ints) [0] dq tickets, [1] dq CTAs done, [2] dk/dv
+// tickets, [3] dk/dv CTAs done; then D [B*H*L] fp32; then the partial sums.
+constexpr size_t kCounterBytes = 256;
+
+// One unit chunk: stationary tiles `top` (rows 0..63) and `bot` (rows 64..127,
+// or -1) of head bh against `n` moving tiles.
+struct Unit {
+  int32_t n;
+  int32_t bh;
+  int32_t top, bot;
+  int32_t split;   // partial-sum slot of a split global unit, or -1
+  int32_t first;   // 1: the unit's first chunk (accumulators start from zero)
+  int32_t last;    // 1: the unit's last chunk (epilogue follows)
+  int32_t stop;    // 1: no more units for this CTA
+  int32_t mt[kMaxList];    // moving tiles
+  uint64_t vm[kMaxList];   // dq kernel: validity bits of the moving (key) tile
+  uint8_t hm[kMaxList];    // bit 0: rows 0..63 use the tile, bit 1: rows 64..127
+};
+
+struct Params {
   const uint16_t* q;
   const uint16_t* k;
   const uint16_t* v;
-  const void* out;
   const uint16_t* dout;
-  const float* lse;
+  const float* lse;       // [B*H*L] natural log
+  const float* dd;        // D [B*H*L]
   const int32_t* rand_attn;
   const uint8_t* seq_mask;
-  float* dq;
-  float* dk;
-  float* dv;
-  int H, L, nb, r;
+  float* g1;              // dq (dq kernel) or dv (dk/dv kernel), [B*H*L, 64]
+  float* g2;              // dk (dk/dv kernel)
+  float* part1;           // partial sums of split global units [BH, nsplit, 128, 64] (g1)
+  float* part2;           // ... (g2)
+  int* counters;          // this kernel's [tickets, done]
+  uint32_t* status;
+  int H, L, nb, r, BH;
   int sparse;
-  int out_f32;
-  float scale;  // 1 / sqrt(d)
+  int nsplit;             // ranges per global unit (1: write the gradient directly)
+  int n_mid_per_head;     // middle units per head
+  int n_mid_units;
+  int total_units;
+  float scale_log2;       // log2(e) / sqrt(d)
+  float bias_raw;         // -10000 sqrt(d): the masked-key bias in units of q.k
+  float scale;            // 1 / sqrt(d)
 };
 
-struct Smem {
-  float q[kBlock][kLd];
-  float dout[kBlock][kLd];
-  float k[kBlock][kLd];
-  float v[kBlock][kLd];
-  float p[kBlock][kLd];
-  float ds[kBlock][kLd];
-  float lse[kBlock];
-  float dsum[kBlock];   // D = rowsum(dout * out)
-  float bias[kBlock];   // 0 or -10000 per key of the current block
-  int list[kMaxList];
-  int nlist;
+struct __align__(1024) Smem {
+  uint8_t a1[kRows * kDim * 2];           // Q (dq) or K (dk/dv) of the unit: two tiles
+  uint8_t a2[kRows * kDim * 2];           // dO (dq) or V (dk/dv)
+  uint8_t b1[kStages][kTileBytes];        // K (dq) or Q (dk/dv) of a step
+  uint8_t b2[kStages][kTileBytes];        // V (dq) or dO (dk/dv)
+  uint8_t plo[kRows * kBlock * 2];        // dk/dv: P_lo and dS_lo of the step, [128 rows x 64] bf16,
+  uint8_t dslo[kRows * kBlock * 2];       //   laid out as a TMA box with 128-byte swizzle (an SS-MMA operand)
+  float col_lse[kStages][kBlock];         // dk/dv: lse and D of the step's query tile
+  float col_d[kStages][kBlock];
+  Unit unit[4];
+  uint64_t info_full[4];
+  uint64_t info_empty[4];
+  uint64_t a_full, a_free;
+  uint64_t b_full[kStages], b_empty[kStages];
+  uint64_t x_full;     // S and dP of the step are in TMEM
+  uint64_t p_full;     // P and dS written (4 warps)
+  uint64_t g2_done;    // the step's gradient MMAs are complete (S/dP columns reusable)
+  uint64_t acc_full;   // a unit's accumulators are complete
+  uint64_t acc_free;   // ... and read by the epilogue (4 warps)
+  uint32_t tmem_base;
+  uint32_t rbits[32];  // dk/dv prep: per query block of a scan batch, which key blocks it picked at random
 };
 
-__device__ __forceinline__ float bf16_to_f32(uint16_t x) { return __uint_as_float(static_cast<uint32_t>(x) << 16); }
+__device__ __forceinline__ void flag_timeout(const Params& p) { atomicOr(p.status, kStatusTimeout); }
 
-// A 64x64 bf16 tile (rows row0.., 64 values each) into fp32 shared memory.
-__device__ __forceinline__ void load_tile(float (&dst)[kBlock][kLd], const uint16_t* src, size_t row0) {
-  for (int e = threadIdx.x; e < kBlock * kDim / 2; e += kThreads) {
-    const int rr = e / (kDim / 2);
-    const int cc = 2 * (e % (kDim / 2));
-    const uint32_t w = reinterpret_cast<const uint32_t*>(src + (row0 + rr) * kDim)[cc / 2];
-    dst[rr][cc] = bf16_to_f32(static_cast<uint16_t>(w & 0xFFFFu));
-    dst[rr][cc + 1] = bf16_to_f32(static_cast<uint16_t>(w >> 16));
-  }
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity) {
+  return __all_sync(0xffffffffu, mbar_wait(bar, parity));
 }
 
-__global__ void __launch_bounds__(kThreads, 2) bigbird_bwd_kernel(const BwdParams p) {
-  extern __shared__ uint8_t smem_raw[];
-  Smem& s = *reinterpret_cast<Smem*>(smem_raw);
-  const int i = blockIdx.x;   // query block
-  const int bh = blockIdx.y;  // b * H + h
-  const int b = bh / p.H;
-  const int h = bh % p.H;
-  const int t = threadIdx.x;
-  const int row = t >> 2;          // row of the D computation (4 threads per row)
-  const int c0 = (t & 3) * 16;     // its 16 columns
-  const int ty = t >> 4;           // 4x4 result tile: rows (or keys) 4ty..4ty+3
-  const int tx = t & 15;           // and columns (keys or dims) 4tx..4tx+3
-  const size_t head = static_cast<size_t>(bh) * p.L;
-  const size_t q0 = head + static_cast<size_t>(i) * kBlock;
+// 1-D bulk copy global -> shared (16-byte aligned, size a multiple of 16),
+// completion counted on the mbarrier in bytes.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+               : "memory");
+}
 
-  // ---- row data: q, dout, lse and D = rowsum(dout * out)
-  load_tile(s.q, p.q, q0);
-  load_tile(s.dout, p.dout, q0);
-  if (t < kBlock) s.lse[t] = p.lse[q0 + t];
-  {
-    // D of row `row`: four threads per row, 16 columns each, combined by shuffles.
-    float acc = 0.f;
-    const size_t o = (q0 + row) * kDim + c0;
-    for (int x = 0; x < 16; ++x) {
-      const float ov = p.out_f32 ? static_cast<const float*>(p.out)[o + x]
-                                 : bf16_to_f32(static_cast<const uint16_t*>(p.out)[o + x]);
-      acc += ov * bf16_to_f32(p.dout[o + x]);
+// 64 validity bits of key block kb of batch b (bit c: seq_mask != 0).
+__device__ __forceinline__ uint64_t key_valid_bits(const uint8_t* seq_mask, int L, int b, int kb) {
+  const uint4* src = reinterpret_cast<const uint4*>(seq_mask + static_cast<size_t>(b) * L + static_cast<size_t>(kb) * kBlock);
+  uint64_t bits = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint4 w = __ldg(src + i);
+    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint32_t m = __vcmpne4(ws[j], 0u) & 0x01010101u;  // one bit per byte
+      bits |= static_cast<uint64_t>((m * 0x01020408u) >> 24) << (16 * i + 4 * j);
     }
-    acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-    acc += __shfl_xor_sync(0xffffffffu, acc, 2);
-    if ((t & 3) == 0) s.dsum[row] = acc;
   }
-  // ---- the row's key blocks
-  const bool all = !p.sparse || i == 0 || i == p.nb - 1;
-  if (t == 0 && !all) {
-    int n = 0;
-    auto add = [&](int kb) {
-      if (kb < 0 || kb >= p.nb) return;  // out of range: skipped (the forward flags it)
-      for (int e = 0; e < n; ++e)
-        if (s.list[e] == kb) return;
-      s.list[n++] = kb;
-    };
-    add(i - 1);
-    add(i);
-    add(i + 1);
-    add(0);
-    add(p.nb - 1);
+  return bits;
+}
+
+// ------------------------------------------------------------ unit building
+
+// Unit u of either kernel when its list fits one chunk: a global unit (the
+// two global blocks stacked against one range of 8 tiles: every row attends
+// every tile), a full-attention unit (blocks 2j, 2j+1 against every tile), or
+// -- dq kernel only -- a middle unit of query blocks (i, i+1) against the
+// union of their key blocks [TFG-BigBird, section "随机块掩码是如何生成的";
+// HF-Pegasus, section "三类注意力组合"], a half mask per tile. In the dk/dv
+// kernel the stationary tiles are key blocks and the moving ones query
+// blocks; a global or full-attention unit decodes the same way (every query
+// attends a global key block, and in full attention every key).
+// Whole warp: the lanes fetch the random entries, lane 0 builds the list.
+__device__ void build_simple(const Params& p, int u, Unit& ui, int lane) {
+  int n = 0;
+  auto add = [&](int t, int hm) {
+    if (t < 0 || t >= p.nb) {
+      atomicOr(p.status, kStatusBadRandAttn);
+      return;
+    }
+    for (int e = 0; e < n; ++e)
+      if (ui.mt[e] == t) {
+        ui.hm[e] |= static_cast<uint8_t>(hm);
+        return;
+      }
+    ui.mt[n] = t;
+    ui.hm[n] = static_cast<uint8_t>(hm);
+    ++n;
+  };
+  int bh, top, bot, split = -1;
+  if (u >= p.n_mid_units) {
+    const int v = u - p.n_mid_units;
+    int t0, t1;
+    if (p.sparse) {
+      bh = v / p.nsplit;
+      const int s = v % p.nsplit;
+      top = 0;
+      bot = p.nb - 1;
+      t0 = s * kSplit;
+      t1 = min(p.nb, t0 + kSplit);
+      split = p.nsplit > 1 ? s : -1;
+    } else {
+      const int npair = (p.nb + 1) / 2;
+      bh = v / npair;
+      const int pp = v % npair;
+      top = 2 * pp;
+      bot = 2 * pp + 1 < p.nb ? 2 * pp + 1 : -1;
+      t0 = 0;
+      t1 = p.nb;
+    }
+    if (lane == 0)
+      for (int t = t0; t < t1; ++t) add(t, bot >= 0 ? 3 : 1);
+  } else {
+    bh = u / p.n_mid_per_head;
+    const int pp = u % p.n_mid_per_head;
+    const int h = bh % p.H;
+    const int i = 1 + 2 * pp;
+    const bool pair = i + 1 <= p.nb - 2;
+    const int both = pair ? 3 : 1;
+    const int nrand = pair ? 2 * p.r : p.r;
     const int32_t* ra = p.rand_attn + (static_cast<size_t>(h) * (p.nb - 2) + (i - 1)) * p.r;
-    for (int e = 0; e < p.r; ++e) add(ra[e]);
-    s.nlist = n;
+    const int rv = lane < nrand ? __ldg(ra + lane) : -1;
+    if (lane == 0) {
+      add(i - 1, 1);
+      add(i, both);
+      add(i + 1, both);
+      if (pair) add(i + 2, 2);
+      add(0, both);
+      add(p.nb - 1, both);
+    }
+    for (int t = 0; t < nrand; ++t) {
+      const int x = __shfl_sync(0xffffffffu, rv, t);
+      if (lane == 0) add(x, t < p.r ? 1 : 2);
+    }
+    top = i;
+    bot = pair ? i + 1 : -1;
   }
-  __syncthreads();
-  const int nkb = all ? p.nb : s.nlist;
-  const float log2e = 1.4426950408889634f;
-
-  float dq[4][4];  // rows 4ty.., dims 4tx..
-#pragma unroll
-  for (int a = 0; a < 4; ++a)
-#pragma unroll
-    for (int c = 0; c < 4; ++c) dq[a][c] = 0.f;
-
-  for (int e = 0; e < nkb; ++e) {
-    const int j = all ? e : s.list[e];
-    const size_t k0 = head + static_cast<size_t>(j) * kBlock;
-    load_tile(s.k, p.k, k0);
-    load_tile(s.v, p.v, k0);
-    if (t < kBlock) s.bias[t] = (p.seq_mask && !p.seq_mask[static_cast<size_t>(b) * p.L + j * kBlock + t]) ? -10000.f : 0.f;
-    __syncthreads();
-    // p and ds for rows 4ty..4ty+3 and keys 4tx..4tx+3 of the block
-    {
-      float sc[4][4], dp[4][4];
-#pragma unroll
-      for (int a = 0; a < 4; ++a)
-#pragma unroll
-        for (int c = 0; c < 4; ++c) sc[a][c] = dp[a][c] = 0.f;
-#pragma unroll 2
-      for (int x = 0; x < kDim; x += 4) {
-        float4 qa[4], ka[4], da[4], va[4];
-#pragma unroll
-        for (int a = 0; a < 4; ++a) {
-          qa[a] = *reinterpret_cast<const float4*>(&s.q[4 * ty + a][x]);
-          da[a] = *reinterpret_cast<const float4*>(&s.dout[4 * ty + a][x]);
-          ka[a] = *reinterpret_cast<const float4*>(&s.k[4 * tx + a][x]);
-          va[a] = *reinterpret_cast<const float4*>(&s.v[4 * tx + a][x]);
-        }
-#pragma unroll
-        for (int a = 0; a < 4; ++a)
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            sc[a][c] = fmaf(qa[a].x, ka[c].x, fmaf(qa[a].y, ka[c].y, fmaf(qa[a].z, ka[c].z, fmaf(qa[a].w, ka[c].w, sc[a][c]))));
-            dp[a][c] = fmaf(da[a].x, va[c].x, fmaf(da[a].y, va[c].y, fmaf(da[a].z, va[c].z, fmaf(da[a].w, va[c].w, dp[a][c]))));
-          }
-      }
-#pragma unroll
-      for (int a = 0; a < 4; ++a) {
-        const int rr = 4 * ty + a;
-        const float lse2 = s.lse[rr] * log2e;
-        const float dr = s.dsum[rr];
-        float4 pv4, ds4;
-        float* pv = reinterpret_cast<float*>(&pv4);
-        float* dsv = reinterpret_cast<float*>(&ds4);
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          pv[c] = exp2f(fmaf(sc[a][c], p.scale, s.bias[4 * tx + c]) * log2e - lse2);
-          dsv[c] = pv[c] * (dp[a][c] - dr);
-        }
-        *reinterpret_cast<float4*>(&s.p[rr][4 * tx]) = pv4;
-        *reinterpret_cast<float4*>(&s.ds[rr][4 * tx]) = ds4;
-      }
-    }
-    __syncthreads();
-    // dq[rows 4ty.., dims 4tx..] += ds[rows, all keys] . k[all keys, dims]
-#pragma unroll 4
-    for (int c = 0; c < kBlock; ++c) {
-      const float4 kv = *reinterpret_cast<const float4*>(&s.k[c][4 * tx]);
-#pragma unroll
-      for (int a = 0; a < 4; ++a) {
-        const float w = s.ds[4 * ty + a][c];
-        dq[a][0] = fmaf(w, kv.x, dq[a][0]);
-        dq[a][1] = fmaf(w, kv.y, dq[a][1]);
-        dq[a][2] = fmaf(w, kv.z, dq[a][2]);
-        dq[a][3] = fmaf(w, kv.w, dq[a][3]);
-      }
-    }
-    // dk[keys 4ty.., dims 4tx..] += ds^T q,  dv[keys 4ty.., dims 4tx..] += p^T dout
-    {
-      float dk[4][4], dv[4][4];
-#pragma unroll
-      for (int a = 0; a < 4; ++a)
-#pragma unroll
-        for (int c = 0; c < 4; ++c) dk[a][c] = dv[a][c] = 0.f;
-#pragma unroll 4
-      for (int rr = 0; rr < kBlock; ++rr) {
-        const float4 w = *reinterpret_cast<const float4*>(&s.ds[rr][4 * ty]);
-        const float4 pw = *reinterpret_cast<const float4*>(&s.p[rr][4 * ty]);
-        const float4 qv = *reinterpret_cast<const float4*>(&s.q[rr][4 * tx]);
-        const float4 dv4 = *reinterpret_cast<const float4*>(&s.dout[rr][4 * tx]);
-        const float ws[4] = {w.x, w.y, w.z, w.w};
-        const float ps[4] = {pw.x, pw.y, pw.z, pw.w};
-#pragma unroll
-        for (int a = 0; a < 4; ++a) {
-          dk[a][0] = fmaf(ws[a], qv.x, dk[a][0]);
-          dk[a][1] = fmaf(ws[a], qv.y, dk[a][1]);
-          dk[a][2] = fmaf(ws[a], qv.z, dk[a][2]);
-          dk[a][3] = fmaf(ws[a], qv.w, dk[a][3]);
-          dv[a][0] = fmaf(ps[a], dv4.x, dv[a][0]);
-          dv[a][1] = fmaf(ps[a], dv4.y, dv[a][1]);
-          dv[a][2] = fmaf(ps[a], dv4.z, dv[a][2]);
-          dv[a][3] = fmaf(ps[a], dv4.w, dv[a][3]);
-        }
-      }
-#pragma unroll
-      for (int a = 0; a < 4; ++a) {
-        float* dkp = p.dk + (k0 + 4 * ty + a) * kDim + 4 * tx;
-        float* dvp = p.dv + (k0 + 4 * ty + a) * kDim + 4 * tx;
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          atomicAdd(dkp + c, dk[a][c] * p.scale);
-          atomicAdd(dvp + c, dv[a][c]);
-        }
-      }
-    }
-    __syncthreads();
+  if (lane == 0) {
+    ui.n = n;
+    ui.bh = bh;
+    ui.top = top;
+    ui.bot = bot;
+    ui.split = split;
+    ui.first = 1;
+    ui.last = 1;
+    ui.stop = 0;
   }
-#pragma unroll
-  for (int a = 0; a < 4; ++a)
-    *reinterpret_cast<float4*>(p.dq + (q0 + 4 * ty + a) * kDim + 4 * tx) =
-        make_float4(dq[a][0] * p.scale, dq[a][1] * p.scale, dq[a][2] * p.scale, dq[a][3] * p.scale);
 }
+
+// ------------------------------------------------------------ preparation
+
+// Unit preparation and scheduling (one warp), up to four chunks ahead: a CTA's
+// first unit is its block index, later ones are tickets from the workspace
+// counter (units numbered longest first). Publishes a stop slot at the end.
+// The dk/dv kernel's middle units -- key blocks (j, j+1) -- list the query
+// blocks that attend either: the two global query blocks, the window
+// neighbours, and every middle query block whose random entries pick j or
+// j+1, found by scanning rand_attn 32 query blocks at a time (set semantics:
+// repeated or window-overlapping picks add nothing). A list longer than a
+// chunk goes out as several chunks; only the first starts the accumulators
+// from zero and only the last is followed by the epilogue.
+template <bool kKV>
+__device__ void prep_role(Smem& s, const Params& p) {
+  const int lane = threadIdx.x & 31;
+  uint32_t ut = 0;  // chunks published so far
+  auto acquire = [&]() -> Unit* {
+    int ok = 1;
+    if (lane == 0) ok = mbar_wait(smem_u32(&s.info_empty[ut & 3]), ((ut >> 2) & 1) ^ 1);
+    if (!__shfl_sync(0xffffffffu, ok, 0)) return nullptr;
+    return &s.unit[ut & 3];
+  };
+  auto finish = [&](Unit& ui) {
+    __syncwarp();
+    const int n = ui.n;
+    const int b = ui.bh / p.H;
+    if (!kKV)
+      for (int e = lane; e < n; e += 32) ui.vm[e] = p.seq_mask ? key_valid_bits(p.seq_mask, p.L, b, ui.mt[e]) : ~0ull;
+    __syncwarp();
+    if (lane == 0) mbar_arrive(smem_u32(&s.info_full[ut & 3]));
+    ++ut;
+    // the moving tiles into L2 ahead of the TMA loads
+    const size_t row0 = static_cast<size_t>(ui.bh) * p.L;
+    for (int t = lane; t < 2 * n; t += 32) {
+      const uint16_t* base = t < n ? (kKV ? p.q : p.k) : (kKV ? p.dout : p.v);
+      prefetch_l2_bulk(base + (row0 + static_cast<size_t>(ui.mt[t < n ? t : t - n]) * kBlock) * kDim, kTileBytes);
+    }
+  };
+  int u = blockIdx.x;
+  s.rbits[lane] = 0;
+  __syncwarp();
+  for (;;) {
+    Unit* ui = acquire();
+    if (!ui) {
+      if (lane == 0) flag_timeout(p);
+      return;
+    }
+    if (u >= p.total_units) {
+      if (lane == 0) {
+        ui->stop = 1;
+        mbar_arrive(smem_u32(&s.info_full[ut & 3]));
+      }
+      return;
+    }
+    int next = 0;
+    if (lane == 0) next = static_cast<int>(gridDim.x) + atomicAdd(&p.counters[0], 1);
+    if (!kKV || u >= p.n_mid_units) {
+      build_simple(p, u, *ui, lane);
+      finish(*ui);
+    } else {
+      const int bh = u / p.n_mid_per_head;
+      const int pp = u % p.n_mid_per_head;
+      const int h = bh % p.H;
+      const int j = 1 + 2 * pp;
+      const bool pair = j + 1 <= p.nb - 2;
+      auto header = [&](Unit& c, int first) {
+        if (lane == 0) {
+          c.bh = bh;
+          c.top = j;
+          c.bot = pair ? j + 1 : -1;
+          c.split = -1;
+          c.first = first;
+          c.last = 0;
+          c.stop = 0;
+        }
+      };
+      header(*ui, 1);
+      int n = 0;
+      bool ok = true;
+      for (int base = 0; base < p.nb && ok; base += 32) {
+        const int q = base + lane;
+        int hm = 0;
+        if (q < p.nb) {
+          if (q == 0 || q == p.nb - 1) {
+            hm = pair ? 3 : 1;
+          } else {
+            hm = (abs(q - j) <= 1 ? 1 : 0) | (pair && abs(q - (j + 1)) <= 1 ? 2 : 0);
+          }
+        }
+        // random picks of the middle query blocks qlo .. qhi-1 of this batch
+        const int qlo = max(base, 1), qhi = min(base + 32, p.nb - 1);
+        if (qhi > qlo) {
+          const int cnt = (qhi - qlo) * p.r;
+          const int32_t* ra = p.rand_attn + (static_cast<size_t>(h) * (p.nb - 2) + (qlo - 1)) * p.r;
+          for (int e = lane; e < cnt; e += 32) {
+            const int x = __ldg(ra + e);
+            if (x < 0 || x >= p.nb) atomicOr(p.status, kStatusBadRandAttn);
+            const int bits = (x == j ? 1 : 0) | (pair && x == j + 1 ? 2 : 0);
+            // lanes holding entries of the same query block meet here: atomic
+            if (bits) atomicOr(&s.rbits[qlo - base + e / p.r], static_cast<unsigned int>(bits));
+          }
+        }
+        __syncwarp();
+        hm |= static_cast<int>(s.rbits[lane]);
+        __syncwarp();
+        s.rbits[lane] = 0;
+        __syncwarp();
+        const uint32_t mask = __ballot_sync(0xffffffffu, hm != 0);
+        const int c = __popc(mask);
+        if (n + c > kMaxList) {
+          if (lane == 0) ui->n = n;
+          finish(*ui);
+          ui = acquire();
+          if (!ui) {
+            ok = false;
+            break;
+          }
+          header(*ui, 0);
+          n = 0;
+        }
+        if (hm) {
+          const int pos = n + __popc(mask & ((1u << lane) - 1u));
+          ui->mt[pos] = q;
+          ui->hm[pos] = static_cast<uint8_t>(hm);
+        }
+        n += c;
+      }
+      if (!ok) {
+        if (lane == 0) flag_timeout(p);
+        return;
+      }
+      if (lane == 0) {
+        ui->n = n;
+        ui->last = 1;
+      }
+      finish(*ui);
+    }
+    u = __shfl_sync(0xffffffffu, next, 0);
+  }
+}
+
+// ------------------------------------------------------------ TMA
+
+// Stationary tiles once per unit (after the previous unit's last S/dP MMAs
+// have read them), then the two moving tiles of every step (and, in the dk/dv
+// kernel, the query tile's lse and D) into a 2-deep ring.
+// dq kernel: A1 = Q, A2 = dO, B1 = K, B2 = V. dk/dv kernel: A1 = K, A2 = V,
+// B1 = Q, B2 = dO.
+template <bool kKV>
+__device__ void producer_role(Smem& s, const Params& p, const CUtensorMap* tmA1, const CUtensorMap* tmA2,
+                              const CUtensorMap* tmB1, const CUtensorMap* tmB2) {
+  const int lane = threadIdx.x & 31;
+  const uint64_t pol_a = l2_policy_evict_first();
+  const uint64_t pol_b = l2_policy_evict_last();
+  uint32_t g = 0, ua = 0;
+  for (uint32_t ut = 0;; ++ut) {
+    if (!warp_wait(smem_u32(&s.info_full[ut & 3]), (ut >> 2) & 1)) {
+      if (lane == 0) flag_timeout(p);
+      return;
+    }
+    const Unit& ui = s.unit[ut & 3];
+    if (ui.stop) break;
+    int ok = 1;
+    if (lane == 0) {
+      const int32_t row0 = ui.bh * p.L;
+      if (ui.first) {
+        ok = mbar_wait(smem_u32(&s.a_free), (ua & 1) ^ 1);
+        if (ok) {
+          const uint32_t bar = smem_u32(&s.a_full);
+          mbar_arrive_expect_tx(bar, (ui.bot >= 0 ? 4 : 2) * kTileBytes);
+          tma_load_2d(smem_u32(s.a1), tmA1, bar, 0, row0 + ui.top * kBlock, pol_a);
+          tma_load_2d(smem_u32(s.a2), tmA2, bar, 0, row0 + ui.top * kBlock, pol_a);
+          if (ui.bot >= 0) {
+            tma_load_2d(smem_u32(s.a1) + kTileBytes, tmA1, bar, 0, row0 + ui.bot * kBlock, pol_a);
+            tma_load_2d(smem_u32(s.a2) + kTileBytes, tmA2, bar, 0, row0 + ui.bot * kBlock, pol_a);
+          }
+        }
+        ++ua;
+      }
+      for (int e = 0; e < ui.n && ok; ++e, ++g) {
+        const int st = g % kStages;
+        ok = mbar_wait(smem_u32(&s.b_empty[st]), ((g / kStages) & 1) ^ 1);
+        if (!ok) break;
+        const uint32_t bar = smem_u32(&s.b_full[st]);
+        const int32_t row = row0 + ui.mt[e] * kBlock;
+        mbar_arrive_expect_tx(bar, 2 * kTileBytes + (kKV ? 2 * kBlock * 4 : 0));
+        tma_load_2d(smem_u32(s.b1[st]), tmB1, bar, 0, row, pol_b);
+        tma_load_2d(smem_u32(s.b2[st]), tmB2, bar, 0, row, pol_b);
+        if (kKV) {
+          bulk_load(smem_u32(s.col_lse[st]), p.lse + row, kBlock * 4, bar);
+          bulk_load(smem_u32(s.col_d[st]), p.dd + row, kBlock * 4, bar);
+        }
+      }
+    }
+    if (!__shfl_sync(0xffffffffu, ok, 0)) {
+      if (lane == 0) flag_timeout(p);
+      return;
+    }
+    g = __shfl_sync(0xffffffffu, g, 0);
+    ua = __shfl_sync(0xffffffffu, ua, 0);
+    __syncwarp();
+    if (lane == 0) mbar_arrive(smem_u32(&s.info_empty[ut & 3]));
+  }
+}
+
+// ------------------------------------------------------------ MMA
+
+// One thread. Per step: X = A1 B1^T, Y = A2 B2^T (SS, M = 128, N = 64,
+// K = 64), once the previous step's gradient MMAs have read P and dS out of
+// those columns; then, once P and dS are written, the gradient MMAs (TS, the
+// moving tile as B with d contiguous, K = 64 moving rows; P and dS in two
+// terms, hi from TMEM, lo from TMEM (dq) or shared memory (dk/dv, SS-MMAs)):
+//   dq kernel:   acc1 += (dS_hi + dS_lo) B1                          (dQ += dS K)
+//   dk/dv kernel: acc1 += (P_hi + P_lo) B2, acc2 += (dS_hi + dS_lo) B1 (dV += P^T dO, dK += dS^T Q)
+template <bool kKV>
+__device__ void mma_role(Smem& s, const Params& p, uint32_t tmem) {
+  const uint32_t idesc1 = idesc_f32acc(kRows, kBlock, true, false);
+  const uint32_t idesc2 = idesc_f32acc(kRows, kDim, true, true);
+  const uint32_t a1 = smem_u32(s.a1), a2 = smem_u32(s.a2);
+  uint32_t g = 0, ua = 0;
+  bool ok = true;
+  for (uint32_t ut = 0; ok; ++ut) {
+    if (!mbar_wait(smem_u32(&s.info_full[ut & 3]), (ut >> 2) & 1)) { ok = false; break; }
+    const Unit& ui = s.unit[ut & 3];
+    if (ui.stop) break;
+    const int n = ui.n;
+    const bool first = ui.first, last = ui.last;
+    if (first && !mbar_wait(smem_u32(&s.a_full), ua & 1)) { ok = false; break; }
+    for (int e = 0; e < n; ++e, ++g) {
+      const int st = g % kStages;
+      if (!mbar_wait(smem_u32(&s.b_full[st]), (g / kStages) & 1)) { ok = false; break; }
+      if (g >= 1 && !mbar_wait(smem_u32(&s.g2_done), (g - 1) & 1)) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t b1 = smem_u32(s.b1[st]), b2 = smem_u32(s.b2[st]);
+#pragma unroll
+      for (int kk = 0; kk < kDim / 16; ++kk)
+        mma_ss(tmem + kColX, sdesc_sw128(a1 + kk * 32, 16, 1024), sdesc_sw128(b1 + kk * 32, 16, 1024), idesc1,
+               kk > 0 ? 1u : 0u);
+#pragma unroll
+      for (int kk = 0; kk < kDim / 16; ++kk)
+        mma_ss(tmem + kColY, sdesc_sw128(a2 + kk * 32, 16, 1024), sdesc_sw128(b2 + kk * 32, 16, 1024), idesc1,
+               kk > 0 ? 1u : 0u);
+      mma_commit(smem_u32(&s.x_full));
+      if (last && e == n - 1) mma_commit(smem_u32(&s.a_free));
+      // the unit's first step overwrites the accumulators, once the previous
+      // unit's epilogue has read them
+      const bool zero = first && e == 0;
+      if (zero && !mbar_wait(smem_u32(&s.acc_free), (ua & 1) ^ 1)) { ok = false; break; }
+      if (!mbar_wait(smem_u32(&s.p_full), g & 1)) { ok = false; break; }
+      tc_fence_after();
+      if (kKV) {
+#pragma unroll
+        for (int kk = 0; kk < kBlock / 16; ++kk)
+          mma_ts(tmem + kColA1, tmem + kColX + kk * 8, sdesc_sw128(b2 + kk * 2048, 8192, 1024), idesc2,
+                 (zero && kk == 0) ? 0u : 1u);
+#pragma unroll
+        for (int kk = 0; kk < kBlock / 16; ++kk)
+          mma_ts(tmem + kColA2, tmem + kColY + kk * 8, sdesc_sw128(b1 + kk * 2048, 8192, 1024), idesc2,
+                 (zero && kk == 0) ? 0u : 1u);
+        const uint32_t plo = smem_u32(s.plo), dslo = smem_u32(s.dslo);
+#pragma unroll
+        for (int kk = 0; kk < kBlock / 16; ++kk)
+          mma_ss(tmem + kColA1, sdesc_sw128(plo + kk * 32, 16, 1024), sdesc_sw128(b2 + kk * 2048, 8192, 1024), idesc2,
+                 1u);
+#pragma unroll
+        for (int kk = 0; kk < kBlock / 16; ++kk)
+          mma_ss(tmem + kColA2, sdesc_sw128(dslo + kk * 32, 16, 1024), sdesc_sw128(b1 + kk * 2048, 8192, 1024), idesc2,
+                 1u);
+      } else {
+#pragma unroll
+        for (int kk = 0; kk < kBlock / 16; ++kk)
+          mma_ts(tmem + kColA1, tmem + kColY + kk * 8, sdesc_sw128(b1 + kk * 2048, 8192, 1024), idesc2,
+                 (zero && kk == 0) ? 0u : 1u);
+#pragma unroll
+        for (int kk = 0; kk < kBlock / 16; ++kk)
+          mma_ts(tmem + kColA1, tmem + kColX + 32 + kk * 8, sdesc_sw128(b1 + kk * 2048, 8192, 1024), idesc2, 1u);
+      }
+      mma_commit(smem_u32(&s.g2_done));
+      mma_commit(smem_u32(&s.b_empty[st]));
+      if (last && e == n - 1) mma_commit(smem_u32(&s.acc_full));
+    }
+    if (!ok) break;
+    if (first) ++ua;
+    mbar_arrive(smem_u32(&s.info_empty[ut & 3]));
+  }
+  if (!ok) flag_timeout(p);
+}
+
+// ------------------------------------------------------------ elementwise
+
+// 16 columns of one row: P = exp2((x + bias) scale_log2 - lse2) and
+// dS = P (y - D), each as two bf16 terms, hi = bf16(x) and lo = bf16(x - hi),
+// packed in pairs: the products then see about 16 significant bits of P and
+// dS. (One bf16 rounding leaves about 2^-9 relative error in each term, and
+// dq, dk and dv are sums of terms of either sign, so that error would reach
+// the gradients nearly undiminished.)
+template <bool kKV>
+__device__ __forceinline__ void piece_pds(const uint32_t (&x)[16], const uint32_t (&y)[16], int c0, uint64_t vm,
+                                          float row_bias, float row_lse2, float row_d, const float* col_lse,
+                                          const float* col_d, const Params& p, uint32_t (&pk)[8],
+                                          uint32_t (&pl)[8], uint32_t (&dk)[8], uint32_t (&dl)[8]) {
+  constexpr float kLog2e = 1.4426950408889634f;
+#pragma unroll
+  for (int c = 0; c < 16; c += 2) {
+    float pv[2], dv[2];
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+      const int col = c0 + c + t;
+      float bias, lse2, dd;
+      if (kKV) {
+        bias = row_bias;
+        lse2 = col_lse[col] * kLog2e;
+        dd = col_d[col];
+      } else {
+        bias = ((vm >> col) & 1ull) ? 0.f : p.bias_raw;
+        lse2 = row_lse2;
+        dd = row_d;
+      }
+      const float pr = ex2_approx(fmaf(__uint_as_float(x[c + t]) + bias, p.scale_log2, -lse2));
+      pv[t] = pr;
+      dv[t] = pr * (__uint_as_float(y[c + t]) - dd);
+    }
+    const uint32_t phi = pack_bf16x2(pv[0], pv[1]);
+    pk[c / 2] = phi;
+    pl[c / 2] = pack_bf16x2(pv[0] - __uint_as_float(phi << 16), pv[1] - __uint_as_float(phi & 0xFFFF0000u));
+    const uint32_t hi = pack_bf16x2(dv[0], dv[1]);
+    dk[c / 2] = hi;
+    dl[c / 2] = pack_bf16x2(dv[0] - __uint_as_float(hi << 16), dv[1] - __uint_as_float(hi & 0xFFFF0000u));
+  }
+}
+
+// Warps 0-3, one stationary row per thread (TMEM lane). Per step: read S and
+// dP (64 columns each) and write P and dS_hi as bf16 over their first 32
+// columns and dS_lo over the last 32 of S (once all of S is read); a half
+// whose rows do not use the tile writes zeros. After a unit's
+// last step: the epilogue (dq = acc1 / sqrt(d); dv = acc1, dk = acc2 /
+// sqrt(d)), raw into the partial-sum slot for a split global unit.
+template <bool kKV>
+__device__ void elem_role(Smem& s, const Params& p, uint32_t tmem) {
+  constexpr float kLog2e = 1.4426950408889634f;
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
+  const int half = warp >> 1;
+  const uint32_t lane_addr = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+  uint32_t g = 0, ua = 0;
+  float row_lse2 = 0.f, row_d = 0.f, row_bias = 0.f;
+  for (uint32_t ut = 0;; ++ut) {
+    if (!warp_wait(smem_u32(&s.info_full[ut & 3]), (ut >> 2) & 1)) { if (lane == 0) flag_timeout(p); return; }
+    const Unit& ui = s.unit[ut & 3];
+    if (ui.stop) break;
+    const int n = ui.n;
+    const int stile = half ? ui.bot : ui.top;
+    const bool exists = stile >= 0;
+    const int bh = ui.bh;
+    const size_t row = static_cast<size_t>(bh) * p.L + static_cast<size_t>(exists ? stile : 0) * kBlock + (tid & 63);
+    if (ui.first && exists) {
+      if (kKV) {
+        const int b = bh / p.H;
+        const bool valid = !p.seq_mask || p.seq_mask[static_cast<size_t>(b) * p.L + (row - static_cast<size_t>(bh) * p.L)] != 0;
+        row_bias = valid ? 0.f : p.bias_raw;
+      } else {
+        row_lse2 = __ldg(p.lse + row) * kLog2e;
+        row_d = __ldg(p.dd + row);
+      }
+    }
+    for (int e = 0; e < n; ++e, ++g) {
+      const bool used = exists && ((ui.hm[e] >> half) & 1);
+      if (!warp_wait(smem_u32(&s.x_full), g & 1)) { if (lane == 0) flag_timeout(p); return; }
+      tc_fence_after();
+      const int st = g % kStages;
+      if (kKV && !warp_wait(smem_u32(&s.b_full[st]), (g / kStages) & 1)) { if (lane == 0) flag_timeout(p); return; }
+      if (used && kKV) {
+        // P_hi, dS_hi into TMEM over S^T and dP^T; P_lo, dS_lo into shared
+        // memory (row tid, 16-byte chunk c at chunk c ^ (tid & 7))
+        uint8_t* rp = s.plo + (tid >> 3) * 1024 + (tid & 7) * 128;
+        uint8_t* rd = s.dslo + (tid >> 3) * 1024 + (tid & 7) * 128;
+#pragma unroll 1
+        for (int q = 0; q < 4; ++q) {
+          uint32_t x[16], y[16], pk[8], pl[8], dk[8], dl[8];
+          tmem_ld16(lane_addr + kColX + 16 * q, x);
+          tmem_ld16(lane_addr + kColY + 16 * q, y);
+          tmem_wait_ld();
+          piece_pds<kKV>(x, y, 16 * q, ~0ull, row_bias, row_lse2, row_d, s.col_lse[st], s.col_d[st], p, pk, pl, dk,
+                         dl);
+          tmem_st8(lane_addr + kColX + 8 * q, pk);
+          tmem_st8(lane_addr + kColY + 8 * q, dk);
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int chunk = (2 * q + h) ^ (tid & 7);
+            *reinterpret_cast<uint4*>(rp + chunk * 16) = make_uint4(pl[4 * h], pl[4 * h + 1], pl[4 * h + 2], pl[4 * h + 3]);
+            *reinterpret_cast<uint4*>(rd + chunk * 16) = make_uint4(dl[4 * h], dl[4 * h + 1], dl[4 * h + 2], dl[4 * h + 3]);
+          }
+        }
+        fence_proxy_async_smem();
+      } else if (used) {
+        const uint64_t vm = ui.vm[e];
+        uint32_t lo[4][8];  // dS_lo, written once every S column has been read
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          uint32_t x[16], y[16], pk[8], pl[8], dk[8];
+          tmem_ld16(lane_addr + kColX + 16 * q, x);
+          tmem_ld16(lane_addr + kColY + 16 * q, y);
+          tmem_wait_ld();
+          piece_pds<kKV>(x, y, 16 * q, vm, row_bias, row_lse2, row_d, s.col_lse[st], s.col_d[st], p, pk, pl, dk,
+                         lo[q]);
+          tmem_st8(lane_addr + kColX + 8 * q, pk);
+          tmem_st8(lane_addr + kColY + 8 * q, dk);
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) tmem_st8(lane_addr + kColX + 32 + 8 * q, lo[q]);
+      } else {
+        uint32_t z[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) z[i] = 0u;
+        tmem_st16(lane_addr + kColX, z);
+        tmem_st16(lane_addr + kColX + 16, z);
+        tmem_st16(lane_addr + kColX + 32, z);
+        tmem_st16(lane_addr + kColX + 48, z);
+        tmem_st16(lane_addr + kColY, z);
+        tmem_st16(lane_addr + kColY + 16, z);
+        if (kKV) {
+          uint4* rp = reinterpret_cast<uint4*>(s.plo + (tid >> 3) * 1024 + (tid & 7) * 128);
+          uint4* rd = reinterpret_cast<uint4*>(s.dslo + (tid >> 3) * 1024 + (tid & 7) * 128);
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            rp[c] = make_uint4(0u, 0u, 0u, 0u);
+            rd[c] = make_uint4(0u, 0u, 0u, 0u);
+          }
+          fence_proxy_async_smem();
+        }
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&s.p_full));
+    }
+    const bool last = ui.last;
+    const int split = ui.split;
+    __syncwarp();
+    if (lane == 0) mbar_arrive(smem_u32(&s.info_empty[ut & 3]));
+    if (!last) continue;
+    // ---- epilogue
+    if (!warp_wait(smem_u32(&s.acc_full), ua & 1)) { if (lane == 0) flag_timeout(p); return; }
+    tc_fence_after();
+    if (exists) {
+      const size_t prow = (static_cast<size_t>(bh) * p.nsplit + (split >= 0 ? split : 0)) * kRows + tid;
+#pragma unroll 1
+      for (int a = 0; a < (kKV ? 2 : 1); ++a) {
+        // acc1: dq (dq kernel) or dv; acc2: dk
+        const float f = (split >= 0 || (kKV && a == 0)) ? 1.f : p.scale;
+        float* dst = split >= 0 ? (a == 0 ? p.part1 : p.part2) + prow * kDim : (a == 0 ? p.g1 : p.g2) + row * kDim;
+#pragma unroll 1
+        for (int c0 = 0; c0 < kDim; c0 += 16) {
+          uint32_t o[16];
+          tmem_ld16(lane_addr + (a == 0 ? kColA1 : kColA2) + c0, o);
+          tmem_wait_ld();
+          float4* d4 = reinterpret_cast<float4*>(dst + c0);
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+            d4[c] = make_float4(__uint_as_float(o[4 * c]) * f, __uint_as_float(o[4 * c + 1]) * f,
+                                __uint_as_float(o[4 * c + 2]) * f, __uint_as_float(o[4 * c + 3]) * f);
+        }
+      }
+    }
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(smem_u32(&s.acc_free));
+    ++ua;
+  }
+}
+
+// ------------------------------------------------------------ kernels
+
+// kKV = false: dq. kKV = true: dk and dv.
+template <bool kKV>
+__global__ void __launch_bounds__(kThreads, kCtasPerSm)
+bwd_kernel(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmA2,
+           const __grid_constant__ CUtensorMap tmB1, const __grid_constant__ CUtensorMap tmB2,
+           const __grid_constant__ Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  Smem& s = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  if (warp == 5) {
+    tmem_alloc(smem_u32(&s.tmem_base), kTmemCols);
+    tmem_relinquish();
+  }
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 4; ++i) {
+      mbar_init(smem_u32(&s.info_full[i]), 1);
+      mbar_init(smem_u32(&s.info_empty[i]), 1 + 1 + 4);  // TMA, MMA, 4 elementwise warps
+    }
+    mbar_init(smem_u32(&s.a_full), 1);
+    mbar_init(smem_u32(&s.a_free), 1);
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(smem_u32(&s.b_full[i]), 1);
+      mbar_init(smem_u32(&s.b_empty[i]), 1);
+    }
+    mbar_init(smem_u32(&s.x_full), 1);
+    mbar_init(smem_u32(&s.p_full), 4);
+    mbar_init(smem_u32(&s.g2_done), 1);
+    mbar_init(smem_u32(&s.acc_full), 1);
+    mbar_init(smem_u32(&s.acc_free), 4);
+    fence_barrier_init();
+  }
+  if (warp == 4 && lane == 0) {
+    tma_prefetch_desc(&tmA1);
+    tma_prefetch_desc(&tmA2);
+    tma_prefetch_desc(&tmB1);
+    tma_prefetch_desc(&tmB2);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s.tmem_base;
+  if (warp < 4) {
+    elem_role<kKV>(s, p, tmem);
+  } else if (warp == 4) {
+    producer_role<kKV>(s, p, &tmA1, &tmA2, &tmB1, &tmB2);
+  } else if (warp == 5) {
+    if (lane == 0) mma_role<kKV>(s, p, tmem);
+  } else if (warp == 6) {
+    prep_role<kKV>(s, p);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 5) {
+    __syncwarp();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+  // the CTA that finishes last sets this kernel's counters back to zero
+  if (threadIdx.x == 0) {
+    __threadfence();
+    if (atomicAdd(&p.counters[1], 1) == static_cast<int>(gridDim.x) - 1) {
+      p.counters[0] = 0;
+      p.counters[1] = 0;
+    }
+  }
+}
+
+// D[row] = sum_c dout[row, c] * out[row, c]: 16 threads per row, 4 columns
+// each; a CTA of 256 threads covers 16 rows.
+__global__ void __launch_bounds__(256)
+bwd_rowdot_kernel(const uint16_t* __restrict__ dout, const void* __restrict__ out, int out_f32, float* __restrict__ dd,
+                  size_t rows) {
+  const size_t row = static_cast<size_t>(blockIdx.x) * 16 + (threadIdx.x >> 4);
+  const int c4 = threadIdx.x & 15;
+  float acc = 0.f;
+  if (row < rows) {
+    const uint2 g = __ldg(reinterpret_cast<const uint2*>(dout + row * kDim) + c4);
+    float o[4];
+    if (out_f32) {
+      const float4 t = __ldg(reinterpret_cast<const float4*>(static_cast<const float*>(out) + row * kDim) + c4);
+      o[0] = t.x; o[1] = t.y; o[2] = t.z; o[3] = t.w;
+    } else {
+      const uint2 t = __ldg(reinterpret_cast<const uint2*>(static_cast<const uint16_t*>(out) + row * kDim) + c4);
+      o[0] = __uint_as_float(t.x << 16); o[1] = __uint_as_float(t.x & 0xFFFF0000u);
+      o[2] = __uint_as_float(t.y << 16); o[3] = __uint_as_float(t.y & 0xFFFF0000u);
+    }
+    acc = __uint_as_float(g.x << 16) * o[0] + __uint_as_float(g.x & 0xFFFF0000u) * o[1] +
+          __uint_as_float(g.y << 16) * o[2] + __uint_as_float(g.y & 0xFFFF0000u) * o[3];
+  }
+#pragma unroll
+  for (int off = 8; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+  if (row < rows && c4 == 0) dd[row] = acc;
+}
+
+// The split global units' partial sums: rows 0..63 of a unit belong to tile 0
+// and rows 64..127 to tile nb-1 of head bh; dst = f * sum over the ranges.
+// 16 threads per row, 4 columns each; grid (B*H, 128 / 16).
+__global__ void __launch_bounds__(256)
+bwd_sum_kernel(const float* __restrict__ part, float* __restrict__ dst, int nsplit, int L, int nb, float f) {
+  const int bh = blockIdx.x;
+  const int r = blockIdx.y * 16 + (threadIdx.x >> 4);
+  const int c4 = threadIdx.x & 15;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int sidx = 0; sidx < nsplit; ++sidx) {
+    const float4 t =
+        __ldg(reinterpret_cast<const float4*>(part + ((static_cast<size_t>(bh) * nsplit + sidx) * kRows + r) * kDim) + c4);
+    acc.x += t.x;
+    acc.y += t.y;
+    acc.z += t.z;
+    acc.w += t.w;
+  }
+  const int tile = r < kBlock ? 0 : nb - 1;
+  const size_t row = static_cast<size_t>(bh) * L + static_cast<size_t>(tile) * kBlock + (r & (kBlock - 1));
+  reinterpret_cast<float4*>(dst + row * kDim)[c4] = make_float4(acc.x * f, acc.y * f, acc.z * f, acc.w * f);
+}
+
+static_assert(sizeof(Smem) + 1024 <= kSmemRequest, "shared memory request below the kernel's use");
+static_assert(3 * (kSmemRequest + 1024) > 228 * 1024, "a third CTA per SM would wait for TMEM");
 
 }  // namespace bbw
+
+// ------------------------------------------------------------ host
+
+namespace {
+
+struct BwdPlan {
+  int nb = 0;
+  bool sparse = false;
+  int nsplit = 1;
+  size_t d_off = 0, partq_off = 0, partv_off = 0, partk_off = 0, bytes = 0;
+};
+
+int bwd_plan(int B, int H, int L, int d, int block, int r, unsigned flags, BwdPlan& pl) {
+  using namespace bbw;
+  if (B <= 0 || H <= 0 || L <= 0 || d <= 0 || block <= 0 || r < 1 || L % block != 0) return BB_ERR_INVALID_ARG;
+  if (d != kDim || block != kBlock || r > kMaxR) return BB_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(B) * H * L >= (int64_t(1) << 31)) return BB_ERR_UNSUPPORTED;
+  pl.nb = L / block;
+  pl.sparse = (flags & BB_FLAG_FORCE_SPARSE) || pl.nb > 5 + 2 * r;
+  if (pl.sparse && pl.nb < 5 + r) return BB_ERR_INVALID_ARG;
+  // a full-attention unit lists every block: nb <= 5 + 2r <= kMaxList
+  pl.nsplit = pl.sparse ? (pl.nb + kSplit - 1) / kSplit : 1;
+  auto round256 = [](size_t x) { return (x + 255) / 256 * 256; };
+  const size_t bhl = static_cast<size_t>(B) * H * L;
+  pl.d_off = kCounterBytes;
+  size_t off = pl.d_off + round256(bhl * sizeof(float));
+  if (pl.nsplit > 1) {
+    const size_t part = static_cast<size_t>(B) * H * pl.nsplit * kRows * kDim * sizeof(float);
+    pl.partq_off = off;
+    pl.partv_off = off + part;
+    pl.partk_off = off + 2 * part;
+    off += 3 * part;
+  }
+  pl.bytes = off;
+  return BB_OK;
+}
+
+bool set_attributes(int dev) {
+  using namespace bbw;
+  static bool done[64] = {};
+  if (dev < 0 || dev >= 64) return false;
+  if (done[dev]) return true;
+  const int smem = kSmemRequest;
+  for (const void* fn : {reinterpret_cast<const void*>(bwd_kernel<false>), reinterpret_cast<const void*>(bwd_kernel<true>)}) {
+    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) return false;
+    if (cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout, 100) != cudaSuccess) return false;
+  }
+  done[dev] = true;
+  return true;
+}
+
+}  // namespace
+
+extern "C" size_t bigbird_attn_bwd_workspace_size(int B, int H, int L, int d, int block, int r, unsigned flags) {
+  BwdPlan pl;
+  return bwd_plan(B, H, L, d, block, r, flags, pl) == BB_OK ? pl.bytes : 0;
+}
+
+extern "C" int bigbird_attn_bwd_ex(const void* q, const void* k, const void* v, const void* out, const void* dout,
+                                   const float* lse, const int32_t* rand_attn, const uint8_t* seq_mask, float* dq,
+                                   float* dk, float* dv, int B, int H, int L, int d, int block, int r, int out_dtype,
+                                   unsigned flags, void* workspace, size_t workspace_bytes, void* stream_) {
+  using namespace bbw;
+  BwdPlan pl;
+  const int st = bwd_plan(B, H, L, d, block, r, flags, pl);
+  if (st != BB_OK) return st;
+  if (!q || !k || !v || !out || !dout || !lse || !dq || !dk || !dv) return BB_ERR_INVALID_ARG;
+  if (out_dtype != BB_OUT_BF16 && out_dtype != BB_OUT_F32) return BB_ERR_INVALID_ARG;
+  if (pl.sparse && !rand_attn) return BB_ERR_INVALID_ARG;
+  auto misaligned = [](const void* ptr, uintptr_t a) { return (reinterpret_cast<uintptr_t>(ptr) & (a - 1)) != 0; };
+  if (misaligned(q, 16) || misaligned(k, 16) || misaligned(v, 16) || misaligned(out, 16) || misaligned(dout, 16) ||
+      misaligned(lse, 16) || misaligned(dq, 16) || misaligned(dk, 16) || misaligned(dv, 16))
+    return BB_ERR_UNSUPPORTED;
+  if (workspace && (misaligned(workspace, 256) || workspace_bytes < pl.bytes)) return BB_ERR_INVALID_ARG;
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  int dev = 0, major = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return BB_ERR_CUDA;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return BB_ERR_CUDA;
+  if (major != 10) return BB_ERR_UNSUPPORTED;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return BB_ERR_CUDA;
+  uint32_t* status = status_word(dev);
+  if (!status || !set_attributes(dev)) return BB_ERR_CUDA;
+
+  const size_t rows = static_cast<size_t>(B) * H * L;
+  CUtensorMap tq, tk, tv, tdo;
+  if (!make_tile_map(&tq, q, rows) || !make_tile_map(&tk, k, rows) || !make_tile_map(&tv, v, rows) ||
+      !make_tile_map(&tdo, dout, rows))
+    return BB_ERR_CUDA;
+
+  void* ws = workspace;
+  bool owned = false;
+  if (!ws) {
+    if (cudaMallocAsync(&ws, pl.bytes, stream) != cudaSuccess) return BB_ERR_CUDA;
+    owned = true;
+    if (cudaMemsetAsync(ws, 0, kCounterBytes, stream) != cudaSuccess) {
+      cudaFreeAsync(ws, stream);
+      return BB_ERR_CUDA;
+    }
+  }
+  uint8_t* wsb = static_cast<uint8_t*>(ws);
+  float* dd = reinterpret_cast<float*>(wsb + pl.d_off);
+
+  Params p{};
+  p.q = static_cast<const uint16_t*>(q);
+  p.k = static_cast<const uint16_t*>(k);
+  p.v = static_cast<const uint16_t*>(v);
+  p.dout = static_cast<const uint16_t*>(dout);
+  p.lse = lse;
+  p.dd = dd;
+  p.rand_attn = rand_attn;
+  p.seq_mask = seq_mask;
+  p.status = status;
+  p.H = H;
+  p.L = L;
+  p.nb = pl.nb;
+  p.r = r;
+  p.BH = B * H;
+  p.sparse = pl.sparse ? 1 : 0;
+  p.nsplit = pl.nsplit;
+  p.n_mid_per_head = pl.sparse ? (pl.nb - 2 + 1) / 2 : 0;
+  p.n_mid_units = p.BH * p.n_mid_per_head;
+  p.total_units = p.n_mid_units + p.BH * (pl.sparse ? pl.nsplit : (pl.nb + 1) / 2);
+  p.scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(d));
+  p.bias_raw = -10000.0f * sqrtf(static_cast<float>(d));
+  p.scale = 1.0f / sqrtf(static_cast<float>(d));
+
+  const int grid = std::min(p.total_units, kCtasPerSm * sms);
+  const size_t smem = kSmemRequest;
+  bwd_rowdot_kernel<<<static_cast<unsigned>((rows + 15) / 16), 256, 0, stream>>>(
+      static_cast<const uint16_t*>(dout), out, out_dtype == BB_OUT_F32 ? 1 : 0, dd, rows);
+  // dq
+  Params pq = p;
+  pq.g1 = dq;
+  pq.part1 = pl.nsplit > 1 ? reinterpret_cast<float*>(wsb + pl.partq_off) : nullptr;
+  pq.counters = reinterpret_cast<int*>(wsb);
+  bwd_kernel<false><<<grid, kThreads, smem, stream>>>(tq, tdo, tk, tv, pq);
+  // dk, dv
+  Params pk = p;
+  pk.g1 = dv;
+  pk.g2 = dk;
+  pk.part1 = pl.nsplit > 1 ? reinterpret_cast<float*>(wsb + pl.partv_off) : nullptr;
+  pk.part2 = pl.nsplit > 1 ? reinterpret_cast<float*>(wsb + pl.partk_off) : nullptr;
+  pk.counters = reinterpret_cast<int*>(wsb) + 2;
+  bwd_kernel<true><<<grid, kThreads, smem, stream>>>(tk, tv, tq, tdo, pk);
+  if (pl.nsplit > 1) {
+    const dim3 sg(p.BH, kRows / 16);
+    bwd_sum_kernel<<<sg, 256, 0, stream>>>(pq.part1, dq, pl.nsplit, L, pl.nb, p.scale);
+    bwd_sum_kernel<<<sg, 256, 0, stream>>>(pk.part1, dv, pl.nsplit, L, pl.nb, 1.0f);
+    bwd_sum_kernel<<<sg, 256, 0, stream>>>(pk.part2, dk, pl.nsplit, L, pl.nb, p.scale);
+  }
+  const cudaError_t e = cudaGetLastError();
+  if (owned) cudaFreeAsync(ws, stream);
+  return e == cudaSuccess ? BB_OK : BB_ERR_CUDA;
+}
 
 extern "C" int bigbird_attn_bwd(const void* q, const void* k, const void* v, const void* out, const void* dout,
                                 const float* lse, const int32_t* rand_attn, const uint8_t* seq_mask, float* dq,
                                 float* dk, float* dv, int B, int H, int L, int d, int block, int r, int out_dtype,
-                                unsigned flags, void* stream_) {
-  using namespace bbw;
-  if (B <= 0 || H <= 0 || L <= 0 || d <= 0 || block <= 0 || r < 1 || L % block != 0) return BB_ERR_INVALID_ARG;
-  if (d != kDim || block != kBlock || r > 16) return BB_ERR_UNSUPPORTED;
-  if (static_cast<int64_t>(B) * H * L >= (int64_t(1) << 31)) return BB_ERR_UNSUPPORTED;
-  if (!q || !k || !v || !out || !dout || !lse || !dq || !dk || !dv) return BB_ERR_INVALID_ARG;
-  if (out_dtype != BB_OUT_BF16 && out_dtype != BB_OUT_F32) return BB_ERR_INVALID_ARG;
-  const int nb = L / block;
-  const bool sparse = (flags & BB_FLAG_FORCE_SPARSE) || nb > 5 + 2 * r;
-  if (sparse && nb < 5 + r) return BB_ERR_INVALID_ARG;
-  if (sparse && !rand_attn) return BB_ERR_INVALID_ARG;
-  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
-  const size_t bytes = static_cast<size_t>(B) * H * L * d * sizeof(float);
-  if (cudaMemsetAsync(dk, 0, bytes, stream) != cudaSuccess) return BB_ERR_CUDA;
-  if (cudaMemsetAsync(dv, 0, bytes, stream) != cudaSuccess) return BB_ERR_CUDA;
-  // (set on every call: the attribute is per device and the call is cheap)
-  const int smem = static_cast<int>(sizeof(Smem));
-  if (cudaFuncSetAttribute(bigbird_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-    return BB_ERR_CUDA;
-  BwdParams p{};
-  p.q = static_cast<const uint16_t*>(q);
-  p.k = static_cast<const uint16_t*>(k);
-  p.v = static_cast<const uint16_t*>(v);
-  p.out = out;
-  p.dout = static_cast<const uint16_t*>(dout);
-  p.lse = lse;
-  p.rand_attn = rand_attn;
-  p.seq_mask = seq_mask;
-  p.dq = dq;
-  p.dk = dk;
-  p.dv = dv;
-  p.H = H;
-  p.L = L;
-  p.nb = nb;
-  p.r = r;
-  p.sparse = sparse ? 1 : 0;
-  p.out_f32 = out_dtype == BB_OUT_F32 ? 1 : 0;
-  p.scale = 1.0f / sqrtf(static_cast<float>(d));
-  bigbird_bwd_kernel<<<dim3(nb, B * H), kThreads, smem, stream>>>(p);
-  return cudaGetLastError() == cudaSuccess ? BB_OK : BB_ERR_CUDA;
+                                unsigned flags, void* stream) {
+  return bigbird_attn_bwd_ex(q, k, v, out, dout, lse, rand_attn, seq_mask, dq, dk, dv, B, H, L, d, block, r, out_dtype,
+                             flags, nullptr, 0, stream);
 }

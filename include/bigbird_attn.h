@@ -157,20 +157,48 @@ int bigbird_attn_fwd_train(const void* q, const void* k, const void* v, const in
  * through each row's softmax (p recomputed as exp(s - lse)):
  *   dv = p^T dout,  dp = dout v^T,  ds = p (dp - rowsum(dout * out)),
  *   dq = ds k / sqrt(d),  dk = ds^T q / sqrt(d).
- *   q, k, v, dout  device bf16 [B, H, L, d] (dout: gradient of out).
+ *   q, k, v, dout  device bf16 [B, H, L, d] (dout: gradient of out), 16-byte aligned.
  *   out            device [B, H, L, d]: the forward's output, bf16 or fp32 (out_dtype).
  *   lse            device fp32 [B, H, L] from bigbird_attn_fwd_train.
  *   rand_attn, seq_mask, B, H, L, d, block, r, BB_FLAG_FORCE_SPARSE: as the forward.
- *   dq, dk, dv     device fp32 [B, H, L, d], written in full (dk and dv are
- *                  zeroed with cudaMemsetAsync on `stream`, then accumulated).
- * Asynchronous on `stream`; nothing is allocated. Errors as the forward
- * (d != 64 or block != 64 -> BB_ERR_UNSUPPORTED). Out-of-range rand_attn
- * entries are skipped.
+ *   dq, dk, dv     device fp32 [B, H, L, d], written in full, 16-byte aligned.
+ * Tensor cores (tcgen05, bf16 operands, fp32 accumulation): a row-dot
+ * kernel (D = rowsum(dout * out)), a query-stationary dq kernel, a
+ * key-stationary dk/dv kernel and, when the global rows are split into key
+ * ranges, a kernel summing their partial results -- no atomics, so the
+ * gradients are the same bit for bit on every run. The workspace (counters,
+ * D and the partial sums; bigbird_attn_bwd_workspace_size) is taken with
+ * cudaMallocAsync on `stream`, its counters zeroed with cudaMemsetAsync, and
+ * released with cudaFreeAsync; bigbird_attn_bwd_ex takes the caller's.
+ * Asynchronous on `stream`. Errors as the forward (d != 64 or block != 64 ->
+ * BB_ERR_UNSUPPORTED). Out-of-range rand_attn entries are skipped and flagged
+ * in bigbird_device_status.
  */
 int bigbird_attn_bwd(const void* q, const void* k, const void* v, const void* out, const void* dout,
                      const float* lse, const int32_t* rand_attn, const uint8_t* seq_mask, float* dq, float* dk,
                      float* dv, int B, int H, int L, int d, int block, int r, int out_dtype, unsigned flags,
                      void* stream);
+
+/*
+ * Bytes of device workspace bigbird_attn_bwd_ex needs (0 for invalid or
+ * unsupported sizes): 256 bytes of counters, D [B*H*L] fp32 (rounded up to
+ * 256 bytes) and, when the global rows are split into key ranges (sparse
+ * pattern, nb > 8), three partial-sum arrays [B*H, ceil(nb / 8), 128, 64]
+ * fp32 (dq of the global query blocks, dv and dk of the global key blocks).
+ */
+size_t bigbird_attn_bwd_workspace_size(int B, int H, int L, int d, int block, int r, unsigned flags);
+
+/*
+ * bigbird_attn_bwd_ex -- bigbird_attn_bwd with a caller-provided workspace:
+ * device, 256-byte aligned, at least bigbird_attn_bwd_workspace_size(...)
+ * bytes, zero-filled before its first use (every call that completes leaves
+ * its counters at zero again); NULL allocates one as bigbird_attn_bwd does.
+ * Calls that share a workspace must not overlap on the GPU.
+ */
+int bigbird_attn_bwd_ex(const void* q, const void* k, const void* v, const void* out, const void* dout,
+                        const float* lse, const int32_t* rand_attn, const uint8_t* seq_mask, float* dq, float* dk,
+                        float* dv, int B, int H, int L, int d, int block, int r, int out_dtype, unsigned flags,
+                        void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * Attention probabilities (the output_attentions path). The block-sparse model

@@ -135,3 +135,26 @@ def test_backward_full_size_head_and_identities():
             dv_sum_err=float(np.abs(dv.sum(axis=2) - dsum).max()))
     assert np.abs(dk.sum(axis=2)).max() <= 2e-4 * scale_k
     assert np.abs(dv.sum(axis=2) - dsum).max() <= 2e-4 * np.abs(dsum).max()
+
+
+def test_backward_deterministic_and_long_transposed_lists():
+    """The gradients are the same bit for bit on a second run (no atomics),
+    and a key block picked by every middle row's random entries (a transposed
+    list longer than one chunk of the dk/dv kernel) is handled."""
+    w = Workload("bwd_chunks", 1, 2, 64 * 64, pad=("fixed", [3900]), seed=21)
+    inp = make_inputs(w)
+    ra = oracle.rand_attn_generate(w.H, w.L, w.block, w.r, seed=6)
+    nb = w.nb
+    for h in range(w.H):  # every middle row outside block 5's window picks block 5 (set semantics elsewhere)
+        for i in range(1, nb - 1):
+            if abs(i - 5) > 1:
+                ra[h, i - 1, 0] = 5
+    do = _dout(w, 8)
+    first = _run(inp, w, ra, do)
+    again = _run(inp, w, ra, do)
+    for a, b in zip(first[2:], again[2:]):
+        assert np.array_equal(a, b)
+    out, lse, dq, dk, dv = first
+    gq, gk, gv = oracle.attention_backward(inp["q"], inp["k"], inp["v"], ra, inp["seq_mask"], w.block, w.r, do)
+    for name, got, want in (("dq", dq, gq), ("dk", dk, gk), ("dv", dv, gv)):
+        _check_grad(name, got, want, w.name)
