@@ -29,10 +29,11 @@
 //      are split over ranges; their partial sums (workspace) are added here.
 //
 // Both attention kernels are persistent (2 CTAs per SM, 256 TMEM columns:
-// S | dP | accumulator 1 | accumulator 2) and warp-specialised: warps 0-3 the
-// elementwise part and the epilogue, warp 4 TMA, warp 5 the MMAs (one
-// thread), warp 6 unit preparation and scheduling (tickets from a workspace
-// counter, reset by the CTA that finishes last). Every wait is bounded.
+// S | dP | accumulator 1 | accumulator 2) and warp-specialised: warps 0-7 the
+// elementwise part and the epilogue (two warps per row, 32 columns each),
+// warp 8 TMA, warp 9 the MMAs (one thread), warp 10 unit preparation and
+// scheduling (tickets from a workspace counter, reset by the CTA that
+// finishes last). Every wait is bounded.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -55,14 +56,15 @@ constexpr int kStages = 2;     // moving-tile ring depth
 constexpr int kMaxList = 42;   // moving tiles per unit chunk
 constexpr int kMaxR = 16;
 constexpr int kSplit = 8;      // tiles per range of a global unit
-constexpr int kThreads = 256;
+constexpr int kThreads = 384;  // warps 0-7 elementwise, 8 TMA, 9 MMA, 10 prep, 11 idle
+constexpr int kElemWarps = 8;
 constexpr int kCtasPerSm = 2;
 // Dynamic shared memory requested per CTA: more than the kernel uses, so that
 // at most two CTAs share an SM (each allocates half of its TMEM).
 constexpr int kSmemRequest = 112 * 1024;
 constexpr uint32_t kTileBytes = kBlock * kDim * 2;  // 8 KB
 constexpr uint32_t kTmemCols = 256;
-constexpr uint32_t kColX = 0;     // S (or S^T): 64 fp32 columns; P (bf16) overwrites the first 32, dS_lo the last 32
+constexpr uint32_t kColX = 0;     // S (or S^T): 64 fp32 columns; P_hi (bf16) overwrites the first 32
 constexpr uint32_t kColY = 64;    // dP (or dP^T): 64 fp32 columns; dS_hi (bf16) overwrites the first 32
 constexpr uint32_t kColA1 = 128;  // dQ, or dV
 constexpr uint32_t kColA2 = 192;  // dK
@@ -120,8 +122,8 @@ struct __align__(1024) Smem {
   uint8_t a2[kRows * kDim * 2];           // dO (dq) or V (dk/dv)
   uint8_t b1[kStages][kTileBytes];        // K (dq) or Q (dk/dv) of a step
   uint8_t b2[kStages][kTileBytes];        // V (dq) or dO (dk/dv)
-  uint8_t plo[kRows * kBlock * 2];        // dk/dv: P_lo and dS_lo of the step, [128 rows x 64] bf16,
-  uint8_t dslo[kRows * kBlock * 2];       //   laid out as a TMA box with 128-byte swizzle (an SS-MMA operand)
+  uint8_t plo[kRows * kBlock * 2];        // P_lo (dk/dv) and dS_lo of the step, [128 rows x 64] bf16, laid
+  uint8_t dslo[kRows * kBlock * 2];       //   out as a TMA box with 128-byte swizzle (an SS-MMA operand)
   float col_lse[kStages][kBlock];         // dk/dv: lse and D of the step's query tile
   float col_d[kStages][kBlock];
   Unit unit[4];
@@ -131,7 +133,7 @@ struct __align__(1024) Smem {
   uint64_t b_full[kStages], b_empty[kStages];
   uint64_t x_full;     // S and dP of the step are in TMEM
   uint64_t p_full;     // P and dS written (4 warps)
-  uint64_t g2_done;    // the step's gradient MMAs are complete (S/dP columns reusable)
+  uint64_t xy_free;    // the step's MMAs reading P_hi and dS_hi from TMEM are complete (S/dP columns reusable)
   uint64_t acc_full;   // a unit's accumulators are complete
   uint64_t acc_free;   // ... and read by the epilogue (4 warps)
   uint32_t tmem_base;
@@ -398,6 +400,12 @@ __device__ void prep_role(Smem& s, const Params& p) {
   }
 }
 
+// Columns 16q .. 16q+15 of the S / dP tiles: the hi terms of piece q go to
+// TMEM columns hi_col(q) .. +7 (packed pairs), which the warp that owns the
+// piece has already read: pieces 0, 1 (one warp) to 0..15, pieces 2, 3 (the
+// other warp of the same rows) to 32..47.
+__device__ __forceinline__ uint32_t hi_col(int q) { return 8 * q + 16 * (q >> 1); }
+
 // ------------------------------------------------------------ TMA
 
 // Stationary tiles once per unit (after the previous unit's last S/dP MMAs
@@ -465,10 +473,13 @@ __device__ void producer_role(Smem& s, const Params& p, const CUtensorMap* tmA1,
 // ------------------------------------------------------------ MMA
 
 // One thread. Per step: X = A1 B1^T, Y = A2 B2^T (SS, M = 128, N = 64,
-// K = 64), once the previous step's gradient MMAs have read P and dS out of
-// those columns; then, once P and dS are written, the gradient MMAs (TS, the
-// moving tile as B with d contiguous, K = 64 moving rows; P and dS in two
-// terms, hi from TMEM, lo from TMEM (dq) or shared memory (dk/dv, SS-MMAs)):
+// K = 64), once the previous step's hi-term MMAs have read P_hi and dS_hi
+// out of those columns; then, once P and dS are written, the gradient MMAs
+// (the moving tile as B with d contiguous, K = 64 moving rows; P and dS in
+// two terms, hi from TMEM (TS), lo from shared memory (SS)). The next step's
+// X and Y are issued behind the lo terms, which write other accumulators.
+// (MMAs of one thread complete in order, so x_full of the next step also
+// means the lo terms have read shared memory.)
 //   dq kernel:   acc1 += (dS_hi + dS_lo) B1                          (dQ += dS K)
 //   dk/dv kernel: acc1 += (P_hi + P_lo) B2, acc2 += (dS_hi + dS_lo) B1 (dV += P^T dO, dK += dS^T Q)
 template <bool kKV>
@@ -488,7 +499,7 @@ __device__ void mma_role(Smem& s, const Params& p, uint32_t tmem) {
     for (int e = 0; e < n; ++e, ++g) {
       const int st = g % kStages;
       if (!mbar_wait(smem_u32(&s.b_full[st]), (g / kStages) & 1)) { ok = false; break; }
-      if (g >= 1 && !mbar_wait(smem_u32(&s.g2_done), (g - 1) & 1)) { ok = false; break; }
+      if (g >= 1 && !mbar_wait(smem_u32(&s.xy_free), (g - 1) & 1)) { ok = false; break; }
       tc_fence_after();
       const uint32_t b1 = smem_u32(s.b1[st]), b2 = smem_u32(s.b2[st]);
 #pragma unroll
@@ -507,16 +518,26 @@ __device__ void mma_role(Smem& s, const Params& p, uint32_t tmem) {
       if (zero && !mbar_wait(smem_u32(&s.acc_free), (ua & 1) ^ 1)) { ok = false; break; }
       if (!mbar_wait(smem_u32(&s.p_full), g & 1)) { ok = false; break; }
       tc_fence_after();
+      // hi terms from TMEM first: once they are done the next step's S and
+      // dP may overwrite those columns while the lo terms (shared memory) run
       if (kKV) {
 #pragma unroll
         for (int kk = 0; kk < kBlock / 16; ++kk)
-          mma_ts(tmem + kColA1, tmem + kColX + kk * 8, sdesc_sw128(b2 + kk * 2048, 8192, 1024), idesc2,
+          mma_ts(tmem + kColA1, tmem + kColX + hi_col(kk), sdesc_sw128(b2 + kk * 2048, 8192, 1024), idesc2,
                  (zero && kk == 0) ? 0u : 1u);
 #pragma unroll
         for (int kk = 0; kk < kBlock / 16; ++kk)
-          mma_ts(tmem + kColA2, tmem + kColY + kk * 8, sdesc_sw128(b1 + kk * 2048, 8192, 1024), idesc2,
+          mma_ts(tmem + kColA2, tmem + kColY + hi_col(kk), sdesc_sw128(b1 + kk * 2048, 8192, 1024), idesc2,
                  (zero && kk == 0) ? 0u : 1u);
-        const uint32_t plo = smem_u32(s.plo), dslo = smem_u32(s.dslo);
+      } else {
+#pragma unroll
+        for (int kk = 0; kk < kBlock / 16; ++kk)
+          mma_ts(tmem + kColA1, tmem + kColY + hi_col(kk), sdesc_sw128(b1 + kk * 2048, 8192, 1024), idesc2,
+                 (zero && kk == 0) ? 0u : 1u);
+      }
+      mma_commit(smem_u32(&s.xy_free));
+      const uint32_t plo = smem_u32(s.plo), dslo = smem_u32(s.dslo);
+      if (kKV) {
 #pragma unroll
         for (int kk = 0; kk < kBlock / 16; ++kk)
           mma_ss(tmem + kColA1, sdesc_sw128(plo + kk * 32, 16, 1024), sdesc_sw128(b2 + kk * 2048, 8192, 1024), idesc2,
@@ -528,13 +549,9 @@ __device__ void mma_role(Smem& s, const Params& p, uint32_t tmem) {
       } else {
 #pragma unroll
         for (int kk = 0; kk < kBlock / 16; ++kk)
-          mma_ts(tmem + kColA1, tmem + kColY + kk * 8, sdesc_sw128(b1 + kk * 2048, 8192, 1024), idesc2,
-                 (zero && kk == 0) ? 0u : 1u);
-#pragma unroll
-        for (int kk = 0; kk < kBlock / 16; ++kk)
-          mma_ts(tmem + kColA1, tmem + kColX + 32 + kk * 8, sdesc_sw128(b1 + kk * 2048, 8192, 1024), idesc2, 1u);
+          mma_ss(tmem + kColA1, sdesc_sw128(dslo + kk * 32, 16, 1024), sdesc_sw128(b1 + kk * 2048, 8192, 1024), idesc2,
+                 1u);
       }
-      mma_commit(smem_u32(&s.g2_done));
       mma_commit(smem_u32(&s.b_empty[st]));
       if (last && e == n - 1) mma_commit(smem_u32(&s.acc_full));
     }
@@ -547,63 +564,74 @@ __device__ void mma_role(Smem& s, const Params& p, uint32_t tmem) {
 
 // ------------------------------------------------------------ elementwise
 
-// 16 columns of one row: P = exp2((x + bias) scale_log2 - lse2) and
-// dS = P (y - D), each as two bf16 terms, hi = bf16(x) and lo = bf16(x - hi),
-// packed in pairs: the products then see about 16 significant bits of P and
-// dS. (One bf16 rounding leaves about 2^-9 relative error in each term, and
-// dq, dk and dv are sums of terms of either sign, so that error would reach
-// the gradients nearly undiminished.)
+// 16 columns of one row: P = exp2(x scale_log2 + c) with c = bias scale_log2
+// - lse log2(e) (bias -10000 sqrt(d) for a padded key), and dS = P (y - D),
+// each as two bf16 terms, hi = bf16(v) and lo = bf16(v - hi), packed in
+// pairs: the products then see about 16 significant bits of P and dS. (One
+// bf16 rounding leaves about 2^-9 relative error in each term, and dq, dk and
+// dv are sums of terms of either sign, so that error would reach the
+// gradients nearly undiminished.) Pairs of columns in packed f32x2 arithmetic.
 template <bool kKV>
 __device__ __forceinline__ void piece_pds(const uint32_t (&x)[16], const uint32_t (&y)[16], int c0, uint64_t vm,
-                                          float row_bias, float row_lse2, float row_d, const float* col_lse,
-                                          const float* col_d, const Params& p, uint32_t (&pk)[8],
+                                          float row_c, float row_cmask, float row_d, const float* col_lse,
+                                          const float* col_d, float row_bias_l2, float scale_log2, uint32_t (&pk)[8],
                                           uint32_t (&pl)[8], uint32_t (&dk)[8], uint32_t (&dl)[8]) {
   constexpr float kLog2e = 1.4426950408889634f;
+  const uint64_t sc2 = f2_pack(scale_log2, scale_log2);
 #pragma unroll
   for (int c = 0; c < 16; c += 2) {
-    float pv[2], dv[2];
-#pragma unroll
-    for (int t = 0; t < 2; ++t) {
-      const int col = c0 + c + t;
-      float bias, lse2, dd;
-      if (kKV) {
-        bias = row_bias;
-        lse2 = col_lse[col] * kLog2e;
-        dd = col_d[col];
-      } else {
-        bias = ((vm >> col) & 1ull) ? 0.f : p.bias_raw;
-        lse2 = row_lse2;
-        dd = row_d;
-      }
-      const float pr = ex2_approx(fmaf(__uint_as_float(x[c + t]) + bias, p.scale_log2, -lse2));
-      pv[t] = pr;
-      dv[t] = pr * (__uint_as_float(y[c + t]) - dd);
+    const int col = c0 + c;
+    uint64_t cc, dd;
+    if (kKV) {
+      // per query column: c = row bias - lse log2(e), D
+      const float2 l = *reinterpret_cast<const float2*>(col_lse + col);
+      const float2 d = *reinterpret_cast<const float2*>(col_d + col);
+      cc = f2_fma(f2_pack(l.x, l.y), f2_pack(-kLog2e, -kLog2e), f2_pack(row_bias_l2, row_bias_l2));
+      dd = f2_pack(-d.x, -d.y);
+    } else {
+      // per key column: the row's c, or with the masked-key bias
+      cc = f2_pack(((vm >> col) & 1ull) ? row_c : row_cmask, ((vm >> (col + 1)) & 1ull) ? row_c : row_cmask);
+      dd = f2_pack(-row_d, -row_d);
     }
-    const uint32_t phi = pack_bf16x2(pv[0], pv[1]);
+    float t0, t1;
+    f2_unpack(f2_fma(f2_pack(__uint_as_float(x[c]), __uint_as_float(x[c + 1])), sc2, cc), t0, t1);
+    const float p0 = ex2_approx(t0), p1 = ex2_approx(t1);
+    const uint64_t pp = f2_pack(p0, p1);
+    float d0, d1;
+    f2_unpack(f2_mul(pp, f2_add(f2_pack(__uint_as_float(y[c]), __uint_as_float(y[c + 1])), dd)), d0, d1);
+    const uint32_t phi = pack_bf16x2(p0, p1);
     pk[c / 2] = phi;
-    pl[c / 2] = pack_bf16x2(pv[0] - __uint_as_float(phi << 16), pv[1] - __uint_as_float(phi & 0xFFFF0000u));
-    const uint32_t hi = pack_bf16x2(dv[0], dv[1]);
+    float r0, r1;
+    f2_unpack(f2_add(pp, f2_pack(-__uint_as_float(phi << 16), -__uint_as_float(phi & 0xFFFF0000u))), r0, r1);
+    pl[c / 2] = pack_bf16x2(r0, r1);
+    const uint32_t hi = pack_bf16x2(d0, d1);
     dk[c / 2] = hi;
-    dl[c / 2] = pack_bf16x2(dv[0] - __uint_as_float(hi << 16), dv[1] - __uint_as_float(hi & 0xFFFF0000u));
+    f2_unpack(f2_add(f2_pack(d0, d1), f2_pack(-__uint_as_float(hi << 16), -__uint_as_float(hi & 0xFFFF0000u))), r0, r1);
+    dl[c / 2] = pack_bf16x2(r0, r1);
   }
 }
 
-// Warps 0-3, one stationary row per thread (TMEM lane). Per step: read S and
-// dP (64 columns each) and write P and dS_hi as bf16 over their first 32
-// columns and dS_lo over the last 32 of S (once all of S is read); a half
-// whose rows do not use the tile writes zeros. After a unit's
-// last step: the epilogue (dq = acc1 / sqrt(d); dv = acc1, dk = acc2 /
-// sqrt(d)), raw into the partial-sum slot for a split global unit.
+// Warps 0-7: warps w and w + 4 share the 32 stationary rows of TMEM lanes
+// 32 (w & 3) .. +31 (one row per thread) and take columns 0..31 and 32..63
+// of them. Per step: read S and dP, write P_hi (dk/dv kernel) and dS_hi as
+// bf16 into TMEM (hi_col) and P_lo, dS_lo into shared memory; a half whose
+// rows do not use the tile writes zeros. After a unit's last step: the
+// epilogue, each warp its 32 of the 64 columns (dq = acc1 / sqrt(d); dv =
+// acc1, dk = acc2 / sqrt(d); raw into the partial-sum slot of a split global
+// unit).
 template <bool kKV>
 __device__ void elem_role(Smem& s, const Params& p, uint32_t tmem) {
   constexpr float kLog2e = 1.4426950408889634f;
-  const int tid = threadIdx.x;
-  const int warp = tid >> 5;
-  const int lane = tid & 31;
-  const int half = warp >> 1;
-  const uint32_t lane_addr = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int quad = warp & 3;
+  const int chalf = warp >> 2;          // columns 32 chalf .. 32 chalf + 31
+  const int rowi = quad * 32 + lane;    // stationary row 0..127 (TMEM lane)
+  const int half = quad >> 1;           // rows 0..63 or 64..127
+  const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quad * 32) << 16);
+  const float row_bias_l2_masked = p.bias_raw * p.scale_log2;
   uint32_t g = 0, ua = 0;
-  float row_lse2 = 0.f, row_d = 0.f, row_bias = 0.f;
+  float row_c = 0.f, row_cmask = 0.f, row_d = 0.f, row_bias_l2 = 0.f;
   for (uint32_t ut = 0;; ++ut) {
     if (!warp_wait(smem_u32(&s.info_full[ut & 3]), (ut >> 2) & 1)) { if (lane == 0) flag_timeout(p); return; }
     const Unit& ui = s.unit[ut & 3];
@@ -612,83 +640,64 @@ __device__ void elem_role(Smem& s, const Params& p, uint32_t tmem) {
     const int stile = half ? ui.bot : ui.top;
     const bool exists = stile >= 0;
     const int bh = ui.bh;
-    const size_t row = static_cast<size_t>(bh) * p.L + static_cast<size_t>(exists ? stile : 0) * kBlock + (tid & 63);
+    const size_t row = static_cast<size_t>(bh) * p.L + static_cast<size_t>(exists ? stile : 0) * kBlock + (rowi & 63);
     if (ui.first && exists) {
       if (kKV) {
         const int b = bh / p.H;
         const bool valid = !p.seq_mask || p.seq_mask[static_cast<size_t>(b) * p.L + (row - static_cast<size_t>(bh) * p.L)] != 0;
-        row_bias = valid ? 0.f : p.bias_raw;
+        row_bias_l2 = valid ? 0.f : row_bias_l2_masked;
       } else {
-        row_lse2 = __ldg(p.lse + row) * kLog2e;
+        const float lse2 = __ldg(p.lse + row) * kLog2e;
+        row_c = -lse2;
+        row_cmask = row_bias_l2_masked - lse2;
         row_d = __ldg(p.dd + row);
       }
     }
+    uint8_t* rp = s.plo + (rowi >> 3) * 1024 + (rowi & 7) * 128;
+    uint8_t* rd = s.dslo + (rowi >> 3) * 1024 + (rowi & 7) * 128;
     for (int e = 0; e < n; ++e, ++g) {
       const bool used = exists && ((ui.hm[e] >> half) & 1);
       if (!warp_wait(smem_u32(&s.x_full), g & 1)) { if (lane == 0) flag_timeout(p); return; }
       tc_fence_after();
       const int st = g % kStages;
       if (kKV && !warp_wait(smem_u32(&s.b_full[st]), (g / kStages) & 1)) { if (lane == 0) flag_timeout(p); return; }
-      if (used && kKV) {
-        // P_hi, dS_hi into TMEM over S^T and dP^T; P_lo, dS_lo into shared
-        // memory (row tid, 16-byte chunk c at chunk c ^ (tid & 7))
-        uint8_t* rp = s.plo + (tid >> 3) * 1024 + (tid & 7) * 128;
-        uint8_t* rd = s.dslo + (tid >> 3) * 1024 + (tid & 7) * 128;
+      if (used) {
+        const uint64_t vm = kKV ? ~0ull : ui.vm[e];
 #pragma unroll 1
-        for (int q = 0; q < 4; ++q) {
+        for (int q = 2 * chalf; q < 2 * chalf + 2; ++q) {
           uint32_t x[16], y[16], pk[8], pl[8], dk[8], dl[8];
           tmem_ld16(lane_addr + kColX + 16 * q, x);
           tmem_ld16(lane_addr + kColY + 16 * q, y);
           tmem_wait_ld();
-          piece_pds<kKV>(x, y, 16 * q, ~0ull, row_bias, row_lse2, row_d, s.col_lse[st], s.col_d[st], p, pk, pl, dk,
-                         dl);
-          tmem_st8(lane_addr + kColX + 8 * q, pk);
-          tmem_st8(lane_addr + kColY + 8 * q, dk);
+          piece_pds<kKV>(x, y, 16 * q, vm, row_c, row_cmask, row_d, s.col_lse[st], s.col_d[st], row_bias_l2,
+                         p.scale_log2, pk, pl, dk, dl);
+          if (kKV) tmem_st8(lane_addr + kColX + hi_col(q), pk);
+          tmem_st8(lane_addr + kColY + hi_col(q), dk);
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
-            const int chunk = (2 * q + h) ^ (tid & 7);
-            *reinterpret_cast<uint4*>(rp + chunk * 16) = make_uint4(pl[4 * h], pl[4 * h + 1], pl[4 * h + 2], pl[4 * h + 3]);
+            const int chunk = (2 * q + h) ^ (rowi & 7);
+            if (kKV)
+              *reinterpret_cast<uint4*>(rp + chunk * 16) = make_uint4(pl[4 * h], pl[4 * h + 1], pl[4 * h + 2], pl[4 * h + 3]);
             *reinterpret_cast<uint4*>(rd + chunk * 16) = make_uint4(dl[4 * h], dl[4 * h + 1], dl[4 * h + 2], dl[4 * h + 3]);
           }
         }
-        fence_proxy_async_smem();
-      } else if (used) {
-        const uint64_t vm = ui.vm[e];
-        uint32_t lo[4][8];  // dS_lo, written once every S column has been read
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          uint32_t x[16], y[16], pk[8], pl[8], dk[8];
-          tmem_ld16(lane_addr + kColX + 16 * q, x);
-          tmem_ld16(lane_addr + kColY + 16 * q, y);
-          tmem_wait_ld();
-          piece_pds<kKV>(x, y, 16 * q, vm, row_bias, row_lse2, row_d, s.col_lse[st], s.col_d[st], p, pk, pl, dk,
-                         lo[q]);
-          tmem_st8(lane_addr + kColX + 8 * q, pk);
-          tmem_st8(lane_addr + kColY + 8 * q, dk);
-        }
-#pragma unroll
-        for (int q = 0; q < 4; ++q) tmem_st8(lane_addr + kColX + 32 + 8 * q, lo[q]);
       } else {
-        uint32_t z[16];
+        uint32_t z[8];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) z[i] = 0u;
-        tmem_st16(lane_addr + kColX, z);
-        tmem_st16(lane_addr + kColX + 16, z);
-        tmem_st16(lane_addr + kColX + 32, z);
-        tmem_st16(lane_addr + kColX + 48, z);
-        tmem_st16(lane_addr + kColY, z);
-        tmem_st16(lane_addr + kColY + 16, z);
-        if (kKV) {
-          uint4* rp = reinterpret_cast<uint4*>(s.plo + (tid >> 3) * 1024 + (tid & 7) * 128);
-          uint4* rd = reinterpret_cast<uint4*>(s.dslo + (tid >> 3) * 1024 + (tid & 7) * 128);
+        for (int i = 0; i < 8; ++i) z[i] = 0u;
 #pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            rp[c] = make_uint4(0u, 0u, 0u, 0u);
-            rd[c] = make_uint4(0u, 0u, 0u, 0u);
+        for (int q = 2 * chalf; q < 2 * chalf + 2; ++q) {
+          if (kKV) tmem_st8(lane_addr + kColX + hi_col(q), z);
+          tmem_st8(lane_addr + kColY + hi_col(q), z);
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int chunk = (2 * q + h) ^ (rowi & 7);
+            if (kKV) *reinterpret_cast<uint4*>(rp + chunk * 16) = make_uint4(0u, 0u, 0u, 0u);
+            *reinterpret_cast<uint4*>(rd + chunk * 16) = make_uint4(0u, 0u, 0u, 0u);
           }
-          fence_proxy_async_smem();
         }
       }
+      fence_proxy_async_smem();
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
@@ -699,18 +708,18 @@ __device__ void elem_role(Smem& s, const Params& p, uint32_t tmem) {
     __syncwarp();
     if (lane == 0) mbar_arrive(smem_u32(&s.info_empty[ut & 3]));
     if (!last) continue;
-    // ---- epilogue
+    // ---- epilogue: this warp's 32 columns of each accumulator
     if (!warp_wait(smem_u32(&s.acc_full), ua & 1)) { if (lane == 0) flag_timeout(p); return; }
     tc_fence_after();
     if (exists) {
-      const size_t prow = (static_cast<size_t>(bh) * p.nsplit + (split >= 0 ? split : 0)) * kRows + tid;
+      const size_t prow = (static_cast<size_t>(bh) * p.nsplit + (split >= 0 ? split : 0)) * kRows + rowi;
 #pragma unroll 1
       for (int a = 0; a < (kKV ? 2 : 1); ++a) {
         // acc1: dq (dq kernel) or dv; acc2: dk
         const float f = (split >= 0 || (kKV && a == 0)) ? 1.f : p.scale;
         float* dst = split >= 0 ? (a == 0 ? p.part1 : p.part2) + prow * kDim : (a == 0 ? p.g1 : p.g2) + row * kDim;
 #pragma unroll 1
-        for (int c0 = 0; c0 < kDim; c0 += 16) {
+        for (int c0 = 32 * chalf; c0 < 32 * chalf + 32; c0 += 16) {
           uint32_t o[16];
           tmem_ld16(lane_addr + (a == 0 ? kColA1 : kColA2) + c0, o);
           tmem_wait_ld();
@@ -741,14 +750,14 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUt
   Smem& s = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  if (warp == 5) {
+  if (warp == 9) {
     tmem_alloc(smem_u32(&s.tmem_base), kTmemCols);
     tmem_relinquish();
   }
   if (threadIdx.x == 0) {
     for (int i = 0; i < 4; ++i) {
       mbar_init(smem_u32(&s.info_full[i]), 1);
-      mbar_init(smem_u32(&s.info_empty[i]), 1 + 1 + 4);  // TMA, MMA, 4 elementwise warps
+      mbar_init(smem_u32(&s.info_empty[i]), 1 + 1 + kElemWarps);  // TMA, MMA, elementwise warps
     }
     mbar_init(smem_u32(&s.a_full), 1);
     mbar_init(smem_u32(&s.a_free), 1);
@@ -757,13 +766,13 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUt
       mbar_init(smem_u32(&s.b_empty[i]), 1);
     }
     mbar_init(smem_u32(&s.x_full), 1);
-    mbar_init(smem_u32(&s.p_full), 4);
-    mbar_init(smem_u32(&s.g2_done), 1);
+    mbar_init(smem_u32(&s.p_full), kElemWarps);
+    mbar_init(smem_u32(&s.xy_free), 1);
     mbar_init(smem_u32(&s.acc_full), 1);
-    mbar_init(smem_u32(&s.acc_free), 4);
+    mbar_init(smem_u32(&s.acc_free), kElemWarps);
     fence_barrier_init();
   }
-  if (warp == 4 && lane == 0) {
+  if (warp == 8 && lane == 0) {
     tma_prefetch_desc(&tmA1);
     tma_prefetch_desc(&tmA2);
     tma_prefetch_desc(&tmB1);
@@ -773,19 +782,19 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUt
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = s.tmem_base;
-  if (warp < 4) {
+  if (warp < kElemWarps) {
     elem_role<kKV>(s, p, tmem);
-  } else if (warp == 4) {
+  } else if (warp == 8) {
     producer_role<kKV>(s, p, &tmA1, &tmA2, &tmB1, &tmB2);
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     if (lane == 0) mma_role<kKV>(s, p, tmem);
-  } else if (warp == 6) {
+  } else if (warp == 10) {
     prep_role<kKV>(s, p);
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 5) {
+  if (warp == 9) {
     __syncwarp();
     tmem_dealloc(tmem, kTmemCols);
   }
