@@ -64,8 +64,8 @@ constexpr int kCtasPerSm = 2;
 constexpr int kSmemRequest = 112 * 1024;
 constexpr uint32_t kTileBytes = kBlock * kDim * 2;  // 8 KB
 constexpr uint32_t kTmemCols = 256;
-constexpr uint32_t kColX = 0;     // S (or S^T): 64 fp32 columns; P_hi (bf16) overwrites the first 32
-constexpr uint32_t kColY = 64;    // dP (or dP^T): 64 fp32 columns; dS_hi (bf16) overwrites the first 32
+constexpr uint32_t kColX = 0;     // S (or S^T): 64 fp32 columns; then P_hi and P_lo (bf16 pairs)
+constexpr uint32_t kColY = 64;    // dP (or dP^T): 64 fp32 columns; then dS_hi and dS_lo
 constexpr uint32_t kColA1 = 128;  // dQ, or dV
 constexpr uint32_t kColA2 = 192;  // dK
 
@@ -122,8 +122,6 @@ struct __align__(1024) Smem {
   uint8_t a2[kRows * kDim * 2];           // dO (dq) or V (dk/dv)
   uint8_t b1[kStages][kTileBytes];        // K (dq) or Q (dk/dv) of a step
   uint8_t b2[kStages][kTileBytes];        // V (dq) or dO (dk/dv)
-  uint8_t plo[kRows * kBlock * 2];        // P_lo (dk/dv) and dS_lo of the step, [128 rows x 64] bf16, laid
-  uint8_t dslo[kRows * kBlock * 2];       //   out as a TMA box with 128-byte swizzle (an SS-MMA operand)
   float col_lse[kStages][kBlock];         // dk/dv: lse and D of the step's query tile
   float col_d[kStages][kBlock];
   Unit unit[4];
@@ -133,7 +131,7 @@ struct __align__(1024) Smem {
   uint64_t b_full[kStages], b_empty[kStages];
   uint64_t x_full;     // S and dP of the step are in TMEM
   uint64_t p_full;     // P and dS written (4 warps)
-  uint64_t xy_free;    // the step's MMAs reading P_hi and dS_hi from TMEM are complete (S/dP columns reusable)
+  uint64_t xy_free;    // the step's gradient MMAs are complete (S/dP columns reusable)
   uint64_t acc_full;   // a unit's accumulators are complete
   uint64_t acc_free;   // ... and read by the epilogue (4 warps)
   uint32_t tmem_base;
@@ -400,11 +398,11 @@ __device__ void prep_role(Smem& s, const Params& p) {
   }
 }
 
-// Columns 16q .. 16q+15 of the S / dP tiles: the hi terms of piece q go to
-// TMEM columns hi_col(q) .. +7 (packed pairs), which the warp that owns the
-// piece has already read: pieces 0, 1 (one warp) to 0..15, pieces 2, 3 (the
-// other warp of the same rows) to 32..47.
-__device__ __forceinline__ uint32_t hi_col(int q) { return 8 * q + 16 * (q >> 1); }
+// Columns 16q .. 16q+15 of the S / dP tiles (piece q, read by one warp) are
+// replaced by that piece's hi terms (columns 16q .. 16q+7, packed pairs) and
+// lo terms (16q+8 .. 16q+15).
+__device__ __forceinline__ uint32_t hi_col(int q) { return 16 * q; }
+__device__ __forceinline__ uint32_t lo_col(int q) { return 16 * q + 8; }
 
 // ------------------------------------------------------------ TMA
 
@@ -473,13 +471,10 @@ __device__ void producer_role(Smem& s, const Params& p, const CUtensorMap* tmA1,
 // ------------------------------------------------------------ MMA
 
 // One thread. Per step: X = A1 B1^T, Y = A2 B2^T (SS, M = 128, N = 64,
-// K = 64), once the previous step's hi-term MMAs have read P_hi and dS_hi
-// out of those columns; then, once P and dS are written, the gradient MMAs
-// (the moving tile as B with d contiguous, K = 64 moving rows; P and dS in
-// two terms, hi from TMEM (TS), lo from shared memory (SS)). The next step's
-// X and Y are issued behind the lo terms, which write other accumulators.
-// (MMAs of one thread complete in order, so x_full of the next step also
-// means the lo terms have read shared memory.)
+// K = 64), once the previous step's gradient MMAs have read P and dS out of
+// those columns; then, once P and dS are written, the gradient MMAs (TS, A =
+// the hi and lo terms from TMEM, B = the moving tile with d contiguous, K =
+// 64 moving rows):
 //   dq kernel:   acc1 += (dS_hi + dS_lo) B1                          (dQ += dS K)
 //   dk/dv kernel: acc1 += (P_hi + P_lo) B2, acc2 += (dS_hi + dS_lo) B1 (dV += P^T dO, dK += dS^T Q)
 template <bool kKV>
@@ -518,40 +513,28 @@ __device__ void mma_role(Smem& s, const Params& p, uint32_t tmem) {
       if (zero && !mbar_wait(smem_u32(&s.acc_free), (ua & 1) ^ 1)) { ok = false; break; }
       if (!mbar_wait(smem_u32(&s.p_full), g & 1)) { ok = false; break; }
       tc_fence_after();
-      // hi terms from TMEM first: once they are done the next step's S and
-      // dP may overwrite those columns while the lo terms (shared memory) run
       if (kKV) {
 #pragma unroll
-        for (int kk = 0; kk < kBlock / 16; ++kk)
+        for (int kk = 0; kk < kBlock / 16; ++kk) {
           mma_ts(tmem + kColA1, tmem + kColX + hi_col(kk), sdesc_sw128(b2 + kk * 2048, 8192, 1024), idesc2,
                  (zero && kk == 0) ? 0u : 1u);
+          mma_ts(tmem + kColA1, tmem + kColX + lo_col(kk), sdesc_sw128(b2 + kk * 2048, 8192, 1024), idesc2, 1u);
+        }
 #pragma unroll
-        for (int kk = 0; kk < kBlock / 16; ++kk)
+        for (int kk = 0; kk < kBlock / 16; ++kk) {
           mma_ts(tmem + kColA2, tmem + kColY + hi_col(kk), sdesc_sw128(b1 + kk * 2048, 8192, 1024), idesc2,
                  (zero && kk == 0) ? 0u : 1u);
+          mma_ts(tmem + kColA2, tmem + kColY + lo_col(kk), sdesc_sw128(b1 + kk * 2048, 8192, 1024), idesc2, 1u);
+        }
       } else {
 #pragma unroll
-        for (int kk = 0; kk < kBlock / 16; ++kk)
+        for (int kk = 0; kk < kBlock / 16; ++kk) {
           mma_ts(tmem + kColA1, tmem + kColY + hi_col(kk), sdesc_sw128(b1 + kk * 2048, 8192, 1024), idesc2,
                  (zero && kk == 0) ? 0u : 1u);
+          mma_ts(tmem + kColA1, tmem + kColY + lo_col(kk), sdesc_sw128(b1 + kk * 2048, 8192, 1024), idesc2, 1u);
+        }
       }
       mma_commit(smem_u32(&s.xy_free));
-      const uint32_t plo = smem_u32(s.plo), dslo = smem_u32(s.dslo);
-      if (kKV) {
-#pragma unroll
-        for (int kk = 0; kk < kBlock / 16; ++kk)
-          mma_ss(tmem + kColA1, sdesc_sw128(plo + kk * 32, 16, 1024), sdesc_sw128(b2 + kk * 2048, 8192, 1024), idesc2,
-                 1u);
-#pragma unroll
-        for (int kk = 0; kk < kBlock / 16; ++kk)
-          mma_ss(tmem + kColA2, sdesc_sw128(dslo + kk * 32, 16, 1024), sdesc_sw128(b1 + kk * 2048, 8192, 1024), idesc2,
-                 1u);
-      } else {
-#pragma unroll
-        for (int kk = 0; kk < kBlock / 16; ++kk)
-          mma_ss(tmem + kColA1, sdesc_sw128(dslo + kk * 32, 16, 1024), sdesc_sw128(b1 + kk * 2048, 8192, 1024), idesc2,
-                 1u);
-      }
       mma_commit(smem_u32(&s.b_empty[st]));
       if (last && e == n - 1) mma_commit(smem_u32(&s.acc_full));
     }
@@ -613,9 +596,9 @@ __device__ __forceinline__ void piece_pds(const uint32_t (&x)[16], const uint32_
 
 // Warps 0-7: warps w and w + 4 share the 32 stationary rows of TMEM lanes
 // 32 (w & 3) .. +31 (one row per thread) and take columns 0..31 and 32..63
-// of them. Per step: read S and dP, write P_hi (dk/dv kernel) and dS_hi as
-// bf16 into TMEM (hi_col) and P_lo, dS_lo into shared memory; a half whose
-// rows do not use the tile writes zeros. After a unit's last step: the
+// of them. Per step: read S and dP and write P (dk/dv kernel) and dS over
+// them as bf16 hi and lo terms; a half whose rows do not use the tile writes
+// zeros. After a unit's last step: the
 // epilogue, each warp its 32 of the 64 columns (dq = acc1 / sqrt(d); dv =
 // acc1, dk = acc2 / sqrt(d); raw into the partial-sum slot of a split global
 // unit).
@@ -653,8 +636,6 @@ __device__ void elem_role(Smem& s, const Params& p, uint32_t tmem) {
         row_d = __ldg(p.dd + row);
       }
     }
-    uint8_t* rp = s.plo + (rowi >> 3) * 1024 + (rowi & 7) * 128;
-    uint8_t* rd = s.dslo + (rowi >> 3) * 1024 + (rowi & 7) * 128;
     for (int e = 0; e < n; ++e, ++g) {
       const bool used = exists && ((ui.hm[e] >> half) & 1);
       if (!warp_wait(smem_u32(&s.x_full), g & 1)) { if (lane == 0) flag_timeout(p); return; }
@@ -671,33 +652,23 @@ __device__ void elem_role(Smem& s, const Params& p, uint32_t tmem) {
           tmem_wait_ld();
           piece_pds<kKV>(x, y, 16 * q, vm, row_c, row_cmask, row_d, s.col_lse[st], s.col_d[st], row_bias_l2,
                          p.scale_log2, pk, pl, dk, dl);
-          if (kKV) tmem_st8(lane_addr + kColX + hi_col(q), pk);
-          tmem_st8(lane_addr + kColY + hi_col(q), dk);
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const int chunk = (2 * q + h) ^ (rowi & 7);
-            if (kKV)
-              *reinterpret_cast<uint4*>(rp + chunk * 16) = make_uint4(pl[4 * h], pl[4 * h + 1], pl[4 * h + 2], pl[4 * h + 3]);
-            *reinterpret_cast<uint4*>(rd + chunk * 16) = make_uint4(dl[4 * h], dl[4 * h + 1], dl[4 * h + 2], dl[4 * h + 3]);
+          if (kKV) {
+            tmem_st8(lane_addr + kColX + hi_col(q), pk);
+            tmem_st8(lane_addr + kColX + lo_col(q), pl);
           }
+          tmem_st8(lane_addr + kColY + hi_col(q), dk);
+          tmem_st8(lane_addr + kColY + lo_col(q), dl);
         }
       } else {
-        uint32_t z[8];
+        uint32_t z[16];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) z[i] = 0u;
+        for (int i = 0; i < 16; ++i) z[i] = 0u;
 #pragma unroll
         for (int q = 2 * chalf; q < 2 * chalf + 2; ++q) {
-          if (kKV) tmem_st8(lane_addr + kColX + hi_col(q), z);
-          tmem_st8(lane_addr + kColY + hi_col(q), z);
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const int chunk = (2 * q + h) ^ (rowi & 7);
-            if (kKV) *reinterpret_cast<uint4*>(rp + chunk * 16) = make_uint4(0u, 0u, 0u, 0u);
-            *reinterpret_cast<uint4*>(rd + chunk * 16) = make_uint4(0u, 0u, 0u, 0u);
-          }
+          if (kKV) tmem_st16(lane_addr + kColX + 16 * q, z);
+          tmem_st16(lane_addr + kColY + 16 * q, z);
         }
       }
-      fence_proxy_async_smem();
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
