@@ -36,7 +36,10 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one forward
 # kernel launch per workload, from an ncu capture of the current kernel
 # source; an entry is removed whenever the kernel changes.
-FWD_DRAM_BYTES_PER_LAUNCH: dict = {}
+FWD_DRAM_BYTES_PER_LAUNCH: dict = {
+    # 78.00 MB read + 8.70 MB written, fp16 instance at d = 64, one launch
+    "bigbird_base_l4096": 86.699008e6,
+}
 
 
 def _peaks():
@@ -538,10 +541,11 @@ def run_probs(args):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32 (bf16 inputs)",
         "data": "synthetic", "pass": "probs",
         "config": _config(w, 1), "l2": L2_NOTE,
-        # traffic: null -- the kernel changed (warp-parallel unit planning)
-        # after its last ncu capture.
+        # traffic: one fp32 export launch at the BigBird-base workload, ncu
+        # (59.05 MB read + 431.25 MB written)
         "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s", "frac": gbs / peak,
-                     "traffic": None, "kernel": "bigbird_probs_kernel",
+                     "traffic": 490.295296e6 if w.name == "bigbird_base_l4096" else None,
+                     "kernel": "bigbird_probs_kernel",
                      "algorithmic_bytes": out_bytes + in_bytes,
                      "peak_source": f"{src} HBM copy bandwidth"},
         "pairs_per_s": pairs / (ms * 1e-3),
