@@ -455,10 +455,11 @@ def run_bwd(args):
         "data": "synthetic", "pass": "bwd",
         "config": _config(w, 1), "l2": L2_NOTE,
         "roofline": {"bound": "tensor", "achieved": value, "peak": peak, "unit": "TFLOP/s", "frac": value / peak,
-                     "traffic": None,
+                     # DRAM bytes of one dk/dv launch (the larger kernel), ncu: 148.96 MB read + 78.63 MB written
+                     "traffic": 227.583744e6 if w.name == "bigbird_base_l4096" else None,
                      "kernel": "bwd_kernel<dq> + bwd_kernel<dk,dv> (tcgen05, bf16 operands); the duration is the "
                                "whole call (row dot and partial sums included), the work the algorithmic 5 GEMM-"
-                               "shaped products",
+                               "shaped products; traffic is the dk/dv kernel's",
                      "peak_source": f"{src} bf16 dense burst"},
         "gpu_launches": steps * launches, "clocks": clocks,
     }
