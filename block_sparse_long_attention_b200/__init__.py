@@ -58,6 +58,8 @@ def _load():
         "bigbird_attn_bwd": (I, [P, P, P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, U, P]),
         "bigbird_attn_bwd_ex": (I, [P, P, P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, U, P, Z, P]),
         "bigbird_attn_bwd_workspace_size": (Z, [I, I, I, I, I, I, U]),
+        "bigbird_attn_fwd_host": (I, [P, P, P, P, P, P, I, I, I, I, I, I, I, U, P, Z, P]),
+        "bigbird_attn_fwd_host_scratch_bytes": (Z, [I, I, I, I, I, I, U]),
         "bigbird_wait_probe": (I, [U, P]),
         "bigbird_attn_probs_layout": (I, [I, I, I, I, U, ctypes.POINTER(I), ctypes.POINTER(I), ctypes.POINTER(I)]),
         "bigbird_attn_probs": (I, [P, P, P, P, P, P, P, I, I, I, I, I, I, I, U, P]),
@@ -197,6 +199,49 @@ def fwd_train(q, k, v, rand_attn, seq_mask=None, *, block: int = 64, r: int = 3,
                                      workspace.data_ptr(), ws_bytes, _stream_handle(stream))
     _check(st, "bigbird_attn_fwd_train")
     return out, lse
+
+
+def fwd_host_scratch_bytes(B: int, H: int, L: int, d: int = 64, block: int = 64, r: int = 3,
+                           force_sparse: bool = False) -> int:
+    flags = BB_FLAG_FORCE_SPARSE if force_sparse else 0
+    return int(_load().bigbird_attn_fwd_host_scratch_bytes(B, H, L, d, block, r, flags))
+
+
+def fwd_host(q, k, v, rand_attn, seq_mask, out, *, block: int = 64, r: int = 3, scratch=None,
+             force_sparse: bool = False, stream=None):
+    """bigbird_attn_fwd_host: q, k, v (bf16 [B, H, L, d]), rand_attn (int32
+    [H, nb-2, r] or None), seq_mask (uint8 [B, L] or None) and out (bf16 or
+    fp32, q's shape) are CPU tensors, page-locked for the copies to overlap
+    compute; scratch a uint8 CUDA tensor of fwd_host_scratch_bytes(...) bytes.
+    Runs on the current torch stream (or `stream`); synchronise it before
+    reading out."""
+    import torch
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if t.is_cuda or t.dtype != torch.bfloat16 or not t.is_contiguous() or t.dim() != 4:
+            raise ValueError(f"{name} must be a contiguous bf16 CPU tensor [B, H, L, d]")
+    if k.shape != q.shape or v.shape != q.shape or out.shape != q.shape or out.is_cuda or not out.is_contiguous():
+        raise ValueError("k, v and out must be contiguous CPU tensors of q's shape")
+    if out.dtype not in (torch.bfloat16, torch.float32):
+        raise ValueError("out must be bf16 or fp32")
+    B, H, L, d = q.shape
+    flags = BB_FLAG_FORCE_SPARSE if force_sparse else 0
+    need = fwd_host_scratch_bytes(B, H, L, d, block, r, force_sparse)
+    if scratch is None or not scratch.is_cuda or scratch.numel() * scratch.element_size() < need:
+        raise ValueError(f"scratch must be a CUDA tensor of at least {need} bytes")
+    ra = None
+    if rand_attn is not None:
+        ra = torch.as_tensor(rand_attn, dtype=torch.int32).contiguous()
+        if ra.is_cuda:
+            raise ValueError("rand_attn must be on the host")
+    if seq_mask is not None and (seq_mask.is_cuda or seq_mask.dtype != torch.uint8 or not seq_mask.is_contiguous()):
+        raise ValueError("seq_mask must be a contiguous uint8 CPU tensor [B, L]")
+    st = _load().bigbird_attn_fwd_host(q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                       None if ra is None else ra.data_ptr(),
+                                       None if seq_mask is None else seq_mask.data_ptr(), out.data_ptr(),
+                                       B, H, L, d, block, r, BB_OUT_F32 if out.dtype == torch.float32 else BB_OUT_BF16,
+                                       flags, scratch.data_ptr(), need, _stream_handle(stream))
+    _check(st, "bigbird_attn_fwd_host")
+    return out
 
 
 def bwd_workspace_size(B: int, H: int, L: int, d: int = 64, block: int = 64, r: int = 3,

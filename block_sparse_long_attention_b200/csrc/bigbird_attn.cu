@@ -1388,3 +1388,153 @@ extern "C" int bigbird_attn_fwd_noalloc(const void* q, const void* k, const void
 }
 
 extern "C" size_t bigbird_attn_noalloc_scratch_bytes(void) { return bb::kStaticScratchBytes; }
+
+// ------------------------------------------------------------ host buffers
+
+// bigbird_attn_fwd_host: inputs and output in host memory. The batch is
+// processed one sequence at a time through two device slots, on three
+// streams of the library's own (host-to-device copies, the forward, device-to-
+// host copies), so that copying sequence b+1 in, computing b and copying b-1
+// out overlap; the caller's stream waits for the whole call at the end.
+
+namespace bb {
+
+struct HostPipe {
+  std::mutex mu;  // one call at a time enqueues on the device's streams and events
+  cudaStream_t h2d = nullptr, comp = nullptr, d2h = nullptr;
+  cudaEvent_t start = nullptr, in_done[2] = {}, comp_done[2] = {}, out_done[2] = {}, finish = nullptr;
+  bool ok = false;
+};
+
+static HostPipe* host_pipe(int dev) {
+  static HostPipe pipes[64];
+  static std::once_flag once[64];
+  if (dev < 0 || dev >= 64) return nullptr;
+  std::call_once(once[dev], [dev] {
+    HostPipe& hp = pipes[dev];
+    bool ok = cudaStreamCreateWithFlags(&hp.h2d, cudaStreamNonBlocking) == cudaSuccess &&
+              cudaStreamCreateWithFlags(&hp.comp, cudaStreamNonBlocking) == cudaSuccess &&
+              cudaStreamCreateWithFlags(&hp.d2h, cudaStreamNonBlocking) == cudaSuccess &&
+              cudaEventCreateWithFlags(&hp.start, cudaEventDisableTiming) == cudaSuccess &&
+              cudaEventCreateWithFlags(&hp.finish, cudaEventDisableTiming) == cudaSuccess;
+    for (int i = 0; i < 2 && ok; ++i)
+      ok = cudaEventCreateWithFlags(&hp.in_done[i], cudaEventDisableTiming) == cudaSuccess &&
+           cudaEventCreateWithFlags(&hp.comp_done[i], cudaEventDisableTiming) == cudaSuccess &&
+           cudaEventCreateWithFlags(&hp.out_done[i], cudaEventDisableTiming) == cudaSuccess;
+    hp.ok = ok;
+  });
+  return pipes[dev].ok ? &pipes[dev] : nullptr;
+}
+
+struct HostLayout {
+  size_t ra = 0, slot = 0, q = 0, k = 0, v = 0, out = 0, mask = 0, ws = 0, ws_bytes = 0, total = 0;
+};
+
+static size_t r256(size_t x) { return (x + 255) / 256 * 256; }
+
+// Scratch layout: rand_attn, then two slots of one sequence's q, k, v, out
+// (fp32-sized), seq_mask and forward workspace. 0 if the sizes are invalid.
+static bool host_layout(int B, int H, int L, int d, int block, int r, unsigned flags, HostLayout& hl) {
+  if (B <= 0 || H <= 0 || L <= 0 || d <= 0 || block <= 0 || r < 1 || L % block != 0) return false;
+  const size_t rows = static_cast<size_t>(H) * L;
+  const int nb = L / block;
+  hl.ws_bytes = bigbird_attn_workspace_size(1, H, L, d, block, r, flags);
+  hl.ra = 0;
+  size_t off = r256(static_cast<size_t>(H) * (nb > 2 ? nb - 2 : 1) * r * sizeof(int32_t));
+  hl.q = 0;
+  hl.k = r256(rows * d * 2);
+  hl.v = hl.k + r256(rows * d * 2);
+  hl.out = hl.v + r256(rows * d * 2);
+  hl.mask = hl.out + r256(rows * d * 4);
+  hl.ws = hl.mask + r256(static_cast<size_t>(L));
+  hl.slot = hl.ws + r256(hl.ws_bytes);
+  hl.total = off + 2 * hl.slot;
+  hl.ra = 0;
+  // slot s starts at off + s * slot
+  hl.q += off;
+  hl.k += off;
+  hl.v += off;
+  hl.out += off;
+  hl.mask += off;
+  hl.ws += off;
+  return true;
+}
+
+}  // namespace bb
+
+extern "C" size_t bigbird_attn_fwd_host_scratch_bytes(int B, int H, int L, int d, int block, int r, unsigned flags) {
+  bb::HostLayout hl;
+  return bb::host_layout(B, H, L, d, block, r, flags, hl) ? hl.total : 0;
+}
+
+extern "C" int bigbird_attn_fwd_host(const void* q, const void* k, const void* v, const int32_t* rand_attn,
+                                     const uint8_t* seq_mask, void* out, int B, int H, int L, int d, int block, int r,
+                                     int out_dtype, unsigned flags, void* scratch, size_t scratch_bytes,
+                                     void* stream_) {
+  using namespace bb;
+  HostLayout hl;
+  if (!host_layout(B, H, L, d, block, r, flags, hl)) return BB_ERR_INVALID_ARG;
+  if (!q || !k || !v || !out || !scratch) return BB_ERR_INVALID_ARG;
+  if (out_dtype != BB_OUT_BF16 && out_dtype != BB_OUT_F32) return BB_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(scratch) & 255) != 0 || scratch_bytes < hl.total) return BB_ERR_INVALID_ARG;
+  const int nb = L / block;
+  const bool sparse = (flags & BB_FLAG_FORCE_SPARSE) || nb > 5 + 2 * r;
+  if (sparse && !rand_attn) return BB_ERR_INVALID_ARG;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return BB_ERR_CUDA;
+  HostPipe* hp = host_pipe(dev);
+  if (!hp) return BB_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(hp->mu);
+  cudaStream_t caller = static_cast<cudaStream_t>(stream_);
+  uint8_t* base = static_cast<uint8_t*>(scratch);
+  const size_t seq_in = static_cast<size_t>(H) * L * d * 2;
+  const size_t seq_out = static_cast<size_t>(H) * L * d * (out_dtype == BB_OUT_F32 ? 4 : 2);
+  // everything already queued on the caller's stream (earlier users of the
+  // scratch) comes first
+  if (cudaEventRecord(hp->start, caller) != cudaSuccess) return BB_ERR_CUDA;
+  for (cudaStream_t s : {hp->h2d, hp->comp, hp->d2h})
+    if (cudaStreamWaitEvent(s, hp->start, 0) != cudaSuccess) return BB_ERR_CUDA;
+  int32_t* ra_d = reinterpret_cast<int32_t*>(base + hl.ra);
+  if (sparse && cudaMemcpyAsync(ra_d, rand_attn, static_cast<size_t>(H) * (nb - 2) * r * sizeof(int32_t),
+                                cudaMemcpyHostToDevice, hp->h2d) != cudaSuccess)
+    return BB_ERR_CUDA;
+  // a fresh call's workspace counters start at zero
+  for (int sl = 0; sl < 2; ++sl)
+    if (hl.ws_bytes && cudaMemsetAsync(base + sl * hl.slot + hl.ws, 0, kCounterBytes, hp->h2d) != cudaSuccess)
+      return BB_ERR_CUDA;
+  int st = BB_OK;
+  for (int b = 0; b < B && st == BB_OK; ++b) {
+    const int sl = b & 1;
+    uint8_t* slot = base + sl * hl.slot;
+    // slot sl is free once sequence b-2 has been copied out
+    if (b >= 2 && cudaStreamWaitEvent(hp->h2d, hp->out_done[sl], 0) != cudaSuccess) return BB_ERR_CUDA;
+    const size_t off = static_cast<size_t>(b) * seq_in;
+    if (cudaMemcpyAsync(slot + hl.q, static_cast<const uint8_t*>(q) + off, seq_in, cudaMemcpyHostToDevice, hp->h2d) !=
+            cudaSuccess ||
+        cudaMemcpyAsync(slot + hl.k, static_cast<const uint8_t*>(k) + off, seq_in, cudaMemcpyHostToDevice, hp->h2d) !=
+            cudaSuccess ||
+        cudaMemcpyAsync(slot + hl.v, static_cast<const uint8_t*>(v) + off, seq_in, cudaMemcpyHostToDevice, hp->h2d) !=
+            cudaSuccess)
+      return BB_ERR_CUDA;
+    if (seq_mask && cudaMemcpyAsync(slot + hl.mask, seq_mask + static_cast<size_t>(b) * L, static_cast<size_t>(L),
+                                    cudaMemcpyHostToDevice, hp->h2d) != cudaSuccess)
+      return BB_ERR_CUDA;
+    if (cudaEventRecord(hp->in_done[sl], hp->h2d) != cudaSuccess) return BB_ERR_CUDA;
+    if (cudaStreamWaitEvent(hp->comp, hp->in_done[sl], 0) != cudaSuccess) return BB_ERR_CUDA;
+    st = bigbird_attn_fwd_ex(slot + hl.q, slot + hl.k, slot + hl.v, sparse ? ra_d : nullptr,
+                             seq_mask ? slot + hl.mask : nullptr, slot + hl.out, 1, H, L, d, block, r, out_dtype,
+                             flags & ~static_cast<unsigned>(BB_FLAG_DEBUG_CHECKS),
+                             hl.ws_bytes ? slot + hl.ws : nullptr, hl.ws_bytes, hp->comp);
+    if (st != BB_OK) break;
+    if (cudaEventRecord(hp->comp_done[sl], hp->comp) != cudaSuccess) return BB_ERR_CUDA;
+    if (cudaStreamWaitEvent(hp->d2h, hp->comp_done[sl], 0) != cudaSuccess) return BB_ERR_CUDA;
+    if (cudaMemcpyAsync(static_cast<uint8_t*>(out) + static_cast<size_t>(b) * seq_out, slot + hl.out, seq_out,
+                        cudaMemcpyDeviceToHost, hp->d2h) != cudaSuccess)
+      return BB_ERR_CUDA;
+    if (cudaEventRecord(hp->out_done[sl], hp->d2h) != cudaSuccess) return BB_ERR_CUDA;
+  }
+  // the caller's stream waits for the last copy out (and so for everything)
+  if (cudaEventRecord(hp->finish, hp->d2h) != cudaSuccess) return BB_ERR_CUDA;
+  if (cudaStreamWaitEvent(caller, hp->finish, 0) != cudaSuccess) return BB_ERR_CUDA;
+  return st;
+}

@@ -138,6 +138,31 @@ int bigbird_attn_fwd_ex(const void* q, const void* k, const void* v, const int32
                         int out_dtype, unsigned flags, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * bigbird_attn_fwd_host -- bigbird_attn_fwd_ex with q, k, v, rand_attn,
+ * seq_mask and out in HOST memory (page-locked for the copies to overlap):
+ * layouts as bigbird_attn_fwd_ex, out bf16 or fp32 per out_dtype. The batch
+ * goes through the GPU one sequence at a time in two device slots, on three
+ * streams of the library's own (copies in, the forward, copies out), so that
+ * copying sequence b+1 in, computing b and copying b-1 out overlap; the
+ * results are those of bigbird_attn_fwd_ex on the whole batch, bit for bit.
+ *   scratch  device, 256-byte aligned, at least
+ *            bigbird_attn_fwd_host_scratch_bytes(...) bytes; no initialisation
+ *            needed (the call zeroes the workspace counters it uses).
+ *   stream   the caller's stream: the call starts after the work queued on it
+ *            and the stream waits for the call's last copy; synchronise it
+ *            before reading out.
+ * Calls for one device are enqueued one at a time (a mutex); calls that share
+ * a scratch must not overlap on the GPU. Errors as bigbird_attn_fwd_ex
+ * (BB_FLAG_DEBUG_CHECKS is ignored: rand_attn is on the host already).
+ */
+int bigbird_attn_fwd_host(const void* q, const void* k, const void* v, const int32_t* rand_attn,
+                          const uint8_t* seq_mask, void* out, int B, int H, int L, int d, int block, int r,
+                          int out_dtype, unsigned flags, void* scratch, size_t scratch_bytes, void* stream);
+
+/* Bytes of device scratch bigbird_attn_fwd_host needs (0 if the sizes are invalid). */
+size_t bigbird_attn_fwd_host_scratch_bytes(int B, int H, int L, int d, int block, int r, unsigned flags);
+
+/*
  * bigbird_attn_fwd_train -- bigbird_attn_fwd_ex that also writes, for the
  * backward pass, each row's natural-log log-sum-exp of its scores:
  *   lse[b,h,t] = log sum_k exp(s[t,k]),  s = q.k / sqrt(d) + bias
