@@ -62,6 +62,31 @@ def test_noalloc_matches_allocating_entry_point_twice():
         assert torch.equal(out, ref)
 
 
+@pytest.mark.parametrize("block,d", [(128, 64), (64, 128), (128, 128)], ids=["b128_d64", "b64_d128", "b128_d128"])
+def test_noalloc_other_tensor_core_sizes(block, d):
+    """Blocks of 128 and d = 128 run the tensor-core kernel too: the scratch
+    region holds their workspace (partials of 128 columns at d = 128)."""
+    from block_sparse_long_attention_b200.workloads import Workload
+    w = Workload(f"noalloc_b{block}_d{d}", 2, 3, 24 * block, d=d, block=block, value_scale=1.0,
+                 pad=("fixed", [24 * block - 100, 12 * block]), seed=61)
+    lib = bb.lib()
+    need = bb.workspace_size(w.B, w.H, w.L, d, block)
+    assert 256 < need <= lib.bigbird_attn_noalloc_scratch_bytes()
+    inp = make_inputs(w)
+    q, k, v = (inp[x].cuda() for x in "qkv")
+    sm = inp["seq_mask"].cuda()
+    ra = torch.from_numpy(bb.rand_attn_generate(w.H, w.L, w.block, w.r, seed=w.seed)).cuda()
+    ref = bb.fwd(q, k, v, ra, sm, block=block, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    for _ in range(2):
+        out = torch.full_like(ref, float("nan"))
+        st = _noalloc(lib, q, k, v, ra, sm, out, w, bb.BB_OUT_F32)
+        assert st == bb.BB_OK, bb.status_string(st)
+        torch.cuda.synchronize()
+        assert bb.device_status() == 0
+        assert torch.equal(out, ref)
+
+
 def test_noalloc_rejects_what_does_not_fit():
     lib = bb.lib()
     w = WORKLOADS["tiny_l1024"]
