@@ -12,6 +12,9 @@ namespace bb {
 // swizzle (one box = one block of one head). False if the driver entry point
 // is missing or the encoding is rejected.
 bool make_tile_map(CUtensorMap* map, const void* base, uint64_t rows);
+// The same over a [rows, d] matrix (d = 64 or 128): 64x64 boxes, one per
+// 64-column chunk (x = 64 c).
+bool make_tile_map_d(CUtensorMap* map, const void* base, uint64_t rows, int d);
 
 // Device address of the library's status word on the current device `dev`
 // (bit 1: an out-of-range rand_attn entry was skipped; bit 2: a bounded wait

@@ -1083,6 +1083,7 @@ static DeviceInfo* device_info(int dev) {
 }
 
 bool make_tile_map(CUtensorMap* map, const void* base, uint64_t rows) { return make_map(map, base, rows, 64); }
+bool make_tile_map_d(CUtensorMap* map, const void* base, uint64_t rows, int d) { return make_map(map, base, rows, d); }
 
 uint32_t* status_word(int dev) {
   DeviceInfo* di = device_info(dev);

@@ -49,8 +49,7 @@ namespace bbw {
 
 using namespace bb;
 
-constexpr int kBlock = 64;     // tokens per block (one 64x64 tile)
-constexpr int kDim = 64;       // head dimension
+constexpr int kBlock = 64;     // tokens per tile: a block of 64, or half a block of 128
 constexpr int kRows = 128;     // stationary rows per unit (two tiles)
 constexpr int kStages = 2;     // moving-tile ring depth
 constexpr int kMaxList = 42;   // moving tiles per unit chunk
@@ -58,16 +57,27 @@ constexpr int kMaxR = 16;
 constexpr int kSplit = 8;      // tiles per range of a global unit
 constexpr int kThreads = 384;  // warps 0-7 elementwise, 8 TMA, 9 MMA, 10 prep, 11 idle
 constexpr int kElemWarps = 8;
-constexpr int kCtasPerSm = 2;
-// Dynamic shared memory requested per CTA: more than the kernel uses, so that
-// at most two CTAs share an SM (each allocates half of its TMEM).
-constexpr int kSmemRequest = 112 * 1024;
-constexpr uint32_t kTileBytes = kBlock * kDim * 2;  // 8 KB
-constexpr uint32_t kTmemCols = 256;
+constexpr uint32_t kChunkBytes = kBlock * 64 * 2;  // 64 rows x 64 columns bf16: one TMA box
 constexpr uint32_t kColX = 0;     // S (or S^T): 64 fp32 columns; then P_hi and P_lo (bf16 pairs)
 constexpr uint32_t kColY = 64;    // dP (or dP^T): 64 fp32 columns; then dS_hi and dS_lo
-constexpr uint32_t kColA1 = 128;  // dQ, or dV
-constexpr uint32_t kColA2 = 192;  // dK
+constexpr uint32_t kColA1 = 128;  // dQ, or dV: d fp32 columns; dK follows
+
+// Sizes that follow from the head dimension d (64 or 128): a row of d values
+// is cut into d / 64 chunks (chunk c of a 64-row tile at c * 8 KB, of the
+// unit's 128 stationary rows at c * 16 KB). At d = 64 two CTAs share an SM
+// (256 TMEM columns each; more shared memory is requested than used so that a
+// third never waits for TMEM); at d = 128 the two stationary operands alone
+// take 64 KB, so one CTA per SM (512 TMEM columns for dk/dv: S | dP | dV | dK).
+template <int kD>
+struct BGeo {
+  static constexpr int kChunks = kD / 64;
+  static constexpr uint32_t kTileBytes = kBlock * kD * 2;
+  static constexpr uint32_t kAChunkBytes = kRows * 64 * 2;
+  static constexpr int kCtasPerSm = kD == 64 ? 2 : 1;
+  static constexpr uint32_t kColA2 = kColA1 + kD;
+  __host__ __device__ static constexpr uint32_t tmem_cols(bool kv) { return kD == 64 ? 256u : (kv ? 512u : 256u); }
+};
+constexpr int kSmemRequest64 = 112 * 1024;
 
 constexpr uint32_t kStatusBadRandAttn = 1u;
 constexpr uint32_t kStatusTimeout = 2u;
@@ -100,15 +110,18 @@ struct Params {
   const float* dd;        // D [B*H*L]
   const int32_t* rand_attn;
   const uint8_t* seq_mask;
-  float* g1;              // dq (dq kernel) or dv (dk/dv kernel), [B*H*L, 64]
+  float* g1;              // dq (dq kernel) or dv (dk/dv kernel), [B*H*L, d]
   float* g2;              // dk (dk/dv kernel)
-  float* part1;           // partial sums of split global units [BH, nsplit, 128, 64] (g1)
+  float* part1;           // partial sums of split global units [BH, nparts, 128, d] (g1)
   float* part2;           // ... (g2)
   int* counters;          // this kernel's [tickets, done]
   uint32_t* status;
   int H, L, nb, r, BH;
+  int nt;                 // 64-token tiles per sequence
   int sparse;
   int nsplit;             // ranges per global unit (1: write the gradient directly)
+  int n_glob;             // global units per range: 1 (block 64: both global blocks) or 2 (block 128)
+  int nparts;             // n_glob * nsplit
   int n_mid_per_head;     // middle units per head
   int n_mid_units;
   int total_units;
@@ -117,11 +130,12 @@ struct Params {
   float scale;            // 1 / sqrt(d)
 };
 
+template <int kD>
 struct __align__(1024) Smem {
-  uint8_t a1[kRows * kDim * 2];           // Q (dq) or K (dk/dv) of the unit: two tiles
-  uint8_t a2[kRows * kDim * 2];           // dO (dq) or V (dk/dv)
-  uint8_t b1[kStages][kTileBytes];        // K (dq) or Q (dk/dv) of a step
-  uint8_t b2[kStages][kTileBytes];        // V (dq) or dO (dk/dv)
+  uint8_t a1[kRows * kD * 2];                   // Q (dq) or K (dk/dv) of the unit: two tiles
+  uint8_t a2[kRows * kD * 2];                   // dO (dq) or V (dk/dv)
+  uint8_t b1[kStages][BGeo<kD>::kTileBytes];    // K (dq) or Q (dk/dv) of a step
+  uint8_t b2[kStages][BGeo<kD>::kTileBytes];    // V (dq) or dO (dk/dv)
   float col_lse[kStages][kBlock];         // dk/dv: lse and D of the step's query tile
   float col_d[kStages][kBlock];
   Unit unit[4];
@@ -171,23 +185,25 @@ __device__ __forceinline__ uint64_t key_valid_bits(const uint8_t* seq_mask, int 
 
 // ------------------------------------------------------------ unit building
 
-// Unit u of either kernel when its list fits one chunk: a global unit (the
-// two global blocks stacked against one range of 8 tiles: every row attends
-// every tile), a full-attention unit (blocks 2j, 2j+1 against every tile), or
-// -- dq kernel only -- a middle unit of query blocks (i, i+1) against the
-// union of their key blocks [TFG-BigBird, section "随机块掩码是如何生成的";
-// HF-Pegasus, section "三类注意力组合"], a half mask per tile. In the dk/dv
-// kernel the stationary tiles are key blocks and the moving ones query
-// blocks; a global or full-attention unit decodes the same way (every query
-// attends a global key block, and in full attention every key).
-// Whole warp: the lanes fetch the random entries, lane 0 builds the list.
+// Everything is counted in 64-token tiles: a block of 64 is one tile (kBt =
+// 1), a block of 128 two (kBt = 2). Unit u of either kernel when its list fits
+// one chunk: a global unit (the global rows stacked against one range of 8
+// tiles, every row attending every tile: both global blocks in one unit at
+// block 64, one unit per global block at block 128), a full-attention unit
+// (tiles 2j, 2j+1 against every tile), or -- dq kernel only -- a middle unit:
+// query blocks (i, i+1) against the union of their key blocks with a half
+// mask per tile (block 64), or query block i against its own key blocks
+// (block 128) [TFG-BigBird, section "随机块掩码是如何生成的"; HF-Pegasus,
+// section "三类注意力组合"]. In the dk/dv kernel the stationary tiles are key
+// tiles and the moving ones query tiles; a global or full-attention unit
+// decodes the same way (every query attends a global key block, and in full
+// attention every key). Whole warp: the lanes fetch the random entries, lane
+// 0 builds the list.
+template <int kBt>
 __device__ void build_simple(const Params& p, int u, Unit& ui, int lane) {
   int n = 0;
-  auto add = [&](int t, int hm) {
-    if (t < 0 || t >= p.nb) {
-      atomicOr(p.status, kStatusBadRandAttn);
-      return;
-    }
+  // one tile, merging the half masks of a tile listed twice (set semantics)
+  auto add_tile = [&](int t, int hm) {
     for (int e = 0; e < n; ++e)
       if (ui.mt[e] == t) {
         ui.hm[e] |= static_cast<uint8_t>(hm);
@@ -197,53 +213,88 @@ __device__ void build_simple(const Params& p, int u, Unit& ui, int lane) {
     ui.hm[n] = static_cast<uint8_t>(hm);
     ++n;
   };
+  // one block of the pattern; an entry outside [0, nb) is skipped and reported
+  auto add_block = [&](int kb, int hm) {
+    if (kb < 0 || kb >= p.nb) {
+      atomicOr(p.status, kStatusBadRandAttn);
+      return;
+    }
+#pragma unroll
+    for (int t = 0; t < kBt; ++t) add_tile(kb * kBt + t, hm);
+  };
   int bh, top, bot, split = -1;
   if (u >= p.n_mid_units) {
     const int v = u - p.n_mid_units;
     int t0, t1;
     if (p.sparse) {
-      bh = v / p.nsplit;
-      const int s = v % p.nsplit;
-      top = 0;
-      bot = p.nb - 1;
+      bh = v / p.nparts;
+      const int part = v % p.nparts;
+      const int g = part / p.nsplit;
+      const int s = part % p.nsplit;
+      if (p.n_glob == 1) {
+        top = 0;
+        bot = p.nt - 1;
+      } else {
+        top = g == 0 ? 0 : p.nt - 2;
+        bot = top + 1;
+      }
       t0 = s * kSplit;
-      t1 = min(p.nb, t0 + kSplit);
-      split = p.nsplit > 1 ? s : -1;
+      t1 = min(p.nt, t0 + kSplit);
+      split = p.nsplit > 1 ? part : -1;
     } else {
-      const int npair = (p.nb + 1) / 2;
+      const int npair = (p.nt + 1) / 2;
       bh = v / npair;
       const int pp = v % npair;
       top = 2 * pp;
-      bot = 2 * pp + 1 < p.nb ? 2 * pp + 1 : -1;
+      bot = 2 * pp + 1 < p.nt ? 2 * pp + 1 : -1;
       t0 = 0;
-      t1 = p.nb;
+      t1 = p.nt;
     }
     if (lane == 0)
-      for (int t = t0; t < t1; ++t) add(t, bot >= 0 ? 3 : 1);
+      for (int t = t0; t < t1; ++t) add_tile(t, bot >= 0 ? 3 : 1);
   } else {
     bh = u / p.n_mid_per_head;
     const int pp = u % p.n_mid_per_head;
     const int h = bh % p.H;
-    const int i = 1 + 2 * pp;
-    const bool pair = i + 1 <= p.nb - 2;
-    const int both = pair ? 3 : 1;
-    const int nrand = pair ? 2 * p.r : p.r;
-    const int32_t* ra = p.rand_attn + (static_cast<size_t>(h) * (p.nb - 2) + (i - 1)) * p.r;
-    const int rv = lane < nrand ? __ldg(ra + lane) : -1;
-    if (lane == 0) {
-      add(i - 1, 1);
-      add(i, both);
-      add(i + 1, both);
-      if (pair) add(i + 2, 2);
-      add(0, both);
-      add(p.nb - 1, both);
+    if (kBt == 1) {
+      const int i = 1 + 2 * pp;
+      const bool pair = i + 1 <= p.nb - 2;
+      const int both = pair ? 3 : 1;
+      const int nrand = pair ? 2 * p.r : p.r;
+      const int32_t* ra = p.rand_attn + (static_cast<size_t>(h) * (p.nb - 2) + (i - 1)) * p.r;
+      const int rv = lane < nrand ? __ldg(ra + lane) : -1;
+      if (lane == 0) {
+        add_block(i - 1, 1);
+        add_block(i, both);
+        add_block(i + 1, both);
+        if (pair) add_block(i + 2, 2);
+        add_block(0, both);
+        add_block(p.nb - 1, both);
+      }
+      for (int t = 0; t < nrand; ++t) {
+        const int x = __shfl_sync(0xffffffffu, rv, t);
+        if (lane == 0) add_block(x, t < p.r ? 1 : 2);
+      }
+      top = i;
+      bot = pair ? i + 1 : -1;
+    } else {
+      const int i = 1 + pp;
+      const int32_t* ra = p.rand_attn + (static_cast<size_t>(h) * (p.nb - 2) + (i - 1)) * p.r;
+      const int rv = lane < p.r ? __ldg(ra + lane) : -1;
+      if (lane == 0) {
+        add_block(i - 1, 3);
+        add_block(i, 3);
+        add_block(i + 1, 3);
+        add_block(0, 3);
+        add_block(p.nb - 1, 3);
+      }
+      for (int t = 0; t < p.r; ++t) {
+        const int x = __shfl_sync(0xffffffffu, rv, t);
+        if (lane == 0) add_block(x, 3);
+      }
+      top = 2 * i;
+      bot = 2 * i + 1;
     }
-    for (int t = 0; t < nrand; ++t) {
-      const int x = __shfl_sync(0xffffffffu, rv, t);
-      if (lane == 0) add(x, t < p.r ? 1 : 2);
-    }
-    top = i;
-    bot = pair ? i + 1 : -1;
   }
   if (lane == 0) {
     ui.n = n;
@@ -262,15 +313,16 @@ __device__ void build_simple(const Params& p, int u, Unit& ui, int lane) {
 // Unit preparation and scheduling (one warp), up to four chunks ahead: a CTA's
 // first unit is its block index, later ones are tickets from the workspace
 // counter (units numbered longest first). Publishes a stop slot at the end.
-// The dk/dv kernel's middle units -- key blocks (j, j+1) -- list the query
-// blocks that attend either: the two global query blocks, the window
-// neighbours, and every middle query block whose random entries pick j or
-// j+1, found by scanning rand_attn 32 query blocks at a time (set semantics:
-// repeated or window-overlapping picks add nothing). A list longer than a
-// chunk goes out as several chunks; only the first starts the accumulators
-// from zero and only the last is followed by the epilogue.
-template <bool kKV>
-__device__ void prep_role(Smem& s, const Params& p) {
+// The dk/dv kernel's middle units -- key blocks (j, j+1) at block 64, key
+// block j (two tiles) at block 128 -- list the query tiles of the query
+// blocks that attend them: the two global query blocks, the window
+// neighbours, and every middle query block whose random entries pick one of
+// them, found by scanning rand_attn 32 (block 128: 16) query blocks at a time
+// (set semantics: repeated or window-overlapping picks add nothing). A list
+// longer than a chunk goes out as several chunks; only the first starts the
+// accumulators from zero and only the last is followed by the epilogue.
+template <int kD, int kBt, bool kKV>
+__device__ void prep_role(Smem<kD>& s, const Params& p) {
   const int lane = threadIdx.x & 31;
   uint32_t ut = 0;  // chunks published so far
   auto acquire = [&]() -> Unit* {
@@ -292,7 +344,8 @@ __device__ void prep_role(Smem& s, const Params& p) {
     const size_t row0 = static_cast<size_t>(ui.bh) * p.L;
     for (int t = lane; t < 2 * n; t += 32) {
       const uint16_t* base = t < n ? (kKV ? p.q : p.k) : (kKV ? p.dout : p.v);
-      prefetch_l2_bulk(base + (row0 + static_cast<size_t>(ui.mt[t < n ? t : t - n]) * kBlock) * kDim, kTileBytes);
+      prefetch_l2_bulk(base + (row0 + static_cast<size_t>(ui.mt[t < n ? t : t - n]) * kBlock) * kD,
+                       BGeo<kD>::kTileBytes);
     }
   };
   int u = blockIdx.x;
@@ -314,19 +367,21 @@ __device__ void prep_role(Smem& s, const Params& p) {
     int next = 0;
     if (lane == 0) next = static_cast<int>(gridDim.x) + atomicAdd(&p.counters[0], 1);
     if (!kKV || u >= p.n_mid_units) {
-      build_simple(p, u, *ui, lane);
+      build_simple<kBt>(p, u, *ui, lane);
       finish(*ui);
     } else {
+      constexpr int kBatch = kBt == 1 ? 32 : 16;  // query blocks per scan batch (kBt tiles each)
       const int bh = u / p.n_mid_per_head;
       const int pp = u % p.n_mid_per_head;
       const int h = bh % p.H;
-      const int j = 1 + 2 * pp;
-      const bool pair = j + 1 <= p.nb - 2;
+      // key blocks j and j + 1 (block 64) or key block j (block 128)
+      const int j = kBt == 1 ? 1 + 2 * pp : 1 + pp;
+      const bool pair = kBt == 1 && j + 1 <= p.nb - 2;
       auto header = [&](Unit& c, int first) {
         if (lane == 0) {
           c.bh = bh;
-          c.top = j;
-          c.bot = pair ? j + 1 : -1;
+          c.top = kBt * j;
+          c.bot = kBt == 2 ? 2 * j + 1 : (pair ? j + 1 : -1);
           c.split = -1;
           c.first = first;
           c.last = 0;
@@ -336,25 +391,28 @@ __device__ void prep_role(Smem& s, const Params& p) {
       header(*ui, 1);
       int n = 0;
       bool ok = true;
-      for (int base = 0; base < p.nb && ok; base += 32) {
+      // at block 128 both tiles of key block j are used by every row of an
+      // attending query block: bits 1 and 2 together
+      const int jbits = kBt == 1 ? 1 : 3;
+      for (int base = 0; base < p.nb && ok; base += kBatch) {
         const int q = base + lane;
         int hm = 0;
-        if (q < p.nb) {
+        if (lane < kBatch && q < p.nb) {
           if (q == 0 || q == p.nb - 1) {
-            hm = pair ? 3 : 1;
+            hm = kBt == 2 || pair ? 3 : 1;
           } else {
-            hm = (abs(q - j) <= 1 ? 1 : 0) | (pair && abs(q - (j + 1)) <= 1 ? 2 : 0);
+            hm = (abs(q - j) <= 1 ? jbits : 0) | (pair && abs(q - (j + 1)) <= 1 ? 2 : 0);
           }
         }
         // random picks of the middle query blocks qlo .. qhi-1 of this batch
-        const int qlo = max(base, 1), qhi = min(base + 32, p.nb - 1);
+        const int qlo = max(base, 1), qhi = min(base + kBatch, p.nb - 1);
         if (qhi > qlo) {
           const int cnt = (qhi - qlo) * p.r;
           const int32_t* ra = p.rand_attn + (static_cast<size_t>(h) * (p.nb - 2) + (qlo - 1)) * p.r;
           for (int e = lane; e < cnt; e += 32) {
             const int x = __ldg(ra + e);
             if (x < 0 || x >= p.nb) atomicOr(p.status, kStatusBadRandAttn);
-            const int bits = (x == j ? 1 : 0) | (pair && x == j + 1 ? 2 : 0);
+            const int bits = (x == j ? jbits : 0) | (pair && x == j + 1 ? 2 : 0);
             // lanes holding entries of the same query block meet here: atomic
             if (bits) atomicOr(&s.rbits[qlo - base + e / p.r], static_cast<unsigned int>(bits));
           }
@@ -365,7 +423,7 @@ __device__ void prep_role(Smem& s, const Params& p) {
         s.rbits[lane] = 0;
         __syncwarp();
         const uint32_t mask = __ballot_sync(0xffffffffu, hm != 0);
-        const int c = __popc(mask);
+        const int c = kBt * __popc(mask);  // tiles this batch adds
         if (n + c > kMaxList) {
           if (lane == 0) ui->n = n;
           finish(*ui);
@@ -378,9 +436,12 @@ __device__ void prep_role(Smem& s, const Params& p) {
           n = 0;
         }
         if (hm) {
-          const int pos = n + __popc(mask & ((1u << lane) - 1u));
-          ui->mt[pos] = q;
-          ui->hm[pos] = static_cast<uint8_t>(hm);
+          const int pos = n + kBt * __popc(mask & ((1u << lane) - 1u));
+#pragma unroll
+          for (int t = 0; t < kBt; ++t) {
+            ui->mt[pos + t] = kBt * q + t;
+            ui->hm[pos + t] = static_cast<uint8_t>(hm);
+          }
         }
         n += c;
       }
@@ -411,9 +472,10 @@ __device__ __forceinline__ uint32_t lo_col(int q) { return 16 * q + 8; }
 // kernel, the query tile's lse and D) into a 2-deep ring.
 // dq kernel: A1 = Q, A2 = dO, B1 = K, B2 = V. dk/dv kernel: A1 = K, A2 = V,
 // B1 = Q, B2 = dO.
-template <bool kKV>
-__device__ void producer_role(Smem& s, const Params& p, const CUtensorMap* tmA1, const CUtensorMap* tmA2,
+template <int kD, bool kKV>
+__device__ void producer_role(Smem<kD>& s, const Params& p, const CUtensorMap* tmA1, const CUtensorMap* tmA2,
                               const CUtensorMap* tmB1, const CUtensorMap* tmB2) {
+  using G = BGeo<kD>;
   const int lane = threadIdx.x & 31;
   const uint64_t pol_a = l2_policy_evict_first();
   const uint64_t pol_b = l2_policy_evict_last();
@@ -432,12 +494,17 @@ __device__ void producer_role(Smem& s, const Params& p, const CUtensorMap* tmA1,
         ok = mbar_wait(smem_u32(&s.a_free), (ua & 1) ^ 1);
         if (ok) {
           const uint32_t bar = smem_u32(&s.a_full);
-          mbar_arrive_expect_tx(bar, (ui.bot >= 0 ? 4 : 2) * kTileBytes);
-          tma_load_2d(smem_u32(s.a1), tmA1, bar, 0, row0 + ui.top * kBlock, pol_a);
-          tma_load_2d(smem_u32(s.a2), tmA2, bar, 0, row0 + ui.top * kBlock, pol_a);
-          if (ui.bot >= 0) {
-            tma_load_2d(smem_u32(s.a1) + kTileBytes, tmA1, bar, 0, row0 + ui.bot * kBlock, pol_a);
-            tma_load_2d(smem_u32(s.a2) + kTileBytes, tmA2, bar, 0, row0 + ui.bot * kBlock, pol_a);
+          mbar_arrive_expect_tx(bar, (ui.bot >= 0 ? 4 : 2) * G::kTileBytes);
+          // chunk c of the unit's rows at c * 16 KB: the top tile, then the bottom one
+#pragma unroll
+          for (int c = 0; c < G::kChunks; ++c) {
+            const uint32_t off = c * G::kAChunkBytes;
+            tma_load_2d(smem_u32(s.a1) + off, tmA1, bar, 64 * c, row0 + ui.top * kBlock, pol_a);
+            tma_load_2d(smem_u32(s.a2) + off, tmA2, bar, 64 * c, row0 + ui.top * kBlock, pol_a);
+            if (ui.bot >= 0) {
+              tma_load_2d(smem_u32(s.a1) + off + kChunkBytes, tmA1, bar, 64 * c, row0 + ui.bot * kBlock, pol_a);
+              tma_load_2d(smem_u32(s.a2) + off + kChunkBytes, tmA2, bar, 64 * c, row0 + ui.bot * kBlock, pol_a);
+            }
           }
         }
         ++ua;
@@ -448,9 +515,12 @@ __device__ void producer_role(Smem& s, const Params& p, const CUtensorMap* tmA1,
         if (!ok) break;
         const uint32_t bar = smem_u32(&s.b_full[st]);
         const int32_t row = row0 + ui.mt[e] * kBlock;
-        mbar_arrive_expect_tx(bar, 2 * kTileBytes + (kKV ? 2 * kBlock * 4 : 0));
-        tma_load_2d(smem_u32(s.b1[st]), tmB1, bar, 0, row, pol_b);
-        tma_load_2d(smem_u32(s.b2[st]), tmB2, bar, 0, row, pol_b);
+        mbar_arrive_expect_tx(bar, 2 * G::kTileBytes + (kKV ? 2 * kBlock * 4 : 0));
+#pragma unroll
+        for (int c = 0; c < G::kChunks; ++c) {
+          tma_load_2d(smem_u32(s.b1[st]) + c * kChunkBytes, tmB1, bar, 64 * c, row, pol_b);
+          tma_load_2d(smem_u32(s.b2[st]) + c * kChunkBytes, tmB2, bar, 64 * c, row, pol_b);
+        }
         if (kKV) {
           bulk_load(smem_u32(s.col_lse[st]), p.lse + row, kBlock * 4, bar);
           bulk_load(smem_u32(s.col_d[st]), p.dd + row, kBlock * 4, bar);
@@ -477,10 +547,11 @@ __device__ void producer_role(Smem& s, const Params& p, const CUtensorMap* tmA1,
 // 64 moving rows):
 //   dq kernel:   acc1 += (dS_hi + dS_lo) B1                          (dQ += dS K)
 //   dk/dv kernel: acc1 += (P_hi + P_lo) B2, acc2 += (dS_hi + dS_lo) B1 (dV += P^T dO, dK += dS^T Q)
-template <bool kKV>
-__device__ void mma_role(Smem& s, const Params& p, uint32_t tmem) {
+template <int kD, bool kKV>
+__device__ void mma_role(Smem<kD>& s, const Params& p, uint32_t tmem) {
+  using G = BGeo<kD>;
   const uint32_t idesc1 = idesc_f32acc(kRows, kBlock, true, false);
-  const uint32_t idesc2 = idesc_f32acc(kRows, kDim, true, true);
+  const uint32_t idesc2 = idesc_f32acc(kRows, 64, true, true);  // one 64-column chunk of d
   const uint32_t a1 = smem_u32(s.a1), a2 = smem_u32(s.a2);
   uint32_t g = 0, ua = 0;
   bool ok = true;
@@ -497,14 +568,15 @@ __device__ void mma_role(Smem& s, const Params& p, uint32_t tmem) {
       if (g >= 1 && !mbar_wait(smem_u32(&s.xy_free), (g - 1) & 1)) { ok = false; break; }
       tc_fence_after();
       const uint32_t b1 = smem_u32(s.b1[st]), b2 = smem_u32(s.b2[st]);
+      // K = d in steps of 16: four per 64-column chunk
 #pragma unroll
-      for (int kk = 0; kk < kDim / 16; ++kk)
-        mma_ss(tmem + kColX, sdesc_sw128(a1 + kk * 32, 16, 1024), sdesc_sw128(b1 + kk * 32, 16, 1024), idesc1,
-               kk > 0 ? 1u : 0u);
+      for (int kk = 0; kk < kD / 16; ++kk)
+        mma_ss(tmem + kColX, sdesc_sw128(a1 + (kk >> 2) * G::kAChunkBytes + (kk & 3) * 32, 16, 1024),
+               sdesc_sw128(b1 + (kk >> 2) * kChunkBytes + (kk & 3) * 32, 16, 1024), idesc1, kk > 0 ? 1u : 0u);
 #pragma unroll
-      for (int kk = 0; kk < kDim / 16; ++kk)
-        mma_ss(tmem + kColY, sdesc_sw128(a2 + kk * 32, 16, 1024), sdesc_sw128(b2 + kk * 32, 16, 1024), idesc1,
-               kk > 0 ? 1u : 0u);
+      for (int kk = 0; kk < kD / 16; ++kk)
+        mma_ss(tmem + kColY, sdesc_sw128(a2 + (kk >> 2) * G::kAChunkBytes + (kk & 3) * 32, 16, 1024),
+               sdesc_sw128(b2 + (kk >> 2) * kChunkBytes + (kk & 3) * 32, 16, 1024), idesc1, kk > 0 ? 1u : 0u);
       mma_commit(smem_u32(&s.x_full));
       if (last && e == n - 1) mma_commit(smem_u32(&s.a_free));
       // the unit's first step overwrites the accumulators, once the previous
@@ -513,25 +585,33 @@ __device__ void mma_role(Smem& s, const Params& p, uint32_t tmem) {
       if (zero && !mbar_wait(smem_u32(&s.acc_free), (ua & 1) ^ 1)) { ok = false; break; }
       if (!mbar_wait(smem_u32(&s.p_full), g & 1)) { ok = false; break; }
       tc_fence_after();
-      if (kKV) {
+      // accumulator columns 64 c .. 64 c + 63 from chunk c of the moving tile
 #pragma unroll
-        for (int kk = 0; kk < kBlock / 16; ++kk) {
-          mma_ts(tmem + kColA1, tmem + kColX + hi_col(kk), sdesc_sw128(b2 + kk * 2048, 8192, 1024), idesc2,
-                 (zero && kk == 0) ? 0u : 1u);
-          mma_ts(tmem + kColA1, tmem + kColX + lo_col(kk), sdesc_sw128(b2 + kk * 2048, 8192, 1024), idesc2, 1u);
-        }
+      for (int c = 0; c < G::kChunks; ++c) {
+        const uint32_t boff = c * kChunkBytes;
+        if (kKV) {
 #pragma unroll
-        for (int kk = 0; kk < kBlock / 16; ++kk) {
-          mma_ts(tmem + kColA2, tmem + kColY + hi_col(kk), sdesc_sw128(b1 + kk * 2048, 8192, 1024), idesc2,
-                 (zero && kk == 0) ? 0u : 1u);
-          mma_ts(tmem + kColA2, tmem + kColY + lo_col(kk), sdesc_sw128(b1 + kk * 2048, 8192, 1024), idesc2, 1u);
-        }
-      } else {
+          for (int kk = 0; kk < kBlock / 16; ++kk) {
+            mma_ts(tmem + kColA1 + 64 * c, tmem + kColX + hi_col(kk), sdesc_sw128(b2 + boff + kk * 2048, 8192, 1024),
+                   idesc2, (zero && kk == 0) ? 0u : 1u);
+            mma_ts(tmem + kColA1 + 64 * c, tmem + kColX + lo_col(kk), sdesc_sw128(b2 + boff + kk * 2048, 8192, 1024),
+                   idesc2, 1u);
+          }
 #pragma unroll
-        for (int kk = 0; kk < kBlock / 16; ++kk) {
-          mma_ts(tmem + kColA1, tmem + kColY + hi_col(kk), sdesc_sw128(b1 + kk * 2048, 8192, 1024), idesc2,
-                 (zero && kk == 0) ? 0u : 1u);
-          mma_ts(tmem + kColA1, tmem + kColY + lo_col(kk), sdesc_sw128(b1 + kk * 2048, 8192, 1024), idesc2, 1u);
+          for (int kk = 0; kk < kBlock / 16; ++kk) {
+            mma_ts(tmem + G::kColA2 + 64 * c, tmem + kColY + hi_col(kk),
+                   sdesc_sw128(b1 + boff + kk * 2048, 8192, 1024), idesc2, (zero && kk == 0) ? 0u : 1u);
+            mma_ts(tmem + G::kColA2 + 64 * c, tmem + kColY + lo_col(kk),
+                   sdesc_sw128(b1 + boff + kk * 2048, 8192, 1024), idesc2, 1u);
+          }
+        } else {
+#pragma unroll
+          for (int kk = 0; kk < kBlock / 16; ++kk) {
+            mma_ts(tmem + kColA1 + 64 * c, tmem + kColY + hi_col(kk), sdesc_sw128(b1 + boff + kk * 2048, 8192, 1024),
+                   idesc2, (zero && kk == 0) ? 0u : 1u);
+            mma_ts(tmem + kColA1 + 64 * c, tmem + kColY + lo_col(kk), sdesc_sw128(b1 + boff + kk * 2048, 8192, 1024),
+                   idesc2, 1u);
+          }
         }
       }
       mma_commit(smem_u32(&s.xy_free));
@@ -602,8 +682,8 @@ __device__ __forceinline__ void piece_pds(const uint32_t (&x)[16], const uint32_
 // epilogue, each warp its 32 of the 64 columns (dq = acc1 / sqrt(d); dv =
 // acc1, dk = acc2 / sqrt(d); raw into the partial-sum slot of a split global
 // unit).
-template <bool kKV>
-__device__ void elem_role(Smem& s, const Params& p, uint32_t tmem) {
+template <int kD, bool kKV>
+__device__ void elem_role(Smem<kD>& s, const Params& p, uint32_t tmem) {
   constexpr float kLog2e = 1.4426950408889634f;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -679,20 +759,20 @@ __device__ void elem_role(Smem& s, const Params& p, uint32_t tmem) {
     __syncwarp();
     if (lane == 0) mbar_arrive(smem_u32(&s.info_empty[ut & 3]));
     if (!last) continue;
-    // ---- epilogue: this warp's 32 columns of each accumulator
+    // ---- epilogue: this warp's d / 2 columns of each accumulator
     if (!warp_wait(smem_u32(&s.acc_full), ua & 1)) { if (lane == 0) flag_timeout(p); return; }
     tc_fence_after();
     if (exists) {
-      const size_t prow = (static_cast<size_t>(bh) * p.nsplit + (split >= 0 ? split : 0)) * kRows + rowi;
+      const size_t prow = (static_cast<size_t>(bh) * p.nparts + (split >= 0 ? split : 0)) * kRows + rowi;
 #pragma unroll 1
       for (int a = 0; a < (kKV ? 2 : 1); ++a) {
         // acc1: dq (dq kernel) or dv; acc2: dk
         const float f = (split >= 0 || (kKV && a == 0)) ? 1.f : p.scale;
-        float* dst = split >= 0 ? (a == 0 ? p.part1 : p.part2) + prow * kDim : (a == 0 ? p.g1 : p.g2) + row * kDim;
+        float* dst = split >= 0 ? (a == 0 ? p.part1 : p.part2) + prow * kD : (a == 0 ? p.g1 : p.g2) + row * kD;
 #pragma unroll 1
-        for (int c0 = 32 * chalf; c0 < 32 * chalf + 32; c0 += 16) {
+        for (int c0 = (kD / 2) * chalf; c0 < (kD / 2) * (chalf + 1); c0 += 16) {
           uint32_t o[16];
-          tmem_ld16(lane_addr + (a == 0 ? kColA1 : kColA2) + c0, o);
+          tmem_ld16(lane_addr + (a == 0 ? kColA1 : BGeo<kD>::kColA2) + c0, o);
           tmem_wait_ld();
           float4* d4 = reinterpret_cast<float4*>(dst + c0);
 #pragma unroll
@@ -711,14 +791,15 @@ __device__ void elem_role(Smem& s, const Params& p, uint32_t tmem) {
 
 // ------------------------------------------------------------ kernels
 
-// kKV = false: dq. kKV = true: dk and dv.
-template <bool kKV>
-__global__ void __launch_bounds__(kThreads, kCtasPerSm)
+// kKV = false: dq. kKV = true: dk and dv. kD: head dimension; kBt: tiles per block.
+template <int kD, int kBt, bool kKV>
+__global__ void __launch_bounds__(kThreads, BGeo<kD>::kCtasPerSm)
 bwd_kernel(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmA2,
            const __grid_constant__ CUtensorMap tmB1, const __grid_constant__ CUtensorMap tmB2,
            const __grid_constant__ Params p) {
+  constexpr uint32_t kTmemCols = BGeo<kD>::tmem_cols(kKV);
   extern __shared__ uint8_t smem_raw[];
-  Smem& s = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Smem<kD>& s = *reinterpret_cast<Smem<kD>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   if (warp == 9) {
@@ -754,13 +835,13 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUt
   tc_fence_after();
   const uint32_t tmem = s.tmem_base;
   if (warp < kElemWarps) {
-    elem_role<kKV>(s, p, tmem);
+    elem_role<kD, kKV>(s, p, tmem);
   } else if (warp == 8) {
-    producer_role<kKV>(s, p, &tmA1, &tmA2, &tmB1, &tmB2);
+    producer_role<kD, kKV>(s, p, &tmA1, &tmA2, &tmB1, &tmB2);
   } else if (warp == 9) {
-    if (lane == 0) mma_role<kKV>(s, p, tmem);
+    if (lane == 0) mma_role<kD, kKV>(s, p, tmem);
   } else if (warp == 10) {
-    prep_role<kKV>(s, p);
+    prep_role<kD, kBt, kKV>(s, p);
   }
   tc_fence_before();
   __syncthreads();
@@ -779,22 +860,24 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUt
   }
 }
 
-// D[row] = sum_c dout[row, c] * out[row, c]: 16 threads per row, 4 columns
-// each; a CTA of 256 threads covers 16 rows.
+// D[row] = sum_c dout[row, c] * out[row, c]: d / 4 threads per row, 4
+// columns each; a CTA of 256 threads covers 1024 / d rows.
+template <int kD>
 __global__ void __launch_bounds__(256)
 bwd_rowdot_kernel(const uint16_t* __restrict__ dout, const void* __restrict__ out, int out_f32, float* __restrict__ dd,
                   size_t rows) {
-  const size_t row = static_cast<size_t>(blockIdx.x) * 16 + (threadIdx.x >> 4);
-  const int c4 = threadIdx.x & 15;
+  constexpr int kTpr = kD / 4;
+  const size_t row = static_cast<size_t>(blockIdx.x) * (256 / kTpr) + threadIdx.x / kTpr;
+  const int c4 = threadIdx.x % kTpr;
   float acc = 0.f;
   if (row < rows) {
-    const uint2 g = __ldg(reinterpret_cast<const uint2*>(dout + row * kDim) + c4);
+    const uint2 g = __ldg(reinterpret_cast<const uint2*>(dout + row * kD) + c4);
     float o[4];
     if (out_f32) {
-      const float4 t = __ldg(reinterpret_cast<const float4*>(static_cast<const float*>(out) + row * kDim) + c4);
+      const float4 t = __ldg(reinterpret_cast<const float4*>(static_cast<const float*>(out) + row * kD) + c4);
       o[0] = t.x; o[1] = t.y; o[2] = t.z; o[3] = t.w;
     } else {
-      const uint2 t = __ldg(reinterpret_cast<const uint2*>(static_cast<const uint16_t*>(out) + row * kDim) + c4);
+      const uint2 t = __ldg(reinterpret_cast<const uint2*>(static_cast<const uint16_t*>(out) + row * kD) + c4);
       o[0] = __uint_as_float(t.x << 16); o[1] = __uint_as_float(t.x & 0xFFFF0000u);
       o[2] = __uint_as_float(t.y << 16); o[3] = __uint_as_float(t.y & 0xFFFF0000u);
     }
@@ -802,34 +885,45 @@ bwd_rowdot_kernel(const uint16_t* __restrict__ dout, const void* __restrict__ ou
           __uint_as_float(g.y << 16) * o[2] + __uint_as_float(g.y & 0xFFFF0000u) * o[3];
   }
 #pragma unroll
-  for (int off = 8; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+  for (int off = kTpr / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
   if (row < rows && c4 == 0) dd[row] = acc;
 }
 
-// The split global units' partial sums: rows 0..63 of a unit belong to tile 0
-// and rows 64..127 to tile nb-1 of head bh; dst = f * sum over the ranges.
-// 16 threads per row, 4 columns each; grid (B*H, 128 / 16).
+// The split global units' partial sums, dst = f * sum over the ranges. Rows
+// 0..63 and 64..127 of global unit g of head bh are tiles 0 and nt-1 (block
+// 64: both global blocks in one unit), or the two tiles of block 0 (g = 0) or
+// of block nb-1 (block 128). d / 4 threads per row, 4 columns each; grid
+// (B*H*n_glob, 128 d / 1024).
+template <int kD>
 __global__ void __launch_bounds__(256)
-bwd_sum_kernel(const float* __restrict__ part, float* __restrict__ dst, int nsplit, int L, int nb, float f) {
-  const int bh = blockIdx.x;
-  const int r = blockIdx.y * 16 + (threadIdx.x >> 4);
-  const int c4 = threadIdx.x & 15;
+bwd_sum_kernel(const float* __restrict__ part, float* __restrict__ dst, int nsplit, int n_glob, int L, int nt,
+               float f) {
+  constexpr int kTpr = kD / 4;
+  const int bh = blockIdx.x / n_glob;
+  const int g = blockIdx.x % n_glob;
+  const int r = blockIdx.y * (256 / kTpr) + static_cast<int>(threadIdx.x) / kTpr;
+  const int c4 = static_cast<int>(threadIdx.x) % kTpr;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  const size_t base = (static_cast<size_t>(bh) * n_glob + g) * nsplit;
   for (int sidx = 0; sidx < nsplit; ++sidx) {
-    const float4 t =
-        __ldg(reinterpret_cast<const float4*>(part + ((static_cast<size_t>(bh) * nsplit + sidx) * kRows + r) * kDim) + c4);
+    const float4 t = __ldg(reinterpret_cast<const float4*>(part + ((base + sidx) * kRows + r) * kD) + c4);
     acc.x += t.x;
     acc.y += t.y;
     acc.z += t.z;
     acc.w += t.w;
   }
-  const int tile = r < kBlock ? 0 : nb - 1;
+  const int tile = n_glob == 1 ? (r < kBlock ? 0 : nt - 1) : (g == 0 ? 0 : nt - 2) + r / kBlock;
   const size_t row = static_cast<size_t>(bh) * L + static_cast<size_t>(tile) * kBlock + (r & (kBlock - 1));
-  reinterpret_cast<float4*>(dst + row * kDim)[c4] = make_float4(acc.x * f, acc.y * f, acc.z * f, acc.w * f);
+  reinterpret_cast<float4*>(dst + row * kD)[c4] = make_float4(acc.x * f, acc.y * f, acc.z * f, acc.w * f);
 }
 
-static_assert(sizeof(Smem) + 1024 <= kSmemRequest, "shared memory request below the kernel's use");
-static_assert(3 * (kSmemRequest + 1024) > 228 * 1024, "a third CTA per SM would wait for TMEM");
+template <int kD>
+constexpr int smem_request() {
+  return kD == 64 ? kSmemRequest64 : static_cast<int>(sizeof(Smem<kD>) + 1024);
+}
+static_assert(sizeof(Smem<64>) + 1024 <= kSmemRequest64, "shared memory request below the kernel's use");
+static_assert(3 * (kSmemRequest64 + 1024) > 228 * 1024, "a third CTA per SM would wait for TMEM");
+static_assert(2 * (sizeof(Smem<128>) + 2048) > 228 * 1024, "d = 128: one CTA per SM");
 
 }  // namespace bbw
 
@@ -838,28 +932,33 @@ static_assert(3 * (kSmemRequest + 1024) > 228 * 1024, "a third CTA per SM would 
 namespace {
 
 struct BwdPlan {
-  int nb = 0;
+  int nb = 0, nt = 0, bt = 1;
   bool sparse = false;
-  int nsplit = 1;
+  int nsplit = 1, n_glob = 1;
   size_t d_off = 0, partq_off = 0, partv_off = 0, partk_off = 0, bytes = 0;
 };
 
+// Blocks of 64 or 128 at d = 64 or 128; full attention wider than one unit's
+// list (block 128 with r > 8) is not supported.
 int bwd_plan(int B, int H, int L, int d, int block, int r, unsigned flags, BwdPlan& pl) {
   using namespace bbw;
   if (B <= 0 || H <= 0 || L <= 0 || d <= 0 || block <= 0 || r < 1 || L % block != 0) return BB_ERR_INVALID_ARG;
-  if (d != kDim || block != kBlock || r > kMaxR) return BB_ERR_UNSUPPORTED;
+  if ((d != 64 && d != 128) || (block != kBlock && block != 2 * kBlock) || r > kMaxR) return BB_ERR_UNSUPPORTED;
   if (static_cast<int64_t>(B) * H * L >= (int64_t(1) << 31)) return BB_ERR_UNSUPPORTED;
   pl.nb = L / block;
+  pl.bt = block / kBlock;
+  pl.nt = L / kBlock;
   pl.sparse = (flags & BB_FLAG_FORCE_SPARSE) || pl.nb > 5 + 2 * r;
   if (pl.sparse && pl.nb < 5 + r) return BB_ERR_INVALID_ARG;
-  // a full-attention unit lists every block: nb <= 5 + 2r <= kMaxList
-  pl.nsplit = pl.sparse ? (pl.nb + kSplit - 1) / kSplit : 1;
+  if (!pl.sparse && pl.nt > kMaxList) return BB_ERR_UNSUPPORTED;
+  pl.nsplit = pl.sparse ? (pl.nt + kSplit - 1) / kSplit : 1;
+  pl.n_glob = pl.sparse && pl.bt == 2 ? 2 : 1;
   auto round256 = [](size_t x) { return (x + 255) / 256 * 256; };
   const size_t bhl = static_cast<size_t>(B) * H * L;
   pl.d_off = kCounterBytes;
   size_t off = pl.d_off + round256(bhl * sizeof(float));
   if (pl.nsplit > 1) {
-    const size_t part = static_cast<size_t>(B) * H * pl.nsplit * kRows * kDim * sizeof(float);
+    const size_t part = static_cast<size_t>(B) * H * pl.n_glob * pl.nsplit * kRows * d * sizeof(float);
     pl.partq_off = off;
     pl.partv_off = off + part;
     pl.partk_off = off + 2 * part;
@@ -869,18 +968,51 @@ int bwd_plan(int B, int H, int L, int d, int block, int r, unsigned flags, BwdPl
   return BB_OK;
 }
 
-bool set_attributes(int dev) {
+template <int kD>
+bool set_attributes_d() {
   using namespace bbw;
-  static bool done[64] = {};
-  if (dev < 0 || dev >= 64) return false;
-  if (done[dev]) return true;
-  const int smem = kSmemRequest;
-  for (const void* fn : {reinterpret_cast<const void*>(bwd_kernel<false>), reinterpret_cast<const void*>(bwd_kernel<true>)}) {
+  const int smem = smem_request<kD>();
+  for (const void* fn : {reinterpret_cast<const void*>(bwd_kernel<kD, 1, false>),
+                         reinterpret_cast<const void*>(bwd_kernel<kD, 1, true>),
+                         reinterpret_cast<const void*>(bwd_kernel<kD, 2, false>),
+                         reinterpret_cast<const void*>(bwd_kernel<kD, 2, true>)}) {
     if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) return false;
     if (cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout, 100) != cudaSuccess) return false;
   }
+  return true;
+}
+
+bool set_attributes(int dev) {
+  static bool done[64] = {};
+  if (dev < 0 || dev >= 64) return false;
+  if (done[dev]) return true;
+  if (!set_attributes_d<64>() || !set_attributes_d<128>()) return false;
   done[dev] = true;
   return true;
+}
+
+// The launches of one backward call: row dot, dq kernel, dk/dv kernel, then
+// the partial sums of the split global units.
+template <int kD, int kBt>
+cudaError_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tdo,
+                       const bbw::Params& pq, const bbw::Params& pk, const BwdPlan& pl, int sms, const void* dout,
+                       const void* out, int out_f32, float* dd, size_t rows, float* dq, float* dk, float* dv, int L,
+                       cudaStream_t stream) {
+  using namespace bbw;
+  const int grid = std::min(pq.total_units, BGeo<kD>::kCtasPerSm * sms);
+  const size_t smem = smem_request<kD>();
+  constexpr int kRowsPerCta = 256 / (kD / 4);
+  bwd_rowdot_kernel<kD><<<static_cast<unsigned>((rows + kRowsPerCta - 1) / kRowsPerCta), 256, 0, stream>>>(
+      static_cast<const uint16_t*>(dout), out, out_f32, dd, rows);
+  bwd_kernel<kD, kBt, false><<<grid, kThreads, smem, stream>>>(tq, tdo, tk, tv, pq);
+  bwd_kernel<kD, kBt, true><<<grid, kThreads, smem, stream>>>(tk, tv, tq, tdo, pk);
+  if (pl.nsplit > 1) {
+    const dim3 sg(pq.BH * pl.n_glob, kRows / kRowsPerCta);
+    bwd_sum_kernel<kD><<<sg, 256, 0, stream>>>(pq.part1, dq, pl.nsplit, pl.n_glob, L, pl.nt, pq.scale);
+    bwd_sum_kernel<kD><<<sg, 256, 0, stream>>>(pk.part1, dv, pl.nsplit, pl.n_glob, L, pl.nt, 1.0f);
+    bwd_sum_kernel<kD><<<sg, 256, 0, stream>>>(pk.part2, dk, pl.nsplit, pl.n_glob, L, pl.nt, pq.scale);
+  }
+  return cudaGetLastError();
 }
 
 }  // namespace
@@ -917,8 +1049,8 @@ extern "C" int bigbird_attn_bwd_ex(const void* q, const void* k, const void* v, 
 
   const size_t rows = static_cast<size_t>(B) * H * L;
   CUtensorMap tq, tk, tv, tdo;
-  if (!make_tile_map(&tq, q, rows) || !make_tile_map(&tk, k, rows) || !make_tile_map(&tv, v, rows) ||
-      !make_tile_map(&tdo, dout, rows))
+  if (!make_tile_map_d(&tq, q, rows, d) || !make_tile_map_d(&tk, k, rows, d) || !make_tile_map_d(&tv, v, rows, d) ||
+      !make_tile_map_d(&tdo, dout, rows, d))
     return BB_ERR_CUDA;
 
   void* ws = workspace;
@@ -949,40 +1081,37 @@ extern "C" int bigbird_attn_bwd_ex(const void* q, const void* k, const void* v, 
   p.nb = pl.nb;
   p.r = r;
   p.BH = B * H;
+  p.nt = pl.nt;
   p.sparse = pl.sparse ? 1 : 0;
   p.nsplit = pl.nsplit;
-  p.n_mid_per_head = pl.sparse ? (pl.nb - 2 + 1) / 2 : 0;
+  p.n_glob = pl.n_glob;
+  p.nparts = pl.n_glob * pl.nsplit;
+  // middle units: pairs of blocks (block 64) or single blocks (block 128)
+  p.n_mid_per_head = pl.sparse ? (pl.bt == 1 ? (pl.nb - 2 + 1) / 2 : pl.nb - 2) : 0;
   p.n_mid_units = p.BH * p.n_mid_per_head;
-  p.total_units = p.n_mid_units + p.BH * (pl.sparse ? pl.nsplit : (pl.nb + 1) / 2);
+  p.total_units = p.n_mid_units + p.BH * (pl.sparse ? p.nparts : (pl.nt + 1) / 2);
   p.scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(d));
   p.bias_raw = -10000.0f * sqrtf(static_cast<float>(d));
   p.scale = 1.0f / sqrtf(static_cast<float>(d));
 
-  const int grid = std::min(p.total_units, kCtasPerSm * sms);
-  const size_t smem = kSmemRequest;
-  bwd_rowdot_kernel<<<static_cast<unsigned>((rows + 15) / 16), 256, 0, stream>>>(
-      static_cast<const uint16_t*>(dout), out, out_dtype == BB_OUT_F32 ? 1 : 0, dd, rows);
-  // dq
   Params pq = p;
   pq.g1 = dq;
   pq.part1 = pl.nsplit > 1 ? reinterpret_cast<float*>(wsb + pl.partq_off) : nullptr;
   pq.counters = reinterpret_cast<int*>(wsb);
-  bwd_kernel<false><<<grid, kThreads, smem, stream>>>(tq, tdo, tk, tv, pq);
-  // dk, dv
   Params pk = p;
   pk.g1 = dv;
   pk.g2 = dk;
   pk.part1 = pl.nsplit > 1 ? reinterpret_cast<float*>(wsb + pl.partv_off) : nullptr;
   pk.part2 = pl.nsplit > 1 ? reinterpret_cast<float*>(wsb + pl.partk_off) : nullptr;
   pk.counters = reinterpret_cast<int*>(wsb) + 2;
-  bwd_kernel<true><<<grid, kThreads, smem, stream>>>(tk, tv, tq, tdo, pk);
-  if (pl.nsplit > 1) {
-    const dim3 sg(p.BH, kRows / 16);
-    bwd_sum_kernel<<<sg, 256, 0, stream>>>(pq.part1, dq, pl.nsplit, L, pl.nb, p.scale);
-    bwd_sum_kernel<<<sg, 256, 0, stream>>>(pk.part1, dv, pl.nsplit, L, pl.nb, 1.0f);
-    bwd_sum_kernel<<<sg, 256, 0, stream>>>(pk.part2, dk, pl.nsplit, L, pl.nb, p.scale);
-  }
-  const cudaError_t e = cudaGetLastError();
+  const int of32 = out_dtype == BB_OUT_F32 ? 1 : 0;
+  cudaError_t e;
+  if (d == 64)
+    e = pl.bt == 1 ? launch_bwd<64, 1>(tq, tk, tv, tdo, pq, pk, pl, sms, dout, out, of32, dd, rows, dq, dk, dv, L, stream)
+                   : launch_bwd<64, 2>(tq, tk, tv, tdo, pq, pk, pl, sms, dout, out, of32, dd, rows, dq, dk, dv, L, stream);
+  else
+    e = pl.bt == 1 ? launch_bwd<128, 1>(tq, tk, tv, tdo, pq, pk, pl, sms, dout, out, of32, dd, rows, dq, dk, dv, L, stream)
+                   : launch_bwd<128, 2>(tq, tk, tv, tdo, pq, pk, pl, sms, dout, out, of32, dd, rows, dq, dk, dv, L, stream);
   if (owned) cudaFreeAsync(ws, stream);
   return e == cudaSuccess ? BB_OK : BB_ERR_CUDA;
 }

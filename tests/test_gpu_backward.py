@@ -158,3 +158,43 @@ def test_backward_deterministic_and_long_transposed_lists():
     gq, gk, gv = oracle.attention_backward(inp["q"], inp["k"], inp["v"], ra, inp["seq_mask"], w.block, w.r, do)
     for name, got, want in (("dq", dq, gq), ("dk", dk, gk), ("dv", dv, gv)):
         _check_grad(name, got, want, w.name)
+
+
+OTHER_SIZES = [(128, 64), (64, 128), (128, 128)]  # (block, d)
+
+
+def _run_bd(inp, w, ra, dout):
+    q, k, v = (inp[x].cuda() for x in "qkv")
+    sm = None if inp["seq_mask"] is None else inp["seq_mask"].cuda()
+    ra_d = None if ra is None else torch.from_numpy(np.ascontiguousarray(ra)).cuda()
+    out, lse = bb.fwd_train(q, k, v, ra_d, sm, block=w.block, r=w.r, out_dtype=torch.float32)
+    grads = bb.bwd(q, k, v, out, dout.cuda(), lse, ra_d, sm, block=w.block, r=w.r)
+    torch.cuda.synchronize()
+    assert bb.device_status() == 0
+    return [t.double().cpu().numpy() for t in grads]
+
+
+@pytest.mark.parametrize("block,d", OTHER_SIZES, ids=[f"b{b}_d{d}" for b, d in OTHER_SIZES])
+def test_backward_other_sizes(block, d):
+    """Blocks of 128 (two 64-token tiles: the dk/dv kernel's units are single
+    key blocks) and d = 128 (two 64-column chunks; one CTA per SM): a padded
+    sparse case with split global rows and a full-attention case, against
+    the oracle, and a bit-exact second run."""
+    cases = [
+        Workload(f"bwd_sparse_b{block}_d{d}", 2, 2, 14 * block, d=d, block=block, value_scale=1.0,
+                 pad=("fixed", [14 * block - 70, 9 * block + 5]), seed=71 + d + block),
+        Workload(f"bwd_fallback_b{block}_d{d}", 1, 2, 8 * block, d=d, block=block, pad=("fixed", [8 * block - 3]),
+                 seed=72 + d + block),
+    ]
+    for w in cases:
+        inp = make_inputs(w)
+        ra = None if oracle.is_fallback(w.L, w.block, w.r) else bb.rand_attn_generate(w.H, w.L, w.block, w.r,
+                                                                                      seed=w.seed)
+        do = torch.randn(w.B, w.H, w.L, d, generator=torch.Generator().manual_seed(w.seed)).to(torch.bfloat16)
+        dq, dk, dv = _run_bd(inp, w, ra, do)
+        again = _run_bd(inp, w, ra, do)
+        for a, b in zip((dq, dk, dv), again):
+            assert np.array_equal(a, b)
+        gq, gk, gv = oracle.attention_backward(inp["q"], inp["k"], inp["v"], ra, inp["seq_mask"], w.block, w.r, do)
+        for name, got, want in (("dq", dq, gq), ("dk", dk, gk), ("dv", dv, gv)):
+            _check_grad(name, got, want, w.name)
