@@ -195,9 +195,12 @@ int bigbird_attn_fwd_train(const void* q, const void* k, const void* v, const in
  * D and the partial sums; bigbird_attn_bwd_workspace_size) is taken with
  * cudaMallocAsync on `stream`, its counters zeroed with cudaMemsetAsync, and
  * released with cudaFreeAsync; bigbird_attn_bwd_ex takes the caller's.
- * Asynchronous on `stream`. Errors as the forward (d != 64 or block != 64 ->
- * BB_ERR_UNSUPPORTED). Out-of-range rand_attn entries are skipped and flagged
- * in bigbird_device_status.
+ * Sizes: d 64 or 128, block 64 or 128 (a block of 128 is two 64-token tiles,
+ * d 128 two 64-column chunks; at d 128 one CTA per SM); other sizes, and full
+ * attention over more than 42 tiles (block 128 with r > 8), return
+ * BB_ERR_UNSUPPORTED. Asynchronous on `stream`. Other errors as the forward.
+ * Out-of-range rand_attn entries are skipped and flagged in
+ * bigbird_device_status.
  */
 int bigbird_attn_bwd(const void* q, const void* k, const void* v, const void* out, const void* dout,
                      const float* lse, const int32_t* rand_attn, const uint8_t* seq_mask, float* dq, float* dk,
@@ -208,8 +211,10 @@ int bigbird_attn_bwd(const void* q, const void* k, const void* v, const void* ou
  * Bytes of device workspace bigbird_attn_bwd_ex needs (0 for invalid or
  * unsupported sizes): 256 bytes of counters, D [B*H*L] fp32 (rounded up to
  * 256 bytes) and, when the global rows are split into key ranges (sparse
- * pattern, nb > 8), three partial-sum arrays [B*H, ceil(nb / 8), 128, 64]
- * fp32 (dq of the global query blocks, dv and dk of the global key blocks).
+ * pattern), three partial-sum arrays [B*H, n_glob * ceil(L / 512), 128, d]
+ * fp32 (dq of the global query blocks, dv and dk of the global key blocks;
+ * n_glob = 1 at block 64, where one unit holds both global blocks, 2 at
+ * block 128).
  */
 size_t bigbird_attn_bwd_workspace_size(int B, int H, int L, int d, int block, int r, unsigned flags);
 
