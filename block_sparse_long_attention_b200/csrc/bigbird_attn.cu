@@ -6,8 +6,8 @@
 //   * global units: query blocks 0 and nb-1 (or a pair of blocks in the
 //     full-attention fallback) against a contiguous range of key blocks; with
 //     more than one range per head the unit writes a partial (unnormalised
-//     output, running max, running sum) that a small merge kernel combines by
-//     log-sum-exp [TFG-BigBird, section "BigBird：从二次方注意力到线性稀疏注意力":
+//     output, running max, running sum) that the bf16 instance's grid
+//     (launched behind this one) combines by log-sum-exp [TFG-BigBird, section "BigBird：从二次方注意力到线性稀疏注意力":
 //     the first and last blocks attend to the whole K/V];
 //   * pair units: query blocks i and i+1 (1 <= i <= nb-2) against the union of
 //     their key blocks -- window, the two global blocks and their random blocks
@@ -109,7 +109,7 @@ constexpr uint32_t kBigExpField = 143u << 7;
 // out beyond gridDim.x, [1] CTAs finished, [2] set when a V value fp16 cannot
 // represent was seen (the bf16 instance then recomputes the call).
 constexpr size_t kCounterBytes = 256;
-constexpr int kCtrTickets = 0, kCtrDone = 1, kCtrBigV = 2;
+constexpr int kCtrTickets = 0, kCtrDone = 1, kCtrBigV = 2, kCtrParts = 3;
 
 // status word bits
 constexpr uint32_t kStatusBadRandAttn = 1u;
@@ -367,10 +367,16 @@ __device__ void prep_unit(const FwdParams& p, int u, UnitInfo& ui, int lane) {
 // ticket from a device-wide counter (units are numbered longest first), so
 // CTAs that run faster take more units and all finish together. Once the
 // tickets run out it publishes a stop slot, which ends every role's loop.
-template <int kD>
+template <int kD, bool kAllTickets>
 __device__ void prep_role(SharedStorage<kD>& s, const FwdParams& p, int bt) {
   const int lane = threadIdx.x & 31;
+  // kAllTickets: the first unit is a ticket too, so every unit is held by a
+  // CTA that is running (what the bf16 instance's wait before its merge needs)
   int u = blockIdx.x;
+  if (kAllTickets) {
+    if (lane == 0) u = atomicAdd(&p.counters[kCtrTickets], 1);
+    u = __shfl_sync(0xffffffffu, u, 0);
+  }
   for (uint32_t ut = 0;; ++ut) {
     const int slot = ut & 3;
     int ok = 1;
@@ -389,7 +395,7 @@ __device__ void prep_role(SharedStorage<kD>& s, const FwdParams& p, int bt) {
     }
     // Claim the next unit now, so the atomic's round trip overlaps this one's preparation.
     int next = 0;
-    if (lane == 0) next = static_cast<int>(gridDim.x) + atomicAdd(&p.counters[kCtrTickets], 1);
+    if (lane == 0) next = (kAllTickets ? 0 : static_cast<int>(gridDim.x)) + atomicAdd(&p.counters[kCtrTickets], 1);
     if (bt == 1) prep_unit<1>(p, u, ui, lane);
     else prep_unit<2>(p, u, ui, lane);
     if (lane == 0) mbar_arrive(smem_u32(&s.info_full[slot]));
@@ -825,6 +831,14 @@ __device__ void softmax_role(SharedStorage<kD>& s, const FwdParams& p, uint32_t 
                                __uint_as_float(o[4 * c + 3]));
       }
       reinterpret_cast<float2*>(p.part_ml)[base] = make_float2(m_ref, l_run);
+      if (kBf16) {
+        // the bf16 instance merges inside its own grid: count this warp's rows of the partial as written
+        __syncwarp();
+        if (lane == 0) {
+          __threadfence();
+          atomicAdd(&p.counters[kCtrParts], 1);
+        }
+      }
     } else if (exists) {
       const float inv = 1.f / l_run;
       const size_t row = static_cast<size_t>(bh) * p.L + static_cast<size_t>(qblk) * kBlock + (tid & 63);
@@ -844,9 +858,84 @@ __device__ void softmax_role(SharedStorage<kD>& s, const FwdParams& p, uint32_t 
   }
 }
 
+// Combine the partial results of the key ranges of the global rows by
+// log-sum-exp (log2 units) and write those rows' output and lse. Called by
+// every thread of a CTA; the grid's CTAs deal the rows out among themselves,
+// d / 4 threads per row (4 columns each), which take the row's ranges in
+// order, four at a time with their loads in flight together. The result does
+// not depend on which CTA merges a row.
+template <int kD>
+__device__ void merge_ranges(const FwdParams& p, int cta, int ncta) {
+  constexpr int kTpr = kD / 4;
+  constexpr int kRowsPerPass = kThreads / kTpr;
+  constexpr int kBatch = 4;
+  const int c4 = static_cast<int>(threadIdx.x) % kTpr;
+  const int total = p.BH * p.n_glob * kRows;
+  const float2* ml = reinterpret_cast<const float2*>(p.part_ml);
+#pragma unroll 1
+  for (int R = cta * kRowsPerPass + static_cast<int>(threadIdx.x) / kTpr; R < total; R += ncta * kRowsPerPass) {
+    const int unit = R / kRows;  // b * H * n_glob + global unit
+    const int row = R % kRows;
+    const size_t base = static_cast<size_t>(unit) * p.nsplit * kRows + row;
+    float m = kNegInit, l = 0.f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 1
+    for (int s0 = 0; s0 < p.nsplit; s0 += kBatch) {
+      float2 e[kBatch];
+      float4 o[kBatch];
+#pragma unroll
+      for (int i = 0; i < kBatch; ++i) {
+        if (s0 + i < p.nsplit) {
+          const size_t idx = base + static_cast<size_t>(s0 + i) * kRows;
+          e[i] = __ldcg(ml + idx);
+          o[i] = __ldcg(reinterpret_cast<const float4*>(p.part_o + idx * kD) + c4);
+        } else {
+          e[i] = make_float2(kNegInit, 0.f);
+          o[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+      }
+      float mb = m;
+#pragma unroll
+      for (int i = 0; i < kBatch; ++i) mb = fmaxf(mb, e[i].x);
+      const float f = ex2_approx(m - mb);
+      l *= f;
+      acc.x *= f;
+      acc.y *= f;
+      acc.z *= f;
+      acc.w *= f;
+#pragma unroll
+      for (int i = 0; i < kBatch; ++i) {
+        const float w = ex2_approx(e[i].x - mb);
+        l += w * e[i].y;
+        acc.x += w * o[i].x;
+        acc.y += w * o[i].y;
+        acc.z += w * o[i].z;
+        acc.w += w * o[i].w;
+      }
+      m = mb;
+    }
+    const int g = unit % p.n_glob;
+    const int bh = unit / p.n_glob;
+    const float inv = 1.f / l;
+    // rows 0..63 and 64..127 of the unit: tiles 0 and nt-1 (block 64: blocks 0
+    // and nb-1 stacked), or the two tiles of block 0 (g = 0) or of block nb-1
+    const int qtile = p.n_glob == 1 ? (row < kBlock ? 0 : p.nt - 1) : (g == 0 ? 0 : p.nt - 2) + row / kBlock;
+    const size_t orow = static_cast<size_t>(bh) * p.L + static_cast<size_t>(qtile) * kBlock + (row & (kBlock - 1));
+    if (p.lse && c4 == 0) p.lse[orow] = (m + log2f(l)) * 0.69314718055994531f;
+    if (p.out_f32) {
+      reinterpret_cast<float4*>(static_cast<float*>(p.out) + orow * kD)[c4] =
+          make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+    } else {
+      reinterpret_cast<uint2*>(static_cast<uint16_t*>(p.out) + orow * kD)[c4] =
+          make_uint2(pack_bf16x2(acc.x * inv, acc.y * inv), pack_bf16x2(acc.z * inv, acc.w * inv));
+    }
+  }
+}
+
 // kBf16 = false: the fp16 instance (every call). kBf16 = true: the bf16
-// instance, launched behind it as its programmatic dependent, which does the
-// call again only when the fp16 instance saw a V value fp16 cannot represent.
+// instance, launched behind it as its programmatic dependent, which merges the
+// fp16 instance's global-row ranges, or, when the fp16 instance saw a V value
+// fp16 cannot represent, does the whole call again and then merges its own.
 // kD: the head dimension (64 or 128).
 template <int kD, bool kBf16>
 __global__ void __launch_bounds__(kThreads, Geo<kD>::kCtasPerSm)
@@ -862,7 +951,12 @@ bigbird_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     // do the call again only if it set the flag.
     asm volatile("griddepcontrol.launch_dependents;");
     asm volatile("griddepcontrol.wait;" ::: "memory");
-    if (threadIdx.x == 0) s.abort_flag = *reinterpret_cast<volatile int*>(&p.counters[kCtrBigV]);
+    // Merge the fp16 instance's ranges at once (the flag's load overlaps the
+    // merge); when the flag is set the call is redone and merged again.
+    int big_v = 0;
+    if (threadIdx.x == 0) big_v = *reinterpret_cast<volatile int*>(&p.counters[kCtrBigV]);
+    if (p.nsplit > 1) merge_ranges<kD>(p, blockIdx.x, gridDim.x);
+    if (threadIdx.x == 0) s.abort_flag = big_v;
     __syncthreads();
     if (s.abort_flag == 0) return;
     __syncthreads();
@@ -915,7 +1009,7 @@ bigbird_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
   } else if (warp == 5) {
     if (lane == 0) mma_role<kD, kBf16>(s, p, tmem);
   } else if (warp == 6) {
-    prep_role<kD>(s, p, p.bt);
+    prep_role<kD, kBf16>(s, p, p.bt);
   } else {
     convert_role<kD, kBf16>(s, p);
   }
@@ -926,6 +1020,27 @@ bigbird_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     __syncwarp();
     tmem_dealloc(tmem, Geo<kD>::kTmemCols);
   }
+  if (kBf16 && p.nsplit > 1) {
+    // Every unit was claimed by ticket, so each is held by a running CTA: wait
+    // (bounded) until all partials of the recomputed ranges are written, then
+    // merge this CTA's share of the rows.
+    if (threadIdx.x == 0) {
+      const int want = 4 * p.BH * p.nparts;  // four softmax warps per range
+      const volatile int* cnt = &p.counters[kCtrParts];
+      const uint64_t t0 = globaltimer_ns();
+      while (*cnt < want) {
+        if ((*reinterpret_cast<volatile uint32_t*>(p.status) & kStatusTimeout) ||
+            globaltimer_ns() - t0 > kWaitTimeoutNs) {
+          atomicOr(p.status, kStatusTimeout);
+          break;
+        }
+        __nanosleep(256);
+      }
+      __threadfence();
+    }
+    __syncthreads();
+    merge_ranges<kD>(p, blockIdx.x, gridDim.x);
+  }
   // The CTA that finishes last puts the workspace counters back to zero for
   // the next call (every other CTA is done with them).
   // (The flag is left for the bf16 instance, which clears it when it runs.)
@@ -934,62 +1049,11 @@ bigbird_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     if (atomicAdd(&p.counters[kCtrDone], 1) == static_cast<int>(gridDim.x) - 1) {
       p.counters[kCtrTickets] = 0;
       p.counters[kCtrDone] = 0;
-      if (kBf16) p.counters[kCtrBigV] = 0;
+      if (kBf16) {
+        p.counters[kCtrBigV] = 0;
+        p.counters[kCtrParts] = 0;
+      }
     }
-  }
-}
-
-// Combine the partial results of the key ranges of the global rows by
-// log-sum-exp (log2 units). d / 4 threads per query row, 4 columns each; a
-// CTA of 256 threads covers 1024 / d rows of one global unit, grid =
-// (B*H*n_glob, 128 d / 1024).
-template <int kD>
-struct MergeGeo {
-  static constexpr int kThreadsPerRow = kD / 4;
-  static constexpr int kRowsPerCta = 256 / kThreadsPerRow;
-};
-
-template <int kD>
-__global__ void __launch_bounds__(256)
-bigbird_merge_kernel(const float* __restrict__ part_o, const float* __restrict__ part_ml, void* out, float* lse,
-                     int nsplit, int n_glob, int L, int nt, int out_f32) {
-  constexpr int kTpr = MergeGeo<kD>::kThreadsPerRow;
-  // Launched as a programmatic dependent of the attention kernel: wait until
-  // that grid has completed and its partials are visible.
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-  const int bh = blockIdx.x / n_glob;
-  const int g = blockIdx.x % n_glob;  // global unit: its partials follow those of unit g - 1
-  const int row = blockIdx.y * MergeGeo<kD>::kRowsPerCta + static_cast<int>(threadIdx.x) / kTpr;
-  const int c4 = static_cast<int>(threadIdx.x) % kTpr;
-  const size_t base = (static_cast<size_t>(bh) * n_glob + g) * nsplit * kRows + row;
-  const float2* ml = reinterpret_cast<const float2*>(part_ml);
-  float mmax = kNegInit;
-  for (int s = 0; s < nsplit; ++s) mmax = fmaxf(mmax, __ldg(&ml[base + static_cast<size_t>(s) * kRows].x));
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  float l = 0.f;
-  for (int s = 0; s < nsplit; ++s) {
-    const size_t idx = base + static_cast<size_t>(s) * kRows;
-    const float2 e = __ldg(&ml[idx]);
-    const float w = ex2_approx(e.x - mmax);
-    l += w * e.y;
-    const float4 t = __ldg(reinterpret_cast<const float4*>(part_o + idx * kD) + c4);
-    acc.x += w * t.x;
-    acc.y += w * t.y;
-    acc.z += w * t.z;
-    acc.w += w * t.w;
-  }
-  const float inv = 1.f / l;
-  // rows 0..63 and 64..127 of the unit: tiles 0 and nt-1 (block 64: blocks 0
-  // and nb-1 stacked), or the two tiles of block 0 (g = 0) or of block nb-1
-  const int qtile = n_glob == 1 ? (row < kBlock ? 0 : nt - 1) : (g == 0 ? 0 : nt - 2) + row / kBlock;
-  const size_t orow = static_cast<size_t>(bh) * L + static_cast<size_t>(qtile) * kBlock + (row & (kBlock - 1));
-  if (lse && c4 == 0) lse[orow] = (mmax + log2f(l)) * 0.69314718055994531f;
-  if (out_f32) {
-    reinterpret_cast<float4*>(static_cast<float*>(out) + orow * kD)[c4] =
-        make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
-  } else {
-    reinterpret_cast<uint2*>(static_cast<uint16_t*>(out) + orow * kD)[c4] =
-        make_uint2(pack_bf16x2(acc.x * inv, acc.y * inv), pack_bf16x2(acc.z * inv, acc.w * inv));
   }
 }
 
@@ -1136,15 +1200,13 @@ static int make_plan(int B, int H, int L, int d, int block, int r, unsigned flag
 }
 
 // The launches of one call at head dimension kD: the fp16 instance, then the
-// bf16 instance and (split global rows) the merge.
+// bf16 instance (which also merges split global rows) as its programmatic
+// dependent: launched while the fp16 grid runs, it waits
+// (griddepcontrol.wait) for that grid's completion before it reads what the
+// grid wrote, which hides the launch gap.
 template <int kD>
 static cudaError_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const FwdParams& p,
-                              const Plan& pl, int sms, void* out, int L, cudaStream_t stream) {
-  // The fp16 instance, then the bf16 instance and the merge, each a
-  // programmatic dependent of the kernel before it: launched while its
-  // predecessor runs, it waits (griddepcontrol.wait) for the predecessor's
-  // completion before it reads what that grid wrote, which hides the launch
-  // gaps.
+                              int sms, cudaStream_t stream) {
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
@@ -1161,18 +1223,6 @@ static cudaError_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, cons
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     e = cudaLaunchKernelEx(&cfg, bigbird_fwd_kernel<kD, true>, tq, tk, tv, p);
-  }
-  if (e == cudaSuccess && pl.nsplit > 1) {
-    cudaLaunchConfig_t cfg{};
-    cfg.gridDim = dim3(p.BH * p.n_glob, kRows / MergeGeo<kD>::kRowsPerCta);
-    cfg.blockDim = dim3(256);
-    cfg.dynamicSmemBytes = 0;
-    cfg.stream = stream;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, bigbird_merge_kernel<kD>, static_cast<const float*>(p.part_o),
-                           static_cast<const float*>(p.part_ml), out, p.lse, pl.nsplit, pl.n_glob, L, pl.nt,
-                           p.out_f32);
   }
   return e;
 }
@@ -1280,8 +1330,8 @@ static int fwd_impl(const void* q, const void* k, const void* v, const int32_t* 
     p.part_o = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + kCounterBytes);
     p.part_ml = p.part_o + static_cast<size_t>(p.BH) * p.nparts * kRows * d;
   }
-  const cudaError_t e = d == 64 ? launch_fwd<64>(tq, tk, tv, p, pl, di->sms, out, L, stream)
-                                : launch_fwd<128>(tq, tk, tv, p, pl, di->sms, out, L, stream);
+  const cudaError_t e = d == 64 ? launch_fwd<64>(tq, tk, tv, p, di->sms, stream)
+                                : launch_fwd<128>(tq, tk, tv, p, di->sms, stream);
   if (owned) cudaFreeAsync(ws, stream);
   return e == cudaSuccess ? BB_OK : BB_ERR_CUDA;
 }

@@ -90,9 +90,9 @@ enum {
  * shared memory); when V holds a value of magnitude >= 65536, which fp16
  * cannot represent, the call is done again with bf16 P and V (8 significant
  * bits of P instead of 11), which about doubles its time. A call launches the
- * fp16 kernel, then its bf16 instance (which returns at once unless that
- * recompute is needed) and, when the global rows are split into key ranges,
- * the merge of the ranges, each a programmatic dependent of the one before.
+ * fp16 kernel, then its bf16 instance as its programmatic dependent: that
+ * grid merges the key ranges of the split global rows (when the recompute is
+ * needed, after doing the call again) and otherwise returns at once.
  * The workspace (the work-unit counters and,
  * for split global rows, their partial results; see
  * bigbird_attn_workspace_size) is taken with cudaMallocAsync on `stream`,
@@ -115,7 +115,9 @@ int bigbird_attn_fwd(const void* q, const void* k, const void* v, const int32_t*
  * ranges of 8 tiles of 64 keys) each range's partial result follows, per
  * global unit (one unit holds both global blocks at block 64, one unit per
  * global block at block 128): output normalised by its own sum [128 rows, d],
- * running max and running sum, merged by log-sum-exp in a separate kernel.
+ * running max and running sum, merged by log-sum-exp by the bf16 instance.
+ * A fourth counter (the ranges the bf16 instance has redone) is used only on
+ * the recompute path and is zero between calls like the others.
  */
 size_t bigbird_attn_workspace_size(int B, int H, int L, int d, int block, int r, unsigned flags);
 

@@ -267,6 +267,40 @@ def test_v_beyond_fp16_range(vmax, out_dtype):
         assert (err[0, h, attends] <= bar).all(), (h, float((err[0, h, attends] / bar).max()))
 
 
+def test_v_beyond_fp16_range_many_ranges():
+    """The recompute path at L = 4096 with more work units than CTAs: eight key
+    ranges per global row, each redone by the bf16 instance, which waits until
+    every range is written and then merges them. Key block 0 (a global block,
+    attended by every row) holds V at 1e5, so every row carries that path's
+    error bar: |err| <= 1e-2 + 2^-7 * mass0 * max|v0| (mass0 = the row's weight
+    on block 0). Two calls give the same bits: the merge of a row does not
+    depend on which CTA does it. Heads (b 0, h 0) and (b 1, h 7) are checked
+    against the oracle, every head for finiteness."""
+    w = Workload("bigv_l4096", 2, 8, 4096, pad=("fixed", [4096, 3001]), seed=23)
+    inp = make_inputs(w)
+    ra_c, ra_o = _rand_attn_pair(w)
+    v = inp["v"].clone()
+    big = torch.randn(w.B, w.H, 64, 64, generator=torch.Generator().manual_seed(7))
+    v[:, :, :64] = (big / big.abs().max() * 1.0e5).to(torch.bfloat16)
+    inp = dict(inp, v=v)
+    got = _cuda_fwd(inp, w, ra_c, torch.float32)
+    again = _cuda_fwd(inp, w, ra_c, torch.float32)
+    assert np.isfinite(got).all()
+    assert np.array_equal(got, again)
+    vmax0 = float(v[:, :, :64].float().abs().max())
+    for b, h in [(0, 0), (1, 7)]:
+        sl = {x: inp[x][b:b + 1, h:h + 1] for x in "qk"}
+        vb = v[b:b + 1, h:h + 1]
+        sm = inp["seq_mask"][b:b + 1]
+        ra_h = ra_o[h:h + 1]
+        want = oracle.attention(sl["q"], sl["k"], vb, ra_h, sm, w.block, w.r)
+        ind = np.zeros(vb.shape, np.float64)
+        ind[:, :, :64] = 1.0
+        mass = oracle.attention(sl["q"], sl["k"], ind, ra_h, sm, w.block, w.r)[..., :1]
+        err = np.abs(got[b:b + 1, h:h + 1].astype(np.float64) - want)
+        assert (err <= 1e-2 + 2.0 ** -7 * mass * vmax0).all(), (b, h, float((err / (1e-2 + 2.0 ** -7 * mass * vmax0)).max()))
+
+
 def test_out_of_range_rand_attn_is_flagged():
     w = Workload("oor", 1, 1, 16 * 64, seed=18)
     inp = make_inputs(w)
