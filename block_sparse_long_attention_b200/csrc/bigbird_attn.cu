@@ -1,7 +1,7 @@
 // BigBird ITC block-sparse attention forward for B200 (sm_100a).
 //
-// One persistent, warp-specialised kernel processes "units" of 128 query rows
-// (two 64-row query blocks stacked, so every tensor-core MMA has M = 128):
+// Persistent, warp-specialised kernels process "units" of 128 query rows (two
+// 64-row query blocks stacked, so every tensor-core MMA has M = 128):
 //
 //   * global units: query blocks 0 and nb-1 (or a pair of blocks in the
 //     full-attention fallback) against a contiguous range of key blocks; with
@@ -20,40 +20,41 @@
 // block index, later ones are tickets from a counter in the workspace; the
 // CTA that finishes last sets the workspace counters back to zero.
 //
-// A unit's key blocks are processed one at a time through a serial chain:
-// S = Q K^T (tcgen05 SS-MMA, 128x64x16 steps) -> softmax -> fp16 P written
-// back over the S columns -> O += P V (TS-MMA, A = P from TMEM). Each CTA
-// needs only 128 TMEM columns, so four CTAs (four independent chains) share
-// an SM and interleave on its tensor pipe, exp unit and issue slots.
+// Per key block the chain is S = Q K^T (tcgen05 SS-MMA, 128x64x16 steps) ->
+// softmax -> fp16 P written back over the S columns it was read from -> O +=
+// P V (TS-MMA, A = P from TMEM). Two kernels run it:
 //
-// Warp roles (256 threads, 64 registers, four CTAs per SM):
-//   warps 0-3  softmax and epilogue, one query row per thread (thread t owns
-//              TMEM lane t);
-//   warp 4     TMA: Q per unit (one buffer, loaded once the previous unit's
-//              last S is done), K and V per block on 2-deep rings;
-//   warp 5     TMEM allocation and the tcgen05 MMAs (one thread);
-//   warp 6     scheduling and unit preparation (key-block list, half masks,
-//              key-validity bits) up to four units ahead, plus L2 prefetch,
-//              so its dependent global loads never stall the pipeline;
-//   warp 7     converts each V block bf16 -> fp16 in shared memory.
+//   * d = 64: bigbird_fwd2_kernel, two CTAs per SM, 384 threads (80
+//     registers). Each row's 64 keys per block are split between two softmax
+//     warps (keys 0..31 and 32..63), each with its own reference max, running
+//     sum and O accumulator (O_a, O_b), combined once per unit; S is
+//     double-buffered in TMEM (S0, S1, O_a, O_b: 256 columns), so S(g+1) is
+//     computed while the softmax works on block g. Warps 0-7 softmax and
+//     epilogue, 8 TMA (Q double-buffered, K and V on 2-deep rings released by
+//     the S and P.V completions themselves), 9 TMEM and the MMAs (one
+//     thread), 10 unit preparation, 11 V conversion.
+//   * d = 128: bigbird_fwd_kernel, two CTAs per SM, 256 threads, one softmax
+//     thread per row over the whole block, S [0,64) and O [64,192) in 256
+//     TMEM columns; the next S waits for the P.V that reads P (tcgen05 only
+//     orders MMAs that share an accumulator). Warps 0-3 softmax, 4 TMA, 5
+//     MMA, 6 unit preparation, 7 V conversion.
 //
-// TMEM (128 columns): S [0,64) fp32, with P (fp16, 32 columns) written over
-// [0,32) once read; O [64,128) fp32. The next S waits for the P.V that reads
-// P (tcgen05 only orders MMAs that share an accumulator).
+// The prep warp schedules and prepares units (key-block list, half masks,
+// key-validity bits) up to four units ahead, plus L2 prefetch, so its
+// dependent global loads never stall the pipeline.
 //
-// Softmax: one pass over each block's 64 columns, 16 at a time; the
-// reference max moves only when a score exceeds it by more than 2^14 (rare:
-// then the P pieces already written in the block are rescaled in TMEM, and O
-// once the previous P.V has landed; the final O / l is exact either way).
-// Padded keys get -10000 added to the scaled score. P.V runs in fp16: P is
-// written as fp16 and each V tile is converted bf16 -> fp16 in shared memory
-// (exact in the fp16 normal range), which keeps three more mantissa bits of P
-// than bf16. fp16 cannot represent a magnitude >= 65536: the converter flags
-// such a value (in the workspace) as it converts, and a second instance of
-// this kernel, launched behind the first as its programmatic dependent, then
-// recomputes the whole call with bf16 P and V as loaded (8 significant bits of
-// P), so every finite bf16 V is taken. Without the flag the second instance
-// returns at once.
+// Softmax: 16 columns at a time; the reference max moves only when a score
+// exceeds it by more than 2^14 (rare: then the P pieces already written in
+// the block are rescaled in TMEM, and O once the previous P.V has landed; the
+// final O / l is exact either way). Padded keys get -10000 added to the scaled
+// score. P.V runs in fp16: P is written as fp16 and each V tile is converted
+// bf16 -> fp16 in shared memory (exact in the fp16 normal range), which keeps
+// three more mantissa bits of P than bf16. fp16 cannot represent a magnitude
+// >= 65536: the converter flags such a value (in the workspace) as it
+// converts, and a second instance of the kernel, launched behind the first as
+// its programmatic dependent, then recomputes the whole call with bf16 P and
+// V as loaded (8 significant bits of P), so every finite bf16 V is taken.
+// Without the flag the second instance only merges the global rows' ranges.
 #include <cuda.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -162,14 +163,20 @@ struct FwdParams {
 
 template <int kD>
 struct __align__(1024) SharedStorage {
-  uint8_t q[kRows * kD * 2];                   // Q of the current unit (chunks of two 64x64 tiles, SW128)
+  static constexpr int kDim = kD;
+  static constexpr int kQBufs = 1;  // Q buffers (units whose Q is resident at once)
+  static constexpr int kKSt = kKStages;
+  static constexpr int kVSt = kVStages;
+  static constexpr int kSoftmaxWarps = 4;
+  static constexpr bool kFusedRelease = false;  // K/V stages released by their own barriers
+  uint8_t q[kQBufs][kRows * kD * 2];           // Q of the current unit (chunks of two 64x64 tiles, SW128)
   uint8_t k[kKStages][Geo<kD>::kTileBytes];    // K tiles
   uint8_t v[kVStages][Geo<kD>::kTileBytes];    // V tiles, converted to fp16 in place
   UnitInfo unit[4];
   uint64_t info_full[4];
   uint64_t info_empty[4];
-  uint64_t q_full;
-  uint64_t q_free;
+  uint64_t q_full[kQBufs];
+  uint64_t q_free[kQBufs];
   uint64_t k_full[kKStages];
   uint64_t k_empty[kKStages];
   uint64_t v_full[kVStages];
@@ -180,6 +187,53 @@ struct __align__(1024) SharedStorage {
   uint64_t pv_done;  // P.V of the current key block is complete (S/P columns reusable)
   uint64_t o_full;
   uint64_t o_free;
+  uint32_t tmem_base;
+  int32_t abort_flag;
+};
+
+// The d = 64 kernel with split rows (two CTAs per SM, 384 threads): each
+// query row's 64 keys per block are shared by two softmax warps (keys 0..31
+// and 32..63), each with its own reference max, running sum and O
+// accumulator, combined once per unit; S is double-buffered in TMEM so that
+// S(g+1) is computed while the softmax works on block g. TMEM columns (256):
+// S/P buffers at 0 and 64 (half h of a buffer at +32h, its fp16 P over the
+// first 16 of those columns), O of keys 0..31 at 128, of keys 32..63 at 192.
+constexpr int kThreads2 = 384;
+constexpr uint32_t kColOa = 128;
+constexpr uint32_t kColOb = 192;
+constexpr uint32_t kTmemCols2 = 256;
+
+struct __align__(1024) SharedStorage2 {
+  static constexpr int kDim = 64;
+  static constexpr int kQBufs = 2;  // the next unit's Q loads while this unit runs
+  // Two K and two V stages, as many as S buffers: a K stage is free again once
+  // the S that read it is complete (s_full), a V stage once its P.V is
+  // (pv_done), and the converter's arrival joins the softmax warps' on p_full,
+  // so the MMA thread waits and commits once per event.
+  static constexpr int kKSt = 2;
+  static constexpr int kVSt = 2;
+  static constexpr int kSoftmaxWarps = 8;
+  static constexpr bool kFusedRelease = true;
+  uint8_t q[kQBufs][kRows * 64 * 2];
+  uint8_t k[kKSt][kBlock * 64 * 2];
+  uint8_t v[kVSt][kBlock * 64 * 2];  // converted to fp16 in place
+  UnitInfo unit[4];
+  float2 mlx[2][2][kRows];  // (max, sum) per unit parity, column half, row: the halves' combine
+  uint64_t info_full[4];
+  uint64_t info_empty[4];
+  uint64_t q_full[kQBufs];
+  uint64_t q_free[kQBufs];
+  uint64_t k_full[kKSt];
+  uint64_t k_empty[kKSt];
+  uint64_t v_full[kVSt];
+  uint64_t v_conv[kVSt];
+  uint64_t v_empty[kVSt];
+  uint64_t s_full[2];   // S(g) is in buffer g & 1
+  uint64_t p_full[2];   // all eight softmax warps have written P(g) into buffer g & 1
+  uint64_t pv_done[2];  // P.V(g) is complete (buffer g & 1 reusable)
+  uint64_t o_full;
+  uint64_t o_free;
+  uint64_t ml_ready;    // both halves' (max, sum) of the unit are in mlx
   uint32_t tmem_base;
   int32_t abort_flag;
 };
@@ -367,8 +421,9 @@ __device__ void prep_unit(const FwdParams& p, int u, UnitInfo& ui, int lane) {
 // ticket from a device-wide counter (units are numbered longest first), so
 // CTAs that run faster take more units and all finish together. Once the
 // tickets run out it publishes a stop slot, which ends every role's loop.
-template <int kD, bool kAllTickets>
-__device__ void prep_role(SharedStorage<kD>& s, const FwdParams& p, int bt) {
+template <class S, bool kAllTickets>
+__device__ void prep_role(S& s, const FwdParams& p, int bt) {
+  constexpr int kD = S::kDim;
   const int lane = threadIdx.x & 31;
   // kAllTickets: the first unit is a ticket too, so every unit is held by a
   // CTA that is running (what the bf16 instance's wait before its merge needs)
@@ -422,17 +477,24 @@ __device__ void prep_role(SharedStorage<kD>& s, const FwdParams& p, int bt) {
 // cannot represent, sets the workspace flag that makes the bf16 instance
 // recompute the call. The bf16 instance converts nothing: this warp only
 // keeps the unit bookkeeping.
-template <int kD, bool kBf16>
-__device__ void convert_role(SharedStorage<kD>& s, const FwdParams& p) {
+template <class S, bool kBf16>
+__device__ void convert_role(S& s, const FwdParams& p) {
+  constexpr int kD = S::kDim;
   const int lane = threadIdx.x & 31;
   uint32_t gv = 0;
   for (uint32_t ut = 0;; ++ut) {
     if (!warp_wait(smem_u32(&s.info_full[ut & 3]), (ut >> 2) & 1)) { if (lane == 0) flag_timeout(s, p); return; }
     if (s.unit[ut & 3].stop) break;
     const int n = s.unit[ut & 3].n;
-    for (int e = 0; e < n && !kBf16; ++e, ++gv) {
-      const int st = gv % kVStages;
-      if (!warp_wait(smem_u32(&s.v_full[st]), (gv / kVStages) & 1)) { if (lane == 0) flag_timeout(s, p); return; }
+    for (int e = 0; e < n && (!kBf16 || S::kFusedRelease); ++e, ++gv) {
+      const int st = gv % S::kVSt;
+      if (!warp_wait(smem_u32(&s.v_full[st]), (gv / S::kVSt) & 1)) { if (lane == 0) flag_timeout(s, p); return; }
+      if (kBf16) {  // nothing to convert: only the arrival on p_full
+        __syncwarp();
+        if constexpr (S::kFusedRelease)
+          if (lane == 0) mbar_arrive(smem_u32(&s.p_full[gv & 1]));
+        continue;
+      }
       uint4* vp = reinterpret_cast<uint4*>(s.v[st]) + lane;
       uint32_t ex = 0;  // largest bf16 exponent field seen, per 16-bit half
 #pragma unroll 4
@@ -452,7 +514,11 @@ __device__ void convert_role(SharedStorage<kD>& s, const FwdParams& p) {
       if (__any_sync(0xffffffffu, max(ex & 0xFFFFu, ex >> 16) >= kBigExpField) && lane == 0)
         atomicExch(&p.counters[kCtrBigV], 1);
       __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&s.v_conv[st]));
+      if constexpr (S::kFusedRelease) {
+        if (lane == 0) mbar_arrive(smem_u32(&s.p_full[gv & 1]));
+      } else {
+        if (lane == 0) mbar_arrive(smem_u32(&s.v_conv[st]));
+      }
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(smem_u32(&s.info_empty[ut & 3]));
@@ -464,9 +530,10 @@ __device__ void convert_role(SharedStorage<kD>& s, const FwdParams& p) {
 // the unit (single Q buffer: after every S of the previous unit is done).
 // Loads every chunk of a tile: K and V tiles are 64 rows x d, stored chunk by
 // chunk (x = 64 c of the tensor map, 8 KB apart).
-template <int kD>
-__device__ void producer_role(SharedStorage<kD>& s, const FwdParams& p, const CUtensorMap* tmQ, const CUtensorMap* tmK,
+template <class S>
+__device__ void producer_role(S& s, const FwdParams& p, const CUtensorMap* tmQ, const CUtensorMap* tmK,
                               const CUtensorMap* tmV) {
+  constexpr int kD = S::kDim;
   const int lane = threadIdx.x & 31;
   const uint64_t pol_kv = l2_policy_evict_last();
   const uint64_t pol_q = l2_policy_evict_first();
@@ -480,8 +547,13 @@ __device__ void producer_role(SharedStorage<kD>& s, const FwdParams& p, const CU
       const UnitInfo& ui = s.unit[vut & 3];
       int ok = 1;
       if (lane == 0) {
-        const int st = gv % kVStages;
-        ok = mbar_wait(smem_u32(&s.v_empty[st]), ((gv / kVStages) & 1) ^ 1);
+        const int st = gv % S::kVSt;
+        if constexpr (S::kFusedRelease) {
+          // the stage's previous tile (block gv - 2) is free once its P.V is complete
+          ok = gv < 2 || mbar_wait(smem_u32(&s.pv_done[st]), ((gv >> 1) - 1) & 1);
+        } else {
+          ok = mbar_wait(smem_u32(&s.v_empty[st]), ((gv / S::kVSt) & 1) ^ 1);
+        }
         if (ok) {
           const uint32_t vbar = smem_u32(&s.v_full[st]);
           mbar_arrive_expect_tx(vbar, Geo<kD>::kTileBytes);
@@ -519,22 +591,28 @@ __device__ void producer_role(SharedStorage<kD>& s, const FwdParams& p, const CU
       const int32_t row0 = ui.bh * p.L;
       if (lane == 0) {
         if (ke == 0) {
-          ok = mbar_wait(smem_u32(&s.q_free), (kut & 1) ^ 1);
+          const int qb = kut % S::kQBufs;
+          ok = mbar_wait(smem_u32(&s.q_free[qb]), ((kut / S::kQBufs) & 1) ^ 1);
           if (ok) {
-            const uint32_t qbar = smem_u32(&s.q_full);
+            const uint32_t qbar = smem_u32(&s.q_full[qb]);
             mbar_arrive_expect_tx(qbar, (ui.qbot >= 0 ? 2 : 1) * Geo<kD>::kTileBytes);
 #pragma unroll
             for (int c = 0; c < Geo<kD>::kChunks; ++c) {
               // chunk c of the unit's 128 rows: the top tile, then the bottom one
-              const uint32_t qdst = smem_u32(s.q) + c * Geo<kD>::kQChunkBytes;
+              const uint32_t qdst = smem_u32(s.q[qb]) + c * Geo<kD>::kQChunkBytes;
               tma_load_2d(qdst, tmQ, qbar, 64 * c, row0 + ui.qtop * kBlock, pol_q);
               if (ui.qbot >= 0) tma_load_2d(qdst + kChunkBytes, tmQ, qbar, 64 * c, row0 + ui.qbot * kBlock, pol_q);
             }
           }
         }
         if (ok) {
-          const int st = gk % kKStages;
-          ok = mbar_wait(smem_u32(&s.k_empty[st]), ((gk / kKStages) & 1) ^ 1);
+          const int st = gk % S::kKSt;
+          if constexpr (S::kFusedRelease) {
+            // the stage's previous tile (block gk - 2) is free once its S is complete
+            ok = gk < 2 || mbar_wait(smem_u32(&s.s_full[st]), ((gk >> 1) - 1) & 1);
+          } else {
+            ok = mbar_wait(smem_u32(&s.k_empty[st]), ((gk / S::kKSt) & 1) ^ 1);
+          }
           if (ok) {
             const uint32_t kbar = smem_u32(&s.k_full[st]);
             mbar_arrive_expect_tx(kbar, Geo<kD>::kTileBytes);
@@ -568,13 +646,13 @@ __device__ void mma_role(SharedStorage<kD>& s, const FwdParams& p, uint32_t tmem
   const uint32_t idesc_s = idesc_f32acc(kRows, kBlock, true, false);    // bf16 Q . K^T, N = 64
   // fp16 P . fp16 V, or bf16 P . bf16 V in the bf16 instance; N = 64 per chunk of d
   const uint32_t idesc_o = idesc_f32acc(kRows, 64, kBf16, true);
-  const uint32_t q_addr = smem_u32(s.q);
+  const uint32_t q_addr = smem_u32(s.q[0]);
   uint32_t g = 0;
   bool ok = true;
   for (uint32_t ut = 0; ok; ++ut) {
     if (!mbar_wait(smem_u32(&s.info_full[ut & 3]), (ut >> 2) & 1)) { ok = false; break; }
     if (s.unit[ut & 3].stop) break;
-    if (!mbar_wait(smem_u32(&s.q_full), ut & 1)) { ok = false; break; }
+    if (!mbar_wait(smem_u32(&s.q_full[0]), ut & 1)) { ok = false; break; }
     const int n = s.unit[ut & 3].n;
     for (int e = 0; e < n; ++e, ++g) {
       const int kst = g % kKStages;
@@ -589,7 +667,7 @@ __device__ void mma_role(SharedStorage<kD>& s, const FwdParams& p, uint32_t tmem
                sdesc_sw128(k_addr + (kk >> 2) * kChunkBytes + (kk & 3) * 32, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
       mma_commit(smem_u32(&s.s_full));
       mma_commit(smem_u32(&s.k_empty[kst]));
-      if (e == n - 1) mma_commit(smem_u32(&s.q_free));
+      if (e == n - 1) mma_commit(smem_u32(&s.q_free[0]));
       const int vst = g % kVStages;
       // the V tile: converted (fp16), or as loaded (bf16 instance)
       if (!mbar_wait(smem_u32(kBf16 ? &s.v_full[vst] : &s.v_conv[vst]), (g / kVStages) & 1)) { ok = false; break; }
@@ -858,16 +936,239 @@ __device__ void softmax_role(SharedStorage<kD>& s, const FwdParams& p, uint32_t 
   }
 }
 
+// ---------------------------------------------------------------- split-row kernel (d = 64)
+
+// Per key block g of this CTA: S(g) = Q . K(g)^T into S buffer g & 1 once
+// P.V(g - 2), which read the P held there, has completed; then P.V(g - 1),
+// once all eight softmax warps have written P(g - 1) and the converter has
+// converted V(g - 1) (both arrive on p_full): keys 0..31 into O_a,
+// keys 32..63 into O_b. S(g) goes out before P.V(g - 1), so that it is ready
+// when the softmax finishes block g - 1.
+template <bool kBf16>
+__device__ void mma2_role(SharedStorage2& s, const FwdParams& p, uint32_t tmem) {
+  constexpr int kK = SharedStorage2::kKSt;
+  constexpr int kV = SharedStorage2::kVSt;
+  const uint32_t idesc_s = idesc_f32acc(kRows, kBlock, true, false);  // bf16 Q . K^T, N = 64
+  const uint32_t idesc_o = idesc_f32acc(kRows, 64, kBf16, true);      // fp16 (or bf16) P . V, N = 64
+  // P.V of block gb: first / last block of its unit, the unit's index
+  auto issue_pv = [&](uint32_t gb, bool first, bool last, uint32_t put) -> bool {
+    const int vst = gb % kV;
+    if (first && !mbar_wait(smem_u32(&s.o_free), (put & 1) ^ 1)) return false;
+    if (!mbar_wait(smem_u32(&s.p_full[gb & 1]), (gb >> 1) & 1)) return false;
+    tc_fence_after();
+    const uint32_t v_addr = smem_u32(s.v[vst]);
+    const uint32_t pb = tmem + 64 * (gb & 1);
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+      for (int kk = 0; kk < 2; ++kk)  // keys 32h + 16kk .. +15: P columns 32h + 8kk, V rows 2048 bytes apart
+        mma_ts(tmem + kColOa + 64 * h, pb + 32 * h + 8 * kk, sdesc_sw128(v_addr + (2 * h + kk) * 2048, 8192, 1024),
+               idesc_o, (!first || kk > 0) ? 1u : 0u);
+    mma_commit(smem_u32(&s.pv_done[gb & 1]));
+    if (last) mma_commit(smem_u32(&s.o_full));
+    return true;
+  };
+  uint32_t g = 0;
+  bool pend = false, pend_first = false, pend_last = false;
+  uint32_t pend_ut = 0;
+  bool ok = true;
+  for (uint32_t ut = 0; ok; ++ut) {
+    if (!mbar_wait(smem_u32(&s.info_full[ut & 3]), (ut >> 2) & 1)) { ok = false; break; }
+    if (s.unit[ut & 3].stop) break;
+    const int qb = ut & 1;
+    if (!mbar_wait(smem_u32(&s.q_full[qb]), (ut >> 1) & 1)) { ok = false; break; }
+    const uint32_t q_addr = smem_u32(s.q[qb]);
+    const int n = s.unit[ut & 3].n;
+    for (int e = 0; e < n; ++e, ++g) {
+      const int kst = g % kK;
+      if (!mbar_wait(smem_u32(&s.k_full[kst]), (g / kK) & 1)) { ok = false; break; }
+      if (g >= 2 && !mbar_wait(smem_u32(&s.pv_done[g & 1]), ((g >> 1) - 1) & 1)) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t k_addr = smem_u32(s.k[kst]);
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk)
+        mma_ss(tmem + 64 * (g & 1), sdesc_sw128(q_addr + kk * 32, 16, 1024), sdesc_sw128(k_addr + kk * 32, 16, 1024),
+               idesc_s, kk > 0 ? 1u : 0u);
+      mma_commit(smem_u32(&s.s_full[g & 1]));
+      if (e == n - 1) mma_commit(smem_u32(&s.q_free[qb]));
+      if (pend && !issue_pv(g - 1, pend_first, pend_last, pend_ut)) { ok = false; break; }
+      pend = true;
+      pend_first = e == 0;
+      pend_last = e == n - 1;
+      pend_ut = ut;
+    }
+    if (!ok) break;
+    mbar_arrive(smem_u32(&s.info_empty[ut & 3]));
+  }
+  if (ok && pend && !issue_pv(g - 1, pend_first, pend_last, pend_ut)) ok = false;
+  if (!ok) flag_timeout(s, p);
+}
+
+// Warps 0..7: warp w takes rows 32 (w % 4) .. + 31 (its TMEM lanes) and keys
+// 32 (w / 4) .. + 31 of every block: one pass over those 32 S columns, 16 at a
+// time (max, a change of its own reference max when a score exceeds it by
+// more than 2^14, exponentials, fp16 P written over the columns already
+// read), then the block goes to the MMA. At the end of a unit the two halves
+// of a row exchange (max, sum) through shared memory; each writes 32 of the
+// row's output columns, O_a and O_b scaled to the common max.
+template <bool kBf16>
+__device__ void softmax2_role(SharedStorage2& s, const FwdParams& p, uint32_t tmem) {
+  const int wid = threadIdx.x >> 5;  // 0..7
+  const int h = wid >> 2;            // key half of each block
+  const int row = threadIdx.x & 127; // TMEM lane == row of the unit
+  const int lane = threadIdx.x & 31;
+  const int rhalf = (wid & 3) >> 1;  // 0: rows 0..63, 1: rows 64..127
+  const uint32_t lane_addr = tmem + (static_cast<uint32_t>((wid & 3) * 32) << 16);
+  const uint64_t scale2 = f2_pack(p.scale_log2, p.scale_log2);
+  uint32_t g = 0;
+  for (uint32_t ut = 0;; ++ut) {
+    if (!warp_wait(smem_u32(&s.info_full[ut & 3]), (ut >> 2) & 1)) { flag_timeout(s, p); return; }
+    const UnitInfo& ui = s.unit[ut & 3];
+    if (ui.stop) break;
+    const int n = ui.n;
+    const int bh = ui.bh;
+    const int qblk = rhalf ? ui.qbot : ui.qtop;
+    const int split = ui.split;
+    const bool exists = qblk >= 0;
+    float m_ref = kNegInit;
+    float l_run = 0.f;
+    for (int e = 0; e < n; ++e, ++g) {
+      const bool used = exists && ((ui.hm[e] >> rhalf) & 1);
+      if (!warp_wait(smem_u32(&s.s_full[g & 1]), (g >> 1) & 1)) { flag_timeout(s, p); return; }
+      tc_fence_after();
+      const uint32_t s_addr = lane_addr + 64 * (g & 1) + 32 * h;
+      if (used) {
+        const uint32_t vm = static_cast<uint32_t>(ui.vm[e] >> (32 * h));
+        const bool mixed = vm != 0xFFFFFFFFu && vm != 0u;
+        const float off_s = (vm == 0u ? p.bias_raw : 0.f) * p.scale_log2;
+        float o_factor = 1.f;  // rescale owed to O (the P.V of the earlier blocks)
+        uint64_t acc0 = 0ull, acc1 = 0ull;
+        uint32_t r0[16], r1[16];
+        tmem_ld16(s_addr, r0);
+        tmem_wait_ld();
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          uint32_t (&cur)[16] = q ? r1 : r0;
+          if (q == 0) tmem_ld16(s_addr + 16, r1);
+          const float mx =
+              fmaf(piece16_prepare(cur, mixed, (vm >> (16 * q)) & 0xFFFFu, p.bias_raw), p.scale_log2, off_s);
+          const bool need = mx > m_ref + kRescaleThreshold;
+          if (__any_sync(0xffffffffu, need)) {
+            float f = 1.f;
+            if (need) {
+              f = ex2_approx(m_ref - mx);
+              m_ref = mx;
+            }
+            l_run *= f;
+            const uint64_t f2 = f2_pack(f, f);
+            acc0 = f2_fma(acc0, f2, 0ull);
+            acc1 = f2_fma(acc1, f2, 0ull);
+            o_factor *= f;
+            if (q > 0 && __any_sync(0xffffffffu, f != 1.f)) rescale_p<kBf16>(s_addr, q, f);
+          }
+          const float o = off_s - m_ref;
+          uint32_t pk[8];
+          piece16_exp<kBf16>(cur, scale2, f2_pack(o, o), pk, acc0, acc1);
+          if (q == 0) tmem_wait_ld();
+          tmem_st8(s_addr + 8 * q, pk);
+        }
+        float a0, a1, b0, b1;
+        f2_unpack(acc0, a0, a1);
+        f2_unpack(acc1, b0, b1);
+        l_run += (a0 + a1) + (b0 + b1);
+        // this half's O holds the P.V of the earlier blocks (none yet for e == 0);
+        // rescale it once that P.V is done
+        if (e > 0 && __any_sync(0xffffffffu, o_factor != 1.f)) {
+          if (!warp_wait(smem_u32(&s.pv_done[(g - 1) & 1]), ((g - 1) >> 1) & 1)) { flag_timeout(s, p); return; }
+          tc_fence_after();
+          rescale_o<64>(lane_addr + kColOa + 64 * h, o_factor);
+        }
+      } else {
+        // No row of this warp uses the block: P = 0.
+        uint32_t z[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) z[i] = 0u;
+        tmem_st16(s_addr, z);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&s.p_full[g & 1]));
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(smem_u32(&s.info_empty[ut & 3]));
+
+    // ---- epilogue: combine the halves, each writes 32 columns of its row
+    if (!warp_wait(smem_u32(&s.o_full), ut & 1)) { flag_timeout(s, p); return; }
+    tc_fence_after();
+    s.mlx[ut & 1][h][row] = make_float2(m_ref, l_run);
+    __syncwarp();
+    if (lane == 0) mbar_arrive(smem_u32(&s.ml_ready));
+    if (!warp_wait(smem_u32(&s.ml_ready), ut & 1)) { flag_timeout(s, p); return; }
+    const float2 A = s.mlx[ut & 1][0][row];
+    const float2 B = s.mlx[ut & 1][1][row];
+    const float m = fmaxf(A.x, B.x);
+    const float fa = ex2_approx(A.x - m);
+    const float fb = ex2_approx(B.x - m);
+    const float l = A.y * fa + B.y * fb;
+    const int c_base = 32 * h;
+    if (split >= 0) {
+      const size_t base = (static_cast<size_t>(bh) * p.nparts + split) * kRows + row;
+#pragma unroll 1
+      for (int c0 = 0; c0 < 32; c0 += 16) {
+        uint32_t oa[16], ob[16];
+        tmem_ld16(lane_addr + kColOa + c_base + c0, oa);
+        tmem_ld16(lane_addr + kColOb + c_base + c0, ob);
+        tmem_wait_ld();
+        float4* dst = reinterpret_cast<float4*>(p.part_o + base * 64 + c_base + c0);
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          dst[c] = make_float4(__uint_as_float(oa[4 * c]) * fa + __uint_as_float(ob[4 * c]) * fb,
+                               __uint_as_float(oa[4 * c + 1]) * fa + __uint_as_float(ob[4 * c + 1]) * fb,
+                               __uint_as_float(oa[4 * c + 2]) * fa + __uint_as_float(ob[4 * c + 2]) * fb,
+                               __uint_as_float(oa[4 * c + 3]) * fa + __uint_as_float(ob[4 * c + 3]) * fb);
+      }
+      if (h == 0) reinterpret_cast<float2*>(p.part_ml)[base] = make_float2(m, l);
+      if (kBf16) {
+        // the bf16 instance merges inside its own grid: count this warp's rows of the partial as written
+        __syncwarp();
+        if (lane == 0) {
+          __threadfence();
+          atomicAdd(&p.counters[kCtrParts], 1);
+        }
+      }
+    } else if (exists) {
+      const float inv = 1.f / l;
+      const size_t orow = static_cast<size_t>(bh) * p.L + static_cast<size_t>(qblk) * kBlock + (row & 63);
+      // log sum_k exp(s_k) = ln 2 * (m + log2 l), the scores in log2 units being s * log2(e).
+      if (h == 0 && p.lse) p.lse[orow] = (m + log2f(l)) * 0.69314718055994531f;
+#pragma unroll 1
+      for (int c0 = 0; c0 < 32; c0 += 16) {
+        uint32_t oa[16], ob[16];
+        tmem_ld16(lane_addr + kColOa + c_base + c0, oa);
+        tmem_ld16(lane_addr + kColOb + c_base + c0, ob);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) oa[i] = __float_as_uint(__uint_as_float(oa[i]) * fa + __uint_as_float(ob[i]) * fb);
+        store16<64>(p, orow, c_base + c0, oa, inv);
+      }
+    }
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(smem_u32(&s.o_free));
+  }
+}
+
 // Combine the partial results of the key ranges of the global rows by
 // log-sum-exp (log2 units) and write those rows' output and lse. Called by
 // every thread of a CTA; the grid's CTAs deal the rows out among themselves,
 // d / 4 threads per row (4 columns each), which take the row's ranges in
 // order, four at a time with their loads in flight together. The result does
 // not depend on which CTA merges a row.
-template <int kD>
+template <int kD, int kNT>
 __device__ void merge_ranges(const FwdParams& p, int cta, int ncta) {
   constexpr int kTpr = kD / 4;
-  constexpr int kRowsPerPass = kThreads / kTpr;
+  constexpr int kRowsPerPass = kNT / kTpr;
   constexpr int kBatch = 4;
   const int c4 = static_cast<int>(threadIdx.x) % kTpr;
   const int total = p.BH * p.n_glob * kRows;
@@ -955,7 +1256,7 @@ bigbird_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     // merge); when the flag is set the call is redone and merged again.
     int big_v = 0;
     if (threadIdx.x == 0) big_v = *reinterpret_cast<volatile int*>(&p.counters[kCtrBigV]);
-    if (p.nsplit > 1) merge_ranges<kD>(p, blockIdx.x, gridDim.x);
+    if (p.nsplit > 1) merge_ranges<kD, kThreads>(p, blockIdx.x, gridDim.x);
     if (threadIdx.x == 0) s.abort_flag = big_v;
     __syncthreads();
     if (s.abort_flag == 0) return;
@@ -970,8 +1271,8 @@ bigbird_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       mbar_init(smem_u32(&s.info_full[i]), 1);
       mbar_init(smem_u32(&s.info_empty[i]), 1 + 1 + 4 + 1);  // TMA, MMA, 4 softmax warps, converter
     }
-    mbar_init(smem_u32(&s.q_full), 1);
-    mbar_init(smem_u32(&s.q_free), 1);
+    mbar_init(smem_u32(&s.q_full[0]), 1);
+    mbar_init(smem_u32(&s.q_free[0]), 1);
     for (int i = 0; i < kKStages; ++i) {
       mbar_init(smem_u32(&s.k_full[i]), 1);
       mbar_init(smem_u32(&s.k_empty[i]), 1);
@@ -1005,13 +1306,13 @@ bigbird_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
   if (warp < 4) {
     softmax_role<kD, kBf16>(s, p, tmem);
   } else if (warp == 4) {
-    producer_role<kD>(s, p, &tmQ, &tmK, &tmV);
+    producer_role(s, p, &tmQ, &tmK, &tmV);
   } else if (warp == 5) {
     if (lane == 0) mma_role<kD, kBf16>(s, p, tmem);
   } else if (warp == 6) {
-    prep_role<kD, kBf16>(s, p, p.bt);
+    prep_role<SharedStorage<kD>, kBf16>(s, p, p.bt);
   } else {
-    convert_role<kD, kBf16>(s, p);
+    convert_role<SharedStorage<kD>, kBf16>(s, p);
   }
   tc_fence_before();
   __syncthreads();
@@ -1025,7 +1326,7 @@ bigbird_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     // (bounded) until all partials of the recomputed ranges are written, then
     // merge this CTA's share of the rows.
     if (threadIdx.x == 0) {
-      const int want = 4 * p.BH * p.nparts;  // four softmax warps per range
+      const int want = SharedStorage<kD>::kSoftmaxWarps * p.BH * p.nparts;  // each softmax warp counts its rows
       const volatile int* cnt = &p.counters[kCtrParts];
       const uint64_t t0 = globaltimer_ns();
       while (*cnt < want) {
@@ -1039,11 +1340,138 @@ bigbird_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       __threadfence();
     }
     __syncthreads();
-    merge_ranges<kD>(p, blockIdx.x, gridDim.x);
+    merge_ranges<kD, kThreads>(p, blockIdx.x, gridDim.x);
   }
   // The CTA that finishes last puts the workspace counters back to zero for
   // the next call (every other CTA is done with them).
   // (The flag is left for the bf16 instance, which clears it when it runs.)
+  if (threadIdx.x == 0) {
+    __threadfence();
+    if (atomicAdd(&p.counters[kCtrDone], 1) == static_cast<int>(gridDim.x) - 1) {
+      p.counters[kCtrTickets] = 0;
+      p.counters[kCtrDone] = 0;
+      if (kBf16) {
+        p.counters[kCtrBigV] = 0;
+        p.counters[kCtrParts] = 0;
+      }
+    }
+  }
+}
+
+// The split-row kernel at d = 64 (fp16 instance, or the bf16 instance with
+// the merge of the global rows' ranges): the same units, scheduling, workspace
+// and bf16 recompute as bigbird_fwd_kernel, with 12 warps -- 0..7 softmax
+// (two per row), 8 TMA, 9 MMA (and TMEM), 10 unit preparation, 11 V
+// conversion -- and two CTAs per SM.
+template <bool kBf16>
+__global__ void __launch_bounds__(kThreads2, 2)
+bigbird_fwd2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                    const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  SharedStorage2& s =
+      *reinterpret_cast<SharedStorage2*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  if (kBf16) {
+    // Merge the fp16 instance's ranges at once (the flag's load overlaps the
+    // merge); when the flag is set the call is redone and merged again.
+    asm volatile("griddepcontrol.launch_dependents;");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    int big_v = 0;
+    if (threadIdx.x == 0) big_v = *reinterpret_cast<volatile int*>(&p.counters[kCtrBigV]);
+    if (p.nsplit > 1) merge_ranges<64, kThreads2>(p, blockIdx.x, gridDim.x);
+    if (threadIdx.x == 0) s.abort_flag = big_v;
+    __syncthreads();
+    if (s.abort_flag == 0) return;
+    __syncthreads();
+  }
+  if (warp == 9) {
+    tmem_alloc(smem_u32(&s.tmem_base), kTmemCols2);
+    tmem_relinquish();
+  }
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 4; ++i) {
+      mbar_init(smem_u32(&s.info_full[i]), 1);
+      mbar_init(smem_u32(&s.info_empty[i]), 1 + 1 + 8 + 1);  // TMA, MMA, 8 softmax warps, converter
+    }
+    for (int i = 0; i < SharedStorage2::kQBufs; ++i) {
+      mbar_init(smem_u32(&s.q_full[i]), 1);
+      mbar_init(smem_u32(&s.q_free[i]), 1);
+    }
+    for (int i = 0; i < SharedStorage2::kKSt; ++i) {
+      mbar_init(smem_u32(&s.k_full[i]), 1);
+      mbar_init(smem_u32(&s.k_empty[i]), 1);
+    }
+    for (int i = 0; i < SharedStorage2::kVSt; ++i) {
+      mbar_init(smem_u32(&s.v_full[i]), 1);
+      mbar_init(smem_u32(&s.v_conv[i]), 1);
+      mbar_init(smem_u32(&s.v_empty[i]), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(&s.s_full[i]), 1);
+      mbar_init(smem_u32(&s.p_full[i]), 8 + 1);  // eight softmax warps and the converter
+      mbar_init(smem_u32(&s.pv_done[i]), 1);
+    }
+    mbar_init(smem_u32(&s.o_full), 1);
+    mbar_init(smem_u32(&s.o_free), 8);
+    mbar_init(smem_u32(&s.ml_ready), 8);
+    s.abort_flag = 0;
+    fence_barrier_init();
+  }
+  // The dependent grid (the bf16 instance) may launch now; it waits for this
+  // grid's completion.
+  if (!kBf16) asm volatile("griddepcontrol.launch_dependents;");
+  if (warp == 8 && lane == 0) {
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s.tmem_base;
+
+  if (warp < 8) {
+    softmax2_role<kBf16>(s, p, tmem);
+  } else if (warp == 8) {
+    producer_role(s, p, &tmQ, &tmK, &tmV);
+  } else if (warp == 9) {
+    if (lane == 0) mma2_role<kBf16>(s, p, tmem);
+  } else if (warp == 10) {
+    prep_role<SharedStorage2, kBf16>(s, p, p.bt);
+  } else {
+    convert_role<SharedStorage2, kBf16>(s, p);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 9) {
+    __syncwarp();
+    tmem_dealloc(tmem, kTmemCols2);
+  }
+  if (kBf16 && p.nsplit > 1) {
+    // Every unit was claimed by ticket, so each is held by a running CTA: wait
+    // (bounded) until all partials of the recomputed ranges are written, then
+    // merge this CTA's share of the rows.
+    if (threadIdx.x == 0) {
+      const int want = SharedStorage2::kSoftmaxWarps * p.BH * p.nparts;  // each softmax warp counts its rows
+      const volatile int* cnt = &p.counters[kCtrParts];
+      const uint64_t t0 = globaltimer_ns();
+      while (*cnt < want) {
+        if ((*reinterpret_cast<volatile uint32_t*>(p.status) & kStatusTimeout) ||
+            globaltimer_ns() - t0 > kWaitTimeoutNs) {
+          atomicOr(p.status, kStatusTimeout);
+          break;
+        }
+        __nanosleep(256);
+      }
+      __threadfence();
+    }
+    __syncthreads();
+    merge_ranges<64, kThreads2>(p, blockIdx.x, gridDim.x);
+  }
+  // The CTA that finishes last puts the workspace counters back to zero for
+  // the next call (every other CTA is done with them).
   if (threadIdx.x == 0) {
     __threadfence();
     if (atomicAdd(&p.counters[kCtrDone], 1) == static_cast<int>(gridDim.x) - 1) {
@@ -1123,15 +1551,15 @@ static DeviceInfo* device_info(int dev) {
     di.ok = (major == 10);
     di.sms = sms;
     if (di.ok) {
-      // Four (d 64) or two (d 128) CTAs per SM need the largest shared-memory carve-out.
+      // Two CTAs per SM (either kernel) need the largest shared-memory carve-out.
       const struct {
         const void* fn;
         int smem;
       } kernels[] = {
-          {reinterpret_cast<const void*>(bigbird_fwd_kernel<64, false>), static_cast<int>(sizeof(SharedStorage<64>) + 1024)},
-          {reinterpret_cast<const void*>(bigbird_fwd_kernel<64, true>), static_cast<int>(sizeof(SharedStorage<64>) + 1024)},
           {reinterpret_cast<const void*>(bigbird_fwd_kernel<128, false>), static_cast<int>(sizeof(SharedStorage<128>) + 1024)},
           {reinterpret_cast<const void*>(bigbird_fwd_kernel<128, true>), static_cast<int>(sizeof(SharedStorage<128>) + 1024)},
+          {reinterpret_cast<const void*>(bigbird_fwd2_kernel<false>), static_cast<int>(sizeof(SharedStorage2) + 1024)},
+          {reinterpret_cast<const void*>(bigbird_fwd2_kernel<true>), static_cast<int>(sizeof(SharedStorage2) + 1024)},
       };
       for (const auto& kf : kernels) {
         if (cudaFuncSetAttribute(kf.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, kf.smem) != cudaSuccess)
@@ -1223,6 +1651,30 @@ static cudaError_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, cons
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     e = cudaLaunchKernelEx(&cfg, bigbird_fwd_kernel<kD, true>, tq, tk, tv, p);
+  }
+  return e;
+}
+
+// The d = 64 launches: the split-row kernel's fp16 instance, then its bf16
+// instance as the programmatic dependent (as in launch_fwd).
+static cudaError_t launch_fwd2(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const FwdParams& p,
+                               int sms, cudaStream_t stream) {
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  const int grid = std::min(p.total_units, 2 * sms);
+  const size_t smem = sizeof(SharedStorage2) + 1024;
+  bigbird_fwd2_kernel<false><<<grid, kThreads2, smem, stream>>>(tq, tk, tv, p);
+  cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess) {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kThreads2);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, bigbird_fwd2_kernel<true>, tq, tk, tv, p);
   }
   return e;
 }
@@ -1330,7 +1782,7 @@ static int fwd_impl(const void* q, const void* k, const void* v, const int32_t* 
     p.part_o = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + kCounterBytes);
     p.part_ml = p.part_o + static_cast<size_t>(p.BH) * p.nparts * kRows * d;
   }
-  const cudaError_t e = d == 64 ? launch_fwd<64>(tq, tk, tv, p, di->sms, stream)
+  const cudaError_t e = d == 64 ? launch_fwd2(tq, tk, tv, p, di->sms, stream)
                                 : launch_fwd<128>(tq, tk, tv, p, di->sms, stream);
   if (owned) cudaFreeAsync(ws, stream);
   return e == cudaSuccess ? BB_OK : BB_ERR_CUDA;
