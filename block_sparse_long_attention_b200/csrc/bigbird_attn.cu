@@ -217,6 +217,7 @@ struct __align__(1024) SharedStorage2 {
   uint8_t q[kQBufs][kRows * 64 * 2];
   uint8_t k[kKSt][kBlock * 64 * 2];
   uint8_t v[kVSt][kBlock * 64 * 2];  // converted to fp16 in place
+  uint8_t ostage[kRows * 64 * 2];    // a unit's bf16 output tile (two 64-row TMA boxes, 128-byte swizzle)
   UnitInfo unit[4];
   float2 mlx[2][2][kRows];  // (max, sum) per unit parity, column half, row: the halves' combine
   uint64_t info_full[4];
@@ -234,6 +235,7 @@ struct __align__(1024) SharedStorage2 {
   uint64_t o_full;
   uint64_t o_free;
   uint64_t ml_ready;    // both halves' (max, sum) of the unit are in mlx
+  uint64_t tile_ready;  // all eight softmax warps have written their part of ostage
   uint32_t tmem_base;
   int32_t abort_flag;
 };
@@ -1012,7 +1014,7 @@ __device__ void mma2_role(SharedStorage2& s, const FwdParams& p, uint32_t tmem) 
 // of a row exchange (max, sum) through shared memory; each writes 32 of the
 // row's output columns, O_a and O_b scaled to the common max.
 template <bool kBf16>
-__device__ void softmax2_role(SharedStorage2& s, const FwdParams& p, uint32_t tmem) {
+__device__ void softmax2_role(SharedStorage2& s, const FwdParams& p, uint32_t tmem, const CUtensorMap* tmO) {
   const int wid = threadIdx.x >> 5;  // 0..7
   const int h = wid >> 2;            // key half of each block
   const int row = threadIdx.x & 127; // TMEM lane == row of the unit
@@ -1021,13 +1023,16 @@ __device__ void softmax2_role(SharedStorage2& s, const FwdParams& p, uint32_t tm
   const uint32_t lane_addr = tmem + (static_cast<uint32_t>((wid & 3) * 32) << 16);
   const uint64_t scale2 = f2_pack(p.scale_log2, p.scale_log2);
   uint32_t g = 0;
+  uint32_t staged = 0;  // units whose output tile went out through ostage
   for (uint32_t ut = 0;; ++ut) {
     if (!warp_wait(smem_u32(&s.info_full[ut & 3]), (ut >> 2) & 1)) { flag_timeout(s, p); return; }
     const UnitInfo& ui = s.unit[ut & 3];
     if (ui.stop) break;
     const int n = ui.n;
     const int bh = ui.bh;
-    const int qblk = rhalf ? ui.qbot : ui.qtop;
+    const int qtop = ui.qtop;  // kept: the unit slot is released before the epilogue
+    const int qbot = ui.qbot;
+    const int qblk = rhalf ? qbot : qtop;
     const int split = ui.split;
     const bool exists = qblk >= 0;
     float m_ref = kNegInit;
@@ -1041,37 +1046,31 @@ __device__ void softmax2_role(SharedStorage2& s, const FwdParams& p, uint32_t tm
         const uint32_t vm = static_cast<uint32_t>(ui.vm[e] >> (32 * h));
         const bool mixed = vm != 0xFFFFFFFFu && vm != 0u;
         const float off_s = (vm == 0u ? p.bias_raw : 0.f) * p.scale_log2;
-        float o_factor = 1.f;  // rescale owed to O (the P.V of the earlier blocks)
-        uint64_t acc0 = 0ull, acc1 = 0ull;
         uint32_t r0[16], r1[16];
         tmem_ld16(s_addr, r0);
+        tmem_ld16(s_addr + 16, r1);
         tmem_wait_ld();
-#pragma unroll
-        for (int q = 0; q < 2; ++q) {
-          uint32_t (&cur)[16] = q ? r1 : r0;
-          if (q == 0) tmem_ld16(s_addr + 16, r1);
-          const float mx =
-              fmaf(piece16_prepare(cur, mixed, (vm >> (16 * q)) & 0xFFFFu, p.bias_raw), p.scale_log2, off_s);
-          const bool need = mx > m_ref + kRescaleThreshold;
-          if (__any_sync(0xffffffffu, need)) {
-            float f = 1.f;
-            if (need) {
-              f = ex2_approx(m_ref - mx);
-              m_ref = mx;
-            }
-            l_run *= f;
-            const uint64_t f2 = f2_pack(f, f);
-            acc0 = f2_fma(acc0, f2, 0ull);
-            acc1 = f2_fma(acc1, f2, 0ull);
-            o_factor *= f;
-            if (q > 0 && __any_sync(0xffffffffu, f != 1.f)) rescale_p<kBf16>(s_addr, q, f);
+        // one reference-max decision for the 32 scores: it moves only when one
+        // exceeds it by more than 2^14 (rare after a unit's first block)
+        const float mx = fmaf(fmaxf(piece16_prepare(r0, mixed, vm & 0xFFFFu, p.bias_raw),
+                                    piece16_prepare(r1, mixed, vm >> 16, p.bias_raw)),
+                              p.scale_log2, off_s);
+        const bool need = mx > m_ref + kRescaleThreshold;
+        float o_factor = 1.f;  // rescale owed to O (the P.V of the earlier blocks)
+        if (__any_sync(0xffffffffu, need)) {
+          if (need) {
+            o_factor = ex2_approx(m_ref - mx);
+            m_ref = mx;
           }
-          const float o = off_s - m_ref;
-          uint32_t pk[8];
-          piece16_exp<kBf16>(cur, scale2, f2_pack(o, o), pk, acc0, acc1);
-          if (q == 0) tmem_wait_ld();
-          tmem_st8(s_addr + 8 * q, pk);
+          l_run *= o_factor;
         }
+        const float o = off_s - m_ref;
+        uint64_t acc0 = 0ull, acc1 = 0ull;
+        uint32_t pk0[8], pk1[8];
+        piece16_exp<kBf16>(r0, scale2, f2_pack(o, o), pk0, acc0, acc1);
+        piece16_exp<kBf16>(r1, scale2, f2_pack(o, o), pk1, acc0, acc1);
+        tmem_st8(s_addr, pk0);
+        tmem_st8(s_addr + 8, pk1);
         float a0, a1, b0, b1;
         f2_unpack(acc0, a0, a1);
         f2_unpack(acc1, b0, b1);
@@ -1101,6 +1100,8 @@ __device__ void softmax2_role(SharedStorage2& s, const FwdParams& p, uint32_t tm
     // ---- epilogue: combine the halves, each writes 32 columns of its row
     if (!warp_wait(smem_u32(&s.o_full), ut & 1)) { flag_timeout(s, p); return; }
     tc_fence_after();
+    // the previous tile's TMA store has read ostage before anyone writes it again
+    if (wid == 0 && lane == 0) bulk_wait_read_all();
     s.mlx[ut & 1][h][row] = make_float2(m_ref, l_run);
     __syncwarp();
     if (lane == 0) mbar_arrive(smem_u32(&s.ml_ready));
@@ -1137,21 +1138,65 @@ __device__ void softmax2_role(SharedStorage2& s, const FwdParams& p, uint32_t tm
           atomicAdd(&p.counters[kCtrParts], 1);
         }
       }
-    } else if (exists) {
-      const float inv = 1.f / l;
-      const size_t orow = static_cast<size_t>(bh) * p.L + static_cast<size_t>(qblk) * kBlock + (row & 63);
-      // log sum_k exp(s_k) = ln 2 * (m + log2 l), the scores in log2 units being s * log2(e).
-      if (h == 0 && p.lse) p.lse[orow] = (m + log2f(l)) * 0.69314718055994531f;
+    } else if (p.out_f32) {
+      if (exists) {
+        const float inv = 1.f / l;
+        const size_t orow = static_cast<size_t>(bh) * p.L + static_cast<size_t>(qblk) * kBlock + (row & 63);
+        // log sum_k exp(s_k) = ln 2 * (m + log2 l), the scores in log2 units being s * log2(e).
+        if (h == 0 && p.lse) p.lse[orow] = (m + log2f(l)) * 0.69314718055994531f;
 #pragma unroll 1
-      for (int c0 = 0; c0 < 32; c0 += 16) {
-        uint32_t oa[16], ob[16];
-        tmem_ld16(lane_addr + kColOa + c_base + c0, oa);
-        tmem_ld16(lane_addr + kColOb + c_base + c0, ob);
-        tmem_wait_ld();
+        for (int c0 = 0; c0 < 32; c0 += 16) {
+          uint32_t oa[16], ob[16];
+          tmem_ld16(lane_addr + kColOa + c_base + c0, oa);
+          tmem_ld16(lane_addr + kColOb + c_base + c0, ob);
+          tmem_wait_ld();
 #pragma unroll
-        for (int i = 0; i < 16; ++i) oa[i] = __float_as_uint(__uint_as_float(oa[i]) * fa + __uint_as_float(ob[i]) * fb);
-        store16<64>(p, orow, c_base + c0, oa, inv);
+          for (int i = 0; i < 16; ++i)
+            oa[i] = __float_as_uint(__uint_as_float(oa[i]) * fa + __uint_as_float(ob[i]) * fb);
+          store16<64>(p, orow, c_base + c0, oa, inv);
+        }
       }
+    } else {
+      // bf16 output: each thread puts its 32 columns (four 16-byte chunks of
+      // its 128-byte row) into ostage, swizzled as the tensor map expects;
+      // warp 0 then stores the tile's one or two 64-row boxes with TMA.
+      if (exists) {
+        const float inv = 1.f / l;
+        if (h == 0 && p.lse) {
+          const size_t orow = static_cast<size_t>(bh) * p.L + static_cast<size_t>(qblk) * kBlock + (row & 63);
+          p.lse[orow] = (m + log2f(l)) * 0.69314718055994531f;
+        }
+        const int rr = row & 63;
+        uint8_t* srow = s.ostage + (row >> 6) * (kBlock * 128) + rr * 128;
+#pragma unroll 1
+        for (int c0 = 0; c0 < 32; c0 += 16) {
+          uint32_t oa[16], ob[16];
+          tmem_ld16(lane_addr + kColOa + c_base + c0, oa);
+          tmem_ld16(lane_addr + kColOb + c_base + c0, ob);
+          tmem_wait_ld();
+          uint32_t w[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            w[i] = pack_bf16x2((__uint_as_float(oa[2 * i]) * fa + __uint_as_float(ob[2 * i]) * fb) * inv,
+                               (__uint_as_float(oa[2 * i + 1]) * fa + __uint_as_float(ob[2 * i + 1]) * fb) * inv);
+          const int cc = (c_base + c0) >> 3;  // 16-byte chunk of the row
+          *reinterpret_cast<uint4*>(srow + ((cc ^ (rr & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+          *reinterpret_cast<uint4*>(srow + (((cc + 1) ^ (rr & 7)) << 4)) = make_uint4(w[4], w[5], w[6], w[7]);
+        }
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&s.tile_ready));
+      if (wid == 0) {
+        if (!warp_wait(smem_u32(&s.tile_ready), staged & 1)) { flag_timeout(s, p); return; }
+        if (lane == 0) {
+          const int32_t row0 = bh * p.L;
+          tma_store_2d(tmO, smem_u32(s.ostage), 0, row0 + qtop * kBlock);
+          if (qbot >= 0) tma_store_2d(tmO, smem_u32(s.ostage) + kBlock * 128, 0, row0 + qbot * kBlock);
+          bulk_commit();
+        }
+      }
+      ++staged;
     }
     tc_fence_before();
     __syncwarp();
@@ -1366,7 +1411,8 @@ bigbird_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
 template <bool kBf16>
 __global__ void __launch_bounds__(kThreads2, 2)
 bigbird_fwd2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                    const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
+                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+                    const FwdParams p) {
   extern __shared__ uint8_t smem_raw[];
   SharedStorage2& s =
       *reinterpret_cast<SharedStorage2*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -1415,6 +1461,7 @@ bigbird_fwd2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     mbar_init(smem_u32(&s.o_full), 1);
     mbar_init(smem_u32(&s.o_free), 8);
     mbar_init(smem_u32(&s.ml_ready), 8);
+    mbar_init(smem_u32(&s.tile_ready), 8);
     s.abort_flag = 0;
     fence_barrier_init();
   }
@@ -1425,6 +1472,7 @@ bigbird_fwd2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     tma_prefetch_desc(&tmQ);
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
+    if (!p.out_f32) tma_prefetch_desc(&tmO);
   }
   tc_fence_before();
   __syncthreads();
@@ -1432,7 +1480,9 @@ bigbird_fwd2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
   const uint32_t tmem = s.tmem_base;
 
   if (warp < 8) {
-    softmax2_role<kBf16>(s, p, tmem);
+    softmax2_role<kBf16>(s, p, tmem, &tmO);
+    // the bf16 output tiles' TMA stores read shared memory until they complete
+    if (warp == 0 && lane == 0) bulk_wait_all();
   } else if (warp == 8) {
     producer_role(s, p, &tmQ, &tmK, &tmV);
   } else if (warp == 9) {
@@ -1657,14 +1707,14 @@ static cudaError_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, cons
 
 // The d = 64 launches: the split-row kernel's fp16 instance, then its bf16
 // instance as the programmatic dependent (as in launch_fwd).
-static cudaError_t launch_fwd2(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const FwdParams& p,
-                               int sms, cudaStream_t stream) {
+static cudaError_t launch_fwd2(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                               const CUtensorMap& to, const FwdParams& p, int sms, cudaStream_t stream) {
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   const int grid = std::min(p.total_units, 2 * sms);
   const size_t smem = sizeof(SharedStorage2) + 1024;
-  bigbird_fwd2_kernel<false><<<grid, kThreads2, smem, stream>>>(tq, tk, tv, p);
+  bigbird_fwd2_kernel<false><<<grid, kThreads2, smem, stream>>>(tq, tk, tv, to, p);
   cudaError_t e = cudaGetLastError();
   if (e == cudaSuccess) {
     cudaLaunchConfig_t cfg{};
@@ -1674,7 +1724,7 @@ static cudaError_t launch_fwd2(const CUtensorMap& tq, const CUtensorMap& tk, con
     cfg.stream = stream;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, bigbird_fwd2_kernel<true>, tq, tk, tv, p);
+    e = cudaLaunchKernelEx(&cfg, bigbird_fwd2_kernel<true>, tq, tk, tv, to, p);
   }
   return e;
 }
@@ -1725,9 +1775,15 @@ static int fwd_impl(const void* q, const void* k, const void* v, const int32_t* 
     if (vs != BB_OK) return vs;
   }
 
-  CUtensorMap tq, tk, tv;
+  CUtensorMap tq, tk, tv, to;
   const uint64_t rows = static_cast<uint64_t>(B) * H * L;
   if (!make_map(&tq, q, rows, d) || !make_map(&tk, k, rows, d) || !make_map(&tv, v, rows, d)) return BB_ERR_CUDA;
+  // the bf16 output at d = 64 leaves through TMA stores (64-row boxes, like Q)
+  if (d == 64 && out_dtype != BB_OUT_F32) {
+    if (!make_map(&to, out, rows, 64)) return BB_ERR_CUDA;
+  } else {
+    to = tq;  // not used
+  }
 
   FwdParams p{};
   p.q = static_cast<const uint16_t*>(q);
@@ -1782,7 +1838,7 @@ static int fwd_impl(const void* q, const void* k, const void* v, const int32_t* 
     p.part_o = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + kCounterBytes);
     p.part_ml = p.part_o + static_cast<size_t>(p.BH) * p.nparts * kRows * d;
   }
-  const cudaError_t e = d == 64 ? launch_fwd2(tq, tk, tv, p, di->sms, stream)
+  const cudaError_t e = d == 64 ? launch_fwd2(tq, tk, tv, to, p, di->sms, stream)
                                 : launch_fwd<128>(tq, tk, tv, p, di->sms, stream);
   if (owned) cudaFreeAsync(ws, stream);
   return e == cudaSuccess ? BB_OK : BB_ERR_CUDA;
