@@ -15,6 +15,9 @@ bool make_tile_map(CUtensorMap* map, const void* base, uint64_t rows);
 // The same over a [rows, d] matrix (d = 64 or 128): 64x64 boxes, one per
 // 64-column chunk (x = 64 c).
 bool make_tile_map_d(CUtensorMap* map, const void* base, uint64_t rows, int d);
+// Tensor map over a [rows, 64] fp32 matrix with boxes of 64 rows x 32 columns
+// (128 bytes) and 128-byte swizzle, for TMA stores of gradient tiles.
+bool make_f32_map(CUtensorMap* map, const void* base, uint64_t rows);
 
 // Device address of the library's status word on the current device `dev`
 // (bit 1: an out-of-range rand_attn entry was skipped; bit 2: a bounded wait

@@ -1627,6 +1627,18 @@ static DeviceInfo* device_info(int dev) {
 bool make_tile_map(CUtensorMap* map, const void* base, uint64_t rows) { return make_map(map, base, rows, 64); }
 bool make_tile_map_d(CUtensorMap* map, const void* base, uint64_t rows, int d) { return make_map(map, base, rows, d); }
 
+bool make_f32_map(CUtensorMap* map, const void* base, uint64_t rows) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {64, static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {64 * 4};
+  const cuuint32_t box[2] = {32u, static_cast<cuuint32_t>(kBlock)};
+  const cuuint32_t es[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 uint32_t* status_word(int dev) {
   DeviceInfo* di = device_info(dev);
   return di && di->ok ? di->status : nullptr;

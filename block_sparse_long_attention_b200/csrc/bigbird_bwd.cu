@@ -130,12 +130,21 @@ struct Params {
   float scale;            // 1 / sqrt(d)
 };
 
+// TMA store maps of the gradient tiles at d = 64 ([rows, 64] fp32, boxes of
+// 64 rows x 32 columns): the direct outputs g1, g2 and the partial sums.
+struct StoreMaps {
+  CUtensorMap o1, o2, p1, p2;
+};
+
 template <int kD>
 struct __align__(1024) Smem {
   uint8_t a1[kRows * kD * 2];                   // Q (dq) or K (dk/dv) of the unit: two tiles
   uint8_t a2[kRows * kD * 2];                   // dO (dq) or V (dk/dv)
   uint8_t b1[kStages][BGeo<kD>::kTileBytes];    // K (dq) or Q (dk/dv) of a step
   uint8_t b2[kStages][BGeo<kD>::kTileBytes];    // V (dq) or dO (dk/dv)
+  // d = 64: one fp32 accumulator tile of the unit (four boxes of 64 rows x
+  // 32 columns, 128-byte swizzle) on its way out through TMA stores
+  uint8_t ostage[kD == 64 ? kRows * 64 * 4 : 1024];
   float col_lse[kStages][kBlock];         // dk/dv: lse and D of the step's query tile
   float col_d[kStages][kBlock];
   Unit unit[4];
@@ -148,6 +157,8 @@ struct __align__(1024) Smem {
   uint64_t xy_free;    // the step's gradient MMAs are complete (S/dP columns reusable)
   uint64_t acc_full;   // a unit's accumulators are complete
   uint64_t acc_free;   // ... and read by the epilogue (4 warps)
+  uint64_t stage_free; // d = 64: ostage may be written (the previous tile's stores have read it)
+  uint64_t tile_ready; // d = 64: the elementwise warps have written their part of ostage
   uint32_t tmem_base;
   uint32_t rbits[32];  // dk/dv prep: per query block of a scan batch, which key blocks it picked at random
 };
@@ -683,7 +694,7 @@ __device__ __forceinline__ void piece_pds(const uint32_t (&x)[16], const uint32_
 // acc1, dk = acc2 / sqrt(d); raw into the partial-sum slot of a split global
 // unit).
 template <int kD, bool kKV>
-__device__ void elem_role(Smem<kD>& s, const Params& p, uint32_t tmem) {
+__device__ void elem_role(Smem<kD>& s, const Params& p, uint32_t tmem, const StoreMaps* smaps) {
   constexpr float kLog2e = 1.4426950408889634f;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -694,6 +705,7 @@ __device__ void elem_role(Smem<kD>& s, const Params& p, uint32_t tmem) {
   const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quad * 32) << 16);
   const float row_bias_l2_masked = p.bias_raw * p.scale_log2;
   uint32_t g = 0, ua = 0;
+  uint32_t staged = 0;  // d = 64: accumulator tiles that went out through ostage
   float row_c = 0.f, row_cmask = 0.f, row_d = 0.f, row_bias_l2 = 0.f;
   for (uint32_t ut = 0;; ++ut) {
     if (!warp_wait(smem_u32(&s.info_full[ut & 3]), (ut >> 2) & 1)) { if (lane == 0) flag_timeout(p); return; }
@@ -701,6 +713,7 @@ __device__ void elem_role(Smem<kD>& s, const Params& p, uint32_t tmem) {
     if (ui.stop) break;
     const int n = ui.n;
     const int stile = half ? ui.bot : ui.top;
+    const int top_tile = ui.top, bot_tile = ui.bot;  // kept: the unit slot is released before the epilogue
     const bool exists = stile >= 0;
     const int bh = ui.bh;
     const size_t row = static_cast<size_t>(bh) * p.L + static_cast<size_t>(exists ? stile : 0) * kBlock + (rowi & 63);
@@ -762,26 +775,85 @@ __device__ void elem_role(Smem<kD>& s, const Params& p, uint32_t tmem) {
     // ---- epilogue: this warp's d / 2 columns of each accumulator
     if (!warp_wait(smem_u32(&s.acc_full), ua & 1)) { if (lane == 0) flag_timeout(p); return; }
     tc_fence_after();
-    if (exists) {
-      const size_t prow = (static_cast<size_t>(bh) * p.nparts + (split >= 0 ? split : 0)) * kRows + rowi;
+    if constexpr (kD == 64) {
+      // Each accumulator goes out through ostage: every thread writes its 32
+      // columns (eight 16-byte chunks of one 128-byte box row, swizzled as the
+      // tensor map expects), then warp 0 stores the tile's boxes with TMA.
+      const int rr = rowi & 63;
+      uint8_t* srow = s.ostage + ((rowi >> 6) * 2 + chalf) * (kBlock * 128) + rr * 128;
 #pragma unroll 1
       for (int a = 0; a < (kKV ? 2 : 1); ++a) {
         // acc1: dq (dq kernel) or dv; acc2: dk
         const float f = (split >= 0 || (kKV && a == 0)) ? 1.f : p.scale;
-        float* dst = split >= 0 ? (a == 0 ? p.part1 : p.part2) + prow * kD : (a == 0 ? p.g1 : p.g2) + row * kD;
+        if (warp == 0 && lane == 0) {
+          bulk_wait_read_all();  // the previous tile's stores have read ostage
+          mbar_arrive(smem_u32(&s.stage_free));
+        }
+        if (!warp_wait(smem_u32(&s.stage_free), staged & 1)) { if (lane == 0) flag_timeout(p); return; }
+        if (exists) {
 #pragma unroll 1
-        for (int c0 = (kD / 2) * chalf; c0 < (kD / 2) * (chalf + 1); c0 += 16) {
-          uint32_t o[16];
-          tmem_ld16(lane_addr + (a == 0 ? kColA1 : BGeo<kD>::kColA2) + c0, o);
-          tmem_wait_ld();
-          float4* d4 = reinterpret_cast<float4*>(dst + c0);
+          for (int c0 = 0; c0 < 32; c0 += 16) {
+            uint32_t o[16];
+            tmem_ld16(lane_addr + (a == 0 ? kColA1 : BGeo<kD>::kColA2) + 32 * chalf + c0, o);
+            tmem_wait_ld();
 #pragma unroll
-          for (int c = 0; c < 4; ++c)
-            d4[c] = make_float4(__uint_as_float(o[4 * c]) * f, __uint_as_float(o[4 * c + 1]) * f,
-                                __uint_as_float(o[4 * c + 2]) * f, __uint_as_float(o[4 * c + 3]) * f);
+            for (int j = 0; j < 4; ++j) {
+              const int cc = (c0 >> 2) + j;  // 16-byte chunk (four floats) of the box row
+              *reinterpret_cast<float4*>(srow + ((cc ^ (rr & 7)) << 4)) =
+                  make_float4(__uint_as_float(o[4 * j]) * f, __uint_as_float(o[4 * j + 1]) * f,
+                              __uint_as_float(o[4 * j + 2]) * f, __uint_as_float(o[4 * j + 3]) * f);
+            }
+          }
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&s.tile_ready));
+        if (warp == 0) {
+          if (!warp_wait(smem_u32(&s.tile_ready), staged & 1)) { if (lane == 0) flag_timeout(p); return; }
+          if (lane == 0) {
+            const CUtensorMap* map = split >= 0 ? (a == 0 ? &smaps->p1 : &smaps->p2) : (a == 0 ? &smaps->o1 : &smaps->o2);
+            const uint32_t src = smem_u32(s.ostage);
+            int32_t y0, y1;
+            if (split >= 0) {
+              y0 = (bh * p.nparts + split) * kRows;
+              y1 = y0 + kBlock;
+            } else {
+              y0 = bh * p.L + top_tile * kBlock;
+              y1 = bot_tile >= 0 ? bh * p.L + bot_tile * kBlock : -1;
+            }
+            tma_store_2d(map, src, 0, y0);
+            tma_store_2d(map, src + kBlock * 128, 32, y0);
+            if (y1 >= 0) {
+              tma_store_2d(map, src + 2 * kBlock * 128, 0, y1);
+              tma_store_2d(map, src + 3 * kBlock * 128, 32, y1);
+            }
+            bulk_commit();
+          }
+        }
+        ++staged;
+      }
+    } else {
+      if (exists) {
+        const size_t prow = (static_cast<size_t>(bh) * p.nparts + (split >= 0 ? split : 0)) * kRows + rowi;
+  #pragma unroll 1
+        for (int a = 0; a < (kKV ? 2 : 1); ++a) {
+          // acc1: dq (dq kernel) or dv; acc2: dk
+          const float f = (split >= 0 || (kKV && a == 0)) ? 1.f : p.scale;
+          float* dst = split >= 0 ? (a == 0 ? p.part1 : p.part2) + prow * kD : (a == 0 ? p.g1 : p.g2) + row * kD;
+  #pragma unroll 1
+          for (int c0 = (kD / 2) * chalf; c0 < (kD / 2) * (chalf + 1); c0 += 16) {
+            uint32_t o[16];
+            tmem_ld16(lane_addr + (a == 0 ? kColA1 : BGeo<kD>::kColA2) + c0, o);
+            tmem_wait_ld();
+            float4* d4 = reinterpret_cast<float4*>(dst + c0);
+  #pragma unroll
+            for (int c = 0; c < 4; ++c)
+              d4[c] = make_float4(__uint_as_float(o[4 * c]) * f, __uint_as_float(o[4 * c + 1]) * f,
+                                  __uint_as_float(o[4 * c + 2]) * f, __uint_as_float(o[4 * c + 3]) * f);
+          }
         }
       }
-    }
+}
     tc_fence_before();
     __syncwarp();
     if (lane == 0) mbar_arrive(smem_u32(&s.acc_free));
@@ -796,7 +868,7 @@ template <int kD, int kBt, bool kKV>
 __global__ void __launch_bounds__(kThreads, BGeo<kD>::kCtasPerSm)
 bwd_kernel(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmA2,
            const __grid_constant__ CUtensorMap tmB1, const __grid_constant__ CUtensorMap tmB2,
-           const __grid_constant__ Params p) {
+           const __grid_constant__ StoreMaps smaps, const __grid_constant__ Params p) {
   constexpr uint32_t kTmemCols = BGeo<kD>::tmem_cols(kKV);
   extern __shared__ uint8_t smem_raw[];
   Smem<kD>& s = *reinterpret_cast<Smem<kD>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -822,6 +894,8 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUt
     mbar_init(smem_u32(&s.xy_free), 1);
     mbar_init(smem_u32(&s.acc_full), 1);
     mbar_init(smem_u32(&s.acc_free), kElemWarps);
+    mbar_init(smem_u32(&s.stage_free), 1);
+    mbar_init(smem_u32(&s.tile_ready), kElemWarps);
     fence_barrier_init();
   }
   if (warp == 8 && lane == 0) {
@@ -835,7 +909,9 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUt
   tc_fence_after();
   const uint32_t tmem = s.tmem_base;
   if (warp < kElemWarps) {
-    elem_role<kD, kKV>(s, p, tmem);
+    elem_role<kD, kKV>(s, p, tmem, &smaps);
+    // the gradient tiles' TMA stores read shared memory until they complete
+    if (kD == 64 && warp == 0 && lane == 0) bulk_wait_all();
   } else if (warp == 8) {
     producer_role<kD, kKV>(s, p, &tmA1, &tmA2, &tmB1, &tmB2);
   } else if (warp == 9) {
@@ -995,7 +1071,8 @@ bool set_attributes(int dev) {
 // the partial sums of the split global units.
 template <int kD, int kBt>
 cudaError_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tdo,
-                       const bbw::Params& pq, const bbw::Params& pk, const BwdPlan& pl, int sms, const void* dout,
+                       const bbw::StoreMaps& smq, const bbw::StoreMaps& smk, const bbw::Params& pq,
+                       const bbw::Params& pk, const BwdPlan& pl, int sms, const void* dout,
                        const void* out, int out_f32, float* dd, size_t rows, float* dq, float* dk, float* dv, int L,
                        cudaStream_t stream) {
   using namespace bbw;
@@ -1004,8 +1081,8 @@ cudaError_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUten
   constexpr int kRowsPerCta = 256 / (kD / 4);
   bwd_rowdot_kernel<kD><<<static_cast<unsigned>((rows + kRowsPerCta - 1) / kRowsPerCta), 256, 0, stream>>>(
       static_cast<const uint16_t*>(dout), out, out_f32, dd, rows);
-  bwd_kernel<kD, kBt, false><<<grid, kThreads, smem, stream>>>(tq, tdo, tk, tv, pq);
-  bwd_kernel<kD, kBt, true><<<grid, kThreads, smem, stream>>>(tk, tv, tq, tdo, pk);
+  bwd_kernel<kD, kBt, false><<<grid, kThreads, smem, stream>>>(tq, tdo, tk, tv, smq, pq);
+  bwd_kernel<kD, kBt, true><<<grid, kThreads, smem, stream>>>(tk, tv, tq, tdo, smk, pk);
   if (pl.nsplit > 1) {
     const dim3 sg(pq.BH * pl.n_glob, kRows / kRowsPerCta);
     bwd_sum_kernel<kD><<<sg, 256, 0, stream>>>(pq.part1, dq, pl.nsplit, pl.n_glob, L, pl.nt, pq.scale);
@@ -1105,13 +1182,34 @@ extern "C" int bigbird_attn_bwd_ex(const void* q, const void* k, const void* v, 
   pk.part2 = pl.nsplit > 1 ? reinterpret_cast<float*>(wsb + pl.partk_off) : nullptr;
   pk.counters = reinterpret_cast<int*>(wsb) + 2;
   const int of32 = out_dtype == BB_OUT_F32 ? 1 : 0;
+  // d = 64: the gradient tiles leave through TMA stores (maps over dq, dv, dk
+  // and the three partial-sum arrays; unused entries repeat a valid map)
+  StoreMaps smq{}, smk{};
+  if (d == 64) {
+    const uint64_t prow = static_cast<uint64_t>(B) * H * pl.n_glob * pl.nsplit * kRows;
+    bool ok = make_f32_map(&smq.o1, dq, rows) && make_f32_map(&smk.o1, dv, rows) && make_f32_map(&smk.o2, dk, rows);
+    if (ok && pl.nsplit > 1) {
+      ok = make_f32_map(&smq.p1, pq.part1, prow) && make_f32_map(&smk.p1, pk.part1, prow) &&
+           make_f32_map(&smk.p2, pk.part2, prow);
+    } else {
+      smq.p1 = smq.o1;
+      smk.p1 = smk.o1;
+      smk.p2 = smk.o2;
+    }
+    smq.o2 = smq.o1;
+    smq.p2 = smq.p1;
+    if (!ok) {
+      if (owned) cudaFreeAsync(ws, stream);
+      return BB_ERR_CUDA;
+    }
+  }
   cudaError_t e;
   if (d == 64)
-    e = pl.bt == 1 ? launch_bwd<64, 1>(tq, tk, tv, tdo, pq, pk, pl, sms, dout, out, of32, dd, rows, dq, dk, dv, L, stream)
-                   : launch_bwd<64, 2>(tq, tk, tv, tdo, pq, pk, pl, sms, dout, out, of32, dd, rows, dq, dk, dv, L, stream);
+    e = pl.bt == 1 ? launch_bwd<64, 1>(tq, tk, tv, tdo, smq, smk, pq, pk, pl, sms, dout, out, of32, dd, rows, dq, dk, dv, L, stream)
+                   : launch_bwd<64, 2>(tq, tk, tv, tdo, smq, smk, pq, pk, pl, sms, dout, out, of32, dd, rows, dq, dk, dv, L, stream);
   else
-    e = pl.bt == 1 ? launch_bwd<128, 1>(tq, tk, tv, tdo, pq, pk, pl, sms, dout, out, of32, dd, rows, dq, dk, dv, L, stream)
-                   : launch_bwd<128, 2>(tq, tk, tv, tdo, pq, pk, pl, sms, dout, out, of32, dd, rows, dq, dk, dv, L, stream);
+    e = pl.bt == 1 ? launch_bwd<128, 1>(tq, tk, tv, tdo, smq, smk, pq, pk, pl, sms, dout, out, of32, dd, rows, dq, dk, dv, L, stream)
+                   : launch_bwd<128, 2>(tq, tk, tv, tdo, smq, smk, pq, pk, pl, sms, dout, out, of32, dd, rows, dq, dk, dv, L, stream);
   if (owned) cudaFreeAsync(ws, stream);
   return e == cudaSuccess ? BB_OK : BB_ERR_CUDA;
 }
