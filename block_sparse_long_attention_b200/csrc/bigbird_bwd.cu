@@ -8,8 +8,10 @@
 //   dp = dout v^T,  ds = p (dp - D),
 //   dq = ds k / sqrt(d),  dk = ds^T q / sqrt(d),  dv = p^T dout.
 //
-// Four launches, in stream order, nothing accumulated with atomics (the
-// gradients are the same bit for bit on every run):
+// Four launches, in stream order (the dk/dv kernel as the dq kernel's
+// programmatic dependent, free to start on the SMs the dq kernel leaves, as
+// it needs nothing the dq kernel writes), nothing accumulated with atomics
+// (the gradients are the same bit for bit on every run):
 //   1. bwd_rowdot_kernel: D = rowsum(dout * out) into the workspace;
 //   2. bwd_kernel<false> (dq): query-stationary. A unit is the forward's: 128
 //      query rows (query blocks i, i+1, or the two global blocks against one
@@ -26,12 +28,14 @@
 //      one thread per key row (the query's lse and D from shared memory), then
 //      dV += P^T dO and dK += dS^T Q (two TS-MMAs);
 //   4. bwd_sum_kernel: the global rows' dq and the global key blocks' dk, dv
-//      are split over ranges; their partial sums (workspace) are added here.
+//      are split over ranges; their partial sums (workspace) are added here,
+//      all three in one launch.
 //
 // Both attention kernels are persistent (2 CTAs per SM, 256 TMEM columns:
 // S | dP | accumulator 1 | accumulator 2) and warp-specialised: warps 0-7 the
 // elementwise part and the epilogue (two warps per row, 32 columns each),
-// warp 8 TMA, warp 9 the MMAs (one thread), warp 10 unit preparation and
+// warp 8 TMA, warps 9 and 11 the MMAs (one thread each: S and its product,
+// dP and its product), warp 10 unit preparation and
 // scheduling (tickets from a workspace counter, reset by the CTA that
 // finishes last). Every wait is bounded.
 #include <cuda.h>
@@ -55,7 +59,7 @@ constexpr int kStages = 2;     // moving-tile ring depth
 constexpr int kMaxList = 42;   // moving tiles per unit chunk
 constexpr int kMaxR = 16;
 constexpr int kSplit = 8;      // tiles per range of a global unit
-constexpr int kThreads = 384;  // warps 0-7 elementwise, 8 TMA, 9 MMA, 10 prep, 11 idle
+constexpr int kThreads = 384;  // warps 0-7 elementwise, 8 TMA, 9 and 11 MMA, 10 prep
 constexpr int kElemWarps = 8;
 constexpr uint32_t kChunkBytes = kBlock * 64 * 2;  // 64 rows x 64 columns bf16: one TMA box
 constexpr uint32_t kColX = 0;     // S (or S^T): 64 fp32 columns; then P_hi and P_lo (bf16 pairs)
@@ -154,7 +158,7 @@ struct __align__(1024) Smem {
   uint64_t b_full[kStages], b_empty[kStages];
   uint64_t x_full;     // S and dP of the step are in TMEM
   uint64_t p_full;     // P and dS written (4 warps)
-  uint64_t xy_free;    // the step's gradient MMAs are complete (S/dP columns reusable)
+  uint64_t xy_free[2]; // a part's gradient MMAs of the step are complete (its columns reusable)
   uint64_t acc_full;   // a unit's accumulators are complete
   uint64_t acc_free;   // ... and read by the epilogue (4 warps)
   uint64_t stage_free; // d = 64: ostage may be written (the previous tile's stores have read it)
@@ -558,12 +562,20 @@ __device__ void producer_role(Smem<kD>& s, const Params& p, const CUtensorMap* t
 // 64 moving rows):
 //   dq kernel:   acc1 += (dS_hi + dS_lo) B1                          (dQ += dS K)
 //   dk/dv kernel: acc1 += (P_hi + P_lo) B2, acc2 += (dS_hi + dS_lo) B1 (dV += P^T dO, dK += dS^T Q)
-template <int kD, bool kKV>
+template <int kD, bool kKV, int kPart>
 __device__ void mma_role(Smem<kD>& s, const Params& p, uint32_t tmem) {
   using G = BGeo<kD>;
+  // Two issuing threads (warps 9 and 11), each with its own products:
+  //   dk/dv: part 0 S^T -> dV += P^T dO;  part 1 dP^T -> dK += dS^T Q;
+  //   dq:    part 0 S   -> dQ += dS K;     part 1 dP.
+  // A part reuses its S or dP columns once its own gradient MMAs that read
+  // them are complete (dk/dv: xy_free[part]; dq: dP waits for dQ, xy_free[0],
+  // while S's columns are read by no MMA and free once P(g) is written).
+  constexpr bool kHasGrad = kKV || kPart == 0;
   const uint32_t idesc1 = idesc_f32acc(kRows, kBlock, true, false);
   const uint32_t idesc2 = idesc_f32acc(kRows, 64, true, true);  // one 64-column chunk of d
-  const uint32_t a1 = smem_u32(s.a1), a2 = smem_u32(s.a2);
+  const uint32_t a_src = smem_u32(kPart == 0 ? s.a1 : s.a2);
+  const uint32_t x_col = kPart == 0 ? kColX : kColY;  // this part's S or dP columns
   uint32_t g = 0, ua = 0;
   bool ok = true;
   for (uint32_t ut = 0; ok; ++ut) {
@@ -576,58 +588,49 @@ __device__ void mma_role(Smem<kD>& s, const Params& p, uint32_t tmem) {
     for (int e = 0; e < n; ++e, ++g) {
       const int st = g % kStages;
       if (!mbar_wait(smem_u32(&s.b_full[st]), (g / kStages) & 1)) { ok = false; break; }
-      if (g >= 1 && !mbar_wait(smem_u32(&s.xy_free), (g - 1) & 1)) { ok = false; break; }
+      if (g >= 1) {
+        if (kKV && !mbar_wait(smem_u32(&s.xy_free[kPart]), (g - 1) & 1)) { ok = false; break; }
+        if (!kKV && kPart == 1 && !mbar_wait(smem_u32(&s.xy_free[0]), (g - 1) & 1)) { ok = false; break; }
+      }
       tc_fence_after();
       const uint32_t b1 = smem_u32(s.b1[st]), b2 = smem_u32(s.b2[st]);
+      const uint32_t b_src = kPart == 0 ? b1 : b2;
       // K = d in steps of 16: four per 64-column chunk
 #pragma unroll
       for (int kk = 0; kk < kD / 16; ++kk)
-        mma_ss(tmem + kColX, sdesc_sw128(a1 + (kk >> 2) * G::kAChunkBytes + (kk & 3) * 32, 16, 1024),
-               sdesc_sw128(b1 + (kk >> 2) * kChunkBytes + (kk & 3) * 32, 16, 1024), idesc1, kk > 0 ? 1u : 0u);
-#pragma unroll
-      for (int kk = 0; kk < kD / 16; ++kk)
-        mma_ss(tmem + kColY, sdesc_sw128(a2 + (kk >> 2) * G::kAChunkBytes + (kk & 3) * 32, 16, 1024),
-               sdesc_sw128(b2 + (kk >> 2) * kChunkBytes + (kk & 3) * 32, 16, 1024), idesc1, kk > 0 ? 1u : 0u);
+        mma_ss(tmem + x_col, sdesc_sw128(a_src + (kk >> 2) * G::kAChunkBytes + (kk & 3) * 32, 16, 1024),
+               sdesc_sw128(b_src + (kk >> 2) * kChunkBytes + (kk & 3) * 32, 16, 1024), idesc1, kk > 0 ? 1u : 0u);
       mma_commit(smem_u32(&s.x_full));
       if (last && e == n - 1) mma_commit(smem_u32(&s.a_free));
-      // the unit's first step overwrites the accumulators, once the previous
-      // unit's epilogue has read them
-      const bool zero = first && e == 0;
-      if (zero && !mbar_wait(smem_u32(&s.acc_free), (ua & 1) ^ 1)) { ok = false; break; }
-      if (!mbar_wait(smem_u32(&s.p_full), g & 1)) { ok = false; break; }
-      tc_fence_after();
-      // accumulator columns 64 c .. 64 c + 63 from chunk c of the moving tile
+      if (kHasGrad) {
+        // the unit's first step overwrites the accumulator, once the previous
+        // unit's epilogue has read it
+        const bool zero = first && e == 0;
+        if (zero && !mbar_wait(smem_u32(&s.acc_free), (ua & 1) ^ 1)) { ok = false; break; }
+        if (!mbar_wait(smem_u32(&s.p_full), g & 1)) { ok = false; break; }
+        tc_fence_after();
+        // dk/dv part 0: dV += (P_hi + P_lo) dO (P in the S columns, B = b2);
+        // dk/dv part 1: dK += (dS_hi + dS_lo) Q (dS in the dP columns, B = b1);
+        // dq: dQ += (dS_hi + dS_lo) K (dS in the dP columns, B = b1)
+        const uint32_t acc = kKV && kPart == 1 ? G::kColA2 : kColA1;
+        const uint32_t pcol = kKV && kPart == 0 ? kColX : kColY;
+        const uint32_t bsrc = kKV && kPart == 0 ? b2 : b1;
+        // accumulator columns 64 c .. 64 c + 63 from chunk c of the moving tile
 #pragma unroll
-      for (int c = 0; c < G::kChunks; ++c) {
-        const uint32_t boff = c * kChunkBytes;
-        if (kKV) {
+        for (int c = 0; c < G::kChunks; ++c) {
+          const uint32_t boff = c * kChunkBytes;
 #pragma unroll
           for (int kk = 0; kk < kBlock / 16; ++kk) {
-            mma_ts(tmem + kColA1 + 64 * c, tmem + kColX + hi_col(kk), sdesc_sw128(b2 + boff + kk * 2048, 8192, 1024),
+            mma_ts(tmem + acc + 64 * c, tmem + pcol + hi_col(kk), sdesc_sw128(bsrc + boff + kk * 2048, 8192, 1024),
                    idesc2, (zero && kk == 0) ? 0u : 1u);
-            mma_ts(tmem + kColA1 + 64 * c, tmem + kColX + lo_col(kk), sdesc_sw128(b2 + boff + kk * 2048, 8192, 1024),
-                   idesc2, 1u);
-          }
-#pragma unroll
-          for (int kk = 0; kk < kBlock / 16; ++kk) {
-            mma_ts(tmem + G::kColA2 + 64 * c, tmem + kColY + hi_col(kk),
-                   sdesc_sw128(b1 + boff + kk * 2048, 8192, 1024), idesc2, (zero && kk == 0) ? 0u : 1u);
-            mma_ts(tmem + G::kColA2 + 64 * c, tmem + kColY + lo_col(kk),
-                   sdesc_sw128(b1 + boff + kk * 2048, 8192, 1024), idesc2, 1u);
-          }
-        } else {
-#pragma unroll
-          for (int kk = 0; kk < kBlock / 16; ++kk) {
-            mma_ts(tmem + kColA1 + 64 * c, tmem + kColY + hi_col(kk), sdesc_sw128(b1 + boff + kk * 2048, 8192, 1024),
-                   idesc2, (zero && kk == 0) ? 0u : 1u);
-            mma_ts(tmem + kColA1 + 64 * c, tmem + kColY + lo_col(kk), sdesc_sw128(b1 + boff + kk * 2048, 8192, 1024),
+            mma_ts(tmem + acc + 64 * c, tmem + pcol + lo_col(kk), sdesc_sw128(bsrc + boff + kk * 2048, 8192, 1024),
                    idesc2, 1u);
           }
         }
+        mma_commit(smem_u32(&s.xy_free[kPart]));
+        if (last && e == n - 1) mma_commit(smem_u32(&s.acc_full));
       }
-      mma_commit(smem_u32(&s.xy_free));
       mma_commit(smem_u32(&s.b_empty[st]));
-      if (last && e == n - 1) mma_commit(smem_u32(&s.acc_full));
     }
     if (!ok) break;
     if (first) ++ua;
@@ -881,23 +884,28 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUt
   if (threadIdx.x == 0) {
     for (int i = 0; i < 4; ++i) {
       mbar_init(smem_u32(&s.info_full[i]), 1);
-      mbar_init(smem_u32(&s.info_empty[i]), 1 + 1 + kElemWarps);  // TMA, MMA, elementwise warps
+      mbar_init(smem_u32(&s.info_empty[i]), 1 + 2 + kElemWarps);  // TMA, two MMA threads, elementwise warps
     }
     mbar_init(smem_u32(&s.a_full), 1);
-    mbar_init(smem_u32(&s.a_free), 1);
+    mbar_init(smem_u32(&s.a_free), 2);  // both MMA threads read the stationary operands
     for (int i = 0; i < kStages; ++i) {
       mbar_init(smem_u32(&s.b_full[i]), 1);
-      mbar_init(smem_u32(&s.b_empty[i]), 1);
+      mbar_init(smem_u32(&s.b_empty[i]), 2);
     }
-    mbar_init(smem_u32(&s.x_full), 1);
+    mbar_init(smem_u32(&s.x_full), 2);  // S and dP, one MMA thread each
     mbar_init(smem_u32(&s.p_full), kElemWarps);
-    mbar_init(smem_u32(&s.xy_free), 1);
-    mbar_init(smem_u32(&s.acc_full), 1);
+    mbar_init(smem_u32(&s.xy_free[0]), 1);
+    mbar_init(smem_u32(&s.xy_free[1]), 1);
+    mbar_init(smem_u32(&s.acc_full), kKV ? 2 : 1);  // dk/dv: two accumulators, one per MMA thread
     mbar_init(smem_u32(&s.acc_free), kElemWarps);
     mbar_init(smem_u32(&s.stage_free), 1);
     mbar_init(smem_u32(&s.tile_ready), kElemWarps);
     fence_barrier_init();
   }
+  // The dk/dv kernel follows the dq kernel as its programmatic dependent: it
+  // reads nothing the dq kernel writes, so its CTAs may take the SMs the dq
+  // kernel's CTAs leave (they never wait for the dq grid).
+  if (!kKV) asm volatile("griddepcontrol.launch_dependents;");
   if (warp == 8 && lane == 0) {
     tma_prefetch_desc(&tmA1);
     tma_prefetch_desc(&tmA2);
@@ -915,9 +923,11 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUt
   } else if (warp == 8) {
     producer_role<kD, kKV>(s, p, &tmA1, &tmA2, &tmB1, &tmB2);
   } else if (warp == 9) {
-    if (lane == 0) mma_role<kD, kKV>(s, p, tmem);
+    if (lane == 0) mma_role<kD, kKV, 0>(s, p, tmem);
   } else if (warp == 10) {
     prep_role<kD, kBt, kKV>(s, p);
+  } else if (warp == 11) {
+    if (lane == 0) mma_role<kD, kKV, 1>(s, p, tmem);
   }
   tc_fence_before();
   __syncthreads();
@@ -969,12 +979,21 @@ bwd_rowdot_kernel(const uint16_t* __restrict__ dout, const void* __restrict__ ou
 // 0..63 and 64..127 of global unit g of head bh are tiles 0 and nt-1 (block
 // 64: both global blocks in one unit), or the two tiles of block 0 (g = 0) or
 // of block nb-1 (block 128). d / 4 threads per row, 4 columns each; grid
-// (B*H*n_glob, 128 d / 1024).
+// (B*H*n_glob, 128 d / 1024, 3): the three gradients in one launch.
+struct SumJobs {
+  const float* part[3];
+  float* dst[3];
+  float f[3];
+};
+
 template <int kD>
 __global__ void __launch_bounds__(256)
-bwd_sum_kernel(const float* __restrict__ part, float* __restrict__ dst, int nsplit, int n_glob, int L, int nt,
-               float f) {
+bwd_sum_kernel(const __grid_constant__ SumJobs jobs, int nsplit, int n_glob, int L, int nt) {
   constexpr int kTpr = kD / 4;
+  // blockIdx.z: which gradient (dq, dv, dk)
+  const float* __restrict__ part = jobs.part[blockIdx.z];
+  float* __restrict__ dst = jobs.dst[blockIdx.z];
+  const float f = jobs.f[blockIdx.z];
   const int bh = blockIdx.x / n_glob;
   const int g = blockIdx.x % n_glob;
   const int r = blockIdx.y * (256 / kTpr) + static_cast<int>(threadIdx.x) / kTpr;
@@ -1082,12 +1101,26 @@ cudaError_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUten
   bwd_rowdot_kernel<kD><<<static_cast<unsigned>((rows + kRowsPerCta - 1) / kRowsPerCta), 256, 0, stream>>>(
       static_cast<const uint16_t*>(dout), out, out_f32, dd, rows);
   bwd_kernel<kD, kBt, false><<<grid, kThreads, smem, stream>>>(tq, tdo, tk, tv, smq, pq);
-  bwd_kernel<kD, kBt, true><<<grid, kThreads, smem, stream>>>(tk, tv, tq, tdo, smk, pk);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  // the dk/dv kernel as the dq kernel's programmatic dependent (see the kernel)
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, bwd_kernel<kD, kBt, true>, tk, tv, tq, tdo, smk, pk);
+  if (e != cudaSuccess) return e;
   if (pl.nsplit > 1) {
-    const dim3 sg(pq.BH * pl.n_glob, kRows / kRowsPerCta);
-    bwd_sum_kernel<kD><<<sg, 256, 0, stream>>>(pq.part1, dq, pl.nsplit, pl.n_glob, L, pl.nt, pq.scale);
-    bwd_sum_kernel<kD><<<sg, 256, 0, stream>>>(pk.part1, dv, pl.nsplit, pl.n_glob, L, pl.nt, 1.0f);
-    bwd_sum_kernel<kD><<<sg, 256, 0, stream>>>(pk.part2, dk, pl.nsplit, pl.n_glob, L, pl.nt, pq.scale);
+    // a normal launch: it waits for both attention kernels
+    const dim3 sg(pq.BH * pl.n_glob, kRows / kRowsPerCta, 3);
+    SumJobs jobs{{pq.part1, pk.part1, pk.part2}, {dq, dv, dk}, {pq.scale, 1.0f, pq.scale}};
+    bwd_sum_kernel<kD><<<sg, 256, 0, stream>>>(jobs, pl.nsplit, pl.n_glob, L, pl.nt);
   }
   return cudaGetLastError();
 }
