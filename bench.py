@@ -40,6 +40,10 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # launch list of the same workload (cold-cache, serialised launches: the share,
 # not the absolute, carries over to the live timing).
 FWD_KERNEL_SHARE: dict = {"bigbird_base_l4096": 103.06 / (103.06 + 8.90)}
+BWD_DRAM_BYTES_PER_LAUNCH: dict = {
+    # 163.28 MB read + 84.44 MB written, one dk/dv launch (d = 64)
+    "bigbird_base_l4096": 247.724544e6,
+}
 FWD_DRAM_BYTES_PER_LAUNCH: dict = {
     # 83.69 MB read + 12.83 MB written, split-row kernel's fp16 instance (d = 64), one launch
     "bigbird_base_l4096": 96.514304e6,
@@ -453,9 +457,9 @@ def run_bwd(args):
     value = flops / (ms * 1e-3) / 1e12
     peaks, src = _peaks()
     peak = float(peaks["bf16_tflops"])
-    # row dot, dq kernel, dk/dv kernel, and the three partial-sum launches
-    # when the global rows are split into key ranges
-    launches = 3 + (3 if bb.bwd_workspace_size(w.B, w.H, w.L) > 256 + 4 * w.B * w.H * w.L + 255 else 0)
+    # row dot, dq kernel, dk/dv kernel, and the partial-sum launch when the
+    # global rows are split into key ranges
+    launches = 3 + (1 if bb.bwd_workspace_size(w.B, w.H, w.L) > 256 + 4 * w.B * w.H * w.L + 255 else 0)
     line = {
         "metric": "block-sparse attention backward TFLOP/s (dq, dk, dv) at L=4096, 1xB200", "value": value,
         "unit": UNIT, "n_gpus": 1, "steps": steps, "warmup": args.warmup, "ms_per_step": ms,
@@ -463,8 +467,9 @@ def run_bwd(args):
         "data": "synthetic", "pass": "bwd",
         "config": _config(w, 1), "l2": L2_NOTE,
         "roofline": {"bound": "tensor", "achieved": value, "peak": peak, "unit": "TFLOP/s", "frac": value / peak,
-                     # DRAM bytes of one dk/dv launch (the larger kernel), ncu: 148.96 MB read + 78.63 MB written
-                     "traffic": 227.583744e6 if w.name == "bigbird_base_l4096" else None,
+                     # DRAM bytes of one dk/dv launch (the larger kernel), from an ncu capture of
+                     # the current source (None until one is taken)
+                     "traffic": BWD_DRAM_BYTES_PER_LAUNCH.get(w.name),
                      "kernel": "bwd_kernel<dq> + bwd_kernel<dk,dv> (tcgen05, bf16 operands); the duration is the "
                                "whole call (row dot and partial sums included), the work the algorithmic 5 GEMM-"
                                "shaped products; traffic is the dk/dv kernel's",
