@@ -946,33 +946,42 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUt
   }
 }
 
-// D[row] = sum_c dout[row, c] * out[row, c]: d / 4 threads per row, 4
-// columns each; a CTA of 256 threads covers 1024 / d rows.
+// D[row] = sum_c dout[row, c] * out[row, c]: d / 8 threads per row, 8
+// columns (16 bytes of each bf16 operand) each; a CTA of 256 threads covers
+// 2048 / d rows.
 template <int kD>
 __global__ void __launch_bounds__(256)
 bwd_rowdot_kernel(const uint16_t* __restrict__ dout, const void* __restrict__ out, int out_f32, float* __restrict__ dd,
                   size_t rows) {
-  constexpr int kTpr = kD / 4;
+  constexpr int kTpr = kD / 8;
   const size_t row = static_cast<size_t>(blockIdx.x) * (256 / kTpr) + threadIdx.x / kTpr;
-  const int c4 = threadIdx.x % kTpr;
+  const int c8 = threadIdx.x % kTpr;
   float acc = 0.f;
   if (row < rows) {
-    const uint2 g = __ldg(reinterpret_cast<const uint2*>(dout + row * kD) + c4);
-    float o[4];
+    const uint4 g = __ldg(reinterpret_cast<const uint4*>(dout + row * kD) + c8);
+    float o[8];
     if (out_f32) {
-      const float4 t = __ldg(reinterpret_cast<const float4*>(static_cast<const float*>(out) + row * kD) + c4);
-      o[0] = t.x; o[1] = t.y; o[2] = t.z; o[3] = t.w;
+      const float4* src = reinterpret_cast<const float4*>(static_cast<const float*>(out) + row * kD) + 2 * c8;
+      const float4 t0 = __ldg(src), t1 = __ldg(src + 1);
+      o[0] = t0.x; o[1] = t0.y; o[2] = t0.z; o[3] = t0.w;
+      o[4] = t1.x; o[5] = t1.y; o[6] = t1.z; o[7] = t1.w;
     } else {
-      const uint2 t = __ldg(reinterpret_cast<const uint2*>(static_cast<const uint16_t*>(out) + row * kD) + c4);
-      o[0] = __uint_as_float(t.x << 16); o[1] = __uint_as_float(t.x & 0xFFFF0000u);
-      o[2] = __uint_as_float(t.y << 16); o[3] = __uint_as_float(t.y & 0xFFFF0000u);
+      const uint4 t = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(out) + row * kD) + c8);
+      const uint32_t w[4] = {t.x, t.y, t.z, t.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        o[2 * i] = __uint_as_float(w[i] << 16);
+        o[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+      }
     }
-    acc = __uint_as_float(g.x << 16) * o[0] + __uint_as_float(g.x & 0xFFFF0000u) * o[1] +
-          __uint_as_float(g.y << 16) * o[2] + __uint_as_float(g.y & 0xFFFF0000u) * o[3];
+    const uint32_t gw[4] = {g.x, g.y, g.z, g.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      acc += __uint_as_float(gw[i] << 16) * o[2 * i] + __uint_as_float(gw[i] & 0xFFFF0000u) * o[2 * i + 1];
   }
 #pragma unroll
   for (int off = kTpr / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-  if (row < rows && c4 == 0) dd[row] = acc;
+  if (row < rows && c8 == 0) dd[row] = acc;
 }
 
 // The split global units' partial sums, dst = f * sum over the ranges. Rows
@@ -1097,8 +1106,9 @@ cudaError_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUten
   using namespace bbw;
   const int grid = std::min(pq.total_units, BGeo<kD>::kCtasPerSm * sms);
   const size_t smem = smem_request<kD>();
-  constexpr int kRowsPerCta = 256 / (kD / 4);
-  bwd_rowdot_kernel<kD><<<static_cast<unsigned>((rows + kRowsPerCta - 1) / kRowsPerCta), 256, 0, stream>>>(
+  constexpr int kRowsPerCta = 256 / (kD / 4);        // partial sums: d / 4 threads per row
+  constexpr int kDotRowsPerCta = 256 / (kD / 8);     // row dot: d / 8 threads per row
+  bwd_rowdot_kernel<kD><<<static_cast<unsigned>((rows + kDotRowsPerCta - 1) / kDotRowsPerCta), 256, 0, stream>>>(
       static_cast<const uint16_t*>(dout), out, out_f32, dd, rows);
   bwd_kernel<kD, kBt, false><<<grid, kThreads, smem, stream>>>(tq, tdo, tk, tv, smq, pq);
   cudaError_t e = cudaGetLastError();
