@@ -203,6 +203,14 @@ constexpr uint32_t kColOa = 128;
 constexpr uint32_t kColOb = 192;
 constexpr uint32_t kTmemCols2 = 256;
 
+// TMA store maps of the split-row kernel's output tiles: `out` (bf16 with
+// 64x64 boxes, or fp32 with 64-row x 32-column boxes) and the ranges'
+// partial outputs (fp32, 64-row x 32-column boxes).
+struct OutMaps {
+  CUtensorMap out;
+  CUtensorMap part;
+};
+
 struct __align__(1024) SharedStorage2 {
   static constexpr int kDim = 64;
   static constexpr int kQBufs = 2;  // the next unit's Q loads while this unit runs
@@ -217,7 +225,10 @@ struct __align__(1024) SharedStorage2 {
   uint8_t q[kQBufs][kRows * 64 * 2];
   uint8_t k[kKSt][kBlock * 64 * 2];
   uint8_t v[kVSt][kBlock * 64 * 2];  // converted to fp16 in place
-  uint8_t ostage[kRows * 64 * 2];    // a unit's bf16 output tile (two 64-row TMA boxes, 128-byte swizzle)
+  // a unit's output tile on its way out through TMA stores (128-byte swizzle):
+  // bf16, two boxes of 64 rows x 64 columns; or fp32 (fp32 output, or the
+  // partial result of a global-row range), four boxes of 64 rows x 32 columns
+  uint8_t ostage[kRows * 64 * 4];
   UnitInfo unit[4];
   float2 mlx[2][2][kRows];  // (max, sum) per unit parity, column half, row: the halves' combine
   uint64_t info_full[4];
@@ -1014,7 +1025,7 @@ __device__ void mma2_role(SharedStorage2& s, const FwdParams& p, uint32_t tmem) 
 // of a row exchange (max, sum) through shared memory; each writes 32 of the
 // row's output columns, O_a and O_b scaled to the common max.
 template <bool kBf16>
-__device__ void softmax2_role(SharedStorage2& s, const FwdParams& p, uint32_t tmem, const CUtensorMap* tmO) {
+__device__ void softmax2_role(SharedStorage2& s, const FwdParams& p, uint32_t tmem, const OutMaps* tmO) {
   const int wid = threadIdx.x >> 5;  // 0..7
   const int h = wid >> 2;            // key half of each block
   const int row = threadIdx.x & 127; // TMEM lane == row of the unit
@@ -1113,37 +1124,26 @@ __device__ void softmax2_role(SharedStorage2& s, const FwdParams& p, uint32_t tm
     const float fb = ex2_approx(B.x - m);
     const float l = A.y * fa + B.y * fb;
     const int c_base = 32 * h;
-    if (split >= 0) {
-      const size_t base = (static_cast<size_t>(bh) * p.nparts + split) * kRows + row;
-#pragma unroll 1
-      for (int c0 = 0; c0 < 32; c0 += 16) {
-        uint32_t oa[16], ob[16];
-        tmem_ld16(lane_addr + kColOa + c_base + c0, oa);
-        tmem_ld16(lane_addr + kColOb + c_base + c0, ob);
-        tmem_wait_ld();
-        float4* dst = reinterpret_cast<float4*>(p.part_o + base * 64 + c_base + c0);
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-          dst[c] = make_float4(__uint_as_float(oa[4 * c]) * fa + __uint_as_float(ob[4 * c]) * fb,
-                               __uint_as_float(oa[4 * c + 1]) * fa + __uint_as_float(ob[4 * c + 1]) * fb,
-                               __uint_as_float(oa[4 * c + 2]) * fa + __uint_as_float(ob[4 * c + 2]) * fb,
-                               __uint_as_float(oa[4 * c + 3]) * fa + __uint_as_float(ob[4 * c + 3]) * fb);
-      }
-      if (h == 0) reinterpret_cast<float2*>(p.part_ml)[base] = make_float2(m, l);
-      if (kBf16) {
-        // the bf16 instance merges inside its own grid: count this warp's rows of the partial as written
-        __syncwarp();
-        if (lane == 0) {
-          __threadfence();
-          atomicAdd(&p.counters[kCtrParts], 1);
+    if (split >= 0 || p.out_f32) {
+      // fp32 (a range's partial result, or fp32 output): each thread puts its
+      // 32 columns (eight 16-byte chunks, one 128-byte box row) into ostage,
+      // swizzled as the tensor map expects; warp 0 then stores the tile's
+      // boxes with TMA.
+      const bool has = split >= 0 || exists;
+      if (has) {
+        const float inv = split >= 0 ? 1.f : 1.f / l;  // a partial stays unnormalised
+        if (split >= 0) {
+          if (h == 0) {
+            const size_t base = (static_cast<size_t>(bh) * p.nparts + split) * kRows + row;
+            reinterpret_cast<float2*>(p.part_ml)[base] = make_float2(m, l);
+          }
+        } else if (h == 0 && p.lse) {
+          const size_t orow = static_cast<size_t>(bh) * p.L + static_cast<size_t>(qblk) * kBlock + (row & 63);
+          // log sum_k exp(s_k) = ln 2 * (m + log2 l), the scores in log2 units being s * log2(e).
+          p.lse[orow] = (m + log2f(l)) * 0.69314718055994531f;
         }
-      }
-    } else if (p.out_f32) {
-      if (exists) {
-        const float inv = 1.f / l;
-        const size_t orow = static_cast<size_t>(bh) * p.L + static_cast<size_t>(qblk) * kBlock + (row & 63);
-        // log sum_k exp(s_k) = ln 2 * (m + log2 l), the scores in log2 units being s * log2(e).
-        if (h == 0 && p.lse) p.lse[orow] = (m + log2f(l)) * 0.69314718055994531f;
+        const int rr = row & 63;
+        uint8_t* srow = s.ostage + ((row >> 6) * 2 + h) * (kBlock * 128) + rr * 128;
 #pragma unroll 1
         for (int c0 = 0; c0 < 32; c0 += 16) {
           uint32_t oa[16], ob[16];
@@ -1151,11 +1151,51 @@ __device__ void softmax2_role(SharedStorage2& s, const FwdParams& p, uint32_t tm
           tmem_ld16(lane_addr + kColOb + c_base + c0, ob);
           tmem_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 16; ++i)
-            oa[i] = __float_as_uint(__uint_as_float(oa[i]) * fa + __uint_as_float(ob[i]) * fb);
-          store16<64>(p, orow, c_base + c0, oa, inv);
+          for (int j = 0; j < 4; ++j) {
+            const int cc = (c0 >> 2) + j;  // 16-byte chunk (four floats) of the box row
+            *reinterpret_cast<float4*>(srow + ((cc ^ (rr & 7)) << 4)) =
+                make_float4((__uint_as_float(oa[4 * j]) * fa + __uint_as_float(ob[4 * j]) * fb) * inv,
+                            (__uint_as_float(oa[4 * j + 1]) * fa + __uint_as_float(ob[4 * j + 1]) * fb) * inv,
+                            (__uint_as_float(oa[4 * j + 2]) * fa + __uint_as_float(ob[4 * j + 2]) * fb) * inv,
+                            (__uint_as_float(oa[4 * j + 3]) * fa + __uint_as_float(ob[4 * j + 3]) * fb) * inv);
+          }
         }
       }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&s.tile_ready));
+      if (wid == 0) {
+        if (!warp_wait(smem_u32(&s.tile_ready), staged & 1)) { flag_timeout(s, p); return; }
+        if (lane == 0) {
+          const CUtensorMap* map = split >= 0 ? &tmO->part : &tmO->out;
+          int32_t y0, y1;
+          if (split >= 0) {
+            y0 = (bh * p.nparts + split) * kRows;
+            y1 = y0 + kBlock;
+          } else {
+            y0 = bh * p.L + qtop * kBlock;
+            y1 = qbot >= 0 ? bh * p.L + qbot * kBlock : -1;
+          }
+          const uint32_t src = smem_u32(s.ostage);
+          tma_store_2d(map, src, 0, y0);
+          tma_store_2d(map, src + kBlock * 128, 32, y0);
+          if (y1 >= 0) {
+            tma_store_2d(map, src + 2 * kBlock * 128, 0, y1);
+            tma_store_2d(map, src + 3 * kBlock * 128, 32, y1);
+          }
+          bulk_commit();
+          if (kBf16 && split >= 0) {
+            // the bf16 instance merges inside its own grid: count the range's
+            // partial as written once the stores have completed (eight
+            // softmax warps' rows; the (max, sum) pairs were written before
+            // tile_ready)
+            bulk_wait_all();
+            __threadfence();
+            atomicAdd(&p.counters[kCtrParts], SharedStorage2::kSoftmaxWarps);
+          }
+        }
+      }
+      ++staged;
     } else {
       // bf16 output: each thread puts its 32 columns (four 16-byte chunks of
       // its 128-byte row) into ostage, swizzled as the tensor map expects;
@@ -1191,8 +1231,8 @@ __device__ void softmax2_role(SharedStorage2& s, const FwdParams& p, uint32_t tm
         if (!warp_wait(smem_u32(&s.tile_ready), staged & 1)) { flag_timeout(s, p); return; }
         if (lane == 0) {
           const int32_t row0 = bh * p.L;
-          tma_store_2d(tmO, smem_u32(s.ostage), 0, row0 + qtop * kBlock);
-          if (qbot >= 0) tma_store_2d(tmO, smem_u32(s.ostage) + kBlock * 128, 0, row0 + qbot * kBlock);
+          tma_store_2d(&tmO->out, smem_u32(s.ostage), 0, row0 + qtop * kBlock);
+          if (qbot >= 0) tma_store_2d(&tmO->out, smem_u32(s.ostage) + kBlock * 128, 0, row0 + qbot * kBlock);
           bulk_commit();
         }
       }
@@ -1411,7 +1451,7 @@ bigbird_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
 template <bool kBf16>
 __global__ void __launch_bounds__(kThreads2, 2)
 bigbird_fwd2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ OutMaps tmO,
                     const FwdParams p) {
   extern __shared__ uint8_t smem_raw[];
   SharedStorage2& s =
@@ -1472,7 +1512,8 @@ bigbird_fwd2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     tma_prefetch_desc(&tmQ);
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
-    if (!p.out_f32) tma_prefetch_desc(&tmO);
+    tma_prefetch_desc(&tmO.out);
+    if (p.nsplit > 1) tma_prefetch_desc(&tmO.part);
   }
   tc_fence_before();
   __syncthreads();
@@ -1720,7 +1761,7 @@ static cudaError_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, cons
 // The d = 64 launches: the split-row kernel's fp16 instance, then its bf16
 // instance as the programmatic dependent (as in launch_fwd).
 static cudaError_t launch_fwd2(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                               const CUtensorMap& to, const FwdParams& p, int sms, cudaStream_t stream) {
+                               const OutMaps& to, const FwdParams& p, int sms, cudaStream_t stream) {
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
@@ -1787,15 +1828,9 @@ static int fwd_impl(const void* q, const void* k, const void* v, const int32_t* 
     if (vs != BB_OK) return vs;
   }
 
-  CUtensorMap tq, tk, tv, to;
+  CUtensorMap tq, tk, tv;
   const uint64_t rows = static_cast<uint64_t>(B) * H * L;
   if (!make_map(&tq, q, rows, d) || !make_map(&tk, k, rows, d) || !make_map(&tv, v, rows, d)) return BB_ERR_CUDA;
-  // the bf16 output at d = 64 leaves through TMA stores (64-row boxes, like Q)
-  if (d == 64 && out_dtype != BB_OUT_F32) {
-    if (!make_map(&to, out, rows, 64)) return BB_ERR_CUDA;
-  } else {
-    to = tq;  // not used
-  }
 
   FwdParams p{};
   p.q = static_cast<const uint16_t*>(q);
@@ -1850,8 +1885,18 @@ static int fwd_impl(const void* q, const void* k, const void* v, const int32_t* 
     p.part_o = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + kCounterBytes);
     p.part_ml = p.part_o + static_cast<size_t>(p.BH) * p.nparts * kRows * d;
   }
-  const cudaError_t e = d == 64 ? launch_fwd2(tq, tk, tv, to, p, di->sms, stream)
-                                : launch_fwd<128>(tq, tk, tv, p, di->sms, stream);
+  cudaError_t e = cudaSuccess;
+  if (d == 64) {
+    // the split-row kernel's output tiles leave through TMA stores: out (bf16
+    // 64x64 boxes, or fp32 64-row x 32-column boxes) and the ranges' partials
+    OutMaps om;
+    bool ok = p.out_f32 ? make_f32_map(&om.out, out, rows) : make_map(&om.out, out, rows, 64);
+    if (ok && pl.nsplit > 1) ok = make_f32_map(&om.part, p.part_o, static_cast<uint64_t>(p.BH) * p.nparts * kRows);
+    else om.part = om.out;  // not used
+    e = ok ? launch_fwd2(tq, tk, tv, om, p, di->sms, stream) : cudaErrorInvalidValue;
+  } else {
+    e = launch_fwd<128>(tq, tk, tv, p, di->sms, stream);
+  }
   if (owned) cudaFreeAsync(ws, stream);
   return e == cudaSuccess ? BB_OK : BB_ERR_CUDA;
 }
