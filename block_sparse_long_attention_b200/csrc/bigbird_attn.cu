@@ -79,7 +79,6 @@ constexpr int kMaxList = 42;           // key tiles per unit
 constexpr int kMaxR = 16;              // random blocks per row supported
 constexpr int kSplitBlocks = 8;        // key tiles per global-row range
 constexpr int kThreads = 256;
-constexpr uint32_t kColS = 0;          // S of one key tile: 64 fp32 columns; P (16-bit) overwrites the first 32
 constexpr uint32_t kColO = 64;         // O: d fp32 columns
 constexpr uint32_t kChunkBytes = kBlock * 64 * 2;  // 64 rows x 64 columns bf16: one TMA box, one 128-byte swizzle span
 
@@ -95,6 +94,11 @@ struct Geo {
   // per SM: four at d = 64, two at d = 128 (TMEM and shared memory)
   static constexpr uint32_t kTmemCols = kD == 64 ? 128 : 256;
   static constexpr int kCtasPerSm = kD == 64 ? 4 : 2;
+  // S buffers of bigbird_fwd_kernel: at d = 128 the second one sits in the 64
+  // columns after O (S(g+1) is computed while the softmax works on block g);
+  // at d = 64 there is one
+  static constexpr int kSBufs = kD == 128 ? 2 : 1;
+  __host__ __device__ static constexpr uint32_t s_col(uint32_t g) { return (kSBufs == 2 && (g & 1)) ? 192u : 0u; }
 };
 // The reference max moves only when a score exceeds it by more than 2^14: P
 // (fp16, largest finite 65504) then stays <= 2^14 with headroom, and the
@@ -182,9 +186,9 @@ struct __align__(1024) SharedStorage {
   uint64_t v_full[kVStages];
   uint64_t v_conv[kVStages];
   uint64_t v_empty[kVStages];
-  uint64_t s_full;   // S of the current key block is in TMEM
-  uint64_t p_full;   // P of the current key block is in TMEM (4 softmax warps)
-  uint64_t pv_done;  // P.V of the current key block is complete (S/P columns reusable)
+  uint64_t s_full[2];   // S(g) is in S buffer g & 1
+  uint64_t p_full[2];   // P(g) is in S buffer g & 1 (4 softmax warps)
+  uint64_t pv_done[2];  // P.V(g) is complete (S buffer g & 1 reusable)
   uint64_t o_full;
   uint64_t o_free;
   uint32_t tmem_base;
@@ -656,11 +660,36 @@ __device__ void producer_role(S& s, const FwdParams& p, const CUtensorMap* tmQ, 
 // CTA; the four CTAs of an SM interleave on the tensor pipe.
 template <int kD, bool kBf16>
 __device__ void mma_role(SharedStorage<kD>& s, const FwdParams& p, uint32_t tmem) {
+  using Gm = Geo<kD>;
+  constexpr int kB = Gm::kSBufs;
   const uint32_t idesc_s = idesc_f32acc(kRows, kBlock, true, false);    // bf16 Q . K^T, N = 64
   // fp16 P . fp16 V, or bf16 P . bf16 V in the bf16 instance; N = 64 per chunk of d
   const uint32_t idesc_o = idesc_f32acc(kRows, 64, kBf16, true);
   const uint32_t q_addr = smem_u32(s.q[0]);
+  // P.V of block gb (first / last block of its unit ut)
+  auto issue_pv = [&](uint32_t gb, bool first, bool last, uint32_t put) -> bool {
+    const int vst = gb % kVStages;
+    // the V tile: converted (fp16), or as loaded (bf16 instance)
+    if (!mbar_wait(smem_u32(kBf16 ? &s.v_full[vst] : &s.v_conv[vst]), (gb / kVStages) & 1)) return false;
+    if (first && !mbar_wait(smem_u32(&s.o_free), (put & 1) ^ 1)) return false;
+    if (!mbar_wait(smem_u32(&s.p_full[gb % kB]), (gb / kB) & 1)) return false;
+    tc_fence_after();
+    const uint32_t v_addr = smem_u32(s.v[vst]);
+    // O columns 64 c .. 64 c + 63 from V chunk c; K = 64 keys in steps of 16
+#pragma unroll
+    for (int c = 0; c < Gm::kChunks; ++c)
+#pragma unroll
+      for (int kk = 0; kk < kBlock / 16; ++kk)
+        mma_ts(tmem + kColO + 64 * c, tmem + Gm::s_col(gb) + kk * 8,
+               sdesc_sw128(v_addr + c * kChunkBytes + kk * 2048, 8192, 1024), idesc_o, (!first || kk > 0) ? 1u : 0u);
+    mma_commit(smem_u32(&s.pv_done[gb % kB]));
+    mma_commit(smem_u32(&s.v_empty[vst]));
+    if (last) mma_commit(smem_u32(&s.o_full));
+    return true;
+  };
   uint32_t g = 0;
+  bool pend = false, pend_first = false, pend_last = false;
+  uint32_t pend_ut = 0;
   bool ok = true;
   for (uint32_t ut = 0; ok; ++ut) {
     if (!mbar_wait(smem_u32(&s.info_full[ut & 3]), (ut >> 2) & 1)) { ok = false; break; }
@@ -670,38 +699,35 @@ __device__ void mma_role(SharedStorage<kD>& s, const FwdParams& p, uint32_t tmem
     for (int e = 0; e < n; ++e, ++g) {
       const int kst = g % kKStages;
       if (!mbar_wait(smem_u32(&s.k_full[kst]), (g / kKStages) & 1)) { ok = false; break; }
-      if (g >= 1 && !mbar_wait(smem_u32(&s.pv_done), (g - 1) & 1)) { ok = false; break; }
+      // S(g) overwrites the P that P.V(g - kB) reads
+      if (g >= kB && !mbar_wait(smem_u32(&s.pv_done[g % kB]), ((g / kB) - 1) & 1)) { ok = false; break; }
       tc_fence_after();
       const uint32_t k_addr = smem_u32(s.k[kst]);
       // K = d in steps of 16: four steps (32 bytes apart) per 64-column chunk
 #pragma unroll
       for (int kk = 0; kk < kD / 16; ++kk)
-        mma_ss(tmem + kColS, sdesc_sw128(q_addr + (kk >> 2) * Geo<kD>::kQChunkBytes + (kk & 3) * 32, 16, 1024),
+        mma_ss(tmem + Gm::s_col(g), sdesc_sw128(q_addr + (kk >> 2) * Gm::kQChunkBytes + (kk & 3) * 32, 16, 1024),
                sdesc_sw128(k_addr + (kk >> 2) * kChunkBytes + (kk & 3) * 32, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
-      mma_commit(smem_u32(&s.s_full));
+      mma_commit(smem_u32(&s.s_full[g % kB]));
       mma_commit(smem_u32(&s.k_empty[kst]));
       if (e == n - 1) mma_commit(smem_u32(&s.q_free[0]));
-      const int vst = g % kVStages;
-      // the V tile: converted (fp16), or as loaded (bf16 instance)
-      if (!mbar_wait(smem_u32(kBf16 ? &s.v_full[vst] : &s.v_conv[vst]), (g / kVStages) & 1)) { ok = false; break; }
-      if (e == 0 && !mbar_wait(smem_u32(&s.o_free), (ut & 1) ^ 1)) { ok = false; break; }
-      if (!mbar_wait(smem_u32(&s.p_full), g & 1)) { ok = false; break; }
-      tc_fence_after();
-      const uint32_t v_addr = smem_u32(s.v[vst]);
-      // O columns 64 c .. 64 c + 63 from V chunk c; K = 64 keys in steps of 16
-#pragma unroll
-      for (int c = 0; c < Geo<kD>::kChunks; ++c)
-#pragma unroll
-        for (int kk = 0; kk < kBlock / 16; ++kk)
-          mma_ts(tmem + kColO + 64 * c, tmem + kColS + kk * 8,
-                 sdesc_sw128(v_addr + c * kChunkBytes + kk * 2048, 8192, 1024), idesc_o, (e > 0 || kk > 0) ? 1u : 0u);
-      mma_commit(smem_u32(&s.pv_done));
-      mma_commit(smem_u32(&s.v_empty[vst]));
-      if (e == n - 1) mma_commit(smem_u32(&s.o_full));
+      if (kB == 1) {
+        // one S buffer: P.V(g) right behind S(g)
+        if (!issue_pv(g, e == 0, e == n - 1, ut)) { ok = false; break; }
+      } else {
+        // two: S(g) goes out before P.V(g - 1), so that it is ready when the
+        // softmax finishes block g - 1
+        if (pend && !issue_pv(g - 1, pend_first, pend_last, pend_ut)) { ok = false; break; }
+        pend = true;
+        pend_first = e == 0;
+        pend_last = e == n - 1;
+        pend_ut = ut;
+      }
     }
     if (!ok) break;
     mbar_arrive(smem_u32(&s.info_empty[ut & 3]));
   }
+  if (ok && pend && !issue_pv(g - 1, pend_first, pend_last, pend_ut)) ok = false;
   if (!ok) flag_timeout(s, p);
 }
 
@@ -818,7 +844,7 @@ __device__ void softmax_role(SharedStorage<kD>& s, const FwdParams& p, uint32_t 
   const int lane = tid & 31;
   const int half = warp >> 1;   // 0: rows 0..63, 1: rows 64..127
   const uint32_t lane_addr = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-  const uint32_t s_addr = lane_addr + kColS;
+  constexpr int kB = Geo<kD>::kSBufs;
   const uint64_t scale2 = f2_pack(p.scale_log2, p.scale_log2);
   uint32_t g = 0;
   for (uint32_t ut = 0;; ++ut) {
@@ -834,8 +860,9 @@ __device__ void softmax_role(SharedStorage<kD>& s, const FwdParams& p, uint32_t 
     float l_run = 0.f;
     for (int e = 0; e < n; ++e, ++g) {
       const bool used = exists && ((ui.hm[e] >> half) & 1);
-      if (!warp_wait(smem_u32(&s.s_full), g & 1)) { flag_timeout(s, p); return; }
+      if (!warp_wait(smem_u32(&s.s_full[g % kB]), (g / kB) & 1)) { flag_timeout(s, p); return; }
       tc_fence_after();
+      const uint32_t s_addr = lane_addr + Geo<kD>::s_col(g);
       if (used) {
         const uint64_t vm = ui.vm[e];
         const bool mixed = block_mixed(vm);
@@ -885,7 +912,7 @@ __device__ void softmax_role(SharedStorage<kD>& s, const FwdParams& p, uint32_t 
         // O holds the P.V of the earlier blocks (none yet for e == 0: the
         // first P.V of the unit overwrites O); rescale it once that P.V is done.
         if (e > 0 && __any_sync(0xffffffffu, o_factor != 1.f)) {
-          if (!warp_wait(smem_u32(&s.pv_done), (g - 1) & 1)) { flag_timeout(s, p); return; }
+          if (!warp_wait(smem_u32(&s.pv_done[(g - 1) % kB]), ((g - 1) / kB) & 1)) { flag_timeout(s, p); return; }
           tc_fence_after();
           rescale_o<kD>(lane_addr + kColO, o_factor);
         }
@@ -900,7 +927,7 @@ __device__ void softmax_role(SharedStorage<kD>& s, const FwdParams& p, uint32_t 
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&s.p_full));
+      if (lane == 0) mbar_arrive(smem_u32(&s.p_full[g % kB]));
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(smem_u32(&s.info_empty[ut & 3]));
@@ -1367,9 +1394,11 @@ bigbird_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       mbar_init(smem_u32(&s.v_conv[i]), 1);
       mbar_init(smem_u32(&s.v_empty[i]), 1);
     }
-    mbar_init(smem_u32(&s.s_full), 1);
-    mbar_init(smem_u32(&s.p_full), 4);
-    mbar_init(smem_u32(&s.pv_done), 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(&s.s_full[i]), 1);
+      mbar_init(smem_u32(&s.p_full[i]), 4);
+      mbar_init(smem_u32(&s.pv_done[i]), 1);
+    }
     mbar_init(smem_u32(&s.o_full), 1);
     mbar_init(smem_u32(&s.o_free), 4);
     s.abort_flag = 0;
