@@ -55,15 +55,15 @@ using namespace bb;
 
 constexpr int kBlock = 64;     // tokens per tile: a block of 64, or half a block of 128
 constexpr int kRows = 128;     // stationary rows per unit (two tiles)
-constexpr int kStages = 2;     // moving-tile ring depth
 constexpr int kMaxList = 42;   // moving tiles per unit chunk
 constexpr int kMaxR = 16;
 constexpr int kSplit = 8;      // tiles per range of a global unit
 constexpr int kThreads = 384;  // warps 0-7 elementwise, 8 TMA, 9 and 11 MMA, 10 prep
 constexpr int kElemWarps = 8;
 constexpr uint32_t kChunkBytes = kBlock * 64 * 2;  // 64 rows x 64 columns bf16: one TMA box
-constexpr uint32_t kColX = 0;     // S (or S^T): 64 fp32 columns; then P_hi and P_lo (bf16 pairs)
-constexpr uint32_t kColY = 64;    // dP (or dP^T): 64 fp32 columns; then dS_hi and dS_lo
+// TMEM columns: S (or S^T) of a step, 64 fp32 columns, then P_hi and P_lo
+// (bf16 pairs) over them; dP (or dP^T) in the next 64, then dS_hi and dS_lo
+// (BGeo::x_col gives the S columns of each buffer); the accumulators:
 constexpr uint32_t kColA1 = 128;  // dQ, or dV: d fp32 columns; dK follows
 
 // Sizes that follow from the head dimension d (64 or 128): a row of d values
@@ -79,7 +79,16 @@ struct BGeo {
   static constexpr uint32_t kAChunkBytes = kRows * 64 * 2;
   static constexpr int kCtasPerSm = kD == 64 ? 2 : 1;
   static constexpr uint32_t kColA2 = kColA1 + kD;
-  __host__ __device__ static constexpr uint32_t tmem_cols(bool kv) { return kD == 64 ? 256u : (kv ? 512u : 256u); }
+  // At d = 128 (one CTA per SM) S and dP are double-buffered: step g uses
+  // buffer g % 2, the second pair in the columns after the accumulators, so
+  // the next step's S and dP are computed while the elementwise warps work on
+  // this one; the moving-tile ring is then three deep (a stage stays in use
+  // until the previous step's gradient MMAs are complete).
+  static constexpr int kBufs = kD == 128 ? 2 : 1;
+  static constexpr int kStages = kD == 128 ? 3 : 2;
+  __host__ __device__ static constexpr uint32_t tmem_cols(bool) { return kD == 64 ? 256u : 512u; }
+  // S (X) columns of buffer b; dP (Y) follow at + 64
+  __host__ __device__ static constexpr uint32_t x_col(uint32_t b, bool kv) { return b == 0 ? 0u : (kv ? 384u : 256u); }
 };
 constexpr int kSmemRequest64 = 112 * 1024;
 
@@ -144,21 +153,21 @@ template <int kD>
 struct __align__(1024) Smem {
   uint8_t a1[kRows * kD * 2];                   // Q (dq) or K (dk/dv) of the unit: two tiles
   uint8_t a2[kRows * kD * 2];                   // dO (dq) or V (dk/dv)
-  uint8_t b1[kStages][BGeo<kD>::kTileBytes];    // K (dq) or Q (dk/dv) of a step
-  uint8_t b2[kStages][BGeo<kD>::kTileBytes];    // V (dq) or dO (dk/dv)
+  uint8_t b1[BGeo<kD>::kStages][BGeo<kD>::kTileBytes];    // K (dq) or Q (dk/dv) of a step
+  uint8_t b2[BGeo<kD>::kStages][BGeo<kD>::kTileBytes];    // V (dq) or dO (dk/dv)
   // d = 64: one fp32 accumulator tile of the unit (four boxes of 64 rows x
   // 32 columns, 128-byte swizzle) on its way out through TMA stores
   uint8_t ostage[kD == 64 ? kRows * 64 * 4 : 1024];
-  float col_lse[kStages][kBlock];         // dk/dv: lse and D of the step's query tile
-  float col_d[kStages][kBlock];
+  float col_lse[BGeo<kD>::kStages][kBlock];         // dk/dv: lse and D of the step's query tile
+  float col_d[BGeo<kD>::kStages][kBlock];
   Unit unit[4];
   uint64_t info_full[4];
   uint64_t info_empty[4];
   uint64_t a_full, a_free;
-  uint64_t b_full[kStages], b_empty[kStages];
-  uint64_t x_full;     // S and dP of the step are in TMEM
-  uint64_t p_full;     // P and dS written (4 warps)
-  uint64_t xy_free[2]; // a part's gradient MMAs of the step are complete (its columns reusable)
+  uint64_t b_full[BGeo<kD>::kStages], b_empty[BGeo<kD>::kStages];
+  uint64_t x_full[2];     // S and dP of step g are in TMEM buffer g % kBufs
+  uint64_t p_full[2];     // P and dS of step g written (elementwise warps)
+  uint64_t xy_free[2][2]; // [part][buffer]: a part's gradient MMAs of the step are complete
   uint64_t acc_full;   // a unit's accumulators are complete
   uint64_t acc_free;   // ... and read by the epilogue (4 warps)
   uint64_t stage_free; // d = 64: ostage may be written (the previous tile's stores have read it)
@@ -525,8 +534,8 @@ __device__ void producer_role(Smem<kD>& s, const Params& p, const CUtensorMap* t
         ++ua;
       }
       for (int e = 0; e < ui.n && ok; ++e, ++g) {
-        const int st = g % kStages;
-        ok = mbar_wait(smem_u32(&s.b_empty[st]), ((g / kStages) & 1) ^ 1);
+        const int st = g % BGeo<kD>::kStages;
+        ok = mbar_wait(smem_u32(&s.b_empty[st]), ((g / BGeo<kD>::kStages) & 1) ^ 1);
         if (!ok) break;
         const uint32_t bar = smem_u32(&s.b_full[st]);
         const int32_t row = row0 + ui.mt[e] * kBlock;
@@ -565,18 +574,58 @@ __device__ void producer_role(Smem<kD>& s, const Params& p, const CUtensorMap* t
 template <int kD, bool kKV, int kPart>
 __device__ void mma_role(Smem<kD>& s, const Params& p, uint32_t tmem) {
   using G = BGeo<kD>;
+  constexpr int kSt = G::kStages;
+  constexpr int kNB = G::kBufs;
   // Two issuing threads (warps 9 and 11), each with its own products:
   //   dk/dv: part 0 S^T -> dV += P^T dO;  part 1 dP^T -> dK += dS^T Q;
   //   dq:    part 0 S   -> dQ += dS K;     part 1 dP.
-  // A part reuses its S or dP columns once its own gradient MMAs that read
-  // them are complete (dk/dv: xy_free[part]; dq: dP waits for dQ, xy_free[0],
-  // while S's columns are read by no MMA and free once P(g) is written).
+  // A part reuses its S or dP columns (buffer g % kNB) once the gradient MMAs
+  // that read them, kNB steps back, are complete (dk/dv: its own,
+  // xy_free[part]; dq: dP waits for dQ, xy_free[0], while S's columns are
+  // read by no MMA and free once P is written). With two buffers a step's S
+  // and dP go out before the previous step's gradient MMAs.
   constexpr bool kHasGrad = kKV || kPart == 0;
   const uint32_t idesc1 = idesc_f32acc(kRows, kBlock, true, false);
   const uint32_t idesc2 = idesc_f32acc(kRows, 64, true, true);  // one 64-column chunk of d
   const uint32_t a_src = smem_u32(kPart == 0 ? s.a1 : s.a2);
-  const uint32_t x_col = kPart == 0 ? kColX : kColY;  // this part's S or dP columns
+  // gradient MMAs of step gb (zero: its unit's first step, the accumulator is
+  // overwritten once the unit before has been read out, acc_free phase uab;
+  // last: its unit's last step), then the moving stage is released
+  auto issue_grad = [&](uint32_t gb, bool zero, bool last, uint32_t uab) -> bool {
+    const int st = gb % kSt;
+    const uint32_t bb = gb % kNB;
+    if (kHasGrad) {
+      if (zero && !mbar_wait(smem_u32(&s.acc_free), (uab & 1) ^ 1)) return false;
+      if (!mbar_wait(smem_u32(&s.p_full[bb]), (gb / kNB) & 1)) return false;
+      tc_fence_after();
+      const uint32_t b1 = smem_u32(s.b1[st]), b2 = smem_u32(s.b2[st]);
+      // dk/dv part 0: dV += (P_hi + P_lo) dO (P in the S columns, B = b2);
+      // dk/dv part 1: dK += (dS_hi + dS_lo) Q (dS in the dP columns, B = b1);
+      // dq: dQ += (dS_hi + dS_lo) K (dS in the dP columns, B = b1)
+      const uint32_t acc = kKV && kPart == 1 ? G::kColA2 : kColA1;
+      const uint32_t pcol = G::x_col(bb, kKV) + (kKV && kPart == 0 ? 0u : 64u);
+      const uint32_t bsrc = kKV && kPart == 0 ? b2 : b1;
+      // accumulator columns 64 c .. 64 c + 63 from chunk c of the moving tile
+#pragma unroll
+      for (int c = 0; c < G::kChunks; ++c) {
+        const uint32_t boff = c * kChunkBytes;
+#pragma unroll
+        for (int kk = 0; kk < kBlock / 16; ++kk) {
+          mma_ts(tmem + acc + 64 * c, tmem + pcol + hi_col(kk), sdesc_sw128(bsrc + boff + kk * 2048, 8192, 1024),
+                 idesc2, (zero && kk == 0) ? 0u : 1u);
+          mma_ts(tmem + acc + 64 * c, tmem + pcol + lo_col(kk), sdesc_sw128(bsrc + boff + kk * 2048, 8192, 1024),
+                 idesc2, 1u);
+        }
+      }
+      mma_commit(smem_u32(&s.xy_free[kPart][bb]));
+      if (last) mma_commit(smem_u32(&s.acc_full));
+    }
+    mma_commit(smem_u32(&s.b_empty[st]));
+    return true;
+  };
   uint32_t g = 0, ua = 0;
+  bool pend = false, pend_zero = false, pend_last = false;
+  uint32_t pend_g = 0, pend_ua = 0;
   bool ok = true;
   for (uint32_t ut = 0; ok; ++ut) {
     if (!mbar_wait(smem_u32(&s.info_full[ut & 3]), (ut >> 2) & 1)) { ok = false; break; }
@@ -586,56 +635,42 @@ __device__ void mma_role(Smem<kD>& s, const Params& p, uint32_t tmem) {
     const bool first = ui.first, last = ui.last;
     if (first && !mbar_wait(smem_u32(&s.a_full), ua & 1)) { ok = false; break; }
     for (int e = 0; e < n; ++e, ++g) {
-      const int st = g % kStages;
-      if (!mbar_wait(smem_u32(&s.b_full[st]), (g / kStages) & 1)) { ok = false; break; }
-      if (g >= 1) {
-        if (kKV && !mbar_wait(smem_u32(&s.xy_free[kPart]), (g - 1) & 1)) { ok = false; break; }
-        if (!kKV && kPart == 1 && !mbar_wait(smem_u32(&s.xy_free[0]), (g - 1) & 1)) { ok = false; break; }
+      const int st = g % kSt;
+      const uint32_t bb = g % kNB;
+      if (!mbar_wait(smem_u32(&s.b_full[st]), (g / kSt) & 1)) { ok = false; break; }
+      if (g >= static_cast<uint32_t>(kNB)) {
+        const uint32_t ph = ((g / kNB) - 1) & 1;  // step g - kNB
+        if (kKV && !mbar_wait(smem_u32(&s.xy_free[kPart][bb]), ph)) { ok = false; break; }
+        if (!kKV && kPart == 1 && !mbar_wait(smem_u32(&s.xy_free[0][bb]), ph)) { ok = false; break; }
       }
       tc_fence_after();
-      const uint32_t b1 = smem_u32(s.b1[st]), b2 = smem_u32(s.b2[st]);
-      const uint32_t b_src = kPart == 0 ? b1 : b2;
+      const uint32_t b_src = smem_u32(kPart == 0 ? s.b1[st] : s.b2[st]);
+      const uint32_t x_col = G::x_col(bb, kKV) + (kPart == 0 ? 0u : 64u);  // this part's S or dP columns
       // K = d in steps of 16: four per 64-column chunk
 #pragma unroll
       for (int kk = 0; kk < kD / 16; ++kk)
         mma_ss(tmem + x_col, sdesc_sw128(a_src + (kk >> 2) * G::kAChunkBytes + (kk & 3) * 32, 16, 1024),
                sdesc_sw128(b_src + (kk >> 2) * kChunkBytes + (kk & 3) * 32, 16, 1024), idesc1, kk > 0 ? 1u : 0u);
-      mma_commit(smem_u32(&s.x_full));
+      mma_commit(smem_u32(&s.x_full[bb]));
       if (last && e == n - 1) mma_commit(smem_u32(&s.a_free));
-      if (kHasGrad) {
-        // the unit's first step overwrites the accumulator, once the previous
-        // unit's epilogue has read it
-        const bool zero = first && e == 0;
-        if (zero && !mbar_wait(smem_u32(&s.acc_free), (ua & 1) ^ 1)) { ok = false; break; }
-        if (!mbar_wait(smem_u32(&s.p_full), g & 1)) { ok = false; break; }
-        tc_fence_after();
-        // dk/dv part 0: dV += (P_hi + P_lo) dO (P in the S columns, B = b2);
-        // dk/dv part 1: dK += (dS_hi + dS_lo) Q (dS in the dP columns, B = b1);
-        // dq: dQ += (dS_hi + dS_lo) K (dS in the dP columns, B = b1)
-        const uint32_t acc = kKV && kPart == 1 ? G::kColA2 : kColA1;
-        const uint32_t pcol = kKV && kPart == 0 ? kColX : kColY;
-        const uint32_t bsrc = kKV && kPart == 0 ? b2 : b1;
-        // accumulator columns 64 c .. 64 c + 63 from chunk c of the moving tile
-#pragma unroll
-        for (int c = 0; c < G::kChunks; ++c) {
-          const uint32_t boff = c * kChunkBytes;
-#pragma unroll
-          for (int kk = 0; kk < kBlock / 16; ++kk) {
-            mma_ts(tmem + acc + 64 * c, tmem + pcol + hi_col(kk), sdesc_sw128(bsrc + boff + kk * 2048, 8192, 1024),
-                   idesc2, (zero && kk == 0) ? 0u : 1u);
-            mma_ts(tmem + acc + 64 * c, tmem + pcol + lo_col(kk), sdesc_sw128(bsrc + boff + kk * 2048, 8192, 1024),
-                   idesc2, 1u);
-          }
-        }
-        mma_commit(smem_u32(&s.xy_free[kPart]));
-        if (last && e == n - 1) mma_commit(smem_u32(&s.acc_full));
+      const bool zero = first && e == 0;
+      const bool lst = last && e == n - 1;
+      if (kNB == 1) {
+        if (!issue_grad(g, zero, lst, ua)) { ok = false; break; }
+      } else {
+        if (pend && !issue_grad(pend_g, pend_zero, pend_last, pend_ua)) { ok = false; break; }
+        pend = true;
+        pend_g = g;
+        pend_zero = zero;
+        pend_last = lst;
+        pend_ua = ua;
       }
-      mma_commit(smem_u32(&s.b_empty[st]));
     }
     if (!ok) break;
     if (first) ++ua;
     mbar_arrive(smem_u32(&s.info_empty[ut & 3]));
   }
+  if (ok && pend && !issue_grad(pend_g, pend_zero, pend_last, pend_ua)) ok = false;
   if (!ok) flag_timeout(p);
 }
 
@@ -734,26 +769,29 @@ __device__ void elem_role(Smem<kD>& s, const Params& p, uint32_t tmem, const Sto
     }
     for (int e = 0; e < n; ++e, ++g) {
       const bool used = exists && ((ui.hm[e] >> half) & 1);
-      if (!warp_wait(smem_u32(&s.x_full), g & 1)) { if (lane == 0) flag_timeout(p); return; }
+      const uint32_t bb = g % BGeo<kD>::kBufs;
+      if (!warp_wait(smem_u32(&s.x_full[bb]), (g / BGeo<kD>::kBufs) & 1)) { if (lane == 0) flag_timeout(p); return; }
       tc_fence_after();
-      const int st = g % kStages;
-      if (kKV && !warp_wait(smem_u32(&s.b_full[st]), (g / kStages) & 1)) { if (lane == 0) flag_timeout(p); return; }
+      const int st = g % BGeo<kD>::kStages;
+      if (kKV && !warp_wait(smem_u32(&s.b_full[st]), (g / BGeo<kD>::kStages) & 1)) { if (lane == 0) flag_timeout(p); return; }
+      // this step's S and dP columns
+      const uint32_t xcol = BGeo<kD>::x_col(bb, kKV), ycol = xcol + 64;
       if (used) {
         const uint64_t vm = kKV ? ~0ull : ui.vm[e];
 #pragma unroll 1
         for (int q = 2 * chalf; q < 2 * chalf + 2; ++q) {
           uint32_t x[16], y[16], pk[8], pl[8], dk[8], dl[8];
-          tmem_ld16(lane_addr + kColX + 16 * q, x);
-          tmem_ld16(lane_addr + kColY + 16 * q, y);
+          tmem_ld16(lane_addr + xcol + 16 * q, x);
+          tmem_ld16(lane_addr + ycol + 16 * q, y);
           tmem_wait_ld();
           piece_pds<kKV>(x, y, 16 * q, vm, row_c, row_cmask, row_d, s.col_lse[st], s.col_d[st], row_bias_l2,
                          p.scale_log2, pk, pl, dk, dl);
           if (kKV) {
-            tmem_st8(lane_addr + kColX + hi_col(q), pk);
-            tmem_st8(lane_addr + kColX + lo_col(q), pl);
+            tmem_st8(lane_addr + xcol + hi_col(q), pk);
+            tmem_st8(lane_addr + xcol + lo_col(q), pl);
           }
-          tmem_st8(lane_addr + kColY + hi_col(q), dk);
-          tmem_st8(lane_addr + kColY + lo_col(q), dl);
+          tmem_st8(lane_addr + ycol + hi_col(q), dk);
+          tmem_st8(lane_addr + ycol + lo_col(q), dl);
         }
       } else {
         uint32_t z[16];
@@ -761,14 +799,14 @@ __device__ void elem_role(Smem<kD>& s, const Params& p, uint32_t tmem, const Sto
         for (int i = 0; i < 16; ++i) z[i] = 0u;
 #pragma unroll
         for (int q = 2 * chalf; q < 2 * chalf + 2; ++q) {
-          if (kKV) tmem_st16(lane_addr + kColX + 16 * q, z);
-          tmem_st16(lane_addr + kColY + 16 * q, z);
+          if (kKV) tmem_st16(lane_addr + xcol + 16 * q, z);
+          tmem_st16(lane_addr + ycol + 16 * q, z);
         }
       }
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&s.p_full));
+      if (lane == 0) mbar_arrive(smem_u32(&s.p_full[bb]));
     }
     const bool last = ui.last;
     const int split = ui.split;
@@ -888,14 +926,16 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUt
     }
     mbar_init(smem_u32(&s.a_full), 1);
     mbar_init(smem_u32(&s.a_free), 2);  // both MMA threads read the stationary operands
-    for (int i = 0; i < kStages; ++i) {
+    for (int i = 0; i < BGeo<kD>::kStages; ++i) {
       mbar_init(smem_u32(&s.b_full[i]), 1);
       mbar_init(smem_u32(&s.b_empty[i]), 2);
     }
-    mbar_init(smem_u32(&s.x_full), 2);  // S and dP, one MMA thread each
-    mbar_init(smem_u32(&s.p_full), kElemWarps);
-    mbar_init(smem_u32(&s.xy_free[0]), 1);
-    mbar_init(smem_u32(&s.xy_free[1]), 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(&s.x_full[i]), 2);  // S and dP, one MMA thread each
+      mbar_init(smem_u32(&s.p_full[i]), kElemWarps);
+      mbar_init(smem_u32(&s.xy_free[0][i]), 1);
+      mbar_init(smem_u32(&s.xy_free[1][i]), 1);
+    }
     mbar_init(smem_u32(&s.acc_full), kKV ? 2 : 1);  // dk/dv: two accumulators, one per MMA thread
     mbar_init(smem_u32(&s.acc_free), kElemWarps);
     mbar_init(smem_u32(&s.stage_free), 1);
