@@ -90,13 +90,14 @@ struct Geo {
   static constexpr int kChunks = kD / 64;
   static constexpr uint32_t kTileBytes = kBlock * kD * 2;    // one 64-token tile of K or V
   static constexpr uint32_t kQChunkBytes = kRows * 64 * 2;   // one chunk of the unit's Q
-  // TMEM columns per CTA (S 64 + O d, rounded up to a power of two) and CTAs
-  // per SM: four at d = 64, two at d = 128 (TMEM and shared memory)
+  // bigbird_fwd_kernel (d = 128; d = 64 runs on bigbird_fwd2_kernel): TMEM
+  // columns per CTA and CTAs per SM (TMEM and shared memory). The template
+  // also describes the single-buffered d = 64 form (S 64 + O 64 in 128
+  // columns, four CTAs per SM), which is no longer launched.
   static constexpr uint32_t kTmemCols = kD == 64 ? 128 : 256;
   static constexpr int kCtasPerSm = kD == 64 ? 4 : 2;
-  // S buffers of bigbird_fwd_kernel: at d = 128 the second one sits in the 64
-  // columns after O (S(g+1) is computed while the softmax works on block g);
-  // at d = 64 there is one
+  // its S buffers: at d = 128 the second one sits in the 64 columns after O
+  // (S(g+1) is computed while the softmax works on block g)
   static constexpr int kSBufs = kD == 128 ? 2 : 1;
   __host__ __device__ static constexpr uint32_t s_col(uint32_t g) { return (kSBufs == 2 && (g & 1)) ? 192u : 0u; }
 };
@@ -1354,6 +1355,7 @@ template <int kD, bool kBf16>
 __global__ void __launch_bounds__(kThreads, Geo<kD>::kCtasPerSm)
 bigbird_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
+  static_assert(kD == 128, "d = 64 runs on bigbird_fwd2_kernel");
   extern __shared__ uint8_t smem_raw[];
   SharedStorage<kD>& s =
       *reinterpret_cast<SharedStorage<kD>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
