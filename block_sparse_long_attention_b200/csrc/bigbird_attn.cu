@@ -655,10 +655,12 @@ __device__ void producer_role(S& s, const FwdParams& p, const CUtensorMap* tmQ, 
 
 // ---------------------------------------------------------------- MMA issuer
 
-// Per key block g of this CTA: S(g) = Q . K(g)^T into the S columns once the
-// previous block's P.V has consumed the P that shares them, then, once the
-// softmax has written P(g), O += P(g) . V(g). The chain is serial within a
-// CTA; the four CTAs of an SM interleave on the tensor pipe.
+// Per key block g of this CTA: S(g) = Q . K(g)^T into S buffer g % kSBufs
+// once the P.V that read the P sharing those columns (kSBufs blocks back) is
+// complete, then, once the softmax has written P(g), O += P(g) . V(g). With
+// two buffers (d = 128) S(g) goes out before P.V(g - 1), so that it is ready
+// when the softmax finishes block g - 1; the two CTAs of an SM interleave on
+// the tensor pipe.
 template <int kD, bool kBf16>
 __device__ void mma_role(SharedStorage<kD>& s, const FwdParams& p, uint32_t tmem) {
   using Gm = Geo<kD>;
