@@ -159,13 +159,22 @@ def test_determinism_and_batch_slices():
         assert np.array_equal(a[bi:bi + 1], c)
 
 
-def test_key_set_probe_exact():
+@pytest.mark.parametrize("L,bs,r,plant", [(4096, 64, 3, False), (4096, 64, 16, True), (8192, 128, 16, True)],
+                         ids=["block64_r3", "block64_r16_dups", "block128_r16_dups"])
+def test_key_set_probe_exact(L, bs, r, plant):
     """Q = 0 and V one-hot by key block (d = nb = 64): every row's output is the
     fraction of its valid keys in each block, so the per-block key counts of
-    every row are recovered exactly from the fp32 output."""
-    B, H, L, bs, r = 2, 3, 4096, 64, 3
+    every row are recovered exactly from the fp32 output. With r = 16 a pair
+    of query blocks has 38 candidate key blocks (window, global, 32 random),
+    more than one per lane of the warp that builds the list; the planted
+    entries repeat blocks listed earlier (the row's own first entry, a global
+    block, a window block, the previous row's entry), some of them with
+    another half mask, which set semantics merges [TFG-BigBird, section
+    "随机块掩码是如何生成的"]."""
+    B, H = 2, 3
     nb = L // bs
-    vl = [4096, 2500]
+    assert nb == 64
+    vl = [L, L * 5 // 8]
     sm = mask_from_lengths(B, L, vl)
     q = torch.zeros(B, H, L, 64, dtype=torch.bfloat16)
     k = torch.randn(B, H, L, 64, generator=torch.Generator().manual_seed(5)).to(torch.bfloat16)
@@ -173,7 +182,16 @@ def test_key_set_probe_exact():
     for j in range(nb):
         v[:, :, j * bs:(j + 1) * bs, j] = 1.0
     ra = bb.rand_attn_generate(H, L, bs, r, seed=21)
-    w = Workload("probe", B, H, L, seed=0)
+    if plant:
+        for x in range(nb - 2):  # row x: query block x + 1
+            e = ra[1, x]
+            e[10] = e[0]
+            e[11] = 0
+            e[12] = x
+            e[13] = ra[1, x - 1, 3] if x >= 1 else nb - 1
+            e[14] = nb - 1
+            e[15] = e[14]
+    w = Workload("probe", B, H, L, block=bs, r=r, seed=0)
     got = _cuda_fwd({"q": q, "k": k, "v": v, "seq_mask": sm}, w, ra, torch.float32)
     for b in range(B):
         valid = np.arange(L) < vl[b]
