@@ -40,7 +40,7 @@
 //     MMA, 6 unit preparation, 7 V conversion.
 //
 // The prep warp schedules and prepares units (key-block list, half masks,
-// key-validity bits) up to four units ahead, plus L2 prefetch, so its
+// key-validity bits) up to two units ahead, plus L2 prefetch, so its
 // dependent global loads never stall the pipeline.
 //
 // Softmax: 16 columns at a time; the reference max moves only when a score
@@ -433,12 +433,14 @@ __device__ void prep_unit(const FwdParams& p, int u, UnitInfo& ui, int lane) {
   __syncwarp();
 }
 
-// Unit preparation, up to four units ahead of the TMA warp: slot ut & 3 is
-// refilled once every consumer of unit ut - 4 has released it. The prep warp
-// also schedules: a CTA's first unit is blockIdx.x, every later one is a
-// ticket from a device-wide counter (units are numbered longest first), so
-// CTAs that run faster take more units and all finish together. Once the
-// tickets run out it publishes a stop slot, which ends every role's loop.
+// Unit preparation, up to two units ahead of the consumers: unit ut is
+// claimed and prepared (into slot ut & 3) once every consumer has released
+// unit ut - 2. The prep warp also schedules: a CTA's first unit is
+// blockIdx.x, every later one is a ticket from a device-wide counter (units
+// are numbered longest first), so CTAs that run faster take more units and
+// all finish together; claiming only two ahead keeps the work a CTA holds
+// when the tickets run out, and so the spread of finish times, small. Once
+// the tickets run out it publishes a stop slot, which ends every role's loop.
 template <class S, bool kAllTickets>
 __device__ void prep_role(S& s, const FwdParams& p, int bt) {
   constexpr int kD = S::kDim;
@@ -453,7 +455,8 @@ __device__ void prep_role(S& s, const FwdParams& p, int bt) {
   for (uint32_t ut = 0;; ++ut) {
     const int slot = ut & 3;
     int ok = 1;
-    if (lane == 0) ok = mbar_wait(smem_u32(&s.info_empty[slot]), ((ut >> 2) & 1) ^ 1);
+    // at most two units ahead: unit ut - 2 released (which implies ut - 4)
+    if (lane == 0) ok = ut < 2 || mbar_wait(smem_u32(&s.info_empty[(ut - 2) & 3]), ((ut - 2) >> 2) & 1);
     if (!__shfl_sync(0xffffffffu, ok, 0)) {
       if (lane == 0) flag_timeout(s, p);
       return;
@@ -472,7 +475,7 @@ __device__ void prep_role(S& s, const FwdParams& p, int bt) {
     if (bt == 1) prep_unit<1>(p, u, ui, lane);
     else prep_unit<2>(p, u, ui, lane);
     if (lane == 0) mbar_arrive(smem_u32(&s.info_full[slot]));
-    // Pull the unit's tiles into L2 now (it is up to four units ahead of the
+    // Pull the unit's tiles into L2 now (it is up to two units ahead of the
     // TMA warp), so its TMA loads hit L2 instead of HBM: one tile per
     // lane, lanes 0..n-1 K, n..2n-1 V, 2n and 2n+1 the query blocks.
     const size_t row0 = static_cast<size_t>(ui.bh) * p.L;

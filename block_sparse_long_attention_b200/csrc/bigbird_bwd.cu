@@ -334,7 +334,7 @@ __device__ void build_simple(const Params& p, int u, Unit& ui, int lane) {
 
 // ------------------------------------------------------------ preparation
 
-// Unit preparation and scheduling (one warp), up to four chunks ahead: a CTA's
+// Unit preparation and scheduling (one warp), up to two chunks ahead: a CTA's
 // first unit is its block index, later ones are tickets from the workspace
 // counter (units numbered longest first). Publishes a stop slot at the end.
 // The dk/dv kernel's middle units -- key blocks (j, j+1) at block 64, key
@@ -351,7 +351,8 @@ __device__ void prep_role(Smem<kD>& s, const Params& p) {
   uint32_t ut = 0;  // chunks published so far
   auto acquire = [&]() -> Unit* {
     int ok = 1;
-    if (lane == 0) ok = mbar_wait(smem_u32(&s.info_empty[ut & 3]), ((ut >> 2) & 1) ^ 1);
+    // at most two chunks ahead: chunk ut - 2 released (which implies ut - 4)
+    if (lane == 0) ok = ut < 2 || mbar_wait(smem_u32(&s.info_empty[(ut - 2) & 3]), ((ut - 2) >> 2) & 1);
     if (!__shfl_sync(0xffffffffu, ok, 0)) return nullptr;
     return &s.unit[ut & 3];
   };
