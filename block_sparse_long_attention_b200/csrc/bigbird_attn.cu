@@ -1281,13 +1281,13 @@ __device__ void softmax2_role(SharedStorage2& s, const FwdParams& p, uint32_t tm
 // log-sum-exp (log2 units) and write those rows' output and lse. Called by
 // every thread of a CTA; the grid's CTAs deal the rows out among themselves,
 // d / 4 threads per row (4 columns each), which take the row's ranges in
-// order, four at a time with their loads in flight together. The result does
+// order, eight at a time with their loads in flight together. The result does
 // not depend on which CTA merges a row.
 template <int kD, int kNT>
 __device__ void merge_ranges(const FwdParams& p, int cta, int ncta) {
   constexpr int kTpr = kD / 4;
   constexpr int kRowsPerPass = kNT / kTpr;
-  constexpr int kBatch = 4;
+  constexpr int kBatch = 8;
   const int c4 = static_cast<int>(threadIdx.x) % kTpr;
   const int total = p.BH * p.n_glob * kRows;
   const float2* ml = reinterpret_cast<const float2*>(p.part_ml);
