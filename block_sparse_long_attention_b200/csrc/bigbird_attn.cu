@@ -1069,7 +1069,7 @@ __device__ void softmax2_role(SharedStorage2& s, const FwdParams& p, uint32_t tm
   uint32_t g = 0;
   uint32_t staged = 0;  // units whose output tile went out through ostage
   for (uint32_t ut = 0;; ++ut) {
-    if (!warp_wait(smem_u32(&s.info_full[ut & 3]), (ut >> 2) & 1)) { flag_timeout(s, p); return; }
+    if (__builtin_expect(!warp_wait(smem_u32(&s.info_full[ut & 3]), (ut >> 2) & 1), 0)) { flag_timeout(s, p); return; }
     const UnitInfo& ui = s.unit[ut & 3];
     if (ui.stop) break;
     const int n = ui.n;
@@ -1083,7 +1083,7 @@ __device__ void softmax2_role(SharedStorage2& s, const FwdParams& p, uint32_t tm
     float l_run = 0.f;
     for (int e = 0; e < n; ++e, ++g) {
       const bool used = exists && ((ui.hm[e] >> rhalf) & 1);
-      if (!warp_wait(smem_u32(&s.s_full[g & 1]), (g >> 1) & 1)) { flag_timeout(s, p); return; }
+      if (__builtin_expect(!warp_wait(smem_u32(&s.s_full[g & 1]), (g >> 1) & 1), 0)) { flag_timeout(s, p); return; }
       tc_fence_after();
       const uint32_t s_addr = lane_addr + 64 * (g & 1) + 32 * h;
       if (used) {
@@ -1101,7 +1101,7 @@ __device__ void softmax2_role(SharedStorage2& s, const FwdParams& p, uint32_t tm
                               p.scale_log2, off_s);
         const bool need = mx > m_ref + kRescaleThreshold;
         float o_factor = 1.f;  // rescale owed to O (the P.V of the earlier blocks)
-        if (__any_sync(0xffffffffu, need)) {
+        if (__builtin_expect(__any_sync(0xffffffffu, need), 0)) {
           if (need) {
             o_factor = ex2_approx(m_ref - mx);
             m_ref = mx;
@@ -1121,8 +1121,8 @@ __device__ void softmax2_role(SharedStorage2& s, const FwdParams& p, uint32_t tm
         l_run += (a0 + a1) + (b0 + b1);
         // this half's O holds the P.V of the earlier blocks (none yet for e == 0);
         // rescale it once that P.V is done
-        if (e > 0 && __any_sync(0xffffffffu, o_factor != 1.f)) {
-          if (!warp_wait(smem_u32(&s.pv_done[(g - 1) & 1]), ((g - 1) >> 1) & 1)) { flag_timeout(s, p); return; }
+        if (__builtin_expect(e > 0 && __any_sync(0xffffffffu, o_factor != 1.f), 0)) {
+          if (__builtin_expect(!warp_wait(smem_u32(&s.pv_done[(g - 1) & 1]), ((g - 1) >> 1) & 1), 0)) { flag_timeout(s, p); return; }
           tc_fence_after();
           rescale_o<64>(lane_addr + kColOa + 64 * h, o_factor);
         }
@@ -1142,14 +1142,14 @@ __device__ void softmax2_role(SharedStorage2& s, const FwdParams& p, uint32_t tm
     if (lane == 0) mbar_arrive(smem_u32(&s.info_empty[ut & 3]));
 
     // ---- epilogue: combine the halves, each writes 32 columns of its row
-    if (!warp_wait(smem_u32(&s.o_full), ut & 1)) { flag_timeout(s, p); return; }
+    if (__builtin_expect(!warp_wait(smem_u32(&s.o_full), ut & 1), 0)) { flag_timeout(s, p); return; }
     tc_fence_after();
     // the previous tile's TMA store has read ostage before anyone writes it again
     if (wid == 0 && lane == 0) bulk_wait_read_all();
     s.mlx[ut & 1][h][row] = make_float2(m_ref, l_run);
     __syncwarp();
     if (lane == 0) mbar_arrive(smem_u32(&s.ml_ready));
-    if (!warp_wait(smem_u32(&s.ml_ready), ut & 1)) { flag_timeout(s, p); return; }
+    if (__builtin_expect(!warp_wait(smem_u32(&s.ml_ready), ut & 1), 0)) { flag_timeout(s, p); return; }
     const float2 A = s.mlx[ut & 1][0][row];
     const float2 B = s.mlx[ut & 1][1][row];
     const float m = fmaxf(A.x, B.x);
@@ -1198,7 +1198,7 @@ __device__ void softmax2_role(SharedStorage2& s, const FwdParams& p, uint32_t tm
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&s.tile_ready));
       if (wid == 0) {
-        if (!warp_wait(smem_u32(&s.tile_ready), staged & 1)) { flag_timeout(s, p); return; }
+        if (__builtin_expect(!warp_wait(smem_u32(&s.tile_ready), staged & 1), 0)) { flag_timeout(s, p); return; }
         if (lane == 0) {
           const CUtensorMap* map = split >= 0 ? &tmO->part : &tmO->out;
           int32_t y0, y1;
@@ -1261,7 +1261,7 @@ __device__ void softmax2_role(SharedStorage2& s, const FwdParams& p, uint32_t tm
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&s.tile_ready));
       if (wid == 0) {
-        if (!warp_wait(smem_u32(&s.tile_ready), staged & 1)) { flag_timeout(s, p); return; }
+        if (__builtin_expect(!warp_wait(smem_u32(&s.tile_ready), staged & 1), 0)) { flag_timeout(s, p); return; }
         if (lane == 0) {
           const int32_t row0 = bh * p.L;
           tma_store_2d(&tmO->out, smem_u32(s.ostage), 0, row0 + qtop * kBlock);
