@@ -747,7 +747,7 @@ __device__ void elem_role(Smem<kD>& s, const Params& p, uint32_t tmem, const Sto
   uint32_t staged = 0;  // d = 64: accumulator tiles that went out through ostage
   float row_c = 0.f, row_cmask = 0.f, row_d = 0.f, row_bias_l2 = 0.f;
   for (uint32_t ut = 0;; ++ut) {
-    if (!warp_wait(smem_u32(&s.info_full[ut & 3]), (ut >> 2) & 1)) { if (lane == 0) flag_timeout(p); return; }
+    if (__builtin_expect(!warp_wait(smem_u32(&s.info_full[ut & 3]), (ut >> 2) & 1), 0)) { if (lane == 0) flag_timeout(p); return; }
     const Unit& ui = s.unit[ut & 3];
     if (ui.stop) break;
     const int n = ui.n;
@@ -771,10 +771,10 @@ __device__ void elem_role(Smem<kD>& s, const Params& p, uint32_t tmem, const Sto
     for (int e = 0; e < n; ++e, ++g) {
       const bool used = exists && ((ui.hm[e] >> half) & 1);
       const uint32_t bb = g % BGeo<kD>::kBufs;
-      if (!warp_wait(smem_u32(&s.x_full[bb]), (g / BGeo<kD>::kBufs) & 1)) { if (lane == 0) flag_timeout(p); return; }
+      if (__builtin_expect(!warp_wait(smem_u32(&s.x_full[bb]), (g / BGeo<kD>::kBufs) & 1), 0)) { if (lane == 0) flag_timeout(p); return; }
       tc_fence_after();
       const int st = g % BGeo<kD>::kStages;
-      if (kKV && !warp_wait(smem_u32(&s.b_full[st]), (g / BGeo<kD>::kStages) & 1)) { if (lane == 0) flag_timeout(p); return; }
+      if (__builtin_expect(kKV && !warp_wait(smem_u32(&s.b_full[st]), (g / BGeo<kD>::kStages) & 1), 0)) { if (lane == 0) flag_timeout(p); return; }
       // this step's S and dP columns
       const uint32_t xcol = BGeo<kD>::x_col(bb, kKV), ycol = xcol + 64;
       if (used) {
@@ -815,7 +815,7 @@ __device__ void elem_role(Smem<kD>& s, const Params& p, uint32_t tmem, const Sto
     if (lane == 0) mbar_arrive(smem_u32(&s.info_empty[ut & 3]));
     if (!last) continue;
     // ---- epilogue: this warp's d / 2 columns of each accumulator
-    if (!warp_wait(smem_u32(&s.acc_full), ua & 1)) { if (lane == 0) flag_timeout(p); return; }
+    if (__builtin_expect(!warp_wait(smem_u32(&s.acc_full), ua & 1), 0)) { if (lane == 0) flag_timeout(p); return; }
     tc_fence_after();
     if constexpr (kD == 64) {
       // Each accumulator goes out through ostage: every thread writes its 32
@@ -831,7 +831,7 @@ __device__ void elem_role(Smem<kD>& s, const Params& p, uint32_t tmem, const Sto
           bulk_wait_read_all();  // the previous tile's stores have read ostage
           mbar_arrive(smem_u32(&s.stage_free));
         }
-        if (!warp_wait(smem_u32(&s.stage_free), staged & 1)) { if (lane == 0) flag_timeout(p); return; }
+        if (__builtin_expect(!warp_wait(smem_u32(&s.stage_free), staged & 1), 0)) { if (lane == 0) flag_timeout(p); return; }
         if (exists) {
 #pragma unroll 1
           for (int c0 = 0; c0 < 32; c0 += 16) {
@@ -851,7 +851,7 @@ __device__ void elem_role(Smem<kD>& s, const Params& p, uint32_t tmem, const Sto
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&s.tile_ready));
         if (warp == 0) {
-          if (!warp_wait(smem_u32(&s.tile_ready), staged & 1)) { if (lane == 0) flag_timeout(p); return; }
+          if (__builtin_expect(!warp_wait(smem_u32(&s.tile_ready), staged & 1), 0)) { if (lane == 0) flag_timeout(p); return; }
           if (lane == 0) {
             const CUtensorMap* map = split >= 0 ? (a == 0 ? &smaps->p1 : &smaps->p2) : (a == 0 ? &smaps->o1 : &smaps->o2);
             const uint32_t src = smem_u32(s.ostage);
