@@ -39,14 +39,14 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # Share of one forward call taken by the fp16 attention kernel in the ncu
 # launch list of the same workload (cold-cache, serialised launches: the share,
 # not the absolute, carries over to the live timing).
-FWD_KERNEL_SHARE: dict = {"bigbird_base_l4096": 103.60 / (103.60 + 10.23)}
+FWD_KERNEL_SHARE: dict = {"bigbird_base_l4096": 103.23 / (103.23 + 10.19)}
 BWD_DRAM_BYTES_PER_LAUNCH: dict = {
-    # 146.68 MB read + 80.67 MB written, dk/dv launch (d = 64), mean of 8 launches
-    "bigbird_base_l4096": 227.357984e6,
+    # 146.56 MB read + 81.01 MB written, dk/dv launch (d = 64), mean of 11 launches
+    "bigbird_base_l4096": 227.567476e6,
 }
 FWD_DRAM_BYTES_PER_LAUNCH: dict = {
-    # 84.34 MB read + 9.98 MB written, split-row kernel's fp16 instance (d = 64), mean of 30 launches
-    "bigbird_base_l4096": 94.318345e6,
+    # 84.66 MB read + 10.06 MB written, split-row kernel's fp16 instance (d = 64), mean of 30 launches
+    "bigbird_base_l4096": 94.724471e6,
 }
 
 
