@@ -198,3 +198,42 @@ def test_backward_other_sizes(block, d):
         gq, gk, gv = oracle.attention_backward(inp["q"], inp["k"], inp["v"], ra, inp["seq_mask"], w.block, w.r, do)
         for name, got, want in (("dq", dq, gq), ("dk", dk, gk), ("dv", dv, gv)):
             _check_grad(name, got, want, w.name)
+
+
+@pytest.mark.parametrize("block", [64, 128], ids=["b64", "b128"])
+def test_forward_and_backward_at_max_r(block):
+    """r = 16, the largest supported: a pair of 64-token query blocks has 38
+    candidate key blocks (window, global, 32 random), and a key block of the
+    dk/dv kernel is picked by many query blocks. Entries 10..15 of every row
+    repeat blocks listed before them (the row's first entry, a global block,
+    its own window block, the previous row's entry), some with the other
+    half of a pair, which set semantics merges [TFG-BigBird, section
+    "随机块掩码是如何生成的"]. Forward output and lse, and dq, dk, dv against
+    the oracle; the gradients the same on a second run."""
+    nb = 40
+    w = Workload(f"max_r_b{block}", 1, 2, nb * block, block=block, r=16, pad=("fixed", [nb * block - 150]),
+                 seed=91 + block)
+    inp = make_inputs(w)
+    ra = oracle.rand_attn_generate(w.H, w.L, w.block, w.r, seed=5)
+    for x in range(nb - 2):  # row x: query block x + 1
+        e = ra[1, x]
+        e[10] = e[0]
+        e[11] = 0
+        e[12] = x
+        e[13] = ra[1, x - 1, 3] if x >= 1 else nb - 1
+        e[14] = nb - 1
+        e[15] = e[14]
+    do = _dout(w, 13)
+    out, lse, dq, dk, dv = _run(inp, w, ra, do)
+    want = oracle.attention(inp["q"], inp["k"], inp["v"], ra, inp["seq_mask"], w.block, w.r)
+    ferr = np.abs(out - want)
+    _report(case=w.name, grad="out", max_err=float(ferr.max()), mean_err=float(ferr.mean()))
+    assert ferr.max() <= 1e-2 and ferr.mean() <= 1e-3, (float(ferr.max()), float(ferr.mean()))
+    want_lse = oracle.attention_lse(inp["q"], inp["k"], ra, inp["seq_mask"], w.block, w.r)
+    assert np.abs(lse - want_lse).max() <= LSE_MAX_ABS
+    again = _run(inp, w, ra, do)
+    for a, b in zip((dq, dk, dv), again[2:]):
+        assert np.array_equal(a, b)
+    gq, gk, gv = oracle.attention_backward(inp["q"], inp["k"], inp["v"], ra, inp["seq_mask"], w.block, w.r, do)
+    for name, got, want_g in (("dq", dq, gq), ("dk", dk, gk), ("dv", dv, gv)):
+        _check_grad(name, got, want_g, w.name)
