@@ -230,3 +230,34 @@ def test_probs_out_of_range_rand_attn_is_flagged():
     ra_d[0, 3, 1] = 999
     bb.probs(q, k, lse, ra_d, sm, block=64, r=w.r)
     assert bb.device_status() & 1
+
+
+def test_probs_max_r_with_duplicates():
+    """r = 16, the largest supported (21 candidate key blocks per query
+    block), with entries 10..15 of every row repeating blocks listed before
+    them (the row's first entry, a global block, its window block, the
+    previous row's entry): every element of the packed and dense layouts
+    against the oracle's weights (set semantics: a repeated block is listed
+    once) [TFG-BigBird, section "随机块掩码是如何生成的"]."""
+    nb = 40
+    w = Workload("probs_max_r", 1, 2, nb * 64, r=16, pad=("fixed", [nb * 64 - 150]), seed=23)
+    inp = make_inputs(w)
+    ra = oracle.rand_attn_generate(w.H, w.L, w.block, w.r, seed=5)
+    for x in range(nb - 2):  # row x: query block x + 1
+        e = ra[1, x]
+        e[10] = e[0]
+        e[11] = 0
+        e[12] = x
+        e[13] = ra[1, x - 1, 3] if x >= 1 else nb - 1
+        e[14] = nb - 1
+        e[15] = e[14]
+    q, k, lse, ra_d, sm = _gpu_lse(inp, w, ra)
+    pg, pb = bb.probs(q, k, lse, ra_d, sm, block=64, r=w.r)
+    pd = bb.probs_dense(q, k, lse, ra_d, sm, block=64, r=w.r)
+    torch.cuda.synchronize()
+    assert bb.device_status() == 0
+    P = oracle.attention_probs(inp["q"], inp["k"], ra, inp["seq_mask"], w.block, w.r)
+    glob, band = _pack(P, ra, w)
+    _close(pg.cpu().numpy(), glob, REL_F32, "global rows")
+    _close(pb.cpu().numpy(), band, REL_F32, "band tiles")
+    _close(pd.cpu().numpy(), P, REL_F32, "dense")
