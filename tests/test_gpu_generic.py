@@ -215,3 +215,31 @@ def test_d128_v_beyond_fp16_range(block, d):
     assert off.any() and (~off).any()
     assert err[off].max() <= 1e-2 and err[off].mean() <= 1e-3, float(err[off].max())
     assert (err <= 1e-2 + 2.0 ** -7 * mass * vmax).all()
+
+
+@pytest.mark.parametrize("block,d", [(32, 64), (32, 128), (64, 128)], ids=["b32_d64", "b32_d128", "b64_d128"])
+def test_max_r_with_duplicates(block, d):
+    """r = 16, the largest supported, on the CUDA-core kernel (block 32) and
+    the d = 128 tensor-core kernel: entries 10..15 of every row repeat blocks
+    listed before them (the row's first entry, a global block, its window
+    block, the previous row's entry), which set semantics lists once
+    [TFG-BigBird, section "随机块掩码是如何生成的"]; output and lse against the
+    oracle."""
+    nb = 40
+    w = Workload(f"max_r_b{block}_d{d}", 1, 2, nb * block, d=d, block=block, value_scale=1.0,
+                 pad=("fixed", [nb * block - 3 * block // 2]), r=16, seed=31 + block + d)
+    inp = make_inputs(w)
+    ra = oracle.rand_attn_generate(w.H, w.L, w.block, w.r, seed=5)
+    for x in range(nb - 2):  # row x: query block x + 1
+        e = ra[1, x]
+        e[10] = e[0]
+        e[11] = 0
+        e[12] = x
+        e[13] = ra[1, x - 1, 3] if x >= 1 else nb - 1
+        e[14] = nb - 1
+        e[15] = e[14]
+    want = oracle.attention(inp["q"], inp["k"], inp["v"], ra, inp["seq_mask"], w.block, w.r)
+    got, lse = _run(w, inp, ra, torch.float32, train=True)
+    _check_f32(block, d, np.abs(got - want), w.name)
+    want_lse = oracle.attention_lse(inp["q"], inp["k"], ra, inp["seq_mask"], w.block, w.r)
+    assert np.abs(lse - want_lse).max() <= 1e-5, (w.name, float(np.abs(lse - want_lse).max()))
