@@ -78,6 +78,7 @@ constexpr int kVStages = 2;            // V ring depth (blocks)
 constexpr int kMaxList = 42;           // key tiles per unit
 constexpr int kMaxR = 16;              // random blocks per row supported
 constexpr int kSplitBlocks = 8;        // key tiles per global-row range
+constexpr int kSplitBlocksLong = 12;   // ... at block 64, d 64 with 256 or more tiles (L >= 16384)
 constexpr int kThreads = 256;
 constexpr uint32_t kColO = 64;         // O: d fp32 columns
 constexpr uint32_t kChunkBytes = kBlock * 64 * 2;  // 64 rows x 64 columns bf16: one TMA box, one 128-byte swizzle span
@@ -1747,8 +1748,10 @@ static int make_plan(int B, int H, int L, int d, int block, int r, unsigned flag
   if (pl.sparse) {
     // a middle unit lists at most 6 + 2r tiles (block 64: two query blocks'
     // union) or 2 (5 + r) (block 128); both fit kMaxList for r <= kMaxR
-    pl.split_tiles = kSplitBlocks;
-    pl.nsplit = (pl.nt + kSplitBlocks - 1) / kSplitBlocks;
+    // longer ranges for long sequences: fewer partial results to write and
+    // merge, while the many middle units still balance the grid's tail
+    pl.split_tiles = (pl.bt == 1 && d == 64 && pl.nt >= 256) ? kSplitBlocksLong : kSplitBlocks;
+    pl.nsplit = (pl.nt + pl.split_tiles - 1) / pl.split_tiles;
     pl.n_glob = pl.bt == 1 ? 1 : 2;
   } else {
     // full attention in one range: nt <= (5 + 2r) bt tiles must fit the list
