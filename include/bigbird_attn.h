@@ -112,7 +112,8 @@ int bigbird_attn_fwd(const void* q, const void* k, const void* v, const int32_t*
  * finds the CTA finishing last (which sets the counters back to zero), and
  * the flag that asks for the bf16 recompute (cleared by the bf16 instance when
  * it runs). When the global rows are split into key ranges (sparse pattern:
- * ranges of 8 tiles of 64 keys) each range's partial result follows, per
+ * ranges of 8 tiles of 64 keys; 12 tiles at block 64, d 64 when the sequence
+ * has 256 or more tiles) each range's partial result follows, per
  * global unit (one unit holds both global blocks at block 64, one unit per
  * global block at block 128): output normalised by its own sum [128 rows, d],
  * running max and running sum, merged by log-sum-exp by the bf16 instance.
