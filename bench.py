@@ -41,8 +41,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # not the absolute, carries over to the live timing).
 FWD_KERNEL_SHARE: dict = {"bigbird_base_l4096": 103.23 / (103.23 + 10.19)}
 BWD_DRAM_BYTES_PER_LAUNCH: dict = {
-    # 146.56 MB read + 81.01 MB written, dk/dv launch (d = 64), mean of 11 launches
-    "bigbird_base_l4096": 227.567476e6,
+    # 146.70 MB read + 81.14 MB written, dk/dv launch (d = 64), mean of 11 launches
+    "bigbird_base_l4096": 227.842141e6,
 }
 FWD_DRAM_BYTES_PER_LAUNCH: dict = {
     # 84.66 MB read + 10.06 MB written, split-row kernel's fp16 instance (d = 64), mean of 30 launches
@@ -467,7 +467,7 @@ def run_bwd(args):
     value = flops / (ms * 1e-3) / 1e12
     peaks, src = _peaks()
     peak = float(peaks["bf16_tflops"])
-    # row dot, dq kernel, dk/dv kernel, and the partial-sum launch when the
+    # row dot, dk/dv kernel, dq kernel, and the partial-sum launch when the
     # global rows are split into key ranges
     launches = 3 + (1 if bb.bwd_workspace_size(w.B, w.H, w.L) > 256 + 4 * w.B * w.H * w.L + 255 else 0)
     line = {

@@ -8,25 +8,27 @@
 //   dp = dout v^T,  ds = p (dp - D),
 //   dq = ds k / sqrt(d),  dk = ds^T q / sqrt(d),  dv = p^T dout.
 //
-// Four launches, in stream order (the dk/dv kernel as the dq kernel's
-// programmatic dependent, free to start on the SMs the dq kernel leaves, as
-// it needs nothing the dq kernel writes), nothing accumulated with atomics
-// (the gradients are the same bit for bit on every run):
+// Four launches, in stream order (the dq kernel as the dk/dv kernel's
+// programmatic dependent, free to start on the SMs the dk/dv kernel leaves,
+// as it needs nothing the dk/dv kernel writes; the dk/dv kernel, whose units
+// are the larger, goes first so that the finer dq units fill the end),
+// nothing accumulated with atomics (the gradients are the same bit for bit
+// on every run):
 //   1. bwd_rowdot_kernel: D = rowsum(dout * out) into the workspace;
-//   2. bwd_kernel<false> (dq): query-stationary. A unit is the forward's: 128
-//      query rows (query blocks i, i+1, or the two global blocks against one
-//      range of key tiles) against a list of 64-key tiles. Per key tile:
-//      S = Q K^T and dP = dO V^T (tcgen05 SS-MMAs, M = 128, N = 64, K = 64,
-//      fp32 in TMEM), P and dS by one thread per query row (bf16, written
-//      back over the S and dP columns), then dQ += dS K (TS-MMA, dS from TMEM,
-//      K as loaded, d contiguous);
-//   3. bwd_kernel<true> (dk, dv): key-stationary. A unit is 128 key rows (key
+//   2. bwd_kernel<true> (dk, dv): key-stationary. A unit is 128 key rows (key
 //      blocks j, j+1, or the two global key blocks against one range of query
 //      tiles) against the query tiles that attend either block -- the pattern
 //      transposed, found by scanning rand_attn (a long list goes out in
 //      chunks). Per query tile: S^T = K Q^T and dP^T = V dO^T, P^T and dS^T by
 //      one thread per key row (the query's lse and D from shared memory), then
 //      dV += P^T dO and dK += dS^T Q (two TS-MMAs);
+//   3. bwd_kernel<false> (dq): query-stationary. A unit is the forward's: 128
+//      query rows (query blocks i, i+1, or the two global blocks against one
+//      range of key tiles) against a list of 64-key tiles. Per key tile:
+//      S = Q K^T and dP = dO V^T (tcgen05 SS-MMAs, M = 128, N = 64, K = 64,
+//      fp32 in TMEM), P and dS by one thread per query row (bf16, written
+//      back over the S and dP columns), then dQ += dS K (TS-MMA, dS from TMEM,
+//      K as loaded, d contiguous);
 //   4. bwd_sum_kernel: the global rows' dq and the global key blocks' dk, dv
 //      are split over ranges; their partial sums (workspace) are added here,
 //      all three in one launch.
@@ -943,10 +945,11 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUt
     mbar_init(smem_u32(&s.tile_ready), kElemWarps);
     fence_barrier_init();
   }
-  // The dk/dv kernel follows the dq kernel as its programmatic dependent: it
-  // reads nothing the dq kernel writes, so its CTAs may take the SMs the dq
-  // kernel's CTAs leave (they never wait for the dq grid).
-  if (!kKV) asm volatile("griddepcontrol.launch_dependents;");
+  // The dq kernel follows the dk/dv kernel as its programmatic dependent: it
+  // reads nothing the dk/dv kernel writes, so its CTAs may take the SMs the
+  // dk/dv kernel's CTAs leave (they never wait for the dk/dv grid; both read
+  // D, which the row dot, launched before them in stream order, wrote).
+  if (kKV) asm volatile("griddepcontrol.launch_dependents;");
   if (warp == 8 && lane == 0) {
     tma_prefetch_desc(&tmA1);
     tma_prefetch_desc(&tmA2);
@@ -1136,8 +1139,9 @@ bool set_attributes(int dev) {
   return true;
 }
 
-// The launches of one backward call: row dot, dq kernel, dk/dv kernel, then
-// the partial sums of the split global units.
+// The launches of one backward call: row dot, dk/dv kernel, dq kernel (its
+// programmatic dependent), then the partial sums of the split global units
+// (a normal launch: it waits for both attention kernels).
 template <int kD, int kBt>
 cudaError_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tdo,
                        const bbw::StoreMaps& smq, const bbw::StoreMaps& smk, const bbw::Params& pq,
@@ -1151,10 +1155,11 @@ cudaError_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUten
   constexpr int kDotRowsPerCta = 256 / (kD / 8);     // row dot: d / 8 threads per row
   bwd_rowdot_kernel<kD><<<static_cast<unsigned>((rows + kDotRowsPerCta - 1) / kDotRowsPerCta), 256, 0, stream>>>(
       static_cast<const uint16_t*>(dout), out, out_f32, dd, rows);
-  bwd_kernel<kD, kBt, false><<<grid, kThreads, smem, stream>>>(tq, tdo, tk, tv, smq, pq);
+  const int grid_kv = std::min(pk.total_units, BGeo<kD>::kCtasPerSm * sms);
+  bwd_kernel<kD, kBt, true><<<grid_kv, kThreads, smem, stream>>>(tk, tv, tq, tdo, smk, pk);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  // the dk/dv kernel as the dq kernel's programmatic dependent (see the kernel)
+  // the dq kernel as the dk/dv kernel's programmatic dependent (see the kernel)
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
@@ -1165,7 +1170,7 @@ cudaError_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUten
   cfg.stream = stream;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, bwd_kernel<kD, kBt, true>, tk, tv, tq, tdo, smk, pk);
+  e = cudaLaunchKernelEx(&cfg, bwd_kernel<kD, kBt, false>, tq, tdo, tk, tv, smq, pq);
   if (e != cudaSuccess) return e;
   if (pl.nsplit > 1) {
     // a normal launch: it waits for both attention kernels
